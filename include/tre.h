@@ -1,0 +1,214 @@
+/*
+ * tre.h — C ABI of the persistent tile engine for batch-1 LLM decode (sm_100a).
+ *
+ * One decode step of a whole decoder stack runs as ONE persistent kernel launch that
+ * executes a static, host-planned list of tile tasks.  Each task waits on a dependency
+ * counter in global memory, streams its weight (or KV) tiles through a shared-memory
+ * ring filled by a bulk-copy producer warp, computes, publishes its outputs and bumps
+ * its output counter, so later tiles start as soon as the tiles they read are done.
+ *
+ * Sources (the pages describe the method only in prose; they print no formula):
+ *   [SC]  "Static Compilation for LLM Inference: from ASIC Graph Compile to Persistent
+ *         Engine Kernel" — §1 (the whole model is statically unrolled ahead of time into
+ *         one Persistent Engine Kernel; the tile is the scheduling unit), §5.1 (tile
+ *         pipeline: shared memory holds one tile at a time), §5.2 (warp-group roles:
+ *         a TMA copy group stands in for the DMA engine, a compute group with the
+ *         activation fused in), §5.4 table (bs=1 GEMM is memory bound, fuse norm+GEMM),
+ *         §6 (launch overhead dominates bs=1 decode).
+ *   [TA]  "TileRT code audit" (tile-ai-tilert page) — blog-vs-code table (host launches
+ *         once; fused ops RMSNormProjxWqkvia, UnProjOAllReduce, ExpertSelectUpGateSiLU,
+ *         ExpertDownAllReduce, FlashSparseMLA with batch == 1; inject_cache() takes an
+ *         external KV cache as raw tensors).
+ *   [SI]  "Speed is intelligence" talk transcript (TileRT team) — section on breaking
+ *         the kernel boundary: tasks whose dependencies are met start early; the model
+ *         is a dataflow graph lowered to tile micro-kernels and an execution engine.
+ *
+ * Conventions for every call:
+ *   - All pointers named *_dev are device pointers on the engine's device; *_host are
+ *     host pointers.  Weight and KV memory is OWNED BY THE CALLER and must outlive the
+ *     engine; the engine never frees it.  The engine owns its plan, task list,
+ *     counters, activation scratch and split-KV partial buffers.
+ *   - Every call returns a tre_status.  Errors detectable on the host are returned
+ *     before anything is enqueued.  Errors found on the device (a dependency wait that
+ *     ran out of time, a bounds check) are recorded in a device status word: they are
+ *     returned by the next tre_decode_step / tre_layers_step (which then launches
+ *     nothing) and by tre_get_status; tre_reset clears them.
+ *   - An engine is not thread safe: calls on one engine must not overlap.
+ *   - Weights, embedding, norm gains and KV caches are bf16 (raw 16-bit words,
+ *     round-to-nearest-even).  Activations, the residual stream, attention partials and
+ *     logits are fp32.  Matrices are row-major W[N][K] (N outputs, K inputs), the
+ *     layout of torch.nn.Linear.weight; every K must be a multiple of 8 (16-byte rows)
+ *     and every pointer 16-byte aligned.
+ */
+#ifndef TRE_H
+#define TRE_H
+
+#include <stdint.h>
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tre_engine tre_engine;          /* opaque, library owned */
+typedef struct CUstream_st* tre_stream;        /* a cudaStream_t (NULL = legacy default) */
+
+typedef enum {
+  TRE_OK = 0,
+  TRE_ERR_INVALID_ARG = -1,   /* bad config value, NULL or misaligned pointer        */
+  TRE_ERR_CUDA = -2,          /* a CUDA runtime call failed (see tre_last_error)     */
+  TRE_ERR_OCCUPANCY = -3,     /* one CTA per SM cannot be co-resident                */
+  TRE_ERR_DEP_TIMEOUT = -4,   /* a device wait ran out of time (device status word)  */
+  TRE_ERR_POS_RANGE = -5,     /* pos (+ tokens) beyond the KV capacity               */
+  TRE_ERR_UNSUPPORTED = -6,   /* config outside what this build implements           */
+  TRE_ERR_BOUNDS = -7,        /* device bounds check fired (device status word)      */
+  TRE_ERR_STATE = -8          /* previous device error not yet cleared by tre_reset  */
+} tre_status;
+
+/* Layer kinds.  GQA: Llama-style pre-norm attention + SwiGLU MLP.  MOE: the same
+ * attention with a routed mixture-of-experts MLP.  MLA: absorbed multi-head latent
+ * attention only (no MLP). */
+enum { TRE_LAYER_GQA = 0, TRE_LAYER_MLA = 1, TRE_LAYER_MOE = 2 };
+
+/* debug_flags bits */
+enum {
+  TRE_DEBUG_HIDDEN = 1,        /* keep the residual stream after every layer          */
+  TRE_DEBUG_TRACE = 2,         /* record per-task start / ready / end timestamps      */
+  TRE_DEBUG_FAULT_INJECT = 4,  /* plan one dependency that can never be met (tests the
+                                  bounded-wait error path; the step returns
+                                  TRE_ERR_DEP_TIMEOUT and the context stays usable)   */
+  TRE_DEBUG_NO_OVERLAP = 8     /* producer waits for each task's dependency before
+                                  streaming its tiles (removes cross-op prefetch; for
+                                  measurement only)                                   */
+};
+
+typedef struct {
+  int32_t kind;                 /* TRE_LAYER_*  (one kind for the whole stack)          */
+  int32_t n_layers;
+  int32_t hidden;               /* d                                                    */
+  int32_t n_q_heads;            /* Hq (MLA: heads)                                      */
+  int32_t n_kv_heads;           /* Hkv (GQA/MOE); Hq % Hkv == 0                         */
+  int32_t head_dim;             /* D (GQA/MOE): 64 or 128                               */
+  int32_t ffn;                  /* F, SwiGLU hidden (GQA)                               */
+  int32_t vocab;                /* V (0 when has_embed_lm_head == 0)                    */
+  int32_t q_lora, kv_lora, rope_dim, nope_dim, v_dim;          /* MLA                   */
+  int32_t n_experts, top_k, n_shared, expert_ffn;              /* MOE                   */
+  int32_t kv_capacity;          /* positions allocated in each KV cache                 */
+  int32_t max_tokens_per_step;  /* M, 1..4                                              */
+  float rope_theta;
+  float norm_eps;
+  int32_t has_embed_lm_head;    /* 1: token in, logits out; 0: hidden in, hidden out    */
+  int32_t debug_flags;          /* TRE_DEBUG_*                                          */
+  int32_t dep_timeout_us;       /* bound on every device wait; 0 = 1,000,000 us         */
+  int32_t num_sms;              /* CTAs of the persistent grid; 0 = every SM            */
+  int32_t kv_splits;            /* split-KV chunks per kv head; 0 = planner's choice    */
+  int32_t stage_bytes;          /* bytes per ring stage; 0 = 32768                      */
+  int32_t ring_stages;          /* ring depth; 0 = as many as shared memory allows      */
+  int32_t reserved[8];          /* must be zero                                         */
+} tre_config;
+
+/* Per-layer tensor slots.  layer_w[l * TRE_W_SLOTS + slot] is the device pointer of
+ * tensor `slot` of layer l (NULL for slots the layer kind does not use).
+ *   GQA : ATTN_NORM[d], WQ[Hq*D][d], WK[Hkv*D][d], WV[Hkv*D][d], WO[d][Hq*D],
+ *         FFN_NORM[d], WGATE[F][d], WUP[F][d], WDOWN[d][F]
+ * KV caches (bf16, written at pos by every step, caller owned):
+ *   GQA/MOE : k_cache[l], v_cache[l] = [Hkv][kv_capacity][D]
+ */
+enum {
+  TRE_W_ATTN_NORM = 0, TRE_W_Q = 1, TRE_W_K = 2, TRE_W_V = 3, TRE_W_O = 4,
+  TRE_W_FFN_NORM = 5, TRE_W_GATE = 6, TRE_W_UP = 7, TRE_W_DOWN = 8,
+  TRE_W_SLOTS = 16
+};
+
+typedef struct {
+  const void* embed;              /* [V][d] bf16                                        */
+  const void* final_norm;         /* [d] bf16                                           */
+  const void* lm_head;            /* [V][d] bf16                                        */
+  const void* const* layer_w;     /* host array of n_layers * TRE_W_SLOTS device ptrs   */
+  void* const* k_cache;           /* host array of n_layers device ptrs                 */
+  void* const* v_cache;           /* host array of n_layers device ptrs (MLA: unused)   */
+} tre_weights;
+
+/* Summary of a plan, filled by tre_plan_inspect (host only, needs no GPU). */
+typedef struct {
+  int32_t num_sms;                /* CTAs planned                                       */
+  int32_t num_tasks;              /* tasks in the whole step                            */
+  int32_t num_counters;
+  int32_t kv_splits;
+  int32_t ring_stages, stage_bytes, smem_bytes;
+  int32_t max_tasks_per_sm;
+  int64_t weight_bytes;           /* weight bytes streamed per step                     */
+  int64_t kv_bytes_at_capacity;   /* KV bytes streamed per step at pos = capacity - M   */
+  int64_t max_sm_bytes, min_sm_bytes;  /* per-CTA streamed bytes (balance)              */
+} tre_plan_info;
+
+/* ---- lifecycle ---------------------------------------------------------------- */
+
+/* Validate cfg and the weight pointers, build the static tile task list (the "AOT
+ * compile" of [SC] §1 / [SI] dataflow-graph-to-engine section), allocate the engine's
+ * device state on `device` and check that one CTA per SM is co-resident.  On success
+ * *out receives the engine.  Ownership: the engine copies cfg and the pointer tables;
+ * the pointed-to device memory stays the caller's. */
+tre_status tre_create(const tre_config* cfg, const tre_weights* w, int device,
+                      tre_engine** out);
+
+/* Free everything the engine owns (not the caller's weights / caches).  NULL is a no-op. */
+void tre_destroy(tre_engine* e);
+
+/* ---- the hot path ------------------------------------------------------------- */
+
+/* One batch-1 decode step of the whole stack as ONE persistent launch on `stream`
+ * ([SC] §1; [TA] blog-vs-code table: the host launches once per token).
+ *   token        input token id, 0 <= token < vocab (kernel argument, no copy)
+ *   pos          position of this token; the KV caches hold positions [0, pos) on
+ *                entry and [0, pos] on return; 0 <= pos < kv_capacity
+ *   logits_dev   device fp32[vocab] or NULL (then only token_dev is produced)
+ *   token_dev    device int32[1] or NULL: greedy argmax of the logits (lowest index
+ *                on ties)
+ * Enqueues asynchronously; returns the previous step's device error, if any, without
+ * launching.  Requires has_embed_lm_head == 1. */
+tre_status tre_decode_step(tre_engine* e, int32_t token, int32_t pos, tre_stream stream,
+                           float* logits_dev, int32_t* token_dev);
+
+/* The same step driven from host memory: copies nothing in (the token is a kernel
+ * argument), runs the step, copies the argmax token (and the logits when logits_host
+ * is not NULL) back into host memory and waits for them.  This is the call a greedy
+ * generation loop makes once per token. */
+tre_status tre_decode_step_host(tre_engine* e, int32_t token, int32_t pos, tre_stream stream,
+                                float* logits_host, int32_t* token_host);
+
+/* ---- status / debug ----------------------------------------------------------- */
+
+/* Wait for the engine's last stream, then report the device status word: 0, or a
+ * negative tre_status (TRE_ERR_DEP_TIMEOUT / TRE_ERR_BOUNDS).  *detail_out (may be
+ * NULL) receives the global index of the task that recorded it. */
+tre_status tre_get_status(tre_engine* e, int32_t* device_status, int32_t* detail_out);
+
+/* Clear the device status word, the dependency counters and the epoch so that the
+ * engine can step again after a device error.  Enqueued on `stream`. */
+tre_status tre_reset(tre_engine* e, tre_stream stream);
+
+/* Copy the residual stream after every layer of the last step ([n_layers][d] fp32,
+ * device) — requires TRE_DEBUG_HIDDEN. */
+tre_status tre_debug_hidden(tre_engine* e, float* hidden_dev, tre_stream stream);
+
+/* Copy the per-task trace of the last step to host memory: 4 int64 per task
+ * (start ns, dependency met ns, end ns, sm id), in global task order.  Requires
+ * TRE_DEBUG_TRACE.  *n_tasks receives the task count; trace_host may be NULL to query. */
+tre_status tre_debug_trace(tre_engine* e, int64_t* trace_host, int32_t* n_tasks);
+
+/* Bytes a step at `pos` streams from HBM (weights + KV read + KV written + logits). */
+tre_status tre_step_bytes(const tre_engine* e, int32_t pos, int64_t* bytes);
+
+/* Plan without a GPU: run the planner for cfg on a hypothetical device with `num_sms`
+ * SMs and `smem_per_block` bytes of opt-in shared memory, and summarise the plan. */
+tre_status tre_plan_inspect(const tre_config* cfg, int32_t num_sms, int32_t smem_per_block,
+                            tre_plan_info* info);
+
+/* Human-readable text of the last host-side error of this thread. */
+const char* tre_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TRE_H */

@@ -1,0 +1,174 @@
+"""CPU ORACLE of the batch-1 decode step — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import this package.  The product (``persistent_tile_pipelined_b200``) never imports it,
+and it imports nothing from the product except the seeded input generator's recipes
+(which hold no decode arithmetic).
+
+``oracle.c`` is the plain definition of a decoder step (see its header for the readings
+of the pages and for the pins).  This module only marshals numpy arrays through ctypes.
+Every function here is pinned by ``tests/test_oracle_pins.py``; nothing is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+
+
+def lib_path(bits: int) -> str:
+    return os.path.join(_HERE, f"liboracle{bits}.so")
+
+
+def build(force: bool = False) -> None:
+    """Compile oracle.c twice (fp64 and fp32 `real`) with gcc + OpenMP."""
+    for bits, real in ((64, "double"), (32, "float")):
+        out = lib_path(bits)
+        if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+            subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                                   f"-DORC_REAL={real}", _SRC, "-o", out, "-lm"])
+
+
+class _GqaConfig(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("ffn", ctypes.c_int32),
+                ("vocab", ctypes.c_int32), ("kv_capacity", ctypes.c_int32),
+                ("rope_theta", ctypes.c_double), ("norm_eps", ctypes.c_double)]
+
+
+class _GqaLayer(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "wgate", "wup", "wdown",
+                 "k_cache", "v_cache")]
+
+
+_SLOT_NAMES = ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "wgate", "wup", "wdown")
+
+
+def _ptr(a: np.ndarray) -> ctypes.c_void_p:
+    assert a.flags.c_contiguous, "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """The oracle at one precision: bits=64 (parity reference) or bits=32."""
+
+    def __init__(self, bits: int = 64):
+        assert bits in (32, 64)
+        build()
+        self.bits = bits
+        self.real = np.float64 if bits == 64 else np.float32
+        self.lib = ctypes.CDLL(lib_path(bits))
+        L = self.lib
+        vp, i32, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        creal = ctypes.c_double if bits == 64 else ctypes.c_float
+        L.orc_real_bytes.restype = ctypes.c_int
+        assert L.orc_real_bytes() == bits // 8
+        L.orc_bf16_to_real.argtypes = [ctypes.c_uint16]
+        L.orc_bf16_to_real.restype = creal
+        L.orc_round_bf16.argtypes = [creal]
+        L.orc_round_bf16.restype = ctypes.c_uint16
+        L.orc_rmsnorm.argtypes = [i32, vp, vp, dbl, vp]
+        L.orc_gemv.argtypes = [i32, i32, vp, vp, vp]
+        L.orc_rope.argtypes = [i32, i32, dbl, vp]
+        L.orc_silu.argtypes = [creal]
+        L.orc_silu.restype = creal
+        L.orc_attention.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+        L.orc_argmax.argtypes = [i32, vp]
+        L.orc_argmax.restype = i32
+        L.orc_gqa_layer_step.argtypes = [vp, vp, i32, vp]
+        L.orc_gqa_layers_step.argtypes = [vp, vp, i32, vp, vp]
+        L.orc_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp]
+
+    # -- pieces ------------------------------------------------------------------
+    def _r(self, a) -> np.ndarray:
+        return np.ascontiguousarray(a, dtype=self.real)
+
+    def round_bf16(self, v: float) -> int:
+        return int(self.lib.orc_round_bf16(v))
+
+    def bf16_to_real(self, w: int) -> float:
+        return float(self.lib.orc_bf16_to_real(w))
+
+    def rmsnorm(self, x, g_bf16, eps):
+        x = self._r(x)
+        g = np.ascontiguousarray(g_bf16, dtype=np.uint16)
+        out = np.empty_like(x)
+        self.lib.orc_rmsnorm(x.size, _ptr(x), _ptr(g), float(eps), _ptr(out))
+        return out
+
+    def gemv(self, W_bf16, x):
+        W = np.ascontiguousarray(W_bf16, dtype=np.uint16)
+        x = self._r(x)
+        N, K = W.shape
+        assert x.size == K
+        y = np.empty(N, dtype=self.real)
+        self.lib.orc_gemv(N, K, _ptr(W), _ptr(x), _ptr(y))
+        return y
+
+    def rope(self, v, pos, theta):
+        v = self._r(v).copy()
+        self.lib.orc_rope(v.size, int(pos), float(theta), _ptr(v))
+        return v
+
+    def silu(self, z: float) -> float:
+        return float(self.lib.orc_silu(z))
+
+    def attention(self, q, k_cache, v_cache, P, want_probs=False):
+        """q [Hq][D]; caches [Hkv][cap][D] bf16 words; attends positions [0, P)."""
+        q = self._r(q)
+        kc = np.ascontiguousarray(k_cache, dtype=np.uint16)
+        vc = np.ascontiguousarray(v_cache, dtype=np.uint16)
+        Hq, D = q.shape
+        Hkv, cap, D2 = kc.shape
+        assert D2 == D and vc.shape == kc.shape and 0 <= P <= cap
+        out = np.empty((Hq, D), dtype=self.real)
+        probs = np.empty((Hq, max(P, 1)), dtype=self.real) if want_probs else None
+        self.lib.orc_attention(Hq, Hkv, D, int(P), cap, _ptr(q), _ptr(kc), _ptr(vc), _ptr(out),
+                               _ptr(probs) if probs is not None else None)
+        return (out, probs[:, :P]) if want_probs else out
+
+    def argmax(self, v) -> int:
+        v = self._r(v)
+        return int(self.lib.orc_argmax(v.size, _ptr(v)))
+
+    # -- the stack ---------------------------------------------------------------
+    def _gqa_structs(self, wl, model):
+        cfg = _GqaConfig(wl.n_layers, wl.hidden, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                         wl.ffn, wl.vocab, wl.kv_capacity, float(wl.rope_theta),
+                         float(wl.norm_eps))
+        layers = (_GqaLayer * wl.n_layers)()
+        for l in range(wl.n_layers):
+            t = model["layers"][l]
+            for slot, name in enumerate(_SLOT_NAMES):
+                setattr(layers[l], name, _ptr(t[slot]).value)
+            layers[l].k_cache = _ptr(model["k_cache"][l]).value
+            layers[l].v_cache = _ptr(model["v_cache"][l]).value
+        return cfg, layers
+
+    def decode_step(self, wl, model, token: int, pos: int, want_hidden: bool = True):
+        """One decode step; writes this token's k, v into model's caches at pos.
+        Returns (logits[V], hidden[L][d] or None)."""
+        cfg, layers = self._gqa_structs(wl, model)
+        logits = np.empty(wl.vocab, dtype=self.real)
+        hidden = np.empty((wl.n_layers, wl.hidden), dtype=self.real) if want_hidden else None
+        self.lib.orc_decode_step(ctypes.byref(cfg), _ptr(model["embed"]),
+                                 _ptr(model["final_norm"]), _ptr(model["lm_head"]), layers,
+                                 int(token), int(pos), _ptr(logits),
+                                 _ptr(hidden) if hidden is not None else None)
+        return logits, hidden
+
+    def layers_step(self, wl, model, x, pos: int):
+        """Layers only: returns (x_out[d], hidden[L][d])."""
+        cfg, layers = self._gqa_structs(wl, model)
+        x = self._r(x).copy()
+        hidden = np.empty((wl.n_layers, wl.hidden), dtype=self.real)
+        self.lib.orc_gqa_layers_step(ctypes.byref(cfg), layers, int(pos), _ptr(x), _ptr(hidden))
+        return x, hidden

@@ -1,0 +1,238 @@
+/*
+ * oracle.c — the CPU ORACLE of the batch-1 decode step.  TEST INFRASTRUCTURE ONLY:
+ * nothing in the product links or calls it; the tests, the smoke check and the
+ * CPU-baseline leg of the benchmark do.  It shares no code, header, table or constant
+ * with the GPU engine.
+ *
+ * It is the plain definition of one decoder forward step, written out with loops in
+ * the order the math states, with no blocking, fusion or reordering.  Compiled twice:
+ * ORC_REAL=double (liboracle64.so, the parity reference) and ORC_REAL=float
+ * (liboracle32.so, the fp32 decoder stack).  OpenMP only splits independent output rows
+ * (matrix-vector rows, attention heads) across threads.
+ *
+ * What the pages fix and what is read into them.  The pages name the fused ops whose
+ * math this is — RMSNorm + QKV projection ("rmsnorm_projx_wqkvia", Static Compilation
+ * for LLM Inference §5.4; "RMSNormProjxWqkvia", TileRT code audit, fused-op list),
+ * output projection ("UnProjO…"), expert select + up/gate + SiLU and expert down
+ * (TileRT code audit, blog-vs-code table and MoE section), the batch-1 decode
+ * attention ("FlashSparseMLA", batch == 1) — but print no formula.  The standard
+ * Llama-style decoder math is taken: RMSNorm x*g/sqrt(mean(x^2)+eps), half-split RoPE
+ * with theta_i = theta^(-2i/D), softmax(q.k/sqrt(D)) attention with q head h reading kv
+ * head h / (Hq/Hkv), SwiGLU silu(Wg x)*(Wu x), residual adds, final RMSNorm and LM
+ * head.  Storage: weights, gains, embedding and KV cache are bf16; the k and v of the
+ * current token are rounded to bf16 when appended to the cache and read back from it;
+ * every other value stays in `real`.
+ *
+ * Pins (tests/test_oracle_pins.py): bf16 rounding vs torch and vs the two neighbours;
+ * RMSNorm unit RMS; matrix-vector vs numpy matmul; RoPE identity at pos 0, norm
+ * preservation, relative-position property and the complex-rotation form; attention
+ * brute force in pure Python, one position returns V, equal keys return the mean of V,
+ * softmax rows sum to 1; SiLU special values; the decode step against closed forms
+ * when Wo / Wdown are zero, at pos 0, and under hidden-unit / head permutations.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef ORC_REAL
+#define ORC_REAL double
+#endif
+typedef ORC_REAL real;
+
+/* ------------------------------------------------------------------ storage -------- */
+
+/* bf16 word -> value: the word is the upper half of an IEEE binary32. */
+static real bf16_val(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (real)f;
+}
+
+real orc_bf16_to_real(uint16_t h) { return bf16_val(h); }
+
+/* value -> bf16 word, round to nearest, ties to even, directly from `real` (no
+ * intermediate rounding): keep 8 significant bits of the binary significand. */
+uint16_t orc_round_bf16(real v) {
+  double x = (double)v;
+  if (isnan(x)) return 0x7fc0;
+  if (x == 0.0) return signbit(x) ? 0x8000 : 0x0000;
+  int e;
+  double m = frexp(fabs(x), &e);          /* |x| = m * 2^e, m in [0.5, 1)          */
+  if (e < -125) {                          /* below binary32's normal range: the     */
+    double q = ldexp(1.0, -133);           /* bf16 subnormal step is 2^-133          */
+    double r = nearbyint(fabs(x) / q) * q;
+    float f = (float)r;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)((u >> 16) | (signbit(x) ? 0x8000 : 0));
+  }
+  double r = ldexp(nearbyint(ldexp(m, 8)), e - 8); /* 8 significant bits, RNE        */
+  float f = (float)r;                      /* exact unless it overflows to inf       */
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  u |= signbit(x) ? 0x80000000u : 0u;
+  return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------ pieces --------- */
+
+/* RMSNorm: out = x * g / sqrt(mean(x^2) + eps). */
+void orc_rmsnorm(int n, const real* x, const uint16_t* g, double eps, real* out) {
+  real ss = 0;
+  for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+  real r = (real)(1.0 / sqrt((double)ss / n + eps));
+  for (int i = 0; i < n; ++i) out[i] = x[i] * r * bf16_val(g[i]);
+}
+
+/* y = W x, W row-major [N][K] bf16. */
+void orc_gemv(int N, int K, const uint16_t* W, const real* x, real* y) {
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n) {
+    const uint16_t* row = W + (size_t)n * K;
+    real acc = 0;
+    for (int k = 0; k < K; ++k) acc += bf16_val(row[k]) * x[k];
+    y[n] = acc;
+  }
+}
+
+/* Half-split rotary embedding of one head vector v[D] at position pos: the pair
+ * (v[i], v[i + D/2]) is rotated by the angle pos * theta^(-2i/D). */
+void orc_rope(int D, int pos, double theta, real* v) {
+  int h = D / 2;
+  for (int i = 0; i < h; ++i) {
+    double ang = (double)pos * pow(theta, -2.0 * i / D);
+    real c = (real)cos(ang), s = (real)sin(ang);
+    real x0 = v[i], x1 = v[i + h];
+    v[i] = x0 * c - x1 * s;
+    v[i + h] = x0 * s + x1 * c;
+  }
+}
+
+real orc_silu(real z) { return z / ((real)1 + (real)exp(-(double)z)); }
+
+/* Decode attention of Hq query heads over P cached positions of Hkv kv heads.
+ * Cache layout [Hkv][cap][D] bf16.  Query head h reads kv head h / (Hq / Hkv).
+ * out[h*D + d] = sum_t p_t V[t][d],  p = softmax_t(q_h . K[t] / sqrt(D)).
+ * probs (optional, [Hq][P]) receives p. */
+void orc_attention(int Hq, int Hkv, int D, int P, int cap, const real* q,
+                   const uint16_t* kc, const uint16_t* vc, real* out, real* probs) {
+  int G = Hq / Hkv;
+  real scale = (real)(1.0 / sqrt((double)D));
+#pragma omp parallel for schedule(static)
+  for (int h = 0; h < Hq; ++h) {
+    int g = h / G;
+    real* s = (real*)malloc(sizeof(real) * (size_t)(P > 0 ? P : 1));
+    real m = -INFINITY;
+    for (int t = 0; t < P; ++t) {
+      const uint16_t* krow = kc + ((size_t)g * cap + t) * D;
+      real acc = 0;
+      for (int d = 0; d < D; ++d) acc += q[(size_t)h * D + d] * bf16_val(krow[d]);
+      s[t] = acc * scale;
+      if (s[t] > m) m = s[t];
+    }
+    real l = 0;
+    for (int t = 0; t < P; ++t) {
+      s[t] = (real)exp((double)(s[t] - m));
+      l += s[t];
+    }
+    for (int t = 0; t < P; ++t) s[t] /= l;
+    for (int d = 0; d < D; ++d) {
+      real acc = 0;
+      for (int t = 0; t < P; ++t) acc += s[t] * bf16_val(vc[((size_t)g * cap + t) * D + d]);
+      out[(size_t)h * D + d] = acc;
+    }
+    if (probs)
+      for (int t = 0; t < P; ++t) probs[(size_t)h * P + t] = s[t];
+    free(s);
+  }
+}
+
+int orc_argmax(int n, const real* v) {
+  int best = 0;
+  for (int i = 1; i < n; ++i)
+    if (v[i] > v[best]) best = i;
+  return best;
+}
+
+/* ------------------------------------------------------------------ the stack ------ */
+
+typedef struct {
+  int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab, kv_capacity;
+  double rope_theta, norm_eps;
+} orc_gqa_config;
+
+typedef struct {
+  const uint16_t *attn_norm, *wq, *wk, *wv, *wo, *ffn_norm, *wgate, *wup, *wdown;
+  uint16_t *k_cache, *v_cache; /* [Hkv][cap][D] bf16, written at pos */
+} orc_gqa_layer;
+
+/* One pre-norm GQA decoder layer at position pos, residual x[d] updated in place:
+ *   xn = RMSNorm(x); q,k,v = Wq xn, Wk xn, Wv xn; RoPE(q, k at pos);
+ *   cache[pos] = bf16(k), bf16(v); o = attention over positions [0, pos];
+ *   h1 = x + Wo o; x = h1 + Wdown (silu(Wgate RMSNorm(h1)) * (Wup RMSNorm(h1))). */
+void orc_gqa_layer_step(const orc_gqa_config* c, const orc_gqa_layer* L, int pos, real* x) {
+  int d = c->hidden, Hq = c->n_q_heads, Hkv = c->n_kv_heads, D = c->head_dim, F = c->ffn;
+  int cap = c->kv_capacity;
+  real* xn = (real*)malloc(sizeof(real) * d);
+  real* q = (real*)malloc(sizeof(real) * (size_t)Hq * D);
+  real* k = (real*)malloc(sizeof(real) * (size_t)Hkv * D);
+  real* v = (real*)malloc(sizeof(real) * (size_t)Hkv * D);
+  real* o = (real*)malloc(sizeof(real) * (size_t)Hq * D);
+  real* h1 = (real*)malloc(sizeof(real) * d);
+  real* g = (real*)malloc(sizeof(real) * F);
+  real* u = (real*)malloc(sizeof(real) * F);
+  real* y = (real*)malloc(sizeof(real) * d);
+
+  orc_rmsnorm(d, x, L->attn_norm, c->norm_eps, xn);
+  orc_gemv(Hq * D, d, L->wq, xn, q);
+  orc_gemv(Hkv * D, d, L->wk, xn, k);
+  orc_gemv(Hkv * D, d, L->wv, xn, v);
+  for (int h = 0; h < Hq; ++h) orc_rope(D, pos, c->rope_theta, q + (size_t)h * D);
+  for (int h = 0; h < Hkv; ++h) orc_rope(D, pos, c->rope_theta, k + (size_t)h * D);
+  for (int h = 0; h < Hkv; ++h)
+    for (int i = 0; i < D; ++i) {
+      L->k_cache[((size_t)h * cap + pos) * D + i] = orc_round_bf16(k[(size_t)h * D + i]);
+      L->v_cache[((size_t)h * cap + pos) * D + i] = orc_round_bf16(v[(size_t)h * D + i]);
+    }
+  orc_attention(Hq, Hkv, D, pos + 1, cap, q, L->k_cache, L->v_cache, o, NULL);
+  orc_gemv(d, Hq * D, L->wo, o, y);
+  for (int i = 0; i < d; ++i) h1[i] = x[i] + y[i];
+
+  orc_rmsnorm(d, h1, L->ffn_norm, c->norm_eps, xn);
+  orc_gemv(F, d, L->wgate, xn, g);
+  orc_gemv(F, d, L->wup, xn, u);
+  for (int i = 0; i < F; ++i) g[i] = orc_silu(g[i]) * u[i];
+  orc_gemv(d, F, L->wdown, g, y);
+  for (int i = 0; i < d; ++i) x[i] = h1[i] + y[i];
+
+  free(xn); free(q); free(k); free(v); free(o); free(h1); free(g); free(u); free(y);
+}
+
+/* Layers only: x[d] in, x[d] out, hidden[l*d] (optional) after every layer. */
+void orc_gqa_layers_step(const orc_gqa_config* c, const orc_gqa_layer* layers, int pos,
+                         real* x, real* hidden) {
+  for (int l = 0; l < c->n_layers; ++l) {
+    orc_gqa_layer_step(c, &layers[l], pos, x);
+    if (hidden) memcpy(hidden + (size_t)l * c->hidden, x, sizeof(real) * c->hidden);
+  }
+}
+
+/* One batch-1 decode step of the whole stack: x = E[token]; the layers; logits =
+ * W_lm RMSNorm(x).  hidden (optional) receives the residual after every layer. */
+void orc_decode_step(const orc_gqa_config* c, const uint16_t* embed, const uint16_t* final_norm,
+                     const uint16_t* lm_head, const orc_gqa_layer* layers, int token, int pos,
+                     real* logits, real* hidden) {
+  int d = c->hidden;
+  real* x = (real*)malloc(sizeof(real) * d);
+  real* xn = (real*)malloc(sizeof(real) * d);
+  for (int i = 0; i < d; ++i) x[i] = bf16_val(embed[(size_t)token * d + i]);
+  orc_gqa_layers_step(c, layers, pos, x, hidden);
+  orc_rmsnorm(d, x, final_norm, c->norm_eps, xn);
+  orc_gemv(c->vocab, d, lm_head, xn, logits);
+  free(x);
+  free(xn);
+}
+
+int orc_real_bytes(void) { return (int)sizeof(real); }

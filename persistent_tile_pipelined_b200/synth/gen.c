@@ -1,0 +1,100 @@
+/*
+ * Seeded synthetic inputs: one counter-based generator that both the GPU engine's
+ * uploads and the CPU oracle consume, so the two sides see bit-identical bf16 data.
+ * It holds none of the decode arithmetic: it only turns (seed, tensor id, index) into
+ * numbers.
+ *
+ * Definition (every value is a pure function of seed, tensor_id and its index):
+ *   mix64      the SplitMix64 output function (Steele, Lea & Flood, "Fast splittable
+ *              pseudorandom number generators", OOPSLA 2014): two xor-shift-multiply
+ *              rounds and a final xor-shift.
+ *   key        mix64(seed + G) ^ mix64(tensor_id * G + C)        G = 0x9E3779B97F4A7C15
+ *   draw(i)    mix64(key + (i + 1) * G)                            (SplitMix64 stream)
+ *   normal     Box-Muller on the pair (draw(2p), draw(2p+1)):
+ *                u1 = ((d0 >> 11) + 1) * 2^-53  in (0, 1]
+ *                u2 =  (d1 >> 11)      * 2^-53  in [0, 1)
+ *                z[2p] = sqrt(-2 ln u1) cos(2 pi u2),  z[2p+1] = sqrt(-2 ln u1) sin(2 pi u2)
+ *              value = mean + std * z, computed in double
+ *   bf16       double -> float (C conversion, round to nearest even) -> bf16 by round to
+ *              nearest even on the upper 16 bits.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define GOLDEN 0x9E3779B97F4A7C15ULL
+#define KEYC 0x632BE59BD9B4E019ULL
+
+static inline uint64_t mix64(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+static inline uint64_t stream_key(uint64_t seed, uint64_t tensor_id) {
+  return mix64(seed + GOLDEN) ^ mix64(tensor_id * GOLDEN + KEYC);
+}
+
+static inline uint64_t draw(uint64_t key, uint64_t i) { return mix64(key + (i + 1) * GOLDEN); }
+
+static inline void normal_pair(uint64_t key, uint64_t p, double* z0, double* z1) {
+  const double two53 = 1.0 / 9007199254740992.0; /* 2^-53 */
+  uint64_t d0 = draw(key, 2 * p), d1 = draw(key, 2 * p + 1);
+  double u1 = (double)((d0 >> 11) + 1) * two53;
+  double u2 = (double)(d1 >> 11) * two53;
+  double r = sqrt(-2.0 * log(u1));
+  double a = 6.283185307179586476925286766559 * u2;
+  *z0 = r * cos(a);
+  *z1 = r * sin(a);
+}
+
+static inline uint16_t float_to_bf16_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u); /* quiet NaN */
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+uint64_t synth_u64(uint64_t seed, uint64_t tensor_id, uint64_t index) {
+  return draw(stream_key(seed, tensor_id), index);
+}
+
+void synth_normal_f64(uint64_t seed, uint64_t tensor_id, int64_t n, double mean, double std,
+                      double* out) {
+  uint64_t key = stream_key(seed, tensor_id);
+  int64_t pairs = (n + 1) / 2;
+#pragma omp parallel for schedule(static)
+  for (int64_t p = 0; p < pairs; ++p) {
+    double z0, z1;
+    normal_pair(key, (uint64_t)p, &z0, &z1);
+    out[2 * p] = mean + std * z0;
+    if (2 * p + 1 < n) out[2 * p + 1] = mean + std * z1;
+  }
+}
+
+void synth_normal_f32(uint64_t seed, uint64_t tensor_id, int64_t n, double mean, double std,
+                      float* out) {
+  uint64_t key = stream_key(seed, tensor_id);
+  int64_t pairs = (n + 1) / 2;
+#pragma omp parallel for schedule(static)
+  for (int64_t p = 0; p < pairs; ++p) {
+    double z0, z1;
+    normal_pair(key, (uint64_t)p, &z0, &z1);
+    out[2 * p] = (float)(mean + std * z0);
+    if (2 * p + 1 < n) out[2 * p + 1] = (float)(mean + std * z1);
+  }
+}
+
+void synth_normal_bf16(uint64_t seed, uint64_t tensor_id, int64_t n, double mean, double std,
+                       uint16_t* out) {
+  uint64_t key = stream_key(seed, tensor_id);
+  int64_t pairs = (n + 1) / 2;
+#pragma omp parallel for schedule(static)
+  for (int64_t p = 0; p < pairs; ++p) {
+    double z0, z1;
+    normal_pair(key, (uint64_t)p, &z0, &z1);
+    out[2 * p] = float_to_bf16_rne((float)(mean + std * z0));
+    if (2 * p + 1 < n) out[2 * p + 1] = float_to_bf16_rne((float)(mean + std * z1));
+  }
+}

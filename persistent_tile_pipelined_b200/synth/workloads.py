@@ -1,0 +1,141 @@
+"""Workload recipes: shapes, seeds and value distributions of the synthetic decode inputs.
+
+Every tensor is drawn from the seeded generator in this package (one stream per tensor
+id), so the engine's device copy and the oracle's host copy are bit-identical.
+
+Distributions (the workloads' own statement): bf16 weights N(0, 0.02); RMSNorm gains
+1 + N(0, 0.01); KV cache positions [0, prefill) N(0, 1) bf16, later positions zero until
+a decode step writes them; layer-only workloads start from a hidden vector N(0, 1) fp32.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional
+
+import numpy as np
+
+from . import (TID_EMBED, TID_FINAL_NORM, TID_LM_HEAD, TID_X_IN, normal_bf16, normal_f32,
+               tid_kcache, tid_layer, tid_vcache, token_id)
+
+W_STD = 0.02
+GAIN_STD = 0.01
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    kind: str                 # "gqa" | "mla" | "moe"
+    n_layers: int
+    hidden: int
+    n_q_heads: int
+    n_kv_heads: int = 0
+    head_dim: int = 0
+    ffn: int = 0
+    vocab: int = 0
+    prefill: int = 0          # KV positions filled before the first decode step
+    decode_steps: int = 1     # decode steps the workload runs (KV capacity = prefill + steps)
+    rope_theta: float = 1e4
+    norm_eps: float = 1e-5
+    tokens_per_step: int = 1
+    seed: int = 1234
+    # MLA
+    q_lora: int = 0
+    kv_lora: int = 0
+    rope_dim: int = 0
+    nope_dim: int = 0
+    v_dim: int = 0
+    # MoE
+    n_experts: int = 0
+    top_k: int = 0
+    n_shared: int = 0
+    expert_ffn: int = 0
+
+    @property
+    def kv_capacity(self) -> int:
+        return self.prefill + self.decode_steps * self.tokens_per_step
+
+    @property
+    def has_embed_lm_head(self) -> bool:
+        return self.vocab > 0
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# Tiny 2-layer decoder: hidden 256, 4 q / 2 kv heads of dim 64, RoPE theta 1e4, SwiGLU 688,
+# vocab 1024, KV cache 128 positions.
+TINY = Workload(name="tiny-2L-d256", kind="gqa", n_layers=2, hidden=256, n_q_heads=4,
+                n_kv_heads=2, head_dim=64, ffn=688, vocab=1024, prefill=128, decode_steps=64,
+                rope_theta=1e4, norm_eps=1e-5)
+
+# Llama-3-8B-shaped stack: 32 layers, hidden 4096, 32 q / 8 kv heads of dim 128, SwiGLU 14336,
+# vocab 128256, KV cache 4096 positions, 64 greedy decode steps.
+LLAMA8B = Workload(name="llama3-8b-shaped", kind="gqa", n_layers=32, hidden=4096, n_q_heads=32,
+                   n_kv_heads=8, head_dim=128, ffn=14336, vocab=128256, prefill=4096,
+                   decode_steps=64, rope_theta=5e5, norm_eps=1e-5)
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B)}
+
+
+def gqa_layer_shapes(w: Workload) -> List[tuple]:
+    """(slot, shape, kind) of every GQA layer tensor; kind 'w' = weight, 'g' = gain."""
+    d, hq, hkv, dh, f = w.hidden, w.n_q_heads, w.n_kv_heads, w.head_dim, w.ffn
+    return [
+        (0, (d,), "g"),                 # attention RMSNorm gain
+        (1, (hq * dh, d), "w"),         # Wq
+        (2, (hkv * dh, d), "w"),        # Wk
+        (3, (hkv * dh, d), "w"),        # Wv
+        (4, (d, hq * dh), "w"),         # Wo
+        (5, (d,), "g"),                 # MLP RMSNorm gain
+        (6, (f, d), "w"),               # W_gate
+        (7, (f, d), "w"),               # W_up
+        (8, (d, f), "w"),               # W_down
+    ]
+
+
+def gen_tensor(w: Workload, tensor_id: int, shape, kind: str,
+               out: Optional[np.ndarray] = None) -> np.ndarray:
+    if kind == "g":
+        return normal_bf16(w.seed, tensor_id, shape, 1.0, GAIN_STD, out)
+    if kind == "w":
+        return normal_bf16(w.seed, tensor_id, shape, 0.0, W_STD, out)
+    if kind == "kv":
+        return normal_bf16(w.seed, tensor_id, shape, 0.0, 1.0, out)
+    raise ValueError(kind)
+
+
+def gen_gqa_layer(w: Workload, layer: int) -> Dict[int, np.ndarray]:
+    return {slot: gen_tensor(w, tid_layer(layer, slot), shape, kind)
+            for slot, shape, kind in gqa_layer_shapes(w)}
+
+
+def gen_kv_cache(w: Workload, layer: int, which: str) -> np.ndarray:
+    """[Hkv][capacity][D] bf16 words; positions < prefill drawn N(0,1), the rest zero."""
+    cap, hkv, dh = w.kv_capacity, w.n_kv_heads, w.head_dim
+    out = np.zeros((hkv, cap, dh), dtype=np.uint16)
+    tid = tid_kcache(layer) if which == "k" else tid_vcache(layer)
+    if w.prefill:
+        pre = normal_bf16(w.seed, tid, (hkv, w.prefill, dh), 0.0, 1.0)
+        out[:, : w.prefill, :] = pre
+    return out
+
+
+def gen_gqa_model(w: Workload) -> dict:
+    """All host tensors of a GQA decoder workload (bf16 words as uint16 arrays)."""
+    assert w.kind == "gqa"
+    model = {
+        "layers": [gen_gqa_layer(w, l) for l in range(w.n_layers)],
+        "k_cache": [gen_kv_cache(w, l, "k") for l in range(w.n_layers)],
+        "v_cache": [gen_kv_cache(w, l, "v") for l in range(w.n_layers)],
+    }
+    if w.has_embed_lm_head:
+        model["embed"] = gen_tensor(w, TID_EMBED, (w.vocab, w.hidden), "w")
+        model["final_norm"] = gen_tensor(w, TID_FINAL_NORM, (w.hidden,), "g")
+        model["lm_head"] = gen_tensor(w, TID_LM_HEAD, (w.vocab, w.hidden), "w")
+    else:
+        model["x_in"] = normal_f32(w.seed, TID_X_IN, (w.hidden,), 0.0, 1.0)
+    return model
+
+
+def first_token(w: Workload) -> int:
+    return token_id(w.seed, w.vocab)
