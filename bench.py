@@ -1,0 +1,411 @@
+"""Benchmark: batch-1 decode tokens/s and achieved HBM GB/s of the persistent engine.
+
+Workload: the Llama-3-8B-shaped stack (32 layers, hidden 4096, 32 q / 8 kv heads of dim
+128, SwiGLU 14336, vocab 128256), bf16 random-init weights N(0, 0.02), KV cache of 4096
+positions N(0, 1) bf16, batch 1.  One step = one decode step of the whole stack = one
+launch of the persistent engine kernel.  Inputs are synthetic (seeded generator) and
+resident in HBM; every step streams ~15.5 GB, far more than the 126 MB L2, so no flush
+is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl engine|reference]
+
+For N > 1 it runs under torch.distributed.run, one process per GPU; the path does not
+shard, so every rank runs an independent replica (no collective on the data path) and
+`value` is the sum over ranks of tokens / the slowest rank's time.
+
+Numbers printed (one JSON line on rank 0):
+  value        tokens/s over the K timed steps, launches back to back on the device
+               (CUDA events on the launching stream, barrier + synchronize on both sides,
+               max over ranks)
+  e2e          the greedy generation loop through the C ABI call tre_decode_step_host:
+               the token goes in as a kernel argument, the argmax token comes back to the
+               host every step; host wall time, max over ranks
+  roofline     the engine kernel's algorithmic bytes per launch / average launch time,
+               against the measured HBM copy bandwidth of this machine
+  cpu_baseline the CPU oracle (tests-only code) timed on this machine's cores on a bounded
+               sample of the same workload (rank 0, N = 1)
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "batch-1 decode tokens/s and achieved HBM GB/s (fraction of ~8 TB/s roofline)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="engine", choices=["engine", "reference"])
+    ap.add_argument("--workload", default="llama3-8b-shaped")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-layers", type=int, default=4)
+    ap.add_argument("--trace", default="", help="write a per-task trace of one step (JSON)")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "persistent_tile_pipelined_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "engine_kernel_llama8b.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m_src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
+    m_tr = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", txt)
+    if not (m_src and m_tr) or m_src.group(1) != kernel_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed regions run."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.windows = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "50"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if self.windows and not any(a - 0.05 <= ts <= b + 0.05 for a, b in self.windows):
+                continue
+            try:
+                sm.append(float(parts[2]))
+                mx = float(parts[3])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload -------------
+
+def build_engine(wl, device: int, debug_flags: int = 0):
+    """Generate the synthetic model tensor by tensor (host generator -> device) so the
+    host holds at most one tensor at a time."""
+    import torch
+
+    from persistent_tile_pipelined_b200 import tre
+    from persistent_tile_pipelined_b200.synth import (TID_EMBED, TID_FINAL_NORM, TID_LM_HEAD,
+                                                      tid_layer)
+    from persistent_tile_pipelined_b200.synth import workloads as W
+
+    dev = f"cuda:{device}"
+
+    def up(words):
+        t = torch.from_numpy(words.view(np.int16)).view(torch.bfloat16)
+        return t.to(dev)
+
+    model = {"layers": [], "k_cache": [], "v_cache": []}
+    for l in range(wl.n_layers):
+        model["layers"].append({slot: up(W.gen_tensor(wl, tid_layer(l, slot), shape, kind))
+                                for slot, shape, kind in W.gqa_layer_shapes(wl)})
+        model["k_cache"].append(up(W.gen_kv_cache(wl, l, "k")))
+        model["v_cache"].append(up(W.gen_kv_cache(wl, l, "v")))
+    model["embed"] = up(W.gen_tensor(wl, TID_EMBED, (wl.vocab, wl.hidden), "w"))
+    model["final_norm"] = up(W.gen_tensor(wl, TID_FINAL_NORM, (wl.hidden,), "g"))
+    model["lm_head"] = up(W.gen_tensor(wl, TID_LM_HEAD, (wl.vocab, wl.hidden), "w"))
+    torch.cuda.synchronize(device)
+    cfg = tre.config_from_workload(wl, debug_flags=debug_flags)
+    return tre.Engine(cfg, model, device), model
+
+
+def cpu_baseline(wl, sample_layers: int, reps: int = 1):
+    """The oracle (as it stands) on this machine's cores: one decode step of a
+    `sample_layers`-layer slice of the workload (same layer shapes, same LM head, same KV
+    length) and the same slice's layers alone; the full 32-layer step time is scaled from
+    the per-layer time plus the embedding / final-norm / LM-head time.  With reps > 1 the
+    sample is timed reps times on one generated model and the list is returned."""
+    import oracle
+    from persistent_tile_pipelined_b200.synth import workloads as W
+
+    sw = wl.replace(n_layers=sample_layers, decode_steps=1)
+    model = W.gen_gqa_model(sw)
+    orc = oracle.Oracle(32)
+    if reps > 1:
+        return [_time_sample(orc, wl, sw, model, sample_layers) for _ in range(reps)]
+    return _time_sample(orc, wl, sw, model, sample_layers)
+
+
+def _time_sample(orc, wl, sw, model, sample_layers):
+    from persistent_tile_pipelined_b200.synth import workloads as W
+    tok = W.first_token(sw)
+    t0 = time.perf_counter()
+    orc.decode_step(sw, model, tok, sw.prefill, want_hidden=False)
+    t_step = time.perf_counter() - t0
+    x = np.zeros(sw.hidden, dtype=np.float32)
+    t0 = time.perf_counter()
+    orc.layers_step(sw, model, x + 0.01, sw.prefill)
+    t_layers = time.perf_counter() - t0
+    per_layer = t_layers / sample_layers
+    t_full = per_layer * wl.n_layers + max(t_step - t_layers, 0.0)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": 1.0 / t_full, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"fp32 oracle, {sample_layers} of {wl.n_layers} layers + LM head, one "
+                       f"decode step at pos {sw.prefill} (step {t_step:.2f} s, layers-only "
+                       f"{t_layers:.2f} s), scaled to the full stack: {t_full:.2f} s/token"),
+            "seconds_per_token": t_full}
+
+
+# ---------------------------------------------------------------- engine arm ----------
+
+def run_engine(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from persistent_tile_pipelined_b200.synth import token_id
+    from persistent_tile_pipelined_b200.synth import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    wl = W.WORKLOADS[args.workload]
+    K, Wm = args.steps, args.warmup
+    wl = wl.replace(decode_steps=K + Wm, seed=wl.seed + rank)
+    eng, model = build_engine(wl, local_rank)
+    stream = torch.cuda.current_stream(local_rank)
+    s_ptr = stream.cuda_stream
+    tokens = [token_id(wl.seed, wl.vocab, i) for i in range(K + Wm)]
+    positions = [wl.prefill + i for i in range(K + Wm)]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(local_rank)
+
+    # warm-up
+    for i in range(Wm):
+        eng.step(tokens[i], positions[i], stream=s_ptr)
+    torch.cuda.synchronize(local_rank)
+    assert eng.status() == (0, 0), eng.status()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.2)
+
+    # ---- device-timed region: K launches back to back
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    barrier()
+    tw0 = time.time()
+    ev[0].record(stream)
+    for i in range(K):
+        eng.step(tokens[Wm + i], positions[Wm + i], stream=s_ptr)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(local_rank)
+    tw1 = time.time()
+    barrier()
+    sampler.mark(tw0, tw1)
+    dev_s = ev[0].elapsed_time(ev[K]) / 1e3
+    launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    st = eng.status()
+    assert st == (0, 0), st
+
+    # ---- end to end through the C ABI: greedy loop, token back to the host every step
+    tok = tokens[0]
+    barrier()
+    tw0 = time.time()
+    t0 = time.perf_counter()
+    for i in range(K):
+        tok = eng.step_host(tok, positions[Wm + i], stream=s_ptr)
+    e2e_s = time.perf_counter() - t0
+    tw1 = time.time()
+    barrier()
+    sampler.mark(tw0, tw1)
+    clocks = sampler.stop()
+
+    step_bytes = float(np.mean([eng.step_bytes(positions[Wm + i]) for i in range(K)]))
+    trace_path = args.trace if rank == 0 else ""
+    eng.close()
+    del model
+    torch.cuda.empty_cache()
+
+    if trace_path:
+        write_trace(wl, local_rank, trace_path)
+
+    t = torch.tensor([dev_s, e2e_s, float(np.mean(launch_ms))], dtype=torch.float64,
+                     device=f"cuda:{local_rank}")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev_s, e2e_s, launch_ms_avg = t.tolist()
+    return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
+
+
+def write_trace(wl, device, path):
+    """One traced step (debug flag on a fresh engine): per-task start / ready / end."""
+    import torch
+
+    from persistent_tile_pipelined_b200 import tre
+    eng, model = build_engine(wl.replace(decode_steps=2), device, tre.TRE_DEBUG_TRACE)
+    eng.step(1, wl.prefill)
+    eng.step(2, wl.prefill + 1)
+    torch.cuda.synchronize(device)
+    tr = eng.trace()
+    eng.close()
+    with open(path, "w") as f:
+        json.dump({"workload": wl.name, "trace": tr.tolist()}, f)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus:
+        args.gpus = world
+
+    if args.impl == "reference":
+        return main_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device(f"cuda:{local_rank}"))
+    wl, dev_s, e2e_s, launch_ms, step_bytes, clocks = run_engine(args, rank, world, local_rank)
+    K = args.steps
+    peak, peak_kind = peaks()
+    achieved = step_bytes / (launch_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": world * K / dev_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": dev_s / K * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
+        "config": {
+            "workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions",
+            "layers": wl.n_layers, "hidden": wl.hidden, "q_heads": wl.n_q_heads,
+            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "ffn": wl.ffn,
+            "vocab": wl.vocab, "kv_positions": wl.prefill, "batch": 1,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"not flushed: each step streams {step_bytes / 1e9:.2f} GB >> 126 MB L2",
+        },
+        "hbm_gbs": step_bytes / (dev_s / K) / 1e9,
+        "hbm_frac_of_8tbs": step_bytes / (dev_s / K) / 1e9 / NOMINAL_HBM_GBS,
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": peak_kind,
+            "traffic": profiled_traffic(args.workload),
+            "kernel": "tre::engine_kernel",
+            "algorithmic_bytes_per_launch": step_bytes,
+        },
+        "e2e": {"value": world * K / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 4,
+                "d2h_bytes_per_step": 4,
+                "note": "greedy loop via tre_decode_step_host: token in as a kernel argument, "
+                        "argmax token back to pinned-less host memory, host wall time"},
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_layers)
+        except Exception as exc:  # report, do not hide
+            line["cpu_baseline"] = {"error": repr(exc)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on this machine's host cores, on a
+    bounded sample per step of the same workload.  Rank 0 only."""
+    if rank != 0:
+        return
+    from persistent_tile_pipelined_b200.synth import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    K = max(2, min(args.steps, 3))
+    vals = cpu_baseline(wl, args.cpu_sample_layers, reps=K)
+    v = float(np.median([x["value"] for x in vals]))
+    line = {
+        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": 0, "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions",
+                   "batch": 1, "parallelism": "host cores"},
+        "impl": "reference",
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
+                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

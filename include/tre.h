@@ -205,6 +205,14 @@ tre_status tre_step_bytes(const tre_engine* e, int32_t pos, int64_t* bytes);
 tre_status tre_plan_inspect(const tre_config* cfg, int32_t num_sms, int32_t smem_per_block,
                             tre_plan_info* info);
 
+/* Plan without a GPU and dump the task descriptors: 8 int32 per task in per-SM queue
+ * order — word 0 packs type (bits 0-7), op (8-15) and layer (16-31); then dep, dep_count,
+ * out, r0, r1, aux, id — and the per-SM queue offsets (num_sms + 1 int32).  Returns the
+ * task count or a negative tre_status; out_tasks is written only when max_tasks is at
+ * least the task count, out_sm_begin whenever it is not NULL. */
+int32_t tre_plan_tasks(const tre_config* cfg, int32_t num_sms, int32_t smem_per_block,
+                       int32_t* out_tasks, int32_t max_tasks, int32_t* out_sm_begin);
+
 /* Human-readable text of the last host-side error of this thread. */
 const char* tre_last_error(void);
 

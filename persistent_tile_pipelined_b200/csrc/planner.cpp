@@ -1,0 +1,288 @@
+// Host AOT planner: flattens the decoder stack into a static list of tile tasks.
+//
+// The pages' engine is compiled ahead of time: the whole model is unrolled into one
+// persistent kernel whose scheduling unit is the tile (Static Compilation for LLM
+// Inference, §1 and §5.1), and the dataflow graph is lowered to tile micro-kernels plus
+// an engine that maps tasks onto hardware units (Speed is intelligence talk, section on
+// breaking the kernel boundary).  This planner is that step for one GPU:
+//
+//   * every GEMV op (Q, K, V, O, gate/up, down, LM head) is cut into one contiguous row
+//     range per SM; ranges are sized so that each SM's cumulative streamed bytes over
+//     the step stay level (the SMs then finish every op at about the same time);
+//   * the attention of each layer is cut into (kv head, KV split) tasks, placed on the
+//     SMs with the least streamed bytes so far;
+//   * each task waits on one counter (the op it reads from, all of its tasks) and bumps
+//     one counter; counters only grow, so step e waits for e * count;
+//   * each SM's queue is in global topological order, so with every CTA resident the
+//     lowest unfinished task always has its inputs ready (no deadlock).
+#include <algorithm>
+#include <cmath>
+#include <numeric>
+#include <string>
+#include <vector>
+
+#include "tre_internal.h"
+
+namespace tre {
+
+static thread_local std::string g_err;
+void set_error(const std::string& m) { g_err = m; }
+const char* last_error_cstr() { return g_err.c_str(); }
+
+static tre_status fail(tre_status s, const std::string& m) {
+  set_error(m);
+  return s;
+}
+
+static inline int counter_of(int layer, int kind) { return layer * C_PER_LAYER + kind; }
+
+// Split N rows of `row_bytes` each over the SMs, levelling cumulative bytes `cum`.
+static std::vector<std::pair<int, int>> assign_rows(int N, int64_t row_bytes,
+                                                    std::vector<int64_t>& cum) {
+  const int n = (int)cum.size();
+  double total = (double)N * (double)row_bytes;
+  for (int64_t c : cum) total += (double)c;
+  const double target = total / n;
+  std::vector<double> want(n);
+  double sw = 0;
+  for (int i = 0; i < n; ++i) {
+    want[i] = std::max(0.0, (target - (double)cum[i]) / (double)row_bytes);
+    sw += want[i];
+  }
+  for (int i = 0; i < n; ++i) want[i] = sw > 0 ? want[i] * N / sw : (double)N / n;
+  std::vector<int> rows(n);
+  int s = 0;
+  for (int i = 0; i < n; ++i) {
+    rows[i] = (int)std::floor(want[i]);
+    s += rows[i];
+  }
+  std::vector<int> idx(n);
+  std::iota(idx.begin(), idx.end(), 0);
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) {
+    double fa = want[a] - rows[a], fb = want[b] - rows[b];
+    if (fa != fb) return fa > fb;
+    return cum[a] < cum[b];
+  });
+  for (int k = 0; s < N; ++k, ++s) rows[idx[k % n]]++;
+  std::vector<std::pair<int, int>> ranges(n);
+  int r = 0;
+  for (int i = 0; i < n; ++i) {
+    ranges[i] = {r, r + rows[i]};
+    r += rows[i];
+    cum[i] += (int64_t)rows[i] * row_bytes;
+  }
+  return ranges;
+}
+
+struct Builder {
+  int nsm;
+  std::vector<std::vector<Task>> q;  // per SM
+  std::vector<int64_t> cum;          // streamed bytes per SM
+  int next_id = 0;
+
+  explicit Builder(int n) : nsm(n), q(n), cum(n, 0) {}
+
+  Task make(uint8_t type, uint8_t op, int layer, int dep, uint32_t dep_count, int out) {
+    Task t{};
+    t.type = type;
+    t.op = op;
+    t.layer = (uint16_t)layer;
+    t.dep = dep;
+    t.dep_count = dep_count;
+    t.out = out;
+    t.id = next_id++;
+    return t;
+  }
+
+  // Returns the number of tasks created.
+  int gemv(uint8_t op, int layer, int N, int64_t row_bytes, int dep, uint32_t dep_count,
+           int out) {
+    auto ranges = assign_rows(N, row_bytes, cum);
+    int n = 0;
+    for (int s = 0; s < nsm; ++s) {
+      if (ranges[s].second <= ranges[s].first) continue;
+      Task t = make(T_GEMV, op, layer, dep, dep_count, out);
+      t.r0 = ranges[s].first;
+      t.r1 = ranges[s].second;
+      q[s].push_back(t);
+      ++n;
+    }
+    return n;
+  }
+
+  void attention(int layer, int Hkv, int S, int64_t bytes_per_task, int dep, uint32_t dep_count,
+                 int out) {
+    for (int g = 0; g < Hkv; ++g)
+      for (int s = 0; s < S; ++s) {
+        int best = (int)(std::min_element(cum.begin(), cum.end()) - cum.begin());
+        Task t = make(T_ATTN, 0, layer, dep, dep_count, out);
+        t.r0 = g;
+        t.r1 = s;
+        t.aux = S;
+        q[best].push_back(t);
+        cum[best] += bytes_per_task;
+      }
+  }
+};
+
+static tre_status validate(const tre_config& c) {
+  if (c.kind == TRE_LAYER_MLA || c.kind == TRE_LAYER_MOE)
+    return fail(TRE_ERR_UNSUPPORTED, "layer kind not implemented in this build (GQA only)");
+  if (c.kind != TRE_LAYER_GQA) return fail(TRE_ERR_INVALID_ARG, "unknown layer kind");
+  for (int r : c.reserved)
+    if (r != 0) return fail(TRE_ERR_INVALID_ARG, "reserved config fields must be zero");
+  if (c.n_layers < 1 || c.n_layers > 1024) return fail(TRE_ERR_INVALID_ARG, "n_layers out of range");
+  if (c.hidden < 8 || c.hidden % 8) return fail(TRE_ERR_INVALID_ARG, "hidden must be a positive multiple of 8");
+  if (c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads)
+    return fail(TRE_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+  int G = c.n_q_heads / c.n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(TRE_ERR_UNSUPPORTED, "q heads per kv head must be 1, 2, 4 or 8");
+  if (c.head_dim != 64 && c.head_dim != 128)
+    return fail(TRE_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (c.ffn < 8 || c.ffn % 8) return fail(TRE_ERR_INVALID_ARG, "ffn must be a positive multiple of 8");
+  if (c.has_embed_lm_head != 0 && c.has_embed_lm_head != 1)
+    return fail(TRE_ERR_INVALID_ARG, "has_embed_lm_head must be 0 or 1");
+  if (c.has_embed_lm_head && c.vocab < 1) return fail(TRE_ERR_INVALID_ARG, "vocab must be >= 1");
+  if (c.kv_capacity < 1) return fail(TRE_ERR_INVALID_ARG, "kv_capacity must be >= 1");
+  if (c.max_tokens_per_step > 1)
+    return fail(TRE_ERR_UNSUPPORTED, "multi-token steps are not implemented in this build");
+  if (c.max_tokens_per_step < 0) return fail(TRE_ERR_INVALID_ARG, "max_tokens_per_step < 0");
+  if (!(c.rope_theta > 0.f)) return fail(TRE_ERR_INVALID_ARG, "rope_theta must be > 0");
+  if (!(c.norm_eps >= 0.f)) return fail(TRE_ERR_INVALID_ARG, "norm_eps must be >= 0");
+  if (c.dep_timeout_us < 0) return fail(TRE_ERR_INVALID_ARG, "dep_timeout_us < 0");
+  if (c.num_sms < 0 || c.kv_splits < 0 || c.stage_bytes < 0 || c.ring_stages < 0)
+    return fail(TRE_ERR_INVALID_ARG, "negative launch-shape field");
+  if (c.stage_bytes && (c.stage_bytes % 1024 || c.stage_bytes > kMaxStageBytes))
+    return fail(TRE_ERR_INVALID_ARG, "stage_bytes must be a multiple of 1024, <= 65536");
+  return TRE_OK;
+}
+
+tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* shape,
+                      std::vector<Task>* tasks_out, std::vector<int32_t>* sm_begin,
+                      std::vector<int64_t>* sm_bytes) {
+  tre_status st = validate(c);
+  if (st != TRE_OK) return st;
+  if (nsm < 1) return fail(TRE_ERR_INVALID_ARG, "no SMs to plan for");
+  if (smem_limit > kSmemLimit) smem_limit = kSmemLimit;
+
+  PlanShape s{};
+  s.d = c.hidden;
+  s.Hq = c.n_q_heads;
+  s.Hkv = c.n_kv_heads;
+  s.D = c.head_dim;
+  s.F = c.ffn;
+  s.V = c.has_embed_lm_head ? c.vocab : 0;
+  s.L = c.n_layers;
+  s.cap = c.kv_capacity;
+  s.M = c.max_tokens_per_step < 1 ? 1 : c.max_tokens_per_step;
+  s.nsm = nsm;
+  s.has_lm = c.has_embed_lm_head;
+  const int G = s.Hq / s.Hkv;
+
+  // Largest bytes one ring stage must hold: a full row (or the gate+up row pair).
+  int64_t need = std::max<int64_t>({2LL * s.d * 2, (int64_t)s.F * 2, (int64_t)s.Hq * s.D * 2,
+                                     4LL * s.D /* one KV position, K and V */});
+  int sb = c.stage_bytes ? c.stage_bytes : kDefaultStageBytes;
+  while (sb < need && sb < kMaxStageBytes) sb += 1024;
+  if (sb < need)
+    return fail(TRE_ERR_UNSUPPORTED, "a weight row is wider than the largest ring stage (64 KiB)");
+  s.stage_bytes = sb;
+  s.pos_per_stage = std::min(kMaxPosPerStage, sb / (4 * s.D));
+
+  s.xs_floats = std::max({s.d, s.Hq * s.D, s.F});
+  s.xs_floats = (s.xs_floats + 7) / 8 * 8;
+  s.attn_floats = G * s.D + 2 * s.D + kConsumerWarps * (2 * G + G * s.D) + 16;
+  const int ubuf_floats = (std::max(s.xs_floats, s.attn_floats) + 7) / 8 * 8;
+  s.ub_floats = ubuf_floats;
+  const int misc_bytes = 1024;
+  const int fixed = ubuf_floats * 4 + misc_bytes;
+  int ns = c.ring_stages;
+  if (!ns) ns = std::min(16, (smem_limit - fixed - 1024) / (sb + 20));
+  if (ns < 2) return fail(TRE_ERR_UNSUPPORTED, "shared memory too small for a 2-stage ring");
+  s.ring_stages = ns;
+  s.smem_bytes = ns * sb + ((2 * ns * 8 + ns * 4 + 127) / 128) * 128 + fixed;
+  if (s.smem_bytes > smem_limit)
+    return fail(TRE_ERR_UNSUPPORTED, "ring + buffers exceed the shared memory per block");
+
+  // KV splits: enough (kv head, split) tasks to cover the SMs, but no split shorter than
+  // one stage of positions at full capacity.
+  int S = c.kv_splits;
+  if (!S) {
+    S = std::max(1, nsm / s.Hkv);
+    int max_s = std::max(1, (s.cap - 1 + s.pos_per_stage - 1) / s.pos_per_stage);
+    S = std::min(S, max_s);
+  }
+  s.kv_splits = S;
+
+  Builder b(nsm);
+  const int64_t d2 = (int64_t)s.d * 2;
+  int prev_down = -1;
+  uint32_t prev_down_count = 0;
+  for (int l = 0; l < s.L; ++l) {
+    const int cq = counter_of(l, C_QKV), ca = counter_of(l, C_ATTN), co = counter_of(l, C_O),
+              cg = counter_of(l, C_GU), cd = counter_of(l, C_DOWN);
+    int nqkv = 0;
+    nqkv += b.gemv(OP_Q, l, s.Hq * s.D, d2, prev_down, prev_down_count, cq);
+    nqkv += b.gemv(OP_K, l, s.Hkv * s.D, d2, prev_down, prev_down_count, cq);
+    nqkv += b.gemv(OP_V, l, s.Hkv * s.D, d2, prev_down, prev_down_count, cq);
+    const int64_t kv_task_bytes = (int64_t)(s.cap - s.M) / S * s.D * 2 * 2;
+    b.attention(l, s.Hkv, S, kv_task_bytes, cq, (uint32_t)nqkv, ca);
+    int no = b.gemv(OP_O, l, s.d, (int64_t)s.Hq * s.D * 2, ca, (uint32_t)s.Hkv, co);
+    int ng = b.gemv(OP_GU, l, s.F, 2 * d2, co, (uint32_t)no, cg);
+    int nd = b.gemv(OP_DOWN, l, s.d, (int64_t)s.F * 2, cg, (uint32_t)ng, cd);
+    prev_down = cd;
+    prev_down_count = (uint32_t)nd;
+  }
+  const int c_lm = s.L * C_PER_LAYER, c_fault = c_lm + 1;
+  s.n_counters = c_lm + 2;
+  if (s.has_lm) {
+    int first = b.next_id;
+    int nlm = b.gemv(OP_LM, s.L - 1, s.V, d2, prev_down, prev_down_count, c_lm);
+    s.n_lm_tasks = nlm;
+    for (auto& qq : b.q)
+      for (auto& t : qq)
+        if (t.id >= first && t.type == T_GEMV && t.op == OP_LM) t.aux = nlm;
+  }
+  if (c.debug_flags & TRE_DEBUG_FAULT_INJECT) {
+    // the first O-projection task of layer 0 waits on a counter nothing bumps
+    for (auto& qq : b.q) {
+      bool done = false;
+      for (auto& t : qq)
+        if (t.type == T_GEMV && t.op == OP_O && t.layer == 0) {
+          t.dep = c_fault;
+          t.dep_count = 1;
+          done = true;
+          break;
+        }
+      if (done) break;
+    }
+  }
+
+  tasks_out->clear();
+  sm_begin->assign(nsm + 1, 0);
+  size_t mx = 0;
+  for (int i = 0; i < nsm; ++i) {
+    (*sm_begin)[i] = (int32_t)tasks_out->size();
+    tasks_out->insert(tasks_out->end(), b.q[i].begin(), b.q[i].end());
+    mx = std::max(mx, b.q[i].size());
+  }
+  (*sm_begin)[nsm] = (int32_t)tasks_out->size();
+  if (sm_bytes) *sm_bytes = b.cum;
+  *shape = s;
+  (void)mx;
+  return TRE_OK;
+}
+
+int64_t step_bytes(const PlanShape& s, int pos) {
+  const int64_t d = s.d, D = s.D;
+  int64_t per_layer = ((int64_t)(s.Hq + 2 * s.Hkv) * D * d + d * s.Hq * D + 3LL * s.F * d) * 2 +
+                      2 * d * 2;
+  int64_t bytes = per_layer * s.L;
+  bytes += (int64_t)s.L * s.Hkv * (int64_t)pos * D * 2 * 2;  // K and V read
+  bytes += (int64_t)s.L * s.Hkv * D * 2 * 2;                 // this token's K and V written
+  if (s.has_lm) bytes += (int64_t)s.V * d * 2 + d * 2 + d * 2 + (int64_t)s.V * 4;
+  return bytes;
+}
+
+}  // namespace tre

@@ -1,0 +1,464 @@
+// C ABI of the engine (declared in include/tre.h): create / step / status / destroy.
+//
+// The caller owns weights, KV caches and streams (the pages' inject_cache() likewise
+// takes an external KV cache as raw tensors — TileRT code audit, KV-cache section); the
+// engine owns its plan, counters and activation scratch.  One decode step is one
+// cooperative launch of the persistent kernel (Static Compilation for LLM Inference, §1).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "tre_internal.h"
+
+namespace tre {
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm);
+cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream);
+const char* last_error_cstr();
+}  // namespace tre
+
+using namespace tre;
+
+struct tre_engine {
+  tre_config cfg;
+  int device = 0;
+  PlanShape shape{};
+  int n_tasks = 0;
+  uint32_t epoch = 0;
+  cudaStream_t last_stream = nullptr;
+  void* block = nullptr;         // one device allocation for all engine-owned state
+  size_t block_bytes = 0;
+  int32_t* status_host = nullptr;  // mapped pinned [4]
+  int32_t* status_dev = nullptr;
+  Params base{};
+  int32_t* token_buf = nullptr;
+  float* logits_buf = nullptr;
+};
+
+#define TRE_EXPORT extern "C" __attribute__((visibility("default")))
+
+static tre_status cuda_fail(cudaError_t e, const char* what) {
+  set_error(std::string(what) + ": " + cudaGetErrorString(e));
+  return TRE_ERR_CUDA;
+}
+
+#define CK(call)                                          \
+  do {                                                    \
+    cudaError_t _e = (call);                              \
+    if (_e != cudaSuccess) return cuda_fail(_e, #call);   \
+  } while (0)
+
+static bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+namespace {
+struct Carve {  // bump allocator over the engine's single device block
+  size_t off = 0;
+  template <class T>
+  size_t take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    size_t at = off;
+    off += count * sizeof(T);
+    return at;
+  }
+};
+}  // namespace
+
+TRE_EXPORT const char* tre_last_error(void) { return last_error_cstr(); }
+
+TRE_EXPORT tre_status tre_plan_inspect(const tre_config* cfg, int32_t num_sms,
+                                       int32_t smem_per_block, tre_plan_info* info) {
+  if (!cfg || !info) {
+    set_error("tre_plan_inspect: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  PlanShape s;
+  std::vector<Task> tasks;
+  std::vector<int32_t> begin;
+  std::vector<int64_t> bytes;
+  int nsm = cfg->num_sms ? std::min<int>(cfg->num_sms, num_sms) : num_sms;
+  tre_status st = plan_build(*cfg, nsm, smem_per_block, &s, &tasks, &begin, &bytes);
+  if (st != TRE_OK) return st;
+  std::memset(info, 0, sizeof(*info));
+  info->num_sms = s.nsm;
+  info->num_tasks = (int32_t)tasks.size();
+  info->num_counters = s.n_counters;
+  info->kv_splits = s.kv_splits;
+  info->ring_stages = s.ring_stages;
+  info->stage_bytes = s.stage_bytes;
+  info->smem_bytes = s.smem_bytes;
+  int mx = 0;
+  for (int i = 0; i < s.nsm; ++i) mx = std::max(mx, begin[i + 1] - begin[i]);
+  info->max_tasks_per_sm = mx;
+  info->weight_bytes = step_bytes(s, 0) - (int64_t)s.L * s.Hkv * s.D * 4 -
+                       (s.has_lm ? (int64_t)s.V * 4 + 2LL * s.d : 0);
+  info->kv_bytes_at_capacity = (int64_t)s.L * s.Hkv * (int64_t)(s.cap - s.M) * s.D * 4;
+  int64_t lo = INT64_MAX, hi = 0;
+  for (int64_t b : bytes) {
+    lo = std::min(lo, b);
+    hi = std::max(hi, b);
+  }
+  info->max_sm_bytes = hi;
+  info->min_sm_bytes = lo;
+  return TRE_OK;
+}
+
+// Dump the planned task descriptors (8 int32 per task, the Task layout) and the per-SM
+// queue offsets; returns the task count (or a negative tre_status).  Host only.
+TRE_EXPORT int32_t tre_plan_tasks(const tre_config* cfg, int32_t num_sms, int32_t smem_per_block,
+                       int32_t* out_tasks, int32_t max_tasks, int32_t* out_sm_begin) {
+  if (!cfg) return TRE_ERR_INVALID_ARG;
+  PlanShape s;
+  std::vector<Task> tasks;
+  std::vector<int32_t> begin;
+  int nsm = cfg->num_sms ? std::min<int>(cfg->num_sms, num_sms) : num_sms;
+  tre_status st = plan_build(*cfg, nsm, smem_per_block, &s, &tasks, &begin, nullptr);
+  if (st != TRE_OK) return st;
+  if (out_tasks && max_tasks >= (int32_t)tasks.size())
+    std::memcpy(out_tasks, tasks.data(), tasks.size() * sizeof(Task));
+  if (out_sm_begin) std::memcpy(out_sm_begin, begin.data(), begin.size() * sizeof(int32_t));
+  return (int32_t)tasks.size();
+}
+
+TRE_EXPORT void tre_destroy(tre_engine* e) {
+  if (!e) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(e->device);
+  if (e->last_stream) cudaStreamSynchronize(e->last_stream);
+  cudaDeviceSynchronize();
+  if (e->block) cudaFree(e->block);
+  if (e->status_host) cudaFreeHost(e->status_host);
+  cudaSetDevice(prev);
+  delete e;
+}
+
+TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, int device,
+                                 tre_engine** out) {
+  if (!cfg || !w || !out) {
+    set_error("tre_create: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  *out = nullptr;
+  int ndev = 0;
+  CK(cudaGetDeviceCount(&ndev));
+  if (device < 0 || device >= ndev) {
+    set_error("tre_create: no such device");
+    return TRE_ERR_INVALID_ARG;
+  }
+  CK(cudaSetDevice(device));
+  int sms = 0, smem_optin = 0, coop = 0;
+  CK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device));
+  CK(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device));
+  CK(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device));
+  if (!coop) {
+    set_error("tre_create: device lacks cooperative launch");
+    return TRE_ERR_UNSUPPORTED;
+  }
+  const int nsm = cfg->num_sms ? std::min(cfg->num_sms, sms) : sms;
+
+  PlanShape s;
+  std::vector<Task> tasks;
+  std::vector<int32_t> begin;
+  tre_status st = plan_build(*cfg, nsm, smem_optin, &s, &tasks, &begin, nullptr);
+  if (st != TRE_OK) return st;
+
+  // ---- pointer validation: everything the plan reads must be present and 16B-aligned.
+  if (!w->layer_w || !w->k_cache || !w->v_cache) {
+    set_error("tre_create: layer_w / k_cache / v_cache tables must be non-NULL");
+    return TRE_ERR_INVALID_ARG;
+  }
+  static const int gqa_slots[] = {TRE_W_ATTN_NORM, TRE_W_Q,        TRE_W_K,  TRE_W_V,   TRE_W_O,
+                                  TRE_W_FFN_NORM,  TRE_W_GATE,     TRE_W_UP, TRE_W_DOWN};
+  std::vector<LayerPtrs> lp(s.L);
+  for (int l = 0; l < s.L; ++l) {
+    std::memset(&lp[l], 0, sizeof(LayerPtrs));
+    for (int slot : gqa_slots) {
+      const void* p = w->layer_w[(size_t)l * TRE_W_SLOTS + slot];
+      if (!aligned16(p)) {
+        set_error("tre_create: layer " + std::to_string(l) + " slot " + std::to_string(slot) +
+                  " is NULL or not 16-byte aligned");
+        return TRE_ERR_INVALID_ARG;
+      }
+      lp[l].w[slot] = static_cast<const uint16_t*>(p);
+    }
+    if (!aligned16(w->k_cache[l]) || !aligned16(w->v_cache[l])) {
+      set_error("tre_create: KV cache of layer " + std::to_string(l) + " NULL or misaligned");
+      return TRE_ERR_INVALID_ARG;
+    }
+    lp[l].k_cache = static_cast<uint16_t*>(w->k_cache[l]);
+    lp[l].v_cache = static_cast<uint16_t*>(w->v_cache[l]);
+  }
+  if (s.has_lm && (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(w->lm_head))) {
+    set_error("tre_create: embed / final_norm / lm_head NULL or not 16-byte aligned");
+    return TRE_ERR_INVALID_ARG;
+  }
+
+  int bps = 0;
+  CK(engine_configure(s.smem_bytes, &bps));
+  if (bps < 1) {
+    set_error("tre_create: the persistent CTA does not fit on an SM");
+    return TRE_ERR_OCCUPANCY;
+  }
+
+  tre_engine* e = new tre_engine();
+  e->cfg = *cfg;
+  e->device = device;
+  e->shape = s;
+  e->n_tasks = (int)tasks.size();
+
+  // ---- one device block for all engine-owned state
+  const int qkv_n = (s.Hq + 2 * s.Hkv) * s.D;
+  Carve cv;
+  size_t o_tasks = cv.take<Task>(tasks.size());
+  size_t o_begin = cv.take<int32_t>(begin.size());
+  size_t o_layers = cv.take<LayerPtrs>(s.L);
+  size_t o_ctr = cv.take<uint32_t>(s.n_counters);
+  size_t o_tick = cv.take<uint32_t>(s.Hkv);
+  size_t o_lmt = cv.take<uint32_t>(1);
+  size_t o_arg = cv.take<unsigned long long>(1);
+  size_t o_err = cv.take<int32_t>(2);
+  size_t o_x = cv.take<float>(s.d);
+  size_t o_h1 = cv.take<float>(s.d);
+  size_t o_qkv = cv.take<float>(qkv_n);
+  size_t o_attn = cv.take<float>((size_t)s.Hq * s.D);
+  size_t o_u = cv.take<float>(s.F);
+  size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (s.D + 2));
+  size_t o_logits = cv.take<float>(s.V > 0 ? s.V : 1);
+  size_t o_tok = cv.take<int32_t>(1);
+  size_t o_inv = cv.take<double>(s.D / 2);
+  const bool dbg_hidden = cfg->debug_flags & TRE_DEBUG_HIDDEN;
+  const bool dbg_trace = cfg->debug_flags & TRE_DEBUG_TRACE;
+  size_t o_hidden = dbg_hidden ? cv.take<float>((size_t)s.L * s.d) : 0;
+  size_t o_trace = dbg_trace ? cv.take<long long>((size_t)tasks.size() * 4) : 0;
+  e->block_bytes = cv.off;
+  cudaError_t ce = cudaMalloc(&e->block, e->block_bytes);
+  if (ce != cudaSuccess) {
+    delete e;
+    return cuda_fail(ce, "cudaMalloc(engine state)");
+  }
+  uint8_t* B = static_cast<uint8_t*>(e->block);
+  auto fail_free = [&](cudaError_t err, const char* what) {
+    tre_status r = cuda_fail(err, what);
+    tre_destroy(e);
+    return r;
+  };
+  if ((ce = cudaMemset(e->block, 0, e->block_bytes)) != cudaSuccess)
+    return fail_free(ce, "cudaMemset(engine state)");
+  if ((ce = cudaMemcpy(B + o_tasks, tasks.data(), tasks.size() * sizeof(Task),
+                       cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail_free(ce, "upload tasks");
+  if ((ce = cudaMemcpy(B + o_begin, begin.data(), begin.size() * sizeof(int32_t),
+                       cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail_free(ce, "upload queues");
+  if ((ce = cudaMemcpy(B + o_layers, lp.data(), lp.size() * sizeof(LayerPtrs),
+                       cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail_free(ce, "upload layer table");
+  std::vector<double> inv(s.D / 2);
+  for (int i = 0; i < s.D / 2; ++i)
+    inv[i] = std::pow((double)cfg->rope_theta, -2.0 * i / (double)s.D);
+  if ((ce = cudaMemcpy(B + o_inv, inv.data(), inv.size() * sizeof(double),
+                       cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail_free(ce, "upload rope table");
+  if ((ce = cudaHostAlloc(reinterpret_cast<void**>(&e->status_host), 4 * sizeof(int32_t),
+                          cudaHostAllocMapped)) != cudaSuccess)
+    return fail_free(ce, "cudaHostAlloc(status)");
+  std::memset(e->status_host, 0, 4 * sizeof(int32_t));
+  if ((ce = cudaHostGetDevicePointer(reinterpret_cast<void**>(&e->status_dev), e->status_host,
+                                     0)) != cudaSuccess)
+    return fail_free(ce, "cudaHostGetDevicePointer(status)");
+
+  Params& p = e->base;
+  p.tasks = reinterpret_cast<const Task*>(B + o_tasks);
+  p.sm_begin = reinterpret_cast<const int32_t*>(B + o_begin);
+  p.counters = reinterpret_cast<uint32_t*>(B + o_ctr);
+  p.tickets = reinterpret_cast<uint32_t*>(B + o_tick);
+  p.lm_ticket = reinterpret_cast<uint32_t*>(B + o_lmt);
+  p.argmax_slot = reinterpret_cast<unsigned long long*>(B + o_arg);
+  p.layers = reinterpret_cast<const LayerPtrs*>(B + o_layers);
+  p.embed = static_cast<const uint16_t*>(w->embed);
+  p.final_norm = static_cast<const uint16_t*>(w->final_norm);
+  p.lm_head = static_cast<const uint16_t*>(w->lm_head);
+  p.x = reinterpret_cast<float*>(B + o_x);
+  p.h1 = reinterpret_cast<float*>(B + o_h1);
+  p.qkv = reinterpret_cast<float*>(B + o_qkv);
+  p.attn = reinterpret_cast<float*>(B + o_attn);
+  p.u = reinterpret_cast<float*>(B + o_u);
+  p.part = reinterpret_cast<float*>(B + o_part);
+  p.logits = reinterpret_cast<float*>(B + o_logits);
+  e->logits_buf = p.logits;
+  e->token_buf = reinterpret_cast<int32_t*>(B + o_tok);
+  p.hidden = dbg_hidden ? reinterpret_cast<float*>(B + o_hidden) : nullptr;
+  p.trace = dbg_trace ? reinterpret_cast<long long*>(B + o_trace) : nullptr;
+  p.rope_inv_freq = reinterpret_cast<const double*>(B + o_inv);
+  p.err = reinterpret_cast<int32_t*>(B + o_err);
+  p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
+  p.status_host = e->status_dev;
+  p.d = s.d; p.Hq = s.Hq; p.Hkv = s.Hkv; p.D = s.D; p.F = s.F; p.V = s.V; p.L = s.L;
+  p.cap = s.cap;
+  p.nsplit = s.kv_splits;
+  p.pps = s.pos_per_stage;
+  p.stage_bytes = s.stage_bytes;
+  p.ring_stages = s.ring_stages;
+  p.xs_floats = s.xs_floats;
+  p.ub_floats = s.ub_floats;
+  p.eps = cfg->norm_eps;
+  p.flags = cfg->debug_flags;
+  p.timeout_ns = 1000LL * (cfg->dep_timeout_us ? cfg->dep_timeout_us : 1000000);
+  *out = e;
+  return TRE_OK;
+}
+
+static tre_status pending_device_error(tre_engine* e) {
+  const int32_t code = *reinterpret_cast<volatile int32_t*>(e->status_host);
+  if (code == 0) return TRE_OK;
+  set_error("a previous step recorded device error " + std::to_string(code) + " (task " +
+            std::to_string(reinterpret_cast<volatile int32_t*>(e->status_host)[1]) +
+            "); call tre_reset");
+  return (tre_status)code;
+}
+
+static tre_status launch_step(tre_engine* e, int32_t token, int32_t pos, cudaStream_t stream,
+                              float* logits_dev, int32_t* token_dev, const float* x_in,
+                              float* x_out) {
+  tre_status st = pending_device_error(e);
+  if (st != TRE_OK) return st;
+  if (pos < 0 || pos >= e->shape.cap) {
+    set_error("pos outside [0, kv_capacity)");
+    return TRE_ERR_POS_RANGE;
+  }
+  CK(cudaSetDevice(e->device));
+  Params p = e->base;
+  p.token = token;
+  p.pos = pos;
+  p.epoch = ++e->epoch;
+  if (logits_dev) p.logits = logits_dev;
+  p.token_out = token_dev ? token_dev : e->token_buf;
+  p.x_in = x_in;
+  p.x_out = x_out;
+  cudaError_t ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream);
+  if (ce != cudaSuccess) {
+    --e->epoch;
+    return cuda_fail(ce, "launch of the persistent engine");
+  }
+  e->last_stream = stream;
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_decode_step(tre_engine* e, int32_t token, int32_t pos, tre_stream stream,
+                                      float* logits_dev, int32_t* token_dev) {
+  if (!e) {
+    set_error("tre_decode_step: NULL engine");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (!e->shape.has_lm) {
+    set_error("tre_decode_step: engine has no embedding / LM head (use a layers step)");
+    return TRE_ERR_UNSUPPORTED;
+  }
+  if (token < 0 || token >= e->shape.V) {
+    set_error("tre_decode_step: token outside [0, vocab)");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (logits_dev && ((uintptr_t)logits_dev & 15u)) {
+    set_error("tre_decode_step: logits_dev must be 16-byte aligned");
+    return TRE_ERR_INVALID_ARG;
+  }
+  return launch_step(e, token, pos, (cudaStream_t)stream, logits_dev, token_dev, nullptr, nullptr);
+}
+
+TRE_EXPORT tre_status tre_decode_step_host(tre_engine* e, int32_t token, int32_t pos,
+                                           tre_stream stream, float* logits_host,
+                                           int32_t* token_host) {
+  if (!e || !token_host) {
+    set_error("tre_decode_step_host: NULL engine or token_host");
+    return TRE_ERR_INVALID_ARG;
+  }
+  tre_status st = tre_decode_step(e, token, pos, stream, nullptr, nullptr);
+  if (st != TRE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  CK(cudaMemcpyAsync(token_host, e->token_buf, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  if (logits_host)
+    CK(cudaMemcpyAsync(logits_host, e->logits_buf, (size_t)e->shape.V * sizeof(float),
+                       cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return pending_device_error(e);
+}
+
+TRE_EXPORT tre_status tre_get_status(tre_engine* e, int32_t* device_status, int32_t* detail_out) {
+  if (!e || !device_status) {
+    set_error("tre_get_status: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  CK(cudaSetDevice(e->device));
+  if (e->last_stream) CK(cudaStreamSynchronize(e->last_stream));
+  CK(cudaDeviceSynchronize());
+  volatile int32_t* sh = e->status_host;
+  *device_status = sh[0];
+  if (detail_out) *detail_out = sh[1];
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
+  if (!e) {
+    set_error("tre_reset: NULL engine");
+    return TRE_ERR_INVALID_ARG;
+  }
+  CK(cudaSetDevice(e->device));
+  cudaStream_t s = (cudaStream_t)stream;
+  CK(cudaDeviceSynchronize());
+  const Params& p = e->base;
+  CK(cudaMemsetAsync(p.counters, 0, (size_t)e->shape.n_counters * 4, s));
+  CK(cudaMemsetAsync(p.tickets, 0, (size_t)e->shape.Hkv * 4, s));
+  CK(cudaMemsetAsync(p.lm_ticket, 0, 4, s));
+  CK(cudaMemsetAsync(p.argmax_slot, 0, 8, s));
+  CK(cudaMemsetAsync(p.err, 0, 8, s));  // error word + abort flag
+  CK(cudaStreamSynchronize(s));
+  std::memset(e->status_host, 0, 4 * sizeof(int32_t));
+  e->epoch = 0;
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_debug_hidden(tre_engine* e, float* hidden_dev, tre_stream stream) {
+  if (!e || !hidden_dev) {
+    set_error("tre_debug_hidden: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (!e->base.hidden) {
+    set_error("tre_debug_hidden: engine created without TRE_DEBUG_HIDDEN");
+    return TRE_ERR_INVALID_ARG;
+  }
+  CK(cudaSetDevice(e->device));
+  CK(cudaMemcpyAsync(hidden_dev, e->base.hidden, (size_t)e->shape.L * e->shape.d * sizeof(float),
+                     cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_debug_trace(tre_engine* e, int64_t* trace_host, int32_t* n_tasks) {
+  if (!e || !n_tasks) {
+    set_error("tre_debug_trace: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  *n_tasks = e->n_tasks;
+  if (!trace_host) return TRE_OK;
+  if (!e->base.trace) {
+    set_error("tre_debug_trace: engine created without TRE_DEBUG_TRACE");
+    return TRE_ERR_INVALID_ARG;
+  }
+  CK(cudaSetDevice(e->device));
+  CK(cudaDeviceSynchronize());
+  CK(cudaMemcpy(trace_host, e->base.trace, (size_t)e->n_tasks * 4 * sizeof(long long),
+                cudaMemcpyDeviceToHost));
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_step_bytes(const tre_engine* e, int32_t pos, int64_t* bytes) {
+  if (!e || !bytes) {
+    set_error("tre_step_bytes: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  *bytes = step_bytes(e->shape, pos);
+  return TRE_OK;
+}

@@ -1,0 +1,124 @@
+// Internal types of the engine shared by the host planner (planner.cpp), the C ABI
+// (tre_api.cu) and the persistent kernel (engine.cu).
+#pragma once
+#include <stdint.h>
+
+#include "tre.h"
+
+namespace tre {
+
+// ---- compile-time shape of the persistent CTA -------------------------------------
+constexpr int kConsumerWarps = 8;                      // compute warps
+constexpr int kConsumerThreads = kConsumerWarps * 32;  // 256
+constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
+constexpr int kMaxGroup = 8;                           // q heads per kv head (GQA)
+constexpr int kMaxPosPerStage = 64;                    // KV positions per attention stage
+constexpr int kDefaultStageBytes = 32768;
+constexpr int kMaxStageBytes = 65536;
+constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per block
+
+// ---- tasks --------------------------------------------------------------------------
+enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1 };
+
+// GEMV ops: which matrix, which input vector, which epilogue.
+enum GemvOp : uint8_t {
+  OP_Q = 0,     // in: RMSNorm(x; attn_norm)  -> qkv[0 : Hq*D]
+  OP_K = 1,     // in: RMSNorm(x; attn_norm)  -> qkv[Hq*D : +Hkv*D]
+  OP_V = 2,     // in: RMSNorm(x; attn_norm)  -> qkv[(Hq+Hkv)*D : +Hkv*D]
+  OP_O = 3,     // in: attn                   -> h1 = x + Wo attn
+  OP_GU = 4,    // in: RMSNorm(h1; ffn_norm)  -> u = silu(Wg hn) * (Wu hn)   (2 segments)
+  OP_DOWN = 5,  // in: u                      -> x = h1 + Wd u
+  OP_LM = 6,    // in: RMSNorm(x; final_norm) -> logits, greedy argmax
+  OP_COUNT = 7
+};
+
+// Dependency counters: one per (layer, stage of the layer), then the LM head and a
+// counter nothing ever bumps (used only by the fault-injection debug plan).
+enum CounterKind { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, C_PER_LAYER = 5 };
+
+struct Task {          // 32 bytes, 16-byte aligned array
+  uint8_t type;        // TaskType
+  uint8_t op;          // GemvOp (T_GEMV)
+  uint16_t layer;
+  int32_t dep;         // counter to wait on, -1 = none
+  uint32_t dep_count;  // increments of `dep` per step
+  int32_t out;         // counter to bump when done, -1 = none
+  int32_t r0, r1;      // GEMV: output rows [r0, r1).  ATTN: kv head, split index
+  int32_t aux;         // ATTN: number of splits.  LM: number of LM tasks
+  int32_t id;          // global task index (trace rows, error detail)
+};
+static_assert(sizeof(Task) == 32, "task descriptor is 32 bytes");
+
+struct LayerPtrs {     // device-side per-layer pointer table
+  const uint16_t* w[TRE_W_SLOTS];
+  uint16_t* k_cache;
+  uint16_t* v_cache;
+};
+
+// ---- the plan (host side) -----------------------------------------------------------
+struct PlanShape {
+  int d, Hq, Hkv, D, F, V, L, cap, M;
+  int nsm;
+  int stage_bytes, ring_stages;
+  int kv_splits, pos_per_stage;
+  int xs_floats;       // input-vector buffer (floats)
+  int attn_floats;     // attention scratch (floats), aliases the input-vector buffer
+  int ub_floats;       // max(xs_floats, attn_floats): the shared union buffer
+  int smem_bytes;
+  int n_counters;
+  int n_lm_tasks;
+  int has_lm;
+};
+
+// ---- kernel parameters ----------------------------------------------------------------
+struct Params {
+  const Task* tasks;
+  const int32_t* sm_begin;         // [nsm + 1] offsets into tasks
+  uint32_t* counters;
+  uint32_t* tickets;               // [Hkv] split-KV arrival tickets
+  uint32_t* lm_ticket;
+  unsigned long long* argmax_slot;
+  const LayerPtrs* layers;
+  const uint16_t* embed;
+  const uint16_t* final_norm;
+  const uint16_t* lm_head;
+  const float* x_in;               // layer-only input (NULL: embedding row)
+  float* x_out;                    // layer-only output (NULL: none)
+  float* x;                        // residual stream [d]
+  float* h1;                       // after attention [d]
+  float* qkv;                      // [(Hq + 2 Hkv) D]
+  float* attn;                     // [Hq D]
+  float* u;                        // [F]
+  float* part;                     // [Hq][splits][D + 2]
+  float* logits;                   // [V]
+  int32_t* token_out;              // [1] or NULL
+  float* hidden;                   // debug [L][d] or NULL
+  long long* trace;                // debug [n_tasks][4] or NULL
+  const double* rope_inv_freq;     // [D/2]
+  int32_t* err;                    // device word: first error wins
+  volatile int32_t* abort_flag;    // device word
+  volatile int32_t* status_host;   // host-mapped [2]: code, detail
+  int d, Hq, Hkv, D, F, V, L, cap;
+  int nsplit, pps, stage_bytes, ring_stages, xs_floats, ub_floats;
+  float eps;
+  int token, pos;
+  uint32_t epoch;
+  int flags;
+  long long timeout_ns;
+};
+
+}  // namespace tre
+
+// Planner entry (planner.cpp).  Fills shape, tasks (grouped per SM, topological order
+// within each SM) and sm_begin.  Returns TRE_OK or an error with tre_set_error text.
+#ifdef __cplusplus
+#include <string>
+#include <vector>
+namespace tre {
+tre_status plan_build(const tre_config& cfg, int nsm, int smem_limit, PlanShape* shape,
+                      std::vector<Task>* tasks, std::vector<int32_t>* sm_begin,
+                      std::vector<int64_t>* sm_bytes);
+int64_t step_bytes(const PlanShape& s, int pos);
+void set_error(const std::string& msg);
+}  // namespace tre
+#endif

@@ -1,0 +1,297 @@
+"""Python binding of the engine's C ABI (``include/tre.h``): argument marshalling only.
+
+Every step of the decode path runs inside ``libtre.so``; this module converts Python
+objects to the C structs, passes device pointers from torch tensors and raises on error.
+There is no fallback: if the native library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtre.so")
+
+# ---- constants mirrored from tre.h ------------------------------------------------------
+TRE_OK = 0
+TRE_ERR_INVALID_ARG = -1
+TRE_ERR_CUDA = -2
+TRE_ERR_OCCUPANCY = -3
+TRE_ERR_DEP_TIMEOUT = -4
+TRE_ERR_POS_RANGE = -5
+TRE_ERR_UNSUPPORTED = -6
+TRE_ERR_BOUNDS = -7
+TRE_ERR_STATE = -8
+TRE_LAYER_GQA, TRE_LAYER_MLA, TRE_LAYER_MOE = 0, 1, 2
+TRE_DEBUG_HIDDEN, TRE_DEBUG_TRACE, TRE_DEBUG_FAULT_INJECT, TRE_DEBUG_NO_OVERLAP = 1, 2, 4, 8
+TRE_W_SLOTS = 16
+GQA_SLOTS = {"attn_norm": 0, "wq": 1, "wk": 2, "wv": 3, "wo": 4, "ffn_norm": 5, "wgate": 6,
+             "wup": 7, "wdown": 8}
+
+STATUS_NAMES = {0: "TRE_OK", -1: "TRE_ERR_INVALID_ARG", -2: "TRE_ERR_CUDA",
+                -3: "TRE_ERR_OCCUPANCY", -4: "TRE_ERR_DEP_TIMEOUT", -5: "TRE_ERR_POS_RANGE",
+                -6: "TRE_ERR_UNSUPPORTED", -7: "TRE_ERR_BOUNDS", -8: "TRE_ERR_STATE"}
+
+
+class tre_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "kind", "n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
+        "q_lora", "kv_lora", "rope_dim", "nope_dim", "v_dim",
+        "n_experts", "top_k", "n_shared", "expert_ffn",
+        "kv_capacity", "max_tokens_per_step")] + [
+        ("rope_theta", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
+        (n, ctypes.c_int32) for n in (
+            "has_embed_lm_head", "debug_flags", "dep_timeout_us", "num_sms", "kv_splits",
+            "stage_bytes", "ring_stages")] + [("reserved", ctypes.c_int32 * 8)]
+
+
+class tre_weights(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
+                ("lm_head", ctypes.c_void_p), ("layer_w", ctypes.POINTER(ctypes.c_void_p)),
+                ("k_cache", ctypes.POINTER(ctypes.c_void_p)),
+                ("v_cache", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class tre_plan_info(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_sms", "num_tasks", "num_counters", "kv_splits", "ring_stages", "stage_bytes",
+        "smem_bytes", "max_tasks_per_sm")] + [
+        (n, ctypes.c_int64) for n in ("weight_bytes", "kv_bytes_at_capacity", "max_sm_bytes",
+                                      "min_sm_bytes")]
+
+
+EXPORTED = ("tre_create", "tre_destroy", "tre_decode_step", "tre_decode_step_host",
+            "tre_get_status", "tre_reset", "tre_debug_hidden", "tre_debug_trace",
+            "tre_step_bytes", "tre_plan_inspect", "tre_plan_tasks", "tre_last_error")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m persistent_tile_pipelined_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    L.tre_create.argtypes = [ctypes.POINTER(tre_config), ctypes.POINTER(tre_weights), ctypes.c_int,
+                             ctypes.POINTER(vp)]
+    L.tre_destroy.argtypes = [vp]
+    L.tre_destroy.restype = None
+    L.tre_decode_step.argtypes = [vp, i32, i32, vp, vp, vp]
+    L.tre_decode_step_host.argtypes = [vp, i32, i32, vp, vp, vp]
+    L.tre_get_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    L.tre_reset.argtypes = [vp, vp]
+    L.tre_debug_hidden.argtypes = [vp, vp, vp]
+    L.tre_debug_trace.argtypes = [vp, vp, ctypes.POINTER(i32)]
+    L.tre_step_bytes.argtypes = [vp, i32, ctypes.POINTER(i64)]
+    L.tre_plan_inspect.argtypes = [ctypes.POINTER(tre_config), i32, i32,
+                                   ctypes.POINTER(tre_plan_info)]
+    L.tre_plan_tasks.argtypes = [ctypes.POINTER(tre_config), i32, i32, vp, i32, vp]
+    L.tre_plan_tasks.restype = i32
+    L.tre_last_error.argtypes = []
+    L.tre_last_error.restype = ctypes.c_char_p
+    for name in ("tre_create", "tre_decode_step", "tre_decode_step_host", "tre_get_status",
+                 "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
+                 "tre_plan_inspect"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+class TreError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.tre_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+def check(status: int, where: str) -> None:
+    if status != TRE_OK:
+        raise TreError(status, where)
+
+
+# ---- same-named thin wrappers ----------------------------------------------------------------
+def tre_create(cfg: tre_config, weights: tre_weights, device: int = 0) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    check(lib.tre_create(ctypes.byref(cfg), ctypes.byref(weights), device, ctypes.byref(h)),
+          "tre_create")
+    return h
+
+
+def tre_destroy(h) -> None:
+    lib.tre_destroy(h)
+
+
+def tre_decode_step(h, token: int, pos: int, stream: int = 0, logits_dev: int = 0,
+                    token_dev: int = 0) -> int:
+    return lib.tre_decode_step(h, int(token), int(pos), ctypes.c_void_p(stream or None),
+                               ctypes.c_void_p(logits_dev or None), ctypes.c_void_p(token_dev or None))
+
+
+def tre_decode_step_host(h, token: int, pos: int, stream: int = 0,
+                         logits_host: Optional[np.ndarray] = None) -> int:
+    tok = ctypes.c_int32()
+    lp = None
+    if logits_host is not None:
+        assert logits_host.dtype == np.float32 and logits_host.flags.c_contiguous
+        lp = logits_host.ctypes.data_as(ctypes.c_void_p)
+    check(lib.tre_decode_step_host(h, int(token), int(pos), ctypes.c_void_p(stream or None), lp,
+                                   ctypes.byref(tok)), "tre_decode_step_host")
+    return tok.value
+
+
+def tre_get_status(h):
+    st, det = ctypes.c_int32(), ctypes.c_int32()
+    check(lib.tre_get_status(h, ctypes.byref(st), ctypes.byref(det)), "tre_get_status")
+    return st.value, det.value
+
+
+def tre_reset(h, stream: int = 0) -> None:
+    check(lib.tre_reset(h, ctypes.c_void_p(stream or None)), "tre_reset")
+
+
+def tre_step_bytes(h, pos: int) -> int:
+    b = ctypes.c_int64()
+    check(lib.tre_step_bytes(h, int(pos), ctypes.byref(b)), "tre_step_bytes")
+    return b.value
+
+
+def tre_plan_inspect(cfg: tre_config, num_sms: int = 148, smem_per_block: int = 232448):
+    info = tre_plan_info()
+    check(lib.tre_plan_inspect(ctypes.byref(cfg), num_sms, smem_per_block, ctypes.byref(info)),
+          "tre_plan_inspect")
+    return info
+
+
+def tre_plan_tasks(cfg: tre_config, num_sms: int = 148, smem_per_block: int = 232448):
+    """Returns (tasks int32[n][8], sm_begin int32[num_sms+1])."""
+    nsm = min(cfg.num_sms, num_sms) if cfg.num_sms else num_sms
+    begin = np.zeros(nsm + 1, dtype=np.int32)
+    n = lib.tre_plan_tasks(ctypes.byref(cfg), num_sms, smem_per_block, None, 0,
+                           begin.ctypes.data_as(ctypes.c_void_p))
+    if n < 0:
+        raise TreError(n, "tre_plan_tasks")
+    tasks = np.zeros((n, 8), dtype=np.int32)
+    n2 = lib.tre_plan_tasks(ctypes.byref(cfg), num_sms, smem_per_block,
+                            tasks.ctypes.data_as(ctypes.c_void_p), n,
+                            begin.ctypes.data_as(ctypes.c_void_p))
+    assert n2 == n
+    return tasks, begin
+
+
+# ---- convenience ------------------------------------------------------------------------------
+def config_from_workload(wl, **overrides) -> tre_config:
+    c = tre_config()
+    c.kind = {"gqa": TRE_LAYER_GQA, "mla": TRE_LAYER_MLA, "moe": TRE_LAYER_MOE}[wl.kind]
+    for f in ("n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
+              "q_lora", "kv_lora", "rope_dim", "nope_dim", "v_dim", "n_experts", "top_k",
+              "n_shared", "expert_ffn"):
+        setattr(c, f, int(getattr(wl, f)))
+    c.kv_capacity = wl.kv_capacity
+    c.max_tokens_per_step = wl.tokens_per_step
+    c.rope_theta = wl.rope_theta
+    c.norm_eps = wl.norm_eps
+    c.has_embed_lm_head = 1 if wl.has_embed_lm_head else 0
+    for k, v in overrides.items():
+        setattr(c, k, v)
+    return c
+
+
+def _dev_tensor(words: np.ndarray, device):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(words).view(np.int16)).view(torch.bfloat16)
+    return t.to(device, non_blocking=False)
+
+
+def upload_gqa_model(model: dict, device="cuda:0") -> dict:
+    """Copy a host model (bf16 words) to device tensors; the caller keeps them alive."""
+    out = {"layers": [], "k_cache": [], "v_cache": []}
+    for l, layer in enumerate(model["layers"]):
+        out["layers"].append({slot: _dev_tensor(a, device) for slot, a in layer.items()})
+        out["k_cache"].append(_dev_tensor(model["k_cache"][l], device))
+        out["v_cache"].append(_dev_tensor(model["v_cache"][l], device))
+    for k in ("embed", "final_norm", "lm_head"):
+        if k in model:
+            out[k] = _dev_tensor(model[k], device)
+    return out
+
+
+class Engine:
+    """Owns one tre_engine; keeps references to the caller's device tensors."""
+
+    def __init__(self, cfg: tre_config, dev_model: dict, device: int = 0):
+        self.cfg = cfg
+        self.dev_model = dev_model  # keep the caller-owned memory alive
+        L = cfg.n_layers
+        self._layer_w = (ctypes.c_void_p * (L * TRE_W_SLOTS))()
+        for l in range(L):
+            for slot, t in dev_model["layers"][l].items():
+                self._layer_w[l * TRE_W_SLOTS + slot] = t.data_ptr()
+        self._kc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["k_cache"]])
+        self._vc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["v_cache"]])
+        self.weights = tre_weights()
+        for k in ("embed", "final_norm", "lm_head"):
+            if k in dev_model:
+                setattr(self.weights, k, dev_model[k].data_ptr())
+        self.weights.layer_w = ctypes.cast(self._layer_w, ctypes.POINTER(ctypes.c_void_p))
+        self.weights.k_cache = ctypes.cast(self._kc, ctypes.POINTER(ctypes.c_void_p))
+        self.weights.v_cache = ctypes.cast(self._vc, ctypes.POINTER(ctypes.c_void_p))
+        self.device = device
+        self.h = tre_create(cfg, self.weights, device)
+
+    def close(self):
+        if getattr(self, "h", None):
+            tre_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def step(self, token: int, pos: int, logits=None, token_out=None, stream=None) -> None:
+        """Enqueue one decode step on `stream` (default: torch's current stream)."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        check(tre_decode_step(self.h, token, pos, s,
+                              logits.data_ptr() if logits is not None else 0,
+                              token_out.data_ptr() if token_out is not None else 0),
+              "tre_decode_step")
+
+    def step_host(self, token: int, pos: int, logits_host: Optional[np.ndarray] = None,
+                  stream=None) -> int:
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        return tre_decode_step_host(self.h, token, pos, s, logits_host)
+
+    def status(self):
+        return tre_get_status(self.h)
+
+    def reset(self, stream=None):
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        tre_reset(self.h, s)
+
+    def hidden(self):
+        import torch
+        out = torch.empty((self.cfg.n_layers, self.cfg.hidden), dtype=torch.float32,
+                          device=f"cuda:{self.device}")
+        check(lib.tre_debug_hidden(self.h, ctypes.c_void_p(out.data_ptr()),
+                                   ctypes.c_void_p(torch.cuda.current_stream(self.device).cuda_stream)),
+              "tre_debug_hidden")
+        return out
+
+    def trace(self) -> np.ndarray:
+        n = ctypes.c_int32()
+        check(lib.tre_debug_trace(self.h, None, ctypes.byref(n)), "tre_debug_trace")
+        buf = np.zeros((n.value, 4), dtype=np.int64)
+        check(lib.tre_debug_trace(self.h, buf.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)),
+              "tre_debug_trace")
+        return buf
+
+    def step_bytes(self, pos: int) -> int:
+        return tre_step_bytes(self.h, pos)

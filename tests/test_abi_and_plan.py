@@ -1,0 +1,157 @@
+"""The C-ABI library loads and exports every declared symbol; the host planner's task
+graph is a valid, deadlock-free, balanced partition of the step (no GPU needed)."""
+import os
+import re
+from collections import Counter, defaultdict
+
+import numpy as np
+import pytest
+
+from persistent_tile_pipelined_b200 import build
+from persistent_tile_pipelined_b200.synth import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+build.build_engine()
+from persistent_tile_pipelined_b200 import tre  # noqa: E402
+
+T_GEMV, T_ATTN = 0, 1
+OP_Q, OP_K, OP_V, OP_O, OP_GU, OP_DOWN, OP_LM = range(7)
+C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_PER_LAYER = range(6)
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(tre_[a-z_0-9]+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert {"tre_create", "tre_decode_step", "tre_destroy"} <= names
+    for n in names:
+        assert hasattr(tre.lib, n), f"{n} declared in include/ but not exported"
+    assert set(tre.EXPORTED) == names
+
+
+def decode_tasks(tasks):
+    w0 = tasks[:, 0].astype(np.int64) & 0xFFFFFFFF
+    return {
+        "type": w0 & 0xFF, "op": (w0 >> 8) & 0xFF, "layer": (w0 >> 16) & 0xFFFF,
+        "dep": tasks[:, 1], "dep_count": tasks[:, 2].astype(np.int64) & 0xFFFFFFFF,
+        "out": tasks[:, 3], "r0": tasks[:, 4], "r1": tasks[:, 5], "aux": tasks[:, 6],
+        "id": tasks[:, 7],
+    }
+
+
+PLAN_CASES = [
+    (W.TINY, 148), (W.TINY, 7), (W.LLAMA8B, 148), (W.LLAMA8B, 132),
+    (W.TINY.replace(n_q_heads=8, n_kv_heads=1, ffn=696, vocab=1001), 148),
+    (W.TINY.replace(n_q_heads=4, n_kv_heads=4, head_dim=128, vocab=77), 33),
+]
+
+
+@pytest.mark.parametrize("wl,nsm", PLAN_CASES, ids=lambda x: getattr(x, "name", str(x)))
+def test_plan_is_a_valid_task_graph(wl, nsm):
+    cfg = tre.config_from_workload(wl)
+    tasks, begin = tre.tre_plan_tasks(cfg, num_sms=nsm)
+    info = tre.tre_plan_inspect(cfg, num_sms=nsm)
+    assert info.num_tasks == len(tasks) and begin[-1] == len(tasks)
+    T = decode_tasks(tasks)
+    n = len(tasks)
+    # ids are a permutation of 0..n-1, increasing within each SM queue (topological order)
+    assert sorted(T["id"].tolist()) == list(range(n))
+    for s in range(nsm):
+        ids = T["id"][begin[s]:begin[s + 1]]
+        assert (np.diff(ids) > 0).all()
+    # who bumps each counter, and at which global index
+    bumpers = defaultdict(list)
+    for i in range(n):
+        if T["out"][i] >= 0:
+            bumpers[int(T["out"][i])].append(i)
+    for i in range(n):
+        dep = int(T["dep"][i])
+        if dep < 0:
+            continue
+        assert dep < info.num_counters
+        producers = bumpers[dep]
+        # every producer of a dependency precedes its consumer in global order
+        assert all(T["id"][j] < T["id"][i] for j in producers)
+        kind = dep % C_PER_LAYER
+        if T["type"][i] == T_GEMV and T["op"][i] == OP_O:
+            # the attention counter is bumped once per kv head (by the combining split)
+            assert T["dep_count"][i] == wl.n_kv_heads
+        else:
+            assert T["dep_count"][i] == len(producers), (i, dep, kind)
+    # every GEMV op's output rows are partitioned exactly once per layer
+    rows_of = {OP_Q: wl.n_q_heads * wl.head_dim, OP_K: wl.n_kv_heads * wl.head_dim,
+               OP_V: wl.n_kv_heads * wl.head_dim, OP_O: wl.hidden, OP_GU: wl.ffn,
+               OP_DOWN: wl.hidden, OP_LM: wl.vocab}
+    for l in range(wl.n_layers):
+        for op, N in rows_of.items():
+            if op == OP_LM and l != wl.n_layers - 1:
+                continue
+            sel = (T["type"] == T_GEMV) & (T["op"] == op) & (T["layer"] == l)
+            cover = np.zeros(N, dtype=np.int64)
+            for r0, r1 in zip(T["r0"][sel], T["r1"][sel]):
+                assert 0 <= r0 < r1 <= N
+                cover[r0:r1] += 1
+            assert (cover == 1).all(), (l, op)
+        sel = (T["type"] == T_ATTN) & (T["layer"] == l)
+        pairs = Counter(zip(T["r0"][sel].tolist(), T["r1"][sel].tolist()))
+        S = info.kv_splits
+        assert set(pairs) == {(g, s) for g in range(wl.n_kv_heads) for s in range(S)}
+        assert all(v == 1 for v in pairs.values())
+        assert (T["aux"][sel] == S).all()
+    # LM tasks carry the LM task count
+    lm = (T["type"] == T_GEMV) & (T["op"] == OP_LM)
+    assert (T["aux"][lm] == lm.sum()).all()
+    assert info.smem_bytes <= 232448
+
+
+def test_llama8b_plan_is_byte_balanced():
+    cfg = tre.config_from_workload(W.LLAMA8B)
+    info = tre.tre_plan_inspect(cfg, num_sms=148)
+    assert info.kv_splits >= 8
+    assert info.ring_stages >= 4
+    # every SM streams within 1% of the others over the whole step
+    assert info.max_sm_bytes <= 1.01 * info.min_sm_bytes
+    assert info.weight_bytes == pytest.approx(15.01e9, rel=0.01)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("kind", 1, tre.TRE_ERR_UNSUPPORTED), ("kind", 9, tre.TRE_ERR_INVALID_ARG),
+    ("hidden", 260, tre.TRE_ERR_INVALID_ARG), ("n_kv_heads", 3, tre.TRE_ERR_INVALID_ARG),
+    ("head_dim", 96, tre.TRE_ERR_UNSUPPORTED), ("ffn", 690, tre.TRE_ERR_INVALID_ARG),
+    ("kv_capacity", 0, tre.TRE_ERR_INVALID_ARG), ("max_tokens_per_step", 4, tre.TRE_ERR_UNSUPPORTED),
+    ("stage_bytes", 1000, tre.TRE_ERR_INVALID_ARG), ("rope_theta", 0.0, tre.TRE_ERR_INVALID_ARG),
+])
+def test_plan_rejects_bad_configs(field, value, status):
+    cfg = tre.config_from_workload(W.TINY, **{field: value})
+    info = tre.tre_plan_info()
+    import ctypes
+    assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status
+    assert tre.lib.tre_last_error()
+
+
+def test_reserved_fields_must_be_zero():
+    import ctypes
+    cfg = tre.config_from_workload(W.TINY)
+    cfg.reserved[3] = 1
+    info = tre.tre_plan_info()
+    assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448,
+                                    ctypes.byref(info)) == tre.TRE_ERR_INVALID_ARG
+
+
+def test_fault_inject_plans_one_unsatisfiable_wait():
+    cfg = tre.config_from_workload(W.TINY, debug_flags=tre.TRE_DEBUG_FAULT_INJECT)
+    info = tre.tre_plan_inspect(cfg)
+    tasks, _ = tre.tre_plan_tasks(cfg)
+    T = decode_tasks(tasks)
+    fault_ctr = info.num_counters - 1
+    assert (T["dep"] == fault_ctr).sum() == 1
+    assert not (T["out"] == fault_ctr).any()
