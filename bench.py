@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-layers", type=int, default=4)
     ap.add_argument("--trace", default="", help="write a per-task trace of one step (JSON)")
+    ap.add_argument("--flags", type=int, default=0,
+                    help="engine debug flags for the timed engine (8 = no cross-op prefetch)")
     return ap.parse_args()
 
 
@@ -231,7 +233,7 @@ def run_engine(args, rank, world, local_rank):
     wl = W.WORKLOADS[args.workload]
     K, Wm = args.steps, args.warmup
     wl = wl.replace(decode_steps=K + Wm, seed=wl.seed + rank)
-    eng, model = build_engine(wl, local_rank)
+    eng, model = build_engine(wl, local_rank, args.flags)
     stream = torch.cuda.current_stream(local_rank)
     s_ptr = stream.cuda_stream
     tokens = [token_id(wl.seed, wl.vocab, i) for i in range(K + Wm)]
@@ -289,7 +291,7 @@ def run_engine(args, rank, world, local_rank):
     torch.cuda.empty_cache()
 
     if trace_path:
-        write_trace(wl, local_rank, trace_path)
+        write_trace(wl, local_rank, trace_path, args.flags)
 
     t = torch.tensor([dev_s, e2e_s, float(np.mean(launch_ms))], dtype=torch.float64,
                      device=f"cuda:{local_rank}")
@@ -299,19 +301,26 @@ def run_engine(args, rank, world, local_rank):
     return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
 
 
-def write_trace(wl, device, path):
-    """One traced step (debug flag on a fresh engine): per-task start / ready / end."""
+def write_trace(wl, device, path, flags=0):
+    """Three traced steps on a fresh engine (debug flag): per-task start / ready / end of
+    the last one, with the plan and its summary."""
     import torch
 
+    from persistent_tile_pipelined_b200 import trace as trace_mod
     from persistent_tile_pipelined_b200 import tre
-    eng, model = build_engine(wl.replace(decode_steps=2), device, tre.TRE_DEBUG_TRACE)
-    eng.step(1, wl.prefill)
-    eng.step(2, wl.prefill + 1)
+    eng, model = build_engine(wl.replace(decode_steps=3), device, tre.TRE_DEBUG_TRACE | flags)
+    for i in range(3):
+        eng.step(1 + i, wl.prefill + i)
     torch.cuda.synchronize(device)
     tr = eng.trace()
+    nsm = torch.cuda.get_device_properties(device).multi_processor_count
+    tasks, begin = tre.tre_plan_tasks(eng.cfg, num_sms=nsm)
     eng.close()
+    summ = trace_mod.summarize(tr, tasks)
     with open(path, "w") as f:
-        json.dump({"workload": wl.name, "trace": tr.tolist()}, f)
+        json.dump({"workload": wl.name, "summary": summ, "trace": tr.tolist(),
+                   "tasks": tasks.tolist(), "sm_begin": begin.tolist()}, f)
+    print(json.dumps(summ), file=sys.stderr)
 
 
 def main():

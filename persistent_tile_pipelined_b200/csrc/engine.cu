@@ -75,12 +75,12 @@ __device__ bool mbar_wait(const Params& p, uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Wait for ring stage `sidx` to land.  Consumer warps take stages round-robin, so a warp
-// can reach a slot before the slot's previous stage (sidx - NS) was even issued; a parity
-// wait there would match the previous phase.  The producer therefore tags each slot with
-// the stage it claimed (after that slot's previous stage was consumed, which implies its
-// full-barrier phase completed); waiting for the tag first keeps every parity wait at most
-// one phase ahead.
+// Wait for ring stage `sidx` to land.  GEMV stages are taken round-robin by single warps,
+// so a warp can reach a slot before the slot's previous stage (sidx - NS) was even
+// issued; a parity wait there would match the previous phase.  The producer therefore
+// tags each slot with the stage it claimed (after that slot's previous stage was
+// consumed, which implies its full-barrier phase completed); waiting for the tag first
+// keeps every parity wait at most one phase ahead.
 __device__ bool stage_wait(const Params& p, uint64_t* full, const uint32_t* tags, uint32_t sidx) {
   const uint32_t NS = (uint32_t)p.ring_stages, slot = sidx % NS;
   const volatile uint32_t* tag = tags + slot;
@@ -100,25 +100,42 @@ __device__ bool stage_wait(const Params& p, uint64_t* full, const uint32_t* tags
 }
 
 // ---- task geometry (shared by producer and consumers) ---------------------------------------
+// GEMV task: rows [r0, r1) of the op's matrix (gate/up: the same rows of both matrices),
+// streamed as stages of whole contiguous rows (one bulk copy per matrix per stage).
 __device__ __forceinline__ int gemv_K(const Params& p, int op) {
   return op == OP_O ? p.Hq * p.D : (op == OP_DOWN ? p.F : p.d);
 }
-__device__ __forceinline__ int gemv_nseg(int op) { return op == OP_GU ? 2 : 1; }
-__device__ __forceinline__ int gemv_rps(const Params& p, int op) {
-  const int r = p.stage_bytes / (gemv_nseg(op) * gemv_K(p, op) * 2);
-  return r < 1 ? 1 : r;
-}
-__device__ __forceinline__ const uint16_t* gemv_w(const Params& p, int op, int layer, int seg) {
-  if (op == OP_LM) return p.lm_head;
+// Row n of segment `seg` of the op's matrix; *run receives how many rows from n on lie
+// in the same physical matrix (QKV rows cross from Wq into Wk into Wv).
+__device__ __forceinline__ const uint16_t* gemv_row(const Params& p, int op, int layer, int seg,
+                                                    int n, int K, int* run) {
+  *run = 0x7fffffff;
+  if (op == OP_LM) return p.lm_head + (size_t)n * K;
   const LayerPtrs& L = p.layers[layer];
   switch (op) {
-    case OP_Q: return L.w[TRE_W_Q];
-    case OP_K: return L.w[TRE_W_K];
-    case OP_V: return L.w[TRE_W_V];
-    case OP_O: return L.w[TRE_W_O];
-    case OP_GU: return seg ? L.w[TRE_W_UP] : L.w[TRE_W_GATE];
-    default: return L.w[TRE_W_DOWN];
+    case OP_QKV: {
+      const int nq = p.Hq * p.D, nk = p.Hkv * p.D;
+      if (n < nq) { *run = nq - n; return L.w[TRE_W_Q] + (size_t)n * K; }
+      if (n < nq + nk) { *run = nq + nk - n; return L.w[TRE_W_K] + (size_t)(n - nq) * K; }
+      return L.w[TRE_W_V] + (size_t)(n - nq - nk) * K;
+    }
+    case OP_O: return L.w[TRE_W_O] + (size_t)n * K;
+    case OP_GU: return (seg ? L.w[TRE_W_UP] : L.w[TRE_W_GATE]) + (size_t)n * K;
+    default: return L.w[TRE_W_DOWN] + (size_t)n * K;
   }
+}
+
+struct GemvGeom {
+  int K, nseg, rps, nstages;
+};
+
+__device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
+  GemvGeom g;
+  g.K = gemv_K(p, t.op);
+  g.nseg = t.op == OP_GU ? 2 : 1;
+  g.rps = gemv_rows_per_stage(g.K, g.nseg, p.stage_bytes);
+  g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
+  return g;
 }
 
 __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& t0, int& t1) {
@@ -128,56 +145,18 @@ __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& 
 }
 
 __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
-  if (t.type == T_GEMV) {
-    const int rps = gemv_rps(p, t.op);
-    return (t.r1 - t.r0 + rps - 1) / rps;
-  }
+  if (t.type == T_GEMV) return gemv_geom(p, t).nstages;
   int t0, t1;
   attn_range(p, t, t0, t1);
   return (t1 - t0 + p.pps - 1) / p.pps;
 }
 
-struct StageSrc {
-  const uint8_t* src0;
-  const uint8_t* src1;
-  uint32_t bytes0, bytes1, off1;
-};
-
-__device__ __forceinline__ StageSrc stage_desc(const Params& p, const Task& t, int i) {
-  StageSrc s;
-  if (t.type == T_GEMV) {
-    const int K = gemv_K(p, t.op), rps = gemv_rps(p, t.op);
-    const int n0 = t.r0 + i * rps, nr = min(rps, t.r1 - n0);
-    const size_t rowb = (size_t)K * 2;
-    s.src0 = reinterpret_cast<const uint8_t*>(gemv_w(p, t.op, t.layer, 0)) + (size_t)n0 * rowb;
-    s.bytes0 = (uint32_t)(nr * rowb);
-    if (t.op == OP_GU) {
-      s.src1 = reinterpret_cast<const uint8_t*>(gemv_w(p, t.op, t.layer, 1)) + (size_t)n0 * rowb;
-      s.bytes1 = s.bytes0;
-      s.off1 = (uint32_t)(rps * rowb);
-    } else {
-      s.src1 = nullptr;
-      s.bytes1 = 0;
-      s.off1 = 0;
-    }
-  } else {
-    int t0, t1;
-    attn_range(p, t, t0, t1);
-    const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
-    const size_t rowb = (size_t)p.D * 2;
-    const LayerPtrs& L = p.layers[t.layer];
-    const size_t off = ((size_t)t.r0 * p.cap + tt) * rowb;
-    s.src0 = reinterpret_cast<const uint8_t*>(L.k_cache) + off;
-    s.src1 = reinterpret_cast<const uint8_t*>(L.v_cache) + off;
-    s.bytes0 = s.bytes1 = (uint32_t)(n * rowb);
-    s.off1 = (uint32_t)(p.pps * rowb);
-  }
-  return s;
-}
-
 // ---- producer -------------------------------------------------------------------------------
+// The whole producer warp issues a stage: lane 0 claims the slot (waits for its "empty"
+// phase) and announces the stage's byte count on the "full" barrier; lane j then copies
+// segment j (one weight row's K-chunk, or the K / V rows of the stage's positions).
 __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ring,
-                         uint64_t* full, uint64_t* empty, uint32_t* tags) {
+                         uint64_t* full, uint64_t* empty, uint32_t* tags, int lane) {
   const uint64_t pol = l2_policy_evict_first();
   const uint32_t NS = (uint32_t)p.ring_stages;
   const uint32_t SB = (uint32_t)p.stage_bytes;
@@ -185,25 +164,76 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
   bool ok = true;
   for (int ti = 0; ti < ntask && ok; ++ti) {
     const Task t = my[ti];
-    if ((p.flags & TRE_DEBUG_NO_OVERLAP) && !wait_dep(p, t)) {
-      ok = false;
-      break;
+    if (p.flags & TRE_DEBUG_NO_OVERLAP) {
+      bool r = true;
+      if (lane == 0) r = wait_dep(p, t);
+      ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+      if (!ok) break;
     }
     const int ns = task_nstages(p, t);
+    GemvGeom g{};
+    int t0 = 0, t1 = 0;
+    if (t.type == T_GEMV) g = gemv_geom(p, t);
+    else attn_range(p, t, t0, t1);
     for (int i = 0; i < ns; ++i, ++gs) {
       const uint32_t slot = gs % NS, ph = (gs / NS) & 1u;
-      if (!mbar_wait(p, &empty[slot], ph ^ 1u)) {
+      bool r = true;
+      if (lane == 0) r = mbar_wait(p, &empty[slot], ph ^ 1u);
+      if (__shfl_sync(0xffffffffu, r ? 1 : 0, 0) == 0) {
         ok = false;
         break;
       }
-      const StageSrc s = stage_desc(p, t, i);
-      *reinterpret_cast<volatile uint32_t*>(tags + slot) = gs;
-      mbar_arrive_expect_tx(&full[slot], s.bytes0 + s.bytes1);
-      bulk_g2s(ring + (size_t)slot * SB, s.src0, s.bytes0, &full[slot], pol);
-      if (s.bytes1) bulk_g2s(ring + (size_t)slot * SB + s.off1, s.src1, s.bytes1, &full[slot], pol);
+      uint8_t* dst = ring + (size_t)slot * SB;
+      const uint8_t* src = nullptr;
+      uint32_t bytes = 0, total = 0;
+      if (t.type == T_GEMV) {
+        const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
+        const size_t rowb = (size_t)g.K * 2;
+        total = (uint32_t)(g.nseg * nr * rowb);
+        if (g.nseg == 2) {  // gate rows, then up rows at a fixed offset
+          if (lane < 2) {
+            int run;
+            src = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, lane, n0, g.K, &run));
+            dst += (size_t)lane * g.rps * rowb;
+            bytes = (uint32_t)(nr * rowb);
+          }
+        } else if (lane < 3) {  // the stage's rows, cut where they cross physical matrices
+          int n = n0, left = nr, piece = 0;
+          while (left > 0) {
+            int run;
+            const uint16_t* w = gemv_row(p, t.op, t.layer, 0, n, g.K, &run);
+            const int take = min(left, run);
+            if (piece == lane) {
+              src = reinterpret_cast<const uint8_t*>(w);
+              dst += (size_t)(n - n0) * rowb;
+              bytes = (uint32_t)(take * rowb);
+            }
+            n += take;
+            left -= take;
+            ++piece;
+          }
+        }
+      } else {
+        const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
+        const size_t rowb = (size_t)p.D * 2;
+        total = (uint32_t)(2 * n * rowb);
+        if (lane < 2) {
+          const LayerPtrs& L = p.layers[t.layer];
+          const uint16_t* base = lane == 0 ? L.k_cache : L.v_cache;
+          src = reinterpret_cast<const uint8_t*>(base) + ((size_t)t.r0 * p.cap + tt) * rowb;
+          dst += lane * (size_t)p.pps * rowb;
+          bytes = (uint32_t)(n * rowb);
+        }
+      }
+      if (lane == 0) {
+        *reinterpret_cast<volatile uint32_t*>(tags + slot) = gs;
+        mbar_arrive_expect_tx(&full[slot], total);
+      }
+      __syncwarp();
+      if (bytes) bulk_g2s(dst, src, bytes, &full[slot], pol);
     }
   }
-  if (!ok) {
+  if (!ok && lane == 0) {
     // Abort: let the copies still in flight land before the CTA can exit.
     const uint32_t first = gs > NS ? gs - NS : 0u;
     for (uint32_t k = first; k < gs; ++k) {
@@ -243,7 +273,7 @@ __device__ __forceinline__ float resid_in(const Params& p, int layer, int n) {
 __device__ __forceinline__ int input_key(const Task& t) {
   int cls;
   switch (t.op) {
-    case OP_Q: case OP_K: case OP_V: cls = 0; break;
+    case OP_QKV: cls = 0; break;
     case OP_O: cls = 1; break;
     case OP_GU: cls = 2; break;
     case OP_DOWN: cls = 3; break;
@@ -253,14 +283,15 @@ __device__ __forceinline__ int input_key(const Task& t) {
 }
 
 // Stage the GEMV input into the two planes; returns the RMSNorm scale (1 when none).
-__device__ float load_input(const Params& p, const Task& t, float* xlo, float* xhi, float* red,
-                            int ctid) {
+__device__ float load_input(const Params& p, const Task& t, float* ub, float* red, int ctid) {
   const int K = gemv_K(p, t.op);
+  float* xlo = ub;
+  float* xhi = ub + K / 2;
   const float* src = nullptr;
   const uint16_t* src_bf = nullptr;
   const uint16_t* gain = nullptr;
   switch (t.op) {
-    case OP_Q: case OP_K: case OP_V:
+    case OP_QKV:
       gain = p.layers[t.layer].w[TRE_W_ATTN_NORM];
       if (t.layer > 0) src = p.x;
       else if (p.x_in) src = p.x_in;
@@ -318,10 +349,16 @@ __device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float&
   sincosf((float)red, &s, &c);
 }
 
+// One split of the split-KV decode attention for kv head g = t.r0 (split t.r1 of t.aux):
+// the G query heads of the group attend to cached positions [t0, t1) streamed through the
+// ring (every warp takes 8 positions of every stage); the last split also takes the new
+// position pos from this step's k / v, appends them to the caches and merges its partial.
+// The last split of the group to finish (arrival ticket) combines all splits — the fused
+// combine — and publishes the group.
 template <int G, int DPL>
 __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
                           uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
-                          float* red, int* flag, int warp, int lane, int ctid, bool& abort_out) {
+                          int* flag, int warp, int lane, int ctid, bool& abort_out) {
   constexpr int D = 32 * DPL;
   const int g = t.r0, split = t.r1, S = t.aux;
   const bool last = (split == S - 1);
@@ -390,16 +427,18 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   const uint32_t NS = (uint32_t)p.ring_stages;
   int t0, t1;
   attn_range(p, t, t0, t1);
-  const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
-  for (int i = first; i < ns; i += kConsumerWarps) {
+  for (int i = 0; i < ns; ++i) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
     if (!stage_wait(p, full, tags, sidx)) {
       abort_out = true;
       break;
     }
-    const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
-    const uint8_t* kb = ring + (size_t)slot * p.stage_bytes;
-    attn_stage<G, DPL>(kb, kb + (size_t)p.pps * D * 2, n, q, m, l, o, lane);
+    const int n = min(p.pps, t1 - (t0 + i * p.pps));
+    const int nw = min(kPosPerWarp, n - warp * kPosPerWarp);
+    if (nw > 0) {
+      const uint8_t* kb = ring + (size_t)slot * p.stage_bytes + (size_t)warp * kPosPerWarp * D * 2;
+      attn_warp_positions<G, DPL>(kb, kb + (size_t)p.pps * D * 2, nw, q, m, l, o, lane);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
   }
@@ -455,19 +494,29 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   }
   consumer_sync(kConsumerThreads);
   if (*flag) {  // last split of this kv head to finish: combine all splits
+    // (m, l) of every split into shared memory in one round trip (reuses the warp scratch)
+    float* ms = ow;
+    float* ls = ow + G * S;
+    for (int idx = ctid; idx < G * S; idx += kConsumerThreads) {
+      const float* src = p.part + ((size_t)(g * G) * S + idx) * pstride;  // head idx/S, split idx%S
+      ms[idx] = __ldcg(src + D);
+      ls[idx] = __ldcg(src + D + 1);
+    }
+    consumer_sync(kConsumerThreads);
     for (int idx = ctid; idx < G * D; idx += kConsumerThreads) {
       const int h = idx / D, dd = idx % D;
-      const float* src = p.part + (size_t)(g * G + h) * S * pstride;
+      const float* mh = ms + h * S;
+      const float* lh = ls + h * S;
       float M = -INFINITY;
-      for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, __ldcg(src + s2 * pstride + D));
-      float O = 0.f, Ls = 0.f;
+      for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mh[s2]);
+      float Ls = 0.f, O = 0.f;
+      const float* src = p.part + (size_t)(g * G + h) * S * pstride + dd;
+      // independent loads: the splits' outputs are fetched together, not one at a time
+#pragma unroll 8
       for (int s2 = 0; s2 < S; ++s2) {
-        const float ms = __ldcg(src + s2 * pstride + D);
-        if (ms != -INFINITY) {
-          const float sc = exp2f(ms - M);
-          O = fmaf(sc, __ldcg(src + s2 * pstride + dd), O);
-          Ls = fmaf(sc, __ldcg(src + s2 * pstride + D + 1), Ls);
-        }
+        const float w = mh[s2] == -INFINITY ? 0.f : exp2f(mh[s2] - M);
+        Ls = fmaf(w, lh[s2], Ls);
+        O = fmaf(w, __ldcg(src + s2 * pstride), O);
       }
       p.attn[(size_t)(g * G + h) * D + dd] = O / Ls;
     }
@@ -479,23 +528,46 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
 
 __device__ __forceinline__ void run_attn(const Params& p, const Task& t, uint32_t gs, int ns,
                                          uint8_t* ring, uint64_t* full, uint64_t* empty,
-                                         const uint32_t* tags, float* ub, float* red, int* flag,
-                                         int warp, int lane, int ctid, bool& ab) {
+                                         const uint32_t* tags, float* ub, int* flag, int warp,
+                                         int lane, int ctid, bool& ab) {
   const int G = p.Hq / p.Hkv;
+#define TRE_ATTN(GG, DD) \
+  attn_task<GG, DD>(p, t, gs, ns, ring, full, empty, tags, ub, flag, warp, lane, ctid, ab)
   if (p.D == 128) {
     switch (G) {
-      case 1: attn_task<1, 4>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
-      case 2: attn_task<2, 4>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
-      case 4: attn_task<4, 4>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
-      default: attn_task<8, 4>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
+      case 1: TRE_ATTN(1, 4); break;
+      case 2: TRE_ATTN(2, 4); break;
+      case 4: TRE_ATTN(4, 4); break;
+      default: TRE_ATTN(8, 4); break;
     }
   } else {
     switch (G) {
-      case 1: attn_task<1, 2>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
-      case 2: attn_task<2, 2>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
-      case 4: attn_task<4, 2>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
-      default: attn_task<8, 2>(p, t, gs, ns, ring, full, empty, tags, ub, red, flag, warp, lane, ctid, ab); break;
+      case 1: TRE_ATTN(1, 2); break;
+      case 2: TRE_ATTN(2, 2); break;
+      case 4: TRE_ATTN(4, 2); break;
+      default: TRE_ATTN(8, 2); break;
     }
+  }
+#undef TRE_ATTN
+}
+
+// ---- GEMV epilogue ---------------------------------------------------------------------------------
+__device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, int n, float v, float rn,
+                                          Best& best) {
+  switch (t.op) {
+    case OP_QKV: p.qkv[n] = v * rn; break;
+    case OP_O: p.h1[n] = resid_in(p, t.layer, n) + v; break;
+    case OP_DOWN: {
+      const float y = __ldcg(p.h1 + n) + v;
+      p.x[n] = y;
+      if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
+      if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
+    } break;
+    default: {
+      const float y = v * rn;
+      p.logits[n] = y;
+      best_update(best, y, n);
+    } break;
   }
 }
 
@@ -508,9 +580,6 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
   int* flags = reinterpret_cast<int*>(misc + 32);         // [0] abort, [1] ticket
   float* rn_s = misc + 40;
   const uint32_t NS = (uint32_t)p.ring_stages;
-  const int half = p.xs_floats / 2;
-  float* xlo = ub;
-  float* xhi = ub + half;
   uint32_t gs = 0;
   int cur_key = -1;
   bool ab = false;
@@ -533,20 +602,22 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
 
     if (t.type == T_ATTN) {
       cur_key = -1;  // the attention scratch aliases the input-vector planes
-      run_attn(p, t, gs, ns, ring, full, empty, tags, ub, red, flags + 1, warp, lane, ctid, ab);
+      run_attn(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
     } else {
       const int key = input_key(t);
       if (key != cur_key) {
-        const float rn = load_input(p, t, xlo, xhi, red, ctid);
+        const float rn = load_input(p, t, ub, red, ctid);
         if (ctid == 0) *rn_s = rn;
         consumer_sync(kConsumerThreads);
         cur_key = key;
       }
       const float rn = *rn_s;
-      const int op = t.op, K = gemv_K(p, op), K8 = K >> 3, rps = gemv_rps(p, op);
-      const float4* xl = reinterpret_cast<const float4*>(xlo);
-      const float4* xh = reinterpret_cast<const float4*>(xhi);
+      const GemvGeom g = gemv_geom(p, t);
+      const int K8 = g.K >> 3;
+      const float4* xl = reinterpret_cast<const float4*>(ub);
+      const float4* xh = reinterpret_cast<const float4*>(ub + g.K / 2);
       Best best{-INFINITY, 0x7fffffff};
+      // stage gs + i belongs to warp (gs + i) % 8; each warp takes its stages in order
       const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
       for (int i = first; i < ns; i += kConsumerWarps) {
         const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
@@ -554,40 +625,48 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
           ab = true;
           break;
         }
-        const uint8_t* sp = ring + (size_t)slot * p.stage_bytes;
-        const int n0 = t.r0 + i * rps, nr = min(rps, t.r1 - n0);
-        if (op == OP_GU) {
-          gemv_stage_pairs(sp, (size_t)rps * K * 2, K8, nr, xl, xh, lane,
-                           [&](int r, float gt, float up) {
-                             const float a = gt * rn, b = up * rn;
-                             p.u[n0 + r] = a / (1.f + expf(-a)) * b;
-                           });
-        } else {
-          gemv_stage_rows(sp, K8, nr, xl, xh, lane, [&](int r, float v) {
-            const int n = n0 + r;
-            switch (op) {
-              case OP_Q: p.qkv[n] = v * rn; break;
-              case OP_K: p.qkv[(size_t)p.Hq * p.D + n] = v * rn; break;
-              case OP_V: p.qkv[(size_t)(p.Hq + p.Hkv) * p.D + n] = v * rn; break;
-              case OP_O: p.h1[n] = resid_in(p, t.layer, n) + v; break;
-              case OP_DOWN: {
-                const float y = __ldcg(p.h1 + n) + v;
-                p.x[n] = y;
-                if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
-                if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
-              } break;
-              default: {
-                const float y = v * rn;
-                p.logits[n] = y;
-                best_update(best, y, n);
-              } break;
+        const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
+        const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
+        if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+          const uint4* up = sp + (size_t)g.rps * K8;
+          for (int r = 0; r < nr; r += 2) {
+            const int np = min(2, nr - r);
+            float o[4];
+            const uint4* rows[4] = {sp + (size_t)r * K8, sp + (size_t)(r + np - 1) * K8,
+                                    up + (size_t)r * K8, up + (size_t)(r + np - 1) * K8};
+            if (np == 2) {
+              gemv_rows<4, 1>(rows, K8, xl, xh, lane, o);
+            } else {
+              const uint4* rows2[4] = {rows[0], rows[2], rows[2], rows[2]};
+              gemv_rows<2, 2>(rows2, K8, xl, xh, lane, o);
             }
-          });
+            const float v = reduce4(o[0], o[1], o[2], o[3], lane);
+            // np == 2: lanes 0 / 8 hold gate r / r+1, lanes 16 / 24 up r / r+1
+            // np == 1: lane 0 holds gate r, lane 8 up r
+            const float upv = __shfl_xor_sync(0xffffffffu, v, np == 2 ? 16 : 8);
+            const int k = (lane >> 3) & 1;
+            if ((np == 2 && (lane & 23) == 0) || (np == 1 && lane == 0)) {
+              const float a = v * rn, bb = upv * rn;
+              p.u[n0 + r + k] = a / (1.f + expf(-a)) * bb;
+            }
+          }
+        } else {
+          for (int r = 0; r < nr; r += 4) {
+            const int nv = min(4, nr - r);
+            const uint4* rows[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rows[q] = sp + (size_t)(r + min(q, nv - 1)) * K8;
+            float o[4];
+            gemv_rows_n(nv, rows, K8, xl, xh, lane, o);
+            const float v = reduce4(o[0], o[1], o[2], o[3], lane);
+            const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+            if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, n0 + r + idx, v, rn, best);
+          }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (lane == 0) mbar_arrive_n(&empty[slot], kConsumerWarps);
       }
-      if (op == OP_LM) {
+      if (t.op == OP_LM) {
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) {
           Best o;
@@ -602,10 +681,10 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       }
       __threadfence();
       consumer_sync(kConsumerThreads);
-      if (op == OP_LM && ctid == 0) {
-        Best b{-INFINITY, 0x7fffffff};
-        for (int w = 0; w < kConsumerWarps; ++w) best_update(b, red[w], reinterpret_cast<int*>(red)[16 + w]);
-        atomicMax(p.argmax_slot, pack_best(b));
+      if (t.op == OP_LM && ctid == 0) {
+        Best bb{-INFINITY, 0x7fffffff};
+        for (int w = 0; w < kConsumerWarps; ++w) best_update(bb, red[w], reinterpret_cast<int*>(red)[16 + w]);
+        atomicMax(p.argmax_slot, pack_best(bb));
         __threadfence();
         const uint32_t old = atom_acq_rel_gpu_add(p.lm_ticket, 1u);
         if (((old + 1u) % (uint32_t)t.aux) == 0u) {
@@ -638,15 +717,15 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
 
   if (threadIdx.x == 0) {
     for (uint32_t i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&full[i], 1);                 // the producer's arrive + the copies' bytes
+      mbar_init(&empty[i], kConsumerWarps);   // 8 arrivals: all warps, or one warp's 8
       tags[i] = 0xffffffffu;
     }
     fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
-    if (threadIdx.x == kConsumerThreads) producer(p, my, ntask, ring, full, empty, tags);
+    producer(p, my, ntask, ring, full, empty, tags, threadIdx.x & 31);
     return;
   }
   consumer(p, my, ntask, ring, full, empty, tags, ub, misc);

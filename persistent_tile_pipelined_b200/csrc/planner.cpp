@@ -180,13 +180,14 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   s.has_lm = c.has_embed_lm_head;
   const int G = s.Hq / s.Hkv;
 
-  // Largest bytes one ring stage must hold: a full row (or the gate+up row pair).
-  int64_t need = std::max<int64_t>({2LL * s.d * 2, (int64_t)s.F * 2, (int64_t)s.Hq * s.D * 2,
-                                     4LL * s.D /* one KV position, K and V */});
+  // A ring stage holds whole weight rows (gate/up: a row of each matrix), or the K and V
+  // rows of up to 64 cached positions.
+  const int need = std::max({2 * s.d * 2, s.F * 2, s.Hq * s.D * 2, 4 * s.D});
   int sb = c.stage_bytes ? c.stage_bytes : kDefaultStageBytes;
-  while (sb < need && sb < kMaxStageBytes) sb += 1024;
+  if (!c.stage_bytes)
+    while (sb < need && sb < kMaxStageBytes) sb += 1024;
   if (sb < need)
-    return fail(TRE_ERR_UNSUPPORTED, "a weight row is wider than the largest ring stage (64 KiB)");
+    return fail(TRE_ERR_UNSUPPORTED, "a weight row (or gate/up row pair) is wider than a ring stage");
   s.stage_bytes = sb;
   s.pos_per_stage = std::min(kMaxPosPerStage, sb / (4 * s.D));
 
@@ -213,6 +214,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     int max_s = std::max(1, (s.cap - 1 + s.pos_per_stage - 1) / s.pos_per_stage);
     S = std::min(S, max_s);
   }
+  // the combine stages every split's (m, l) in the attention scratch: 2 G S <= 8 G D
+  if (S > 4 * s.D) return fail(TRE_ERR_UNSUPPORTED, "kv_splits above 4 * head_dim");
   s.kv_splits = S;
 
   Builder b(nsm);
@@ -222,10 +225,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   for (int l = 0; l < s.L; ++l) {
     const int cq = counter_of(l, C_QKV), ca = counter_of(l, C_ATTN), co = counter_of(l, C_O),
               cg = counter_of(l, C_GU), cd = counter_of(l, C_DOWN);
-    int nqkv = 0;
-    nqkv += b.gemv(OP_Q, l, s.Hq * s.D, d2, prev_down, prev_down_count, cq);
-    nqkv += b.gemv(OP_K, l, s.Hkv * s.D, d2, prev_down, prev_down_count, cq);
-    nqkv += b.gemv(OP_V, l, s.Hkv * s.D, d2, prev_down, prev_down_count, cq);
+    // Q, K and V as one op over the stacked matrix [Wq; Wk; Wv]
+    const int nqkv = b.gemv(OP_QKV, l, (s.Hq + 2 * s.Hkv) * s.D, d2, prev_down, prev_down_count, cq);
     const int64_t kv_task_bytes = (int64_t)(s.cap - s.M) / S * s.D * 2 * 2;
     b.attention(l, s.Hkv, S, kv_task_bytes, cq, (uint32_t)nqkv, ca);
     int no = b.gemv(OP_O, l, s.d, (int64_t)s.Hq * s.D * 2, ca, (uint32_t)s.Hkv, co);

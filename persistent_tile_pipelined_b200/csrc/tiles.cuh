@@ -1,5 +1,6 @@
-// Tile micro-kernels of the persistent engine: warp-level compute on one shared-memory
-// ring stage.  The stage layouts here must match stage_desc() in engine.cu.
+// Tile micro-kernels of the persistent engine: per-warp compute on one shared-memory ring
+// stage.  Every consumer warp processes every stage (its own rows, or its own positions);
+// the stage layouts here must match the producer's stage_copy() in engine.cu.
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -58,72 +59,62 @@ __device__ __forceinline__ float reduce32(float (&v)[32], int lane) {
   return v[0];
 }
 
-// ---- GEMV on one stage ------------------------------------------------------------------
-// The stage holds rows [n0, n0 + nr) of the op's matrix (and, for the gate/up op, the same
-// rows of the second matrix at byte offset seg1).  x is the input vector in two planes:
-// xl[j] = x[8j : 8j+4], xh[j] = x[8j+4 : 8j+8].  `emit(row, value)` is called by one lane
-// per row with the full dot product (gate/up: emit2(row, gate, up)).
-template <class Emit>
-__device__ __forceinline__ void gemv_stage_rows(const uint8_t* slot, int K8, int nr,
-                                                const float4* __restrict__ xl,
-                                                const float4* __restrict__ xh, int lane,
-                                                Emit&& emit) {
-  const uint4* base = reinterpret_cast<const uint4*>(slot);
-  for (int r = 0; r < nr; r += 4) {
-    const uint4* w0 = base + (size_t)r * K8;
-    const uint4* w1 = base + (size_t)min(r + 1, nr - 1) * K8;
-    const uint4* w2 = base + (size_t)min(r + 2, nr - 1) * K8;
-    const uint4* w3 = base + (size_t)min(r + 3, nr - 1) * K8;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+// ---- GEMV: one warp computes NR (<= 4) whole rows of a stage ------------------------------
+// rows[r] points at row r's K8 16-byte vectors in shared memory; x planes xl[j] = x[8j:8j+4],
+// xh[j] = x[8j+4:8j+8].  NACC independent accumulators per row keep enough FMA chains in
+// flight when a stage holds only one or two (long) rows.
+template <int NR, int NACC>
+__device__ __forceinline__ void gemv_rows(const uint4* const (&rows)[4], int K8,
+                                          const float4* __restrict__ xl,
+                                          const float4* __restrict__ xh, int lane,
+                                          float (&out)[4]) {
+  float acc[NR][NACC];
+#pragma unroll
+  for (int r = 0; r < NR; ++r)
+#pragma unroll
+    for (int a = 0; a < NACC; ++a) acc[r][a] = 0.f;
+  int j = lane;
 #pragma unroll 2
-    for (int j = lane; j < K8; j += 32) {
-      const float4 x0 = xl[j], x1 = xh[j];
-      a0 = dot8(w0[j], x0, x1, a0);
-      a1 = dot8(w1[j], x0, x1, a1);
-      a2 = dot8(w2[j], x0, x1, a2);
-      a3 = dot8(w3[j], x0, x1, a3);
+  for (; j + 32 * (NACC - 1) < K8; j += 32 * NACC) {
+#pragma unroll
+    for (int a = 0; a < NACC; ++a) {
+      const float4 x0 = xl[j + 32 * a], x1 = xh[j + 32 * a];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) acc[r][a] = dot8(rows[r][j + 32 * a], x0, x1, acc[r][a]);
     }
-    const float v = reduce4(a0, a1, a2, a3, lane);
-    const int row = r + ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-    if ((lane & 7) == 0 && row < nr) emit(row, v);
+  }
+  for (; j < K8; j += 32) {
+    const float4 x0 = xl[j], x1 = xh[j];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) acc[r][0] = dot8(rows[r][j], x0, x1, acc[r][0]);
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    float v = 0.f;
+    if (r < NR) {
+#pragma unroll
+      for (int a = 0; a < NACC; ++a) v += acc[r][a];
+    }
+    out[r] = v;
   }
 }
 
-template <class Emit2>
-__device__ __forceinline__ void gemv_stage_pairs(const uint8_t* slot, size_t seg1, int K8, int nr,
-                                                 const float4* __restrict__ xl,
-                                                 const float4* __restrict__ xh, int lane,
-                                                 Emit2&& emit2) {
-  const uint4* g = reinterpret_cast<const uint4*>(slot);
-  const uint4* u = reinterpret_cast<const uint4*>(slot + seg1);
-  for (int r = 0; r < nr; r += 2) {
-    const int rb = min(r + 1, nr - 1);
-    const uint4* g0 = g + (size_t)r * K8;
-    const uint4* g1 = g + (size_t)rb * K8;
-    const uint4* u0 = u + (size_t)r * K8;
-    const uint4* u1 = u + (size_t)rb * K8;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 2
-    for (int j = lane; j < K8; j += 32) {
-      const float4 x0 = xl[j], x1 = xh[j];
-      a0 = dot8(g0[j], x0, x1, a0);
-      a1 = dot8(g1[j], x0, x1, a1);
-      a2 = dot8(u0[j], x0, x1, a2);
-      a3 = dot8(u1[j], x0, x1, a3);
-    }
-    // lanes 0 / 8 hold gate(r) / gate(r+1); lanes 16 / 24 hold up(r) / up(r+1)
-    const float v = reduce4(a0, a1, a2, a3, lane);
-    const float up = __shfl_xor_sync(0xffffffffu, v, 16);
-    const int row = r + ((lane >> 3) & 1);
-    if ((lane & 23) == 0 && row < nr) emit2(row, v, up);
+__device__ __forceinline__ void gemv_rows_n(int nr, const uint4* const (&rows)[4], int K8,
+                                            const float4* xl, const float4* xh, int lane,
+                                            float (&out)[4]) {
+  switch (nr) {
+    case 4: gemv_rows<4, 1>(rows, K8, xl, xh, lane, out); break;
+    case 3: gemv_rows<3, 1>(rows, K8, xl, xh, lane, out); break;
+    case 2: gemv_rows<2, 2>(rows, K8, xl, xh, lane, out); break;
+    default: gemv_rows<1, 4>(rows, K8, xl, xh, lane, out); break;
   }
 }
 
-// ---- split-KV decode attention on one stage -----------------------------------------------
+// ---- split-KV decode attention: a warp's positions of one stage ----------------------------
 // G query heads share one kv head; lane owns dims [lane*DPL, lane*DPL + DPL) of D = 32*DPL.
 // q is pre-scaled by log2(e)/sqrt(D) so scores are in log2 units.  Running state per warp:
-// m[h] (max), l[h] (sum of 2^(s-m)), o[h][:] (sum of 2^(s-m) v).  kb / vb hold n <= 64
-// consecutive positions of K and V rows (bf16, D each).
+// m[h] (max), l[h] (sum of 2^(s-m)), o[h][:] (sum of 2^(s-m) v).  kb / vb point at this
+// warp's first position's K and V rows (bf16, D each); nw <= kPosPerWarp positions.
 template <int DPL>
 __device__ __forceinline__ void load_bf16_row(const uint8_t* p, float (&f)[DPL]) {
   if constexpr (DPL == 4) {
@@ -136,21 +127,24 @@ __device__ __forceinline__ void load_bf16_row(const uint8_t* p, float (&f)[DPL])
 }
 
 template <int G, int DPL>
-__device__ __forceinline__ void attn_stage(const uint8_t* kb, const uint8_t* vb, int n,
-                                           const float (&q)[G][DPL], float (&m)[G], float (&l)[G],
-                                           float (&o)[G][DPL], int lane) {
+__device__ __forceinline__ void attn_warp_positions(const uint8_t* kb, const uint8_t* vb, int nw,
+                                                    const float (&q)[G][DPL], float (&m)[G],
+                                                    float (&l)[G], float (&o)[G][DPL], int lane) {
   constexpr int D = 32 * DPL;
-  constexpr int CP = 32 / G;                 // positions per 32-score chunk
-  constexpr int NCH = kMaxPosPerStage / CP;  // chunks per stage (max)
+  constexpr int CP = 32 / G;                                   // positions per 32 scores
+  constexpr int PPC = CP < kPosPerWarp ? CP : kPosPerWarp;     // positions per chunk
+  constexpr int NCH = kPosPerWarp / PPC;                       // chunks per warp
   float sc[NCH];
 #pragma unroll
   for (int c = 0; c < NCH; ++c) {
     sc[c] = -INFINITY;
-    if (c * CP < n) {
+    if (c * PPC < nw) {
       float v[32];
 #pragma unroll
-      for (int pp = 0; pp < CP; ++pp) {
-        const int t = min(c * CP + pp, n - 1);
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+#pragma unroll
+      for (int pp = 0; pp < PPC; ++pp) {
+        const int t = min(c * PPC + pp, nw - 1);
         float kf[DPL];
         load_bf16_row<DPL>(kb + ((size_t)t * D + lane * DPL) * 2, kf);
 #pragma unroll
@@ -161,11 +155,12 @@ __device__ __forceinline__ void attn_stage(const uint8_t* kb, const uint8_t* vb,
           v[pp * G + h] = a;
         }
       }
-      const float s = reduce32(v, lane);  // score of position c*CP + lane/G, head lane%G
-      if (c * CP + lane / G < n) sc[c] = s;
+      const float s = reduce32(v, lane);  // score of position c*PPC + lane/G, head lane%G
+      const int pp = lane / G;
+      if (pp < PPC && c * PPC + pp < nw) sc[c] = s;
     }
   }
-  // stage max per head (lanes with equal lane % G)
+  // this stage's max per head (lanes with equal lane % G)
   float mx = -INFINITY;
 #pragma unroll
   for (int c = 0; c < NCH; ++c) mx = fmaxf(mx, sc[c]);
@@ -198,19 +193,17 @@ __device__ __forceinline__ void attn_stage(const uint8_t* kb, const uint8_t* vb,
   // o += p V
 #pragma unroll
   for (int c = 0; c < NCH; ++c) {
-    if (c * CP < n) {
 #pragma unroll
-      for (int pp = 0; pp < CP; ++pp) {
-        const int t = c * CP + pp;
-        if (t < n) {
-          float vf[DPL];
-          load_bf16_row<DPL>(vb + ((size_t)t * D + lane * DPL) * 2, vf);
+    for (int pp = 0; pp < PPC; ++pp) {
+      const int t = c * PPC + pp;
+      if (t < nw) {
+        float vf[DPL];
+        load_bf16_row<DPL>(vb + ((size_t)t * D + lane * DPL) * 2, vf);
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pr = __shfl_sync(0xffffffffu, sc[c], pp * G + h);
+        for (int h = 0; h < G; ++h) {
+          const float pr = __shfl_sync(0xffffffffu, sc[c], pp * G + h);
 #pragma unroll
-            for (int j = 0; j < DPL; ++j) o[h][j] = fmaf(pr, vf[j], o[h][j]);
-          }
+          for (int j = 0; j < DPL; ++j) o[h][j] = fmaf(pr, vf[j], o[h][j]);
         }
       }
     }

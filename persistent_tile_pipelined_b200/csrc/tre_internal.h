@@ -12,24 +12,37 @@ constexpr int kConsumerWarps = 8;                      // compute warps
 constexpr int kConsumerThreads = kConsumerWarps * 32;  // 256
 constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
 constexpr int kMaxGroup = 8;                           // q heads per kv head (GQA)
-constexpr int kMaxPosPerStage = 64;                    // KV positions per attention stage
+constexpr int kPosPerWarp = 8;                         // KV positions per warp per stage
+constexpr int kMaxPosPerStage = kConsumerWarps * kPosPerWarp;  // 64
 constexpr int kDefaultStageBytes = 32768;
 constexpr int kMaxStageBytes = 65536;
 constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per block
+
+#ifdef __CUDACC__
+#define TRE_HD __host__ __device__
+#else
+#define TRE_HD
+#endif
+
+// ---- GEMV stage geometry ----------------------------------------------------------------
+// A GEMV stage holds `rows per stage` whole contiguous rows of the op's matrix (gate/up:
+// the same rows of both matrices); one consumer warp computes the whole stage.
+TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes) {
+  const int r = stage_bytes / (nseg * K * 2);
+  return r < 1 ? 1 : r;
+}
 
 // ---- tasks --------------------------------------------------------------------------
 enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1 };
 
 // GEMV ops: which matrix, which input vector, which epilogue.
 enum GemvOp : uint8_t {
-  OP_Q = 0,     // in: RMSNorm(x; attn_norm)  -> qkv[0 : Hq*D]
-  OP_K = 1,     // in: RMSNorm(x; attn_norm)  -> qkv[Hq*D : +Hkv*D]
-  OP_V = 2,     // in: RMSNorm(x; attn_norm)  -> qkv[(Hq+Hkv)*D : +Hkv*D]
-  OP_O = 3,     // in: attn                   -> h1 = x + Wo attn
-  OP_GU = 4,    // in: RMSNorm(h1; ffn_norm)  -> u = silu(Wg hn) * (Wu hn)   (2 segments)
-  OP_DOWN = 5,  // in: u                      -> x = h1 + Wd u
-  OP_LM = 6,    // in: RMSNorm(x; final_norm) -> logits, greedy argmax
-  OP_COUNT = 7
+  OP_QKV = 0,   // in: RMSNorm(x; attn_norm)  -> qkv = [Wq; Wk; Wv] xn  (rows of the stacked matrix)
+  OP_O = 1,     // in: attn                   -> h1 = x + Wo attn
+  OP_GU = 2,    // in: RMSNorm(h1; ffn_norm)  -> u = silu(Wg hn) * (Wu hn)   (2 segments)
+  OP_DOWN = 3,  // in: u                      -> x = h1 + Wd u
+  OP_LM = 4,    // in: RMSNorm(x; final_norm) -> logits, greedy argmax
+  OP_COUNT = 5
 };
 
 // Dependency counters: one per (layer, stage of the layer), then the LM head and a
@@ -63,7 +76,7 @@ struct PlanShape {
   int kv_splits, pos_per_stage;
   int xs_floats;       // input-vector buffer (floats)
   int attn_floats;     // attention scratch (floats), aliases the input-vector buffer
-  int ub_floats;       // max(xs_floats, attn_floats): the shared union buffer
+  int ub_floats;       // the shared union buffer: input planes, or attention scratch
   int smem_bytes;
   int n_counters;
   int n_lm_tasks;

@@ -74,7 +74,11 @@ LLAMA8B = Workload(name="llama3-8b-shaped", kind="gqa", n_layers=32, hidden=4096
                    n_kv_heads=8, head_dim=128, ffn=14336, vocab=128256, prefill=4096,
                    decode_steps=64, rope_theta=5e5, norm_eps=1e-5)
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B)}
+# The same layer shapes with 4 layers: a ~3.8 GB case (well above the 126 MB L2) for
+# profiler captures that must stay small.
+LLAMA8B_4L = LLAMA8B.replace(name="llama3-8b-shaped-4L", n_layers=4)
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L)}
 
 
 def gqa_layer_shapes(w: Workload) -> List[tuple]:

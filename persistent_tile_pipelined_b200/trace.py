@@ -1,0 +1,83 @@
+"""Per-task trace of one engine step: statistics and a Chrome-trace (chrome://tracing) file.
+
+An engine created with TRE_DEBUG_TRACE records, for every task, the global-timer
+nanoseconds when its consumer warps started waiting for its dependency, when the
+dependency was met, when the task finished, and the SM it ran on.  Combined with the plan
+(``tre_plan_tasks``), this gives per-op time, dependency-wait (idle) time and the spread
+of finish times across SMs — the straggler effect at every op boundary.
+"""
+from __future__ import annotations
+
+import json
+from collections import defaultdict
+
+import numpy as np
+
+OP_NAMES = {0: "qkv", 1: "o_proj", 2: "gate_up", 3: "down", 4: "lm_head"}
+
+
+def task_table(tasks: np.ndarray) -> dict:
+    """Decode the 8-int32 task descriptors of ``tre_plan_tasks`` into columns by task id."""
+    w0 = tasks[:, 0].astype(np.int64) & 0xFFFFFFFF
+    order = np.argsort(tasks[:, 7])
+    cols = {"type": w0 & 0xFF, "op": (w0 >> 8) & 0xFF, "layer": (w0 >> 16) & 0xFFFF,
+            "r0": tasks[:, 4], "r1": tasks[:, 5]}
+    return {k: v[order] for k, v in cols.items()}
+
+
+def op_name(tt: dict, i: int) -> str:
+    return "attention" if tt["type"][i] == 1 else OP_NAMES.get(int(tt["op"][i]), "?")
+
+
+def summarize(trace: np.ndarray, tasks: np.ndarray) -> dict:
+    """trace: [n_tasks][4] int64 (start, ready, end, sm) indexed by task id."""
+    tt = task_table(tasks)
+    t0 = trace[:, 0].min()
+    start, ready, end = trace[:, 0] - t0, trace[:, 1] - t0, trace[:, 2] - t0
+    step_ns = float(end.max())
+    per_op = defaultdict(lambda: {"tasks": 0, "wait_ns": 0.0, "busy_ns": 0.0})
+    spans = defaultdict(list)
+    for i in range(len(trace)):
+        name = op_name(tt, i)
+        d = per_op[name]
+        d["tasks"] += 1
+        d["wait_ns"] += float(ready[i] - start[i])
+        d["busy_ns"] += float(end[i] - ready[i])
+        spans[(int(tt["layer"][i]), name)].append((start[i], ready[i], end[i]))
+    # straggler spread: for each (layer, op), last finish minus median finish
+    spread = defaultdict(list)
+    for (layer, name), v in spans.items():
+        ends = np.array([e for _, _, e in v], dtype=np.float64)
+        spread[name].append(float(ends.max() - np.median(ends)))
+    nsm = int(trace[:, 3].max()) + 1
+    busy = np.zeros(nsm)
+    waitt = np.zeros(nsm)
+    for i in range(len(trace)):
+        busy[int(trace[i, 3])] += end[i] - ready[i]
+        waitt[int(trace[i, 3])] += ready[i] - start[i]
+    return {
+        "step_us": step_ns / 1e3,
+        "per_op": {k: {"tasks": v["tasks"], "mean_wait_us": v["wait_ns"] / v["tasks"] / 1e3,
+                       "mean_busy_us": v["busy_ns"] / v["tasks"] / 1e3}
+                   for k, v in per_op.items()},
+        "finish_spread_us": {k: {"mean": float(np.mean(v)) / 1e3, "max": float(np.max(v)) / 1e3}
+                             for k, v in spread.items()},
+        "sm_wait_frac_mean": float(np.mean(waitt) / step_ns),
+        "sm_busy_frac_mean": float(np.mean(busy) / step_ns),
+    }
+
+
+def chrome_trace(trace: np.ndarray, tasks: np.ndarray, path: str) -> None:
+    tt = task_table(tasks)
+    t0 = trace[:, 0].min()
+    ev = []
+    for i in range(len(trace)):
+        s, r, e, sm = (int(x) for x in trace[i])
+        name = f"L{int(tt['layer'][i])}.{op_name(tt, i)}"
+        if r > s:
+            ev.append({"name": "wait", "ph": "X", "ts": (s - t0) / 1e3, "dur": (r - s) / 1e3,
+                       "pid": 0, "tid": sm, "cat": "wait"})
+        ev.append({"name": name, "ph": "X", "ts": (r - t0) / 1e3, "dur": (e - r) / 1e3,
+                   "pid": 0, "tid": sm, "cat": op_name(tt, i)})
+    with open(path, "w") as f:
+        json.dump({"traceEvents": ev, "displayTimeUnit": "ns"}, f)

@@ -16,7 +16,7 @@ build.build_engine()
 from persistent_tile_pipelined_b200 import tre  # noqa: E402
 
 T_GEMV, T_ATTN = 0, 1
-OP_Q, OP_K, OP_V, OP_O, OP_GU, OP_DOWN, OP_LM = range(7)
+OP_QKV, OP_O, OP_GU, OP_DOWN, OP_LM = range(5)
 C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_PER_LAYER = range(6)
 
 
@@ -88,9 +88,8 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
         else:
             assert T["dep_count"][i] == len(producers), (i, dep, kind)
     # every GEMV op's output rows are partitioned exactly once per layer
-    rows_of = {OP_Q: wl.n_q_heads * wl.head_dim, OP_K: wl.n_kv_heads * wl.head_dim,
-               OP_V: wl.n_kv_heads * wl.head_dim, OP_O: wl.hidden, OP_GU: wl.ffn,
-               OP_DOWN: wl.hidden, OP_LM: wl.vocab}
+    rows_of = {OP_QKV: (wl.n_q_heads + 2 * wl.n_kv_heads) * wl.head_dim, OP_O: wl.hidden,
+               OP_GU: wl.ffn, OP_DOWN: wl.hidden, OP_LM: wl.vocab}
     for l in range(wl.n_layers):
         for op, N in rows_of.items():
             if op == OP_LM and l != wl.n_layers - 1:
