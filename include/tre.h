@@ -177,6 +177,31 @@ tre_status tre_decode_step(tre_engine* e, int32_t token, int32_t pos, tre_stream
 tre_status tre_decode_step_host(tre_engine* e, int32_t token, int32_t pos, tre_stream stream,
                                 float* logits_host, int32_t* token_host);
 
+/* One decode step, like tre_decode_step, for callers that cannot allocate GPU memory
+ * (the pages have no counterpart: it exists for this library's users).  Some callers
+ * cannot call cudaMalloc — code running under a framework allocator that must own every
+ * byte, real-time loops where allocation is forbidden, plug-ins handed only raw
+ * pointers — so no engine is created: each call plans the step on the host (ordinary CPU
+ * memory) and keeps everything the kernel needs beyond the caller's tensors (task list,
+ * counters, activations, split-KV partials) in one fixed device array built into the
+ * library, 4 MiB per GPU, held by every GPU that loads the library until the process exits.
+ * The call allocates no GPU memory: no cudaMalloc / cudaMallocAsync / cudaHostAlloc and no
+ * cudaFree.
+ *   cfg, w       as for tre_create (weights and caches caller owned); no debug flags
+ *   token, pos   as for tre_decode_step; the step runs on the CURRENT device
+ *   logits_dev   device fp32[vocab], required;  token_dev  device int32[1] or NULL
+ *   status_dev   device int32[2] or NULL: set to {0, 0}, then on a device error to
+ *                {TRE_ERR_DEP_TIMEOUT or TRE_ERR_BOUNDS, task index}
+ * Returns TRE_ERR_UNSUPPORTED, before enqueuing anything, when the model's plan needs
+ * more than the 4 MiB array.  The first call on a device looks up the array's device
+ * address; make that first call before any stream capture.  Every call shares the array
+ * and leaves the previous call's contents in it (the call clears what must start at
+ * zero): calls whose work overlaps on the GPU — two streams, two threads — race and give
+ * undefined results; calls in one stream are ordered. */
+tre_status tre_decode_step_static(const tre_config* cfg, const tre_weights* w, int32_t token,
+                                  int32_t pos, tre_stream stream, float* logits_dev,
+                                  int32_t* token_dev, int32_t* status_dev);
+
 /* ---- status / debug ----------------------------------------------------------- */
 
 /* Wait for the engine's last stream, then report the device status word: 0, or a

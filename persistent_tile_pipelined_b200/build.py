@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 ENGINE_LIB = os.path.join(PKG, "libtre.so")
 SYNTH_LIB = os.path.join(PKG, "synth", "libtre_synth.so")
 
-ENGINE_SOURCES = ["planner.cpp", "tre_api.cu", "engine.cu"]
+ENGINE_SOURCES = ["planner.cpp", "tre_api.cu", "engine.cu", "noalloc.cu"]
 ENGINE_HEADERS = ["tre_internal.h", "ptx.cuh", "tiles.cuh"]
 
 NVCC_FLAGS = [

@@ -64,6 +64,7 @@ class tre_plan_info(ctypes.Structure):
 
 
 EXPORTED = ("tre_create", "tre_destroy", "tre_decode_step", "tre_decode_step_host",
+            "tre_decode_step_static",
             "tre_get_status", "tre_reset", "tre_debug_hidden", "tre_debug_trace",
             "tre_step_bytes", "tre_plan_inspect", "tre_plan_tasks", "tre_last_error")
 
@@ -80,6 +81,8 @@ def _load() -> ctypes.CDLL:
     L.tre_destroy.restype = None
     L.tre_decode_step.argtypes = [vp, i32, i32, vp, vp, vp]
     L.tre_decode_step_host.argtypes = [vp, i32, i32, vp, vp, vp]
+    L.tre_decode_step_static.argtypes = [ctypes.POINTER(tre_config), ctypes.POINTER(tre_weights),
+                                         i32, i32, vp, vp, vp, vp]
     L.tre_get_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.tre_reset.argtypes = [vp, vp]
     L.tre_debug_hidden.argtypes = [vp, vp, vp]
@@ -91,7 +94,8 @@ def _load() -> ctypes.CDLL:
     L.tre_plan_tasks.restype = i32
     L.tre_last_error.argtypes = []
     L.tre_last_error.restype = ctypes.c_char_p
-    for name in ("tre_create", "tre_decode_step", "tre_decode_step_host", "tre_get_status",
+    for name in ("tre_create", "tre_decode_step", "tre_decode_step_host",
+                 "tre_decode_step_static", "tre_get_status",
                  "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
                  "tre_plan_inspect"):
         getattr(L, name).restype = ctypes.c_int
@@ -141,6 +145,17 @@ def tre_decode_step_host(h, token: int, pos: int, stream: int = 0,
     check(lib.tre_decode_step_host(h, int(token), int(pos), ctypes.c_void_p(stream or None), lp,
                                    ctypes.byref(tok)), "tre_decode_step_host")
     return tok.value
+
+
+def tre_decode_step_static(cfg: tre_config, weights: tre_weights, token: int, pos: int,
+                           stream: int = 0, logits_dev: int = 0, token_dev: int = 0,
+                           status_dev: int = 0) -> int:
+    """One decode step that allocates no GPU memory (see include/tre.h); returns the status."""
+    return lib.tre_decode_step_static(ctypes.byref(cfg), ctypes.byref(weights), int(token),
+                                      int(pos), ctypes.c_void_p(stream or None),
+                                      ctypes.c_void_p(logits_dev or None),
+                                      ctypes.c_void_p(token_dev or None),
+                                      ctypes.c_void_p(status_dev or None))
 
 
 def tre_get_status(h):
@@ -217,6 +232,26 @@ def upload_gqa_model(model: dict, device="cuda:0") -> dict:
         if k in model:
             out[k] = _dev_tensor(model[k], device)
     return out
+
+
+def make_weights(cfg: tre_config, dev_model: dict):
+    """A tre_weights struct over the device tensors of `dev_model`.  Returns (weights,
+    keepalive): keep `keepalive` referenced while the struct is in use."""
+    L = cfg.n_layers
+    layer_w = (ctypes.c_void_p * (L * TRE_W_SLOTS))()
+    for l in range(L):
+        for slot, t in dev_model["layers"][l].items():
+            layer_w[l * TRE_W_SLOTS + slot] = t.data_ptr()
+    kc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["k_cache"]])
+    vc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["v_cache"]])
+    w = tre_weights()
+    for k in ("embed", "final_norm", "lm_head"):
+        if k in dev_model:
+            setattr(w, k, dev_model[k].data_ptr())
+    w.layer_w = ctypes.cast(layer_w, ctypes.POINTER(ctypes.c_void_p))
+    w.k_cache = ctypes.cast(kc, ctypes.POINTER(ctypes.c_void_p))
+    w.v_cache = ctypes.cast(vc, ctypes.POINTER(ctypes.c_void_p))
+    return w, (layer_w, kc, vc, dev_model)
 
 
 class Engine:
