@@ -52,6 +52,18 @@ class _GqaLayer(ctypes.Structure):
 _SLOT_NAMES = ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "wgate", "wup", "wdown")
 
 
+class _MlaConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("hidden", "n_heads", "q_lora", "kv_lora",
+                                               "rope_dim", "nope_dim", "v_dim", "kv_capacity")] + [
+        ("rope_theta", ctypes.c_double), ("norm_eps", ctypes.c_double)]
+
+
+class _MlaLayer(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("attn_norm", "w_dq", "q_norm", "w_uq", "w_dkv", "kv_norm", "w_uk", "w_uv", "w_o",
+                 "latent_cache")]
+
+
 def _ptr(a: np.ndarray) -> ctypes.c_void_p:
     assert a.flags.c_contiguous, "oracle arrays must be C-contiguous"
     return a.ctypes.data_as(ctypes.c_void_p)
@@ -86,6 +98,10 @@ class Oracle:
         L.orc_gqa_layer_step.argtypes = [vp, vp, i32, vp]
         L.orc_gqa_layers_step.argtypes = [vp, vp, i32, vp, vp]
         L.orc_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp]
+        L.orc_gqa_attn_block.argtypes = [vp, vp, i32, vp, vp]
+        L.orc_swiglu_mlp.argtypes = [i32, i32, vp, vp, vp, vp, vp]
+        L.orc_router_topk.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
+        L.orc_mla_layer_step.argtypes = [vp, vp, i32, vp]
 
     # -- pieces ------------------------------------------------------------------
     def _r(self, a) -> np.ndarray:
@@ -164,6 +180,68 @@ class Oracle:
                                  int(token), int(pos), _ptr(logits),
                                  _ptr(hidden) if hidden is not None else None)
         return logits, hidden
+
+    def swiglu_mlp(self, wgate, wup, wdown, hn):
+        wg, wu, wd = (np.ascontiguousarray(a, dtype=np.uint16) for a in (wgate, wup, wdown))
+        F, d = wg.shape
+        assert wu.shape == (F, d) and wd.shape == (d, F)
+        hn = self._r(hn)
+        y = np.empty(d, dtype=self.real)
+        self.lib.orc_swiglu_mlp(d, F, _ptr(wg), _ptr(wu), _ptr(wd), _ptr(hn), _ptr(y))
+        return y
+
+    def router_topk(self, wr, hn, top_k: int):
+        """(idx[top_k], w[top_k], scores[E]) of the sigmoid top-k router."""
+        wr = np.ascontiguousarray(wr, dtype=np.uint16)
+        E, d = wr.shape
+        hn = self._r(hn)
+        idx = np.empty(top_k, dtype=np.int32)
+        w = np.empty(top_k, dtype=self.real)
+        sc = np.empty(E, dtype=self.real)
+        self.lib.orc_router_topk(E, int(top_k), d, _ptr(wr), _ptr(hn), _ptr(idx), _ptr(w), _ptr(sc))
+        return idx, w, sc
+
+    def gqa_attn_block(self, wl, layer: dict, k_cache, v_cache, pos: int, x):
+        """h1 = x + Wo attention(RMSNorm(x)); appends this token's k, v to the caches."""
+        cfg = _GqaConfig(1, wl.hidden, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ffn,
+                         wl.vocab, wl.kv_capacity, float(wl.rope_theta), float(wl.norm_eps))
+        L = _GqaLayer()
+        for slot, name in enumerate(_SLOT_NAMES[:5]):
+            setattr(L, name, _ptr(layer[slot]).value)
+        L.k_cache = _ptr(k_cache).value
+        L.v_cache = _ptr(v_cache).value
+        x = self._r(x)
+        h1 = np.empty_like(x)
+        self.lib.orc_gqa_attn_block(ctypes.byref(cfg), ctypes.byref(L), int(pos), _ptr(x), _ptr(h1))
+        return h1
+
+    def moe_layer_step(self, wl, layer: dict, k_cache, v_cache, experts, pos: int, x):
+        """One MoE decoder layer: the GQA attention block, then
+        x = h1 + sum_i w_i Expert_{idx_i}(hn) + Shared(hn), hn = RMSNorm(h1).
+        `experts(e)` returns routed expert e's (W_gate, W_up, W_down).
+        Returns (x_out, idx, w)."""
+        h1 = self.gqa_attn_block(wl, layer, k_cache, v_cache, pos, x)
+        hn = self.rmsnorm(h1, layer[5], wl.norm_eps)
+        idx, w, _ = self.router_topk(layer[6], hn, wl.top_k)
+        y = np.zeros(wl.hidden, dtype=self.real)
+        for i, e in enumerate(idx):
+            y += w[i] * self.swiglu_mlp(*experts(int(e)), hn)
+        y += self.swiglu_mlp(layer[7], layer[8], layer[9], hn)
+        return h1 + y, idx, w
+
+    def mla_layer_step(self, wl, layer: dict, latent_cache, pos: int, x):
+        """One absorbed-MLA layer (attention only); appends this token's latent row."""
+        cfg = _MlaConfig(wl.hidden, wl.n_q_heads, wl.q_lora, wl.kv_lora, wl.rope_dim,
+                         wl.nope_dim, wl.v_dim, wl.kv_capacity, float(wl.rope_theta),
+                         float(wl.norm_eps))
+        L = _MlaLayer()
+        for slot, name in enumerate(("attn_norm", "w_dq", "q_norm", "w_uq", "w_dkv", "kv_norm",
+                                     "w_uk", "w_uv", "w_o")):
+            setattr(L, name, _ptr(layer[slot]).value)
+        L.latent_cache = _ptr(latent_cache).value
+        x = self._r(x).copy()
+        self.lib.orc_mla_layer_step(ctypes.byref(cfg), ctypes.byref(L), int(pos), _ptr(x))
+        return x
 
     def layers_step(self, wl, model, x, pos: int):
         """Layers only: returns (x_out[d], hidden[L][d])."""

@@ -168,23 +168,20 @@ typedef struct {
   uint16_t *k_cache, *v_cache; /* [Hkv][cap][D] bf16, written at pos */
 } orc_gqa_layer;
 
-/* One pre-norm GQA decoder layer at position pos, residual x[d] updated in place:
+/* The attention block of a pre-norm GQA layer at position pos:
  *   xn = RMSNorm(x); q,k,v = Wq xn, Wk xn, Wv xn; RoPE(q, k at pos);
  *   cache[pos] = bf16(k), bf16(v); o = attention over positions [0, pos];
- *   h1 = x + Wo o; x = h1 + Wdown (silu(Wgate RMSNorm(h1)) * (Wup RMSNorm(h1))). */
-void orc_gqa_layer_step(const orc_gqa_config* c, const orc_gqa_layer* L, int pos, real* x) {
-  int d = c->hidden, Hq = c->n_q_heads, Hkv = c->n_kv_heads, D = c->head_dim, F = c->ffn;
+ *   h1 = x + Wo o. */
+void orc_gqa_attn_block(const orc_gqa_config* c, const orc_gqa_layer* L, int pos, const real* x,
+                        real* h1) {
+  int d = c->hidden, Hq = c->n_q_heads, Hkv = c->n_kv_heads, D = c->head_dim;
   int cap = c->kv_capacity;
   real* xn = (real*)malloc(sizeof(real) * d);
   real* q = (real*)malloc(sizeof(real) * (size_t)Hq * D);
   real* k = (real*)malloc(sizeof(real) * (size_t)Hkv * D);
   real* v = (real*)malloc(sizeof(real) * (size_t)Hkv * D);
   real* o = (real*)malloc(sizeof(real) * (size_t)Hq * D);
-  real* h1 = (real*)malloc(sizeof(real) * d);
-  real* g = (real*)malloc(sizeof(real) * F);
-  real* u = (real*)malloc(sizeof(real) * F);
   real* y = (real*)malloc(sizeof(real) * d);
-
   orc_rmsnorm(d, x, L->attn_norm, c->norm_eps, xn);
   orc_gemv(Hq * D, d, L->wq, xn, q);
   orc_gemv(Hkv * D, d, L->wk, xn, k);
@@ -199,15 +196,35 @@ void orc_gqa_layer_step(const orc_gqa_config* c, const orc_gqa_layer* L, int pos
   orc_attention(Hq, Hkv, D, pos + 1, cap, q, L->k_cache, L->v_cache, o, NULL);
   orc_gemv(d, Hq * D, L->wo, o, y);
   for (int i = 0; i < d; ++i) h1[i] = x[i] + y[i];
+  free(xn); free(q); free(k); free(v); free(o); free(y);
+}
 
-  orc_rmsnorm(d, h1, L->ffn_norm, c->norm_eps, xn);
-  orc_gemv(F, d, L->wgate, xn, g);
-  orc_gemv(F, d, L->wup, xn, u);
+/* A SwiGLU MLP on an already-normalised input: y = Wd (silu(Wg hn) * (Wu hn)), F hidden
+ * units.  Serves the dense MLP, every routed expert and the shared expert. */
+void orc_swiglu_mlp(int d, int F, const uint16_t* wgate, const uint16_t* wup,
+                    const uint16_t* wdown, const real* hn, real* y) {
+  real* g = (real*)malloc(sizeof(real) * F);
+  real* u = (real*)malloc(sizeof(real) * F);
+  orc_gemv(F, d, wgate, hn, g);
+  orc_gemv(F, d, wup, hn, u);
   for (int i = 0; i < F; ++i) g[i] = orc_silu(g[i]) * u[i];
-  orc_gemv(d, F, L->wdown, g, y);
-  for (int i = 0; i < d; ++i) x[i] = h1[i] + y[i];
+  orc_gemv(d, F, wdown, g, y);
+  free(g);
+  free(u);
+}
 
-  free(xn); free(q); free(k); free(v); free(o); free(h1); free(g); free(u); free(y);
+/* One pre-norm GQA decoder layer at position pos, residual x[d] updated in place:
+ * h1 = attention block; x = h1 + SwiGLU(RMSNorm(h1)). */
+void orc_gqa_layer_step(const orc_gqa_config* c, const orc_gqa_layer* L, int pos, real* x) {
+  int d = c->hidden;
+  real* h1 = (real*)malloc(sizeof(real) * d);
+  real* hn = (real*)malloc(sizeof(real) * d);
+  real* y = (real*)malloc(sizeof(real) * d);
+  orc_gqa_attn_block(c, L, pos, x, h1);
+  orc_rmsnorm(d, h1, L->ffn_norm, c->norm_eps, hn);
+  orc_swiglu_mlp(d, c->ffn, L->wgate, L->wup, L->wdown, hn, y);
+  for (int i = 0; i < d; ++i) x[i] = h1[i] + y[i];
+  free(h1); free(hn); free(y);
 }
 
 /* Layers only: x[d] in, x[d] out, hidden[l*d] (optional) after every layer. */
@@ -233,6 +250,131 @@ void orc_decode_step(const orc_gqa_config* c, const uint16_t* embed, const uint1
   orc_gemv(c->vocab, d, lm_head, xn, logits);
   free(x);
   free(xn);
+}
+
+/* ------------------------------------------------------------------ MoE ------------ */
+
+/* Router of a mixture-of-experts MLP (the pages name the fused op ExpertSelectUpGateSiLU,
+ * TileRT code audit, MoE paragraph, but print no formula; read as DeepSeek-style
+ * sigmoid routing): s_e = sigmoid(W_r[e] . hn) for e < E; the top_k experts by s, ties
+ * to the lower index; w_i = s_i / sum of the selected s.  idx[top_k], w[top_k] in
+ * descending score order; scores (optional) receives all E scores. */
+void orc_router_topk(int E, int top_k, int d, const uint16_t* wr, const real* hn, int* idx,
+                     real* w, real* scores) {
+  real* s = (real*)malloc(sizeof(real) * E);
+  orc_gemv(E, d, wr, hn, s);
+  for (int e = 0; e < E; ++e) s[e] = (real)(1.0 / (1.0 + exp(-(double)s[e])));
+  char* taken = (char*)calloc((size_t)E, 1);
+  real tot = 0;
+  for (int i = 0; i < top_k; ++i) {
+    int best = -1;
+    for (int e = 0; e < E; ++e)
+      if (!taken[e] && (best < 0 || s[e] > s[best])) best = e;
+    taken[best] = 1;
+    idx[i] = best;
+    w[i] = s[best];
+    tot += s[best];
+  }
+  for (int i = 0; i < top_k; ++i) w[i] /= tot;
+  if (scores) memcpy(scores, s, sizeof(real) * E);
+  free(taken);
+  free(s);
+}
+
+/* ------------------------------------------------------------------ absorbed MLA ---- */
+
+typedef struct {
+  int32_t hidden, n_heads, q_lora, kv_lora, rope_dim, nope_dim, v_dim, kv_capacity;
+  double rope_theta, norm_eps;
+} orc_mla_config;
+
+typedef struct {
+  const uint16_t *attn_norm; /* [d]                          */
+  const uint16_t *w_dq;      /* [q_lora][d]                  */
+  const uint16_t *q_norm;    /* [q_lora]                     */
+  const uint16_t *w_uq;      /* [H * (nope + rope)][q_lora]  */
+  const uint16_t *w_dkv;     /* [kv_lora + rope][d]          */
+  const uint16_t *kv_norm;   /* [kv_lora]                    */
+  const uint16_t *w_uk;      /* [H * nope][kv_lora]          */
+  const uint16_t *w_uv;      /* [H * v][kv_lora]             */
+  const uint16_t *w_o;       /* [d][H * v]                   */
+  uint16_t *latent_cache;    /* [cap][kv_lora + rope] bf16   */
+} orc_mla_layer;
+
+/* One absorbed multi-head latent attention layer (attention only) at position pos, residual
+ * x[d] updated in place.  The pages name FlashSparseMLA (batch == 1) and TokenSpeed's
+ * q-head folding (TileRT code audit) but print no formula; read as DeepSeek-V2 MLA with the
+ * up-projections absorbed:
+ *   xn = RMSNorm(x); c_q = RMSNorm(W_dq xn; q_norm); [q_nope_h, q_pe_h] = (W_uq c_q)_h;
+ *   [c_kv, k_pe] = W_dkv xn; c_kv = RMSNorm(c_kv; kv_norm); RoPE(q_pe_h), RoPE(k_pe) at pos;
+ *   cache[pos] = bf16([c_kv, k_pe]);
+ *   q_lat_h = W_uk,h^T q_nope_h;  s_h[t] = (q_lat_h . c_kv[t] + q_pe_h . k_pe[t]) / sqrt(nope+rope);
+ *   o_lat_h = sum_t softmax(s_h)[t] c_kv[t];  o_h = W_uv,h o_lat_h;  x = x + W_o [o_h]. */
+void orc_mla_layer_step(const orc_mla_config* c, const orc_mla_layer* L, int pos, real* x) {
+  const int d = c->hidden, H = c->n_heads, QL = c->q_lora, KL = c->kv_lora, R = c->rope_dim;
+  const int NP = c->nope_dim, VD = c->v_dim, QH = NP + R, C = KL + R, cap = c->kv_capacity;
+  real* xn = (real*)malloc(sizeof(real) * d);
+  real* cq = (real*)malloc(sizeof(real) * QL);
+  real* cqn = (real*)malloc(sizeof(real) * QL);
+  real* q = (real*)malloc(sizeof(real) * (size_t)H * QH);
+  real* kv = (real*)malloc(sizeof(real) * C);
+  real* ckv = (real*)malloc(sizeof(real) * KL);
+  real* qlat = (real*)malloc(sizeof(real) * (size_t)H * KL);
+  real* olat = (real*)malloc(sizeof(real) * (size_t)H * KL);
+  real* o = (real*)malloc(sizeof(real) * (size_t)H * VD);
+  real* y = (real*)malloc(sizeof(real) * d);
+  const int P = pos + 1;
+  real* sc = (real*)malloc(sizeof(real) * P);
+
+  orc_rmsnorm(d, x, L->attn_norm, c->norm_eps, xn);
+  orc_gemv(QL, d, L->w_dq, xn, cq);
+  orc_rmsnorm(QL, cq, L->q_norm, c->norm_eps, cqn);
+  orc_gemv(H * QH, QL, L->w_uq, cqn, q);
+  orc_gemv(C, d, L->w_dkv, xn, kv);
+  orc_rmsnorm(KL, kv, L->kv_norm, c->norm_eps, ckv);
+  orc_rope(R, pos, c->rope_theta, kv + KL);
+  for (int h = 0; h < H; ++h) orc_rope(R, pos, c->rope_theta, q + (size_t)h * QH + NP);
+  uint16_t* row = L->latent_cache + (size_t)pos * C;
+  for (int i = 0; i < KL; ++i) row[i] = orc_round_bf16(ckv[i]);
+  for (int i = 0; i < R; ++i) row[KL + i] = orc_round_bf16(kv[KL + i]);
+
+  /* q_lat_h[j] = sum_n W_uk[h*NP + n][j] * q_nope_h[n] */
+  for (int h = 0; h < H; ++h)
+    for (int j = 0; j < KL; ++j) {
+      real acc = 0;
+      for (int n = 0; n < NP; ++n)
+        acc += bf16_val(L->w_uk[((size_t)h * NP + n) * KL + j]) * q[(size_t)h * QH + n];
+      qlat[(size_t)h * KL + j] = acc;
+    }
+  const real scale = (real)(1.0 / sqrt((double)QH));
+  for (int h = 0; h < H; ++h) {
+    real m = -INFINITY;
+    for (int t = 0; t < P; ++t) {
+      const uint16_t* ct = L->latent_cache + (size_t)t * C;
+      real a = 0;
+      for (int j = 0; j < KL; ++j) a += qlat[(size_t)h * KL + j] * bf16_val(ct[j]);
+      for (int j = 0; j < R; ++j) a += q[(size_t)h * QH + NP + j] * bf16_val(ct[KL + j]);
+      sc[t] = a * scale;
+      if (sc[t] > m) m = sc[t];
+    }
+    real l = 0;
+    for (int t = 0; t < P; ++t) {
+      sc[t] = (real)exp((double)(sc[t] - m));
+      l += sc[t];
+    }
+    for (int j = 0; j < KL; ++j) {
+      real acc = 0;
+      for (int t = 0; t < P; ++t) acc += sc[t] / l * bf16_val(L->latent_cache[(size_t)t * C + j]);
+      olat[(size_t)h * KL + j] = acc;
+    }
+  }
+  /* o_h = W_uv,h o_lat_h */
+  for (int h = 0; h < H; ++h)
+    orc_gemv(VD, KL, L->w_uv + (size_t)h * VD * KL, olat + (size_t)h * KL, o + (size_t)h * VD);
+  orc_gemv(d, H * VD, L->w_o, o, y);
+  for (int i = 0; i < d; ++i) x[i] += y[i];
+  free(xn); free(cq); free(cqn); free(q); free(kv); free(ckv); free(qlat); free(olat);
+  free(o); free(y); free(sc);
 }
 
 int orc_real_bytes(void) { return (int)sizeof(real); }

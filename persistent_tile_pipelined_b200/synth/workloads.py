@@ -78,7 +78,19 @@ LLAMA8B = Workload(name="llama3-8b-shaped", kind="gqa", n_layers=32, hidden=4096
 # profiler captures that must stay small.
 LLAMA8B_4L = LLAMA8B.replace(name="llama3-8b-shaped-4L", n_layers=4)
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L)}
+# Absorbed-MLA decode layers x4 (attention only): hidden 7168, 128 heads, q_lora 1536,
+# kv_lora 512, rope 64, nope 128, v 128; latent KV cache 8192 positions; theta 1e4, eps 1e-6.
+MLA4 = Workload(name="mla-4L-d7168", kind="mla", n_layers=4, hidden=7168, n_q_heads=128,
+                q_lora=1536, kv_lora=512, rope_dim=64, nope_dim=128, v_dim=128, prefill=8192,
+                decode_steps=1, rope_theta=1e4, norm_eps=1e-6)
+
+# MoE decode layers x4: hidden 7168, 256 routed experts top-8 + 1 shared, expert SwiGLU 2048,
+# sigmoid router; GQA attention 64 q / 8 kv heads of dim 128 over 4096 positions.
+MOE4 = Workload(name="moe-4L-d7168", kind="moe", n_layers=4, hidden=7168, n_q_heads=64,
+                n_kv_heads=8, head_dim=128, prefill=4096, decode_steps=1, rope_theta=1e4,
+                norm_eps=1e-6, n_experts=256, top_k=8, n_shared=1, expert_ffn=2048)
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L, MLA4, MOE4)}
 
 
 def gqa_layer_shapes(w: Workload) -> List[tuple]:
@@ -95,6 +107,80 @@ def gqa_layer_shapes(w: Workload) -> List[tuple]:
         (7, (f, d), "w"),               # W_up
         (8, (d, f), "w"),               # W_down
     ]
+
+
+def mla_layer_shapes(w: Workload) -> List[tuple]:
+    """(slot, shape, kind) of every absorbed-MLA layer tensor."""
+    d, H, ql, kl, r = w.hidden, w.n_q_heads, w.q_lora, w.kv_lora, w.rope_dim
+    nope, v = w.nope_dim, w.v_dim
+    return [
+        (0, (d,), "g"),                     # attention RMSNorm gain
+        (1, (ql, d), "w"),                  # W_dq
+        (2, (ql,), "g"),                    # q_lora RMSNorm gain
+        (3, (H * (nope + r), ql), "w"),     # W_uq: per head [nope | rope] rows
+        (4, (kl + r, d), "w"),              # W_dkv: [kv_lora | rope] rows
+        (5, (kl,), "g"),                    # kv_lora RMSNorm gain
+        (6, (H * nope, kl), "w"),           # W_uk
+        (7, (H * v, kl), "w"),              # W_uv
+        (8, (d, H * v), "w"),               # W_o
+    ]
+
+
+def moe_layer_shapes(w: Workload) -> List[tuple]:
+    """(slot, shape, kind) of the non-expert tensors of a MoE layer."""
+    d, hq, hkv, dh = w.hidden, w.n_q_heads, w.n_kv_heads, w.head_dim
+    fs = w.expert_ffn * w.n_shared
+    return [
+        (0, (d,), "g"), (1, (hq * dh, d), "w"), (2, (hkv * dh, d), "w"),
+        (3, (hkv * dh, d), "w"), (4, (d, hq * dh), "w"),
+        (5, (d,), "g"),                     # MLP RMSNorm gain
+        (6, (w.n_experts, d), "w"),         # router
+        (7, (fs, d), "w"), (8, (fs, d), "w"), (9, (d, fs), "w"),   # shared expert
+    ]
+
+
+def tid_expert(layer: int, expert: int, which: int) -> int:
+    """Tensor id of routed expert `expert` of `layer`: which 0 = gate, 1 = up, 2 = down."""
+    return 1_000_000 + int(layer) * 100_000 + int(expert) * 4 + int(which)
+
+
+def gen_expert(w: Workload, layer: int, expert: int) -> tuple:
+    """(W_gate [F][d], W_up [F][d], W_down [d][F]) of one routed expert, on demand."""
+    F, d = w.expert_ffn, w.hidden
+    return (gen_tensor(w, tid_expert(layer, expert, 0), (F, d), "w"),
+            gen_tensor(w, tid_expert(layer, expert, 1), (F, d), "w"),
+            gen_tensor(w, tid_expert(layer, expert, 2), (d, F), "w"))
+
+
+def gen_mla_model(w: Workload) -> dict:
+    assert w.kind == "mla"
+    C = w.kv_lora + w.rope_dim
+    model = {"layers": [], "latent_cache": [], "x_in": normal_f32(w.seed, TID_X_IN, (w.hidden,))}
+    for l in range(w.n_layers):
+        model["layers"].append({slot: gen_tensor(w, tid_layer(l, slot), shape, kind)
+                                for slot, shape, kind in mla_layer_shapes(w)})
+        cache = np.zeros((w.kv_capacity, C), dtype=np.uint16)
+        if w.prefill:
+            cache[: w.prefill] = normal_bf16(w.seed, tid_kcache(l), (w.prefill, C), 0.0, 1.0)
+        model["latent_cache"].append(cache)
+    return model
+
+
+def gen_moe_model(w: Workload, with_experts: bool = False) -> dict:
+    """Non-expert tensors, KV caches and x_in; routed experts come from gen_expert on
+    demand (all of them when with_experts)."""
+    assert w.kind == "moe"
+    model = {
+        "layers": [{slot: gen_tensor(w, tid_layer(l, slot), shape, kind)
+                    for slot, shape, kind in moe_layer_shapes(w)} for l in range(w.n_layers)],
+        "k_cache": [gen_kv_cache(w, l, "k") for l in range(w.n_layers)],
+        "v_cache": [gen_kv_cache(w, l, "v") for l in range(w.n_layers)],
+        "x_in": normal_f32(w.seed, TID_X_IN, (w.hidden,), 0.0, 1.0),
+    }
+    if with_experts:
+        model["experts"] = [[gen_expert(w, l, e) for e in range(w.n_experts)]
+                            for l in range(w.n_layers)]
+    return model
 
 
 def gen_tensor(w: Workload, tensor_id: int, shape, kind: str,
