@@ -196,27 +196,36 @@ def cpu_baseline(wl, sample_layers: int, reps: int = 1):
     model = W.gen_gqa_model(sw)
     orc = oracle.Oracle(32)
     if reps > 1:
-        return [_time_sample(orc, wl, sw, model, sample_layers) for _ in range(reps)]
+        return [_time_sample(orc, wl, sw, model, sample_layers, 3.0) for _ in range(reps)]
     return _time_sample(orc, wl, sw, model, sample_layers)
 
 
-def _time_sample(orc, wl, sw, model, sample_layers):
+def _time_sample(orc, wl, sw, model, sample_layers, min_seconds: float = 10.0):
+    """Time the sliced step (and its layers alone) repeatedly until at least
+    `min_seconds` of CPU work has run; scale the median to the full stack."""
     from persistent_tile_pipelined_b200.synth import workloads as W
+
     tok = W.first_token(sw)
-    t0 = time.perf_counter()
-    orc.decode_step(sw, model, tok, sw.prefill, want_hidden=False)
-    t_step = time.perf_counter() - t0
-    x = np.zeros(sw.hidden, dtype=np.float32)
-    t0 = time.perf_counter()
-    orc.layers_step(sw, model, x + 0.01, sw.prefill)
-    t_layers = time.perf_counter() - t0
+    x = np.full(sw.hidden, 0.01, dtype=np.float32)
+    steps, layers = [], []
+    t_start = time.perf_counter()
+    while time.perf_counter() - t_start < min_seconds or len(steps) < 2:
+        t0 = time.perf_counter()
+        orc.decode_step(sw, model, tok, sw.prefill, want_hidden=False)
+        steps.append(time.perf_counter() - t0)
+        t0 = time.perf_counter()
+        orc.layers_step(sw, model, x, sw.prefill)
+        layers.append(time.perf_counter() - t0)
+    t_step, t_layers = float(np.median(steps)), float(np.median(layers))
     per_layer = t_layers / sample_layers
     t_full = per_layer * wl.n_layers + max(t_step - t_layers, 0.0)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    work = time.perf_counter() - t_start
     return {"value": 1.0 / t_full, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"fp32 oracle, {sample_layers} of {wl.n_layers} layers + LM head, one "
-                       f"decode step at pos {sw.prefill} (step {t_step:.2f} s, layers-only "
-                       f"{t_layers:.2f} s), scaled to the full stack: {t_full:.2f} s/token"),
+            "sample": (f"fp32 oracle, {sample_layers} of {wl.n_layers} layers + LM head, decode "
+                       f"step at pos {sw.prefill}, repeated {len(steps)}x ({work:.1f} s of CPU "
+                       f"work; median step {t_step:.3f} s, layers-only {t_layers:.3f} s), "
+                       f"scaled to the full stack: {t_full:.3f} s/token"),
             "seconds_per_token": t_full}
 
 

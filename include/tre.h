@@ -104,7 +104,10 @@ typedef struct {
   int32_t kv_splits;            /* split-KV chunks per kv head; 0 = planner's choice    */
   int32_t stage_bytes;          /* bytes per ring stage; 0 = 32768                      */
   int32_t ring_stages;          /* ring depth; 0 = as many as shared memory allows      */
-  int32_t reserved[8];          /* must be zero                                         */
+  int32_t l2_prefetch_kb;       /* per-SM budget (KiB) for asking L2 for the next task's
+                                   bytes when a task starts; <= 0 = off (the default:
+                                   measured slower on the 8B-shaped stack)              */
+  int32_t reserved[7];          /* must be zero                                         */
 } tre_config;
 
 /* Per-layer tensor slots.  layer_w[l * TRE_W_SLOTS + slot] is the device pointer of
@@ -217,9 +220,12 @@ tre_status tre_reset(tre_engine* e, tre_stream stream);
  * device) — requires TRE_DEBUG_HIDDEN. */
 tre_status tre_debug_hidden(tre_engine* e, float* hidden_dev, tre_stream stream);
 
-/* Copy the per-task trace of the last step to host memory: 4 int64 per task
- * (start ns, dependency met ns, end ns, sm id), in global task order.  Requires
- * TRE_DEBUG_TRACE.  *n_tasks receives the task count; trace_host may be NULL to query. */
+/* Copy the per-task trace of the last step to host memory: 8 int64 per task, in global
+ * task order: start ns (dependency wait begins), dependency met ns, end ns, SM id, then
+ * phase marks — GEMV: input vector staged, last stage consumed; attention: q ready,
+ * stages consumed, partial written and ticket taken — (0 where a mark does not apply).
+ * Requires TRE_DEBUG_TRACE.  *n_tasks receives the task count; trace_host may be NULL to
+ * query. */
 tre_status tre_debug_trace(tre_engine* e, int64_t* trace_host, int32_t* n_tasks);
 
 /* Bytes a step at `pos` streams from HBM (weights + KV read + KV written + logits). */

@@ -87,6 +87,7 @@ __device__ bool stage_wait(const Params& p, uint64_t* full, const uint32_t* tags
   if (*tag != sidx) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1; *tag != sidx; ++it) {
+      __nanosleep(64);  // yield issue slots to the warps that are computing
       if ((it & 63) == 0) {
         if (aborted(p)) return false;
         if ((long long)(globaltimer_ns() - t0) > 2 * p.timeout_ns) {
@@ -126,14 +127,29 @@ __device__ __forceinline__ const uint16_t* gemv_row(const Params& p, int op, int
 }
 
 struct GemvGeom {
-  int K, nseg, rps, nstages;
+  int K;        // full row length (inputs)
+  int nseg;     // 2 for gate/up (a row of each matrix), else 1
+  int np, part; // K-parts of the op and this task's part
+  int k0, Kp;   // this part's input columns [k0, k0 + Kp)
+  int rps;      // rows per ring stage
+  int nstages;
 };
 
 __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   GemvGeom g;
   g.K = gemv_K(p, t.op);
   g.nseg = t.op == OP_GU ? 2 : 1;
-  g.rps = gemv_rows_per_stage(g.K, g.nseg, p.stage_bytes);
+  if (t.op == OP_LM) {
+    g.np = 1;
+    g.part = 0;
+  } else {
+    g.part = t.aux & 0xff;
+    g.np = max(1, t.aux >> 8);
+  }
+  const int len = gemv_part_len(g.K, g.np);
+  g.k0 = g.part * len;
+  g.Kp = min(len, g.K - g.k0);
+  g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes);
   g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
   return g;
 }
@@ -152,24 +168,145 @@ __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
 }
 
 // ---- producer -------------------------------------------------------------------------------
+// Lane `lane`'s piece of stage i of task t: source, byte offset in the stage, bytes (0 = no
+// piece for this lane); *total receives the stage's byte count.  GEMV stages are whole
+// rows (gate/up: the rows of both matrices at a fixed offset; QKV: cut where the stacked
+// rows cross from Wq to Wk to Wv); attention stages are the K and V rows of up to `pps`
+// consecutive cached positions of one kv head.
+__device__ __forceinline__ const uint8_t* stage_piece(const Params& p, const Task& t,
+                                                      const GemvGeom& g, int t0, int t1, int i,
+                                                      int lane, uint32_t* off, uint32_t* bytes,
+                                                      uint32_t* total) {
+  const uint8_t* src = nullptr;
+  *off = 0;
+  *bytes = 0;
+  if (t.type == T_GEMV) {
+    const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
+    const size_t rowb = (size_t)g.Kp * 2;  // bytes of one row's part in the stage
+    *total = (uint32_t)(g.nseg * nr * rowb);
+    if (g.np > 1) {  // K-parts: rows are strided in memory, one copy per row
+      if (lane < nr * g.nseg) {
+        const int seg = lane / nr, r = lane % nr;
+        int run;
+        src = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, seg, n0 + r, g.K, &run) + g.k0);
+        *off = (uint32_t)((seg * g.rps + r) * rowb);
+        *bytes = (uint32_t)rowb;
+      }
+    } else if (g.nseg == 2) {
+      if (lane < 2) {
+        int run;
+        src = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, lane, n0, g.K, &run));
+        *off = (uint32_t)(lane * g.rps * rowb);
+        *bytes = (uint32_t)(nr * rowb);
+      }
+    } else if (lane < 3) {
+      int n = n0, left = nr, piece = 0;
+      while (left > 0) {
+        int run;
+        const uint16_t* w = gemv_row(p, t.op, t.layer, 0, n, g.K, &run);
+        const int take = min(left, run);
+        if (piece == lane) {
+          src = reinterpret_cast<const uint8_t*>(w);
+          *off = (uint32_t)((n - n0) * rowb);
+          *bytes = (uint32_t)(take * rowb);
+        }
+        n += take;
+        left -= take;
+        ++piece;
+      }
+    }
+  } else {
+    const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
+    const size_t rowb = (size_t)p.D * 2;
+    *total = (uint32_t)(2 * n * rowb);
+    if (lane < 2) {
+      const LayerPtrs& L = p.layers[t.layer];
+      const uint16_t* base = lane == 0 ? L.k_cache : L.v_cache;
+      src = reinterpret_cast<const uint8_t*>(base) + ((size_t)t.r0 * p.cap + tt) * rowb;
+      *off = (uint32_t)(lane * p.pps * rowb);
+      *bytes = (uint32_t)(n * rowb);
+    }
+  }
+  return src;
+}
+
+// L2 prefetch of a whole task ahead of its stages: the contiguous byte ranges task t will
+// stream (its rows of each matrix; or the K and V rows of its positions), as a few large
+// requests — a bulk request costs the same fixed time whatever its size, so one request
+// per range rather than one per stage.  At most `budget` bytes; K-part tasks (strided rows)
+// are skipped.
+__device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, int lane,
+                                              long long budget) {
+  const uint8_t* src[3] = {nullptr, nullptr, nullptr};
+  long long bytes[3] = {0, 0, 0};
+  if (t.type == T_GEMV) {
+    const GemvGeom g = gemv_geom(p, t);
+    if (g.np > 1) return;
+    const size_t rowb = (size_t)g.K * 2;
+    if (g.nseg == 2) {
+      for (int s = 0; s < 2; ++s) {
+        int run;
+        src[s] = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, s, t.r0, g.K, &run));
+        bytes[s] = (long long)(t.r1 - t.r0) * rowb;
+      }
+    } else {
+      int n = t.r0, left = t.r1 - t.r0;
+      for (int piece = 0; left > 0 && piece < 3; ++piece) {
+        int run;
+        src[piece] = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, 0, n, g.K, &run));
+        const int take = min(left, run);
+        bytes[piece] = (long long)take * rowb;
+        n += take;
+        left -= take;
+      }
+    }
+  } else {
+    int t0, t1;
+    attn_range(p, t, t0, t1);
+    const size_t rowb = (size_t)p.D * 2;
+    const LayerPtrs& L = p.layers[t.layer];
+    const size_t off = ((size_t)t.r0 * p.cap + t0) * rowb;
+    src[0] = reinterpret_cast<const uint8_t*>(L.k_cache) + off;
+    src[1] = reinterpret_cast<const uint8_t*>(L.v_cache) + off;
+    bytes[0] = bytes[1] = (long long)(t1 - t0) * rowb;
+  }
+  if (lane < 3 && src[lane]) {
+    long long before = 0;  // budget left after the pieces of lower lanes
+    for (int k = 0; k < lane; ++k) before += bytes[k];
+    long long n = min(bytes[lane], budget - before);
+    const uint8_t* a = src[lane];
+    while (n >= 16) {
+      const uint32_t chunk = (uint32_t)min(n, 1LL << 20) & ~15u;
+      bulk_prefetch_l2(a, chunk);
+      a += chunk;
+      n -= chunk;
+    }
+  }
+}
+
 // The whole producer warp issues a stage: lane 0 claims the slot (waits for its "empty"
-// phase) and announces the stage's byte count on the "full" barrier; lane j then copies
-// segment j (one weight row's K-chunk, or the K / V rows of the stage's positions).
+// phase) and announces the stage's byte count on the "full" barrier; each lane then copies
+// its piece.  When it starts a task it first asks L2 for the next task's bytes (up to
+// pf_window): weights and cached KV never depend on this step's activations, so HBM keeps
+// streaming through op boundaries even while the shared-memory ring is full.
 __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, uint32_t* tags, int lane) {
   const uint64_t pol = l2_policy_evict_first();
   const uint32_t NS = (uint32_t)p.ring_stages;
   const uint32_t SB = (uint32_t)p.stage_bytes;
+  const bool no_overlap = (p.flags & TRE_DEBUG_NO_OVERLAP) != 0;
+  const long long window = no_overlap ? 0 : p.pf_window;
   uint32_t gs = 0;
   bool ok = true;
   for (int ti = 0; ti < ntask && ok; ++ti) {
     const Task t = my[ti];
-    if (p.flags & TRE_DEBUG_NO_OVERLAP) {
+    if (no_overlap) {
       bool r = true;
       if (lane == 0) r = wait_dep(p, t);
       ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
       if (!ok) break;
     }
+    if (window > 0 && ti + 1 < ntask) task_prefetch(p, my[ti + 1], lane, window);
     const int ns = task_nstages(p, t);
     GemvGeom g{};
     int t0 = 0, t1 = 0;
@@ -183,54 +320,14 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
         ok = false;
         break;
       }
-      uint8_t* dst = ring + (size_t)slot * SB;
-      const uint8_t* src = nullptr;
-      uint32_t bytes = 0, total = 0;
-      if (t.type == T_GEMV) {
-        const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
-        const size_t rowb = (size_t)g.K * 2;
-        total = (uint32_t)(g.nseg * nr * rowb);
-        if (g.nseg == 2) {  // gate rows, then up rows at a fixed offset
-          if (lane < 2) {
-            int run;
-            src = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, lane, n0, g.K, &run));
-            dst += (size_t)lane * g.rps * rowb;
-            bytes = (uint32_t)(nr * rowb);
-          }
-        } else if (lane < 3) {  // the stage's rows, cut where they cross physical matrices
-          int n = n0, left = nr, piece = 0;
-          while (left > 0) {
-            int run;
-            const uint16_t* w = gemv_row(p, t.op, t.layer, 0, n, g.K, &run);
-            const int take = min(left, run);
-            if (piece == lane) {
-              src = reinterpret_cast<const uint8_t*>(w);
-              dst += (size_t)(n - n0) * rowb;
-              bytes = (uint32_t)(take * rowb);
-            }
-            n += take;
-            left -= take;
-            ++piece;
-          }
-        }
-      } else {
-        const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
-        const size_t rowb = (size_t)p.D * 2;
-        total = (uint32_t)(2 * n * rowb);
-        if (lane < 2) {
-          const LayerPtrs& L = p.layers[t.layer];
-          const uint16_t* base = lane == 0 ? L.k_cache : L.v_cache;
-          src = reinterpret_cast<const uint8_t*>(base) + ((size_t)t.r0 * p.cap + tt) * rowb;
-          dst += lane * (size_t)p.pps * rowb;
-          bytes = (uint32_t)(n * rowb);
-        }
-      }
+      uint32_t off, bytes, total;
+      const uint8_t* src = stage_piece(p, t, g, t0, t1, i, lane, &off, &bytes, &total);
       if (lane == 0) {
         *reinterpret_cast<volatile uint32_t*>(tags + slot) = gs;
         mbar_arrive_expect_tx(&full[slot], total);
       }
       __syncwarp();
-      if (bytes) bulk_g2s(dst, src, bytes, &full[slot], pol);
+      if (bytes) bulk_g2s(ring + (size_t)slot * SB + off, src, bytes, &full[slot], pol);
     }
   }
   if (!ok && lane == 0) {
@@ -279,12 +376,13 @@ __device__ __forceinline__ int input_key(const Task& t) {
     case OP_DOWN: cls = 3; break;
     default: cls = 4; break;
   }
-  return (int)t.layer * 8 + cls;
+  return (((int)t.layer * 8 + cls) << 4) | (t.op == OP_LM ? 0 : (t.aux & 0xf));
 }
 
 // Stage the GEMV input into the two planes; returns the RMSNorm scale (1 when none).
-__device__ float load_input(const Params& p, const Task& t, float* ub, float* red, int ctid) {
-  const int K = gemv_K(p, t.op);
+__device__ float load_input(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
+                            float* red, int ctid) {
+  const int K = gg.Kp;  // this K-part's slice of the input vector
   float* xlo = ub;
   float* xhi = ub + K / 2;
   const float* src = nullptr;
@@ -302,6 +400,7 @@ __device__ float load_input(const Params& p, const Task& t, float* ub, float* re
     case OP_DOWN: src = p.u; break;
     default: src = p.x; gain = p.final_norm; break;
   }
+  if (src) src += gg.k0;        // normalised inputs are single-part (k0 = 0)
   float ss = 0.f;
   const int K8 = K >> 3;
   for (int j = ctid; j < K8; j += kConsumerThreads) {
@@ -404,6 +503,7 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     }
   }
   consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
 
   if (last && warp < G) {  // score of the new position for head `warp`
     float a = 0.f;
@@ -427,20 +527,24 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   const uint32_t NS = (uint32_t)p.ring_stages;
   int t0, t1;
   attn_range(p, t, t0, t1);
-  for (int i = 0; i < ns; ++i) {
+  // a stage of pps positions is taken by wps warps (8 positions each); the 8 warps form
+  // 8 / wps groups that consume alternate stages
+  const int wps = p.pps / kPosPerWarp, ngrp = kConsumerWarps / wps;
+  const int grp = warp / wps, wpos = (warp % wps) * kPosPerWarp;
+  for (int i = grp; i < ns; i += ngrp) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
     if (!stage_wait(p, full, tags, sidx)) {
       abort_out = true;
       break;
     }
     const int n = min(p.pps, t1 - (t0 + i * p.pps));
-    const int nw = min(kPosPerWarp, n - warp * kPosPerWarp);
+    const int nw = min(kPosPerWarp, n - wpos);
     if (nw > 0) {
-      const uint8_t* kb = ring + (size_t)slot * p.stage_bytes + (size_t)warp * kPosPerWarp * D * 2;
+      const uint8_t* kb = ring + (size_t)slot * p.stage_bytes + (size_t)wpos * D * 2;
       attn_warp_positions<G, DPL>(kb, kb + (size_t)p.pps * D * 2, nw, q, m, l, o, lane);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
+    if (lane == 0) mbar_arrive_n(&empty[slot], (uint32_t)(kConsumerWarps / wps));
   }
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -452,6 +556,7 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     for (int j = 0; j < DPL; ++j) ow[(warp * G + h) * D + lane * DPL + j] = o[h][j];
   }
   consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
 
   // merge the warps (and the new position) into this split's partial
   const size_t pstride = (size_t)D + 2;
@@ -491,6 +596,7 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   if (ctid == 0) {
     const uint32_t old = atom_acq_rel_gpu_add(p.tickets + g, 1u);
     *flag = ((old + 1u) % (uint32_t)S) == 0u;
+    if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
   }
   consumer_sync(kConsumerThreads);
   if (*flag) {  // last split of this kv head to finish: combine all splits
@@ -552,16 +658,32 @@ __device__ __forceinline__ void run_attn(const Params& p, const Task& t, uint32_
 }
 
 // ---- GEMV epilogue ---------------------------------------------------------------------------------
-__device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, int n, float v, float rn,
-                                          Best& best) {
+// Residual rows of an O-proj / down task, staged before its stages: part 0 reads the
+// residual stream (x, or for layer 0 the embedding row / layer input; h1 for down), later
+// K-parts read the partial sum the previous part left in the output.
+__device__ __forceinline__ void prefetch_resid(const Params& p, const Task& t, const GemvGeom& g,
+                                               float* resid, int ctid) {
+  for (int r = ctid; r < t.r1 - t.r0; r += kConsumerThreads) {
+    const int n = t.r0 + r;
+    float v;
+    if (t.op == OP_O) v = g.part == 0 ? resid_in(p, t.layer, n) : __ldcg(p.h1 + n);
+    else v = g.part == 0 ? __ldcg(p.h1 + n) : __ldcg(p.x + n);
+    resid[r] = v;
+  }
+}
+
+__device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const GemvGeom& g, int n,
+                                          float v, float rn, const float* resid, Best& best) {
   switch (t.op) {
     case OP_QKV: p.qkv[n] = v * rn; break;
-    case OP_O: p.h1[n] = resid_in(p, t.layer, n) + v; break;
+    case OP_O: p.h1[n] = resid[n - t.r0] + v; break;
     case OP_DOWN: {
-      const float y = __ldcg(p.h1 + n) + v;
+      const float y = resid[n - t.r0] + v;
       p.x[n] = y;
-      if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
-      if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
+      if (g.part == g.np - 1) {
+        if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
+        if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
+      }
     } break;
     default: {
       const float y = v * rn;
@@ -587,7 +709,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     const Task t = my[ti];
     const int ns = task_nstages(p, t);
     if (ctid == 0) {
-      long long* tr = p.trace ? p.trace + (size_t)t.id * 4 : nullptr;
+      long long* tr = p.trace ? p.trace + (size_t)t.id * kTraceCols : nullptr;
       if (tr) tr[0] = (long long)globaltimer_ns();
       const bool ok = !ab && wait_dep(p, t);
       if (ok) fence_acq_rel_gpu();
@@ -604,18 +726,22 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       cur_key = -1;  // the attention scratch aliases the input-vector planes
       run_attn(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
     } else {
+      const GemvGeom g = gemv_geom(p, t);
       const int key = input_key(t);
+      float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
+      const bool has_resid = t.op == OP_O || t.op == OP_DOWN;
+      if (has_resid) prefetch_resid(p, t, g, resid, ctid);
       if (key != cur_key) {
-        const float rn = load_input(p, t, ub, red, ctid);
+        const float rn = load_input(p, t, g, ub, red, ctid);
         if (ctid == 0) *rn_s = rn;
-        consumer_sync(kConsumerThreads);
         cur_key = key;
       }
+      consumer_sync(kConsumerThreads);
+      if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
       const float rn = *rn_s;
-      const GemvGeom g = gemv_geom(p, t);
-      const int K8 = g.K >> 3;
+      const int K8 = g.Kp >> 3;
       const float4* xl = reinterpret_cast<const float4*>(ub);
-      const float4* xh = reinterpret_cast<const float4*>(ub + g.K / 2);
+      const float4* xh = reinterpret_cast<const float4*>(ub + g.Kp / 2);
       Best best{-INFINITY, 0x7fffffff};
       // stage gs + i belongs to warp (gs + i) % 8; each warp takes its stages in order
       const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
@@ -631,16 +757,15 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
           const uint4* up = sp + (size_t)g.rps * K8;
           for (int r = 0; r < nr; r += 2) {
             const int np = min(2, nr - r);
-            float o[4];
-            const uint4* rows[4] = {sp + (size_t)r * K8, sp + (size_t)(r + np - 1) * K8,
-                                    up + (size_t)r * K8, up + (size_t)(r + np - 1) * K8};
+            float o0, o1, o2, o3;
+            const uint4* g0 = sp + (size_t)r * K8;
+            const uint4* u0 = up + (size_t)r * K8;
             if (np == 2) {
-              gemv_rows<4, 1>(rows, K8, xl, xh, lane, o);
+              gemv_rows<4, 1>(g0, g0 + K8, u0, u0 + K8, K8, xl, xh, lane, o0, o1, o2, o3);
             } else {
-              const uint4* rows2[4] = {rows[0], rows[2], rows[2], rows[2]};
-              gemv_rows<2, 2>(rows2, K8, xl, xh, lane, o);
+              gemv_rows<2, 2>(g0, u0, u0, u0, K8, xl, xh, lane, o0, o1, o2, o3);
             }
-            const float v = reduce4(o[0], o[1], o[2], o[3], lane);
+            const float v = reduce4(o0, o1, o2, o3, lane);
             // np == 2: lanes 0 / 8 hold gate r / r+1, lanes 16 / 24 up r / r+1
             // np == 1: lane 0 holds gate r, lane 8 up r
             const float upv = __shfl_xor_sync(0xffffffffu, v, np == 2 ? 16 : 8);
@@ -653,14 +778,13 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         } else {
           for (int r = 0; r < nr; r += 4) {
             const int nv = min(4, nr - r);
-            const uint4* rows[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) rows[q] = sp + (size_t)(r + min(q, nv - 1)) * K8;
-            float o[4];
-            gemv_rows_n(nv, rows, K8, xl, xh, lane, o);
-            const float v = reduce4(o[0], o[1], o[2], o[3], lane);
+            const uint4* r0 = sp + (size_t)r * K8;
+            float o0, o1, o2, o3;
+            gemv_rows_n(nv, r0, r0 + (size_t)min(1, nv - 1) * K8, r0 + (size_t)min(2, nv - 1) * K8,
+                        r0 + (size_t)min(3, nv - 1) * K8, K8, xl, xh, lane, o0, o1, o2, o3);
+            const float v = reduce4(o0, o1, o2, o3, lane);
             const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-            if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, n0 + r + idx, v, rn, best);
+            if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, g, n0 + r + idx, v, rn, resid, best);
           }
         }
         __syncwarp();
@@ -681,6 +805,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       }
       __threadfence();
       consumer_sync(kConsumerThreads);
+      if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
       if (t.op == OP_LM && ctid == 0) {
         Best bb{-INFINITY, 0x7fffffff};
         for (int w = 0; w < kConsumerWarps; ++w) best_update(bb, red[w], reinterpret_cast<int*>(red)[16 + w]);
@@ -694,7 +819,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       }
       if (ctid == 0 && t.out >= 0) red_release_gpu_add(p.counters + t.out, 1u);
     }
-    if (ctid == 0 && p.trace) p.trace[(size_t)t.id * 4 + 2] = (long long)globaltimer_ns();
+    if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 2] = (long long)globaltimer_ns();
     gs += (uint32_t)ns;
   }
 }

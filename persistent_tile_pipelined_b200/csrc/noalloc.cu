@@ -220,6 +220,7 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   p.eps = cfg->norm_eps;
   p.flags = cfg->debug_flags;
   p.timeout_ns = 1000LL * (cfg->dep_timeout_us ? cfg->dep_timeout_us : 1000000);
+  p.pf_window = cfg->l2_prefetch_kb > 0 ? 1024LL * cfg->l2_prefetch_kb : 1024LL * kDefaultPrefetchKB;
   p.token = token;
   p.pos = pos;
   p.epoch = 1;  // counters were just cleared

@@ -94,18 +94,25 @@ struct Builder {
     return t;
   }
 
-  // Returns the number of tasks created.
-  int gemv(uint8_t op, int layer, int N, int64_t row_bytes, int dep, uint32_t dep_count,
-           int out) {
-    auto ranges = assign_rows(N, row_bytes, cum);
+  // Cut N rows (K inputs each, nseg matrices) into per-SM ranges; a range longer than
+  // `cap` rows becomes several sub-ranges, and each sub-range one task per K-part (only
+  // the last part bumps `out`).  Returns the number of tasks that bump `out`.
+  int gemv(uint8_t op, int layer, int N, int K, int nseg, int dep, uint32_t dep_count, int out,
+           int cap) {
+    const int np = op == OP_LM ? 1 : gemv_nparts(K);
+    auto ranges = assign_rows(N, (int64_t)nseg * K * 2, cum);
     int n = 0;
     for (int s = 0; s < nsm; ++s) {
-      if (ranges[s].second <= ranges[s].first) continue;
-      Task t = make(T_GEMV, op, layer, dep, dep_count, out);
-      t.r0 = ranges[s].first;
-      t.r1 = ranges[s].second;
-      q[s].push_back(t);
-      ++n;
+      for (int r = ranges[s].first; r < ranges[s].second; r += cap) {
+        for (int part = 0; part < np; ++part) {
+          Task t = make(T_GEMV, op, layer, dep, dep_count, part == np - 1 ? out : -1);
+          t.r0 = r;
+          t.r1 = std::min(ranges[s].second, r + cap);
+          t.aux = part | (np << 8);
+          q[s].push_back(t);
+          if (part == np - 1) ++n;
+        }
+      }
     }
     return n;
   }
@@ -180,21 +187,34 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   s.has_lm = c.has_embed_lm_head;
   const int G = s.Hq / s.Hkv;
 
-  // A ring stage holds whole weight rows (gate/up: a row of each matrix), or the K and V
-  // rows of up to 64 cached positions.
-  const int need = std::max({2 * s.d * 2, s.F * 2, s.Hq * s.D * 2, 4 * s.D});
+  // Inputs longer than kMaxKPart are staged in K-parts; ops that normalise their input
+  // (QKV, gate/up, LM head) need the whole vector at once.
+  if (s.d > kMaxKPart)
+    return fail(TRE_ERR_UNSUPPORTED, "hidden above 16384 (normalised inputs are staged whole)");
+  const int Ks[OP_COUNT] = {s.d, s.Hq * s.D, s.d, s.F, s.d};
+  const int segs[OP_COUNT] = {1, 1, 2, 1, 1};
+  int xs = 8, need = 4 * s.D * 8;  // a stage holds at least 8 KV positions
+  for (int op = 0; op < OP_COUNT; ++op) {
+    const int kp = gemv_part_len(Ks[op], op == OP_LM ? 1 : gemv_nparts(Ks[op]));
+    xs = std::max(xs, kp);
+    need = std::max(need, segs[op] * kp * 2);
+  }
+  // A ring stage holds whole rows of one K-part (gate/up: a row of each matrix), or the K
+  // and V rows of 8-64 cached positions.
   int sb = c.stage_bytes ? c.stage_bytes : kDefaultStageBytes;
   if (!c.stage_bytes)
     while (sb < need && sb < kMaxStageBytes) sb += 1024;
   if (sb < need)
-    return fail(TRE_ERR_UNSUPPORTED, "a weight row (or gate/up row pair) is wider than a ring stage");
+    return fail(TRE_ERR_UNSUPPORTED, "a weight row part (or gate/up row pair) is wider than a ring stage");
   s.stage_bytes = sb;
-  s.pos_per_stage = std::min(kMaxPosPerStage, sb / (4 * s.D));
+  int pps = 8;  // a power of two, so that every warp of a stage group takes 8 positions
+  while (pps * 2 <= kMaxPosPerStage && pps * 2 * 4 * s.D <= sb) pps *= 2;
+  s.pos_per_stage = pps;
 
-  s.xs_floats = std::max({s.d, s.Hq * s.D, s.F});
-  s.xs_floats = (s.xs_floats + 7) / 8 * 8;
+  s.xs_floats = (xs + 7) / 8 * 8;
+  s.resid_floats = kMaxResidRows;
   s.attn_floats = G * s.D + 2 * s.D + kConsumerWarps * (2 * G + G * s.D) + 16;
-  const int ubuf_floats = (std::max(s.xs_floats, s.attn_floats) + 7) / 8 * 8;
+  const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats, s.attn_floats) + 7) / 8 * 8;
   s.ub_floats = ubuf_floats;
   const int misc_bytes = 1024;
   const int fixed = ubuf_floats * 4 + misc_bytes;
@@ -219,19 +239,20 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   s.kv_splits = S;
 
   Builder b(nsm);
-  const int64_t d2 = (int64_t)s.d * 2;
   int prev_down = -1;
   uint32_t prev_down_count = 0;
   for (int l = 0; l < s.L; ++l) {
     const int cq = counter_of(l, C_QKV), ca = counter_of(l, C_ATTN), co = counter_of(l, C_O),
               cg = counter_of(l, C_GU), cd = counter_of(l, C_DOWN);
     // Q, K and V as one op over the stacked matrix [Wq; Wk; Wv]
-    const int nqkv = b.gemv(OP_QKV, l, (s.Hq + 2 * s.Hkv) * s.D, d2, prev_down, prev_down_count, cq);
+    const int big = 1 << 30;
+    const int nqkv = b.gemv(OP_QKV, l, (s.Hq + 2 * s.Hkv) * s.D, s.d, 1, prev_down,
+                            prev_down_count, cq, big);
     const int64_t kv_task_bytes = (int64_t)(s.cap - s.M) / S * s.D * 2 * 2;
     b.attention(l, s.Hkv, S, kv_task_bytes, cq, (uint32_t)nqkv, ca);
-    int no = b.gemv(OP_O, l, s.d, (int64_t)s.Hq * s.D * 2, ca, (uint32_t)s.Hkv, co);
-    int ng = b.gemv(OP_GU, l, s.F, 2 * d2, co, (uint32_t)no, cg);
-    int nd = b.gemv(OP_DOWN, l, s.d, (int64_t)s.F * 2, cg, (uint32_t)ng, cd);
+    int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)s.Hkv, co, s.resid_floats);
+    int ng = b.gemv(OP_GU, l, s.F, s.d, 2, co, (uint32_t)no, cg, big);
+    int nd = b.gemv(OP_DOWN, l, s.d, s.F, 1, cg, (uint32_t)ng, cd, s.resid_floats);
     prev_down = cd;
     prev_down_count = (uint32_t)nd;
   }
@@ -239,7 +260,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   s.n_counters = c_lm + 2;
   if (s.has_lm) {
     int first = b.next_id;
-    int nlm = b.gemv(OP_LM, s.L - 1, s.V, d2, prev_down, prev_down_count, c_lm);
+    int nlm = b.gemv(OP_LM, s.L - 1, s.V, s.d, 1, prev_down, prev_down_count, c_lm, 1 << 30);
     s.n_lm_tasks = nlm;
     for (auto& qq : b.q)
       for (auto& t : qq)

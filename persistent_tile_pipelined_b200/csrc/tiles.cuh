@@ -64,10 +64,11 @@ __device__ __forceinline__ float reduce32(float (&v)[32], int lane) {
 // xh[j] = x[8j+4:8j+8].  NACC independent accumulators per row keep enough FMA chains in
 // flight when a stage holds only one or two (long) rows.
 template <int NR, int NACC>
-__device__ __forceinline__ void gemv_rows(const uint4* const (&rows)[4], int K8,
-                                          const float4* __restrict__ xl,
-                                          const float4* __restrict__ xh, int lane,
-                                          float (&out)[4]) {
+__device__ __forceinline__ void gemv_rows(const uint4* r0, const uint4* r1, const uint4* r2,
+                                          const uint4* r3, int K8, const float4* __restrict__ xl,
+                                          const float4* __restrict__ xh, int lane, float& o0,
+                                          float& o1, float& o2, float& o3) {
+  const uint4* rp[4] = {r0, r1, r2, r3};
   float acc[NR][NACC];
 #pragma unroll
   for (int r = 0; r < NR; ++r)
@@ -80,14 +81,15 @@ __device__ __forceinline__ void gemv_rows(const uint4* const (&rows)[4], int K8,
     for (int a = 0; a < NACC; ++a) {
       const float4 x0 = xl[j + 32 * a], x1 = xh[j + 32 * a];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) acc[r][a] = dot8(rows[r][j + 32 * a], x0, x1, acc[r][a]);
+      for (int r = 0; r < NR; ++r) acc[r][a] = dot8(rp[r][j + 32 * a], x0, x1, acc[r][a]);
     }
   }
   for (; j < K8; j += 32) {
     const float4 x0 = xl[j], x1 = xh[j];
 #pragma unroll
-    for (int r = 0; r < NR; ++r) acc[r][0] = dot8(rows[r][j], x0, x1, acc[r][0]);
+    for (int r = 0; r < NR; ++r) acc[r][0] = dot8(rp[r][j], x0, x1, acc[r][0]);
   }
+  float out[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     float v = 0.f;
@@ -97,16 +99,21 @@ __device__ __forceinline__ void gemv_rows(const uint4* const (&rows)[4], int K8,
     }
     out[r] = v;
   }
+  o0 = out[0];
+  o1 = out[1];
+  o2 = out[2];
+  o3 = out[3];
 }
 
-__device__ __forceinline__ void gemv_rows_n(int nr, const uint4* const (&rows)[4], int K8,
+__device__ __forceinline__ void gemv_rows_n(int nr, const uint4* r0, const uint4* r1,
+                                            const uint4* r2, const uint4* r3, int K8,
                                             const float4* xl, const float4* xh, int lane,
-                                            float (&out)[4]) {
+                                            float& o0, float& o1, float& o2, float& o3) {
   switch (nr) {
-    case 4: gemv_rows<4, 1>(rows, K8, xl, xh, lane, out); break;
-    case 3: gemv_rows<3, 1>(rows, K8, xl, xh, lane, out); break;
-    case 2: gemv_rows<2, 2>(rows, K8, xl, xh, lane, out); break;
-    default: gemv_rows<1, 4>(rows, K8, xl, xh, lane, out); break;
+    case 4: gemv_rows<4, 1>(r0, r1, r2, r3, K8, xl, xh, lane, o0, o1, o2, o3); break;
+    case 3: gemv_rows<3, 1>(r0, r1, r2, r3, K8, xl, xh, lane, o0, o1, o2, o3); break;
+    case 2: gemv_rows<2, 2>(r0, r1, r2, r3, K8, xl, xh, lane, o0, o1, o2, o3); break;
+    default: gemv_rows<1, 4>(r0, r1, r2, r3, K8, xl, xh, lane, o0, o1, o2, o3); break;
   }
 }
 

@@ -233,7 +233,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   const bool dbg_hidden = cfg->debug_flags & TRE_DEBUG_HIDDEN;
   const bool dbg_trace = cfg->debug_flags & TRE_DEBUG_TRACE;
   size_t o_hidden = dbg_hidden ? cv.take<float>((size_t)s.L * s.d) : 0;
-  size_t o_trace = dbg_trace ? cv.take<long long>((size_t)tasks.size() * 4) : 0;
+  size_t o_trace = dbg_trace ? cv.take<long long>((size_t)tasks.size() * kTraceCols) : 0;
   e->block_bytes = cv.off;
   cudaError_t ce = cudaMalloc(&e->block, e->block_bytes);
   if (ce != cudaSuccess) {
@@ -308,6 +308,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.eps = cfg->norm_eps;
   p.flags = cfg->debug_flags;
   p.timeout_ns = 1000LL * (cfg->dep_timeout_us ? cfg->dep_timeout_us : 1000000);
+  p.pf_window = cfg->l2_prefetch_kb > 0 ? 1024LL * cfg->l2_prefetch_kb : 1024LL * kDefaultPrefetchKB;
   *out = e;
   return TRE_OK;
 }
@@ -449,7 +450,7 @@ TRE_EXPORT tre_status tre_debug_trace(tre_engine* e, int64_t* trace_host, int32_
   }
   CK(cudaSetDevice(e->device));
   CK(cudaDeviceSynchronize());
-  CK(cudaMemcpy(trace_host, e->base.trace, (size_t)e->n_tasks * 4 * sizeof(long long),
+  CK(cudaMemcpy(trace_host, e->base.trace, (size_t)e->n_tasks * kTraceCols * sizeof(long long),
                 cudaMemcpyDeviceToHost));
   return TRE_OK;
 }

@@ -14,7 +14,11 @@ constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
 constexpr int kMaxGroup = 8;                           // q heads per kv head (GQA)
 constexpr int kPosPerWarp = 8;                         // KV positions per warp per stage
 constexpr int kMaxPosPerStage = kConsumerWarps * kPosPerWarp;  // 64
-constexpr int kDefaultStageBytes = 32768;
+constexpr int kDefaultStageBytes = 32768;  // a bulk-copy stage costs ~0.4 us per SM: keep them large
+constexpr int kMaxKPart = 16384;         // longest input slice one GEMV task stages (floats)
+constexpr int kMaxResidRows = 512;       // rows per task of ops that add a residual
+constexpr int kTraceCols = 8;          // int64 per task in the debug trace
+constexpr int kDefaultPrefetchKB = 0;    // next-task L2 prefetch: opt-in (measured 4% slower)
 constexpr int kMaxStageBytes = 65536;
 constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per block
 
@@ -27,6 +31,14 @@ constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per 
 // ---- GEMV stage geometry ----------------------------------------------------------------
 // A GEMV stage holds `rows per stage` whole contiguous rows of the op's matrix (gate/up:
 // the same rows of both matrices); one consumer warp computes the whole stage.
+// Rows longer than kMaxKPart are cut into K-parts: part j of a task covers input columns
+// [j * len, min(K, (j + 1) * len)); the parts of one row range are consecutive tasks on
+// one SM, the first adds the residual and later parts accumulate into the output.
+TRE_HD inline int gemv_nparts(int K) { return (K + kMaxKPart - 1) / kMaxKPart; }
+TRE_HD inline int gemv_part_len(int K, int nparts) {
+  const int l = (K + nparts - 1) / nparts;
+  return (l + 7) / 8 * 8;
+}
 TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes) {
   const int r = stage_bytes / (nseg * K * 2);
   return r < 1 ? 1 : r;
@@ -57,7 +69,8 @@ struct Task {          // 32 bytes, 16-byte aligned array
   uint32_t dep_count;  // increments of `dep` per step
   int32_t out;         // counter to bump when done, -1 = none
   int32_t r0, r1;      // GEMV: output rows [r0, r1).  ATTN: kv head, split index
-  int32_t aux;         // ATTN: number of splits.  LM: number of LM tasks
+  int32_t aux;         // ATTN: number of splits.  LM: number of LM tasks.
+                       // other GEMV: K-part index | (number of K-parts << 8)
   int32_t id;          // global task index (trace rows, error detail)
 };
 static_assert(sizeof(Task) == 32, "task descriptor is 32 bytes");
@@ -74,7 +87,8 @@ struct PlanShape {
   int nsm;
   int stage_bytes, ring_stages;
   int kv_splits, pos_per_stage;
-  int xs_floats;       // input-vector buffer (floats)
+  int xs_floats;       // input-vector buffer (floats): the longest K-part
+  int resid_floats;    // residual rows staged per task (floats)
   int attn_floats;     // attention scratch (floats), aliases the input-vector buffer
   int ub_floats;       // the shared union buffer: input planes, or attention scratch
   int smem_bytes;
@@ -118,6 +132,7 @@ struct Params {
   uint32_t epoch;
   int flags;
   long long timeout_ns;
+  long long pf_window;             // L2 prefetch bytes allowed beyond the ring (0 = off)
 };
 
 }  // namespace tre

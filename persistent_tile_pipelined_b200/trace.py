@@ -30,7 +30,7 @@ def op_name(tt: dict, i: int) -> str:
 
 
 def summarize(trace: np.ndarray, tasks: np.ndarray) -> dict:
-    """trace: [n_tasks][4] int64 (start, ready, end, sm) indexed by task id."""
+    """trace: [n_tasks][8] int64 (start, ready, end, sm, phase marks) by task id."""
     tt = task_table(tasks)
     t0 = trace[:, 0].min()
     start, ready, end = trace[:, 0] - t0, trace[:, 1] - t0, trace[:, 2] - t0
@@ -55,7 +55,19 @@ def summarize(trace: np.ndarray, tasks: np.ndarray) -> dict:
     for i in range(len(trace)):
         busy[int(trace[i, 3])] += end[i] - ready[i]
         waitt[int(trace[i, 3])] += ready[i] - start[i]
+    phases = defaultdict(lambda: [0.0, 0.0, 0.0, 0])
+    if trace.shape[1] >= 7:
+        for i in range(len(trace)):
+            r, e, a, b, c = (int(trace[i, k]) for k in (1, 2, 4, 5, 6))
+            d = phases[op_name(tt, i)]
+            if a and b:
+                d[0] += a - r          # input staged / q ready
+                d[1] += b - a          # stages consumed
+                d[2] += e - (c if c else b)   # tail: epilogue, ticket, combine, publish
+                d[3] += 1
     return {
+        "phases_us": {k: {"prep": v[0] / v[3] / 1e3, "stages": v[1] / v[3] / 1e3,
+                          "tail": v[2] / v[3] / 1e3} for k, v in phases.items() if v[3]},
         "step_us": step_ns / 1e3,
         "per_op": {k: {"tasks": v["tasks"], "mean_wait_us": v["wait_ns"] / v["tasks"] / 1e3,
                        "mean_busy_us": v["busy_ns"] / v["tasks"] / 1e3}

@@ -28,6 +28,7 @@ TRE_ERR_STATE = -8
 TRE_LAYER_GQA, TRE_LAYER_MLA, TRE_LAYER_MOE = 0, 1, 2
 TRE_DEBUG_HIDDEN, TRE_DEBUG_TRACE, TRE_DEBUG_FAULT_INJECT, TRE_DEBUG_NO_OVERLAP = 1, 2, 4, 8
 TRE_W_SLOTS = 16
+TRACE_COLS = 8
 GQA_SLOTS = {"attn_norm": 0, "wq": 1, "wk": 2, "wv": 3, "wo": 4, "ffn_norm": 5, "wgate": 6,
              "wup": 7, "wdown": 8}
 
@@ -45,7 +46,7 @@ class tre_config(ctypes.Structure):
         ("rope_theta", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
         (n, ctypes.c_int32) for n in (
             "has_embed_lm_head", "debug_flags", "dep_timeout_us", "num_sms", "kv_splits",
-            "stage_bytes", "ring_stages")] + [("reserved", ctypes.c_int32 * 8)]
+            "stage_bytes", "ring_stages", "l2_prefetch_kb")] + [("reserved", ctypes.c_int32 * 7)]
 
 
 class tre_weights(ctypes.Structure):
@@ -323,7 +324,7 @@ class Engine:
     def trace(self) -> np.ndarray:
         n = ctypes.c_int32()
         check(lib.tre_debug_trace(self.h, None, ctypes.byref(n)), "tre_debug_trace")
-        buf = np.zeros((n.value, 4), dtype=np.int64)
+        buf = np.zeros((n.value, TRACE_COLS), dtype=np.int64)
         check(lib.tre_debug_trace(self.h, buf.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)),
               "tre_debug_trace")
         return buf

@@ -90,16 +90,25 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
     # every GEMV op's output rows are partitioned exactly once per layer
     rows_of = {OP_QKV: (wl.n_q_heads + 2 * wl.n_kv_heads) * wl.head_dim, OP_O: wl.hidden,
                OP_GU: wl.ffn, OP_DOWN: wl.hidden, OP_LM: wl.vocab}
+    part = np.where(T["op"] == OP_LM, 0, T["aux"] & 0xFF)
+    nparts = np.where(T["op"] == OP_LM, 1, T["aux"] >> 8)
+    gemv = T["type"] == T_GEMV
+    # only the last K-part of a row range publishes
+    assert ((T["out"][gemv] >= 0) == (part[gemv] == nparts[gemv] - 1)).all()
     for l in range(wl.n_layers):
         for op, N in rows_of.items():
             if op == OP_LM and l != wl.n_layers - 1:
                 continue
-            sel = (T["type"] == T_GEMV) & (T["op"] == op) & (T["layer"] == l)
-            cover = np.zeros(N, dtype=np.int64)
-            for r0, r1 in zip(T["r0"][sel], T["r1"][sel]):
-                assert 0 <= r0 < r1 <= N
-                cover[r0:r1] += 1
-            assert (cover == 1).all(), (l, op)
+            sel_op = gemv & (T["op"] == op) & (T["layer"] == l)
+            np_op = int(nparts[sel_op][0])
+            assert (nparts[sel_op] == np_op).all()
+            for pt in range(np_op):
+                sel = sel_op & (part == pt)
+                cover = np.zeros(N, dtype=np.int64)
+                for r0, r1 in zip(T["r0"][sel], T["r1"][sel]):
+                    assert 0 <= r0 < r1 <= N
+                    cover[r0:r1] += 1
+                assert (cover == 1).all(), (l, op, pt)
         sel = (T["type"] == T_ATTN) & (T["layer"] == l)
         pairs = Counter(zip(T["r0"][sel].tolist(), T["r1"][sel].tolist()))
         S = info.kv_splits
