@@ -183,6 +183,121 @@ def build_engine(wl, device: int, debug_flags: int = 0):
     return tre.Engine(cfg, model, device), model
 
 
+def build_layers_engine(wl, device: int, debug_flags: int = 0):
+    """A layers-only stack (MoE or MLA layers, no embedding / LM head): non-expert tensors
+    and caches from the workload generator, routed experts generated one at a time and
+    stacked on the device."""
+    import torch
+
+    from persistent_tile_pipelined_b200 import tre
+    from persistent_tile_pipelined_b200.synth import workloads as W
+
+    dev = f"cuda:{device}"
+    if wl.kind == "moe":
+        model = W.gen_moe_model(wl)
+        dmodel = tre.upload_moe_model(wl, model, dev)
+    else:
+        raise SystemExit(f"layers-only workload kind {wl.kind!r} is not built")
+    torch.cuda.synchronize(device)
+    cfg = tre.config_from_workload(wl, debug_flags=debug_flags)
+    return tre.Engine(cfg, dmodel, device), dmodel
+
+
+def run_layers(args, rank, world, local_rank):
+    """Timed layers-only steps: each step takes a different seeded hidden vector (so MoE
+    routing changes from step to step, as in decode) at the next KV position."""
+    import torch
+    import torch.distributed as dist
+
+    from persistent_tile_pipelined_b200.synth import TID_X_IN, normal_f32
+    from persistent_tile_pipelined_b200.synth import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    K, Wm = args.steps, args.warmup
+    wl = W.WORKLOADS[args.workload].replace(decode_steps=K + Wm)
+    wl = wl.replace(seed=wl.seed + rank)
+    eng, dmodel = build_layers_engine(wl, local_rank, args.flags)
+    stream = torch.cuda.current_stream(local_rank)
+    s_ptr = stream.cuda_stream
+    xs_host = [normal_f32(wl.seed + i, TID_X_IN, (wl.hidden,)) for i in range(K + Wm)]
+    xs = torch.from_numpy(np.stack(xs_host)).to(f"cuda:{local_rank}")
+    out = torch.empty(wl.hidden, dtype=torch.float32, device=f"cuda:{local_rank}")
+    positions = [wl.prefill + i for i in range(K + Wm)]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(local_rank)
+
+    for i in range(Wm):
+        eng.layers_step(xs[i], out, positions[i], stream=s_ptr)
+    torch.cuda.synchronize(local_rank)
+    assert eng.status() == (0, 0), eng.status()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.2)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    barrier()
+    tw0 = time.time()
+    ev[0].record(stream)
+    for i in range(K):
+        eng.layers_step(xs[Wm + i], out, positions[Wm + i], stream=s_ptr)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(local_rank)
+    tw1 = time.time()
+    barrier()
+    sampler.mark(tw0, tw1)
+    dev_s = ev[0].elapsed_time(ev[K]) / 1e3
+    launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    assert eng.status() == (0, 0)
+    # end to end: the hidden vector from pinned host memory in, the result back out
+    x_pin = torch.empty(wl.hidden, dtype=torch.float32).pin_memory()
+    o_pin = torch.empty(wl.hidden, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty(wl.hidden, dtype=torch.float32, device=f"cuda:{local_rank}")
+    barrier()
+    tw0 = time.time()
+    t0 = time.perf_counter()
+    for i in range(K):
+        x_pin.copy_(torch.from_numpy(xs_host[Wm + i]))
+        x_dev.copy_(x_pin, non_blocking=True)
+        eng.layers_step(x_dev, out, positions[Wm + i], stream=s_ptr)
+        o_pin.copy_(out, non_blocking=True)
+        torch.cuda.synchronize(local_rank)
+    e2e_s = time.perf_counter() - t0
+    tw1 = time.time()
+    barrier()
+    sampler.mark(tw0, tw1)
+    clocks = sampler.stop()
+    step_bytes = float(np.mean([eng.step_bytes(positions[Wm + i]) for i in range(K)]))
+    eng.close()
+    if args.trace and rank == 0:
+        # a fresh engine with the trace flag on the same device memory: three steps
+        from persistent_tile_pipelined_b200 import trace as trace_mod
+        from persistent_tile_pipelined_b200 import tre
+        cfg = tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_TRACE | args.flags)
+        teng = tre.Engine(cfg, dmodel, local_rank)
+        for i in range(3):
+            teng.layers_step(xs[i], out, positions[i], stream=s_ptr)
+        torch.cuda.synchronize(local_rank)
+        tr = teng.trace()
+        nsm = torch.cuda.get_device_properties(local_rank).multi_processor_count
+        tasks, begin = tre.tre_plan_tasks(cfg, num_sms=nsm)
+        teng.close()
+        summ = trace_mod.summarize(tr, tasks)
+        with open(args.trace, "w") as f:
+            json.dump({"workload": wl.name, "summary": summ, "trace": tr.tolist(),
+                       "tasks": tasks.tolist(), "sm_begin": begin.tolist()}, f)
+        print(json.dumps(summ), file=sys.stderr)
+    del dmodel
+    torch.cuda.empty_cache()
+    t = torch.tensor([dev_s, e2e_s, float(np.mean(launch_ms))], dtype=torch.float64,
+                     device=f"cuda:{local_rank}")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev_s, e2e_s, launch_ms_avg = t.tolist()
+    return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
+
+
 def cpu_baseline(wl, sample_layers: int, reps: int = 1):
     """The oracle (as it stands) on this machine's cores: one decode step of a
     `sample_layers`-layer slice of the workload (same layer shapes, same LM head, same KV
@@ -348,6 +463,9 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device(f"cuda:{local_rank}"))
+    from persistent_tile_pipelined_b200.synth import workloads as W
+    if W.WORKLOADS[args.workload].kind != "gqa":
+        return main_layers(args, rank, world, local_rank)
     wl, dev_s, e2e_s, launch_ms, step_bytes, clocks = run_engine(args, rank, world, local_rank)
     K = args.steps
     peak, peak_kind = peaks()
@@ -394,6 +512,47 @@ def main():
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_layers)
         except Exception as exc:  # report, do not hide
             line["cpu_baseline"] = {"error": repr(exc)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main_layers(args, rank, world, local_rank):
+    """Layers-only workloads (MoE, MLA): step time of the whole layer stack and the HBM
+    bandwidth it achieves over the bytes a token actually reads."""
+    import torch.distributed as dist
+    wl, dev_s, e2e_s, launch_ms, step_bytes, clocks = run_layers(args, rank, world, local_rank)
+    K = args.steps
+    peak, peak_kind = peaks()
+    achieved = step_bytes / (launch_ms / 1e3) / 1e9
+    cfg = {"workload": f"{wl.name} layers-only step, batch 1, KV {wl.prefill} positions",
+           "kind": wl.kind, "layers": wl.n_layers, "hidden": wl.hidden,
+           "heads": wl.n_q_heads, "batch": 1,
+           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+           "l2": f"not flushed: each step streams {step_bytes / 1e9:.2f} GB >> 126 MB L2"}
+    if wl.kind == "moe":
+        cfg.update(experts=wl.n_experts, top_k=wl.top_k, shared=wl.n_shared,
+                   expert_ffn=wl.expert_ffn, kv_heads=wl.n_kv_heads, head_dim=wl.head_dim)
+    line = {
+        "metric": "layer-stack step time and achieved HBM GB/s over the bytes a token reads",
+        "value": world * K / dev_s, "unit": "steps/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": dev_s / K * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
+        "config": cfg,
+        "hbm_gbs": step_bytes / (dev_s / K) / 1e9,
+        "hbm_frac_of_8tbs": step_bytes / (dev_s / K) / 1e9 / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "tre::engine_kernel",
+                     "algorithmic_bytes_per_launch": step_bytes},
+        "e2e": {"value": world * K / e2e_s, "unit": "steps/s",
+                "h2d_bytes_per_step": 4 * wl.hidden, "d2h_bytes_per_step": 4 * wl.hidden},
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

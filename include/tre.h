@@ -114,12 +114,19 @@ typedef struct {
  * tensor `slot` of layer l (NULL for slots the layer kind does not use).
  *   GQA : ATTN_NORM[d], WQ[Hq*D][d], WK[Hkv*D][d], WV[Hkv*D][d], WO[d][Hq*D],
  *         FFN_NORM[d], WGATE[F][d], WUP[F][d], WDOWN[d][F]
+ *   MOE : slots 0-5 as GQA, then (Fe = expert_ffn, Fs = n_shared * Fe, E = n_experts)
+ *         ROUTER[E][d], SHARED_GATE[Fs][d], SHARED_UP[Fs][d], SHARED_DOWN[d][Fs]
+ *         (NULL when n_shared == 0), and the routed experts stacked expert-major:
+ *         EXPERT_GATE[E][Fe][d], EXPERT_UP[E][Fe][d], EXPERT_DOWN[E][d][Fe]
+ *         (the layout of a fused-MoE weight: expert e's matrix starts at e * Fe * d).
  * KV caches (bf16, written at pos by every step, caller owned):
  *   GQA/MOE : k_cache[l], v_cache[l] = [Hkv][kv_capacity][D]
  */
 enum {
   TRE_W_ATTN_NORM = 0, TRE_W_Q = 1, TRE_W_K = 2, TRE_W_V = 3, TRE_W_O = 4,
   TRE_W_FFN_NORM = 5, TRE_W_GATE = 6, TRE_W_UP = 7, TRE_W_DOWN = 8,
+  TRE_W_ROUTER = 6, TRE_W_SHARED_GATE = 7, TRE_W_SHARED_UP = 8, TRE_W_SHARED_DOWN = 9,
+  TRE_W_EXPERT_GATE = 10, TRE_W_EXPERT_UP = 11, TRE_W_EXPERT_DOWN = 12,
   TRE_W_SLOTS = 16
 };
 
@@ -205,7 +212,26 @@ tre_status tre_decode_step_static(const tre_config* cfg, const tre_weights* w, i
                                   int32_t pos, tre_stream stream, float* logits_dev,
                                   int32_t* token_dev, int32_t* status_dev);
 
+/* One step of a layers-only stack (has_embed_lm_head == 0): the residual stream after
+ * the last layer for one token at `pos`, from the hidden vector entering layer 0.
+ *   x_in_dev    device fp32[hidden], read only (16-byte aligned)
+ *   x_out_dev   device fp32[hidden], written (16-byte aligned; may not alias x_in_dev)
+ *   pos         as for tre_decode_step: the caches hold [0, pos) on entry, [0, pos] after
+ * MoE layers route the token on the device (sigmoid scores, top_k by score with ties to
+ * the lower expert index, weights normalised over the selection; the pages name the
+ * fused op ExpertSelectUpGateSiLU — TileRT code audit, MoE paragraph — and print no
+ * formula): only the selected experts' weights are read.  Enqueues asynchronously and
+ * returns a previous step's device error without launching, like tre_decode_step. */
+tre_status tre_layers_step(tre_engine* e, const float* x_in_dev, float* x_out_dev, int32_t pos,
+                           tre_stream stream);
+
 /* ---- status / debug ----------------------------------------------------------- */
+
+/* MoE engines: copy the routing of the last step to host memory — idx_host int32
+ * [n_layers][top_k] (selected experts in descending score order) and w_host fp32
+ * [n_layers][top_k] (their normalised weights); either may be NULL.  Waits for the
+ * engine's last stream.  TRE_ERR_UNSUPPORTED for other kinds. */
+tre_status tre_debug_routing(tre_engine* e, int32_t* idx_host, float* w_host);
 
 /* Wait for the engine's last stream, then report the device status word: 0, or a
  * negative tre_status (TRE_ERR_DEP_TIMEOUT / TRE_ERR_BOUNDS).  *detail_out (may be

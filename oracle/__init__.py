@@ -215,18 +215,21 @@ class Oracle:
         self.lib.orc_gqa_attn_block(ctypes.byref(cfg), ctypes.byref(L), int(pos), _ptr(x), _ptr(h1))
         return h1
 
-    def moe_layer_step(self, wl, layer: dict, k_cache, v_cache, experts, pos: int, x):
+    def moe_layer_step(self, wl, layer: dict, k_cache, v_cache, experts, pos: int, x,
+                       want_scores: bool = False):
         """One MoE decoder layer: the GQA attention block, then
         x = h1 + sum_i w_i Expert_{idx_i}(hn) + Shared(hn), hn = RMSNorm(h1).
         `experts(e)` returns routed expert e's (W_gate, W_up, W_down).
-        Returns (x_out, idx, w)."""
+        Returns (x_out, idx, w), and the router's scores of all experts when want_scores."""
         h1 = self.gqa_attn_block(wl, layer, k_cache, v_cache, pos, x)
         hn = self.rmsnorm(h1, layer[5], wl.norm_eps)
-        idx, w, _ = self.router_topk(layer[6], hn, wl.top_k)
+        idx, w, scores = self.router_topk(layer[6], hn, wl.top_k)
         y = np.zeros(wl.hidden, dtype=self.real)
         for i, e in enumerate(idx):
             y += w[i] * self.swiglu_mlp(*experts(int(e)), hn)
         y += self.swiglu_mlp(layer[7], layer[8], layer[9], hn)
+        if want_scores:
+            return h1 + y, idx, w, scores
         return h1 + y, idx, w
 
     def mla_layer_step(self, wl, layer: dict, latent_cache, pos: int, x):

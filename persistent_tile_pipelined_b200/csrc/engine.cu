@@ -39,11 +39,11 @@ __device__ __noinline__ void record_error(const Params& p, int code, int detail)
 
 __device__ __forceinline__ bool aborted(const Params& p) { return *p.abort_flag != 0; }
 
-// Wait until counter `t.dep` reaches epoch * t.dep_count (wrap-safe).  Bounded.
-__device__ bool wait_dep(const Params& p, const Task& t) {
-  if (t.dep < 0) return true;
-  const uint32_t target = p.epoch * t.dep_count;
-  const uint32_t* c = p.counters + t.dep;
+// Wait until counter `idx` reaches epoch * count (wrap-safe).  Bounded; on expiry the
+// error names `detail` (a task index).
+__device__ bool wait_counter(const Params& p, int idx, uint32_t count, int detail) {
+  const uint32_t target = p.epoch * count;
+  const uint32_t* c = p.counters + idx;
   if ((int32_t)(ld_acquire_gpu(c) - target) >= 0) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -51,11 +51,17 @@ __device__ bool wait_dep(const Params& p, const Task& t) {
     if ((it & 31) == 0) {
       if (aborted(p)) return false;
       if ((long long)(globaltimer_ns() - t0) > p.timeout_ns) {
-        record_error(p, TRE_ERR_DEP_TIMEOUT, t.id);
+        record_error(p, TRE_ERR_DEP_TIMEOUT, detail);
         return false;
       }
     }
   }
+}
+
+// Wait until the task's dependency counter reaches epoch * t.dep_count.
+__device__ __forceinline__ bool wait_dep(const Params& p, const Task& t) {
+  if (t.dep < 0) return true;
+  return wait_counter(p, t.dep, t.dep_count, t.id);
 }
 
 // Bounded wait on an mbarrier phase; `slack` scales the time budget (ring waits get
@@ -102,30 +108,32 @@ __device__ bool stage_wait(const Params& p, uint64_t* full, const uint32_t* tags
 
 // ---- task geometry (shared by producer and consumers) ---------------------------------------
 // GEMV task: rows [r0, r1) of the op's matrix (gate/up: the same rows of both matrices),
-// streamed as stages of whole contiguous rows (one bulk copy per matrix per stage).
+// streamed as stages of whole contiguous rows (one bulk copy per contiguous run of rows).
 __device__ __forceinline__ int gemv_K(const Params& p, int op) {
-  return op == OP_O ? p.Hq * p.D : (op == OP_DOWN ? p.F : p.d);
-}
-// Row n of segment `seg` of the op's matrix; *run receives how many rows from n on lie
-// in the same physical matrix (QKV rows cross from Wq into Wk into Wv).
-__device__ __forceinline__ const uint16_t* gemv_row(const Params& p, int op, int layer, int seg,
-                                                    int n, int K, int* run) {
-  *run = 0x7fffffff;
-  if (op == OP_LM) return p.lm_head + (size_t)n * K;
-  const LayerPtrs& L = p.layers[layer];
   switch (op) {
-    case OP_QKV: {
-      const int nq = p.Hq * p.D, nk = p.Hkv * p.D;
-      if (n < nq) { *run = nq - n; return L.w[TRE_W_Q] + (size_t)n * K; }
-      if (n < nq + nk) { *run = nq + nk - n; return L.w[TRE_W_K] + (size_t)(n - nq) * K; }
-      return L.w[TRE_W_V] + (size_t)(n - nq - nk) * K;
-    }
-    case OP_O: return L.w[TRE_W_O] + (size_t)n * K;
-    case OP_GU: return (seg ? L.w[TRE_W_UP] : L.w[TRE_W_GATE]) + (size_t)n * K;
-    default: return L.w[TRE_W_DOWN] + (size_t)n * K;
+    case OP_O: return p.Hq * p.D;
+    case OP_DOWN: return p.F;
+    case OP_MDOWN: return (p.nshared + p.topk) * p.Fe;
+    default: return p.d;
   }
 }
 
+// Tasks whose weight addresses depend on this step's routing (the selected experts).
+__device__ __forceinline__ bool needs_route(const Params& p, const Task& t) {
+  return t.type == T_GEMV && (t.op == OP_RGU || (t.op == OP_MDOWN && (t.aux & 0xff) >= p.nshared));
+}
+
+// The expert selected in slot j of `layer` (valid once the layer's route counter is met);
+// an id outside [0, E) records a bounds error and is clamped so no access leaves the
+// expert tensors.
+__device__ __forceinline__ int routed_expert(const Params& p, int layer, int j, int detail) {
+  const int e = __ldcg(p.route_idx + layer * p.topk + j);
+  if (e < 0 || e >= p.E) {
+    record_error(p, TRE_ERR_BOUNDS, detail);
+    return 0;
+  }
+  return e;
+}
 struct GemvGeom {
   int K;        // full row length (inputs)
   int nseg;     // 2 for gate/up (a row of each matrix), else 1
@@ -138,8 +146,8 @@ struct GemvGeom {
 __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   GemvGeom g;
   g.K = gemv_K(p, t.op);
-  g.nseg = t.op == OP_GU ? 2 : 1;
-  if (t.op == OP_LM) {
+  g.nseg = (t.op == OP_GU || t.op == OP_SGU || t.op == OP_RGU) ? 2 : 1;
+  if (t.op == OP_LM || t.op == OP_ROUTER) {
     g.np = 1;
     g.part = 0;
   } else {
@@ -152,6 +160,48 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes);
   g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
   return g;
+}
+
+// Source of this task's K-part of row n of segment `seg`; *contig receives how many rows
+// from n on follow it contiguously in memory (same matrix, row stride = the part length):
+// QKV rows cross from Wq into Wk into Wv, routed rows end at their expert's last row,
+// K-parts of a wider matrix are one row each.
+__device__ __forceinline__ const uint16_t* part_row(const Params& p, const Task& t,
+                                                    const GemvGeom& g, int seg, int n,
+                                                    int* contig) {
+  *contig = 0x7fffffff;
+  if (t.op == OP_LM) return p.lm_head + (size_t)n * g.K;
+  const LayerPtrs& L = p.layers[t.layer];
+  const size_t K = (size_t)g.K;
+  switch (t.op) {
+    case OP_QKV: {
+      const int nq = p.Hq * p.D, nk = p.Hkv * p.D;
+      if (n < nq) { *contig = nq - n; return L.w[TRE_W_Q] + (size_t)n * K; }
+      if (n < nq + nk) { *contig = nq + nk - n; return L.w[TRE_W_K] + (size_t)(n - nq) * K; }
+      return L.w[TRE_W_V] + (size_t)(n - nq - nk) * K;
+    }
+    case OP_O:
+    case OP_DOWN:
+      if (g.np > 1) *contig = 1;
+      return L.w[t.op == OP_O ? TRE_W_O : TRE_W_DOWN] + (size_t)n * K + g.k0;
+    case OP_GU: return L.w[seg ? TRE_W_UP : TRE_W_GATE] + (size_t)n * K;
+    case OP_ROUTER: return L.w[TRE_W_ROUTER] + (size_t)n * K;
+    case OP_SGU: return L.w[seg ? TRE_W_SHARED_UP : TRE_W_SHARED_GATE] + (size_t)n * K;
+    case OP_RGU: {
+      const int j = n / p.Fe, r = n - j * p.Fe;
+      const int e = routed_expert(p, t.layer, j, t.id);
+      *contig = p.Fe - r;
+      return L.w[seg ? TRE_W_EXPERT_UP : TRE_W_EXPERT_GATE] + ((size_t)e * p.Fe + r) * K;
+    }
+    default: {  // OP_MDOWN: part < nshared is a column slice of the shared down matrix
+      if (g.part < p.nshared) {
+        if (p.nshared > 1) *contig = 1;
+        return L.w[TRE_W_SHARED_DOWN] + (size_t)n * p.nshared * p.Fe + (size_t)g.part * p.Fe;
+      }
+      const int e = routed_expert(p, t.layer, g.part - p.nshared, t.id);
+      return L.w[TRE_W_EXPERT_DOWN] + ((size_t)e * p.d + n) * p.Fe;
+    }
+  }
 }
 
 __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& t0, int& t1) {
@@ -168,66 +218,57 @@ __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
 }
 
 // ---- producer -------------------------------------------------------------------------------
-// Lane `lane`'s piece of stage i of task t: source, byte offset in the stage, bytes (0 = no
-// piece for this lane); *total receives the stage's byte count.  GEMV stages are whole
-// rows (gate/up: the rows of both matrices at a fixed offset; QKV: cut where the stacked
-// rows cross from Wq to Wk to Wv); attention stages are the K and V rows of up to `pps`
+// Bytes of stage i of task t.  GEMV stages are whole rows of the task's K-part (gate/up:
+// the rows of both matrices); attention stages are the K and V rows of up to `pps`
 // consecutive cached positions of one kv head.
-__device__ __forceinline__ const uint8_t* stage_piece(const Params& p, const Task& t,
-                                                      const GemvGeom& g, int t0, int t1, int i,
-                                                      int lane, uint32_t* off, uint32_t* bytes,
-                                                      uint32_t* total) {
-  const uint8_t* src = nullptr;
-  *off = 0;
-  *bytes = 0;
+__device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, const GemvGeom& g,
+                                                int t0, int t1, int i) {
   if (t.type == T_GEMV) {
-    const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
-    const size_t rowb = (size_t)g.Kp * 2;  // bytes of one row's part in the stage
-    *total = (uint32_t)(g.nseg * nr * rowb);
-    if (g.np > 1) {  // K-parts: rows are strided in memory, one copy per row
-      if (lane < nr * g.nseg) {
-        const int seg = lane / nr, r = lane % nr;
-        int run;
-        src = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, seg, n0 + r, g.K, &run) + g.k0);
-        *off = (uint32_t)((seg * g.rps + r) * rowb);
-        *bytes = (uint32_t)rowb;
-      }
-    } else if (g.nseg == 2) {
-      if (lane < 2) {
-        int run;
-        src = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, lane, n0, g.K, &run));
-        *off = (uint32_t)(lane * g.rps * rowb);
-        *bytes = (uint32_t)(nr * rowb);
-      }
-    } else if (lane < 3) {
-      int n = n0, left = nr, piece = 0;
-      while (left > 0) {
-        int run;
-        const uint16_t* w = gemv_row(p, t.op, t.layer, 0, n, g.K, &run);
-        const int take = min(left, run);
-        if (piece == lane) {
-          src = reinterpret_cast<const uint8_t*>(w);
-          *off = (uint32_t)((n - n0) * rowb);
-          *bytes = (uint32_t)(take * rowb);
-        }
-        n += take;
-        left -= take;
+    const int nr = min(g.rps, t.r1 - (t.r0 + i * g.rps));
+    return (uint32_t)(g.nseg * nr * g.Kp * 2);
+  }
+  const int n = min(p.pps, t1 - (t0 + i * p.pps));
+  return (uint32_t)(2 * n * p.D * 2);
+}
+
+// Issue the bulk copies of stage i into `dst`: one copy per contiguous run of rows (per
+// segment; gate rows at the stage's start, up rows after `rps` rows), spread over the
+// producer lanes; attention: the K rows then the V rows (lanes 0 and 1).
+__device__ __forceinline__ void issue_stage(const Params& p, const Task& t, const GemvGeom& g,
+                                            int t0, int t1, int i, int lane, uint8_t* dst,
+                                            uint64_t* bar, uint64_t pol) {
+  if (t.type == T_GEMV) {
+    const int n0 = t.r0 + i * g.rps, n1 = min(t.r1, n0 + g.rps);
+    const uint32_t rowb = (uint32_t)g.Kp * 2u;
+    // common case: each segment's rows of the stage are one contiguous run (one lookup
+    // per segment, lanes in parallel)
+    int contig = 0;
+    const uint16_t* w0 = lane < g.nseg ? part_row(p, t, g, lane, n0, &contig) : nullptr;
+    if (__all_sync(0xffffffffu, lane >= g.nseg || contig >= n1 - n0)) {
+      if (lane < g.nseg)
+        bulk_g2s(dst + (size_t)lane * g.rps * rowb, w0, (uint32_t)(n1 - n0) * rowb, bar, pol);
+      return;
+    }
+    int piece = 0;
+    for (int seg = 0; seg < g.nseg; ++seg) {
+      for (int n = n0; n < n1;) {
+        int contig;
+        const uint16_t* w = part_row(p, t, g, seg, n, &contig);
+        const int take = min(n1 - n, contig);
+        if ((piece & 31) == lane)
+          bulk_g2s(dst + (size_t)(seg * g.rps + (n - n0)) * rowb, w, (uint32_t)take * rowb, bar, pol);
         ++piece;
+        n += take;
       }
     }
-  } else {
+  } else if (lane < 2) {
     const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
     const size_t rowb = (size_t)p.D * 2;
-    *total = (uint32_t)(2 * n * rowb);
-    if (lane < 2) {
-      const LayerPtrs& L = p.layers[t.layer];
-      const uint16_t* base = lane == 0 ? L.k_cache : L.v_cache;
-      src = reinterpret_cast<const uint8_t*>(base) + ((size_t)t.r0 * p.cap + tt) * rowb;
-      *off = (uint32_t)(lane * p.pps * rowb);
-      *bytes = (uint32_t)(n * rowb);
-    }
+    const LayerPtrs& L = p.layers[t.layer];
+    const uint16_t* base = lane == 0 ? L.k_cache : L.v_cache;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(base) + ((size_t)t.r0 * p.cap + tt) * rowb;
+    bulk_g2s(dst + (size_t)lane * p.pps * rowb, src, (uint32_t)(n * rowb), bar, pol);
   }
-  return src;
 }
 
 // L2 prefetch of a whole task ahead of its stages: the contiguous byte ranges task t will
@@ -241,19 +282,19 @@ __device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, in
   long long bytes[3] = {0, 0, 0};
   if (t.type == T_GEMV) {
     const GemvGeom g = gemv_geom(p, t);
-    if (g.np > 1) return;
+    if (g.np > 1 || needs_route(p, t)) return;  // strided rows, or addresses not known yet
     const size_t rowb = (size_t)g.K * 2;
     if (g.nseg == 2) {
       for (int s = 0; s < 2; ++s) {
         int run;
-        src[s] = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, s, t.r0, g.K, &run));
+        src[s] = reinterpret_cast<const uint8_t*>(part_row(p, t, g, s, t.r0, &run));
         bytes[s] = (long long)(t.r1 - t.r0) * rowb;
       }
     } else {
       int n = t.r0, left = t.r1 - t.r0;
       for (int piece = 0; left > 0 && piece < 3; ++piece) {
         int run;
-        src[piece] = reinterpret_cast<const uint8_t*>(gemv_row(p, t.op, t.layer, 0, n, g.K, &run));
+        src[piece] = reinterpret_cast<const uint8_t*>(part_row(p, t, g, 0, n, &run));
         const int take = min(left, run);
         bytes[piece] = (long long)take * rowb;
         n += take;
@@ -306,6 +347,12 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
       if (!ok) break;
     }
+    if (needs_route(p, t)) {  // the expert ids pick the addresses: wait for the routing
+      bool r = true;
+      if (lane == 0) r = wait_counter(p, t.layer * C_PER_LAYER + C_ROUTE, 1u, t.id);
+      ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
     if (window > 0 && ti + 1 < ntask) task_prefetch(p, my[ti + 1], lane, window);
     const int ns = task_nstages(p, t);
     GemvGeom g{};
@@ -320,14 +367,12 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
         ok = false;
         break;
       }
-      uint32_t off, bytes, total;
-      const uint8_t* src = stage_piece(p, t, g, t0, t1, i, lane, &off, &bytes, &total);
       if (lane == 0) {
         *reinterpret_cast<volatile uint32_t*>(tags + slot) = gs;
-        mbar_arrive_expect_tx(&full[slot], total);
+        mbar_arrive_expect_tx(&full[slot], stage_total(p, t, g, t0, t1, i));
       }
       __syncwarp();
-      if (bytes) bulk_g2s(ring + (size_t)slot * SB + off, src, bytes, &full[slot], pol);
+      issue_stage(p, t, g, t0, t1, i, lane, ring + (size_t)slot * SB, &full[slot], pol);
     }
   }
   if (!ok && lane == 0) {
@@ -366,17 +411,19 @@ __device__ __forceinline__ float resid_in(const Params& p, int layer, int n) {
   return bf_lo(p.embed[(size_t)p.token * p.d + n]);
 }
 
-// Input-vector identity for reuse across consecutive tasks (same layer, same source).
+// Input-vector identity for reuse across consecutive tasks (same layer, same source,
+// same K-part).  The router, shared and routed gate/up all read RMSNorm(h1).
 __device__ __forceinline__ int input_key(const Task& t) {
   int cls;
   switch (t.op) {
     case OP_QKV: cls = 0; break;
     case OP_O: cls = 1; break;
-    case OP_GU: cls = 2; break;
-    case OP_DOWN: cls = 3; break;
+    case OP_GU: case OP_ROUTER: case OP_SGU: case OP_RGU: cls = 2; break;
+    case OP_DOWN: case OP_MDOWN: cls = 3; break;
     default: cls = 4; break;
   }
-  return (((int)t.layer * 8 + cls) << 4) | (t.op == OP_LM ? 0 : (t.aux & 0xf));
+  const int part = (t.op == OP_LM || t.op == OP_ROUTER) ? 0 : (t.aux & 0xff);
+  return (((int)t.layer * 8 + cls) << 8) | part;
 }
 
 // Stage the GEMV input into the two planes; returns the RMSNorm scale (1 when none).
@@ -396,8 +443,9 @@ __device__ float load_input(const Params& p, const Task& t, const GemvGeom& gg, 
       else src_bf = p.embed + (size_t)p.token * p.d;
       break;
     case OP_O: src = p.attn; break;
-    case OP_GU: src = p.h1; gain = p.layers[t.layer].w[TRE_W_FFN_NORM]; break;
-    case OP_DOWN: src = p.u; break;
+    case OP_GU: case OP_ROUTER: case OP_SGU: case OP_RGU:
+      src = p.h1; gain = p.layers[t.layer].w[TRE_W_FFN_NORM]; break;
+    case OP_DOWN: case OP_MDOWN: src = p.u; break;
     default: src = p.x; gain = p.final_norm; break;
   }
   if (src) src += gg.k0;        // normalised inputs are single-part (k0 = 0)
@@ -667,7 +715,7 @@ __device__ __forceinline__ void prefetch_resid(const Params& p, const Task& t, c
     const int n = t.r0 + r;
     float v;
     if (t.op == OP_O) v = g.part == 0 ? resid_in(p, t.layer, n) : __ldcg(p.h1 + n);
-    else v = g.part == 0 ? __ldcg(p.h1 + n) : __ldcg(p.x + n);
+    else v = g.part == 0 ? __ldcg(p.h1 + n) : __ldcg(p.x + n);  // down / MoE down
     resid[r] = v;
   }
 }
@@ -677,7 +725,9 @@ __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const 
   switch (t.op) {
     case OP_QKV: p.qkv[n] = v * rn; break;
     case OP_O: p.h1[n] = resid[n - t.r0] + v; break;
-    case OP_DOWN: {
+    case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
+    case OP_DOWN:
+    case OP_MDOWN: {
       const float y = resid[n - t.r0] + v;
       p.x[n] = y;
       if (g.part == g.np - 1) {
@@ -691,6 +741,43 @@ __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const 
       best_update(best, y, n);
     } break;
   }
+}
+
+// ---- MoE routing -----------------------------------------------------------------------------------
+// Run by the router task that finishes last (arrival ticket): the top_k experts by score,
+// ties to the lower expert index, in descending order, and their weights normalised over
+// the selection (DeepSeek-style sigmoid routing; the pages name the fused op
+// ExpertSelectUpGateSiLU — TileRT code audit, MoE paragraph).  Warp 0 selects: each lane
+// holds the scores of experts lane, lane + 32, ...; every round is one warp arg-max.
+// Then the layer's route counter is bumped with release semantics.
+__device__ void route_topk(const Params& p, int layer, float* sc, int warp, int lane, int ctid) {
+  for (int e = ctid; e < p.E; e += kConsumerThreads) sc[e] = __ldcg(p.scores + e);
+  consumer_sync(kConsumerThreads);
+  if (warp != 0) return;
+  uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
+  float tot = 0.f, mine = 0.f;
+  for (int j = 0; j < p.topk; ++j) {
+    Best b{-INFINITY, 0x7fffffff};
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = lane + 32 * i;
+      if (e < p.E && !((taken >> i) & 1u)) best_update(b, sc[e], e);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      Best o;
+      o.v = __shfl_xor_sync(0xffffffffu, b.v, off);
+      o.i = __shfl_xor_sync(0xffffffffu, b.i, off);
+      best_update(b, o.v, o.i);
+    }
+    if (b.i != 0x7fffffff && (b.i & 31) == lane) taken |= 1u << (b.i >> 5);
+    tot += b.v;
+    if (lane == j) mine = b.v;
+    if (lane == 0) p.route_idx[layer * p.topk + j] = b.i;
+  }
+  if (lane < p.topk) p.route_w[layer * p.topk + lane] = mine / tot;
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) red_release_gpu_add(p.counters + layer * C_PER_LAYER + C_ROUTE, 1u);
 }
 
 // ---- consumers -----------------------------------------------------------------------------------
@@ -729,7 +816,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       const GemvGeom g = gemv_geom(p, t);
       const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
-      const bool has_resid = t.op == OP_O || t.op == OP_DOWN;
+      const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MDOWN;
       if (has_resid) prefetch_resid(p, t, g, resid, ctid);
       if (key != cur_key) {
         const float rn = load_input(p, t, g, ub, red, ctid);
@@ -755,6 +842,13 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
         if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;
+          // routed experts: the slot's weight folds into u; u holds the shared slices first
+          float wsel = 1.f;
+          int uoff = 0;
+          if (t.op == OP_RGU) {
+            wsel = __ldcg(p.route_w + t.layer * p.topk + t.r0 / p.Fe);
+            uoff = p.nshared * p.Fe;
+          }
           for (int r = 0; r < nr; r += 2) {
             const int np = min(2, nr - r);
             float o0, o1, o2, o3;
@@ -772,7 +866,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
             const int k = (lane >> 3) & 1;
             if ((np == 2 && (lane & 23) == 0) || (np == 1 && lane == 0)) {
               const float a = v * rn, bb = upv * rn;
-              p.u[n0 + r + k] = a / (1.f + expf(-a)) * bb;
+              p.u[uoff + n0 + r + k] = wsel * (a / (1.f + expf(-a)) * bb);
             }
           }
         } else {
@@ -817,7 +911,16 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
           if (p.token_out) *p.token_out = (int32_t)(0xffffffffu - (uint32_t)(w & 0xffffffffull));
         }
       }
-      if (ctid == 0 && t.out >= 0) red_release_gpu_add(p.counters + t.out, 1u);
+      if (t.op == OP_ROUTER) {  // the last router task of the layer selects the experts
+        if (ctid == 0) {
+          const uint32_t old = atom_acq_rel_gpu_add(p.router_ticket, 1u);
+          flags[1] = ((old + 1u) % (uint32_t)t.aux) == 0u;
+        }
+        consumer_sync(kConsumerThreads);
+        if (flags[1]) route_topk(p, t.layer, ub + p.xs_floats, warp, lane, ctid);
+      } else if (ctid == 0 && t.out >= 0) {
+        red_release_gpu_add(p.counters + t.out, 1u);
+      }
     }
     if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 2] = (long long)globaltimer_ns();
     gs += (uint32_t)ns;

@@ -109,6 +109,8 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   if (st != TRE_OK) return st;
   if (!s.has_lm)
     return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: needs an embedding and LM head");
+  if (s.kind != TRE_LAYER_GQA)
+    return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: GQA stacks only");
   if (cfg->debug_flags & (TRE_DEBUG_HIDDEN | TRE_DEBUG_TRACE))
     return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: debug buffers are not available");
 

@@ -95,26 +95,38 @@ struct Builder {
   }
 
   // Cut N rows (K inputs each, nseg matrices) into per-SM ranges; a range longer than
-  // `cap` rows becomes several sub-ranges, and each sub-range one task per K-part (only
-  // the last part bumps `out`).  Returns the number of tasks that bump `out`.
+  // `cap` rows becomes several sub-ranges, a range is also cut at every multiple of
+  // `cut` (> 0: rows of different experts never share a task), and each sub-range is one
+  // task per K-part (only the last part bumps `out`).  `np` > 0 fixes the number of
+  // K-parts (else they follow from K).  Returns the number of tasks that bump `out`.
   int gemv(uint8_t op, int layer, int N, int K, int nseg, int dep, uint32_t dep_count, int out,
-           int cap) {
-    const int np = op == OP_LM ? 1 : gemv_nparts(K);
+           int cap, int np = 0, int cut = 0) {
+    if (np <= 0) np = (op == OP_LM || op == OP_ROUTER) ? 1 : gemv_nparts(K);
     auto ranges = assign_rows(N, (int64_t)nseg * K * 2, cum);
     int n = 0;
     for (int s = 0; s < nsm; ++s) {
-      for (int r = ranges[s].first; r < ranges[s].second; r += cap) {
+      for (int r = ranges[s].first; r < ranges[s].second;) {
+        int e = std::min(ranges[s].second, r + cap);
+        if (cut > 0) e = std::min(e, (r / cut + 1) * cut);
         for (int part = 0; part < np; ++part) {
           Task t = make(T_GEMV, op, layer, dep, dep_count, part == np - 1 ? out : -1);
           t.r0 = r;
-          t.r1 = std::min(ranges[s].second, r + cap);
+          t.r1 = e;
           t.aux = part | (np << 8);
           q[s].push_back(t);
           if (part == np - 1) ++n;
         }
+        r = e;
       }
     }
     return n;
+  }
+
+  // Set aux = count on every task of `op` created since task id `first`.
+  void set_count(int first, uint8_t op, int count) {
+    for (auto& qq : q)
+      for (auto& t : qq)
+        if (t.id >= first && t.type == T_GEMV && t.op == op) t.aux = count;
   }
 
   void attention(int layer, int Hkv, int S, int64_t bytes_per_task, int dep, uint32_t dep_count,
@@ -133,9 +145,20 @@ struct Builder {
 };
 
 static tre_status validate(const tre_config& c) {
-  if (c.kind == TRE_LAYER_MLA || c.kind == TRE_LAYER_MOE)
-    return fail(TRE_ERR_UNSUPPORTED, "layer kind not implemented in this build (GQA only)");
-  if (c.kind != TRE_LAYER_GQA) return fail(TRE_ERR_INVALID_ARG, "unknown layer kind");
+  if (c.kind == TRE_LAYER_MLA)
+    return fail(TRE_ERR_UNSUPPORTED, "layer kind not implemented in this build (GQA, MOE)");
+  if (c.kind != TRE_LAYER_GQA && c.kind != TRE_LAYER_MOE)
+    return fail(TRE_ERR_INVALID_ARG, "unknown layer kind");
+  if (c.kind == TRE_LAYER_MOE) {
+    if (c.n_experts < 1 || c.n_experts > kMaxExperts)
+      return fail(TRE_ERR_UNSUPPORTED, "n_experts must be in [1, 512]");
+    if (c.top_k < 1 || c.top_k > c.n_experts || c.top_k > kMaxTopK)
+      return fail(TRE_ERR_INVALID_ARG, "top_k must be in [1, min(n_experts, 32)]");
+    if (c.n_shared < 0 || c.n_shared > 16)
+      return fail(TRE_ERR_INVALID_ARG, "n_shared must be in [0, 16]");
+    if (c.expert_ffn < 8 || c.expert_ffn % 8)
+      return fail(TRE_ERR_INVALID_ARG, "expert_ffn must be a positive multiple of 8");
+  }
   for (int r : c.reserved)
     if (r != 0) return fail(TRE_ERR_INVALID_ARG, "reserved config fields must be zero");
   if (c.n_layers < 1 || c.n_layers > 1024) return fail(TRE_ERR_INVALID_ARG, "n_layers out of range");
@@ -147,7 +170,8 @@ static tre_status validate(const tre_config& c) {
     return fail(TRE_ERR_UNSUPPORTED, "q heads per kv head must be 1, 2, 4 or 8");
   if (c.head_dim != 64 && c.head_dim != 128)
     return fail(TRE_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
-  if (c.ffn < 8 || c.ffn % 8) return fail(TRE_ERR_INVALID_ARG, "ffn must be a positive multiple of 8");
+  if (c.kind == TRE_LAYER_GQA && (c.ffn < 8 || c.ffn % 8))
+    return fail(TRE_ERR_INVALID_ARG, "ffn must be a positive multiple of 8");
   if (c.has_embed_lm_head != 0 && c.has_embed_lm_head != 1)
     return fail(TRE_ERR_INVALID_ARG, "has_embed_lm_head must be 0 or 1");
   if (c.has_embed_lm_head && c.vocab < 1) return fail(TRE_ERR_INVALID_ARG, "vocab must be >= 1");
@@ -174,6 +198,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   if (smem_limit > kSmemLimit) smem_limit = kSmemLimit;
 
   PlanShape s{};
+  s.kind = c.kind;
   s.d = c.hidden;
   s.Hq = c.n_q_heads;
   s.Hkv = c.n_kv_heads;
@@ -185,19 +210,36 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   s.M = c.max_tokens_per_step < 1 ? 1 : c.max_tokens_per_step;
   s.nsm = nsm;
   s.has_lm = c.has_embed_lm_head;
+  const bool moe = c.kind == TRE_LAYER_MOE;
+  if (moe) {
+    s.F = 0;
+    s.E = c.n_experts;
+    s.topk = c.top_k;
+    s.nshared = c.n_shared;
+    s.Fe = c.expert_ffn;
+  }
+  s.u_floats = moe ? (s.nshared + s.topk) * s.Fe : s.F;
   const int G = s.Hq / s.Hkv;
 
   // Inputs longer than kMaxKPart are staged in K-parts; ops that normalise their input
   // (QKV, gate/up, LM head) need the whole vector at once.
   if (s.d > kMaxKPart)
     return fail(TRE_ERR_UNSUPPORTED, "hidden above 16384 (normalised inputs are staged whole)");
-  const int Ks[OP_COUNT] = {s.d, s.Hq * s.D, s.d, s.F, s.d};
-  const int segs[OP_COUNT] = {1, 1, 2, 1, 1};
+  // (input length, segments, K-part length) of every op the stack uses
+  struct OpShape { int K, nseg, kp; };
+  std::vector<OpShape> ops = {{s.d, 1, 0}, {s.Hq * s.D, 1, 0}, {s.d, 1, s.d}};
+  if (moe) {
+    ops.push_back({s.d, 2, 0});                                  // shared / routed gate-up
+    ops.push_back({(s.nshared + s.topk) * s.Fe, 1, s.Fe});       // MoE down: one part per expert
+  } else {
+    ops.push_back({s.d, 2, 0});
+    ops.push_back({s.F, 1, 0});
+  }
   int xs = 8, need = 4 * s.D * 8;  // a stage holds at least 8 KV positions
-  for (int op = 0; op < OP_COUNT; ++op) {
-    const int kp = gemv_part_len(Ks[op], op == OP_LM ? 1 : gemv_nparts(Ks[op]));
+  for (auto& o : ops) {
+    const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K));
     xs = std::max(xs, kp);
-    need = std::max(need, segs[op] * kp * 2);
+    need = std::max(need, o.nseg * kp * 2);
   }
   // A ring stage holds whole rows of one K-part (gate/up: a row of each matrix), or the K
   // and V rows of 8-64 cached positions.
@@ -251,8 +293,25 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     const int64_t kv_task_bytes = (int64_t)(s.cap - s.M) / S * s.D * 2 * 2;
     b.attention(l, s.Hkv, S, kv_task_bytes, cq, (uint32_t)nqkv, ca);
     int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)s.Hkv, co, s.resid_floats);
-    int ng = b.gemv(OP_GU, l, s.F, s.d, 2, co, (uint32_t)no, cg, big);
-    int nd = b.gemv(OP_DOWN, l, s.d, s.F, 1, cg, (uint32_t)ng, cd, s.resid_floats);
+    int nd;
+    if (!moe) {
+      int ng = b.gemv(OP_GU, l, s.F, s.d, 2, co, (uint32_t)no, cg, big);
+      nd = b.gemv(OP_DOWN, l, s.d, s.F, 1, cg, (uint32_t)ng, cd, s.resid_floats);
+    } else {
+      // Router rows first, then the shared expert (which needs no routing, so its weights
+      // stream while the top-k is decided), then the selected experts' gate/up rows: their
+      // producer waits for the route counter, since the expert ids pick the addresses.
+      const int cr = counter_of(l, C_ROUTE);
+      const int first = b.next_id;
+      const int nr = b.gemv(OP_ROUTER, l, s.E, s.d, 1, co, (uint32_t)no, cr, big);
+      b.set_count(first, OP_ROUTER, nr);
+      int ng = 0;
+      if (s.nshared > 0) ng += b.gemv(OP_SGU, l, s.nshared * s.Fe, s.d, 2, co, (uint32_t)no, cg, big);
+      ng += b.gemv(OP_RGU, l, s.topk * s.Fe, s.d, 2, cr, 1u, cg, big, 0, s.Fe);
+      // down: K-parts of Fe inputs, one per shared-expert slice and per selected expert
+      const int np = s.nshared + s.topk;
+      nd = b.gemv(OP_MDOWN, l, s.d, np * s.Fe, 1, cg, (uint32_t)ng, cd, s.resid_floats, np);
+    }
     prev_down = cd;
     prev_down_count = (uint32_t)nd;
   }
@@ -262,9 +321,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     int first = b.next_id;
     int nlm = b.gemv(OP_LM, s.L - 1, s.V, s.d, 1, prev_down, prev_down_count, c_lm, 1 << 30);
     s.n_lm_tasks = nlm;
-    for (auto& qq : b.q)
-      for (auto& t : qq)
-        if (t.id >= first && t.type == T_GEMV && t.op == OP_LM) t.aux = nlm;
+    b.set_count(first, OP_LM, nlm);
   }
   if (c.debug_flags & TRE_DEBUG_FAULT_INJECT) {
     // the first O-projection task of layer 0 waits on a counter nothing bumps
@@ -298,8 +355,11 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
 
 int64_t step_bytes(const PlanShape& s, int pos) {
   const int64_t d = s.d, D = s.D;
-  int64_t per_layer = ((int64_t)(s.Hq + 2 * s.Hkv) * D * d + d * s.Hq * D + 3LL * s.F * d) * 2 +
-                      2 * d * 2;
+  // MoE: the router, the shared experts and the selected experts only (what one token reads)
+  const int64_t mlp = s.kind == TRE_LAYER_MOE
+                          ? (int64_t)s.E * d + 3LL * (s.nshared + s.topk) * s.Fe * d
+                          : 3LL * s.F * d;
+  int64_t per_layer = ((int64_t)(s.Hq + 2 * s.Hkv) * D * d + d * s.Hq * D + mlp) * 2 + 2 * d * 2;
   int64_t bytes = per_layer * s.L;
   bytes += (int64_t)s.L * s.Hkv * (int64_t)pos * D * 2 * 2;  // K and V read
   bytes += (int64_t)s.L * s.Hkv * D * 2 * 2;                 // this token's K and V written

@@ -173,10 +173,17 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   }
   static const int gqa_slots[] = {TRE_W_ATTN_NORM, TRE_W_Q,        TRE_W_K,  TRE_W_V,   TRE_W_O,
                                   TRE_W_FFN_NORM,  TRE_W_GATE,     TRE_W_UP, TRE_W_DOWN};
+  std::vector<int> slots(gqa_slots, gqa_slots + 9);
+  if (s.kind == TRE_LAYER_MOE) {
+    slots = {TRE_W_ATTN_NORM, TRE_W_Q, TRE_W_K, TRE_W_V, TRE_W_O, TRE_W_FFN_NORM, TRE_W_ROUTER,
+             TRE_W_EXPERT_GATE, TRE_W_EXPERT_UP, TRE_W_EXPERT_DOWN};
+    if (s.nshared > 0)
+      slots.insert(slots.end(), {TRE_W_SHARED_GATE, TRE_W_SHARED_UP, TRE_W_SHARED_DOWN});
+  }
   std::vector<LayerPtrs> lp(s.L);
   for (int l = 0; l < s.L; ++l) {
     std::memset(&lp[l], 0, sizeof(LayerPtrs));
-    for (int slot : gqa_slots) {
+    for (int slot : slots) {
       const void* p = w->layer_w[(size_t)l * TRE_W_SLOTS + slot];
       if (!aligned16(p)) {
         set_error("tre_create: layer " + std::to_string(l) + " slot " + std::to_string(slot) +
@@ -225,7 +232,12 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_h1 = cv.take<float>(s.d);
   size_t o_qkv = cv.take<float>(qkv_n);
   size_t o_attn = cv.take<float>((size_t)s.Hq * s.D);
-  size_t o_u = cv.take<float>(s.F);
+  size_t o_u = cv.take<float>(s.u_floats);
+  const bool moe = s.kind == TRE_LAYER_MOE;
+  size_t o_scores = cv.take<float>(moe ? s.E : 1);
+  size_t o_ridx = cv.take<int32_t>(moe ? (size_t)s.L * s.topk : 1);
+  size_t o_rw = cv.take<float>(moe ? (size_t)s.L * s.topk : 1);
+  size_t o_rtick = cv.take<uint32_t>(1);
   size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (s.D + 2));
   size_t o_logits = cv.take<float>(s.V > 0 ? s.V : 1);
   size_t o_tok = cv.take<int32_t>(1);
@@ -287,6 +299,11 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.qkv = reinterpret_cast<float*>(B + o_qkv);
   p.attn = reinterpret_cast<float*>(B + o_attn);
   p.u = reinterpret_cast<float*>(B + o_u);
+  p.scores = reinterpret_cast<float*>(B + o_scores);
+  p.route_idx = reinterpret_cast<int32_t*>(B + o_ridx);
+  p.route_w = reinterpret_cast<float*>(B + o_rw);
+  p.router_ticket = reinterpret_cast<uint32_t*>(B + o_rtick);
+  p.E = s.E; p.topk = s.topk; p.nshared = s.nshared; p.Fe = s.Fe;
   p.part = reinterpret_cast<float*>(B + o_part);
   p.logits = reinterpret_cast<float*>(B + o_logits);
   e->logits_buf = p.logits;
@@ -388,6 +405,46 @@ TRE_EXPORT tre_status tre_decode_step_host(tre_engine* e, int32_t token, int32_t
   return pending_device_error(e);
 }
 
+TRE_EXPORT tre_status tre_layers_step(tre_engine* e, const float* x_in_dev, float* x_out_dev,
+                                      int32_t pos, tre_stream stream) {
+  if (!e || !x_in_dev || !x_out_dev) {
+    set_error("tre_layers_step: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (e->shape.has_lm) {
+    set_error("tre_layers_step: engine has an embedding / LM head (use tre_decode_step)");
+    return TRE_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(x_in_dev) || !aligned16(x_out_dev)) {
+    set_error("tre_layers_step: x_in_dev / x_out_dev must be 16-byte aligned");
+    return TRE_ERR_INVALID_ARG;
+  }
+  const size_t bytes = (size_t)e->shape.d * sizeof(float);
+  const uintptr_t a = (uintptr_t)x_in_dev, b = (uintptr_t)x_out_dev;
+  if (a < b + bytes && b < a + bytes) {
+    set_error("tre_layers_step: x_out_dev overlaps x_in_dev");
+    return TRE_ERR_INVALID_ARG;
+  }
+  return launch_step(e, 0, pos, (cudaStream_t)stream, nullptr, nullptr, x_in_dev, x_out_dev);
+}
+
+TRE_EXPORT tre_status tre_debug_routing(tre_engine* e, int32_t* idx_host, float* w_host) {
+  if (!e) {
+    set_error("tre_debug_routing: NULL engine");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (e->shape.kind != TRE_LAYER_MOE) {
+    set_error("tre_debug_routing: not a MoE engine");
+    return TRE_ERR_UNSUPPORTED;
+  }
+  CK(cudaSetDevice(e->device));
+  if (e->last_stream) CK(cudaStreamSynchronize(e->last_stream));
+  const size_t n = (size_t)e->shape.L * e->shape.topk;
+  if (idx_host) CK(cudaMemcpy(idx_host, e->base.route_idx, n * 4, cudaMemcpyDeviceToHost));
+  if (w_host) CK(cudaMemcpy(w_host, e->base.route_w, n * 4, cudaMemcpyDeviceToHost));
+  return TRE_OK;
+}
+
 TRE_EXPORT tre_status tre_get_status(tre_engine* e, int32_t* device_status, int32_t* detail_out) {
   if (!e || !device_status) {
     set_error("tre_get_status: NULL argument");
@@ -414,6 +471,7 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
   CK(cudaMemsetAsync(p.counters, 0, (size_t)e->shape.n_counters * 4, s));
   CK(cudaMemsetAsync(p.tickets, 0, (size_t)e->shape.Hkv * 4, s));
   CK(cudaMemsetAsync(p.lm_ticket, 0, 4, s));
+  CK(cudaMemsetAsync(p.router_ticket, 0, 4, s));
   CK(cudaMemsetAsync(p.argmax_slot, 0, 8, s));
   CK(cudaMemsetAsync(p.err, 0, 8, s));  // error word + abort flag
   CK(cudaStreamSynchronize(s));

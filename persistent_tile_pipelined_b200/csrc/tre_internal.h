@@ -18,6 +18,9 @@ constexpr int kDefaultStageBytes = 32768;  // a bulk-copy stage costs ~0.4 us pe
 constexpr int kMaxKPart = 16384;         // longest input slice one GEMV task stages (floats)
 constexpr int kMaxResidRows = 512;       // rows per task of ops that add a residual
 constexpr int kTraceCols = 8;          // int64 per task in the debug trace
+constexpr int kMaxExperts = 512;         // routed experts per MoE layer (scores fit the
+                                         // residual-row buffer for the top-k)
+constexpr int kMaxTopK = 32;
 constexpr int kDefaultPrefetchKB = 0;    // next-task L2 prefetch: opt-in (measured 4% slower)
 constexpr int kMaxStageBytes = 65536;
 constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per block
@@ -49,17 +52,26 @@ enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1 };
 
 // GEMV ops: which matrix, which input vector, which epilogue.
 enum GemvOp : uint8_t {
-  OP_QKV = 0,   // in: RMSNorm(x; attn_norm)  -> qkv = [Wq; Wk; Wv] xn  (rows of the stacked matrix)
-  OP_O = 1,     // in: attn                   -> h1 = x + Wo attn
-  OP_GU = 2,    // in: RMSNorm(h1; ffn_norm)  -> u = silu(Wg hn) * (Wu hn)   (2 segments)
-  OP_DOWN = 3,  // in: u                      -> x = h1 + Wd u
-  OP_LM = 4,    // in: RMSNorm(x; final_norm) -> logits, greedy argmax
-  OP_COUNT = 5
+  OP_QKV = 0,     // in: RMSNorm(x; attn_norm)  -> qkv = [Wq; Wk; Wv] xn  (rows of the stacked matrix)
+  OP_O = 1,       // in: attn                   -> h1 = x + Wo attn
+  OP_GU = 2,      // in: RMSNorm(h1; ffn_norm)  -> u = silu(Wg hn) * (Wu hn)   (2 segments)
+  OP_DOWN = 3,    // in: u                      -> x = h1 + Wd u
+  OP_LM = 4,      // in: RMSNorm(x; final_norm) -> logits, greedy argmax
+  OP_ROUTER = 5,  // in: hn                     -> scores = sigmoid(Wr hn); last task: top-k
+  OP_SGU = 6,     // in: hn                     -> u[0, Fs) = shared expert silu(g) * u
+  OP_RGU = 7,     // in: hn                     -> u[Fs + j Fe + r] = w_j silu(g) * u of the
+                  //                               j-th selected expert (virtual row j Fe + r)
+  OP_MDOWN = 8,   // in: u                      -> x = h1 + sum over K-parts (one per shared
+                  //                               expert slice and per selected expert)
+  OP_COUNT = 9
 };
 
 // Dependency counters: one per (layer, stage of the layer), then the LM head and a
 // counter nothing ever bumps (used only by the fault-injection debug plan).
-enum CounterKind { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, C_PER_LAYER = 5 };
+// C_ROUTE (MoE) is bumped once per step by the router task that finishes last, after it
+// has written the layer's selected experts and weights.
+enum CounterKind { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, C_ROUTE = 5,
+                   C_PER_LAYER = 6 };
 
 struct Task {          // 32 bytes, 16-byte aligned array
   uint8_t type;        // TaskType
@@ -69,7 +81,7 @@ struct Task {          // 32 bytes, 16-byte aligned array
   uint32_t dep_count;  // increments of `dep` per step
   int32_t out;         // counter to bump when done, -1 = none
   int32_t r0, r1;      // GEMV: output rows [r0, r1).  ATTN: kv head, split index
-  int32_t aux;         // ATTN: number of splits.  LM: number of LM tasks.
+  int32_t aux;         // ATTN: number of splits.  LM / ROUTER: number of tasks of the op.
                        // other GEMV: K-part index | (number of K-parts << 8)
   int32_t id;          // global task index (trace rows, error detail)
 };
@@ -83,7 +95,10 @@ struct LayerPtrs {     // device-side per-layer pointer table
 
 // ---- the plan (host side) -----------------------------------------------------------
 struct PlanShape {
+  int kind;
   int d, Hq, Hkv, D, F, V, L, cap, M;
+  int E, topk, nshared, Fe;  // MoE: experts, selected per token, shared, expert FFN
+  int u_floats;        // the SwiGLU activation buffer (MoE: shared then routed slices)
   int nsm;
   int stage_bytes, ring_stages;
   int kv_splits, pos_per_stage;
@@ -115,7 +130,11 @@ struct Params {
   float* h1;                       // after attention [d]
   float* qkv;                      // [(Hq + 2 Hkv) D]
   float* attn;                     // [Hq D]
-  float* u;                        // [F]
+  float* u;                        // [F] (MoE: [nshared Fe + topk Fe])
+  float* scores;                   // MoE router scores [E]
+  int32_t* route_idx;              // MoE selected experts [L][topk]
+  float* route_w;                  // MoE normalised weights [L][topk]
+  uint32_t* router_ticket;         // MoE: arrival ticket of the router tasks
   float* part;                     // [Hq][splits][D + 2]
   float* logits;                   // [V]
   int32_t* token_out;              // [1] or NULL
@@ -126,6 +145,7 @@ struct Params {
   volatile int32_t* abort_flag;    // device word
   volatile int32_t* status_host;   // host-mapped [2]: code, detail
   int d, Hq, Hkv, D, F, V, L, cap;
+  int E, topk, nshared, Fe;
   int nsplit, pps, stage_bytes, ring_stages, xs_floats, ub_floats;
   float eps;
   int token, pos;

@@ -13,7 +13,8 @@ from collections import defaultdict
 
 import numpy as np
 
-OP_NAMES = {0: "qkv", 1: "o_proj", 2: "gate_up", 3: "down", 4: "lm_head"}
+OP_NAMES = {0: "qkv", 1: "o_proj", 2: "gate_up", 3: "down", 4: "lm_head", 5: "router",
+            6: "shared_gate_up", 7: "routed_gate_up", 8: "moe_down"}
 
 
 def task_table(tasks: np.ndarray) -> dict:

@@ -31,6 +31,9 @@ TRE_W_SLOTS = 16
 TRACE_COLS = 8
 GQA_SLOTS = {"attn_norm": 0, "wq": 1, "wk": 2, "wv": 3, "wo": 4, "ffn_norm": 5, "wgate": 6,
              "wup": 7, "wdown": 8}
+MOE_SLOTS = {"attn_norm": 0, "wq": 1, "wk": 2, "wv": 3, "wo": 4, "ffn_norm": 5, "router": 6,
+             "shared_gate": 7, "shared_up": 8, "shared_down": 9, "expert_gate": 10,
+             "expert_up": 11, "expert_down": 12}
 
 STATUS_NAMES = {0: "TRE_OK", -1: "TRE_ERR_INVALID_ARG", -2: "TRE_ERR_CUDA",
                 -3: "TRE_ERR_OCCUPANCY", -4: "TRE_ERR_DEP_TIMEOUT", -5: "TRE_ERR_POS_RANGE",
@@ -65,7 +68,7 @@ class tre_plan_info(ctypes.Structure):
 
 
 EXPORTED = ("tre_create", "tre_destroy", "tre_decode_step", "tre_decode_step_host",
-            "tre_decode_step_static",
+            "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
             "tre_get_status", "tre_reset", "tre_debug_hidden", "tre_debug_trace",
             "tre_step_bytes", "tre_plan_inspect", "tre_plan_tasks", "tre_last_error")
 
@@ -84,6 +87,8 @@ def _load() -> ctypes.CDLL:
     L.tre_decode_step_host.argtypes = [vp, i32, i32, vp, vp, vp]
     L.tre_decode_step_static.argtypes = [ctypes.POINTER(tre_config), ctypes.POINTER(tre_weights),
                                          i32, i32, vp, vp, vp, vp]
+    L.tre_layers_step.argtypes = [vp, vp, vp, i32, vp]
+    L.tre_debug_routing.argtypes = [vp, vp, vp]
     L.tre_get_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.tre_reset.argtypes = [vp, vp]
     L.tre_debug_hidden.argtypes = [vp, vp, vp]
@@ -96,7 +101,8 @@ def _load() -> ctypes.CDLL:
     L.tre_last_error.argtypes = []
     L.tre_last_error.restype = ctypes.c_char_p
     for name in ("tre_create", "tre_decode_step", "tre_decode_step_host",
-                 "tre_decode_step_static", "tre_get_status",
+                 "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
+                 "tre_get_status",
                  "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
                  "tre_plan_inspect"):
         getattr(L, name).restype = ctypes.c_int
@@ -157,6 +163,20 @@ def tre_decode_step_static(cfg: tre_config, weights: tre_weights, token: int, po
                                       ctypes.c_void_p(logits_dev or None),
                                       ctypes.c_void_p(token_dev or None),
                                       ctypes.c_void_p(status_dev or None))
+
+
+def tre_layers_step(h, x_in_dev: int, x_out_dev: int, pos: int, stream: int = 0) -> int:
+    return lib.tre_layers_step(h, ctypes.c_void_p(x_in_dev or None), ctypes.c_void_p(x_out_dev or None),
+                               int(pos), ctypes.c_void_p(stream or None))
+
+
+def tre_debug_routing(h, n_layers: int, top_k: int):
+    """(idx int32[L][top_k], w float32[L][top_k]) of the last step of a MoE engine."""
+    idx = np.zeros((n_layers, top_k), dtype=np.int32)
+    w = np.zeros((n_layers, top_k), dtype=np.float32)
+    check(lib.tre_debug_routing(h, idx.ctypes.data_as(ctypes.c_void_p),
+                                w.ctypes.data_as(ctypes.c_void_p)), "tre_debug_routing")
+    return idx, w
 
 
 def tre_get_status(h):
@@ -235,6 +255,34 @@ def upload_gqa_model(model: dict, device="cuda:0") -> dict:
     return out
 
 
+def upload_moe_model(wl, model: dict, device="cuda:0", expert_fn=None) -> dict:
+    """Copy a host MoE model to device tensors: the non-expert slots as they are, and the
+    routed experts of every layer stacked expert-major into slots 10-12 ([E][Fe][d] gate
+    and up, [E][d][Fe] down).  `expert_fn(layer, e)` returns an expert's host tensors
+    (default: the workload's generator, one expert at a time)."""
+    import torch
+    from .synth import workloads as W
+    expert_fn = expert_fn or (lambda l, e: W.gen_expert(wl, l, e))
+    E, Fe, d = wl.n_experts, wl.expert_ffn, wl.hidden
+    out = {"layers": [], "k_cache": [], "v_cache": []}
+    for l, layer in enumerate(model["layers"]):
+        dev = {slot: _dev_tensor(a, device) for slot, a in layer.items()
+               if not (slot in (7, 8, 9) and a.size == 0)}
+        g = torch.empty((E, Fe, d), dtype=torch.bfloat16, device=device)
+        u = torch.empty((E, Fe, d), dtype=torch.bfloat16, device=device)
+        dn = torch.empty((E, d, Fe), dtype=torch.bfloat16, device=device)
+        for e in range(E):
+            eg, eu, ed = expert_fn(l, e)
+            g[e].copy_(torch.from_numpy(eg.view(np.int16)).view(torch.bfloat16))
+            u[e].copy_(torch.from_numpy(eu.view(np.int16)).view(torch.bfloat16))
+            dn[e].copy_(torch.from_numpy(ed.view(np.int16)).view(torch.bfloat16))
+        dev[10], dev[11], dev[12] = g, u, dn
+        out["layers"].append(dev)
+        out["k_cache"].append(_dev_tensor(model["k_cache"][l], device))
+        out["v_cache"].append(_dev_tensor(model["v_cache"][l], device))
+    return out
+
+
 def make_weights(cfg: tre_config, dev_model: dict):
     """A tre_weights struct over the device tensors of `dev_model`.  Returns (weights,
     keepalive): keep `keepalive` referenced while the struct is in use."""
@@ -303,6 +351,15 @@ class Engine:
         import torch
         s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
         return tre_decode_step_host(self.h, token, pos, s, logits_host)
+
+    def layers_step(self, x_in, x_out, pos: int, stream=None) -> None:
+        """Enqueue one layers-only step: x_out = stack(x_in) (device fp32[hidden] tensors)."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        check(tre_layers_step(self.h, x_in.data_ptr(), x_out.data_ptr(), pos, s), "tre_layers_step")
+
+    def routing(self):
+        return tre_debug_routing(self.h, self.cfg.n_layers, self.cfg.top_k)
 
     def status(self):
         return tre_get_status(self.h)

@@ -16,8 +16,9 @@ build.build_engine()
 from persistent_tile_pipelined_b200 import tre  # noqa: E402
 
 T_GEMV, T_ATTN = 0, 1
-OP_QKV, OP_O, OP_GU, OP_DOWN, OP_LM = range(5)
-C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_PER_LAYER = range(6)
+OP_QKV, OP_O, OP_GU, OP_DOWN, OP_LM, OP_ROUTER, OP_SGU, OP_RGU, OP_MDOWN = range(9)
+C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_ROUTE, C_PER_LAYER = range(7)
+WHOLE_ROW_OPS = (OP_LM, OP_ROUTER)   # aux holds the op's task count, not K-parts
 
 
 def declared_functions():
@@ -48,11 +49,31 @@ def decode_tasks(tasks):
     }
 
 
+MOE_SMALL = W.MOE4.replace(name="moe-small", n_layers=2, hidden=512, n_q_heads=8, n_kv_heads=2,
+                          head_dim=64, prefill=40, n_experts=12, top_k=3, n_shared=1,
+                          expert_ffn=200)
 PLAN_CASES = [
     (W.TINY, 148), (W.TINY, 7), (W.LLAMA8B, 148), (W.LLAMA8B, 132),
     (W.TINY.replace(n_q_heads=8, n_kv_heads=1, ffn=696, vocab=1001), 148),
     (W.TINY.replace(n_q_heads=4, n_kv_heads=4, head_dim=128, vocab=77), 33),
+    (W.MOE4, 148), (MOE_SMALL, 148), (MOE_SMALL, 5),
+    (MOE_SMALL.replace(n_shared=0, top_k=1), 19), (MOE_SMALL.replace(n_shared=2), 64),
 ]
+
+
+def rows_of_ops(wl):
+    """Output rows of every GEMV op of one layer."""
+    rows = {OP_QKV: (wl.n_q_heads + 2 * wl.n_kv_heads) * wl.head_dim, OP_O: wl.hidden}
+    if wl.kind == "moe":
+        rows.update({OP_ROUTER: wl.n_experts, OP_RGU: wl.top_k * wl.expert_ffn,
+                     OP_MDOWN: wl.hidden})
+        if wl.n_shared:
+            rows[OP_SGU] = wl.n_shared * wl.expert_ffn
+    else:
+        rows.update({OP_GU: wl.ffn, OP_DOWN: wl.hidden})
+    if wl.vocab:
+        rows[OP_LM] = wl.vocab
+    return rows
 
 
 @pytest.mark.parametrize("wl,nsm", PLAN_CASES, ids=lambda x: getattr(x, "name", str(x)))
@@ -85,16 +106,32 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
         if T["type"][i] == T_GEMV and T["op"][i] == OP_O:
             # the attention counter is bumped once per kv head (by the combining split)
             assert T["dep_count"][i] == wl.n_kv_heads
+        elif kind == C_ROUTE and dep < wl.n_layers * C_PER_LAYER:
+            # the route counter is bumped once, by the router task that finishes last
+            assert T["dep_count"][i] == 1
+            assert producers and all(T["op"][j] == OP_ROUTER for j in producers)
         else:
             assert T["dep_count"][i] == len(producers), (i, dep, kind)
     # every GEMV op's output rows are partitioned exactly once per layer
-    rows_of = {OP_QKV: (wl.n_q_heads + 2 * wl.n_kv_heads) * wl.head_dim, OP_O: wl.hidden,
-               OP_GU: wl.ffn, OP_DOWN: wl.hidden, OP_LM: wl.vocab}
-    part = np.where(T["op"] == OP_LM, 0, T["aux"] & 0xFF)
-    nparts = np.where(T["op"] == OP_LM, 1, T["aux"] >> 8)
+    rows_of = rows_of_ops(wl)
+    whole = np.isin(T["op"], WHOLE_ROW_OPS)
+    part = np.where(whole, 0, T["aux"] & 0xFF)
+    nparts = np.where(whole, 1, T["aux"] >> 8)
     gemv = T["type"] == T_GEMV
     # only the last K-part of a row range publishes
     assert ((T["out"][gemv] >= 0) == (part[gemv] == nparts[gemv] - 1)).all()
+    if wl.kind == "moe":
+        # one K-part per shared-expert slice and per selected expert
+        md = gemv & (T["op"] == OP_MDOWN)
+        assert (nparts[md] == wl.n_shared + wl.top_k).all()
+        # routed gate/up tasks never straddle two experts; routed work waits for the route
+        rg = np.flatnonzero(gemv & (T["op"] == OP_RGU))
+        for i in rg:
+            assert T["r0"][i] // wl.expert_ffn == (T["r1"][i] - 1) // wl.expert_ffn
+            assert T["dep"][i] % C_PER_LAYER == C_ROUTE
+        for l in range(wl.n_layers):
+            ro = gemv & (T["op"] == OP_ROUTER) & (T["layer"] == l)
+            assert (T["aux"][ro] == ro.sum()).all()
     for l in range(wl.n_layers):
         for op, N in rows_of.items():
             if op == OP_LM and l != wl.n_layers - 1:
@@ -133,6 +170,7 @@ def test_llama8b_plan_is_byte_balanced():
 
 @pytest.mark.parametrize("field,value,status", [
     ("kind", 1, tre.TRE_ERR_UNSUPPORTED), ("kind", 9, tre.TRE_ERR_INVALID_ARG),
+    ("kind", 2, tre.TRE_ERR_UNSUPPORTED),      # MoE with n_experts = 0 (a GQA config)
     ("hidden", 260, tre.TRE_ERR_INVALID_ARG), ("n_kv_heads", 3, tre.TRE_ERR_INVALID_ARG),
     ("head_dim", 96, tre.TRE_ERR_UNSUPPORTED), ("ffn", 690, tre.TRE_ERR_INVALID_ARG),
     ("kv_capacity", 0, tre.TRE_ERR_INVALID_ARG), ("max_tokens_per_step", 4, tre.TRE_ERR_UNSUPPORTED),
@@ -144,6 +182,29 @@ def test_plan_rejects_bad_configs(field, value, status):
     import ctypes
     assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status
     assert tre.lib.tre_last_error()
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("n_experts", 513, tre.TRE_ERR_UNSUPPORTED), ("top_k", 13, tre.TRE_ERR_INVALID_ARG),
+    ("top_k", 0, tre.TRE_ERR_INVALID_ARG), ("n_shared", -1, tre.TRE_ERR_INVALID_ARG),
+    ("expert_ffn", 100, tre.TRE_ERR_INVALID_ARG),
+])
+def test_moe_plan_rejects_bad_configs(field, value, status):
+    import ctypes
+    cfg = tre.config_from_workload(MOE_SMALL, **{field: value})
+    info = tre.tre_plan_info()
+    assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status
+
+
+def test_moe_plan_streams_only_the_selected_experts():
+    wl = W.MOE4
+    info = tre.tre_plan_inspect(tre.config_from_workload(wl))
+    d, dh = wl.hidden, wl.head_dim
+    attn = (wl.n_q_heads + 2 * wl.n_kv_heads) * dh * d + d * wl.n_q_heads * dh
+    mlp = wl.n_experts * d + 3 * (wl.n_shared + wl.top_k) * wl.expert_ffn * d
+    assert info.weight_bytes == wl.n_layers * ((attn + mlp) * 2 + 2 * d * 2)
+    assert info.weight_bytes == pytest.approx(4 * 1.061e9, rel=0.01)
+    assert info.max_sm_bytes <= 1.02 * info.min_sm_bytes
 
 
 def test_reserved_fields_must_be_zero():

@@ -1,0 +1,160 @@
+"""GPU parity of MoE decoder layers (GQA attention + routed experts) through the C ABI's
+layers-only step, against the fp64 CPU oracle.
+
+Bar: max relative error 2e-2 (normwise, max|gpu - oracle| / max|oracle|) on the hidden
+state after every layer, and the same selected experts in the same order.  The routing is
+an integer decision taken from floating-point scores: the GPU takes it in fp32, the oracle
+in fp64, so each case first checks that the oracle's score gap at the selection boundary
+(between the k-th and (k+1)-th expert, and between consecutive selected experts) is far
+above fp32 rounding of the scores (1e-5); then the expert ids must be equal exactly and the
+weights within 1e-4.  Each step feeds both sides the oracle's previous output.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from persistent_tile_pipelined_b200.synth import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from persistent_tile_pipelined_b200 import tre  # noqa: E402
+
+TOL = 2e-2
+ORC = oracle.Oracle(64)
+MARGIN = 1e-5
+
+SMALL = W.MOE4.replace(name="moe-small", n_layers=2, hidden=512, n_q_heads=8, n_kv_heads=2,
+                       head_dim=64, prefill=40, decode_steps=3, n_experts=12, top_k=3,
+                       n_shared=1, expert_ffn=200, seed=2024)
+
+
+def relerr(g, o):
+    g, o = np.asarray(g, np.float64), np.asarray(o, np.float64)
+    return float(np.abs(g - o).max() / max(np.abs(o).max(), 1e-30))
+
+
+def check_margin(scores, k):
+    s = np.sort(np.asarray(scores, np.float64))[::-1]
+    gaps = -np.diff(s[: min(k + 1, len(s))])
+    assert gaps.size == 0 or gaps.min() > MARGIN, f"routing near-tie (gap {gaps.min():.3g})"
+
+
+def run_moe(wl, steps=1, **cfg_over):
+    model = W.gen_moe_model(wl, with_experts=True)
+    ex = model["experts"]
+    dev = tre.upload_moe_model(wl, model, expert_fn=lambda l, e: ex[l][e])
+    cfg = tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_HIDDEN, **cfg_over)
+    eng = tre.Engine(cfg, dev)
+    kc = [c.copy() for c in model["k_cache"]]
+    vc = [c.copy() for c in model["v_cache"]]
+    x = model["x_in"].astype(np.float64)
+    x_dev = torch.empty(wl.hidden, dtype=torch.float32, device="cuda")
+    out_dev = torch.empty(wl.hidden, dtype=torch.float32, device="cuda")
+    worst = 0.0
+    for step in range(steps):
+        pos = wl.prefill + step
+        x_dev.copy_(torch.from_numpy(x.astype(np.float32)))
+        eng.layers_step(x_dev, out_dev, pos)
+        torch.cuda.synchronize()
+        assert eng.status() == (0, 0)
+        hid = eng.hidden().cpu().numpy()
+        gidx, gw = eng.routing()
+        h = x
+        for l in range(wl.n_layers):
+            h, idx, w, sc = ORC.moe_layer_step(wl, model["layers"][l], kc[l], vc[l],
+                                               lambda e, l=l: ex[l][e], pos, h, want_scores=True)
+            check_margin(sc, wl.top_k)
+            assert gidx[l].tolist() == list(idx), f"layer {l} routing {gidx[l]} vs {idx}"
+            np.testing.assert_allclose(gw[l], w, rtol=1e-4, atol=1e-6)
+            e = relerr(hid[l], h)
+            worst = max(worst, e)
+            assert e <= TOL, f"layer {l} hidden rel err {e:.3g} at pos {pos}"
+        g_out = out_dev.cpu().numpy()
+        assert np.array_equal(g_out, hid[-1]), "x_out differs from the last layer's hidden"
+        x = h
+    # appended KV rows: within one bf16 ulp of the row's largest entry (fp32 vs fp64
+    # rounding to bf16); rows before the first step untouched
+    for l in range(wl.n_layers):
+        for name, ref in (("k_cache", kc), ("v_cache", vc)):
+            gw_ = dev[name][l].view(torch.int16).cpu().numpy().view(np.uint16)
+            ow = ref[l]
+            start, end = wl.prefill, wl.prefill + steps
+            assert np.array_equal(gw_[:, :start], ow[:, :start])
+            gv = (gw_[:, start:end].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            ov = (ow[:, start:end].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            row_max = np.abs(ov).max(axis=-1, keepdims=True)
+            assert not (np.abs(gv - ov) > 2.0 ** -8 * row_max).any()
+    eng.close()
+    return worst
+
+
+@pytest.mark.parametrize("over,steps", [
+    (dict(), 3),                                                       # E 12, top 3, Fe 200
+    (dict(hidden=1024, n_q_heads=16, n_kv_heads=2, head_dim=128, n_experts=40, top_k=8,
+          expert_ffn=256, n_layers=1), 2),                             # G 8, D 128, top 8
+    (dict(n_shared=0, top_k=1), 2),                                    # routed expert only
+    (dict(n_shared=2, expert_ffn=64), 2),                              # strided shared parts
+    (dict(hidden=256, n_q_heads=4, n_kv_heads=2, n_experts=300, top_k=32, expert_ffn=48,
+          n_layers=1), 1),                                             # E > 256, top 32
+    (dict(prefill=0, decode_steps=2), 2),                              # pos 0
+], ids=["e12-k3", "e40-k8-d1024", "no-shared-k1", "two-shared", "e300-k32", "pos0"])
+def test_moe_layers(over, steps):
+    run_moe(SMALL.replace(**over), steps=steps)
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(num_sms=5),
+    dict(num_sms=3, ring_stages=2, stage_bytes=8192),
+    dict(kv_splits=1),
+], ids=["sms5", "sms3-ring2-8k", "split1"])
+def test_moe_launch_shapes(cfg):
+    run_moe(SMALL, steps=2, **cfg)
+
+
+def test_moe_layers_step_argument_errors():
+    wl = SMALL.replace(n_layers=1)
+    model = W.gen_moe_model(wl, with_experts=True)
+    ex = model["experts"]
+    dev = tre.upload_moe_model(wl, model, expert_fn=lambda l, e: ex[l][e])
+    eng = tre.Engine(tre.config_from_workload(wl), dev)
+    x = torch.zeros(wl.hidden, dtype=torch.float32, device="cuda")
+    y = torch.zeros(wl.hidden, dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert tre.tre_layers_step(eng.h, x.data_ptr(), x.data_ptr(), wl.prefill, s) == tre.TRE_ERR_INVALID_ARG
+    assert tre.tre_layers_step(eng.h, x.data_ptr(), y.data_ptr(), wl.kv_capacity, s) == tre.TRE_ERR_POS_RANGE
+    assert tre.tre_layers_step(eng.h, x.data_ptr() + 4, y.data_ptr(), wl.prefill, s) == tre.TRE_ERR_INVALID_ARG
+    assert tre.tre_decode_step(eng.h, 0, wl.prefill, s) == tre.TRE_ERR_UNSUPPORTED
+    eng.close()
+
+
+@pytest.mark.slow
+def test_moe_full_size_four_layers():
+    """The full MoE workload: hidden 7168, 256 experts (top 8 + 1 shared, Fe 2048), GQA 64/8
+    heads of dim 128 over 4096 cached positions, 4 layers (~92 GB resident)."""
+    wl = W.MOE4
+    model = W.gen_moe_model(wl)
+    dev = tre.upload_moe_model(wl, model)
+    eng = tre.Engine(tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_HIDDEN), dev)
+    x = model["x_in"].astype(np.float64)
+    x_dev = torch.from_numpy(x.astype(np.float32)).cuda()
+    out_dev = torch.empty_like(x_dev)
+    eng.layers_step(x_dev, out_dev, wl.prefill)
+    torch.cuda.synchronize()
+    assert eng.status() == (0, 0)
+    hid = eng.hidden().cpu().numpy()
+    gidx, gw = eng.routing()
+    h = x
+    for l in range(wl.n_layers):
+        kc, vc = model["k_cache"][l].copy(), model["v_cache"][l].copy()
+        h, idx, w, sc = ORC.moe_layer_step(wl, model["layers"][l], kc, vc,
+                                           lambda e, l=l: W.gen_expert(wl, l, e), wl.prefill, h,
+                                           want_scores=True)
+        check_margin(sc, wl.top_k)
+        assert gidx[l].tolist() == list(idx)
+        np.testing.assert_allclose(gw[l], w, rtol=1e-4, atol=1e-6)
+        assert relerr(hid[l], h) <= TOL
+    eng.close()
