@@ -150,6 +150,9 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   if (t.op == OP_LM || t.op == OP_ROUTER) {
     g.np = 1;
     g.part = 0;
+  } else if (t.op == OP_MDOWN) {  // aux = slot | block << 8
+    g.part = t.aux & 0xff;
+    g.np = p.nshared + p.topk;
   } else {
     g.part = t.aux & 0xff;
     g.np = max(1, t.aux >> 8);
@@ -715,7 +718,7 @@ __device__ __forceinline__ void prefetch_resid(const Params& p, const Task& t, c
     const int n = t.r0 + r;
     float v;
     if (t.op == OP_O) v = g.part == 0 ? resid_in(p, t.layer, n) : __ldcg(p.h1 + n);
-    else v = g.part == 0 ? __ldcg(p.h1 + n) : __ldcg(p.x + n);  // down / MoE down
+    else v = g.part == 0 ? __ldcg(p.h1 + n) : __ldcg(p.x + n);
     resid[r] = v;
   }
 }
@@ -726,8 +729,8 @@ __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const 
     case OP_QKV: p.qkv[n] = v * rn; break;
     case OP_O: p.h1[n] = resid[n - t.r0] + v; break;
     case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
-    case OP_DOWN:
-    case OP_MDOWN: {
+    case OP_MDOWN: p.mpart[(size_t)g.part * p.d + n] = v; break;
+    case OP_DOWN: {
       const float y = resid[n - t.r0] + v;
       p.x[n] = y;
       if (g.part == g.np - 1) {
@@ -780,6 +783,22 @@ __device__ void route_topk(const Params& p, int layer, float* sc, int warp, int 
   if (lane == 0) red_release_gpu_add(p.counters + layer * C_PER_LAYER + C_ROUTE, 1u);
 }
 
+// The last slot of a MoE-down row block to finish: x = h1 + sum of the slots' partial rows
+// in slot order (deterministic), then the block is published.
+__device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
+  const int np = p.nshared + p.topk;
+  for (int n = t.r0 + ctid; n < t.r1; n += kConsumerThreads) {
+    float y = __ldcg(p.h1 + n);
+    for (int j = 0; j < np; ++j) y += __ldcg(p.mpart + (size_t)j * p.d + n);
+    p.x[n] = y;
+    if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
+    if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
+  }
+  __threadfence();
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) red_release_gpu_add(p.counters + t.out, 1u);
+}
+
 // ---- consumers -----------------------------------------------------------------------------------
 __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
@@ -816,7 +835,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       const GemvGeom g = gemv_geom(p, t);
       const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
-      const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MDOWN;
+      const bool has_resid = t.op == OP_O || t.op == OP_DOWN;
       if (has_resid) prefetch_resid(p, t, g, resid, ctid);
       if (key != cur_key) {
         const float rn = load_input(p, t, g, ub, red, ctid);
@@ -918,6 +937,13 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         consumer_sync(kConsumerThreads);
         if (flags[1]) route_topk(p, t.layer, ub + p.xs_floats, warp, lane, ctid);
+      } else if (t.op == OP_MDOWN) {  // the block's last slot sums the partial rows
+        if (ctid == 0) {
+          const uint32_t old = atom_acq_rel_gpu_add(p.down_tickets + (t.aux >> 8), 1u);
+          flags[1] = ((old + 1u) % (uint32_t)(p.nshared + p.topk)) == 0u;
+        }
+        consumer_sync(kConsumerThreads);
+        if (flags[1]) moe_down_combine(p, t, ctid);
       } else if (ctid == 0 && t.out >= 0) {
         red_release_gpu_add(p.counters + t.out, 1u);
       }

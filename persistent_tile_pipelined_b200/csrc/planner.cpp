@@ -6,11 +6,12 @@
 // an engine that maps tasks onto hardware units (Speed is intelligence talk, section on
 // breaking the kernel boundary).  This planner is that step for one GPU:
 //
-//   * every GEMV op (Q, K, V, O, gate/up, down, LM head) is cut into one contiguous row
-//     range per SM; ranges are sized so that each SM's cumulative streamed bytes over
-//     the step stay level (the SMs then finish every op at about the same time);
-//   * the attention of each layer is cut into (kv head, KV split) tasks, placed on the
-//     SMs with the least streamed bytes so far;
+//   * every GEMV op (Q, K, V, O, gate/up, down, LM head, MoE router and experts) is cut
+//     into one contiguous row range per SM of equal size (the SMs then finish the op
+//     together: every op ends at a dependency the next one waits for);
+//   * the attention of each layer is cut into (kv head, KV split) tasks, and the MoE down
+//     into (expert slot, row block) tasks, dealt round robin to the SMs (at most one more
+//     on any SM than on another; the extras to the SMs with the least streamed bytes);
 //   * each task waits on one counter (the op it reads from, all of its tasks) and bumps
 //     one counter; counters only grow, so step e waits for e * count;
 //   * each SM's queue is in global topological order, so with every CTA resident the
@@ -36,34 +37,18 @@ static tre_status fail(tre_status s, const std::string& m) {
 
 static inline int counter_of(int layer, int kind) { return layer * C_PER_LAYER + kind; }
 
-// Split N rows of `row_bytes` each over the SMs, levelling cumulative bytes `cum`.
+// Split N rows of `row_bytes` each over the SMs: every SM gets floor(N / n) rows and the
+// remainder goes one row each to the SMs with the least streamed bytes so far.  Each op
+// ends at a dependency every later op waits for, so it is the op's own balance that sets
+// its time; `cum` (cumulative bytes) only breaks ties.
 static std::vector<std::pair<int, int>> assign_rows(int N, int64_t row_bytes,
                                                     std::vector<int64_t>& cum) {
   const int n = (int)cum.size();
-  double total = (double)N * (double)row_bytes;
-  for (int64_t c : cum) total += (double)c;
-  const double target = total / n;
-  std::vector<double> want(n);
-  double sw = 0;
-  for (int i = 0; i < n; ++i) {
-    want[i] = std::max(0.0, (target - (double)cum[i]) / (double)row_bytes);
-    sw += want[i];
-  }
-  for (int i = 0; i < n; ++i) want[i] = sw > 0 ? want[i] * N / sw : (double)N / n;
-  std::vector<int> rows(n);
-  int s = 0;
-  for (int i = 0; i < n; ++i) {
-    rows[i] = (int)std::floor(want[i]);
-    s += rows[i];
-  }
+  std::vector<int> rows(n, N / n);
   std::vector<int> idx(n);
   std::iota(idx.begin(), idx.end(), 0);
-  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) {
-    double fa = want[a] - rows[a], fb = want[b] - rows[b];
-    if (fa != fb) return fa > fb;
-    return cum[a] < cum[b];
-  });
-  for (int k = 0; s < N; ++k, ++s) rows[idx[k % n]]++;
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cum[a] < cum[b]; });
+  for (int k = 0; k < N % n; ++k) rows[idx[k]]++;
   std::vector<std::pair<int, int>> ranges(n);
   int r = 0;
   for (int i = 0; i < n; ++i) {
@@ -122,6 +107,17 @@ struct Builder {
     return n;
   }
 
+  // SMs for `count` equal tasks of one op: every SM takes floor or ceil(count / nsm) of
+  // them (round robin), in order of the least streamed bytes so far.
+  std::vector<int> spread(int count) const {
+    std::vector<int> idx(nsm);
+    std::iota(idx.begin(), idx.end(), 0);
+    std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cum[a] < cum[b]; });
+    std::vector<int> out(count);
+    for (int k = 0; k < count; ++k) out[k] = idx[k % nsm];
+    return out;
+  }
+
   // Set aux = count on every task of `op` created since task id `first`.
   void set_count(int first, uint8_t op, int count) {
     for (auto& qq : q)
@@ -129,11 +125,31 @@ struct Builder {
         if (t.id >= first && t.type == T_GEMV && t.op == op) t.aux = count;
   }
 
+  // MoE down: np slots x nb row blocks of d rows, each placed on the SM with the least
+  // streamed bytes so far; aux = slot | block << 8.  Returns nb (one bump per block).
+  int moe_down(int layer, int d, int np, int Fe, int nb, int dep, uint32_t dep_count, int out) {
+    const std::vector<int> sms = spread(np * nb);
+    for (int bl = 0; bl < nb; ++bl) {
+      const int r0 = (int)((int64_t)d * bl / nb), r1 = (int)((int64_t)d * (bl + 1) / nb);
+      for (int j = 0; j < np; ++j) {
+        const int best = sms[bl * np + j];
+        Task t = make(T_GEMV, OP_MDOWN, layer, dep, dep_count, out);
+        t.r0 = r0;
+        t.r1 = r1;
+        t.aux = j | (bl << 8);
+        q[best].push_back(t);
+        cum[best] += (int64_t)(r1 - r0) * Fe * 2;
+      }
+    }
+    return nb;
+  }
+
   void attention(int layer, int Hkv, int S, int64_t bytes_per_task, int dep, uint32_t dep_count,
                  int out) {
+    const std::vector<int> sms = spread(Hkv * S);
     for (int g = 0; g < Hkv; ++g)
       for (int s = 0; s < S; ++s) {
-        int best = (int)(std::min_element(cum.begin(), cum.end()) - cum.begin());
+        const int best = sms[g * S + s];
         Task t = make(T_ATTN, 0, layer, dep, dep_count, out);
         t.r0 = g;
         t.r1 = s;
@@ -219,6 +235,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     s.Fe = c.expert_ffn;
   }
   s.u_floats = moe ? (s.nshared + s.topk) * s.Fe : s.F;
+  // MoE down row blocks: enough (slot, block) tasks to cover the SMs once
+  if (moe) s.down_blocks = std::max(1, std::min(s.d / 8, nsm / (s.nshared + s.topk)));
   const int G = s.Hq / s.Hkv;
 
   // Inputs longer than kMaxKPart are staged in K-parts; ops that normalise their input
@@ -308,9 +326,11 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
       int ng = 0;
       if (s.nshared > 0) ng += b.gemv(OP_SGU, l, s.nshared * s.Fe, s.d, 2, co, (uint32_t)no, cg, big);
       ng += b.gemv(OP_RGU, l, s.topk * s.Fe, s.d, 2, cr, 1u, cg, big, 0, s.Fe);
-      // down: K-parts of Fe inputs, one per shared-expert slice and per selected expert
-      const int np = s.nshared + s.topk;
-      nd = b.gemv(OP_MDOWN, l, s.d, np * s.Fe, 1, cg, (uint32_t)ng, cd, s.resid_floats, np);
+      // down: one task per (expert slot j, row block); slot j reads the j-th Fe-slice of u
+      // (shared slices first, then the selected experts).  Each task writes its partial
+      // rows; the last of a block's slots to finish sums them (fixed slot order) with h1
+      // into x and bumps the down counter once per block.
+      nd = b.moe_down(l, s.d, s.nshared + s.topk, s.Fe, s.down_blocks, cg, (uint32_t)ng, cd);
     }
     prev_down = cd;
     prev_down_count = (uint32_t)nd;

@@ -238,6 +238,8 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_ridx = cv.take<int32_t>(moe ? (size_t)s.L * s.topk : 1);
   size_t o_rw = cv.take<float>(moe ? (size_t)s.L * s.topk : 1);
   size_t o_rtick = cv.take<uint32_t>(1);
+  size_t o_mpart = cv.take<float>(moe ? (size_t)(s.nshared + s.topk) * s.d : 1);
+  size_t o_dtick = cv.take<uint32_t>(moe ? s.down_blocks : 1);
   size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (s.D + 2));
   size_t o_logits = cv.take<float>(s.V > 0 ? s.V : 1);
   size_t o_tok = cv.take<int32_t>(1);
@@ -303,6 +305,8 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.route_idx = reinterpret_cast<int32_t*>(B + o_ridx);
   p.route_w = reinterpret_cast<float*>(B + o_rw);
   p.router_ticket = reinterpret_cast<uint32_t*>(B + o_rtick);
+  p.mpart = reinterpret_cast<float*>(B + o_mpart);
+  p.down_tickets = reinterpret_cast<uint32_t*>(B + o_dtick);
   p.E = s.E; p.topk = s.topk; p.nshared = s.nshared; p.Fe = s.Fe;
   p.part = reinterpret_cast<float*>(B + o_part);
   p.logits = reinterpret_cast<float*>(B + o_logits);
@@ -472,6 +476,8 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
   CK(cudaMemsetAsync(p.tickets, 0, (size_t)e->shape.Hkv * 4, s));
   CK(cudaMemsetAsync(p.lm_ticket, 0, 4, s));
   CK(cudaMemsetAsync(p.router_ticket, 0, 4, s));
+  if (e->shape.kind == TRE_LAYER_MOE)
+    CK(cudaMemsetAsync(p.down_tickets, 0, (size_t)e->shape.down_blocks * 4, s));
   CK(cudaMemsetAsync(p.argmax_slot, 0, 8, s));
   CK(cudaMemsetAsync(p.err, 0, 8, s));  // error word + abort flag
   CK(cudaStreamSynchronize(s));

@@ -61,8 +61,9 @@ enum GemvOp : uint8_t {
   OP_SGU = 6,     // in: hn                     -> u[0, Fs) = shared expert silu(g) * u
   OP_RGU = 7,     // in: hn                     -> u[Fs + j Fe + r] = w_j silu(g) * u of the
                   //                               j-th selected expert (virtual row j Fe + r)
-  OP_MDOWN = 8,   // in: u                      -> x = h1 + sum over K-parts (one per shared
-                  //                               expert slice and per selected expert)
+  OP_MDOWN = 8,   // in: u slice j              -> partial rows of slot j (a shared-expert
+                  //                               slice or a selected expert); the block's
+                  //                               last slot sums x = h1 + sum_j partial_j
   OP_COUNT = 9
 };
 
@@ -99,6 +100,7 @@ struct PlanShape {
   int d, Hq, Hkv, D, F, V, L, cap, M;
   int E, topk, nshared, Fe;  // MoE: experts, selected per token, shared, expert FFN
   int u_floats;        // the SwiGLU activation buffer (MoE: shared then routed slices)
+  int down_blocks;     // MoE down: row blocks (each summed by its last slot to finish)
   int nsm;
   int stage_bytes, ring_stages;
   int kv_splits, pos_per_stage;
@@ -135,6 +137,8 @@ struct Params {
   int32_t* route_idx;              // MoE selected experts [L][topk]
   float* route_w;                  // MoE normalised weights [L][topk]
   uint32_t* router_ticket;         // MoE: arrival ticket of the router tasks
+  float* mpart;                    // MoE down partial rows [nshared + topk][d]
+  uint32_t* down_tickets;          // MoE down: arrival ticket per row block
   float* part;                     // [Hq][splits][D + 2]
   float* logits;                   // [V]
   int32_t* token_out;              // [1] or NULL
