@@ -220,6 +220,28 @@ __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
   return (t1 - t0 + p.pps - 1) / p.pps;
 }
 
+// Where a GEMV task's rows come from, resolved once per task (expert ids and layer
+// pointers are looked up here, not per stage): row n of segment s of the task's K-part
+// starts at base[s] + (n - r0) * stride.  QKV rows cross from Wq into Wk into Wv, so QKV
+// stages are resolved per stage instead (lookup = true).
+struct RowSrc {
+  const uint16_t* base[2];
+  long long stride;   // elements between consecutive rows in memory
+  bool lookup;        // resolve every stage with part_row
+};
+
+__device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const GemvGeom& g) {
+  RowSrc r;
+  r.lookup = t.op == OP_QKV;
+  r.stride = g.K;
+  if (t.op == OP_RGU) r.stride = p.d;
+  else if (t.op == OP_MDOWN) r.stride = g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe;
+  int contig;
+  r.base[0] = r.lookup ? nullptr : part_row(p, t, g, 0, t.r0, &contig);
+  r.base[1] = (r.lookup || g.nseg < 2) ? nullptr : part_row(p, t, g, 1, t.r0, &contig);
+  return r;
+}
+
 // ---- producer -------------------------------------------------------------------------------
 // Bytes of stage i of task t.  GEMV stages are whole rows of the task's K-part (gate/up:
 // the rows of both matrices); attention stages are the K and V rows of up to `pps`
@@ -238,13 +260,26 @@ __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, 
 // segment; gate rows at the stage's start, up rows after `rps` rows), spread over the
 // producer lanes; attention: the K rows then the V rows (lanes 0 and 1).
 __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, const GemvGeom& g,
-                                            int t0, int t1, int i, int lane, uint8_t* dst,
-                                            uint64_t* bar, uint64_t pol) {
+                                            const RowSrc& rs, int t0, int t1, int i, int lane,
+                                            uint8_t* dst, uint64_t* bar, uint64_t pol) {
   if (t.type == T_GEMV) {
     const int n0 = t.r0 + i * g.rps, n1 = min(t.r1, n0 + g.rps);
     const uint32_t rowb = (uint32_t)g.Kp * 2u;
-    // common case: each segment's rows of the stage are one contiguous run (one lookup
-    // per segment, lanes in parallel)
+    if (!rs.lookup) {
+      if (rs.stride == g.Kp) {  // rows adjacent in memory: one copy per segment
+        if (lane < g.nseg)
+          bulk_g2s(dst + (size_t)lane * g.rps * rowb, rs.base[lane] + (n0 - t.r0) * rs.stride,
+                   (uint32_t)(n1 - n0) * rowb, bar, pol);
+      } else {                  // strided rows (K-parts): one copy per row
+        for (int k = lane; k < g.nseg * (n1 - n0); k += 32) {
+          const int seg = k / (n1 - n0), r = k % (n1 - n0);
+          bulk_g2s(dst + (size_t)(seg * g.rps + r) * rowb,
+                   rs.base[seg] + (n0 - t.r0 + r) * rs.stride, rowb, bar, pol);
+        }
+      }
+      return;
+    }
+    // QKV: each segment's rows of the stage in at most three runs
     int contig = 0;
     const uint16_t* w0 = lane < g.nseg ? part_row(p, t, g, lane, n0, &contig) : nullptr;
     if (__all_sync(0xffffffffu, lane >= g.nseg || contig >= n1 - n0)) {
@@ -359,9 +394,14 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
     if (window > 0 && ti + 1 < ntask) task_prefetch(p, my[ti + 1], lane, window);
     const int ns = task_nstages(p, t);
     GemvGeom g{};
+    RowSrc rs{};
     int t0 = 0, t1 = 0;
-    if (t.type == T_GEMV) g = gemv_geom(p, t);
-    else attn_range(p, t, t0, t1);
+    if (t.type == T_GEMV) {
+      g = gemv_geom(p, t);
+      rs = row_src(p, t, g);
+    } else {
+      attn_range(p, t, t0, t1);
+    }
     for (int i = 0; i < ns; ++i, ++gs) {
       const uint32_t slot = gs % NS, ph = (gs / NS) & 1u;
       bool r = true;
@@ -375,7 +415,7 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
         mbar_arrive_expect_tx(&full[slot], stage_total(p, t, g, t0, t1, i));
       }
       __syncwarp();
-      issue_stage(p, t, g, t0, t1, i, lane, ring + (size_t)slot * SB, &full[slot], pol);
+      issue_stage(p, t, g, rs, t0, t1, i, lane, ring + (size_t)slot * SB, &full[slot], pol);
     }
   }
   if (!ok && lane == 0) {
@@ -849,6 +889,13 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       const float4* xl = reinterpret_cast<const float4*>(ub);
       const float4* xh = reinterpret_cast<const float4*>(ub + g.Kp / 2);
       Best best{-INFINITY, 0x7fffffff};
+      // routed experts: the slot's weight folds into u; u holds the shared slices first
+      float wsel = 1.f;
+      int uoff = 0;
+      if (t.op == OP_RGU) {
+        wsel = __ldcg(p.route_w + t.layer * p.topk + t.r0 / p.Fe);
+        uoff = p.nshared * p.Fe;
+      }
       // stage gs + i belongs to warp (gs + i) % 8; each warp takes its stages in order
       const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
       for (int i = first; i < ns; i += kConsumerWarps) {
@@ -861,13 +908,6 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
         if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;
-          // routed experts: the slot's weight folds into u; u holds the shared slices first
-          float wsel = 1.f;
-          int uoff = 0;
-          if (t.op == OP_RGU) {
-            wsel = __ldcg(p.route_w + t.layer * p.topk + t.r0 / p.Fe);
-            uoff = p.nshared * p.Fe;
-          }
           for (int r = 0; r < nr; r += 2) {
             const int np = min(2, nr - r);
             float o0, o1, o2, o3;
