@@ -196,6 +196,8 @@ def build_layers_engine(wl, device: int, debug_flags: int = 0):
     if wl.kind == "moe":
         model = W.gen_moe_model(wl)
         dmodel = tre.upload_moe_model(wl, model, dev)
+    elif wl.kind == "mla":
+        dmodel = tre.upload_mla_model(W.gen_mla_model(wl), dev)
     else:
         raise SystemExit(f"layers-only workload kind {wl.kind!r} is not built")
     torch.cuda.synchronize(device)
@@ -535,6 +537,9 @@ def main_layers(args, rank, world, local_rank):
     if wl.kind == "moe":
         cfg.update(experts=wl.n_experts, top_k=wl.top_k, shared=wl.n_shared,
                    expert_ffn=wl.expert_ffn, kv_heads=wl.n_kv_heads, head_dim=wl.head_dim)
+    if wl.kind == "mla":
+        cfg.update(q_lora=wl.q_lora, kv_lora=wl.kv_lora, rope_dim=wl.rope_dim,
+                   nope_dim=wl.nope_dim, v_dim=wl.v_dim, latent_positions=wl.prefill)
     line = {
         "metric": "layer-stack step time and achieved HBM GB/s over the bytes a token reads",
         "value": world * K / dev_s, "unit": "steps/s", "n_gpus": world, "steps": K,

@@ -67,7 +67,10 @@ typedef enum {
 
 /* Layer kinds.  GQA: Llama-style pre-norm attention + SwiGLU MLP.  MOE: the same
  * attention with a routed mixture-of-experts MLP.  MLA: absorbed multi-head latent
- * attention only (no MLP). */
+ * attention only (pre-norm -> MLA -> residual, no MLP); the pages name the fused MLA
+ * kernel FlashSparseMLA with batch == 1 (TileRT code audit, blog-vs-code table) and fold
+ * query heads into one tile (Speed is intelligence talk, section on the attention
+ * kernel); absorbed MLA is read as DeepSeek-V2's. */
 enum { TRE_LAYER_GQA = 0, TRE_LAYER_MLA = 1, TRE_LAYER_MOE = 2 };
 
 /* debug_flags bits */
@@ -86,12 +89,14 @@ typedef struct {
   int32_t kind;                 /* TRE_LAYER_*  (one kind for the whole stack)          */
   int32_t n_layers;
   int32_t hidden;               /* d                                                    */
-  int32_t n_q_heads;            /* Hq (MLA: heads)                                      */
+  int32_t n_q_heads;            /* Hq (MLA: heads H, a multiple of 16)                  */
   int32_t n_kv_heads;           /* Hkv (GQA/MOE); Hq % Hkv == 0                         */
   int32_t head_dim;             /* D (GQA/MOE): 64 or 128                               */
   int32_t ffn;                  /* F, SwiGLU hidden (GQA)                               */
   int32_t vocab;                /* V (0 when has_embed_lm_head == 0)                    */
-  int32_t q_lora, kv_lora, rope_dim, nope_dim, v_dim;          /* MLA                   */
+  int32_t q_lora, kv_lora, rope_dim, nope_dim, v_dim;          /* MLA: kv_lora a multiple
+                                   of 128, rope_dim of 16, kv_lora + rope_dim of 64 and
+                                   <= 768, q_lora / nope_dim / v_dim of 8               */
   int32_t n_experts, top_k, n_shared, expert_ffn;              /* MOE                   */
   int32_t kv_capacity;          /* positions allocated in each KV cache                 */
   int32_t max_tokens_per_step;  /* M, 1..4                                              */
@@ -119,14 +124,22 @@ typedef struct {
  *         (NULL when n_shared == 0), and the routed experts stacked expert-major:
  *         EXPERT_GATE[E][Fe][d], EXPERT_UP[E][Fe][d], EXPERT_DOWN[E][d][Fe]
  *         (the layout of a fused-MoE weight: expert e's matrix starts at e * Fe * d).
+ *   MLA : ATTN_NORM[d], DQ[QL][d], Q_NORM[QL], UQ[H*(NP+R)][QL] (per head: NP nope rows
+ *         then R rope rows), DKV[KL+R][d] (KL latent rows then R rope rows),
+ *         KV_NORM[KL], UK[H*NP][KL], UV[H*VD][KL], MLA_O[d][H*VD]
+ *         (QL = q_lora, KL = kv_lora, R = rope_dim, NP = nope_dim, VD = v_dim)
  * KV caches (bf16, written at pos by every step, caller owned):
  *   GQA/MOE : k_cache[l], v_cache[l] = [Hkv][kv_capacity][D]
+ *   MLA     : k_cache[l] = latent [kv_capacity][KL + R]: RMSNorm(c_kv) then RoPE(k_pe);
+ *             v_cache unused (may be NULL)
  */
 enum {
   TRE_W_ATTN_NORM = 0, TRE_W_Q = 1, TRE_W_K = 2, TRE_W_V = 3, TRE_W_O = 4,
   TRE_W_FFN_NORM = 5, TRE_W_GATE = 6, TRE_W_UP = 7, TRE_W_DOWN = 8,
   TRE_W_ROUTER = 6, TRE_W_SHARED_GATE = 7, TRE_W_SHARED_UP = 8, TRE_W_SHARED_DOWN = 9,
   TRE_W_EXPERT_GATE = 10, TRE_W_EXPERT_UP = 11, TRE_W_EXPERT_DOWN = 12,
+  TRE_W_DQ = 1, TRE_W_Q_NORM = 2, TRE_W_UQ = 3, TRE_W_DKV = 4, TRE_W_KV_NORM = 5,
+  TRE_W_UK = 6, TRE_W_UV = 7, TRE_W_MLA_O = 8,
   TRE_W_SLOTS = 16
 };
 

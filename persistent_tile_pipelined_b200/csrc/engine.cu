@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include "mla.cuh"
 #include "ptx.cuh"
 #include "tiles.cuh"
 #include "tre_internal.h"
@@ -114,6 +115,9 @@ __device__ __forceinline__ int gemv_K(const Params& p, int op) {
     case OP_O: return p.Hq * p.D;
     case OP_DOWN: return p.F;
     case OP_MDOWN: return (p.nshared + p.topk) * p.Fe;
+    case OP_UQ: return p.QL;
+    case OP_UK: case OP_UV: return p.KL;   // W_uk / W_uv rows are KL wide
+    case OP_MO: return p.Hq * p.VD;
     default: return p.d;
   }
 }
@@ -157,7 +161,7 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
     g.part = t.aux & 0xff;
     g.np = max(1, t.aux >> 8);
   }
-  const int len = gemv_part_len(g.K, g.np);
+  const int len = g.np == 1 ? g.K : gemv_part_len(g.K, g.np);
   g.k0 = g.part * len;
   g.Kp = min(len, g.K - g.k0);
   g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes);
@@ -189,6 +193,15 @@ __device__ __forceinline__ const uint16_t* part_row(const Params& p, const Task&
       return L.w[t.op == OP_O ? TRE_W_O : TRE_W_DOWN] + (size_t)n * K + g.k0;
     case OP_GU: return L.w[seg ? TRE_W_UP : TRE_W_GATE] + (size_t)n * K;
     case OP_ROUTER: return L.w[TRE_W_ROUTER] + (size_t)n * K;
+    case OP_MDQKV:
+      if (n < p.QL) { *contig = p.QL - n; return L.w[TRE_W_DQ] + (size_t)n * K; }
+      return L.w[TRE_W_DKV] + (size_t)(n - p.QL) * K;
+    case OP_UQ: return L.w[TRE_W_UQ] + (size_t)n * K;
+    case OP_UK: return L.w[TRE_W_UK] + (size_t)n * K;
+    case OP_UV: return L.w[TRE_W_UV] + (size_t)n * K;
+    case OP_MO:
+      if (g.np > 1) *contig = 1;
+      return L.w[TRE_W_MLA_O] + (size_t)n * K + g.k0;
     case OP_SGU: return L.w[seg ? TRE_W_SHARED_UP : TRE_W_SHARED_GATE] + (size_t)n * K;
     case OP_RGU: {
       const int j = n / p.Fe, r = n - j * p.Fe;
@@ -232,7 +245,7 @@ struct RowSrc {
 
 __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const GemvGeom& g) {
   RowSrc r;
-  r.lookup = t.op == OP_QKV;
+  r.lookup = t.op == OP_QKV || t.op == OP_MDQKV;
   r.stride = g.K;
   if (t.op == OP_RGU) r.stride = p.d;
   else if (t.op == OP_MDOWN) r.stride = g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe;
@@ -252,6 +265,8 @@ __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, 
     const int nr = min(g.rps, t.r1 - (t.r0 + i * g.rps));
     return (uint32_t)(g.nseg * nr * g.Kp * 2);
   }
+  if (t.type == T_MLA_ATTN)  // whole boxes (rows past the cache are zero-filled)
+    return (uint32_t)((p.KL + p.R) / kMlaBox * kMlaPosPerStage * 128);
   const int n = min(p.pps, t1 - (t0 + i * p.pps));
   return (uint32_t)(2 * n * p.D * 2);
 }
@@ -299,6 +314,13 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
         n += take;
       }
     }
+  } else if (t.type == T_MLA_ATTN) {
+    // 64-column boxes of 32 latent rows, 128-byte swizzled (see mla.cuh)
+    if (lane < (p.KL + p.R) / kMlaBox) {
+      const uint8_t* map = static_cast<const uint8_t*>(p.mla_maps) + (size_t)t.layer * 128;
+      tma_load_2d(dst + (size_t)lane * kMlaPosPerStage * 128, map, lane * kMlaBox,
+                  t0 + i * kMlaPosPerStage, bar);
+    }
   } else if (lane < 2) {
     const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
     const size_t rowb = (size_t)p.D * 2;
@@ -318,6 +340,7 @@ __device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, in
                                               long long budget) {
   const uint8_t* src[3] = {nullptr, nullptr, nullptr};
   long long bytes[3] = {0, 0, 0};
+  if (t.type == T_MLA_ATTN) return;  // latent tiles come through the tensor map
   if (t.type == T_GEMV) {
     const GemvGeom g = gemv_geom(p, t);
     if (g.np > 1 || needs_route(p, t)) return;  // strided rows, or addresses not known yet
@@ -455,14 +478,17 @@ __device__ __forceinline__ float resid_in(const Params& p, int layer, int n) {
 }
 
 // Input-vector identity for reuse across consecutive tasks (same layer, same source,
-// same K-part).  The router, shared and routed gate/up all read RMSNorm(h1).
+// same K-part).  The router, shared and routed gate/up all read RMSNorm(h1).  -1: the
+// input depends on the task's rows (MLA per-head ops): always staged again.
 __device__ __forceinline__ int input_key(const Task& t) {
   int cls;
   switch (t.op) {
-    case OP_QKV: cls = 0; break;
-    case OP_O: cls = 1; break;
+    case OP_QKV: case OP_MDQKV: cls = 0; break;
+    case OP_O: case OP_MO: cls = 1; break;
     case OP_GU: case OP_ROUTER: case OP_SGU: case OP_RGU: cls = 2; break;
     case OP_DOWN: case OP_MDOWN: cls = 3; break;
+    case OP_UQ: cls = 5; break;
+    case OP_UK: case OP_UV: return -1;
     default: cls = 4; break;
   }
   const int part = (t.op == OP_LM || t.op == OP_ROUTER) ? 0 : (t.aux & 0xff);
@@ -480,6 +506,7 @@ __device__ float load_input(const Params& p, const Task& t, const GemvGeom& gg, 
   const uint16_t* gain = nullptr;
   switch (t.op) {
     case OP_QKV:
+    case OP_MDQKV:
       gain = p.layers[t.layer].w[TRE_W_ATTN_NORM];
       if (t.layer > 0) src = p.x;
       else if (p.x_in) src = p.x_in;
@@ -489,6 +516,9 @@ __device__ float load_input(const Params& p, const Task& t, const GemvGeom& gg, 
     case OP_GU: case OP_ROUTER: case OP_SGU: case OP_RGU:
       src = p.h1; gain = p.layers[t.layer].w[TRE_W_FFN_NORM]; break;
     case OP_DOWN: case OP_MDOWN: src = p.u; break;
+    case OP_UQ: src = p.cqkv; gain = p.layers[t.layer].w[TRE_W_Q_NORM]; break;
+    case OP_UV: src = p.o_lat + (size_t)(t.r0 / p.VD) * p.KL; break;
+    case OP_MO: src = p.mla_o; break;
     default: src = p.x; gain = p.final_norm; break;
   }
   if (src) src += gg.k0;        // normalised inputs are single-part (k0 = 0)
@@ -532,8 +562,9 @@ __device__ float load_input(const Params& p, const Task& t, const GemvGeom& gg, 
 }
 
 // ---- attention task ----------------------------------------------------------------------------
-__device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float& s) {
-  const double ang = (double)p.pos * p.rope_inv_freq[i];
+__device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float& s,
+                                        const double* inv_freq = nullptr) {
+  const double ang = (double)p.pos * (inv_freq ? inv_freq : p.rope_inv_freq)[i];
   const double two_pi = 6.283185307179586476925286766559;
   const double red = ang - two_pi * rint(ang / two_pi);
   sincosf((float)red, &s, &c);
@@ -748,6 +779,394 @@ __device__ __forceinline__ void run_attn(const Params& p, const Task& t, uint32_
 #undef TRE_ATTN
 }
 
+// ---- absorbed MLA: per-head W_uk contraction ----------------------------------------------------
+// Task = one head h: rows [h NP, (h + 1) NP) of W_uk ([H NP][KL]) stream through the ring,
+// and q_lat[c] = sum_i q_nope[i] W_uk[h NP + i][c] accumulates per warp (lane owns columns
+// 8 lane .. 8 lane + 7 of every 256-column block); the warps' sums are added in warp order.
+// The task also writes RoPE(q_pe) after q_lat, and head 0 appends this token's latent row
+// [RMSNorm(c_kv; kv_norm) | RoPE(k_pe)] (bf16) to the cache and keeps its values for the
+// attention's new position.
+__device__ __noinline__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint32_t gs, int ns,
+                        uint8_t* ring, uint64_t* full, uint64_t* empty, const uint32_t* tags,
+                        float* ub, float* red1, int warp, int lane, int ctid, bool& ab) {
+  const int h = t.r0 / p.NP, KL = p.KL, C = KL + p.R;
+  float* qn = ub;                                  // [NP] q_nope of this head
+  float* red = ub + ((p.NP + 63) / 64) * 64;       // [8][KL] per-warp sums
+  const float* qh = p.qkv + (size_t)h * (p.NP + p.R);
+  for (int i = ctid; i < p.NP; i += kConsumerThreads) qn[i] = __ldcg(qh + i);
+  consumer_sync(kConsumerThreads);
+  const uint32_t NS = (uint32_t)p.ring_stages;
+  const int nblk = KL / 256 + ((KL % 256) ? 1 : 0);   // 256-column blocks (lane: 8 columns each)
+  float acc[3][8];
+#pragma unroll
+  for (int b = 0; b < 3; ++b)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[b][k] = 0.f;
+  const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
+  for (int i = first; i < ns; i += kConsumerWarps) {
+    const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
+    if (!stage_wait(p, full, tags, sidx)) {
+      ab = true;
+      break;
+    }
+    const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
+    const uint8_t* sp = ring + (size_t)slot * p.stage_bytes;
+    for (int r = 0; r < nr; ++r) {
+      const float qv = qn[n0 - t.r0 + r];
+      const uint8_t* row = sp + (size_t)r * KL * 2;
+#pragma unroll
+      for (int b = 0; b < 3; ++b) {
+        const int c0 = b * 256 + lane * 8;
+        if (b < nblk && c0 < KL) {
+          const uint4 w = *reinterpret_cast<const uint4*>(row + (size_t)c0 * 2);
+          acc[b][0] = fmaf(qv, bf_lo(w.x), acc[b][0]);
+          acc[b][1] = fmaf(qv, bf_hi(w.x), acc[b][1]);
+          acc[b][2] = fmaf(qv, bf_lo(w.y), acc[b][2]);
+          acc[b][3] = fmaf(qv, bf_hi(w.y), acc[b][3]);
+          acc[b][4] = fmaf(qv, bf_lo(w.z), acc[b][4]);
+          acc[b][5] = fmaf(qv, bf_hi(w.z), acc[b][5]);
+          acc[b][6] = fmaf(qv, bf_lo(w.w), acc[b][6]);
+          acc[b][7] = fmaf(qv, bf_hi(w.w), acc[b][7]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_n(&empty[slot], kConsumerWarps);
+  }
+#pragma unroll
+  for (int b = 0; b < 3; ++b) {
+    const int c0 = b * 256 + lane * 8;
+    if (b < nblk && c0 < KL)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) red[warp * KL + c0 + k] = acc[b][k];
+  }
+  consumer_sync(kConsumerThreads);
+  float* qf = p.qf + (size_t)h * C;
+  for (int c = ctid; c < KL; c += kConsumerThreads) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) v += red[w * KL + c];
+    qf[c] = v;
+  }
+  const int R2 = p.R / 2;
+  for (int i = ctid; i < R2; i += kConsumerThreads) {
+    const float x0 = __ldcg(qh + p.NP + i), x1 = __ldcg(qh + p.NP + i + R2);
+    float cs, sn;
+    rope_cs(p, i, cs, sn, p.rope_inv_freq_r);
+    qf[KL + i] = x0 * cs - x1 * sn;
+    qf[KL + i + R2] = x0 * sn + x1 * cs;
+  }
+  if (h == 0) {  // this token's latent row
+    const float* kv = p.cqkv + p.QL;
+    const uint16_t* gain = p.layers[t.layer].w[TRE_W_KV_NORM];
+    float ss = 0.f;
+    for (int c = ctid; c < KL; c += kConsumerThreads) ss = fmaf(__ldcg(kv + c), __ldcg(kv + c), ss);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (lane == 0) red1[warp] = ss;
+    consumer_sync(kConsumerThreads);
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) tot += red1[w];
+    const float rn = 1.f / sqrtf(tot / (float)KL + p.eps);
+    __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p.layers[t.layer].k_cache) + (size_t)p.pos * C;
+    for (int c = ctid; c < KL; c += kConsumerThreads) {
+      const __nv_bfloat16 v = __float2bfloat16_rn(__ldcg(kv + c) * rn * bf_lo(gain[c]));
+      row[c] = v;
+      p.lat_new[c] = __bfloat162float(v);
+    }
+    for (int i = ctid; i < R2; i += kConsumerThreads) {
+      const float x0 = __ldcg(kv + KL + i), x1 = __ldcg(kv + KL + i + R2);
+      float cs, sn;
+      rope_cs(p, i, cs, sn, p.rope_inv_freq_r);
+      const __nv_bfloat16 a = __float2bfloat16_rn(x0 * cs - x1 * sn);
+      const __nv_bfloat16 b = __float2bfloat16_rn(x0 * sn + x1 * cs);
+      row[KL + i] = a;
+      row[KL + i + R2] = b;
+      p.lat_new[KL + i] = __bfloat162float(a);
+      p.lat_new[KL + i + R2] = __bfloat162float(b);
+    }
+  }
+  __threadfence();
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) red_release_gpu_add(p.counters + t.out, 1u);
+}
+
+// ---- absorbed MLA: latent attention on tensor cores ---------------------------------------------
+// Task = (head group hg of 16 heads, split s of the cached positions [0, pos)); the last
+// split also takes the new position from lat_new.  Per 32-row latent stage:
+//   scores: warp w multiplies the group's queries (A, hi + lo, held in registers for the
+//           warp's k-steps of the KL + R columns) by the stage's rows (B, ldmatrix from the
+//           swizzled tile); the 8 warps' partial scores are summed through shared memory;
+//   softmax: thread (head, 2 positions) scales to log2 units, masks rows past the split,
+//           updates the head's running max / sum and writes P as bf16 hi + lo;
+//   values: warp w accumulates O[16][KL / 8 columns] += P (hi + lo) x rows (ldmatrix.trans).
+// The split's (m, l, O) go to the partial buffer; the last split of the group to finish
+// (arrival ticket) combines the splits into o_lat.
+__device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
+                              uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
+                              int* flag, int warp, int lane, int ctid, bool& ab) {
+  constexpr int HG = kMlaHeadGroup, PS = kMlaPosPerStage, RP = 36;  // score row pitch (floats)
+  const int KL = p.KL, C = KL + p.R, hg = t.r0, split = t.r1, S = t.aux;
+  const bool last = (split == S - 1);
+  float* red = ub;                                        // [8][16][RP] partial scores
+  __nv_bfloat16* phi = reinterpret_cast<__nv_bfloat16*>(ub + kConsumerWarps * HG * RP);  // [16][40]
+  __nv_bfloat16* plo = phi + HG * 40;                                                    // [16][40]
+  float* mst = reinterpret_cast<float*>(plo + HG * 40);   // [16] running max (log2 units)
+  float* lst = mst + HG;                                  // [16] running sum
+  float* alp = lst + HG;                                  // [16] rescale of this stage
+  float* snw = alp + HG;                                  // [16] score of the new position
+  const float scale = 1.4426950408889634f / sqrtf((float)(p.NP + p.R));
+  const int g8 = lane >> 2, t4 = lane & 3;
+
+  // this warp's k-steps of the score product, and its query fragments (hi, lo)
+  const int KS = C / 16, kb = KS / kConsumerWarps, kr = KS % kConsumerWarps;
+  const int k_begin = warp * kb + min(warp, kr), k_count = kb + (warp < kr ? 1 : 0);
+  uint32_t ahi[kMlaMaxKSteps][4], alo[kMlaMaxKSteps][4];
+  const float* q0 = p.qf + (size_t)(hg * HG + g8) * C;
+  const float* q8 = q0 + (size_t)8 * C;
+#pragma unroll
+  for (int j = 0; j < kMlaMaxKSteps; ++j) {
+    if (j < k_count) {
+      const int k0 = (k_begin + j) * 16 + 2 * t4;
+      split_pair(__ldcg(q0 + k0), __ldcg(q0 + k0 + 1), ahi[j][0], alo[j][0]);
+      split_pair(__ldcg(q8 + k0), __ldcg(q8 + k0 + 1), ahi[j][1], alo[j][1]);
+      split_pair(__ldcg(q0 + k0 + 8), __ldcg(q0 + k0 + 9), ahi[j][2], alo[j][2]);
+      split_pair(__ldcg(q8 + k0 + 8), __ldcg(q8 + k0 + 9), ahi[j][3], alo[j][3]);
+    }
+  }
+  if (ctid < HG) {
+    mst[ctid] = -INFINITY;
+    lst[ctid] = 0.f;
+  }
+  // output accumulators: this warp's KL / 8 columns = KL / 64 n-tiles of 8
+  const int ncol = KL / kConsumerWarps, nt_count = ncol / 8, col0 = warp * ncol;
+  float o[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; ++n)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[n][k] = 0.f;
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
+
+  int t0, t1;
+  attn_range(p, t, t0, t1);
+  const uint32_t NS = (uint32_t)p.ring_stages;
+  for (int i = 0; i < ns; ++i) {
+    const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
+    const bool landed = stage_wait(p, full, tags, sidx);
+    const uint8_t* tile = ring + (size_t)slot * p.stage_bytes;
+    const uint32_t tb = smem_u32(tile);
+    // ---- partial scores over this warp's k-steps, 4 n-tiles of 8 rows
+    float c[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) c[n][k] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMlaMaxKSteps; ++j) {
+      if (landed && j < k_count) {
+        const int ch = (k_begin + j) * 2;  // 16-byte chunk of the step's first 8 columns
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {   // n-tile pairs (rows 16 np .. 16 np + 15)
+          const int m = lane >> 3, r = np * 16 + (m >> 1) * 8 + (lane & 7);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(tb + lat_off(r, ch + (m & 1)), b0, b1, b2, b3);
+          mma_bf16(c[2 * np], ahi[j], b0, b1);
+          mma_bf16(c[2 * np], alo[j], b0, b1);
+          mma_bf16(c[2 * np + 1], ahi[j], b2, b3);
+          mma_bf16(c[2 * np + 1], alo[j], b2, b3);
+        }
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      float* r0 = red + (warp * HG + g8) * RP + n * 8 + 2 * t4;
+      r0[0] = c[n][0];
+      r0[1] = c[n][1];
+      r0[8 * RP] = c[n][2];
+      r0[8 * RP + 1] = c[n][3];
+    }
+    // every warp takes part in every stage: the barrier also agrees on an abort
+    if (consumer_sync_or(!landed, kConsumerThreads)) {
+      ab = true;
+      break;
+    }
+    // ---- softmax: thread = (head hh, rows pp, pp + 1)
+    {
+      const int hh = ctid >> 4, pp = (ctid & 15) * 2;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        s0 += red[(w * HG + hh) * RP + pp];
+        s1 += red[(w * HG + hh) * RP + pp + 1];
+      }
+      const int tt = t0 + i * PS + pp;
+      s0 = tt < t1 ? s0 * scale : -INFINITY;
+      s1 = tt + 1 < t1 ? s1 * scale : -INFINITY;
+      float mx = fmaxf(s0, s1);
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float m_old = mst[hh], m_new = fmaxf(m_old, mx);
+      float p0 = 0.f, p1 = 0.f, a = 1.f;
+      if (m_new != -INFINITY) {
+        p0 = exp2f(s0 - m_new);
+        p1 = exp2f(s1 - m_new);
+        a = exp2f(m_old - m_new);
+      }
+      float ps = p0 + p1;
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      uint32_t hi, lo;
+      split_pair(p0, p1, hi, lo);
+      *reinterpret_cast<uint32_t*>(phi + hh * 40 + pp) = hi;
+      *reinterpret_cast<uint32_t*>(plo + hh * 40 + pp) = lo;
+      __syncwarp();
+      if ((ctid & 15) == 0) {
+        mst[hh] = m_new;
+        lst[hh] = lst[hh] * a + ps;
+        alp[hh] = a;
+      }
+    }
+    consumer_sync(kConsumerThreads);
+    // ---- O += P x rows, this warp's columns
+    {
+      const float a0 = alp[g8], a8 = alp[g8 + 8];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        o[n][0] *= a0;
+        o[n][1] *= a0;
+        o[n][2] *= a8;
+        o[n][3] *= a8;
+      }
+      const uint32_t ph = smem_u32(phi), pl = smem_u32(plo);
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {   // rows 16 ks .. 16 ks + 15
+        const int m = lane >> 3;
+        const uint32_t aoff = (uint32_t)(((m & 1) * 8 + (lane & 7)) * 80 + (ks * 2 + (m >> 1)) * 16);
+        uint32_t ah[4], al[4];
+        ldsm_x4(ph + aoff, ah[0], ah[1], ah[2], ah[3]);
+        ldsm_x4(pl + aoff, al[0], al[1], al[2], al[3]);
+#pragma unroll
+        for (int n = 0; n < 8; n += 2) {
+          if (n < nt_count) {
+            const int r = ks * 16 + (m & 1) * 8 + (lane & 7);
+            const int ch = (col0 + n * 8) / 8 + (m >> 1);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(tb + lat_off(r, ch), b0, b1, b2, b3);
+            mma_bf16(o[n], ah, b0, b1);
+            mma_bf16(o[n], al, b0, b1);
+            mma_bf16(o[n + 1], ah, b2, b3);
+            mma_bf16(o[n + 1], al, b2, b3);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
+  }
+  if (ab) return;
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
+
+  // ---- the new position (last split): score from lat_new, merged into (m, l, O)
+  if (last) {
+    for (int hh = warp * 2; hh < warp * 2 + 2; ++hh) {
+      const float* q = p.qf + (size_t)(hg * HG + hh) * C;
+      float a = 0.f;
+      for (int k = lane; k < C; k += 32) a = fmaf(__ldcg(q + k), __ldcg(p.lat_new + k), a);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+      if (lane == 0) snw[hh] = a * scale;
+    }
+    consumer_sync(kConsumerThreads);
+    float mn[2], an[2], pn[2];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int hh = g8 + 8 * half;
+      const float mo = mst[hh], sv = snw[hh];
+      mn[half] = fmaxf(mo, sv);
+      an[half] = mo == -INFINITY ? 0.f : exp2f(mo - mn[half]);
+      pn[half] = exp2f(sv - mn[half]);
+    }
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      if (n < nt_count) {
+        const int cc = col0 + n * 8 + 2 * t4;
+        const float v0 = __ldcg(p.lat_new + cc), v1 = __ldcg(p.lat_new + cc + 1);
+        o[n][0] = o[n][0] * an[0] + pn[0] * v0;
+        o[n][1] = o[n][1] * an[0] + pn[0] * v1;
+        o[n][2] = o[n][2] * an[1] + pn[1] * v0;
+        o[n][3] = o[n][3] * an[1] + pn[1] * v1;
+      }
+    }
+    consumer_sync(kConsumerThreads);
+    if (ctid < HG) {
+      const float mo = mst[ctid], sv = snw[ctid], m2 = fmaxf(mo, sv);
+      const float a = mo == -INFINITY ? 0.f : exp2f(mo - m2);
+      lst[ctid] = lst[ctid] * a + exp2f(sv - m2);
+      mst[ctid] = m2;
+    }
+    consumer_sync(kConsumerThreads);
+  }
+
+  // ---- this split's partial: O (KL), m, l per head
+  const size_t pstride = (size_t)KL + 2;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    if (n < nt_count) {
+      const int cc = col0 + n * 8 + 2 * t4;
+      float* d0 = p.part + ((size_t)(hg * HG + g8) * S + split) * pstride + cc;
+      float* d8 = p.part + ((size_t)(hg * HG + g8 + 8) * S + split) * pstride + cc;
+      d0[0] = o[n][0];
+      d0[1] = o[n][1];
+      d8[0] = o[n][2];
+      d8[1] = o[n][3];
+    }
+  }
+  if (ctid < HG) {
+    float* d = p.part + ((size_t)(hg * HG + ctid) * S + split) * pstride + KL;
+    d[0] = mst[ctid];
+    d[1] = lst[ctid];
+  }
+  __threadfence();
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) {
+    const uint32_t old = atom_acq_rel_gpu_add(p.tickets + hg, 1u);
+    *flag = ((old + 1u) % (uint32_t)S) == 0u;
+    if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
+  }
+  consumer_sync(kConsumerThreads);
+  if (*flag) {  // last split of the group: combine
+    float* ms = ub;               // [16][S]
+    float* ls = ub + HG * S;      // [16][S]
+    for (int idx = ctid; idx < HG * S; idx += kConsumerThreads) {
+      const float* src = p.part + ((size_t)(hg * HG) * S + idx) * pstride + KL;
+      ms[idx] = __ldcg(src);
+      ls[idx] = __ldcg(src + 1);
+    }
+    consumer_sync(kConsumerThreads);
+    for (int idx = ctid; idx < HG * KL; idx += kConsumerThreads) {
+      const int hh = idx / KL, cc = idx % KL;
+      const float* mh = ms + hh * S;
+      const float* lh = ls + hh * S;
+      float M = -INFINITY;
+      for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mh[s2]);
+      float L = 0.f, O = 0.f;
+      const float* src = p.part + (size_t)(hg * HG + hh) * S * pstride + cc;
+#pragma unroll 8
+      for (int s2 = 0; s2 < S; ++s2) {
+        const float w = mh[s2] == -INFINITY ? 0.f : exp2f(mh[s2] - M);
+        L = fmaf(w, lh[s2], L);
+        O = fmaf(w, __ldcg(src + s2 * pstride), O);
+      }
+      p.o_lat[(size_t)(hg * HG + hh) * KL + cc] = O / L;
+    }
+    __threadfence();
+    consumer_sync(kConsumerThreads);
+    if (ctid == 0) red_release_gpu_add(p.counters + t.out, 1u);
+  }
+}
+
 // ---- GEMV epilogue ---------------------------------------------------------------------------------
 // Residual rows of an O-proj / down task, staged before its stages: part 0 reads the
 // residual stream (x, or for layer 0 the embedding row / layer input; h1 for down), later
@@ -758,6 +1177,7 @@ __device__ __forceinline__ void prefetch_resid(const Params& p, const Task& t, c
     const int n = t.r0 + r;
     float v;
     if (t.op == OP_O) v = g.part == 0 ? resid_in(p, t.layer, n) : __ldcg(p.h1 + n);
+    else if (t.op == OP_MO) v = g.part == 0 ? resid_in(p, t.layer, n) : __ldcg(p.x + n);
     else v = g.part == 0 ? __ldcg(p.h1 + n) : __ldcg(p.x + n);
     resid[r] = v;
   }
@@ -766,11 +1186,14 @@ __device__ __forceinline__ void prefetch_resid(const Params& p, const Task& t, c
 __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const GemvGeom& g, int n,
                                           float v, float rn, const float* resid, Best& best) {
   switch (t.op) {
-    case OP_QKV: p.qkv[n] = v * rn; break;
+    case OP_QKV: case OP_UQ: p.qkv[n] = v * rn; break;
+    case OP_MDQKV: p.cqkv[n] = v * rn; break;
+    case OP_UV: p.mla_o[n] = v; break;
     case OP_O: p.h1[n] = resid[n - t.r0] + v; break;
     case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
     case OP_MDOWN: p.mpart[(size_t)g.part * p.d + n] = v; break;
-    case OP_DOWN: {
+    case OP_DOWN:
+    case OP_MO: {
       const float y = resid[n - t.r0] + v;
       p.x[n] = y;
       if (g.part == g.np - 1) {
@@ -871,13 +1294,19 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     if (t.type == T_ATTN) {
       cur_key = -1;  // the attention scratch aliases the input-vector planes
       run_attn(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
+    } else if (t.type == T_MLA_ATTN) {
+      cur_key = -1;
+      mla_attn_task(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
+    } else if (t.op == OP_UK) {
+      cur_key = -1;
+      uk_task(p, t, gemv_geom(p, t), gs, ns, ring, full, empty, tags, ub, red, warp, lane, ctid, ab);
     } else {
       const GemvGeom g = gemv_geom(p, t);
       const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
-      const bool has_resid = t.op == OP_O || t.op == OP_DOWN;
+      const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MO;
       if (has_resid) prefetch_resid(p, t, g, resid, ctid);
-      if (key != cur_key) {
+      if (key != cur_key || key < 0) {
         const float rn = load_input(p, t, g, ub, red, ctid);
         if (ctid == 0) *rn_s = rn;
         cur_key = key;
@@ -1008,6 +1437,11 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
   const int b = blockIdx.x;
   const Task* my = p.tasks + p.sm_begin[b];
   const int ntask = p.sm_begin[b + 1] - p.sm_begin[b];
+  // the swizzled latent tiles assume 1024-byte aligned ring slots
+  if (p.KL > 0 && (smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) record_error(p, TRE_ERR_BOUNDS, -3);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (uint32_t i = 0; i < NS; ++i) {

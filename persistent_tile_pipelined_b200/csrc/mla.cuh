@@ -1,0 +1,78 @@
+// Absorbed-MLA tiles of the persistent engine: the per-head W_uk contraction and the
+// latent attention on tensor cores.
+//
+// Absorbed MLA (DeepSeek-V2's; the pages name the fused kernel FlashSparseMLA with
+// batch == 1 — TileRT code audit, blog-vs-code table — and fold the query heads of a
+// latent tile together — Speed is intelligence talk, section on the attention kernel) is
+// multi-query attention of H heads over one latent row per position: query head h is
+// [W_uk,h^T q_nope,h | RoPE(q_pe,h)] (KL + R wide), every key is the cached latent row
+// [c_kv | k_pe] and every value its first KL columns.  That is a dense contraction per
+// position tile (16 heads x (KL + R) x 32 positions), so it runs on the tensor cores with
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate).  Keys and values are bf16 already; the
+// fp32 query and probabilities are split into bf16 hi + lo parts and both parts go
+// through the product, which keeps about 16 significand bits of them.
+//
+// A latent stage is 32 cached rows brought in by 2-D tensor copies of 64-column boxes
+// with the 128-byte swizzle, so ldmatrix reads rows 1152 bytes apart without bank
+// conflicts: chunk c (16 bytes) of row r of box b lives at b * 4096 + r * 128 + ((c ^ (r & 7)) << 4).
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+#include "tre_internal.h"
+
+namespace tre {
+
+// ---- tensor-core helpers ------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// d += a * b for one 16x8x16 tile (A row-major 16x16, B column-major 16x8, fp32 C).
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) {
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// x0, x1 -> packed bf16 pairs hi = rn(x), lo = rn(x - hi); the lower column in the low half.
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  hi = bf2_bits(h);
+  lo = bf2_bits(__floats2bfloat162_rn(x0 - hf.x, x1 - hf.y));
+}
+
+// Byte offset of 16-byte chunk `ch` (columns 8 ch .. 8 ch + 7) of row r of a latent stage.
+__device__ __forceinline__ uint32_t lat_off(int r, int ch) {
+  return (uint32_t)((ch >> 3) * (kMlaPosPerStage * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
+// 2-D tensor copy of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+}  // namespace tre

@@ -64,6 +64,7 @@ struct Builder {
   std::vector<std::vector<Task>> q;  // per SM
   std::vector<int64_t> cum;          // streamed bytes per SM
   int next_id = 0;
+  int kpart_max = kMaxKPart;
 
   explicit Builder(int n) : nsm(n), q(n), cum(n, 0) {}
 
@@ -86,7 +87,7 @@ struct Builder {
   // K-parts (else they follow from K).  Returns the number of tasks that bump `out`.
   int gemv(uint8_t op, int layer, int N, int K, int nseg, int dep, uint32_t dep_count, int out,
            int cap, int np = 0, int cut = 0) {
-    if (np <= 0) np = (op == OP_LM || op == OP_ROUTER) ? 1 : gemv_nparts(K);
+    if (np <= 0) np = (op == OP_LM || op == OP_ROUTER) ? 1 : gemv_nparts(K, kpart_max);
     auto ranges = assign_rows(N, (int64_t)nseg * K * 2, cum);
     int n = 0;
     for (int s = 0; s < nsm; ++s) {
@@ -116,6 +117,38 @@ struct Builder {
     std::vector<int> out(count);
     for (int k = 0; k < count; ++k) out[k] = idx[k % nsm];
     return out;
+  }
+
+  // One GEMV task per unit (an MLA head): rows [u * rows, (u + 1) * rows), dealt round
+  // robin to the SMs.  Returns the task count.
+  int per_unit(uint8_t op, int layer, int units, int rows, int64_t bytes_per_unit, int dep,
+               uint32_t dep_count, int out) {
+    const std::vector<int> sms = spread(units);
+    for (int u = 0; u < units; ++u) {
+      Task t = make(T_GEMV, op, layer, dep, dep_count, out);
+      t.r0 = u * rows;
+      t.r1 = (u + 1) * rows;
+      t.aux = 0 | (1 << 8);
+      q[sms[u]].push_back(t);
+      cum[sms[u]] += bytes_per_unit;
+    }
+    return units;
+  }
+
+  // MLA attention: (head group, KV split) tasks dealt round robin; aux = splits.
+  void mla_attention(int layer, int groups, int S, int64_t bytes_per_task, int dep,
+                     uint32_t dep_count, int out) {
+    const std::vector<int> sms = spread(groups * S);
+    for (int g = 0; g < groups; ++g)
+      for (int sp = 0; sp < S; ++sp) {
+        const int best = sms[g * S + sp];
+        Task t = make(T_MLA_ATTN, 0, layer, dep, dep_count, out);
+        t.r0 = g;
+        t.r1 = sp;
+        t.aux = S;
+        q[best].push_back(t);
+        cum[best] += bytes_per_task;
+      }
   }
 
   // Set aux = count on every task of `op` created since task id `first`.
@@ -160,11 +193,31 @@ struct Builder {
   }
 };
 
+static tre_status validate_mla(const tre_config& c) {
+  if (c.n_q_heads < kMlaHeadGroup || c.n_q_heads % kMlaHeadGroup)
+    return fail(TRE_ERR_UNSUPPORTED, "MLA heads must be a positive multiple of 16");
+  if (c.kv_lora < 128 || c.kv_lora % 128)
+    return fail(TRE_ERR_UNSUPPORTED, "MLA kv_lora must be a positive multiple of 128");
+  if (c.rope_dim < 16 || c.rope_dim % 16)
+    return fail(TRE_ERR_UNSUPPORTED, "MLA rope_dim must be a positive multiple of 16");
+  const int C = c.kv_lora + c.rope_dim;
+  if (C % kMlaBox || C > 16 * kMlaMaxKSteps * kConsumerWarps)
+    return fail(TRE_ERR_UNSUPPORTED, "MLA kv_lora + rope_dim must be a multiple of 64, <= 768");
+  if (c.q_lora < 8 || c.q_lora % 8 || c.nope_dim < 8 || c.nope_dim % 8 || c.v_dim < 8 ||
+      c.v_dim % 8)
+    return fail(TRE_ERR_INVALID_ARG, "MLA q_lora, nope_dim and v_dim must be positive multiples of 8");
+  if (c.q_lora > kMaxKPart) return fail(TRE_ERR_UNSUPPORTED, "MLA q_lora above 16384");
+  if (c.nope_dim > kMaxResidRows) return fail(TRE_ERR_UNSUPPORTED, "MLA nope_dim above 512");
+  return TRE_OK;
+}
+
 static tre_status validate(const tre_config& c) {
-  if (c.kind == TRE_LAYER_MLA)
-    return fail(TRE_ERR_UNSUPPORTED, "layer kind not implemented in this build (GQA, MOE)");
-  if (c.kind != TRE_LAYER_GQA && c.kind != TRE_LAYER_MOE)
+  if (c.kind != TRE_LAYER_GQA && c.kind != TRE_LAYER_MOE && c.kind != TRE_LAYER_MLA)
     return fail(TRE_ERR_INVALID_ARG, "unknown layer kind");
+  if (c.kind == TRE_LAYER_MLA) {
+    tre_status st = validate_mla(c);
+    if (st != TRE_OK) return st;
+  }
   if (c.kind == TRE_LAYER_MOE) {
     if (c.n_experts < 1 || c.n_experts > kMaxExperts)
       return fail(TRE_ERR_UNSUPPORTED, "n_experts must be in [1, 512]");
@@ -179,13 +232,15 @@ static tre_status validate(const tre_config& c) {
     if (r != 0) return fail(TRE_ERR_INVALID_ARG, "reserved config fields must be zero");
   if (c.n_layers < 1 || c.n_layers > 1024) return fail(TRE_ERR_INVALID_ARG, "n_layers out of range");
   if (c.hidden < 8 || c.hidden % 8) return fail(TRE_ERR_INVALID_ARG, "hidden must be a positive multiple of 8");
-  if (c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads)
-    return fail(TRE_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
-  int G = c.n_q_heads / c.n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8)
-    return fail(TRE_ERR_UNSUPPORTED, "q heads per kv head must be 1, 2, 4 or 8");
-  if (c.head_dim != 64 && c.head_dim != 128)
-    return fail(TRE_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (c.kind != TRE_LAYER_MLA) {
+    if (c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads)
+      return fail(TRE_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+    int G = c.n_q_heads / c.n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+      return fail(TRE_ERR_UNSUPPORTED, "q heads per kv head must be 1, 2, 4 or 8");
+    if (c.head_dim != 64 && c.head_dim != 128)
+      return fail(TRE_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  }
   if (c.kind == TRE_LAYER_GQA && (c.ffn < 8 || c.ffn % 8))
     return fail(TRE_ERR_INVALID_ARG, "ffn must be a positive multiple of 8");
   if (c.has_embed_lm_head != 0 && c.has_embed_lm_head != 1)
@@ -215,10 +270,21 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
 
   PlanShape s{};
   s.kind = c.kind;
+  const bool mla = c.kind == TRE_LAYER_MLA;
   s.d = c.hidden;
   s.Hq = c.n_q_heads;
-  s.Hkv = c.n_kv_heads;
-  s.D = c.head_dim;
+  s.Hkv = mla ? 1 : c.n_kv_heads;
+  s.D = mla ? 0 : c.head_dim;
+  if (mla) {
+    s.QL = c.q_lora;
+    s.KL = c.kv_lora;
+    s.R = c.rope_dim;
+    s.NP = c.nope_dim;
+    s.VD = c.v_dim;
+  }
+  // an MLA output projection (K = H * v_dim) is staged in halves of at most 8192 inputs,
+  // so that the input planes leave room for a 5-deep ring of 36 KB stages
+  s.kpart_max = mla ? 8192 : kMaxKPart;
   s.F = c.ffn;
   s.V = c.has_embed_lm_head ? c.vocab : 0;
   s.L = c.n_layers;
@@ -246,34 +312,51 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // (input length, segments, K-part length) of every op the stack uses
   struct OpShape { int K, nseg, kp; };
   std::vector<OpShape> ops = {{s.d, 1, 0}, {s.Hq * s.D, 1, 0}, {s.d, 1, s.d}};
-  if (moe) {
+  if (mla) {
+    ops = {{s.d, 1, s.d}, {s.QL, 1, s.QL}, {s.KL, 1, s.KL}, {s.Hq * s.VD, 1, 0},
+           {s.NP, 1, s.NP}};
+    if (s.has_lm) ops.push_back({s.d, 1, s.d});
+  } else if (moe) {
     ops.push_back({s.d, 2, 0});                                  // shared / routed gate-up
     ops.push_back({(s.nshared + s.topk) * s.Fe, 1, s.Fe});       // MoE down: one part per expert
   } else {
     ops.push_back({s.d, 2, 0});
     ops.push_back({s.F, 1, 0});
   }
-  int xs = 8, need = 4 * s.D * 8;  // a stage holds at least 8 KV positions
+  // a stage holds at least 8 KV positions (GQA) or one MLA attention tile
+  int xs = 8, need = mla ? (s.KL + s.R) * kMlaPosPerStage * 2 : 4 * s.D * 8;
   for (auto& o : ops) {
-    const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K));
+    const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max));
     xs = std::max(xs, kp);
     need = std::max(need, o.nseg * kp * 2);
   }
   // A ring stage holds whole rows of one K-part (gate/up: a row of each matrix), or the K
   // and V rows of 8-64 cached positions.
-  int sb = c.stage_bytes ? c.stage_bytes : kDefaultStageBytes;
+  int sb = c.stage_bytes ? c.stage_bytes : std::max(kDefaultStageBytes, (need + 1023) / 1024 * 1024);
   if (!c.stage_bytes)
     while (sb < need && sb < kMaxStageBytes) sb += 1024;
   if (sb < need)
     return fail(TRE_ERR_UNSUPPORTED, "a weight row part (or gate/up row pair) is wider than a ring stage");
   s.stage_bytes = sb;
   int pps = 8;  // a power of two, so that every warp of a stage group takes 8 positions
-  while (pps * 2 <= kMaxPosPerStage && pps * 2 * 4 * s.D <= sb) pps *= 2;
+  if (mla) {
+    pps = kMlaPosPerStage;
+  } else {
+    while (pps * 2 <= kMaxPosPerStage && pps * 2 * 4 * s.D <= sb) pps *= 2;
+  }
   s.pos_per_stage = pps;
 
   s.xs_floats = (xs + 7) / 8 * 8;
   s.resid_floats = kMaxResidRows;
   s.attn_floats = G * s.D + 2 * s.D + kConsumerWarps * (2 * G + G * s.D) + 16;
+  if (mla) {
+    // score partials [8 warps][16][32] + P hi / lo (16 x 40 bf16 each) + head state; the
+    // combine stages (m, l) of every split; the W_uk contraction sums [8][KL]
+    const int Smax = std::max(1, nsm / (s.Hq / kMlaHeadGroup));
+    s.attn_floats = std::max(kConsumerWarps * kMlaHeadGroup * 36 + 640 + 128,
+                             2 * kMlaHeadGroup * Smax);
+    s.attn_floats = std::max(s.attn_floats, kConsumerWarps * s.KL + s.NP + 64);
+  }
   const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats, s.attn_floats) + 7) / 8 * 8;
   s.ub_floats = ubuf_floats;
   const int misc_bytes = 1024;
@@ -287,21 +370,42 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     return fail(TRE_ERR_UNSUPPORTED, "ring + buffers exceed the shared memory per block");
 
   // KV splits: enough (kv head, split) tasks to cover the SMs, but no split shorter than
-  // one stage of positions at full capacity.
+  // one stage of positions at full capacity.  MLA: (head group, split) tasks.
+  const int units = mla ? s.Hq / kMlaHeadGroup : s.Hkv;
   int S = c.kv_splits;
   if (!S) {
-    S = std::max(1, nsm / s.Hkv);
+    S = std::max(1, nsm / units);
     int max_s = std::max(1, (s.cap - 1 + s.pos_per_stage - 1) / s.pos_per_stage);
     S = std::min(S, max_s);
   }
   // the combine stages every split's (m, l) in the attention scratch: 2 G S <= 8 G D
-  if (S > 4 * s.D) return fail(TRE_ERR_UNSUPPORTED, "kv_splits above 4 * head_dim");
+  if (!mla && S > 4 * s.D) return fail(TRE_ERR_UNSUPPORTED, "kv_splits above 4 * head_dim");
+  if (mla && 2 * kMlaHeadGroup * S > s.attn_floats)
+    return fail(TRE_ERR_UNSUPPORTED, "kv_splits too large for the MLA combine");
   s.kv_splits = S;
 
   Builder b(nsm);
+  b.kpart_max = s.kpart_max;
   int prev_down = -1;
   uint32_t prev_down_count = 0;
-  for (int l = 0; l < s.L; ++l) {
+  for (int l = 0; l < s.L && mla; ++l) {
+    // absorbed MLA: down-projections -> q up-projection -> per-head W_uk contraction (+ the
+    // latent append) -> attention over the latent cache -> per-head W_uv -> W_o + residual
+    const int cdq = counter_of(l, C_QKV), cuq = counter_of(l, C_MLA_UQ),
+              cuk = counter_of(l, C_MLA_UK), ca = counter_of(l, C_ATTN),
+              cuv = counter_of(l, C_MLA_UV), co = counter_of(l, C_O);
+    const int big = 1 << 30, C = s.KL + s.R, H = s.Hq, groups = H / kMlaHeadGroup;
+    const int n1 = b.gemv(OP_MDQKV, l, s.QL + C, s.d, 1, prev_down, prev_down_count, cdq, big);
+    const int n2 = b.gemv(OP_UQ, l, H * (s.NP + s.R), s.QL, 1, cdq, (uint32_t)n1, cuq, big);
+    const int n3 = b.per_unit(OP_UK, l, H, s.NP, (int64_t)s.NP * s.KL * 2, cuq, (uint32_t)n2, cuk);
+    const int64_t lat_task = (int64_t)(s.cap - s.M) / S * C * 2;
+    b.mla_attention(l, groups, S, lat_task, cuk, (uint32_t)n3, ca);
+    const int n5 = b.per_unit(OP_UV, l, H, s.VD, (int64_t)s.VD * s.KL * 2, ca, (uint32_t)groups, cuv);
+    const int n6 = b.gemv(OP_MO, l, s.d, H * s.VD, 1, cuv, (uint32_t)n5, co, s.resid_floats);
+    prev_down = co;
+    prev_down_count = (uint32_t)n6;
+  }
+  for (int l = 0; l < s.L && !mla; ++l) {
     const int cq = counter_of(l, C_QKV), ca = counter_of(l, C_ATTN), co = counter_of(l, C_O),
               cg = counter_of(l, C_GU), cd = counter_of(l, C_DOWN);
     // Q, K and V as one op over the stacked matrix [Wq; Wk; Wv]
@@ -375,6 +479,15 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
 
 int64_t step_bytes(const PlanShape& s, int pos) {
   const int64_t d = s.d, D = s.D;
+  if (s.kind == TRE_LAYER_MLA) {
+    const int64_t H = s.Hq, C = s.KL + s.R;
+    const int64_t w = (s.QL + C) * d + H * (s.NP + s.R) * s.QL +
+                      H * s.NP * s.KL + H * s.VD * s.KL + d * H * s.VD;
+    int64_t bytes = (w * 2 + (d + s.QL + s.KL) * 2) * s.L;   // weights and norm gains
+    bytes += (int64_t)s.L * (pos + 1) * C * 2;                // latent rows read + written
+    if (s.has_lm) bytes += (int64_t)s.V * d * 2 + d * 2 + d * 2 + (int64_t)s.V * 4;
+    return bytes;
+  }
   // MoE: the router, the shared experts and the selected experts only (what one token reads)
   const int64_t mlp = s.kind == TRE_LAYER_MOE
                           ? (int64_t)s.E * d + 3LL * (s.nshared + s.topk) * s.Fe * d

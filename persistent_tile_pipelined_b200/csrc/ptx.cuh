@@ -120,6 +120,19 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
+// Named barrier 1 over the consumer threads that also ORs a per-thread flag: returns
+// true on every thread if any thread passed true.
+__device__ __forceinline__ bool consumer_sync_or(bool v, int nthreads) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ uint32_t smid() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%smid;" : "=r"(r));

@@ -4,6 +4,7 @@
 // takes an external KV cache as raw tensors — TileRT code audit, KV-cache section); the
 // engine owns its plan, counters and activation scratch.  One decode step is one
 // cooperative launch of the persistent kernel (Static Compilation for LLM Inference, §1).
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -54,6 +55,40 @@ static tre_status cuda_fail(cudaError_t e, const char* what) {
 
 static bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
 
+// cuTensorMapEncodeTiled from the driver, looked up through the runtime (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static tre_status encode_latent_map(void* cache, int C, int cap, CUtensorMap* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) {
+      set_error("tre_create: cuTensorMapEncodeTiled is not available");
+      return TRE_ERR_CUDA;
+    }
+    fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  // the latent cache [cap][C] bf16 as a 2-D tensor; boxes of 64 columns x 32 rows with the
+  // 128-byte swizzle the MLA tiles read (rows past the cache read as zero)
+  const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)cap};
+  const cuuint64_t strides[1] = {(cuuint64_t)C * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kMlaBox, (cuuint32_t)kMlaPosPerStage};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cache, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("tre_create: cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
+    return TRE_ERR_CUDA;
+  }
+  return TRE_OK;
+}
+
 namespace {
 struct Carve {  // bump allocator over the engine's single device block
   size_t off = 0;
@@ -93,9 +128,11 @@ TRE_EXPORT tre_status tre_plan_inspect(const tre_config* cfg, int32_t num_sms,
   int mx = 0;
   for (int i = 0; i < s.nsm; ++i) mx = std::max(mx, begin[i + 1] - begin[i]);
   info->max_tasks_per_sm = mx;
-  info->weight_bytes = step_bytes(s, 0) - (int64_t)s.L * s.Hkv * s.D * 4 -
+  const int64_t row_new = s.kind == TRE_LAYER_MLA ? (int64_t)(s.KL + s.R) * 2 : (int64_t)s.Hkv * s.D * 4;
+  const int64_t row_read = s.kind == TRE_LAYER_MLA ? (int64_t)(s.KL + s.R) * 2 : (int64_t)s.Hkv * s.D * 4;
+  info->weight_bytes = step_bytes(s, 0) - (int64_t)s.L * row_new -
                        (s.has_lm ? (int64_t)s.V * 4 + 2LL * s.d : 0);
-  info->kv_bytes_at_capacity = (int64_t)s.L * s.Hkv * (int64_t)(s.cap - s.M) * s.D * 4;
+  info->kv_bytes_at_capacity = (int64_t)s.L * (int64_t)(s.cap - s.M) * row_read;
   int64_t lo = INT64_MAX, hi = 0;
   for (int64_t b : bytes) {
     lo = std::min(lo, b);
@@ -167,14 +204,18 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   if (st != TRE_OK) return st;
 
   // ---- pointer validation: everything the plan reads must be present and 16B-aligned.
-  if (!w->layer_w || !w->k_cache || !w->v_cache) {
+  if (!w->layer_w || !w->k_cache || (!w->v_cache && s.kind != TRE_LAYER_MLA)) {
     set_error("tre_create: layer_w / k_cache / v_cache tables must be non-NULL");
     return TRE_ERR_INVALID_ARG;
   }
   static const int gqa_slots[] = {TRE_W_ATTN_NORM, TRE_W_Q,        TRE_W_K,  TRE_W_V,   TRE_W_O,
                                   TRE_W_FFN_NORM,  TRE_W_GATE,     TRE_W_UP, TRE_W_DOWN};
   std::vector<int> slots(gqa_slots, gqa_slots + 9);
-  if (s.kind == TRE_LAYER_MOE) {
+  const bool mla = s.kind == TRE_LAYER_MLA;
+  if (mla) {
+    slots = {TRE_W_ATTN_NORM, TRE_W_DQ, TRE_W_Q_NORM, TRE_W_UQ, TRE_W_DKV, TRE_W_KV_NORM,
+             TRE_W_UK, TRE_W_UV, TRE_W_MLA_O};
+  } else if (s.kind == TRE_LAYER_MOE) {
     slots = {TRE_W_ATTN_NORM, TRE_W_Q, TRE_W_K, TRE_W_V, TRE_W_O, TRE_W_FFN_NORM, TRE_W_ROUTER,
              TRE_W_EXPERT_GATE, TRE_W_EXPERT_UP, TRE_W_EXPERT_DOWN};
     if (s.nshared > 0)
@@ -192,12 +233,12 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
       }
       lp[l].w[slot] = static_cast<const uint16_t*>(p);
     }
-    if (!aligned16(w->k_cache[l]) || !aligned16(w->v_cache[l])) {
+    if (!aligned16(w->k_cache[l]) || (!mla && !aligned16(w->v_cache[l]))) {
       set_error("tre_create: KV cache of layer " + std::to_string(l) + " NULL or misaligned");
       return TRE_ERR_INVALID_ARG;
     }
     lp[l].k_cache = static_cast<uint16_t*>(w->k_cache[l]);
-    lp[l].v_cache = static_cast<uint16_t*>(w->v_cache[l]);
+    lp[l].v_cache = mla ? nullptr : static_cast<uint16_t*>(w->v_cache[l]);
   }
   if (s.has_lm && (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(w->lm_head))) {
     set_error("tre_create: embed / final_norm / lm_head NULL or not 16-byte aligned");
@@ -218,13 +259,19 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   e->n_tasks = (int)tasks.size();
 
   // ---- one device block for all engine-owned state
-  const int qkv_n = (s.Hq + 2 * s.Hkv) * s.D;
+  const int qkv_n = mla ? s.Hq * (s.NP + s.R) : (s.Hq + 2 * s.Hkv) * s.D;
+  const int C = s.KL + s.R;
+  std::vector<CUtensorMap> maps(mla ? s.L : 0);
+  for (int l = 0; l < (mla ? s.L : 0); ++l) {
+    tre_status ms = encode_latent_map(w->k_cache[l], C, s.cap, &maps[l]);
+    if (ms != TRE_OK) return ms;
+  }
   Carve cv;
   size_t o_tasks = cv.take<Task>(tasks.size());
   size_t o_begin = cv.take<int32_t>(begin.size());
   size_t o_layers = cv.take<LayerPtrs>(s.L);
   size_t o_ctr = cv.take<uint32_t>(s.n_counters);
-  size_t o_tick = cv.take<uint32_t>(s.Hkv);
+  size_t o_tick = cv.take<uint32_t>(std::max(s.Hkv, mla ? s.Hq / kMlaHeadGroup : 1));
   size_t o_lmt = cv.take<uint32_t>(1);
   size_t o_arg = cv.take<unsigned long long>(1);
   size_t o_err = cv.take<int32_t>(2);
@@ -240,10 +287,18 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_rtick = cv.take<uint32_t>(1);
   size_t o_mpart = cv.take<float>(moe ? (size_t)(s.nshared + s.topk) * s.d : 1);
   size_t o_dtick = cv.take<uint32_t>(moe ? s.down_blocks : 1);
-  size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (s.D + 2));
+  size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * ((mla ? s.KL : s.D) + 2));
   size_t o_logits = cv.take<float>(s.V > 0 ? s.V : 1);
   size_t o_tok = cv.take<int32_t>(1);
-  size_t o_inv = cv.take<double>(s.D / 2);
+  size_t o_inv = cv.take<double>(std::max(1, s.D / 2));
+  size_t o_invr = cv.take<double>(std::max(1, s.R / 2));
+  size_t o_cqkv = cv.take<float>(mla ? s.QL + C : 1);
+  size_t o_qf = cv.take<float>(mla ? (size_t)s.Hq * C : 1);
+  size_t o_latn = cv.take<float>(mla ? C : 1);
+  size_t o_olat = cv.take<float>(mla ? (size_t)s.Hq * s.KL : 1);
+  size_t o_mlao = cv.take<float>(mla ? (size_t)s.Hq * s.VD : 1);
+  cv.off = (cv.off + 127) & ~size_t(127);
+  size_t o_maps = cv.take<CUtensorMap>(maps.size() ? maps.size() : 1);
   const bool dbg_hidden = cfg->debug_flags & TRE_DEBUG_HIDDEN;
   const bool dbg_trace = cfg->debug_flags & TRE_DEBUG_TRACE;
   size_t o_hidden = dbg_hidden ? cv.take<float>((size_t)s.L * s.d) : 0;
@@ -271,12 +326,20 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   if ((ce = cudaMemcpy(B + o_layers, lp.data(), lp.size() * sizeof(LayerPtrs),
                        cudaMemcpyHostToDevice)) != cudaSuccess)
     return fail_free(ce, "upload layer table");
-  std::vector<double> inv(s.D / 2);
-  for (int i = 0; i < s.D / 2; ++i)
-    inv[i] = std::pow((double)cfg->rope_theta, -2.0 * i / (double)s.D);
-  if ((ce = cudaMemcpy(B + o_inv, inv.data(), inv.size() * sizeof(double),
+  // RoPE frequencies theta^(-2i/D) of the head dim (GQA / MoE) or the rope dim (MLA)
+  for (int which = 0; which < 2; ++which) {
+    const int D = which ? s.R : s.D;
+    if (D < 2) continue;
+    std::vector<double> inv(D / 2);
+    for (int i = 0; i < D / 2; ++i) inv[i] = std::pow((double)cfg->rope_theta, -2.0 * i / (double)D);
+    if ((ce = cudaMemcpy(B + (which ? o_invr : o_inv), inv.data(), inv.size() * sizeof(double),
+                         cudaMemcpyHostToDevice)) != cudaSuccess)
+      return fail_free(ce, "upload rope table");
+  }
+  if (!maps.empty() &&
+      (ce = cudaMemcpy(B + o_maps, maps.data(), maps.size() * sizeof(CUtensorMap),
                        cudaMemcpyHostToDevice)) != cudaSuccess)
-    return fail_free(ce, "upload rope table");
+    return fail_free(ce, "upload tensor maps");
   if ((ce = cudaHostAlloc(reinterpret_cast<void**>(&e->status_host), 4 * sizeof(int32_t),
                           cudaHostAllocMapped)) != cudaSuccess)
     return fail_free(ce, "cudaHostAlloc(status)");
@@ -315,6 +378,15 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.hidden = dbg_hidden ? reinterpret_cast<float*>(B + o_hidden) : nullptr;
   p.trace = dbg_trace ? reinterpret_cast<long long*>(B + o_trace) : nullptr;
   p.rope_inv_freq = reinterpret_cast<const double*>(B + o_inv);
+  p.rope_inv_freq_r = reinterpret_cast<const double*>(B + o_invr);
+  p.cqkv = reinterpret_cast<float*>(B + o_cqkv);
+  p.qf = reinterpret_cast<float*>(B + o_qf);
+  p.lat_new = reinterpret_cast<float*>(B + o_latn);
+  p.o_lat = reinterpret_cast<float*>(B + o_olat);
+  p.mla_o = reinterpret_cast<float*>(B + o_mlao);
+  p.mla_maps = B + o_maps;
+  p.QL = s.QL; p.KL = s.KL; p.R = s.R; p.NP = s.NP; p.VD = s.VD;
+  p.kpart_max = s.kpart_max;
   p.err = reinterpret_cast<int32_t*>(B + o_err);
   p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
   p.status_host = e->status_dev;
@@ -473,7 +545,10 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
   CK(cudaDeviceSynchronize());
   const Params& p = e->base;
   CK(cudaMemsetAsync(p.counters, 0, (size_t)e->shape.n_counters * 4, s));
-  CK(cudaMemsetAsync(p.tickets, 0, (size_t)e->shape.Hkv * 4, s));
+  CK(cudaMemsetAsync(p.tickets, 0,
+                     (size_t)std::max(e->shape.Hkv, e->shape.kind == TRE_LAYER_MLA
+                                                        ? e->shape.Hq / kMlaHeadGroup : 1) * 4,
+                     s));
   CK(cudaMemsetAsync(p.lm_ticket, 0, 4, s));
   CK(cudaMemsetAsync(p.router_ticket, 0, 4, s));
   if (e->shape.kind == TRE_LAYER_MOE)

@@ -37,7 +37,7 @@ constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per 
 // Rows longer than kMaxKPart are cut into K-parts: part j of a task covers input columns
 // [j * len, min(K, (j + 1) * len)); the parts of one row range are consecutive tasks on
 // one SM, the first adds the residual and later parts accumulate into the output.
-TRE_HD inline int gemv_nparts(int K) { return (K + kMaxKPart - 1) / kMaxKPart; }
+TRE_HD inline int gemv_nparts(int K, int kmax = kMaxKPart) { return (K + kmax - 1) / kmax; }
 TRE_HD inline int gemv_part_len(int K, int nparts) {
   const int l = (K + nparts - 1) / nparts;
   return (l + 7) / 8 * 8;
@@ -48,7 +48,7 @@ TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes) {
 }
 
 // ---- tasks --------------------------------------------------------------------------
-enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1 };
+enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1, T_MLA_ATTN = 2 };
 
 // GEMV ops: which matrix, which input vector, which epilogue.
 enum GemvOp : uint8_t {
@@ -64,8 +64,23 @@ enum GemvOp : uint8_t {
   OP_MDOWN = 8,   // in: u slice j              -> partial rows of slot j (a shared-expert
                   //                               slice or a selected expert); the block's
                   //                               last slot sums x = h1 + sum_j partial_j
-  OP_COUNT = 9
+  // absorbed MLA (attention-only layers)
+  OP_MDQKV = 9,   // in: RMSNorm(x; attn_norm)  -> cqkv = [Wdq; Wdkv] xn  (c_q, then c_kv | k_pe)
+  OP_UQ = 10,     // in: RMSNorm(c_q; q_norm)   -> q = Wuq c_q  (per head: nope, rope)
+  OP_UK = 11,     // in: q_nope of one head     -> q_lat = Wuk_h^T q_nope (rows contracted);
+                  //                               also RoPE(q_pe); head 0 appends the latent
+  OP_UV = 12,     // in: o_lat of one head      -> o = Wuv_h o_lat
+  OP_MO = 13,     // in: o                      -> x = x + Wo o
+  OP_COUNT = 14
 };
+
+// MLA counters reuse the per-layer slots: QKV = down-projections, ATTN, O = output
+// projection, and these three.
+enum MlaCounter { C_MLA_UQ = 3, C_MLA_UK = 4, C_MLA_UV = 5 };
+constexpr int kMlaHeadGroup = 16;     // query heads per MLA attention tile (the mma M)
+constexpr int kMlaPosPerStage = 32;   // latent rows per MLA attention stage
+constexpr int kMlaBox = 64;           // latent columns per tensor-map box (128 B, swizzled)
+constexpr int kMlaMaxKSteps = 6;      // 16-column k-steps of the score product per warp
 
 // Dependency counters: one per (layer, stage of the layer), then the LM head and a
 // counter nothing ever bumps (used only by the fault-injection debug plan).
@@ -99,6 +114,8 @@ struct PlanShape {
   int kind;
   int d, Hq, Hkv, D, F, V, L, cap, M;
   int E, topk, nshared, Fe;  // MoE: experts, selected per token, shared, expert FFN
+  int QL, KL, R, NP, VD;  // MLA: q_lora, kv_lora, rope, nope, v dims
+  int kpart_max;       // longest input slice of a GEMV task (floats)
   int u_floats;        // the SwiGLU activation buffer (MoE: shared then routed slices)
   int down_blocks;     // MoE down: row blocks (each summed by its last slot to finish)
   int nsm;
@@ -138,6 +155,14 @@ struct Params {
   float* route_w;                  // MoE normalised weights [L][topk]
   uint32_t* router_ticket;         // MoE: arrival ticket of the router tasks
   float* mpart;                    // MoE down partial rows [nshared + topk][d]
+  // absorbed MLA
+  float* cqkv;                     // [QL + KL + R]: c_q, then c_kv | k_pe (before norm / rope)
+  float* qf;                       // [H][KL + R]: q_lat | RoPE(q_pe), per head
+  float* lat_new;                  // [KL + R]: this token's latent row (bf16 values)
+  float* o_lat;                    // [H][KL]
+  float* mla_o;                    // [H * VD]
+  const void* mla_maps;            // [L] tensor maps (128 B each) over the latent caches
+  const double* rope_inv_freq_r;   // [R / 2]
   uint32_t* down_tickets;          // MoE down: arrival ticket per row block
   float* part;                     // [Hq][splits][D + 2]
   float* logits;                   // [V]
@@ -150,6 +175,7 @@ struct Params {
   volatile int32_t* status_host;   // host-mapped [2]: code, detail
   int d, Hq, Hkv, D, F, V, L, cap;
   int E, topk, nshared, Fe;
+  int QL, KL, R, NP, VD, kpart_max;
   int nsplit, pps, stage_bytes, ring_stages, xs_floats, ub_floats;
   float eps;
   int token, pos;

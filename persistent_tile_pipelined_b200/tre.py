@@ -283,6 +283,15 @@ def upload_moe_model(wl, model: dict, device="cuda:0", expert_fn=None) -> dict:
     return out
 
 
+def upload_mla_model(model: dict, device="cuda:0") -> dict:
+    """Copy a host absorbed-MLA model (bf16 words) to device tensors: the layer slots as
+    they are and each layer's latent cache [capacity][kv_lora + rope] as its k_cache."""
+    return {"layers": [{slot: _dev_tensor(a, device) for slot, a in layer.items()}
+                       for layer in model["layers"]],
+            "k_cache": [_dev_tensor(c, device) for c in model["latent_cache"]],
+            "v_cache": []}
+
+
 def make_weights(cfg: tre_config, dev_model: dict):
     """A tre_weights struct over the device tensors of `dev_model`.  Returns (weights,
     keepalive): keep `keepalive` referenced while the struct is in use."""
@@ -292,14 +301,16 @@ def make_weights(cfg: tre_config, dev_model: dict):
         for slot, t in dev_model["layers"][l].items():
             layer_w[l * TRE_W_SLOTS + slot] = t.data_ptr()
     kc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["k_cache"]])
-    vc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["v_cache"]])
+    vc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["v_cache"]]) \
+        if dev_model.get("v_cache") else None
     w = tre_weights()
     for k in ("embed", "final_norm", "lm_head"):
         if k in dev_model:
             setattr(w, k, dev_model[k].data_ptr())
     w.layer_w = ctypes.cast(layer_w, ctypes.POINTER(ctypes.c_void_p))
     w.k_cache = ctypes.cast(kc, ctypes.POINTER(ctypes.c_void_p))
-    w.v_cache = ctypes.cast(vc, ctypes.POINTER(ctypes.c_void_p))
+    if vc is not None:
+        w.v_cache = ctypes.cast(vc, ctypes.POINTER(ctypes.c_void_p))
     return w, (layer_w, kc, vc, dev_model)
 
 
@@ -315,14 +326,16 @@ class Engine:
             for slot, t in dev_model["layers"][l].items():
                 self._layer_w[l * TRE_W_SLOTS + slot] = t.data_ptr()
         self._kc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["k_cache"]])
-        self._vc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["v_cache"]])
+        self._vc = (ctypes.c_void_p * L)(*[t.data_ptr() for t in dev_model["v_cache"]]) \
+            if dev_model.get("v_cache") else None
         self.weights = tre_weights()
         for k in ("embed", "final_norm", "lm_head"):
             if k in dev_model:
                 setattr(self.weights, k, dev_model[k].data_ptr())
         self.weights.layer_w = ctypes.cast(self._layer_w, ctypes.POINTER(ctypes.c_void_p))
         self.weights.k_cache = ctypes.cast(self._kc, ctypes.POINTER(ctypes.c_void_p))
-        self.weights.v_cache = ctypes.cast(self._vc, ctypes.POINTER(ctypes.c_void_p))
+        if self._vc is not None:
+            self.weights.v_cache = ctypes.cast(self._vc, ctypes.POINTER(ctypes.c_void_p))
         self.device = device
         self.h = tre_create(cfg, self.weights, device)
 

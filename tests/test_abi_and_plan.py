@@ -17,6 +17,8 @@ from persistent_tile_pipelined_b200 import tre  # noqa: E402
 
 T_GEMV, T_ATTN = 0, 1
 OP_QKV, OP_O, OP_GU, OP_DOWN, OP_LM, OP_ROUTER, OP_SGU, OP_RGU, OP_MDOWN = range(9)
+OP_MDQKV, OP_UQ, OP_UK, OP_UV, OP_MO = range(9, 14)
+T_MLA_ATTN = 2
 C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_ROUTE, C_PER_LAYER = range(7)
 WHOLE_ROW_OPS = (OP_LM, OP_ROUTER)   # aux holds the op's task count, not K-parts
 
@@ -52,17 +54,28 @@ def decode_tasks(tasks):
 MOE_SMALL = W.MOE4.replace(name="moe-small", n_layers=2, hidden=512, n_q_heads=8, n_kv_heads=2,
                           head_dim=64, prefill=40, n_experts=12, top_k=3, n_shared=1,
                           expert_ffn=200)
+MLA_SMALL = W.MLA4.replace(name="mla-small", n_layers=2, hidden=512, n_q_heads=32, q_lora=128,
+                          kv_lora=128, rope_dim=64, nope_dim=64, v_dim=64, prefill=100)
 PLAN_CASES = [
     (W.TINY, 148), (W.TINY, 7), (W.LLAMA8B, 148), (W.LLAMA8B, 132),
     (W.TINY.replace(n_q_heads=8, n_kv_heads=1, ffn=696, vocab=1001), 148),
     (W.TINY.replace(n_q_heads=4, n_kv_heads=4, head_dim=128, vocab=77), 33),
     (W.MOE4, 148), (MOE_SMALL, 148), (MOE_SMALL, 5),
     (MOE_SMALL.replace(n_shared=0, top_k=1), 19), (MOE_SMALL.replace(n_shared=2), 64),
+    (W.MLA4, 148), (MLA_SMALL, 148), (MLA_SMALL, 6),
 ]
 
 
 def rows_of_ops(wl):
     """Output rows of every GEMV op of one layer."""
+    if wl.kind == "mla":
+        H = wl.n_q_heads
+        rows = {OP_MDQKV: wl.q_lora + wl.kv_lora + wl.rope_dim,
+                OP_UQ: H * (wl.nope_dim + wl.rope_dim), OP_UK: H * wl.nope_dim,
+                OP_UV: H * wl.v_dim, OP_MO: wl.hidden}
+        if wl.vocab:
+            rows[OP_LM] = wl.vocab
+        return rows
     rows = {OP_QKV: (wl.n_q_heads + 2 * wl.n_kv_heads) * wl.head_dim, OP_O: wl.hidden}
     if wl.kind == "moe":
         rows.update({OP_ROUTER: wl.n_experts, OP_RGU: wl.top_k * wl.expert_ffn,
@@ -103,10 +116,13 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
         # every producer of a dependency precedes its consumer in global order
         assert all(T["id"][j] < T["id"][i] for j in producers)
         kind = dep % C_PER_LAYER
-        if T["type"][i] == T_GEMV and T["op"][i] == OP_O:
+        if T["type"][i] == T_GEMV and T["op"][i] == OP_UV:
+            # the MLA attention counter is bumped once per head group (its combine)
+            assert T["dep_count"][i] == wl.n_q_heads // 16
+        elif T["type"][i] == T_GEMV and T["op"][i] == OP_O:
             # the attention counter is bumped once per kv head (by the combining split)
             assert T["dep_count"][i] == wl.n_kv_heads
-        elif kind == C_ROUTE and dep < wl.n_layers * C_PER_LAYER:
+        elif wl.kind == "moe" and kind == C_ROUTE and dep < wl.n_layers * C_PER_LAYER:
             # the route counter is bumped once, by the router task that finishes last
             assert T["dep_count"][i] == 1
             assert producers and all(T["op"][j] == OP_ROUTER for j in producers)
@@ -165,10 +181,11 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
                     assert 0 <= r0 < r1 <= N
                     cover[r0:r1] += 1
                 assert (cover == 1).all(), (l, op, pt)
-        sel = (T["type"] == T_ATTN) & (T["layer"] == l)
+        sel = (T["type"] == (T_MLA_ATTN if wl.kind == "mla" else T_ATTN)) & (T["layer"] == l)
         pairs = Counter(zip(T["r0"][sel].tolist(), T["r1"][sel].tolist()))
         S = info.kv_splits
-        assert set(pairs) == {(g, s) for g in range(wl.n_kv_heads) for s in range(S)}
+        units = wl.n_q_heads // 16 if wl.kind == "mla" else wl.n_kv_heads
+        assert set(pairs) == {(g, s) for g in range(units) for s in range(S)}
         assert all(v == 1 for v in pairs.values())
         assert (T["aux"][sel] == S).all()
     # per layer, attention and MoE-down tasks are spread evenly: no SM holds more than
@@ -178,7 +195,8 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
         sm_of[T["id"][begin[q]:begin[q + 1]]] = q
     by_id = np.argsort(T["id"])
     for l in range(wl.n_layers):
-        for sel in ((T["type"] == T_ATTN), gemv & mdown):
+        for sel in ((T["type"] == T_ATTN), (T["type"] == T_MLA_ATTN), gemv & mdown,
+                    gemv & (T["op"] == OP_UK), gemv & (T["op"] == OP_UV)):
             ids = T["id"][sel & (T["layer"] == l)]
             if len(ids):
                 counts = np.bincount(sm_of[ids], minlength=nsm)
@@ -200,7 +218,8 @@ def test_llama8b_plan_is_byte_balanced():
 
 
 @pytest.mark.parametrize("field,value,status", [
-    ("kind", 1, tre.TRE_ERR_UNSUPPORTED), ("kind", 9, tre.TRE_ERR_INVALID_ARG),
+    ("kind", 1, tre.TRE_ERR_UNSUPPORTED),      # MLA with the GQA config's zero MLA dims
+    ("kind", 9, tre.TRE_ERR_INVALID_ARG),
     ("kind", 2, tre.TRE_ERR_UNSUPPORTED),      # MoE with n_experts = 0 (a GQA config)
     ("hidden", 260, tre.TRE_ERR_INVALID_ARG), ("n_kv_heads", 3, tre.TRE_ERR_INVALID_ARG),
     ("head_dim", 96, tre.TRE_ERR_UNSUPPORTED), ("ffn", 690, tre.TRE_ERR_INVALID_ARG),
@@ -240,6 +259,32 @@ def test_moe_plan_streams_only_the_selected_experts():
     nb = 148 // (wl.n_shared + wl.top_k)
     task = -(-wl.hidden // nb) * wl.expert_ffn * 2
     assert info.max_sm_bytes - info.min_sm_bytes <= task + 0.01 * info.min_sm_bytes
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("n_q_heads", 24, tre.TRE_ERR_UNSUPPORTED), ("kv_lora", 192, tre.TRE_ERR_UNSUPPORTED),
+    ("rope_dim", 24, tre.TRE_ERR_UNSUPPORTED), ("rope_dim", 32, tre.TRE_ERR_UNSUPPORTED),
+    ("kv_lora", 768, tre.TRE_ERR_UNSUPPORTED), ("v_dim", 12, tre.TRE_ERR_INVALID_ARG),
+    ("q_lora", 0, tre.TRE_ERR_INVALID_ARG),
+])
+def test_mla_plan_rejects_bad_configs(field, value, status):
+    import ctypes
+    cfg = tre.config_from_workload(MLA_SMALL, **{field: value})
+    info = tre.tre_plan_info()
+    assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status
+
+
+def test_mla_plan_bytes_and_stage():
+    wl = W.MLA4
+    info = tre.tre_plan_inspect(tre.config_from_workload(wl))
+    H, d, C = wl.n_q_heads, wl.hidden, wl.kv_lora + wl.rope_dim
+    w = ((wl.q_lora + C) * d + H * (wl.nope_dim + wl.rope_dim) * wl.q_lora +
+         H * wl.nope_dim * wl.kv_lora + H * wl.v_dim * wl.kv_lora + d * H * wl.v_dim)
+    assert info.weight_bytes == wl.n_layers * (w * 2 + (d + wl.q_lora + wl.kv_lora) * 2)
+    assert info.weight_bytes == pytest.approx(4 * 374.2e6, rel=0.01)
+    assert info.stage_bytes == C * 64          # one latent tile of 32 rows per stage
+    assert info.ring_stages >= 5
+    assert info.kv_bytes_at_capacity == wl.n_layers * wl.prefill * C * 2
 
 
 def test_reserved_fields_must_be_zero():

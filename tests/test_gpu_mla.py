@@ -1,0 +1,119 @@
+"""GPU parity of absorbed-MLA decoder layers (attention only) through the C ABI's
+layers-only step, against the fp64 CPU oracle.
+
+Bar: max relative error 2e-2 (normwise, max|gpu - oracle| / max|oracle|) on the hidden
+state after every layer.  The latent row each step appends is checked per row: within one
+bf16 ulp (2^-8) of the row's largest entry, since both sides round fp32 / fp64 values to
+bf16.  Each step feeds both sides the oracle's previous output.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from persistent_tile_pipelined_b200.synth import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from persistent_tile_pipelined_b200 import tre  # noqa: E402
+
+TOL = 2e-2
+ORC = oracle.Oracle(64)
+
+SMALL = W.MLA4.replace(name="mla-small", n_layers=2, hidden=512, n_q_heads=16, q_lora=128,
+                       kv_lora=128, rope_dim=64, nope_dim=64, v_dim=64, prefill=100,
+                       decode_steps=3, seed=77)
+
+
+def relerr(g, o):
+    g, o = np.asarray(g, np.float64), np.asarray(o, np.float64)
+    return float(np.abs(g - o).max() / max(np.abs(o).max(), 1e-30))
+
+
+def words_to_f64(w):
+    return (np.asarray(w, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def run_mla(wl, steps=1, **cfg_over):
+    model = W.gen_mla_model(wl)
+    dev = tre.upload_mla_model(model)
+    eng = tre.Engine(tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_HIDDEN, **cfg_over), dev)
+    caches = [c.copy() for c in model["latent_cache"]]
+    x = model["x_in"].astype(np.float64)
+    x_dev = torch.empty(wl.hidden, dtype=torch.float32, device="cuda")
+    out_dev = torch.empty(wl.hidden, dtype=torch.float32, device="cuda")
+    worst = 0.0
+    for step in range(steps):
+        pos = wl.prefill + step
+        x_dev.copy_(torch.from_numpy(x.astype(np.float32)))
+        eng.layers_step(x_dev, out_dev, pos)
+        torch.cuda.synchronize()
+        assert eng.status() == (0, 0)
+        hid = eng.hidden().cpu().numpy()
+        h = x
+        for l in range(wl.n_layers):
+            h = ORC.mla_layer_step(wl, model["layers"][l], caches[l], pos, h)
+            e = relerr(hid[l], h)
+            worst = max(worst, e)
+            assert e <= TOL, f"layer {l} hidden rel err {e:.3g} at pos {pos}"
+        assert np.array_equal(out_dev.cpu().numpy(), hid[-1])
+        x = h
+    start, end = wl.prefill, wl.prefill + steps
+    for l in range(wl.n_layers):
+        g = dev["k_cache"][l].view(torch.int16).cpu().numpy().view(np.uint16)
+        o = caches[l]
+        assert np.array_equal(g[:start], o[:start])
+        gv, ov = words_to_f64(g[start:end]), words_to_f64(o[start:end])
+        row_max = np.abs(ov).max(axis=-1, keepdims=True)
+        assert not (np.abs(gv - ov) > 2.0 ** -8 * row_max).any()
+    eng.close()
+    return worst
+
+
+@pytest.mark.parametrize("over,steps", [
+    (dict(), 3),                                                        # 1 head group, C 192
+    (dict(n_q_heads=32, kv_lora=256, nope_dim=128, v_dim=128, q_lora=256, hidden=1024,
+          n_layers=1), 2),                                              # 2 groups, C 320
+    (dict(kv_lora=512, nope_dim=128, v_dim=128, q_lora=512, hidden=1024, prefill=300,
+          n_layers=1), 2),                                              # C 576 (9 boxes)
+    (dict(prefill=0, decode_steps=2), 2),                               # pos 0: new row only
+    (dict(prefill=31, decode_steps=3), 3),                              # ragged last tile
+    (dict(rope_dim=128, kv_lora=128, n_layers=1), 1),                   # C 256, wider rope
+], ids=["h16-c192", "h32-c320", "c576", "pos0", "ragged", "rope128"])
+def test_mla_layers(over, steps):
+    run_mla(SMALL.replace(**over), steps=steps)
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(num_sms=5),
+    dict(kv_splits=1),
+    dict(num_sms=3, ring_stages=2),
+], ids=["sms5", "split1", "sms3-ring2"])
+def test_mla_launch_shapes(cfg):
+    run_mla(SMALL, steps=2, **cfg)
+
+
+@pytest.mark.slow
+def test_mla_full_size_four_layers():
+    """The full absorbed-MLA workload: hidden 7168, 128 heads, q_lora 1536, kv_lora 512,
+    rope 64, nope 128, v 128, 4 layers over 8192 cached latent rows."""
+    wl = W.MLA4
+    model = W.gen_mla_model(wl)
+    dev = tre.upload_mla_model(model)
+    eng = tre.Engine(tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_HIDDEN), dev)
+    x = model["x_in"].astype(np.float64)
+    x_dev = torch.from_numpy(x.astype(np.float32)).cuda()
+    out_dev = torch.empty_like(x_dev)
+    eng.layers_step(x_dev, out_dev, wl.prefill)
+    torch.cuda.synchronize()
+    assert eng.status() == (0, 0)
+    hid = eng.hidden().cpu().numpy()
+    h = x
+    for l in range(wl.n_layers):
+        h = ORC.mla_layer_step(wl, model["layers"][l], model["latent_cache"][l].copy(),
+                               wl.prefill, h)
+        assert relerr(hid[l], h) <= TOL
+    eng.close()
