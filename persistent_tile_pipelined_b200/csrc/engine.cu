@@ -901,11 +901,11 @@ __device__ __noinline__ void uk_task(const Params& p, const Task& t, const GemvG
 //   softmax: thread (head, 2 positions) scales to log2 units, masks rows past the split,
 //           updates the head's running max / sum and writes P as bf16 hi + lo;
 //   values: warp w accumulates O[16][KL / 8 columns] += P (hi + lo) x rows (ldmatrix.trans).
-// The split's (m, l, O) go to the partial buffer; the last split of the group to finish
-// (arrival ticket) combines the splits into o_lat.
+// The split's (m, l, O) go to the partial buffer and the split publishes; each head's
+// W_uv task merges the head's splits while it stages its input (mla_combine_input).
 __device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
                               uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
-                              int* flag, int warp, int lane, int ctid, bool& ab) {
+                              int warp, int lane, int ctid, bool& ab) {
   constexpr int HG = kMlaHeadGroup, PS = kMlaPosPerStage, RP = 36;  // score row pitch (floats)
   const int KL = p.KL, C = KL + p.R, hg = t.r0, split = t.r1, S = t.aux;
   const bool last = (split == S - 1);
@@ -952,9 +952,12 @@ __device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint3
   int t0, t1;
   attn_range(p, t, t0, t1);
   const uint32_t NS = (uint32_t)p.ring_stages;
+  long long waited = 0;  // trace: ns warp 0 spent waiting for stages to land
   for (int i = 0; i < ns; ++i) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
+    const long long w0 = p.trace ? (long long)globaltimer_ns() : 0;
     const bool landed = stage_wait(p, full, tags, sidx);
+    if (p.trace) waited += (long long)globaltimer_ns() - w0;
     const uint8_t* tile = ring + (size_t)slot * p.stage_bytes;
     const uint32_t tb = smem_u32(tile);
     // ---- partial scores over this warp's k-steps, 4 n-tiles of 8 rows
@@ -1066,7 +1069,10 @@ __device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint3
     if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
   }
   if (ab) return;
-  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
+  if (ctid == 0 && p.trace) {
+    p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
+    p.trace[(size_t)t.id * kTraceCols + 7] = waited;
+  }
 
   // ---- the new position (last split): score from lat_new, merged into (m, l, O)
   if (last) {
@@ -1110,7 +1116,7 @@ __device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint3
   }
 
   // ---- this split's partial: O (KL), m, l per head
-  const size_t pstride = (size_t)KL + 2;
+  const size_t pstride = (size_t)mla_pstride(KL);
 #pragma unroll
   for (int n = 0; n < 8; ++n) {
     if (n < nt_count) {
@@ -1131,40 +1137,57 @@ __device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint3
   __threadfence();
   consumer_sync(kConsumerThreads);
   if (ctid == 0) {
-    const uint32_t old = atom_acq_rel_gpu_add(p.tickets + hg, 1u);
-    *flag = ((old + 1u) % (uint32_t)S) == 0u;
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
+    red_release_gpu_add(p.counters + t.out, 1u);
+  }
+}
+
+// The W_uv task of head h stages o_lat_h, merging the head's KV splits on the way:
+// o_lat_h = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s (splits that saw no position
+// have m_s = -inf and weigh 0).  128 heads merge on 128 SMs at once.
+__device__ void mla_combine_input(const Params& p, const Task& t, float* ub, float* scratch,
+                                  int ctid) {
+  const int h = t.r0 / p.VD, KL = p.KL, S = p.nsplit;
+  const size_t pstride = (size_t)mla_pstride(KL);
+  const float* base = p.part + (size_t)h * S * pstride;
+  float* ms = scratch;       // [S] split weights 2^(m_s - M)
+  float* ls = scratch + S;  // [1] 1 / sum_s w_s l_s
+  for (int s2 = ctid; s2 < S; s2 += kConsumerThreads) ms[s2] = __ldcg(base + s2 * pstride + KL);
+  consumer_sync(kConsumerThreads);
+  if (ctid < 32) {
+    float M = -INFINITY;
+    for (int s2 = ctid; s2 < S; s2 += 32) M = fmaxf(M, ms[s2]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    for (int s2 = ctid; s2 < S; s2 += 32) {
+      const float w = ms[s2] == -INFINITY ? 0.f : exp2f(ms[s2] - M);
+      L = fmaf(w, __ldcg(base + s2 * pstride + KL + 1), L);
+      ms[s2] = w;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (ctid == 0) ls[0] = 1.f / L;
   }
   consumer_sync(kConsumerThreads);
-  if (*flag) {  // last split of the group: combine
-    float* ms = ub;               // [16][S]
-    float* ls = ub + HG * S;      // [16][S]
-    for (int idx = ctid; idx < HG * S; idx += kConsumerThreads) {
-      const float* src = p.part + ((size_t)(hg * HG) * S + idx) * pstride + KL;
-      ms[idx] = __ldcg(src);
-      ls[idx] = __ldcg(src + 1);
+  const float inv = ls[0];
+  float* xlo = ub;
+  float* xhi = ub + KL / 2;
+  for (int j = ctid; j < KL / 8; j += kConsumerThreads) {
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int s2 = 0; s2 < S; ++s2) {
+      const float w = ms[s2];
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(base + s2 * pstride + 8 * j));
+      const float4 b = __ldcg(reinterpret_cast<const float4*>(base + s2 * pstride + 8 * j + 4));
+      v[0] = fmaf(w, a.x, v[0]); v[1] = fmaf(w, a.y, v[1]); v[2] = fmaf(w, a.z, v[2]);
+      v[3] = fmaf(w, a.w, v[3]); v[4] = fmaf(w, b.x, v[4]); v[5] = fmaf(w, b.y, v[5]);
+      v[6] = fmaf(w, b.z, v[6]); v[7] = fmaf(w, b.w, v[7]);
     }
-    consumer_sync(kConsumerThreads);
-    for (int idx = ctid; idx < HG * KL; idx += kConsumerThreads) {
-      const int hh = idx / KL, cc = idx % KL;
-      const float* mh = ms + hh * S;
-      const float* lh = ls + hh * S;
-      float M = -INFINITY;
-      for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mh[s2]);
-      float L = 0.f, O = 0.f;
-      const float* src = p.part + (size_t)(hg * HG + hh) * S * pstride + cc;
-#pragma unroll 8
-      for (int s2 = 0; s2 < S; ++s2) {
-        const float w = mh[s2] == -INFINITY ? 0.f : exp2f(mh[s2] - M);
-        L = fmaf(w, lh[s2], L);
-        O = fmaf(w, __ldcg(src + s2 * pstride), O);
-      }
-      p.o_lat[(size_t)(hg * HG + hh) * KL + cc] = O / L;
-    }
-    __threadfence();
-    consumer_sync(kConsumerThreads);
-    if (ctid == 0) red_release_gpu_add(p.counters + t.out, 1u);
+    reinterpret_cast<float4*>(xlo)[j] = make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+    reinterpret_cast<float4*>(xhi)[j] = make_float4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
   }
+  consumer_sync(kConsumerThreads);
 }
 
 // ---- GEMV epilogue ---------------------------------------------------------------------------------
@@ -1263,6 +1286,9 @@ __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
 }
 
 // ---- consumers -----------------------------------------------------------------------------------
+// MLA = true: the absorbed-MLA stack's kernel (MLA tiles, no GQA attention); false: GQA /
+// MoE.  Two instantiations keep each kernel's register allocation to its own tiles.
+template <bool MLA>
 __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                          float* misc) {
@@ -1291,22 +1317,29 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     consumer_sync(kConsumerThreads);
     if (flags[0]) break;  // uniform: every consumer thread read the same flag
 
-    if (t.type == T_ATTN) {
+    if (!MLA && t.type == T_ATTN) {
       cur_key = -1;  // the attention scratch aliases the input-vector planes
-      run_attn(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
-    } else if (t.type == T_MLA_ATTN) {
+      if constexpr (!MLA)
+        run_attn(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
+    } else if (MLA && t.type == T_MLA_ATTN) {
       cur_key = -1;
-      mla_attn_task(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
-    } else if (t.op == OP_UK) {
+      if constexpr (MLA)
+        mla_attn_task(p, t, gs, ns, ring, full, empty, tags, ub, warp, lane, ctid, ab);
+    } else if (MLA && t.op == OP_UK) {
       cur_key = -1;
-      uk_task(p, t, gemv_geom(p, t), gs, ns, ring, full, empty, tags, ub, red, warp, lane, ctid, ab);
+      if constexpr (MLA)
+        uk_task(p, t, gemv_geom(p, t), gs, ns, ring, full, empty, tags, ub, red, warp, lane, ctid, ab);
     } else {
       const GemvGeom g = gemv_geom(p, t);
       const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
       const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MO;
       if (has_resid) prefetch_resid(p, t, g, resid, ctid);
-      if (key != cur_key || key < 0) {
+      if (MLA && t.op == OP_UV) {
+        if constexpr (MLA) mla_combine_input(p, t, ub, ub + p.xs_floats, ctid);
+        if (ctid == 0) *rn_s = 1.f;
+        cur_key = -1;
+      } else if (key != cur_key || key < 0) {
         const float rn = load_input(p, t, g, ub, red, ctid);
         if (ctid == 0) *rn_s = rn;
         cur_key = key;
@@ -1423,6 +1456,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
 }
 
 // ---- the kernel ----------------------------------------------------------------------------------
+template <bool MLA>
 __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t NS = (uint32_t)p.ring_stages;
@@ -1456,19 +1490,18 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
     producer(p, my, ntask, ring, full, empty, tags, threadIdx.x & 31);
     return;
   }
-  consumer(p, my, ntask, ring, full, empty, tags, ub, misc);
+  consumer<MLA>(p, my, ntask, ring, full, empty, tags, ub, misc);
 }
 
 // ---- host-side launch helpers ------------------------------------------------------------------
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm) {
-  cudaError_t e = cudaFuncSetAttribute(engine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem_bytes);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla) {
+  auto k = mla ? engine_kernel<true> : engine_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return e;
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, engine_kernel, kThreads,
-                                                       smem_bytes);
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, k, kThreads, smem_bytes);
 }
 
-cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream) {
+cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream, bool mla) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -1479,7 +1512,8 @@ cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, engine_kernel, p);
+  return mla ? cudaLaunchKernelEx(&cfg, engine_kernel<true>, p)
+             : cudaLaunchKernelEx(&cfg, engine_kernel<false>, p);
 }
 
 }  // namespace tre

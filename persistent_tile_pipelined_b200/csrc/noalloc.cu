@@ -21,8 +21,9 @@
 #include "tre_internal.h"
 
 namespace tre {
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm);
-cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla = false);
+cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
+                          bool mla = false);
 }  // namespace tre
 
 using namespace tre;

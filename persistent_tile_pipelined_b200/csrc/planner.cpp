@@ -400,7 +400,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     const int n3 = b.per_unit(OP_UK, l, H, s.NP, (int64_t)s.NP * s.KL * 2, cuq, (uint32_t)n2, cuk);
     const int64_t lat_task = (int64_t)(s.cap - s.M) / S * C * 2;
     b.mla_attention(l, groups, S, lat_task, cuk, (uint32_t)n3, ca);
-    const int n5 = b.per_unit(OP_UV, l, H, s.VD, (int64_t)s.VD * s.KL * 2, ca, (uint32_t)groups, cuv);
+    const int n5 = b.per_unit(OP_UV, l, H, s.VD, (int64_t)s.VD * s.KL * 2, ca,
+                              (uint32_t)(groups * S), cuv);
     const int n6 = b.gemv(OP_MO, l, s.d, H * s.VD, 1, cuv, (uint32_t)n5, co, s.resid_floats);
     prev_down = co;
     prev_down_count = (uint32_t)n6;

@@ -17,8 +17,9 @@
 #include "tre_internal.h"
 
 namespace tre {
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm);
-cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla = false);
+cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
+                          bool mla = false);
 const char* last_error_cstr();
 }  // namespace tre
 
@@ -246,7 +247,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   }
 
   int bps = 0;
-  CK(engine_configure(s.smem_bytes, &bps));
+  CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA));
   if (bps < 1) {
     set_error("tre_create: the persistent CTA does not fit on an SM");
     return TRE_ERR_OCCUPANCY;
@@ -287,7 +288,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_rtick = cv.take<uint32_t>(1);
   size_t o_mpart = cv.take<float>(moe ? (size_t)(s.nshared + s.topk) * s.d : 1);
   size_t o_dtick = cv.take<uint32_t>(moe ? s.down_blocks : 1);
-  size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * ((mla ? s.KL : s.D) + 2));
+  size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (mla ? mla_pstride(s.KL) : s.D + 2));
   size_t o_logits = cv.take<float>(s.V > 0 ? s.V : 1);
   size_t o_tok = cv.take<int32_t>(1);
   size_t o_inv = cv.take<double>(std::max(1, s.D / 2));
@@ -433,7 +434,8 @@ static tre_status launch_step(tre_engine* e, int32_t token, int32_t pos, cudaStr
   p.token_out = token_dev ? token_dev : e->token_buf;
   p.x_in = x_in;
   p.x_out = x_out;
-  cudaError_t ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream);
+  cudaError_t ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream,
+                                 e->shape.kind == TRE_LAYER_MLA);
   if (ce != cudaSuccess) {
     --e->epoch;
     return cuda_fail(ce, "launch of the persistent engine");

@@ -81,6 +81,8 @@ constexpr int kMlaHeadGroup = 16;     // query heads per MLA attention tile (the
 constexpr int kMlaPosPerStage = 32;   // latent rows per MLA attention stage
 constexpr int kMlaBox = 64;           // latent columns per tensor-map box (128 B, swizzled)
 constexpr int kMlaMaxKSteps = 6;      // 16-column k-steps of the score product per warp
+// floats per MLA split partial: O (KL), m, l, 2 pad -> every row starts on 16 bytes
+TRE_HD inline int mla_pstride(int KL) { return KL + 4; }
 
 // Dependency counters: one per (layer, stage of the layer), then the LM head and a
 // counter nothing ever bumps (used only by the fault-injection debug plan).

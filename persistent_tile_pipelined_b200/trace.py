@@ -14,7 +14,8 @@ from collections import defaultdict
 import numpy as np
 
 OP_NAMES = {0: "qkv", 1: "o_proj", 2: "gate_up", 3: "down", 4: "lm_head", 5: "router",
-            6: "shared_gate_up", 7: "routed_gate_up", 8: "moe_down"}
+            6: "shared_gate_up", 7: "routed_gate_up", 8: "moe_down", 9: "mla_down",
+            10: "q_up", 11: "uk", 12: "uv", 13: "mla_o"}
 
 
 def task_table(tasks: np.ndarray) -> dict:
@@ -27,7 +28,11 @@ def task_table(tasks: np.ndarray) -> dict:
 
 
 def op_name(tt: dict, i: int) -> str:
-    return "attention" if tt["type"][i] == 1 else OP_NAMES.get(int(tt["op"][i]), "?")
+    if tt["type"][i] == 1:
+        return "attention"
+    if tt["type"][i] == 2:
+        return "mla_attention"
+    return OP_NAMES.get(int(tt["op"][i]), "?")
 
 
 def summarize(trace: np.ndarray, tasks: np.ndarray) -> dict:

@@ -117,8 +117,8 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
         assert all(T["id"][j] < T["id"][i] for j in producers)
         kind = dep % C_PER_LAYER
         if T["type"][i] == T_GEMV and T["op"][i] == OP_UV:
-            # the MLA attention counter is bumped once per head group (its combine)
-            assert T["dep_count"][i] == wl.n_q_heads // 16
+            # every MLA attention split publishes; W_uv merges a head's splits
+            assert T["dep_count"][i] == (wl.n_q_heads // 16) * info.kv_splits
         elif T["type"][i] == T_GEMV and T["op"][i] == OP_O:
             # the attention counter is bumped once per kv head (by the combining split)
             assert T["dep_count"][i] == wl.n_kv_heads
