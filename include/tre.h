@@ -206,7 +206,8 @@ tre_status tre_decode_step_host(tre_engine* e, int32_t token, int32_t pos, tre_s
  * byte, real-time loops where allocation is forbidden, plug-ins handed only raw
  * pointers — so no engine is created: each call plans the step on the host (ordinary CPU
  * memory) and keeps everything the kernel needs beyond the caller's tensors (task list,
- * counters, activations, split-KV partials) in one fixed device array built into the
+ * tensor maps of the KV caches, counters, activations, split-KV partials) in one fixed
+ * device array built into the
  * library, 4 MiB per GPU, held by every GPU that loads the library until the process exits.
  * The call allocates no GPU memory: no cudaMalloc / cudaMallocAsync / cudaHostAlloc and no
  * cudaFree.

@@ -267,8 +267,7 @@ __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, 
   }
   if (t.type == T_MLA_ATTN)  // whole boxes (rows past the cache are zero-filled)
     return (uint32_t)((p.KL + p.R) / kMlaBox * kMlaPosPerStage * 128);
-  const int n = min(p.pps, t1 - (t0 + i * p.pps));
-  return (uint32_t)(2 * n * p.D * 2);
+  return (uint32_t)(2 * (p.D / 64) * p.pps * 128);  // K and V boxes of pps rows
 }
 
 // Issue the bulk copies of stage i into `dst`: one copy per contiguous run of rows (per
@@ -317,22 +316,25 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
   } else if (t.type == T_MLA_ATTN) {
     // 64-column boxes of 32 latent rows, 128-byte swizzled (see mla.cuh)
     if (lane < (p.KL + p.R) / kMlaBox) {
-      const uint8_t* map = static_cast<const uint8_t*>(p.mla_maps) + (size_t)t.layer * 128;
+      const uint8_t* map = static_cast<const uint8_t*>(p.kv_maps) + (size_t)t.layer * 128;
       tma_load_2d(dst + (size_t)lane * kMlaPosPerStage * 128, map, lane * kMlaBox,
                   t0 + i * kMlaPosPerStage, bar);
     }
-  } else if (lane < 2) {
-    const int tt = t0 + i * p.pps, n = min(p.pps, t1 - tt);
-    const size_t rowb = (size_t)p.D * 2;
-    const LayerPtrs& L = p.layers[t.layer];
-    const uint16_t* base = lane == 0 ? L.k_cache : L.v_cache;
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(base) + ((size_t)t.r0 * p.cap + tt) * rowb;
-    bulk_g2s(dst + (size_t)lane * p.pps * rowb, src, (uint32_t)(n * rowb), bar, pol);
+  } else {
+    // K then V: 64-column boxes of pps rows of kv head r0 (rows of the caches viewed as
+    // [Hkv * capacity][D]; rows past the split are masked by the consumer)
+    const int kb = p.D / 64;
+    if (lane < 2 * kb) {
+      const uint8_t* map = static_cast<const uint8_t*>(p.kv_maps) +
+                           ((size_t)t.layer * 2 + (lane >= kb)) * 128;
+      tma_load_2d(dst + (size_t)lane * p.pps * 128, map, (lane % kb) * 64,
+                  t.r0 * p.cap + t0 + i * p.pps, bar);
+    }
   }
 }
 
-// L2 prefetch of a whole task ahead of its stages: the contiguous byte ranges task t will
-// stream (its rows of each matrix; or the K and V rows of its positions), as a few large
+// L2 prefetch of a whole GEMV task ahead of its stages: the contiguous byte ranges task t
+// will stream (its rows of each matrix), as a few large
 // requests — a bulk request costs the same fixed time whatever its size, so one request
 // per range rather than one per stage.  At most `budget` bytes; K-part tasks (strided rows)
 // are skipped.
@@ -340,8 +342,8 @@ __device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, in
                                               long long budget) {
   const uint8_t* src[3] = {nullptr, nullptr, nullptr};
   long long bytes[3] = {0, 0, 0};
-  if (t.type == T_MLA_ATTN) return;  // latent tiles come through the tensor map
-  if (t.type == T_GEMV) {
+  if (t.type != T_GEMV) return;  // KV tiles come through the tensor maps
+  {
     const GemvGeom g = gemv_geom(p, t);
     if (g.np > 1 || needs_route(p, t)) return;  // strided rows, or addresses not known yet
     const size_t rowb = (size_t)g.K * 2;
@@ -362,15 +364,6 @@ __device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, in
         left -= take;
       }
     }
-  } else {
-    int t0, t1;
-    attn_range(p, t, t0, t1);
-    const size_t rowb = (size_t)p.D * 2;
-    const LayerPtrs& L = p.layers[t.layer];
-    const size_t off = ((size_t)t.r0 * p.cap + t0) * rowb;
-    src[0] = reinterpret_cast<const uint8_t*>(L.k_cache) + off;
-    src[1] = reinterpret_cast<const uint8_t*>(L.v_cache) + off;
-    bytes[0] = bytes[1] = (long long)(t1 - t0) * rowb;
   }
   if (lane < 3 && src[lane]) {
     long long before = 0;  // budget left after the pieces of lower lanes
@@ -576,11 +569,10 @@ __device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float&
 // position pos from this step's k / v, appends them to the caches and merges its partial.
 // The last split of the group to finish (arrival ticket) combines all splits — the fused
 // combine — and publishes the group.
-template <int G, int DPL>
+template <int G, int D>
 __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
                           uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                           int* flag, int warp, int lane, int ctid, bool& abort_out) {
-  constexpr int D = 32 * DPL;
   const int g = t.r0, split = t.r1, S = t.aux;
   const bool last = (split == S - 1);
   float* q_s = ub;                            // [G][D] roped, scaled
@@ -635,47 +627,114 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     if (lane == 0) sn[warp] = a;
   }
 
-  float q[G][DPL], m[G], l[G], o[G][DPL];
+  // ---- tensor-core flash-decode over the split's cached positions
+  // One 16-row A tile carries the group's G <= 8 query heads twice: row h holds head h's
+  // bf16 hi part and row h + 8 its lo part, so S = Q K^T for head h is the sum of the
+  // accumulator rows h and h + 8 — which the same thread holds (c0 + c2, c1 + c3).  P and
+  // the value product use the same packing.  A stage holds 64 positions of K then V as
+  // 64-column swizzled boxes; the 8 warps form two groups taking alternate stages, and warp
+  // (group, quarter) owns positions 16 quarter .. 16 quarter + 15 of its stages with its own
+  // running (m, l, O).  P goes from the score registers straight into the A operand of
+  // O += P V (the m16n8 accumulator layout of two n-tiles is the m16k16 A layout).
+  // Positions past the split are masked (score -inf, value 0).
+  constexpr int KS = D / 16, NT = D / 8, KB = D / 64;  // k-steps, output n-tiles, boxes
+  const int g8 = lane >> 2, t4 = lane & 3;
+  const bool real = g8 < G;
+  uint32_t qa[KS][4];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int j = 0; j < DPL; ++j) {
-      q[h][j] = q_s[h * D + lane * DPL + j];
-      o[h][j] = 0.f;
-    }
+  for (int ks = 0; ks < KS; ++ks) {
+    const int k0 = ks * 16 + 2 * t4;
+    const float* qr = q_s + (real ? g8 : 0) * D;
+    split_pair(real ? qr[k0] : 0.f, real ? qr[k0 + 1] : 0.f, qa[ks][0], qa[ks][1]);
+    split_pair(real ? qr[k0 + 8] : 0.f, real ? qr[k0 + 9] : 0.f, qa[ks][2], qa[ks][3]);
   }
+  float m0 = -INFINITY, l0 = 0.f;   // head g8
+  float o[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   const uint32_t NS = (uint32_t)p.ring_stages;
   int t0, t1;
   attn_range(p, t, t0, t1);
-  // a stage of pps positions is taken by wps warps (8 positions each); the 8 warps form
-  // 8 / wps groups that consume alternate stages
-  const int wps = p.pps / kPosPerWarp, ngrp = kConsumerWarps / wps;
-  const int grp = warp / wps, wpos = (warp % wps) * kPosPerWarp;
-  for (int i = grp; i < ns; i += ngrp) {
+  const int grp = warp >> 2, r0 = (warp & 3) * 16;
+  for (int i = grp; i < ns; i += 2) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
     if (!stage_wait(p, full, tags, sidx)) {
       abort_out = true;
       break;
     }
-    const int n = min(p.pps, t1 - (t0 + i * p.pps));
-    const int nw = min(kPosPerWarp, n - wpos);
-    if (nw > 0) {
-      const uint8_t* kb = ring + (size_t)slot * p.stage_bytes + (size_t)wpos * D * 2;
-      attn_warp_positions<G, DPL>(kb, kb + (size_t)p.pps * D * 2, nw, q, m, l, o, lane);
+    const int valid = min(16, t1 - (t0 + i * p.pps) - r0);
+    if (valid > 0) {
+      const uint32_t tb = smem_u32(ring + (size_t)slot * p.stage_bytes);
+      const int m = lane >> 3;
+      float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int r = r0 + (m >> 1) * 8 + (lane & 7), ch = ks * 2 + (m & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(tb + swz_off(ch >> 3, r, ch & 7, 64), b0, b1, b2, b3);
+        mma_bf16(c[0], qa[ks], b0, b1);
+        mma_bf16(c[1], qa[ks], b2, b3);
+      }
+      // scores of head g8 (hi rows + lo rows); mask positions past the split
+      float sc[2][2];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          sc[n][j] = (n * 8 + 2 * t4 + j < valid) ? c[n][j] + c[n][j + 2] : -INFINITY;
+      float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mn = fmaxf(m0, mx);          // finite: valid > 0
+      const float a0 = exp2f(m0 - mn);          // 0 while m0 = -inf
+      float pv[2][2];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) pv[n][j] = exp2f(sc[n][j] - mn);
+      l0 = l0 * a0 + (pv[0][0] + pv[0][1] + pv[1][0] + pv[1][1]);
+      m0 = mn;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] *= a0;
+        o[n][1] *= a0;
+        o[n][2] *= a0;
+        o[n][3] *= a0;
+      }
+      uint32_t pa[4];
+      split_pair(pv[0][0], pv[0][1], pa[0], pa[1]);
+      split_pair(pv[1][0], pv[1][1], pa[2], pa[3]);
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        const int r = r0 + (m & 1) * 8 + (lane & 7), ch = np * 2 + (m >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(tb + swz_off(KB + (ch >> 3), r, ch & 7, 64), b0, b1, b2, b3);
+        if (valid < 16) {  // value rows past the split may hold anything: zero them
+          const int pa0 = 2 * t4, pb0 = 8 + 2 * t4;
+          if (pa0 >= valid) { b0 &= 0xffff0000u; b2 &= 0xffff0000u; }
+          if (pa0 + 1 >= valid) { b0 &= 0x0000ffffu; b2 &= 0x0000ffffu; }
+          if (pb0 >= valid) { b1 &= 0xffff0000u; b3 &= 0xffff0000u; }
+          if (pb0 + 1 >= valid) { b1 &= 0x0000ffffu; b3 &= 0x0000ffffu; }
+        }
+        mma_bf16(o[2 * np], pa, b0, b1);
+        mma_bf16(o[2 * np + 1], pa, b2, b3);
+      }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive_n(&empty[slot], (uint32_t)(kConsumerWarps / wps));
+    if (lane == 0) mbar_arrive_n(&empty[slot], 2u);  // 4 warps per stage, 8 arrivals
   }
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    if (lane == 0) {
-      mw[warp * G + h] = m[h];
-      lw[warp * G + h] = l[h];
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  if (g8 < G) {
+    if (t4 == 0) {
+      mw[warp * G + g8] = m0;
+      lw[warp * G + g8] = l0;
     }
 #pragma unroll
-    for (int j = 0; j < DPL; ++j) ow[(warp * G + h) * D + lane * DPL + j] = o[h][j];
+    for (int n = 0; n < NT; ++n) {  // hi rows + lo rows
+      ow[(warp * G + g8) * D + n * 8 + 2 * t4] = o[n][0] + o[n][2];
+      ow[(warp * G + g8) * D + n * 8 + 2 * t4 + 1] = o[n][1] + o[n][3];
+    }
   }
   consumer_sync(kConsumerThreads);
   if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
@@ -716,8 +775,9 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   __threadfence();
   consumer_sync(kConsumerThreads);
   if (ctid == 0) {
-    const uint32_t old = atom_acq_rel_gpu_add(p.tickets + g, 1u);
+    const uint32_t old = ticket_add(p.tickets + g, 1u);
     *flag = ((old + 1u) % (uint32_t)S) == 0u;
+    if (*flag) fence_acq_rel_gpu();
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
   }
   consumer_sync(kConsumerThreads);
@@ -750,7 +810,7 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     }
     __threadfence();
     consumer_sync(kConsumerThreads);
-    if (ctid == 0) red_release_gpu_add(p.counters + t.out, 1u);
+    if (ctid == 0) publish_add(p.counters + t.out, 1u);
   }
 }
 
@@ -763,17 +823,17 @@ __device__ __forceinline__ void run_attn(const Params& p, const Task& t, uint32_
   attn_task<GG, DD>(p, t, gs, ns, ring, full, empty, tags, ub, flag, warp, lane, ctid, ab)
   if (p.D == 128) {
     switch (G) {
-      case 1: TRE_ATTN(1, 4); break;
-      case 2: TRE_ATTN(2, 4); break;
-      case 4: TRE_ATTN(4, 4); break;
-      default: TRE_ATTN(8, 4); break;
+      case 1: TRE_ATTN(1, 128); break;
+      case 2: TRE_ATTN(2, 128); break;
+      case 4: TRE_ATTN(4, 128); break;
+      default: TRE_ATTN(8, 128); break;
     }
   } else {
     switch (G) {
-      case 1: TRE_ATTN(1, 2); break;
-      case 2: TRE_ATTN(2, 2); break;
-      case 4: TRE_ATTN(4, 2); break;
-      default: TRE_ATTN(8, 2); break;
+      case 1: TRE_ATTN(1, 64); break;
+      case 2: TRE_ATTN(2, 64); break;
+      case 4: TRE_ATTN(4, 64); break;
+      default: TRE_ATTN(8, 64); break;
     }
   }
 #undef TRE_ATTN
@@ -889,7 +949,7 @@ __device__ __noinline__ void uk_task(const Params& p, const Task& t, const GemvG
   }
   __threadfence();
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) red_release_gpu_add(p.counters + t.out, 1u);
+  if (ctid == 0) publish_add(p.counters + t.out, 1u);
 }
 
 // ---- absorbed MLA: latent attention on tensor cores ---------------------------------------------
@@ -1138,7 +1198,7 @@ __device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint3
   consumer_sync(kConsumerThreads);
   if (ctid == 0) {
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
-    red_release_gpu_add(p.counters + t.out, 1u);
+    publish_add(p.counters + t.out, 1u);
   }
 }
 
@@ -1266,7 +1326,7 @@ __device__ void route_topk(const Params& p, int layer, float* sc, int warp, int 
   if (lane < p.topk) p.route_w[layer * p.topk + lane] = mine / tot;
   __threadfence();
   __syncwarp();
-  if (lane == 0) red_release_gpu_add(p.counters + layer * C_PER_LAYER + C_ROUTE, 1u);
+  if (lane == 0) publish_add(p.counters + layer * C_PER_LAYER + C_ROUTE, 1u);
 }
 
 // The last slot of a MoE-down row block to finish: x = h1 + sum of the slots' partial rows
@@ -1282,7 +1342,7 @@ __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
   }
   __threadfence();
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) red_release_gpu_add(p.counters + t.out, 1u);
+  if (ctid == 0) publish_add(p.counters + t.out, 1u);
 }
 
 // ---- consumers -----------------------------------------------------------------------------------
@@ -1426,28 +1486,31 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         for (int w = 0; w < kConsumerWarps; ++w) best_update(bb, red[w], reinterpret_cast<int*>(red)[16 + w]);
         atomicMax(p.argmax_slot, pack_best(bb));
         __threadfence();
-        const uint32_t old = atom_acq_rel_gpu_add(p.lm_ticket, 1u);
+        const uint32_t old = ticket_add(p.lm_ticket, 1u);
         if (((old + 1u) % (uint32_t)t.aux) == 0u) {
+          fence_acq_rel_gpu();
           const unsigned long long w = atomicExch(p.argmax_slot, 0ull);
           if (p.token_out) *p.token_out = (int32_t)(0xffffffffu - (uint32_t)(w & 0xffffffffull));
         }
       }
       if (t.op == OP_ROUTER) {  // the last router task of the layer selects the experts
         if (ctid == 0) {
-          const uint32_t old = atom_acq_rel_gpu_add(p.router_ticket, 1u);
+          const uint32_t old = ticket_add(p.router_ticket, 1u);
           flags[1] = ((old + 1u) % (uint32_t)t.aux) == 0u;
+          if (flags[1]) fence_acq_rel_gpu();
         }
         consumer_sync(kConsumerThreads);
         if (flags[1]) route_topk(p, t.layer, ub + p.xs_floats, warp, lane, ctid);
       } else if (t.op == OP_MDOWN) {  // the block's last slot sums the partial rows
         if (ctid == 0) {
-          const uint32_t old = atom_acq_rel_gpu_add(p.down_tickets + (t.aux >> 8), 1u);
+          const uint32_t old = ticket_add(p.down_tickets + (t.aux >> 8), 1u);
           flags[1] = ((old + 1u) % (uint32_t)(p.nshared + p.topk)) == 0u;
+          if (flags[1]) fence_acq_rel_gpu();
         }
         consumer_sync(kConsumerThreads);
         if (flags[1]) moe_down_combine(p, t, ctid);
       } else if (ctid == 0 && t.out >= 0) {
-        red_release_gpu_add(p.counters + t.out, 1u);
+        publish_add(p.counters + t.out, 1u);
       }
     }
     if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 2] = (long long)globaltimer_ns();

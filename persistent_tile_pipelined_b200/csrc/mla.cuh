@@ -1,5 +1,5 @@
-// Absorbed-MLA tiles of the persistent engine: the per-head W_uk contraction and the
-// latent attention on tensor cores.
+// Tensor-core helpers of the persistent engine (mma.sync, ldmatrix, swizzled tensor-map
+// tiles) used by the GQA flash-decode tile and the absorbed-MLA latent attention.
 //
 // Absorbed MLA (DeepSeek-V2's; the pages name the fused kernel FlashSparseMLA with
 // batch == 1 — TileRT code audit, blog-vs-code table — and fold the query heads of a
@@ -61,9 +61,15 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   lo = bf2_bits(__floats2bfloat162_rn(x0 - hf.x, x1 - hf.y));
 }
 
+// Byte offset of 16-byte chunk c (0..7) of row r of box b in a stage of `rows`-row boxes
+// of 64 bf16 columns, as the 128-byte swizzle lays them out (boxes 1024-byte aligned).
+__device__ __forceinline__ uint32_t swz_off(int b, int r, int c, int rows) {
+  return (uint32_t)(b * rows * 128 + r * 128 + ((c ^ (r & 7)) << 4));
+}
+
 // Byte offset of 16-byte chunk `ch` (columns 8 ch .. 8 ch + 7) of row r of a latent stage.
 __device__ __forceinline__ uint32_t lat_off(int r, int ch) {
-  return (uint32_t)((ch >> 3) * (kMlaPosPerStage * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+  return swz_off(ch >> 3, r, ch & 7, kMlaPosPerStage);
 }
 
 // 2-D tensor copy of one box into shared memory, completing on `bar`.

@@ -135,6 +135,8 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   const size_t o_u = cv.take<float>(s.F);
   const size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (s.D + 2));
   const size_t o_inv = cv.take<double>(s.D / 2);
+  cv.off = (cv.off + 127) & ~size_t(127);
+  const size_t o_maps = cv.take<uint8_t>((size_t)2 * s.L * 128);  // K and V tensor maps
   if (cv.off > kStaticScratchBytes)
     return fail(TRE_ERR_UNSUPPORTED,
                 "tre_decode_step_static: this model needs " + std::to_string(cv.off) +
@@ -165,6 +167,17 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
     lp[l].v_cache = static_cast<uint16_t*>(w->v_cache[l]);
   }
 
+  // tensor maps over the K and V caches, built on the host (no allocation)
+  std::vector<uint8_t> maps((size_t)2 * s.L * 128);
+  for (int l = 0; l < s.L; ++l) {
+    st = encode_cache_map(w->k_cache[l], s.D, (long long)s.Hkv * s.cap, s.pos_per_stage,
+                          maps.data() + (size_t)2 * l * 128);
+    if (st == TRE_OK)
+      st = encode_cache_map(w->v_cache[l], s.D, (long long)s.Hkv * s.cap, s.pos_per_stage,
+                            maps.data() + (size_t)(2 * l + 1) * 128);
+    if (st != TRE_OK) return st;
+  }
+
   void* scratch = nullptr;
   st = setup_device(dev, &scratch);
   if (st != TRE_OK) return st;
@@ -182,6 +195,8 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
                             cudaMemcpyHostToDevice, sm)) != cudaSuccess ||
       (ce = cudaMemcpyAsync(B + o_inv, inv.data(), inv.size() * sizeof(double),
                             cudaMemcpyHostToDevice, sm)) != cudaSuccess ||
+      (ce = cudaMemcpyAsync(B + o_maps, maps.data(), maps.size(), cudaMemcpyHostToDevice, sm)) !=
+          cudaSuccess ||
       (ce = cudaMemsetAsync(B + o_zero, 0, o_zero_end - o_zero, sm)) != cudaSuccess)
     return cuda_fail(ce, "filling the static scratch");
   if (status_dev && (ce = cudaMemsetAsync(status_dev, 0, 2 * sizeof(int32_t), sm)) != cudaSuccess)
@@ -209,6 +224,7 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   p.logits = logits_dev;
   p.token_out = token_dev;
   p.rope_inv_freq = reinterpret_cast<const double*>(B + o_inv);
+  p.kv_maps = B + o_maps;
   p.err = reinterpret_cast<int32_t*>(B + o_err);
   p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
   p.status_host = status_dev ? status_dev : reinterpret_cast<int32_t*>(B + o_err + 8);

@@ -323,8 +323,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     ops.push_back({s.d, 2, 0});
     ops.push_back({s.F, 1, 0});
   }
-  // a stage holds at least 8 KV positions (GQA) or one MLA attention tile
-  int xs = 8, need = mla ? (s.KL + s.R) * kMlaPosPerStage * 2 : 4 * s.D * 8;
+  // a stage holds one attention tile: 64 K and V rows (GQA) or 32 latent rows (MLA)
+  int xs = 8, need = mla ? (s.KL + s.R) * kMlaPosPerStage * 2 : 4 * s.D * kMaxPosPerStage;
   for (auto& o : ops) {
     const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max));
     xs = std::max(xs, kp);
@@ -338,13 +338,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   if (sb < need)
     return fail(TRE_ERR_UNSUPPORTED, "a weight row part (or gate/up row pair) is wider than a ring stage");
   s.stage_bytes = sb;
-  int pps = 8;  // a power of two, so that every warp of a stage group takes 8 positions
-  if (mla) {
-    pps = kMlaPosPerStage;
-  } else {
-    while (pps * 2 <= kMaxPosPerStage && pps * 2 * 4 * s.D <= sb) pps *= 2;
-  }
-  s.pos_per_stage = pps;
+  // positions per attention stage: MLA 32 latent rows; GQA 64 (four warps x 16 rows)
+  s.pos_per_stage = mla ? kMlaPosPerStage : kMaxPosPerStage;
 
   s.xs_floats = (xs + 7) / 8 * 8;
   s.resid_floats = kMaxResidRows;
@@ -375,7 +370,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   int S = c.kv_splits;
   if (!S) {
     S = std::max(1, nsm / units);
-    int max_s = std::max(1, (s.cap - 1 + s.pos_per_stage - 1) / s.pos_per_stage);
+    int max_s = std::max(1, (s.cap - 1 + s.pos_per_stage - 1) / s.pos_per_stage);  // >= 1 stage each
     S = std::min(S, max_s);
   }
   // the combine stages every split's (m, l) in the attention scratch: 2 G S <= 8 G D

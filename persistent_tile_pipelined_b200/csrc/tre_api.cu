@@ -62,33 +62,36 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-static tre_status encode_latent_map(void* cache, int C, int cap, CUtensorMap* out) {
+// A cache [rows][C] bf16 as a 2-D tensor; boxes of 64 columns x box_rows rows with the
+// 128-byte swizzle the attention tiles read (rows past the cache read as zero).
+namespace tre {
+tre_status encode_cache_map(void* cache, int C, long long rows, int box_rows, void* out128) {
+  CUtensorMap* out = static_cast<CUtensorMap*>(out128);
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
     if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) {
-      set_error("tre_create: cuTensorMapEncodeTiled is not available");
+      set_error("cuTensorMapEncodeTiled is not available");
       return TRE_ERR_CUDA;
     }
     fn = reinterpret_cast<EncodeTiledFn>(f);
   }
-  // the latent cache [cap][C] bf16 as a 2-D tensor; boxes of 64 columns x 32 rows with the
-  // 128-byte swizzle the MLA tiles read (rows past the cache read as zero)
-  const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)cap};
+  const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)C * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kMlaBox, (cuuint32_t)kMlaPosPerStage};
+  const cuuint32_t box[2] = {(cuuint32_t)kMlaBox, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cache, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
-    set_error("tre_create: cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
+    set_error("cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
     return TRE_ERR_CUDA;
   }
   return TRE_OK;
 }
+}  // namespace tre
 
 namespace {
 struct Carve {  // bump allocator over the engine's single device block
@@ -262,9 +265,16 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   // ---- one device block for all engine-owned state
   const int qkv_n = mla ? s.Hq * (s.NP + s.R) : (s.Hq + 2 * s.Hkv) * s.D;
   const int C = s.KL + s.R;
-  std::vector<CUtensorMap> maps(mla ? s.L : 0);
-  for (int l = 0; l < (mla ? s.L : 0); ++l) {
-    tre_status ms = encode_latent_map(w->k_cache[l], C, s.cap, &maps[l]);
+  // MLA: one map per layer over the latent cache; GQA / MoE: K and V maps per layer over
+  // the caches viewed as [Hkv * capacity][D]
+  std::vector<CUtensorMap> maps(mla ? s.L : 2 * s.L);
+  for (int l = 0; l < s.L; ++l) {
+    tre_status ms = mla ? encode_cache_map(w->k_cache[l], C, s.cap, kMlaPosPerStage, &maps[l])
+                        : encode_cache_map(w->k_cache[l], s.D, (long long)s.Hkv * s.cap,
+                                           s.pos_per_stage, &maps[2 * l]);
+    if (ms == TRE_OK && !mla)
+      ms = encode_cache_map(w->v_cache[l], s.D, (long long)s.Hkv * s.cap, s.pos_per_stage,
+                            &maps[2 * l + 1]);
     if (ms != TRE_OK) return ms;
   }
   Carve cv;
@@ -385,7 +395,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.lat_new = reinterpret_cast<float*>(B + o_latn);
   p.o_lat = reinterpret_cast<float*>(B + o_olat);
   p.mla_o = reinterpret_cast<float*>(B + o_mlao);
-  p.mla_maps = B + o_maps;
+  p.kv_maps = B + o_maps;
   p.QL = s.QL; p.KL = s.KL; p.R = s.R; p.NP = s.NP; p.VD = s.VD;
   p.kpart_max = s.kpart_max;
   p.err = reinterpret_cast<int32_t*>(B + o_err);

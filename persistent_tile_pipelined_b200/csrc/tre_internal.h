@@ -12,8 +12,7 @@ constexpr int kConsumerWarps = 8;                      // compute warps
 constexpr int kConsumerThreads = kConsumerWarps * 32;  // 256
 constexpr int kThreads = kConsumerThreads + 32;        // + one producer warp
 constexpr int kMaxGroup = 8;                           // q heads per kv head (GQA)
-constexpr int kPosPerWarp = 8;                         // KV positions per warp per stage
-constexpr int kMaxPosPerStage = kConsumerWarps * kPosPerWarp;  // 64
+constexpr int kMaxPosPerStage = 64;                    // GQA attention stage: 4 warps x 16 rows
 constexpr int kDefaultStageBytes = 32768;  // a bulk-copy stage costs ~0.4 us per SM: keep them large
 constexpr int kMaxKPart = 16384;         // longest input slice one GEMV task stages (floats)
 constexpr int kMaxResidRows = 512;       // rows per task of ops that add a residual
@@ -163,7 +162,8 @@ struct Params {
   float* lat_new;                  // [KL + R]: this token's latent row (bf16 values)
   float* o_lat;                    // [H][KL]
   float* mla_o;                    // [H * VD]
-  const void* mla_maps;            // [L] tensor maps (128 B each) over the latent caches
+  const void* kv_maps;             // tensor maps (128 B each): GQA / MoE [L][K, V] caches,
+                                   // MLA [L] latent caches
   const double* rope_inv_freq_r;   // [R / 2]
   uint32_t* down_tickets;          // MoE down: arrival ticket per row block
   float* part;                     // [Hq][splits][D + 2]
@@ -200,5 +200,8 @@ tre_status plan_build(const tre_config& cfg, int nsm, int smem_limit, PlanShape*
                       std::vector<int64_t>* sm_bytes);
 int64_t step_bytes(const PlanShape& s, int pos);
 void set_error(const std::string& msg);
+// Host only, allocates nothing: a 2-D tensor map (128 bytes at out128) over a bf16 cache
+// [rows][C] with 64-column x box_rows boxes and the 128-byte swizzle (tre_api.cu).
+tre_status encode_cache_map(void* cache, int C, long long rows, int box_rows, void* out128);
 }  // namespace tre
 #endif

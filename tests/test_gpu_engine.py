@@ -121,7 +121,7 @@ def test_shapes(over, steps):
 
 @pytest.mark.parametrize("cfg", [
     dict(num_sms=7),                                   # many tasks per CTA, ring wraps often
-    dict(num_sms=3, ring_stages=2, stage_bytes=4096),  # smallest ring, one row per stage
+    dict(num_sms=3, ring_stages=2, stage_bytes=16384),  # 2-stage ring of one attention tile each
     dict(kv_splits=16),                                # empty splits at small pos
     dict(kv_splits=1),                                 # no split: combine of one partial
 ])

@@ -108,9 +108,9 @@ def test_moe_layers(over, steps):
 
 @pytest.mark.parametrize("cfg", [
     dict(num_sms=5),
-    dict(num_sms=3, ring_stages=2, stage_bytes=8192),
+    dict(num_sms=3, ring_stages=2, stage_bytes=16384),
     dict(kv_splits=1),
-], ids=["sms5", "sms3-ring2-8k", "split1"])
+], ids=["sms5", "sms3-ring2-16k", "split1"])
 def test_moe_launch_shapes(cfg):
     run_moe(SMALL, steps=2, **cfg)
 
