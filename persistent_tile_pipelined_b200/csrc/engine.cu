@@ -772,12 +772,10 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
       dst[D + 1] = Ls;
     }
   }
-  __threadfence();
   consumer_sync(kConsumerThreads);
   if (ctid == 0) {
     const uint32_t old = ticket_add(p.tickets + g, 1u);
     *flag = ((old + 1u) % (uint32_t)S) == 0u;
-    if (*flag) fence_acq_rel_gpu();
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
   }
   consumer_sync(kConsumerThreads);
@@ -808,7 +806,6 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
       }
       p.attn[(size_t)(g * G + h) * D + dd] = O / Ls;
     }
-    __threadfence();
     consumer_sync(kConsumerThreads);
     if (ctid == 0) publish_add(p.counters + t.out, 1u);
   }
@@ -846,7 +843,7 @@ __device__ __forceinline__ void run_attn(const Params& p, const Task& t, uint32_
 // The task also writes RoPE(q_pe) after q_lat, and head 0 appends this token's latent row
 // [RMSNorm(c_kv; kv_norm) | RoPE(k_pe)] (bf16) to the cache and keeps its values for the
 // attention's new position.
-__device__ __noinline__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint32_t gs, int ns,
+__device__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint32_t gs, int ns,
                         uint8_t* ring, uint64_t* full, uint64_t* empty, const uint32_t* tags,
                         float* ub, float* red1, int warp, int lane, int ctid, bool& ab) {
   const int h = t.r0 / p.NP, KL = p.KL, C = KL + p.R;
@@ -947,7 +944,6 @@ __device__ __noinline__ void uk_task(const Params& p, const Task& t, const GemvG
       p.lat_new[KL + i + R2] = __bfloat162float(b);
     }
   }
-  __threadfence();
   consumer_sync(kConsumerThreads);
   if (ctid == 0) publish_add(p.counters + t.out, 1u);
 }
@@ -963,7 +959,7 @@ __device__ __noinline__ void uk_task(const Params& p, const Task& t, const GemvG
 //   values: warp w accumulates O[16][KL / 8 columns] += P (hi + lo) x rows (ldmatrix.trans).
 // The split's (m, l, O) go to the partial buffer and the split publishes; each head's
 // W_uv task merges the head's splits while it stages its input (mla_combine_input).
-__device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
+__device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
                               uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                               int warp, int lane, int ctid, bool& ab) {
   constexpr int HG = kMlaHeadGroup, PS = kMlaPosPerStage, RP = 36;  // score row pitch (floats)
@@ -1194,7 +1190,6 @@ __device__ __noinline__ void mla_attn_task(const Params& p, const Task& t, uint3
     d[0] = mst[ctid];
     d[1] = lst[ctid];
   }
-  __threadfence();
   consumer_sync(kConsumerThreads);
   if (ctid == 0) {
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
@@ -1324,7 +1319,6 @@ __device__ void route_topk(const Params& p, int layer, float* sc, int warp, int 
     if (lane == 0) p.route_idx[layer * p.topk + j] = b.i;
   }
   if (lane < p.topk) p.route_w[layer * p.topk + lane] = mine / tot;
-  __threadfence();
   __syncwarp();
   if (lane == 0) publish_add(p.counters + layer * C_PER_LAYER + C_ROUTE, 1u);
 }
@@ -1340,7 +1334,6 @@ __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
     if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
     if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
   }
-  __threadfence();
   consumer_sync(kConsumerThreads);
   if (ctid == 0) publish_add(p.counters + t.out, 1u);
 }
@@ -1478,17 +1471,14 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
           reinterpret_cast<int*>(red)[16 + warp] = best.i;
         }
       }
-      __threadfence();
       consumer_sync(kConsumerThreads);
       if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
       if (t.op == OP_LM && ctid == 0) {
         Best bb{-INFINITY, 0x7fffffff};
         for (int w = 0; w < kConsumerWarps; ++w) best_update(bb, red[w], reinterpret_cast<int*>(red)[16 + w]);
         atomicMax(p.argmax_slot, pack_best(bb));
-        __threadfence();
         const uint32_t old = ticket_add(p.lm_ticket, 1u);
         if (((old + 1u) % (uint32_t)t.aux) == 0u) {
-          fence_acq_rel_gpu();
           const unsigned long long w = atomicExch(p.argmax_slot, 0ull);
           if (p.token_out) *p.token_out = (int32_t)(0xffffffffu - (uint32_t)(w & 0xffffffffull));
         }
@@ -1497,7 +1487,6 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         if (ctid == 0) {
           const uint32_t old = ticket_add(p.router_ticket, 1u);
           flags[1] = ((old + 1u) % (uint32_t)t.aux) == 0u;
-          if (flags[1]) fence_acq_rel_gpu();
         }
         consumer_sync(kConsumerThreads);
         if (flags[1]) route_topk(p, t.layer, ub + p.xs_floats, warp, lane, ctid);
@@ -1505,7 +1494,6 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         if (ctid == 0) {
           const uint32_t old = ticket_add(p.down_tickets + (t.aux >> 8), 1u);
           flags[1] = ((old + 1u) % (uint32_t)(p.nshared + p.topk)) == 0u;
-          if (flags[1]) fence_acq_rel_gpu();
         }
         consumer_sync(kConsumerThreads);
         if (flags[1]) moe_down_combine(p, t, ctid);

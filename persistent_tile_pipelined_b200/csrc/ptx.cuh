@@ -92,32 +92,23 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-// Publish: bump a dependency counter.  Every call site has each writing thread execute
-// fence.acq_rel.gpu (__threadfence) and then a barrier with the publishing thread before
-// this add (the fence-then-barrier-then-atomic pattern), so the add itself is relaxed: a
-// release form here would fence again, after the producer warp has queued more bulk
-// copies, and was measured to delay the publish by microseconds.
+// Publish: bump a dependency counter with release semantics.  Every call site first has
+// the threads that wrote the published data reach a barrier with the publishing thread;
+// the release is cumulative over what that barrier ordered before it, so one release by
+// one thread covers the whole CTA's writes (no per-thread fences).
 __device__ __forceinline__ void publish_add(uint32_t* p, uint32_t v) {
-  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Arrival ticket: relaxed add returning the old count.  Arrivers fence and barrier before
-// it (as for publish_add); the arriver that finds itself last calls fence_acq_rel_gpu()
-// before it reads what the others wrote.
+// Arrival ticket: acquire-release add returning the old count, by one thread after a
+// barrier (as for publish_add); the arriver that finds itself last may read what the
+// others wrote before their tickets.
 __device__ __forceinline__ uint32_t ticket_add(uint32_t* p, uint32_t v) {
   uint32_t old;
-  asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
 }
 
-__device__ __forceinline__ uint32_t atom_acq_rel_gpu_add(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
 
 __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
