@@ -99,7 +99,8 @@ typedef struct {
                                    <= 768, q_lora / nope_dim / v_dim of 8               */
   int32_t n_experts, top_k, n_shared, expert_ffn;              /* MOE                   */
   int32_t kv_capacity;          /* positions allocated in each KV cache                 */
-  int32_t max_tokens_per_step;  /* M, 1..4                                              */
+  int32_t max_tokens_per_step;  /* M, 0..4 (0 = 1): tokens tre_decode_tokens may take;
+                                   GQA stacks with M x (q heads per kv head) <= 16      */
   float rope_theta;
   float norm_eps;
   int32_t has_embed_lm_head;    /* 1: token in, logits out; 0: hidden in, hidden out    */
@@ -193,6 +194,22 @@ void tre_destroy(tre_engine* e);
 tre_status tre_decode_step(tre_engine* e, int32_t token, int32_t pos, tre_stream stream,
                            float* logits_dev, int32_t* token_dev);
 
+/* One step over m consecutive tokens of one sequence (speculative-style verification:
+ * the pages' multi-token prediction, Speed is intelligence talk, section on tokens per
+ * byte): token v sits at position pos + v and attends to the cached positions [0, pos) and
+ * to the step's own positions pos .. pos + v (causal).  Every weight byte is read once for
+ * all m tokens.  Results equal m successive tre_decode_step calls with the same tokens.
+ *   tokens_host  host int32[m], each in [0, vocab) (kernel arguments, no copy)
+ *   m            1 <= m <= max_tokens_per_step
+ *   pos          the caches hold [0, pos) on entry and [0, pos + m) on return;
+ *                pos + m <= kv_capacity
+ *   logits_dev   device fp32[m][vocab] or NULL
+ *   tokens_dev   device int32[m] or NULL: the greedy argmax of each row of logits
+ * Enqueues asynchronously; returns a previous step's device error without launching.
+ * Requires has_embed_lm_head == 1. */
+tre_status tre_decode_tokens(tre_engine* e, const int32_t* tokens_host, int32_t m, int32_t pos,
+                             tre_stream stream, float* logits_dev, int32_t* tokens_dev);
+
 /* The same step driven from host memory: copies nothing in (the token is a kernel
  * argument), runs the step, copies the argmax token (and the logits when logits_host
  * is not NULL) back into host memory and waits for them.  This is the call a greedy
@@ -256,8 +273,8 @@ tre_status tre_get_status(tre_engine* e, int32_t* device_status, int32_t* detail
  * engine can step again after a device error.  Enqueued on `stream`. */
 tre_status tre_reset(tre_engine* e, tre_stream stream);
 
-/* Copy the residual stream after every layer of the last step ([n_layers][d] fp32,
- * device) — requires TRE_DEBUG_HIDDEN. */
+/* Copy the residual stream after every layer of the last step ([n_layers][m][d] fp32,
+ * device; m = the last step's tokens, 1 for tre_decode_step) — requires TRE_DEBUG_HIDDEN. */
 tre_status tre_debug_hidden(tre_engine* e, float* hidden_dev, tre_stream stream);
 
 /* Copy the per-task trace of the last step to host memory: 8 int64 per task, in global
@@ -269,8 +286,9 @@ tre_status tre_debug_hidden(tre_engine* e, float* hidden_dev, tre_stream stream)
  * query. */
 tre_status tre_debug_trace(tre_engine* e, int64_t* trace_host, int32_t* n_tasks);
 
-/* Bytes a step at `pos` streams from HBM (weights + KV read + KV written + logits). */
-tre_status tre_step_bytes(const tre_engine* e, int32_t pos, int64_t* bytes);
+/* Bytes a step of m tokens at `pos` streams from HBM (weights + KV read + the m tokens' KV
+ * rows written + embedding rows + logits); m = 1 for tre_decode_step / tre_layers_step. */
+tre_status tre_step_bytes(const tre_engine* e, int32_t pos, int32_t m, int64_t* bytes);
 
 /* Plan without a GPU: run the planner for cfg on a hypothetical device with `num_sms`
  * SMs and `smem_per_block` bytes of opt-in shared memory, and summarise the plan. */

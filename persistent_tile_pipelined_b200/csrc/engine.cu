@@ -464,10 +464,12 @@ __device__ __forceinline__ unsigned long long pack_best(const Best& b) {
   return ((unsigned long long)key << 32) | (uint32_t)(0xffffffffu - (uint32_t)b.i);
 }
 
-__device__ __forceinline__ float resid_in(const Params& p, int layer, int n) {
-  if (layer > 0) return __ldcg(p.x + n);
-  if (p.x_in) return __ldcg(p.x_in + n);
-  return bf_lo(p.embed[(size_t)p.token * p.d + n]);
+// Row n of token v's residual stream entering `layer` (layer 0: the embedding row or the
+// layer-only input).
+__device__ __forceinline__ float resid_in(const Params& p, int layer, int n, int v = 0) {
+  if (layer > 0) return __ldcg(p.x + (size_t)v * p.d + n);
+  if (p.x_in) return __ldcg(p.x_in + (size_t)v * p.d + n);
+  return bf_lo(p.embed[(size_t)p.tokens[v] * p.d + n]);
 }
 
 // Input-vector identity for reuse across consecutive tasks (same layer, same source,
@@ -488,76 +490,92 @@ __device__ __forceinline__ int input_key(const Task& t) {
   return (((int)t.layer * 8 + cls) << 8) | part;
 }
 
-// Stage the GEMV input into the two planes; returns the RMSNorm scale (1 when none).
-__device__ float load_input(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
-                            float* red, int ctid) {
+// Stage the GEMV input of each of the MT tokens into its two planes (token v's at
+// ub + v Kp); rn[v] receives token v's RMSNorm scale (1 when the op has no norm).
+template <int MT>
+__device__ void load_input(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
+                           float* red, int ctid, float* rn) {
   const int K = gg.Kp;  // this K-part's slice of the input vector
-  float* xlo = ub;
-  float* xhi = ub + K / 2;
   const float* src = nullptr;
   const uint16_t* src_bf = nullptr;
   const uint16_t* gain = nullptr;
+  size_t vstride = 0;   // floats between consecutive tokens' vectors
   switch (t.op) {
     case OP_QKV:
     case OP_MDQKV:
       gain = p.layers[t.layer].w[TRE_W_ATTN_NORM];
+      vstride = p.d;
       if (t.layer > 0) src = p.x;
       else if (p.x_in) src = p.x_in;
-      else src_bf = p.embed + (size_t)p.token * p.d;
+      else src_bf = p.embed;
       break;
-    case OP_O: src = p.attn; break;
+    case OP_O: src = p.attn; vstride = (size_t)p.Hq * p.D; break;
     case OP_GU: case OP_ROUTER: case OP_SGU: case OP_RGU:
-      src = p.h1; gain = p.layers[t.layer].w[TRE_W_FFN_NORM]; break;
-    case OP_DOWN: case OP_MDOWN: src = p.u; break;
+      src = p.h1; vstride = p.d; gain = p.layers[t.layer].w[TRE_W_FFN_NORM]; break;
+    case OP_DOWN: case OP_MDOWN: src = p.u; vstride = p.F; break;
     case OP_UQ: src = p.cqkv; gain = p.layers[t.layer].w[TRE_W_Q_NORM]; break;
     case OP_UV: src = p.o_lat + (size_t)(t.r0 / p.VD) * p.KL; break;
     case OP_MO: src = p.mla_o; break;
-    default: src = p.x; gain = p.final_norm; break;
+    default: src = p.x; vstride = p.d; gain = p.final_norm; break;
   }
   if (src) src += gg.k0;        // normalised inputs are single-part (k0 = 0)
-  float ss = 0.f;
   const int K8 = K >> 3;
-  for (int j = ctid; j < K8; j += kConsumerThreads) {
-    float v[8];
-    if (src_bf) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(src_bf) + j);
-      v[0] = bf_lo(w.x); v[1] = bf_hi(w.x); v[2] = bf_lo(w.y); v[3] = bf_hi(w.y);
-      v[4] = bf_lo(w.z); v[5] = bf_hi(w.z); v[6] = bf_lo(w.w); v[7] = bf_hi(w.w);
-    } else {
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(src) + 2 * j);
-      const float4 b = __ldcg(reinterpret_cast<const float4*>(src) + 2 * j + 1);
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-    if (gain) {
+  float ss[MT];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) ss = fmaf(v[k], v[k], ss);
-      const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain) + j);
-      v[0] *= bf_lo(g.x); v[1] *= bf_hi(g.x); v[2] *= bf_lo(g.y); v[3] *= bf_hi(g.y);
-      v[4] *= bf_lo(g.z); v[5] *= bf_hi(g.z); v[6] *= bf_lo(g.w); v[7] *= bf_hi(g.w);
+  for (int v = 0; v < MT; ++v) {
+    ss[v] = 0.f;
+    float* xlo = ub + (size_t)v * K;
+    float* xhi = xlo + K / 2;
+    const float* sv = src ? src + v * vstride : nullptr;
+    const uint16_t* bv = src_bf ? src_bf + (size_t)p.tokens[v] * p.d : nullptr;
+    for (int j = ctid; j < K8; j += kConsumerThreads) {
+      float e[8];
+      if (bv) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(bv) + j);
+        e[0] = bf_lo(w.x); e[1] = bf_hi(w.x); e[2] = bf_lo(w.y); e[3] = bf_hi(w.y);
+        e[4] = bf_lo(w.z); e[5] = bf_hi(w.z); e[6] = bf_lo(w.w); e[7] = bf_hi(w.w);
+      } else {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(sv) + 2 * j);
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(sv) + 2 * j + 1);
+        e[0] = a.x; e[1] = a.y; e[2] = a.z; e[3] = a.w; e[4] = b.x; e[5] = b.y; e[6] = b.z; e[7] = b.w;
+      }
+      if (gain) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss[v] = fmaf(e[k], e[k], ss[v]);
+        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain) + j);
+        e[0] *= bf_lo(g.x); e[1] *= bf_hi(g.x); e[2] *= bf_lo(g.y); e[3] *= bf_hi(g.y);
+        e[4] *= bf_lo(g.z); e[5] *= bf_hi(g.z); e[6] *= bf_lo(g.w); e[7] *= bf_hi(g.w);
+      }
+      reinterpret_cast<float4*>(xlo)[j] = make_float4(e[0], e[1], e[2], e[3]);
+      reinterpret_cast<float4*>(xhi)[j] = make_float4(e[4], e[5], e[6], e[7]);
     }
-    reinterpret_cast<float4*>(xlo)[j] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4*>(xhi)[j] = make_float4(v[4], v[5], v[6], v[7]);
   }
-  float rn = 1.f;
   if (gain) {
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if ((ctid & 31) == 0) red[ctid >> 5] = ss;
+    for (int v = 0; v < MT; ++v) {
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) ss[v] += __shfl_xor_sync(0xffffffffu, ss[v], off);
+      if ((ctid & 31) == 0) red[(ctid >> 5) * MT + v] = ss[v];
+    }
   }
   consumer_sync(kConsumerThreads);
-  if (gain) {
-    float tot = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) tot += red[w];
-    rn = 1.f / sqrtf(tot / (float)K + p.eps);
+  for (int v = 0; v < MT; ++v) {
+    float r = 1.f;
+    if (gain) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) tot += red[w * MT + v];
+      r = 1.f / sqrtf(tot / (float)K + p.eps);
+    }
+    rn[v] = r;
   }
-  return rn;
 }
 
 // ---- attention task ----------------------------------------------------------------------------
 __device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float& s,
-                                        const double* inv_freq = nullptr) {
-  const double ang = (double)p.pos * (inv_freq ? inv_freq : p.rope_inv_freq)[i];
+                                        const double* inv_freq = nullptr, int dpos = 0) {
+  const double ang = (double)(p.pos + dpos) * (inv_freq ? inv_freq : p.rope_inv_freq)[i];
   const double two_pi = 6.283185307179586476925286766559;
   const double red = ang - two_pi * rint(ang / two_pi);
   sincosf((float)red, &s, &c);
@@ -569,86 +587,111 @@ __device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float&
 // position pos from this step's k / v, appends them to the caches and merges its partial.
 // The last split of the group to finish (arrival ticket) combines all splits — the fused
 // combine — and publishes the group.
-template <int G, int D>
+template <int G, int D, int MT>
 __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
                           uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                           int* flag, int warp, int lane, int ctid, bool& abort_out) {
+  // query rows r = v G + h: token v (position pos + v) of head g G + h
+  constexpr int ROWS = MT * G;
+  constexpr bool PACK = ROWS <= 8;  // hi / lo packed into rows r and r + 8 of one tile
   const int g = t.r0, split = t.r1, S = t.aux;
   const bool last = (split == S - 1);
-  float* q_s = ub;                            // [G][D] roped, scaled
-  float* kn_s = q_s + G * D;                  // [D]   new k (bf16 value)
-  float* vn_s = kn_s + D;                     // [D]   new v (bf16 value)
-  float* mw = vn_s + D;                       // [warps][G]
-  float* lw = mw + kConsumerWarps * G;        // [warps][G]
-  float* ow = lw + kConsumerWarps * G;        // [warps][G][D]
-  float* sn = ow + kConsumerWarps * G * D;    // [G] score of the new position
+  const int qkv_n = (p.Hq + 2 * p.Hkv) * D;
+  float* q_s = ub;                            // [ROWS][D] roped, scaled
+  float* kn_s = q_s + ROWS * D;               // [MT][D] new k (bf16 values)
+  float* vn_s = kn_s + MT * D;                // [MT][D] new v (bf16 values)
+  float* mw = vn_s + MT * D;                  // [warps][ROWS]
+  float* lw = mw + kConsumerWarps * ROWS;     // [warps][ROWS]
+  float* ow = lw + kConsumerWarps * ROWS;     // [warps][ROWS][D]
+  float* sn = ow + kConsumerWarps * ROWS * D; // [ROWS][MT] scores of the new positions
   const float qscale = 1.4426950408889634f / sqrtf((float)D);
 
-  const float* qsrc = p.qkv + (size_t)g * G * D;
-  for (int idx = ctid; idx < G * (D / 2); idx += kConsumerThreads) {
-    const int h = idx / (D / 2), i = idx % (D / 2);
-    const float x0 = __ldcg(qsrc + h * D + i), x1 = __ldcg(qsrc + h * D + i + D / 2);
+  for (int idx = ctid; idx < ROWS * (D / 2); idx += kConsumerThreads) {
+    const int r = idx / (D / 2), i = idx % (D / 2), v = r / G, h = r % G;
+    const float* qsrc = p.qkv + (size_t)v * qkv_n + (size_t)(g * G + h) * D;
+    const float x0 = __ldcg(qsrc + i), x1 = __ldcg(qsrc + i + D / 2);
     float c, s;
-    rope_cs(p, i, c, s);
-    q_s[h * D + i] = (x0 * c - x1 * s) * qscale;
-    q_s[h * D + i + D / 2] = (x0 * s + x1 * c) * qscale;
+    rope_cs(p, i, c, s, nullptr, v);
+    q_s[r * D + i] = (x0 * c - x1 * s) * qscale;
+    q_s[r * D + i + D / 2] = (x0 * s + x1 * c) * qscale;
   }
-  if (last) {
-    const float* ksrc = p.qkv + (size_t)p.Hq * D + (size_t)g * D;
-    const float* vsrc = ksrc + (size_t)p.Hkv * D;
+  if (last) {  // this step's MT keys and values: RoPE, round to bf16, append at pos + v
     const LayerPtrs& L = p.layers[t.layer];
-    __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(L.k_cache) + ((size_t)g * p.cap + p.pos) * D;
-    __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(L.v_cache) + ((size_t)g * p.cap + p.pos) * D;
-    for (int i = ctid; i < D / 2; i += kConsumerThreads) {
+    for (int idx = ctid; idx < MT * (D / 2); idx += kConsumerThreads) {
+      const int v = idx / (D / 2), i = idx % (D / 2);
+      const float* ksrc = p.qkv + (size_t)v * qkv_n + (size_t)p.Hq * D + (size_t)g * D;
+      __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(L.k_cache) +
+                          ((size_t)g * p.cap + p.pos + v) * D;
       const float x0 = __ldcg(ksrc + i), x1 = __ldcg(ksrc + i + D / 2);
       float c, s;
-      rope_cs(p, i, c, s);
+      rope_cs(p, i, c, s, nullptr, v);
       const __nv_bfloat16 k0 = __float2bfloat16_rn(x0 * c - x1 * s);
       const __nv_bfloat16 k1 = __float2bfloat16_rn(x0 * s + x1 * c);
       kc[i] = k0;
       kc[i + D / 2] = k1;
-      kn_s[i] = __bfloat162float(k0);
-      kn_s[i + D / 2] = __bfloat162float(k1);
+      kn_s[v * D + i] = __bfloat162float(k0);
+      kn_s[v * D + i + D / 2] = __bfloat162float(k1);
     }
-    for (int i = ctid; i < D; i += kConsumerThreads) {
-      const __nv_bfloat16 v = __float2bfloat16_rn(__ldcg(vsrc + i));
-      vc[i] = v;
-      vn_s[i] = __bfloat162float(v);
+    for (int idx = ctid; idx < MT * D; idx += kConsumerThreads) {
+      const int v = idx / D, i = idx % D;
+      const float* vsrc = p.qkv + (size_t)v * qkv_n + (size_t)(p.Hq + p.Hkv) * D + (size_t)g * D;
+      __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(L.v_cache) +
+                          ((size_t)g * p.cap + p.pos + v) * D;
+      const __nv_bfloat16 val = __float2bfloat16_rn(__ldcg(vsrc + i));
+      vc[i] = val;
+      vn_s[v * D + i] = __bfloat162float(val);
     }
   }
   consumer_sync(kConsumerThreads);
   if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
 
-  if (last && warp < G) {  // score of the new position for head `warp`
-    float a = 0.f;
-    for (int i = lane; i < D; i += 32) a = fmaf(q_s[warp * D + i], kn_s[i], a);
+  if (last) {  // scores of the new positions; token v sees new positions j <= v
+    for (int idx = warp; idx < ROWS * MT; idx += kConsumerWarps) {
+      const int r = idx / MT, j = idx % MT;
+      float a = 0.f;
+      for (int i = lane; i < D; i += 32) a = fmaf(q_s[r * D + i], kn_s[j * D + i], a);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-    if (lane == 0) sn[warp] = a;
+      for (int off = 16; off >= 1; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+      if (lane == 0) sn[idx] = j <= r / G ? a : -INFINITY;
+    }
   }
 
   // ---- tensor-core flash-decode over the split's cached positions
-  // One 16-row A tile carries the group's G <= 8 query heads twice: row h holds head h's
-  // bf16 hi part and row h + 8 its lo part, so S = Q K^T for head h is the sum of the
-  // accumulator rows h and h + 8 — which the same thread holds (c0 + c2, c1 + c3).  P and
-  // the value product use the same packing.  A stage holds 64 positions of K then V as
+  // The query rows form one 16-row A tile.  With ROWS <= 8 each row's bf16 hi part sits in
+  // row r and its lo part in row r + 8, so one mma.sync computes both and the thread adds
+  // its two accumulator rows (c0 + c2, c1 + c3); with more rows the hi and lo tiles are
+  // separate and every tile takes two mma.  A stage holds 64 positions of K then V as
   // 64-column swizzled boxes; the 8 warps form two groups taking alternate stages, and warp
   // (group, quarter) owns positions 16 quarter .. 16 quarter + 15 of its stages with its own
-  // running (m, l, O).  P goes from the score registers straight into the A operand of
-  // O += P V (the m16n8 accumulator layout of two n-tiles is the m16k16 A layout).
-  // Positions past the split are masked (score -inf, value 0).
+  // running (m, l, O) per row.  P goes from the score registers straight into the A operand
+  // of O += P V (the m16n8 accumulator layout of two n-tiles is the m16k16 A layout).
+  // Positions past the split are masked (score -inf, value rows zeroed).
   constexpr int KS = D / 16, NT = D / 8, KB = D / 64;  // k-steps, output n-tiles, boxes
+  constexpr int NST = PACK ? 1 : 2;                     // running states per thread
   const int g8 = lane >> 2, t4 = lane & 3;
-  const bool real = g8 < G;
-  uint32_t qa[KS][4];
+  const bool real0 = g8 < ROWS, real1 = !PACK && g8 + 8 < ROWS;
+  uint32_t qh[KS][4], ql[PACK ? 1 : KS][4];
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
     const int k0 = ks * 16 + 2 * t4;
-    const float* qr = q_s + (real ? g8 : 0) * D;
-    split_pair(real ? qr[k0] : 0.f, real ? qr[k0 + 1] : 0.f, qa[ks][0], qa[ks][1]);
-    split_pair(real ? qr[k0 + 8] : 0.f, real ? qr[k0 + 9] : 0.f, qa[ks][2], qa[ks][3]);
+    const float* q0 = q_s + (real0 ? g8 : 0) * D;
+    const float* q1 = q_s + (real1 ? g8 + 8 : 0) * D;
+    if constexpr (PACK) {
+      split_pair(real0 ? q0[k0] : 0.f, real0 ? q0[k0 + 1] : 0.f, qh[ks][0], qh[ks][1]);
+      split_pair(real0 ? q0[k0 + 8] : 0.f, real0 ? q0[k0 + 9] : 0.f, qh[ks][2], qh[ks][3]);
+    } else {
+      split_pair(real0 ? q0[k0] : 0.f, real0 ? q0[k0 + 1] : 0.f, qh[ks][0], ql[ks][0]);
+      split_pair(real1 ? q1[k0] : 0.f, real1 ? q1[k0 + 1] : 0.f, qh[ks][1], ql[ks][1]);
+      split_pair(real0 ? q0[k0 + 8] : 0.f, real0 ? q0[k0 + 9] : 0.f, qh[ks][2], ql[ks][2]);
+      split_pair(real1 ? q1[k0 + 8] : 0.f, real1 ? q1[k0 + 9] : 0.f, qh[ks][3], ql[ks][3]);
+    }
   }
-  float m0 = -INFINITY, l0 = 0.f;   // head g8
+  float mrow[NST], lrow[NST];
+#pragma unroll
+  for (int k = 0; k < NST; ++k) {
+    mrow[k] = -INFINITY;
+    lrow[k] = 0.f;
+  }
   float o[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -672,38 +715,59 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
         const int r = r0 + (m >> 1) * 8 + (lane & 7), ch = ks * 2 + (m & 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(tb + swz_off(ch >> 3, r, ch & 7, 64), b0, b1, b2, b3);
-        mma_bf16(c[0], qa[ks], b0, b1);
-        mma_bf16(c[1], qa[ks], b2, b3);
+        mma_bf16(c[0], qh[ks], b0, b1);
+        mma_bf16(c[1], qh[ks], b2, b3);
+        if constexpr (!PACK) {
+          mma_bf16(c[0], ql[ks], b0, b1);
+          mma_bf16(c[1], ql[ks], b2, b3);
+        }
       }
-      // scores of head g8 (hi rows + lo rows); mask positions past the split
-      float sc[2][2];
+      // scores per state (row g8; unpacked: also row g8 + 8); mask positions past the split
+      float sc[NST][2][2];
 #pragma unroll
       for (int n = 0; n < 2; ++n)
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-          sc[n][j] = (n * 8 + 2 * t4 + j < valid) ? c[n][j] + c[n][j + 2] : -INFINITY;
-      float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float mn = fmaxf(m0, mx);          // finite: valid > 0
-      const float a0 = exp2f(m0 - mn);          // 0 while m0 = -inf
-      float pv[2][2];
+        for (int j = 0; j < 2; ++j) {
+          const bool in = n * 8 + 2 * t4 + j < valid;
+          if constexpr (PACK) {
+            sc[0][n][j] = in ? c[n][j] + c[n][j + 2] : -INFINITY;
+          } else {
+            sc[0][n][j] = in ? c[n][j] : -INFINITY;
+            sc[NST - 1][n][j] = in ? c[n][j + 2] : -INFINITY;
+          }
+        }
+      float alpha[NST], pv[NST][2][2];
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
+      for (int k = 0; k < NST; ++k) {
+        float mx = fmaxf(fmaxf(sc[k][0][0], sc[k][0][1]), fmaxf(sc[k][1][0], sc[k][1][1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(mrow[k], mx);   // finite: valid > 0
+        alpha[k] = exp2f(mrow[k] - mn);        // 0 while the row had no position yet
 #pragma unroll
-        for (int j = 0; j < 2; ++j) pv[n][j] = exp2f(sc[n][j] - mn);
-      l0 = l0 * a0 + (pv[0][0] + pv[0][1] + pv[1][0] + pv[1][1]);
-      m0 = mn;
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) pv[k][n][j] = exp2f(sc[k][n][j] - mn);
+        lrow[k] = lrow[k] * alpha[k] + (pv[k][0][0] + pv[k][0][1] + pv[k][1][0] + pv[k][1][1]);
+        mrow[k] = mn;
+      }
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        o[n][0] *= a0;
-        o[n][1] *= a0;
-        o[n][2] *= a0;
-        o[n][3] *= a0;
+        o[n][0] *= alpha[0];
+        o[n][1] *= alpha[0];
+        o[n][2] *= alpha[NST - 1];
+        o[n][3] *= alpha[NST - 1];
       }
-      uint32_t pa[4];
-      split_pair(pv[0][0], pv[0][1], pa[0], pa[1]);
-      split_pair(pv[1][0], pv[1][1], pa[2], pa[3]);
+      uint32_t ph[4], pl[4];
+      if constexpr (PACK) {
+        split_pair(pv[0][0][0], pv[0][0][1], ph[0], ph[1]);
+        split_pair(pv[0][1][0], pv[0][1][1], ph[2], ph[3]);
+      } else {
+        split_pair(pv[0][0][0], pv[0][0][1], ph[0], pl[0]);
+        split_pair(pv[1][0][0], pv[1][0][1], ph[1], pl[1]);
+        split_pair(pv[0][1][0], pv[0][1][1], ph[2], pl[2]);
+        split_pair(pv[1][1][0], pv[1][1][1], ph[3], pl[3]);
+      }
 #pragma unroll
       for (int np = 0; np < NT / 2; ++np) {
         const int r = r0 + (m & 1) * 8 + (lane & 7), ch = np * 2 + (m >> 1);
@@ -716,56 +780,84 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
           if (pb0 >= valid) { b1 &= 0xffff0000u; b3 &= 0xffff0000u; }
           if (pb0 + 1 >= valid) { b1 &= 0x0000ffffu; b3 &= 0x0000ffffu; }
         }
-        mma_bf16(o[2 * np], pa, b0, b1);
-        mma_bf16(o[2 * np + 1], pa, b2, b3);
+        mma_bf16(o[2 * np], ph, b0, b1);
+        mma_bf16(o[2 * np + 1], ph, b2, b3);
+        if constexpr (!PACK) {
+          mma_bf16(o[2 * np], pl, b0, b1);
+          mma_bf16(o[2 * np + 1], pl, b2, b3);
+        }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive_n(&empty[slot], 2u);  // 4 warps per stage, 8 arrivals
   }
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  if (g8 < G) {
+#pragma unroll
+  for (int k = 0; k < NST; ++k) {
+    lrow[k] += __shfl_xor_sync(0xffffffffu, lrow[k], 1);
+    lrow[k] += __shfl_xor_sync(0xffffffffu, lrow[k], 2);
+  }
+  if (real0) {
     if (t4 == 0) {
-      mw[warp * G + g8] = m0;
-      lw[warp * G + g8] = l0;
+      mw[warp * ROWS + g8] = mrow[0];
+      lw[warp * ROWS + g8] = lrow[0];
     }
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {  // hi rows + lo rows
-      ow[(warp * G + g8) * D + n * 8 + 2 * t4] = o[n][0] + o[n][2];
-      ow[(warp * G + g8) * D + n * 8 + 2 * t4 + 1] = o[n][1] + o[n][3];
+    for (int n = 0; n < NT; ++n) {
+      float* d0 = ow + (warp * ROWS + g8) * D + n * 8 + 2 * t4;
+      if constexpr (PACK) {  // hi rows + lo rows
+        d0[0] = o[n][0] + o[n][2];
+        d0[1] = o[n][1] + o[n][3];
+      } else {
+        d0[0] = o[n][0];
+        d0[1] = o[n][1];
+      }
+    }
+  }
+  if (real1) {
+    if (t4 == 0) {
+      mw[warp * ROWS + g8 + 8] = mrow[NST - 1];
+      lw[warp * ROWS + g8 + 8] = lrow[NST - 1];
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      float* d1 = ow + (warp * ROWS + g8 + 8) * D + n * 8 + 2 * t4;
+      d1[0] = o[n][2];
+      d1[1] = o[n][3];
     }
   }
   consumer_sync(kConsumerThreads);
   if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
 
-  // merge the warps (and the new position) into this split's partial
+  // merge the warps (and, in the last split, the new positions) into this split's partial
   const size_t pstride = (size_t)D + 2;
-  for (int idx = ctid; idx < G * D; idx += kConsumerThreads) {
-    const int h = idx / D, dd = idx % D;
+  for (int idx = ctid; idx < ROWS * D; idx += kConsumerThreads) {
+    const int r = idx / D, dd = idx % D, v = r / G, h = r % G;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mw[w * G + h]);
-    const float snew = last ? sn[h] : -INFINITY;
-    M = fmaxf(M, snew);
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mw[w * ROWS + r]);
+    if (last)
+#pragma unroll
+      for (int j = 0; j < MT; ++j) M = fmaxf(M, sn[r * MT + j]);
     float O = 0.f, Ls = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
-        const float mv = mw[w * G + h];
+        const float mv = mw[w * ROWS + r];
         if (mv != -INFINITY) {
           const float sc = exp2f(mv - M);
-          O = fmaf(sc, ow[(w * G + h) * D + dd], O);
-          Ls = fmaf(sc, lw[w * G + h], Ls);
+          O = fmaf(sc, ow[(w * ROWS + r) * D + dd], O);
+          Ls = fmaf(sc, lw[w * ROWS + r], Ls);
         }
       }
-      if (last) {
-        const float pn = exp2f(snew - M);
-        O = fmaf(pn, vn_s[dd], O);
-        Ls += pn;
-      }
+      if (last)
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+          const float pn = exp2f(sn[r * MT + j] - M);   // 0 for positions after token v
+          O = fmaf(pn, vn_s[j * D + dd], O);
+          Ls += pn;
+        }
     }
-    float* dst = p.part + ((size_t)(g * G + h) * S + split) * pstride;
+    float* dst = p.part + ((size_t)(v * p.Hq + g * G + h) * S + split) * pstride;
     dst[dd] = O;
     if (dd == 0) {
       dst[D] = M;
@@ -782,21 +874,23 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   if (*flag) {  // last split of this kv head to finish: combine all splits
     // (m, l) of every split into shared memory in one round trip (reuses the warp scratch)
     float* ms = ow;
-    float* ls = ow + G * S;
-    for (int idx = ctid; idx < G * S; idx += kConsumerThreads) {
-      const float* src = p.part + ((size_t)(g * G) * S + idx) * pstride;  // head idx/S, split idx%S
+    float* ls = ow + ROWS * S;
+    for (int idx = ctid; idx < ROWS * S; idx += kConsumerThreads) {
+      const int r = idx / S, s2 = idx % S, v = r / G, h = r % G;
+      const float* src = p.part + ((size_t)(v * p.Hq + g * G + h) * S + s2) * pstride;
       ms[idx] = __ldcg(src + D);
       ls[idx] = __ldcg(src + D + 1);
     }
     consumer_sync(kConsumerThreads);
-    for (int idx = ctid; idx < G * D; idx += kConsumerThreads) {
-      const int h = idx / D, dd = idx % D;
-      const float* mh = ms + h * S;
-      const float* lh = ls + h * S;
+    for (int idx = ctid; idx < ROWS * D; idx += kConsumerThreads) {
+      const int r = idx / D, dd = idx % D, v = r / G, h = r % G;
+      const float* mh = ms + r * S;
+      const float* lh = ls + r * S;
       float M = -INFINITY;
       for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mh[s2]);
       float Ls = 0.f, O = 0.f;
-      const float* src = p.part + (size_t)(g * G + h) * S * pstride + dd;
+      const size_t q = (size_t)v * p.Hq + g * G + h;
+      const float* src = p.part + q * S * pstride + dd;
       // independent loads: the splits' outputs are fetched together, not one at a time
 #pragma unroll 8
       for (int s2 = 0; s2 < S; ++s2) {
@@ -804,33 +898,34 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
         Ls = fmaf(w, lh[s2], Ls);
         O = fmaf(w, __ldcg(src + s2 * pstride), O);
       }
-      p.attn[(size_t)(g * G + h) * D + dd] = O / Ls;
+      p.attn[q * D + dd] = O / Ls;
     }
     consumer_sync(kConsumerThreads);
     if (ctid == 0) publish_add(p.counters + t.out, 1u);
   }
 }
 
+template <int MT>
 __device__ __forceinline__ void run_attn(const Params& p, const Task& t, uint32_t gs, int ns,
                                          uint8_t* ring, uint64_t* full, uint64_t* empty,
                                          const uint32_t* tags, float* ub, int* flag, int warp,
                                          int lane, int ctid, bool& ab) {
   const int G = p.Hq / p.Hkv;
 #define TRE_ATTN(GG, DD) \
-  attn_task<GG, DD>(p, t, gs, ns, ring, full, empty, tags, ub, flag, warp, lane, ctid, ab)
+  attn_task<GG, DD, MT>(p, t, gs, ns, ring, full, empty, tags, ub, flag, warp, lane, ctid, ab)
   if (p.D == 128) {
     switch (G) {
       case 1: TRE_ATTN(1, 128); break;
       case 2: TRE_ATTN(2, 128); break;
-      case 4: TRE_ATTN(4, 128); break;
-      default: TRE_ATTN(8, 128); break;
+      case 4: if constexpr (MT <= 4) TRE_ATTN(4, 128); break;
+      default: if constexpr (MT <= 2) TRE_ATTN(8, 128); break;
     }
   } else {
     switch (G) {
       case 1: TRE_ATTN(1, 64); break;
       case 2: TRE_ATTN(2, 64); break;
-      case 4: TRE_ATTN(4, 64); break;
-      default: TRE_ATTN(8, 64); break;
+      case 4: if constexpr (MT <= 4) TRE_ATTN(4, 64); break;
+      default: if constexpr (MT <= 2) TRE_ATTN(8, 64); break;
     }
   }
 #undef TRE_ATTN
@@ -1249,39 +1344,44 @@ __device__ void mla_combine_input(const Params& p, const Task& t, float* ub, flo
 // Residual rows of an O-proj / down task, staged before its stages: part 0 reads the
 // residual stream (x, or for layer 0 the embedding row / layer input; h1 for down), later
 // K-parts read the partial sum the previous part left in the output.
+template <int MT>
 __device__ __forceinline__ void prefetch_resid(const Params& p, const Task& t, const GemvGeom& g,
                                                float* resid, int ctid) {
-  for (int r = ctid; r < t.r1 - t.r0; r += kConsumerThreads) {
-    const int n = t.r0 + r;
-    float v;
-    if (t.op == OP_O) v = g.part == 0 ? resid_in(p, t.layer, n) : __ldcg(p.h1 + n);
-    else if (t.op == OP_MO) v = g.part == 0 ? resid_in(p, t.layer, n) : __ldcg(p.x + n);
-    else v = g.part == 0 ? __ldcg(p.h1 + n) : __ldcg(p.x + n);
-    resid[r] = v;
+  const int nr = t.r1 - t.r0;
+  for (int idx = ctid; idx < MT * nr; idx += kConsumerThreads) {
+    const int v = idx / nr, r = idx % nr, n = t.r0 + r;
+    const size_t off = (size_t)v * p.d + n;
+    float val;
+    if (t.op == OP_O) val = g.part == 0 ? resid_in(p, t.layer, n, v) : __ldcg(p.h1 + off);
+    else if (t.op == OP_MO) val = g.part == 0 ? resid_in(p, t.layer, n, v) : __ldcg(p.x + off);
+    else val = g.part == 0 ? __ldcg(p.h1 + off) : __ldcg(p.x + off);
+    resid[v * kMaxResidRows + r] = val;
   }
 }
 
 __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const GemvGeom& g, int n,
-                                          float v, float rn, const float* resid, Best& best) {
+                                          float v, float rn, const float* resid, Best& best,
+                                          int tok = 0) {
   switch (t.op) {
-    case OP_QKV: case OP_UQ: p.qkv[n] = v * rn; break;
+    case OP_QKV: p.qkv[(size_t)tok * (p.Hq + 2 * p.Hkv) * p.D + n] = v * rn; break;
+    case OP_UQ: p.qkv[n] = v * rn; break;
     case OP_MDQKV: p.cqkv[n] = v * rn; break;
     case OP_UV: p.mla_o[n] = v; break;
-    case OP_O: p.h1[n] = resid[n - t.r0] + v; break;
+    case OP_O: p.h1[(size_t)tok * p.d + n] = resid[n - t.r0] + v; break;
     case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
     case OP_MDOWN: p.mpart[(size_t)g.part * p.d + n] = v; break;
     case OP_DOWN:
     case OP_MO: {
       const float y = resid[n - t.r0] + v;
-      p.x[n] = y;
+      p.x[(size_t)tok * p.d + n] = y;
       if (g.part == g.np - 1) {
-        if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
-        if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
+        if (p.hidden) p.hidden[((size_t)t.layer * p.m + tok) * p.d + n] = y;
+        if (p.x_out && t.layer == p.L - 1) p.x_out[(size_t)tok * p.d + n] = y;
       }
     } break;
     default: {
       const float y = v * rn;
-      p.logits[n] = y;
+      p.logits[(size_t)tok * p.V + n] = y;
       best_update(best, y, n);
     } break;
   }
@@ -1341,14 +1441,14 @@ __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
 // ---- consumers -----------------------------------------------------------------------------------
 // MLA = true: the absorbed-MLA stack's kernel (MLA tiles, no GQA attention); false: GQA /
 // MoE.  Two instantiations keep each kernel's register allocation to its own tiles.
-template <bool MLA>
+template <bool MLA, int MT>
 __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                          float* misc) {
   const int ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
-  float* red = misc;                                      // [32] reductions
-  int* flags = reinterpret_cast<int*>(misc + 32);         // [0] abort, [1] ticket
-  float* rn_s = misc + 40;
+  float* red = misc;                                      // [64] reductions
+  int* flags = reinterpret_cast<int*>(misc + 64);         // [0] abort, [1] ticket
+  float* rn_s = misc + 72;                                // [MT] RMSNorm scales
   const uint32_t NS = (uint32_t)p.ring_stages;
   uint32_t gs = 0;
   int cur_key = -1;
@@ -1373,7 +1473,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     if (!MLA && t.type == T_ATTN) {
       cur_key = -1;  // the attention scratch aliases the input-vector planes
       if constexpr (!MLA)
-        run_attn(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
+        run_attn<MT>(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
     } else if (MLA && t.type == T_MLA_ATTN) {
       cur_key = -1;
       if constexpr (MLA)
@@ -1387,23 +1487,31 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
       const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MO;
-      if (has_resid) prefetch_resid(p, t, g, resid, ctid);
+      if (has_resid) prefetch_resid<MT>(p, t, g, resid, ctid);
       if (MLA && t.op == OP_UV) {
         if constexpr (MLA) mla_combine_input(p, t, ub, ub + p.xs_floats, ctid);
         if (ctid == 0) *rn_s = 1.f;
         cur_key = -1;
       } else if (key != cur_key || key < 0) {
-        const float rn = load_input(p, t, g, ub, red, ctid);
-        if (ctid == 0) *rn_s = rn;
+        float rnv[MT];
+        load_input<MT>(p, t, g, ub, red, ctid, rnv);
+        if (ctid == 0)
+#pragma unroll
+          for (int v = 0; v < MT; ++v) rn_s[v] = rnv[v];
         cur_key = key;
       }
       consumer_sync(kConsumerThreads);
       if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
-      const float rn = *rn_s;
+      float rnt[MT];
+#pragma unroll
+      for (int v = 0; v < MT; ++v) rnt[v] = rn_s[v];
+      const float rn = rnt[0];
       const int K8 = g.Kp >> 3;
       const float4* xl = reinterpret_cast<const float4*>(ub);
       const float4* xh = reinterpret_cast<const float4*>(ub + g.Kp / 2);
-      Best best{-INFINITY, 0x7fffffff};
+      Best best[MT];
+#pragma unroll
+      for (int v = 0; v < MT; ++v) best[v] = Best{-INFINITY, 0x7fffffff};
       // routed experts: the slot's weight folds into u; u holds the shared slices first
       float wsel = 1.f;
       int uoff = 0;
@@ -1421,7 +1529,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
-        if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+        if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;
           for (int r = 0; r < nr; r += 2) {
             const int np = min(2, nr - r);
@@ -1443,7 +1551,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
               p.u[uoff + n0 + r + k] = wsel * (a / (1.f + expf(-a)) * bb);
             }
           }
-        } else {
+        } else if (MT == 1) {
           for (int r = 0; r < nr; r += 4) {
             const int nv = min(4, nr - r);
             const uint4* r0 = sp + (size_t)r * K8;
@@ -1452,7 +1560,44 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
                         r0 + (size_t)min(3, nv - 1) * K8, K8, xl, xh, lane, o0, o1, o2, o3);
             const float v = reduce4(o0, o1, o2, o3, lane);
             const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-            if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, g, n0 + r + idx, v, rn, resid, best);
+            if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
+          }
+        } else if (g.nseg == 2) {  // MT tokens: gate / up rows as above, per token
+          const uint4* up = sp + (size_t)g.rps * K8;
+          const int vs = g.Kp / 4;  // float4 stride between the tokens' planes
+          for (int r = 0; r < nr; r += 2) {
+            const int np = min(2, nr - r);
+            float out[MT][4];
+            const uint4* g0 = sp + (size_t)r * K8;
+            const uint4* u0 = up + (size_t)r * K8;
+            if (np == 2) gemv_rows_mt<4, MT>(g0, g0 + K8, u0, u0 + K8, K8, xl, xh, vs, lane, out);
+            else gemv_rows_mt<2, MT>(g0, u0, u0, u0, K8, xl, xh, vs, lane, out);
+#pragma unroll
+            for (int v = 0; v < MT; ++v) {
+              const float val = reduce4(out[v][0], out[v][1], out[v][2], out[v][3], lane);
+              const float upv = __shfl_xor_sync(0xffffffffu, val, np == 2 ? 16 : 8);
+              const int k = (lane >> 3) & 1;
+              if ((np == 2 && (lane & 23) == 0) || (np == 1 && lane == 0)) {
+                const float a = val * rnt[v], bb = upv * rnt[v];
+                p.u[(size_t)v * p.F + uoff + n0 + r + k] = wsel * (a / (1.f + expf(-a)) * bb);
+              }
+            }
+          }
+        } else {
+          const int vs = g.Kp / 4;
+          for (int r = 0; r < nr; r += 4) {
+            const int nv = min(4, nr - r);
+            const uint4* r0 = sp + (size_t)r * K8;
+            float out[MT][4];
+            gemv_rows_mt_n<MT>(nv, r0, r0 + (size_t)min(1, nv - 1) * K8, r0 + (size_t)min(2, nv - 1) * K8,
+                               r0 + (size_t)min(3, nv - 1) * K8, K8, xl, xh, vs, lane, out);
+            const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+#pragma unroll
+            for (int v = 0; v < MT; ++v) {
+              const float val = reduce4(out[v][0], out[v][1], out[v][2], out[v][3], lane);
+              if ((lane & 7) == 0 && idx < nv)
+                gemv_emit(p, t, g, n0 + r + idx, val, rnt[v], resid + v * kMaxResidRows, best[v], v);
+            }
           }
         }
         __syncwarp();
@@ -1460,27 +1605,37 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       }
       if (t.op == OP_LM) {
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          Best o;
-          o.v = __shfl_xor_sync(0xffffffffu, best.v, off);
-          o.i = __shfl_xor_sync(0xffffffffu, best.i, off);
-          best_update(best, o.v, o.i);
-        }
-        if (lane == 0) {
-          red[warp] = best.v;
-          reinterpret_cast<int*>(red)[16 + warp] = best.i;
+        for (int v = 0; v < MT; ++v) {
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) {
+            Best o;
+            o.v = __shfl_xor_sync(0xffffffffu, best[v].v, off);
+            o.i = __shfl_xor_sync(0xffffffffu, best[v].i, off);
+            best_update(best[v], o.v, o.i);
+          }
+          if (lane == 0) {
+            red[warp * MT + v] = best[v].v;
+            reinterpret_cast<int*>(red)[32 + warp * MT + v] = best[v].i;
+          }
         }
       }
       consumer_sync(kConsumerThreads);
       if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
-      if (t.op == OP_LM && ctid == 0) {
-        Best bb{-INFINITY, 0x7fffffff};
-        for (int w = 0; w < kConsumerWarps; ++w) best_update(bb, red[w], reinterpret_cast<int*>(red)[16 + w]);
-        atomicMax(p.argmax_slot, pack_best(bb));
+      if (t.op == OP_LM && ctid == 0) {  // per token: this task's best, then the last task
+#pragma unroll
+        for (int v = 0; v < MT; ++v) {
+          Best bb{-INFINITY, 0x7fffffff};
+          for (int w = 0; w < kConsumerWarps; ++w)
+            best_update(bb, red[w * MT + v], reinterpret_cast<int*>(red)[32 + w * MT + v]);
+          atomicMax(p.argmax_slot + v, pack_best(bb));
+        }
         const uint32_t old = ticket_add(p.lm_ticket, 1u);
         if (((old + 1u) % (uint32_t)t.aux) == 0u) {
-          const unsigned long long w = atomicExch(p.argmax_slot, 0ull);
-          if (p.token_out) *p.token_out = (int32_t)(0xffffffffu - (uint32_t)(w & 0xffffffffull));
+#pragma unroll
+          for (int v = 0; v < MT; ++v) {
+            const unsigned long long w = atomicExch(p.argmax_slot + v, 0ull);
+            if (p.token_out) p.token_out[v] = (int32_t)(0xffffffffu - (uint32_t)(w & 0xffffffffull));
+          }
         }
       }
       if (t.op == OP_ROUTER) {  // the last router task of the layer selects the experts
@@ -1507,7 +1662,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
 }
 
 // ---- the kernel ----------------------------------------------------------------------------------
-template <bool MLA>
+template <bool MLA, int MT>
 __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t NS = (uint32_t)p.ring_stages;
@@ -1541,15 +1696,35 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
     producer(p, my, ntask, ring, full, empty, tags, threadIdx.x & 31);
     return;
   }
-  consumer<MLA>(p, my, ntask, ring, full, empty, tags, ub, misc);
+  consumer<MLA, MT>(p, my, ntask, ring, full, empty, tags, ub, misc);
 }
 
 // ---- host-side launch helpers ------------------------------------------------------------------
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla) {
-  auto k = mla ? engine_kernel<true> : engine_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
-  if (e != cudaSuccess) return e;
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, k, kThreads, smem_bytes);
+// The kernel instantiation for a stack kind and a number of tokens per step.
+static const void* kernel_for(bool mla, int m) {
+  if (mla) return reinterpret_cast<const void*>(engine_kernel<true, 1>);
+  switch (m) {
+    case 2: return reinterpret_cast<const void*>(engine_kernel<false, 2>);
+    case 3: return reinterpret_cast<const void*>(engine_kernel<false, 3>);
+    case 4: return reinterpret_cast<const void*>(engine_kernel<false, 4>);
+    default: return reinterpret_cast<const void*>(engine_kernel<false, 1>);
+  }
+}
+
+// Configure the instantiations a plan can launch (m = 1 .. max_m) and report how many
+// CTAs of the largest fit on an SM.
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m) {
+  *blocks_per_sm = 1 << 30;
+  for (int m = 1; m <= (mla ? 1 : max_m); ++m) {
+    const void* k = kernel_for(mla, m);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e != cudaSuccess) return e;
+    int b = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, kThreads, smem_bytes);
+    if (e != cudaSuccess) return e;
+    *blocks_per_sm = b < *blocks_per_sm ? b : *blocks_per_sm;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream, bool mla) {
@@ -1563,8 +1738,8 @@ cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return mla ? cudaLaunchKernelEx(&cfg, engine_kernel<true>, p)
-             : cudaLaunchKernelEx(&cfg, engine_kernel<false>, p);
+  void* args[] = {const_cast<Params*>(&p)};
+  return cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m), args);
 }
 
 }  // namespace tre

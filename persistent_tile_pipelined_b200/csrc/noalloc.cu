@@ -21,7 +21,7 @@
 #include "tre_internal.h"
 
 namespace tre {
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla = false);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 }  // namespace tre
@@ -64,7 +64,7 @@ tre_status setup_device(int dev, void** scratch) {
     g_scratch_dev[dev] = ptr;
   }
   int bps = 0;
-  cudaError_t e = engine_configure(kSmemLimit, &bps);
+  cudaError_t e = engine_configure(kSmemLimit, &bps, false, 1);
   if (e != cudaSuccess) return cuda_fail(e, "engine_configure");
   if (bps < 1) return fail(TRE_ERR_OCCUPANCY, "the persistent CTA does not fit on an SM");
   *scratch = g_scratch_dev[dev];
@@ -110,8 +110,8 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   if (st != TRE_OK) return st;
   if (!s.has_lm)
     return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: needs an embedding and LM head");
-  if (s.kind != TRE_LAYER_GQA)
-    return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: GQA stacks only");
+  if (s.kind != TRE_LAYER_GQA || s.M != 1)
+    return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: GQA stacks, one token per step");
   if (cfg->debug_flags & (TRE_DEBUG_HIDDEN | TRE_DEBUG_TRACE))
     return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: debug buffers are not available");
 
@@ -125,7 +125,7 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   const size_t o_ctr = cv.take<uint32_t>(s.n_counters);
   const size_t o_tick = cv.take<uint32_t>(s.Hkv);
   const size_t o_lmt = cv.take<uint32_t>(1);
-  const size_t o_arg = cv.take<unsigned long long>(1);
+  const size_t o_arg = cv.take<unsigned long long>(kMaxTokens);
   const size_t o_err = cv.take<int32_t>(4);  // error word, abort flag, status fallback [2]
   const size_t o_zero_end = cv.off;
   const size_t o_x = cv.take<float>(s.d);
@@ -241,6 +241,8 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   p.timeout_ns = 1000LL * (cfg->dep_timeout_us ? cfg->dep_timeout_us : 1000000);
   p.pf_window = cfg->l2_prefetch_kb > 0 ? 1024LL * cfg->l2_prefetch_kb : 1024LL * kDefaultPrefetchKB;
   p.token = token;
+  p.m = 1;
+  for (int v = 0; v < kMaxTokens; ++v) p.tokens[v] = token;
   p.pos = pos;
   p.epoch = 1;  // counters were just cleared
   if ((ce = engine_launch(p, s.nsm, s.smem_bytes, sm)) != cudaSuccess)

@@ -247,9 +247,14 @@ static tre_status validate(const tre_config& c) {
     return fail(TRE_ERR_INVALID_ARG, "has_embed_lm_head must be 0 or 1");
   if (c.has_embed_lm_head && c.vocab < 1) return fail(TRE_ERR_INVALID_ARG, "vocab must be >= 1");
   if (c.kv_capacity < 1) return fail(TRE_ERR_INVALID_ARG, "kv_capacity must be >= 1");
-  if (c.max_tokens_per_step > 1)
-    return fail(TRE_ERR_UNSUPPORTED, "multi-token steps are not implemented in this build");
-  if (c.max_tokens_per_step < 0) return fail(TRE_ERR_INVALID_ARG, "max_tokens_per_step < 0");
+  if (c.max_tokens_per_step < 0 || c.max_tokens_per_step > kMaxTokens)
+    return fail(TRE_ERR_INVALID_ARG, "max_tokens_per_step must be in [0, 4]");
+  if (c.max_tokens_per_step > 1) {
+    if (c.kind != TRE_LAYER_GQA)
+      return fail(TRE_ERR_UNSUPPORTED, "multi-token steps are implemented for GQA stacks only");
+    if (c.max_tokens_per_step * (c.n_q_heads / c.n_kv_heads) > 16)
+      return fail(TRE_ERR_UNSUPPORTED, "tokens x (q heads per kv head) above 16");
+  }
   if (!(c.rope_theta > 0.f)) return fail(TRE_ERR_INVALID_ARG, "rope_theta must be > 0");
   if (!(c.norm_eps >= 0.f)) return fail(TRE_ERR_INVALID_ARG, "norm_eps must be >= 0");
   if (c.dep_timeout_us < 0) return fail(TRE_ERR_INVALID_ARG, "dep_timeout_us < 0");
@@ -283,13 +288,14 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     s.VD = c.v_dim;
   }
   // an MLA output projection (K = H * v_dim) is staged in halves of at most 8192 inputs,
-  // so that the input planes leave room for a 5-deep ring of 36 KB stages
-  s.kpart_max = mla ? 8192 : kMaxKPart;
+  // so that the input planes leave room for a 5-deep ring of 36 KB stages; with M tokens
+  // per step the M input vectors share the planes
+  s.M = c.max_tokens_per_step < 1 ? 1 : c.max_tokens_per_step;
+  s.kpart_max = mla ? 8192 : (kMaxKPart / s.M) / 8 * 8;
   s.F = c.ffn;
   s.V = c.has_embed_lm_head ? c.vocab : 0;
   s.L = c.n_layers;
   s.cap = c.kv_capacity;
-  s.M = c.max_tokens_per_step < 1 ? 1 : c.max_tokens_per_step;
   s.nsm = nsm;
   s.has_lm = c.has_embed_lm_head;
   const bool moe = c.kind == TRE_LAYER_MOE;
@@ -307,8 +313,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
 
   // Inputs longer than kMaxKPart are staged in K-parts; ops that normalise their input
   // (QKV, gate/up, LM head) need the whole vector at once.
-  if (s.d > kMaxKPart)
-    return fail(TRE_ERR_UNSUPPORTED, "hidden above 16384 (normalised inputs are staged whole)");
+  if (s.d > s.kpart_max)
+    return fail(TRE_ERR_UNSUPPORTED, "hidden above 16384 / tokens per step (normalised inputs are staged whole)");
   // (input length, segments, K-part length) of every op the stack uses
   struct OpShape { int K, nseg, kp; };
   std::vector<OpShape> ops = {{s.d, 1, 0}, {s.Hq * s.D, 1, 0}, {s.d, 1, s.d}};
@@ -341,9 +347,13 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // positions per attention stage: MLA 32 latent rows; GQA 64 (four warps x 16 rows)
   s.pos_per_stage = mla ? kMlaPosPerStage : kMaxPosPerStage;
 
-  s.xs_floats = (xs + 7) / 8 * 8;
-  s.resid_floats = kMaxResidRows;
-  s.attn_floats = G * s.D + 2 * s.D + kConsumerWarps * (2 * G + G * s.D) + 16;
+  s.xs_floats = (s.M * xs + 7) / 8 * 8;
+  s.resid_floats = s.M * kMaxResidRows;
+  // attention scratch: q rows (M tokens x G heads), the M new k / v rows, per-warp
+  // (m, l, O) per row, scores of the new positions
+  const int rows = s.M * G;
+  s.attn_floats = rows * s.D + 2 * s.M * s.D + kConsumerWarps * (2 * rows + rows * s.D) +
+                  rows * s.M + 16;
   if (mla) {
     // score partials [8 warps][16][32] + P hi / lo (16 x 40 bf16 each) + head state; the
     // combine stages (m, l) of every split; the W_uk contraction sums [8][KL]
@@ -397,7 +407,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     b.mla_attention(l, groups, S, lat_task, cuk, (uint32_t)n3, ca);
     const int n5 = b.per_unit(OP_UV, l, H, s.VD, (int64_t)s.VD * s.KL * 2, ca,
                               (uint32_t)(groups * S), cuv);
-    const int n6 = b.gemv(OP_MO, l, s.d, H * s.VD, 1, cuv, (uint32_t)n5, co, s.resid_floats);
+    const int n6 = b.gemv(OP_MO, l, s.d, H * s.VD, 1, cuv, (uint32_t)n5, co, kMaxResidRows);
     prev_down = co;
     prev_down_count = (uint32_t)n6;
   }
@@ -410,11 +420,11 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
                             prev_down_count, cq, big);
     const int64_t kv_task_bytes = (int64_t)(s.cap - s.M) / S * s.D * 2 * 2;
     b.attention(l, s.Hkv, S, kv_task_bytes, cq, (uint32_t)nqkv, ca);
-    int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)s.Hkv, co, s.resid_floats);
+    int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)s.Hkv, co, kMaxResidRows);
     int nd;
     if (!moe) {
       int ng = b.gemv(OP_GU, l, s.F, s.d, 2, co, (uint32_t)no, cg, big);
-      nd = b.gemv(OP_DOWN, l, s.d, s.F, 1, cg, (uint32_t)ng, cd, s.resid_floats);
+      nd = b.gemv(OP_DOWN, l, s.d, s.F, 1, cg, (uint32_t)ng, cd, kMaxResidRows);
     } else {
       // Router rows first, then the shared expert (which needs no routing, so its weights
       // stream while the top-k is decided), then the selected experts' gate/up rows: their
@@ -473,7 +483,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   return TRE_OK;
 }
 
-int64_t step_bytes(const PlanShape& s, int pos) {
+int64_t step_bytes(const PlanShape& s, int pos, int m) {
   const int64_t d = s.d, D = s.D;
   if (s.kind == TRE_LAYER_MLA) {
     const int64_t H = s.Hq, C = s.KL + s.R;
@@ -491,8 +501,8 @@ int64_t step_bytes(const PlanShape& s, int pos) {
   int64_t per_layer = ((int64_t)(s.Hq + 2 * s.Hkv) * D * d + d * s.Hq * D + mlp) * 2 + 2 * d * 2;
   int64_t bytes = per_layer * s.L;
   bytes += (int64_t)s.L * s.Hkv * (int64_t)pos * D * 2 * 2;  // K and V read
-  bytes += (int64_t)s.L * s.Hkv * D * 2 * 2;                 // this token's K and V written
-  if (s.has_lm) bytes += (int64_t)s.V * d * 2 + d * 2 + d * 2 + (int64_t)s.V * 4;
+  bytes += (int64_t)s.L * s.Hkv * D * 2 * 2 * m;             // the m tokens' K and V written
+  if (s.has_lm) bytes += (int64_t)s.V * d * 2 + d * 2 + m * (d * 2 + (int64_t)s.V * 4);
   return bytes;
 }
 

@@ -100,4 +100,48 @@ __device__ __forceinline__ void gemv_rows_n(int nr, const uint4* r0, const uint4
   }
 }
 
+// ---- GEMV for MT tokens: one warp computes NR (<= 4) whole rows against MT input vectors -----
+// Token v's planes start vs float4s after token 0's.  Each weight vector is loaded once and
+// used for every token (the MT tokens give the FMA chains their independence).
+template <int NR, int MT>
+__device__ __forceinline__ void gemv_rows_mt(const uint4* r0, const uint4* r1, const uint4* r2,
+                                             const uint4* r3, int K8, const float4* __restrict__ xl,
+                                             const float4* __restrict__ xh, int vs, int lane,
+                                             float (&out)[MT][4]) {
+  const uint4* rp[4] = {r0, r1, r2, r3};
+  float acc[MT][NR];
+#pragma unroll
+  for (int v = 0; v < MT; ++v)
+#pragma unroll
+    for (int r = 0; r < NR; ++r) acc[v][r] = 0.f;
+  for (int j = lane; j < K8; j += 32) {
+    uint4 w[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) w[r] = rp[r][j];
+#pragma unroll
+    for (int v = 0; v < MT; ++v) {
+      const float4 x0 = xl[v * vs + j], x1 = xh[v * vs + j];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) acc[v][r] = dot8(w[r], x0, x1, acc[v][r]);
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < MT; ++v)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) out[v][r] = r < NR ? acc[v][r] : 0.f;
+}
+
+template <int MT>
+__device__ __forceinline__ void gemv_rows_mt_n(int nr, const uint4* r0, const uint4* r1,
+                                               const uint4* r2, const uint4* r3, int K8,
+                                               const float4* xl, const float4* xh, int vs,
+                                               int lane, float (&out)[MT][4]) {
+  switch (nr) {
+    case 4: gemv_rows_mt<4, MT>(r0, r1, r2, r3, K8, xl, xh, vs, lane, out); break;
+    case 3: gemv_rows_mt<3, MT>(r0, r1, r2, r3, K8, xl, xh, vs, lane, out); break;
+    case 2: gemv_rows_mt<2, MT>(r0, r1, r2, r3, K8, xl, xh, vs, lane, out); break;
+    default: gemv_rows_mt<1, MT>(r0, r1, r2, r3, K8, xl, xh, vs, lane, out); break;
+  }
+}
+
 }  // namespace tre

@@ -17,7 +17,7 @@
 #include "tre_internal.h"
 
 namespace tre {
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla = false);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 const char* last_error_cstr();
@@ -38,6 +38,7 @@ struct tre_engine {
   int32_t* status_dev = nullptr;
   Params base{};
   int32_t* token_buf = nullptr;
+  int last_m = 1;                // tokens of the last step (debug hidden layout)
   float* logits_buf = nullptr;
 };
 
@@ -250,7 +251,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   }
 
   int bps = 0;
-  CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA));
+  CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M));
   if (bps < 1) {
     set_error("tre_create: the persistent CTA does not fit on an SM");
     return TRE_ERR_OCCUPANCY;
@@ -284,13 +285,14 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_ctr = cv.take<uint32_t>(s.n_counters);
   size_t o_tick = cv.take<uint32_t>(std::max(s.Hkv, mla ? s.Hq / kMlaHeadGroup : 1));
   size_t o_lmt = cv.take<uint32_t>(1);
-  size_t o_arg = cv.take<unsigned long long>(1);
+  size_t o_arg = cv.take<unsigned long long>(kMaxTokens);
   size_t o_err = cv.take<int32_t>(2);
-  size_t o_x = cv.take<float>(s.d);
-  size_t o_h1 = cv.take<float>(s.d);
-  size_t o_qkv = cv.take<float>(qkv_n);
-  size_t o_attn = cv.take<float>((size_t)s.Hq * s.D);
-  size_t o_u = cv.take<float>(s.u_floats);
+  const size_t M = (size_t)s.M;  // per-token buffers: [M][...]
+  size_t o_x = cv.take<float>(M * s.d);
+  size_t o_h1 = cv.take<float>(M * s.d);
+  size_t o_qkv = cv.take<float>(M * qkv_n);
+  size_t o_attn = cv.take<float>(M * s.Hq * s.D);
+  size_t o_u = cv.take<float>(M * s.u_floats);
   const bool moe = s.kind == TRE_LAYER_MOE;
   size_t o_scores = cv.take<float>(moe ? s.E : 1);
   size_t o_ridx = cv.take<int32_t>(moe ? (size_t)s.L * s.topk : 1);
@@ -298,9 +300,9 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_rtick = cv.take<uint32_t>(1);
   size_t o_mpart = cv.take<float>(moe ? (size_t)(s.nshared + s.topk) * s.d : 1);
   size_t o_dtick = cv.take<uint32_t>(moe ? s.down_blocks : 1);
-  size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (mla ? mla_pstride(s.KL) : s.D + 2));
-  size_t o_logits = cv.take<float>(s.V > 0 ? s.V : 1);
-  size_t o_tok = cv.take<int32_t>(1);
+  size_t o_part = cv.take<float>(M * s.Hq * s.kv_splits * (mla ? mla_pstride(s.KL) : s.D + 2));
+  size_t o_logits = cv.take<float>(s.V > 0 ? M * s.V : 1);
+  size_t o_tok = cv.take<int32_t>(kMaxTokens);
   size_t o_inv = cv.take<double>(std::max(1, s.D / 2));
   size_t o_invr = cv.take<double>(std::max(1, s.R / 2));
   size_t o_cqkv = cv.take<float>(mla ? s.QL + C : 1);
@@ -312,7 +314,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_maps = cv.take<CUtensorMap>(maps.size() ? maps.size() : 1);
   const bool dbg_hidden = cfg->debug_flags & TRE_DEBUG_HIDDEN;
   const bool dbg_trace = cfg->debug_flags & TRE_DEBUG_TRACE;
-  size_t o_hidden = dbg_hidden ? cv.take<float>((size_t)s.L * s.d) : 0;
+  size_t o_hidden = dbg_hidden ? cv.take<float>((size_t)s.L * M * s.d) : 0;
   size_t o_trace = dbg_trace ? cv.take<long long>((size_t)tasks.size() * kTraceCols) : 0;
   e->block_bytes = cv.off;
   cudaError_t ce = cudaMalloc(&e->block, e->block_bytes);
@@ -398,6 +400,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.kv_maps = B + o_maps;
   p.QL = s.QL; p.KL = s.KL; p.R = s.R; p.NP = s.NP; p.VD = s.VD;
   p.kpart_max = s.kpart_max;
+  p.m = 1;
   p.err = reinterpret_cast<int32_t*>(B + o_err);
   p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
   p.status_host = e->status_dev;
@@ -426,18 +429,20 @@ static tre_status pending_device_error(tre_engine* e) {
   return (tre_status)code;
 }
 
-static tre_status launch_step(tre_engine* e, int32_t token, int32_t pos, cudaStream_t stream,
-                              float* logits_dev, int32_t* token_dev, const float* x_in,
-                              float* x_out) {
+static tre_status launch_step(tre_engine* e, const int32_t* tokens, int m, int32_t pos,
+                              cudaStream_t stream, float* logits_dev, int32_t* token_dev,
+                              const float* x_in, float* x_out) {
   tre_status st = pending_device_error(e);
   if (st != TRE_OK) return st;
-  if (pos < 0 || pos >= e->shape.cap) {
-    set_error("pos outside [0, kv_capacity)");
+  if (pos < 0 || pos + m > e->shape.cap) {
+    set_error("pos .. pos + tokens - 1 outside [0, kv_capacity)");
     return TRE_ERR_POS_RANGE;
   }
   CK(cudaSetDevice(e->device));
   Params p = e->base;
-  p.token = token;
+  p.m = m;
+  for (int v = 0; v < kMaxTokens; ++v) p.tokens[v] = v < m ? tokens[v] : tokens[0];
+  p.token = tokens[0];
   p.pos = pos;
   p.epoch = ++e->epoch;
   if (logits_dev) p.logits = logits_dev;
@@ -450,6 +455,7 @@ static tre_status launch_step(tre_engine* e, int32_t token, int32_t pos, cudaStr
     --e->epoch;
     return cuda_fail(ce, "launch of the persistent engine");
   }
+  e->last_m = m;
   e->last_stream = stream;
   return TRE_OK;
 }
@@ -472,7 +478,36 @@ TRE_EXPORT tre_status tre_decode_step(tre_engine* e, int32_t token, int32_t pos,
     set_error("tre_decode_step: logits_dev must be 16-byte aligned");
     return TRE_ERR_INVALID_ARG;
   }
-  return launch_step(e, token, pos, (cudaStream_t)stream, logits_dev, token_dev, nullptr, nullptr);
+  return launch_step(e, &token, 1, pos, (cudaStream_t)stream, logits_dev, token_dev, nullptr,
+                     nullptr);
+}
+
+TRE_EXPORT tre_status tre_decode_tokens(tre_engine* e, const int32_t* tokens_host, int32_t m,
+                                        int32_t pos, tre_stream stream, float* logits_dev,
+                                        int32_t* tokens_dev) {
+  if (!e || !tokens_host) {
+    set_error("tre_decode_tokens: NULL engine or tokens");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (!e->shape.has_lm) {
+    set_error("tre_decode_tokens: engine has no embedding / LM head");
+    return TRE_ERR_UNSUPPORTED;
+  }
+  if (m < 1 || m > e->shape.M) {
+    set_error("tre_decode_tokens: m outside [1, max_tokens_per_step]");
+    return TRE_ERR_INVALID_ARG;
+  }
+  for (int v = 0; v < m; ++v)
+    if (tokens_host[v] < 0 || tokens_host[v] >= e->shape.V) {
+      set_error("tre_decode_tokens: token outside [0, vocab)");
+      return TRE_ERR_INVALID_ARG;
+    }
+  if (logits_dev && ((uintptr_t)logits_dev & 15u)) {
+    set_error("tre_decode_tokens: logits_dev must be 16-byte aligned");
+    return TRE_ERR_INVALID_ARG;
+  }
+  return launch_step(e, tokens_host, m, pos, (cudaStream_t)stream, logits_dev, tokens_dev,
+                     nullptr, nullptr);
 }
 
 TRE_EXPORT tre_status tre_decode_step_host(tre_engine* e, int32_t token, int32_t pos,
@@ -513,7 +548,9 @@ TRE_EXPORT tre_status tre_layers_step(tre_engine* e, const float* x_in_dev, floa
     set_error("tre_layers_step: x_out_dev overlaps x_in_dev");
     return TRE_ERR_INVALID_ARG;
   }
-  return launch_step(e, 0, pos, (cudaStream_t)stream, nullptr, nullptr, x_in_dev, x_out_dev);
+  const int32_t none = 0;
+  return launch_step(e, &none, 1, pos, (cudaStream_t)stream, nullptr, nullptr, x_in_dev,
+                     x_out_dev);
 }
 
 TRE_EXPORT tre_status tre_debug_routing(tre_engine* e, int32_t* idx_host, float* w_host) {
@@ -565,7 +602,7 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
   CK(cudaMemsetAsync(p.router_ticket, 0, 4, s));
   if (e->shape.kind == TRE_LAYER_MOE)
     CK(cudaMemsetAsync(p.down_tickets, 0, (size_t)e->shape.down_blocks * 4, s));
-  CK(cudaMemsetAsync(p.argmax_slot, 0, 8, s));
+  CK(cudaMemsetAsync(p.argmax_slot, 0, 8 * kMaxTokens, s));
   CK(cudaMemsetAsync(p.err, 0, 8, s));  // error word + abort flag
   CK(cudaStreamSynchronize(s));
   std::memset(e->status_host, 0, 4 * sizeof(int32_t));
@@ -583,7 +620,8 @@ TRE_EXPORT tre_status tre_debug_hidden(tre_engine* e, float* hidden_dev, tre_str
     return TRE_ERR_INVALID_ARG;
   }
   CK(cudaSetDevice(e->device));
-  CK(cudaMemcpyAsync(hidden_dev, e->base.hidden, (size_t)e->shape.L * e->shape.d * sizeof(float),
+  CK(cudaMemcpyAsync(hidden_dev, e->base.hidden,
+                     (size_t)e->shape.L * e->last_m * e->shape.d * sizeof(float),
                      cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
   return TRE_OK;
 }
@@ -606,11 +644,15 @@ TRE_EXPORT tre_status tre_debug_trace(tre_engine* e, int64_t* trace_host, int32_
   return TRE_OK;
 }
 
-TRE_EXPORT tre_status tre_step_bytes(const tre_engine* e, int32_t pos, int64_t* bytes) {
+TRE_EXPORT tre_status tre_step_bytes(const tre_engine* e, int32_t pos, int32_t m, int64_t* bytes) {
   if (!e || !bytes) {
     set_error("tre_step_bytes: NULL argument");
     return TRE_ERR_INVALID_ARG;
   }
-  *bytes = step_bytes(e->shape, pos);
+  if (m < 1 || m > e->shape.M) {
+    set_error("tre_step_bytes: m outside [1, max_tokens_per_step]");
+    return TRE_ERR_INVALID_ARG;
+  }
+  *bytes = step_bytes(e->shape, pos, m);
   return TRE_OK;
 }

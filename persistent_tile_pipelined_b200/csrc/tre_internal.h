@@ -22,6 +22,7 @@ constexpr int kMaxExperts = 512;         // routed experts per MoE layer (scores
 constexpr int kMaxTopK = 32;
 constexpr int kDefaultPrefetchKB = 0;    // next-task L2 prefetch: opt-in (measured 4% slower)
 constexpr int kMaxStageBytes = 65536;
+constexpr int kMaxTokens = 4;            // tokens per step (multi-token verify tiles)
 constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per block
 
 #ifdef __CUDACC__
@@ -139,13 +140,14 @@ struct Params {
   uint32_t* counters;
   uint32_t* tickets;               // [Hkv] split-KV arrival tickets
   uint32_t* lm_ticket;
-  unsigned long long* argmax_slot;
+  unsigned long long* argmax_slot;  // [kMaxTokens]
   const LayerPtrs* layers;
   const uint16_t* embed;
   const uint16_t* final_norm;
   const uint16_t* lm_head;
   const float* x_in;               // layer-only input (NULL: embedding row)
   float* x_out;                    // layer-only output (NULL: none)
+  // per-token buffers are [m][...] (token v's vector at v * length)
   float* x;                        // residual stream [d]
   float* h1;                       // after attention [d]
   float* qkv;                      // [(Hq + 2 Hkv) D]
@@ -181,6 +183,8 @@ struct Params {
   int nsplit, pps, stage_bytes, ring_stages, xs_floats, ub_floats;
   float eps;
   int token, pos;
+  int m;                           // tokens this step (1 .. kMaxTokens): positions pos .. pos + m - 1
+  int32_t tokens[kMaxTokens];
   uint32_t epoch;
   int flags;
   long long timeout_ns;
@@ -198,7 +202,7 @@ namespace tre {
 tre_status plan_build(const tre_config& cfg, int nsm, int smem_limit, PlanShape* shape,
                       std::vector<Task>* tasks, std::vector<int32_t>* sm_begin,
                       std::vector<int64_t>* sm_bytes);
-int64_t step_bytes(const PlanShape& s, int pos);
+int64_t step_bytes(const PlanShape& s, int pos, int m = 1);
 void set_error(const std::string& msg);
 // Host only, allocates nothing: a 2-D tensor map (128 bytes at out128) over a bf16 cache
 // [rows][C] with 64-column x box_rows boxes and the 128-byte swizzle (tre_api.cu).

@@ -69,7 +69,7 @@ class tre_plan_info(ctypes.Structure):
 
 EXPORTED = ("tre_create", "tre_destroy", "tre_decode_step", "tre_decode_step_host",
             "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
-            "tre_get_status", "tre_reset", "tre_debug_hidden", "tre_debug_trace",
+            "tre_decode_tokens", "tre_get_status", "tre_reset", "tre_debug_hidden", "tre_debug_trace",
             "tre_step_bytes", "tre_plan_inspect", "tre_plan_tasks", "tre_last_error")
 
 
@@ -88,12 +88,13 @@ def _load() -> ctypes.CDLL:
     L.tre_decode_step_static.argtypes = [ctypes.POINTER(tre_config), ctypes.POINTER(tre_weights),
                                          i32, i32, vp, vp, vp, vp]
     L.tre_layers_step.argtypes = [vp, vp, vp, i32, vp]
+    L.tre_decode_tokens.argtypes = [vp, vp, i32, i32, vp, vp, vp]
     L.tre_debug_routing.argtypes = [vp, vp, vp]
     L.tre_get_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.tre_reset.argtypes = [vp, vp]
     L.tre_debug_hidden.argtypes = [vp, vp, vp]
     L.tre_debug_trace.argtypes = [vp, vp, ctypes.POINTER(i32)]
-    L.tre_step_bytes.argtypes = [vp, i32, ctypes.POINTER(i64)]
+    L.tre_step_bytes.argtypes = [vp, i32, i32, ctypes.POINTER(i64)]
     L.tre_plan_inspect.argtypes = [ctypes.POINTER(tre_config), i32, i32,
                                    ctypes.POINTER(tre_plan_info)]
     L.tre_plan_tasks.argtypes = [ctypes.POINTER(tre_config), i32, i32, vp, i32, vp]
@@ -102,7 +103,7 @@ def _load() -> ctypes.CDLL:
     L.tre_last_error.restype = ctypes.c_char_p
     for name in ("tre_create", "tre_decode_step", "tre_decode_step_host",
                  "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
-                 "tre_get_status",
+                 "tre_decode_tokens", "tre_get_status",
                  "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
                  "tre_plan_inspect"):
         getattr(L, name).restype = ctypes.c_int
@@ -189,10 +190,18 @@ def tre_reset(h, stream: int = 0) -> None:
     check(lib.tre_reset(h, ctypes.c_void_p(stream or None)), "tre_reset")
 
 
-def tre_step_bytes(h, pos: int) -> int:
+def tre_step_bytes(h, pos: int, m: int = 1) -> int:
     b = ctypes.c_int64()
-    check(lib.tre_step_bytes(h, int(pos), ctypes.byref(b)), "tre_step_bytes")
+    check(lib.tre_step_bytes(h, int(pos), int(m), ctypes.byref(b)), "tre_step_bytes")
     return b.value
+
+
+def tre_decode_tokens(h, tokens, pos: int, stream: int = 0, logits_dev: int = 0,
+                      tokens_dev: int = 0) -> int:
+    arr = (ctypes.c_int32 * len(tokens))(*[int(t) for t in tokens])
+    return lib.tre_decode_tokens(h, arr, len(tokens), int(pos), ctypes.c_void_p(stream or None),
+                                 ctypes.c_void_p(logits_dev or None),
+                                 ctypes.c_void_p(tokens_dev or None))
 
 
 def tre_plan_inspect(cfg: tre_config, num_sms: int = 148, smem_per_block: int = 232448):
@@ -365,6 +374,15 @@ class Engine:
         s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
         return tre_decode_step_host(self.h, token, pos, s, logits_host)
 
+    def step_tokens(self, tokens, pos: int, logits=None, tokens_out=None, stream=None) -> None:
+        """Enqueue one step over len(tokens) consecutive tokens at pos .. pos + m - 1."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        check(tre_decode_tokens(self.h, tokens, pos, s,
+                                logits.data_ptr() if logits is not None else 0,
+                                tokens_out.data_ptr() if tokens_out is not None else 0),
+              "tre_decode_tokens")
+
     def layers_step(self, x_in, x_out, pos: int, stream=None) -> None:
         """Enqueue one layers-only step: x_out = stack(x_in) (device fp32[hidden] tensors)."""
         import torch
@@ -382,10 +400,12 @@ class Engine:
         s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
         tre_reset(self.h, s)
 
-    def hidden(self):
+    def hidden(self, m: int = 1):
+        """Residual stream after every layer of the last step: [L][d] (m = 1) or [L][m][d]."""
         import torch
-        out = torch.empty((self.cfg.n_layers, self.cfg.hidden), dtype=torch.float32,
-                          device=f"cuda:{self.device}")
+        shape = (self.cfg.n_layers, self.cfg.hidden) if m == 1 else \
+            (self.cfg.n_layers, m, self.cfg.hidden)
+        out = torch.empty(shape, dtype=torch.float32, device=f"cuda:{self.device}")
         check(lib.tre_debug_hidden(self.h, ctypes.c_void_p(out.data_ptr()),
                                    ctypes.c_void_p(torch.cuda.current_stream(self.device).cuda_stream)),
               "tre_debug_hidden")
@@ -399,5 +419,5 @@ class Engine:
               "tre_debug_trace")
         return buf
 
-    def step_bytes(self, pos: int) -> int:
-        return tre_step_bytes(self.h, pos)
+    def step_bytes(self, pos: int, m: int = 1) -> int:
+        return tre_step_bytes(self.h, pos, m)

@@ -201,6 +201,9 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
             if len(ids):
                 counts = np.bincount(sm_of[ids], minlength=nsm)
                 assert counts.max() <= -(-len(ids) // nsm), (l, counts.max())
+    # tasks that stage residual rows take at most 512 rows (the per-token residual buffer)
+    resid_ops = gemv & np.isin(T["op"], (OP_O, OP_DOWN, OP_MO))
+    assert ((T["r1"] - T["r0"])[resid_ops] <= 512).all()
     # LM tasks carry the LM task count
     lm = (T["type"] == T_GEMV) & (T["op"] == OP_LM)
     assert (T["aux"][lm] == lm.sum()).all()
@@ -223,7 +226,7 @@ def test_llama8b_plan_is_byte_balanced():
     ("kind", 2, tre.TRE_ERR_UNSUPPORTED),      # MoE with n_experts = 0 (a GQA config)
     ("hidden", 260, tre.TRE_ERR_INVALID_ARG), ("n_kv_heads", 3, tre.TRE_ERR_INVALID_ARG),
     ("head_dim", 96, tre.TRE_ERR_UNSUPPORTED), ("ffn", 690, tre.TRE_ERR_INVALID_ARG),
-    ("kv_capacity", 0, tre.TRE_ERR_INVALID_ARG), ("max_tokens_per_step", 4, tre.TRE_ERR_UNSUPPORTED),
+    ("kv_capacity", 0, tre.TRE_ERR_INVALID_ARG), ("max_tokens_per_step", 5, tre.TRE_ERR_INVALID_ARG),
     ("stage_bytes", 1000, tre.TRE_ERR_INVALID_ARG), ("rope_theta", 0.0, tre.TRE_ERR_INVALID_ARG),
 ])
 def test_plan_rejects_bad_configs(field, value, status):
@@ -285,6 +288,39 @@ def test_mla_plan_bytes_and_stage():
     assert info.stage_bytes == C * 64          # one latent tile of 32 rows per stage
     assert info.ring_stages >= 5
     assert info.kv_bytes_at_capacity == wl.n_layers * wl.prefill * C * 2
+
+
+@pytest.mark.parametrize("wl,m", [(W.TINY, 2), (W.TINY, 4), (W.LLAMA8B, 4),
+                                  (W.TINY.replace(n_q_heads=8, n_kv_heads=1), 2)],
+                         ids=["tiny-m2", "tiny-m4", "8b-m4", "g8-m2"])
+def test_multi_token_plans(wl, m):
+    """M tokens per step: the input planes hold M vectors, so long inputs are cut into
+    K-parts of at most 16384 / M floats; the plan still fits one CTA per SM."""
+    cfg = tre.config_from_workload(wl, max_tokens_per_step=m)
+    info = tre.tre_plan_inspect(cfg)
+    tasks, _ = tre.tre_plan_tasks(cfg)
+    T = decode_tasks(tasks)
+    down = (T["type"] == T_GEMV) & (T["op"] == OP_DOWN)
+    kmax = (16384 // m) // 8 * 8
+    assert (T["aux"][down] >> 8).max() == -(-wl.ffn // kmax)
+    assert info.smem_bytes <= 232448 and info.ring_stages >= 2
+    resid_ops = (T["type"] == T_GEMV) & np.isin(T["op"], (OP_O, OP_DOWN))
+    assert ((T["r1"] - T["r0"])[resid_ops] <= 512).all()
+    # the same weights are streamed whatever the token count
+    one = tre.tre_plan_inspect(tre.config_from_workload(wl))
+    assert info.weight_bytes == one.weight_bytes
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(max_tokens_per_step=4, n_q_heads=8, n_kv_heads=1), tre.TRE_ERR_UNSUPPORTED),  # 32 rows
+    (dict(max_tokens_per_step=2), tre.TRE_ERR_UNSUPPORTED),                            # MoE
+])
+def test_multi_token_rejections(over, status):
+    import ctypes
+    base = W.TINY if "n_q_heads" in over else MOE_SMALL
+    cfg = tre.config_from_workload(base, **over)
+    info = tre.tre_plan_info()
+    assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status
 
 
 def test_reserved_fields_must_be_zero():

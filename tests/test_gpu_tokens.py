@@ -1,0 +1,118 @@
+"""GPU parity of multi-token steps (tre_decode_tokens: m consecutive tokens of one sequence
+per launch, causal among themselves) against the fp64 CPU oracle run as m successive
+single-token decode steps with the same tokens.
+
+Bar: per token, the logits and every layer's hidden state within 2e-2 (normwise), the
+in-kernel argmax equal to the host argmax of the engine's own logits, and the appended K / V
+rows within one bf16 ulp of each row's largest entry.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from persistent_tile_pipelined_b200.synth import token_id
+from persistent_tile_pipelined_b200.synth import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from persistent_tile_pipelined_b200 import tre  # noqa: E402
+
+TOL = 2e-2
+ORC = oracle.Oracle(64)
+
+
+def relerr(g, o):
+    g, o = np.asarray(g, np.float64), np.asarray(o, np.float64)
+    return float(np.abs(g - o).max() / max(np.abs(o).max(), 1e-30))
+
+
+def run_tokens(wl, ms, max_m=4, check_hidden=True, **cfg_over):
+    """Steps of ms[i] tokens each, from pos = prefill; tokens from the seeded stream."""
+    model = W.gen_gqa_model(wl)
+    dev = tre.upload_gqa_model(model)
+    debug = tre.TRE_DEBUG_HIDDEN if check_hidden else 0
+    eng = tre.Engine(tre.config_from_workload(wl, max_tokens_per_step=max_m, debug_flags=debug,
+                                              **cfg_over), dev)
+    logits = torch.empty((max_m, wl.vocab), dtype=torch.float32, device="cuda")
+    toks_dev = torch.empty(max_m, dtype=torch.int32, device="cuda")
+    pos, k = wl.prefill, 0
+    for m in ms:
+        toks = [token_id(wl.seed, wl.vocab, k + v) for v in range(m)]
+        k += m
+        eng.step_tokens(toks, pos, logits[:m], toks_dev[:m])
+        torch.cuda.synchronize()
+        assert eng.status() == (0, 0)
+        g = logits[:m].cpu().numpy()
+        gt = toks_dev[:m].cpu().numpy()
+        hid = eng.hidden(m).cpu().numpy() if check_hidden else None
+        for v in range(m):
+            ref_logits, ref_hidden = ORC.decode_step(wl, model, toks[v], pos + v,
+                                                     want_hidden=check_hidden)
+            e = relerr(g[v], ref_logits)
+            assert e <= TOL, f"token {v} of {m}: logits rel err {e:.3g} at pos {pos + v}"
+            assert gt[v] == int(np.argmax(g[v])), "in-kernel argmax differs from host argmax"
+            if check_hidden:
+                hv = hid[:, v] if m > 1 else hid
+                for l in range(wl.n_layers):
+                    el = relerr(hv[l], ref_hidden[l])
+                    assert el <= TOL, f"token {v}: layer {l} hidden rel err {el:.3g}"
+        pos += m
+    # Appended K / V rows.  Layer 0's rows come from the embedding rows, which both sides
+    # read exactly: each row is within one bf16 ulp (2^-8) of its largest entry (the sides
+    # round fp32 / fp64 values to bf16).  Later layers' rows inherit the layer input's
+    # difference, so they are held to the hidden-state bar (2e-2 normwise per row).
+    start = wl.prefill
+    for l in range(wl.n_layers):
+        for name in ("k_cache", "v_cache"):
+            gw = dev[name][l].view(torch.int16).cpu().numpy().view(np.uint16)
+            ow = model[name][l]
+            assert np.array_equal(gw[:, :start], ow[:, :start])
+            gv = (gw[:, start:pos].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            ov = (ow[:, start:pos].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            row_max = np.abs(ov).max(axis=-1, keepdims=True)
+            worst = float((np.abs(gv - ov) / row_max).max())
+            bound = 2.0 ** -8 if l == 0 else TOL
+            assert worst <= bound, f"{name}[{l}]: row error {worst:.3g} > {bound:.3g}"
+    eng.close()
+
+
+@pytest.mark.parametrize("over,ms,max_m", [
+    (dict(decode_steps=10), [4, 1, 3, 2], 4),                              # G 2: 8 rows, packed
+    (dict(n_q_heads=8, n_kv_heads=2, decode_steps=10), [4, 2, 4], 4),      # G 4: 16 rows
+    (dict(n_q_heads=8, n_kv_heads=1, decode_steps=6), [2, 2, 1], 2),       # G 8: 16 rows
+    (dict(n_q_heads=8, n_kv_heads=4, head_dim=128, decode_steps=8), [4, 3], 4),   # D 128
+    (dict(hidden=264, ffn=696, vocab=1001, decode_steps=7), [3, 4], 4),    # ragged K / N
+    (dict(prefill=0, decode_steps=6), [4, 2], 4),                          # from position 0
+    (dict(prefill=61, decode_steps=4), [4], 4),                            # fills the cache
+], ids=["g2", "g4-16rows", "g8-m2", "d128", "ragged", "pos0", "full-cache"])
+def test_multi_token_steps(over, ms, max_m):
+    run_tokens(W.TINY.replace(**over), ms, max_m)
+
+
+@pytest.mark.parametrize("cfg", [dict(num_sms=5), dict(kv_splits=1), dict(kv_splits=7)],
+                         ids=["sms5", "split1", "split7"])
+def test_multi_token_launch_shapes(cfg):
+    run_tokens(W.TINY.replace(decode_steps=8), [4, 4], 4, **cfg)
+
+
+def test_tokens_argument_errors():
+    wl = W.TINY.replace(decode_steps=4)
+    model = W.gen_gqa_model(wl)
+    dev = tre.upload_gqa_model(model)
+    eng = tre.Engine(tre.config_from_workload(wl, max_tokens_per_step=2), dev)
+    s = torch.cuda.current_stream().cuda_stream
+    assert tre.tre_decode_tokens(eng.h, [1, 2, 3], wl.prefill, s) == tre.TRE_ERR_INVALID_ARG
+    assert tre.tre_decode_tokens(eng.h, [1, wl.vocab], wl.prefill, s) == tre.TRE_ERR_INVALID_ARG
+    assert tre.tre_decode_tokens(eng.h, [1, 2], wl.kv_capacity - 1, s) == tre.TRE_ERR_POS_RANGE
+    eng.close()
+
+
+@pytest.mark.slow
+def test_llama8b_four_token_steps():
+    """The 8B-shaped stack with 4-token steps in the benchmark's launch configuration:
+    every token's logits and layer hidden states over 3 steps."""
+    run_tokens(W.LLAMA8B.replace(decode_steps=12), [4, 4, 4], 4)
