@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="engine", choices=["engine", "reference"])
     ap.add_argument("--workload", default="llama3-8b-shaped")
+    ap.add_argument("--tokens-per-step", type=int, default=1,
+                    help="tokens per launch (1..4): multi-token verify steps via tre_decode_tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-layers", type=int, default=4)
     ap.add_argument("--trace", default="", help="write a per-task trace of one step (JSON)")
@@ -357,13 +359,20 @@ def run_engine(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     wl = W.WORKLOADS[args.workload]
-    K, Wm = args.steps, args.warmup
-    wl = wl.replace(decode_steps=K + Wm, seed=wl.seed + rank)
+    K, Wm, M = args.steps, args.warmup, args.tokens_per_step
+    wl = wl.replace(decode_steps=K + Wm, tokens_per_step=M, seed=wl.seed + rank)
     eng, model = build_engine(wl, local_rank, args.flags)
     stream = torch.cuda.current_stream(local_rank)
     s_ptr = stream.cuda_stream
-    tokens = [token_id(wl.seed, wl.vocab, i) for i in range(K + Wm)]
-    positions = [wl.prefill + i for i in range(K + Wm)]
+    # step i takes tokens i M .. i M + M - 1 of the seeded stream at positions prefill + i M ..
+    tokens = [[token_id(wl.seed, wl.vocab, i * M + v) for v in range(M)] for i in range(K + Wm)]
+    positions = [wl.prefill + i * M for i in range(K + Wm)]
+
+    def launch(i):
+        if M == 1:
+            eng.step(tokens[i][0], positions[i], stream=s_ptr)
+        else:
+            eng.step_tokens(tokens[i], positions[i], stream=s_ptr)
 
     def barrier():
         if world > 1:
@@ -372,7 +381,7 @@ def run_engine(args, rank, world, local_rank):
 
     # warm-up
     for i in range(Wm):
-        eng.step(tokens[i], positions[i], stream=s_ptr)
+        launch(i)
     torch.cuda.synchronize(local_rank)
     assert eng.status() == (0, 0), eng.status()
 
@@ -386,7 +395,7 @@ def run_engine(args, rank, world, local_rank):
     tw0 = time.time()
     ev[0].record(stream)
     for i in range(K):
-        eng.step(tokens[Wm + i], positions[Wm + i], stream=s_ptr)
+        launch(Wm + i)
         ev[i + 1].record(stream)
     torch.cuda.synchronize(local_rank)
     tw1 = time.time()
@@ -397,20 +406,25 @@ def run_engine(args, rank, world, local_rank):
     st = eng.status()
     assert st == (0, 0), st
 
-    # ---- end to end through the C ABI: greedy loop, token back to the host every step
-    tok = tokens[0]
+    # ---- end to end through the C ABI: greedy loop, token(s) back to the host every step
+    tok = tokens[0][0]
+    tok_dev = torch.empty(M, dtype=torch.int32, device=f"cuda:{local_rank}")
     barrier()
     tw0 = time.time()
     t0 = time.perf_counter()
     for i in range(K):
-        tok = eng.step_host(tok, positions[Wm + i], stream=s_ptr)
+        if M == 1:
+            tok = eng.step_host(tok, positions[Wm + i], stream=s_ptr)
+        else:   # verify the next M tokens, read the M argmax tokens back
+            eng.step_tokens(tokens[Wm + i], positions[Wm + i], tokens_out=tok_dev, stream=s_ptr)
+            tok = tok_dev.cpu()
     e2e_s = time.perf_counter() - t0
     tw1 = time.time()
     barrier()
     sampler.mark(tw0, tw1)
     clocks = sampler.stop()
 
-    step_bytes = float(np.mean([eng.step_bytes(positions[Wm + i]) for i in range(K)]))
+    step_bytes = float(np.mean([eng.step_bytes(positions[Wm + i], M) for i in range(K)]))
     trace_path = args.trace if rank == 0 else ""
     eng.close()
     del model
@@ -469,12 +483,12 @@ def main():
     if W.WORKLOADS[args.workload].kind != "gqa":
         return main_layers(args, rank, world, local_rank)
     wl, dev_s, e2e_s, launch_ms, step_bytes, clocks = run_engine(args, rank, world, local_rank)
-    K = args.steps
+    K, M = args.steps, args.tokens_per_step
     peak, peak_kind = peaks()
     achieved = step_bytes / (launch_ms / 1e3) / 1e9
     line = {
         "metric": METRIC,
-        "value": world * K / dev_s,
+        "value": world * K * M / dev_s,
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -486,7 +500,9 @@ def main():
         "dtype": "bf16",
         "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
         "config": {
-            "workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions",
+            "workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions" +
+                        (f", {M} tokens per step (causal verify tiles)" if M > 1 else ""),
+            "tokens_per_step": M,
             "layers": wl.n_layers, "hidden": wl.hidden, "q_heads": wl.n_q_heads,
             "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "ffn": wl.ffn,
             "vocab": wl.vocab, "kv_positions": wl.prefill, "batch": 1,
@@ -502,8 +518,8 @@ def main():
             "kernel": "tre::engine_kernel",
             "algorithmic_bytes_per_launch": step_bytes,
         },
-        "e2e": {"value": world * K / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 4,
-                "d2h_bytes_per_step": 4,
+        "e2e": {"value": world * K * M / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 4 * M,
+                "d2h_bytes_per_step": 4 * M,
                 "note": "greedy loop via tre_decode_step_host: token in as a kernel argument, "
                         "argmax token back to pinned-less host memory, host wall time"},
         "gpu_launches": K,

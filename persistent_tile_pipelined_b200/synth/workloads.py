@@ -90,7 +90,13 @@ MOE4 = Workload(name="moe-4L-d7168", kind="moe", n_layers=4, hidden=7168, n_q_he
                 n_kv_heads=8, head_dim=128, prefill=4096, decode_steps=1, rope_theta=1e4,
                 norm_eps=1e-6, n_experts=256, top_k=8, n_shared=1, expert_ffn=2048)
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L, MLA4, MOE4)}
+# Long-context sweep on the 8B-shaped stack: 8192 / 32768 / 131072 cached positions.
+LLAMA8B_KV8K = LLAMA8B.replace(name="llama3-8b-shaped-kv8k", prefill=8192)
+LLAMA8B_KV32K = LLAMA8B.replace(name="llama3-8b-shaped-kv32k", prefill=32768)
+LLAMA8B_KV128K = LLAMA8B.replace(name="llama3-8b-shaped-kv128k", prefill=131072)
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L, MLA4, MOE4, LLAMA8B_KV8K,
+                                 LLAMA8B_KV32K, LLAMA8B_KV128K)}
 
 
 def gqa_layer_shapes(w: Workload) -> List[tuple]:
