@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-layers", type=int, default=4)
     ap.add_argument("--trace", default="", help="write a per-task trace of one step (JSON)")
+    ap.add_argument("--config", action="append", default=[], metavar="FIELD=VALUE",
+                    help="engine config override (launch shape, K-part limit); repeatable")
     ap.add_argument("--flags", type=int, default=0,
                     help="engine debug flags for the timed engine (8 = no cross-op prefetch)")
     return ap.parse_args()
@@ -155,7 +157,16 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workload -------------
 
-def build_engine(wl, device: int, debug_flags: int = 0):
+def config_overrides(items):
+    """FIELD=VALUE strings -> {field: int}."""
+    out = {}
+    for it in items or []:
+        k, v = it.split("=", 1)
+        out[k.strip()] = int(v)
+    return out
+
+
+def build_engine(wl, device: int, debug_flags: int = 0, overrides=None):
     """Generate the synthetic model tensor by tensor (host generator -> device) so the
     host holds at most one tensor at a time."""
     import torch
@@ -181,11 +192,11 @@ def build_engine(wl, device: int, debug_flags: int = 0):
     model["final_norm"] = up(W.gen_tensor(wl, TID_FINAL_NORM, (wl.hidden,), "g"))
     model["lm_head"] = up(W.gen_tensor(wl, TID_LM_HEAD, (wl.vocab, wl.hidden), "w"))
     torch.cuda.synchronize(device)
-    cfg = tre.config_from_workload(wl, debug_flags=debug_flags)
+    cfg = tre.config_from_workload(wl, debug_flags=debug_flags, **(overrides or {}))
     return tre.Engine(cfg, model, device), model
 
 
-def build_layers_engine(wl, device: int, debug_flags: int = 0):
+def build_layers_engine(wl, device: int, debug_flags: int = 0, overrides=None):
     """A layers-only stack (MoE or MLA layers, no embedding / LM head): non-expert tensors
     and caches from the workload generator, routed experts generated one at a time and
     stacked on the device."""
@@ -203,7 +214,7 @@ def build_layers_engine(wl, device: int, debug_flags: int = 0):
     else:
         raise SystemExit(f"layers-only workload kind {wl.kind!r} is not built")
     torch.cuda.synchronize(device)
-    cfg = tre.config_from_workload(wl, debug_flags=debug_flags)
+    cfg = tre.config_from_workload(wl, debug_flags=debug_flags, **(overrides or {}))
     return tre.Engine(cfg, dmodel, device), dmodel
 
 
@@ -220,7 +231,7 @@ def run_layers(args, rank, world, local_rank):
     K, Wm = args.steps, args.warmup
     wl = W.WORKLOADS[args.workload].replace(decode_steps=K + Wm)
     wl = wl.replace(seed=wl.seed + rank)
-    eng, dmodel = build_layers_engine(wl, local_rank, args.flags)
+    eng, dmodel = build_layers_engine(wl, local_rank, args.flags, config_overrides(args.config))
     stream = torch.cuda.current_stream(local_rank)
     s_ptr = stream.cuda_stream
     xs_host = [normal_f32(wl.seed + i, TID_X_IN, (wl.hidden,)) for i in range(K + Wm)]
@@ -361,7 +372,7 @@ def run_engine(args, rank, world, local_rank):
     wl = W.WORKLOADS[args.workload]
     K, Wm, M = args.steps, args.warmup, args.tokens_per_step
     wl = wl.replace(decode_steps=K + Wm, tokens_per_step=M, seed=wl.seed + rank)
-    eng, model = build_engine(wl, local_rank, args.flags)
+    eng, model = build_engine(wl, local_rank, args.flags, config_overrides(args.config))
     stream = torch.cuda.current_stream(local_rank)
     s_ptr = stream.cuda_stream
     # step i takes tokens i M .. i M + M - 1 of the seeded stream at positions prefill + i M ..
@@ -503,6 +514,7 @@ def main():
             "workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions" +
                         (f", {M} tokens per step (causal verify tiles)" if M > 1 else ""),
             "tokens_per_step": M,
+            "engine_config": config_overrides(args.config),
             "layers": wl.n_layers, "hidden": wl.hidden, "q_heads": wl.n_q_heads,
             "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "ffn": wl.ffn,
             "vocab": wl.vocab, "kv_positions": wl.prefill, "batch": 1,

@@ -113,7 +113,15 @@ typedef struct {
   int32_t l2_prefetch_kb;       /* per-SM budget (KiB) for asking L2 for the next task's
                                    bytes when a task starts; <= 0 = off (the default:
                                    measured slower on the 8B-shaped stack)              */
-  int32_t reserved[7];          /* must be zero                                         */
+  int32_t gemv_kpart_max;       /* longest input slice (floats) a GEMV task stages; longer
+                                   inputs (not the normalised ones) run in K-parts;
+                                   0 = the planner's choice (16384 / tokens per step;
+                                   8192 for MLA)                                         */
+  int32_t stream_policy;        /* when the producer streams the next op's tiles:
+                                   1 = as soon as ring slots free up; 2 = once this SM
+                                   has published the current op (its publish then does
+                                   not wait behind in-flight copies); 0 = default (2)   */
+  int32_t reserved[5];          /* must be zero                                         */
 } tre_config;
 
 /* Per-layer tensor slots.  layer_w[l * TRE_W_SLOTS + slot] is the device pointer of

@@ -384,8 +384,14 @@ __device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, in
 // its piece.  When it starts a task it first asks L2 for the next task's bytes (up to
 // pf_window): weights and cached KV never depend on this step's activations, so HBM keeps
 // streaming through op boundaries even while the shared-memory ring is full.
+// A new op starts at task b (a different op, layer or task type than task a).
+__device__ __forceinline__ bool op_boundary(const Task& a, const Task& b) {
+  return a.type != b.type || a.op != b.op || a.layer != b.layer;
+}
+
 __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ring,
-                         uint64_t* full, uint64_t* empty, uint32_t* tags, int lane) {
+                         uint64_t* full, uint64_t* empty, uint32_t* tags,
+                         const volatile int* done, int lane) {
   const uint64_t pol = l2_policy_evict_first();
   const uint32_t NS = (uint32_t)p.ring_stages;
   const uint32_t SB = (uint32_t)p.stage_bytes;
@@ -398,6 +404,24 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
     if (no_overlap) {
       bool r = true;
       if (lane == 0) r = wait_dep(p, t);
+      ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
+    if (p.hold_next_op && ti > 0 && op_boundary(my[ti - 1], t)) {
+      // hold the next op's tiles until this SM's consumers have finished (and published)
+      // the previous task, so that their publish does not wait behind queued copies
+      bool r = true;
+      if (lane == 0) {
+        const uint64_t w0 = globaltimer_ns();
+        for (uint32_t it = 1; *done < ti; ++it) {
+          __nanosleep(32);
+          if ((it & 63) == 0 && (aborted(p) || (long long)(globaltimer_ns() - w0) > 2 * p.timeout_ns)) {
+            if (!aborted(p)) record_error(p, TRE_ERR_DEP_TIMEOUT, t.id);
+            r = false;
+            break;
+          }
+        }
+      }
       ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
       if (!ok) break;
     }
@@ -882,23 +906,30 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
       ls[idx] = __ldcg(src + D + 1);
     }
     consumer_sync(kConsumerThreads);
-    for (int idx = ctid; idx < ROWS * D; idx += kConsumerThreads) {
-      const int r = idx / D, dd = idx % D, v = r / G, h = r % G;
-      const float* mh = ms + r * S;
-      const float* lh = ls + r * S;
+    if (ctid < ROWS) {  // per row: the splits' weights 2^(m_s - M) and 1 / sum_s w_s l_s
+      float* mh = ms + ctid * S;
+      float* lh = ls + ctid * S;
       float M = -INFINITY;
       for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mh[s2]);
-      float Ls = 0.f, O = 0.f;
+      float Ls = 0.f;
+      for (int s2 = 0; s2 < S; ++s2) {
+        const float w = mh[s2] == -INFINITY ? 0.f : exp2f(mh[s2] - M);
+        mh[s2] = w;
+        Ls = fmaf(w, lh[s2], Ls);
+      }
+      lh[0] = 1.f / Ls;
+    }
+    consumer_sync(kConsumerThreads);
+    for (int idx = ctid; idx < ROWS * D; idx += kConsumerThreads) {
+      const int r = idx / D, dd = idx % D, v = r / G, h = r % G;
+      const float* wh = ms + r * S;
       const size_t q = (size_t)v * p.Hq + g * G + h;
       const float* src = p.part + q * S * pstride + dd;
       // independent loads: the splits' outputs are fetched together, not one at a time
-#pragma unroll 8
-      for (int s2 = 0; s2 < S; ++s2) {
-        const float w = mh[s2] == -INFINITY ? 0.f : exp2f(mh[s2] - M);
-        Ls = fmaf(w, lh[s2], Ls);
-        O = fmaf(w, __ldcg(src + s2 * pstride), O);
-      }
-      p.attn[q * D + dd] = O / Ls;
+      float O = 0.f;
+#pragma unroll 16
+      for (int s2 = 0; s2 < S; ++s2) O = fmaf(wh[s2], __ldcg(src + s2 * pstride), O);
+      p.attn[q * D + dd] = O * ls[r * S];
     }
     consumer_sync(kConsumerThreads);
     if (ctid == 0) publish_add(p.counters + t.out, 1u);
@@ -1656,7 +1687,10 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         publish_add(p.counters + t.out, 1u);
       }
     }
-    if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 2] = (long long)globaltimer_ns();
+    if (ctid == 0) {
+      if (p.trace) p.trace[(size_t)t.id * kTraceCols + 2] = (long long)globaltimer_ns();
+      *reinterpret_cast<volatile int*>(misc + 80) = ti + 1;  // tasks finished (producer reads)
+    }
     gs += (uint32_t)ns;
   }
 }
@@ -1684,6 +1718,7 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
   }
 
   if (threadIdx.x == 0) {
+    *reinterpret_cast<volatile int*>(misc + 80) = 0;
     for (uint32_t i = 0; i < NS; ++i) {
       mbar_init(&full[i], 1);                 // the producer's arrive + the copies' bytes
       mbar_init(&empty[i], kConsumerWarps);   // 8 arrivals: all warps, or one warp's 8
@@ -1693,7 +1728,8 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
-    producer(p, my, ntask, ring, full, empty, tags, threadIdx.x & 31);
+    producer(p, my, ntask, ring, full, empty, tags,
+             reinterpret_cast<const volatile int*>(misc + 80), threadIdx.x & 31);
     return;
   }
   consumer<MLA, MT>(p, my, ntask, ring, full, empty, tags, ub, misc);

@@ -258,6 +258,10 @@ static tre_status validate(const tre_config& c) {
   if (!(c.rope_theta > 0.f)) return fail(TRE_ERR_INVALID_ARG, "rope_theta must be > 0");
   if (!(c.norm_eps >= 0.f)) return fail(TRE_ERR_INVALID_ARG, "norm_eps must be >= 0");
   if (c.dep_timeout_us < 0) return fail(TRE_ERR_INVALID_ARG, "dep_timeout_us < 0");
+  if (c.stream_policy < 0 || c.stream_policy > 2)
+    return fail(TRE_ERR_INVALID_ARG, "stream_policy must be 0, 1 or 2");
+  if (c.gemv_kpart_max < 0 || (c.gemv_kpart_max > 0 && c.gemv_kpart_max < 512))
+    return fail(TRE_ERR_INVALID_ARG, "gemv_kpart_max must be 0 or >= 512");
   if (c.num_sms < 0 || c.kv_splits < 0 || c.stage_bytes < 0 || c.ring_stages < 0)
     return fail(TRE_ERR_INVALID_ARG, "negative launch-shape field");
   if (c.stage_bytes && (c.stage_bytes % 1024 || c.stage_bytes > kMaxStageBytes))
@@ -292,6 +296,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // per step the M input vectors share the planes
   s.M = c.max_tokens_per_step < 1 ? 1 : c.max_tokens_per_step;
   s.kpart_max = mla ? 8192 : (kMaxKPart / s.M) / 8 * 8;
+  if (c.gemv_kpart_max > 0) s.kpart_max = std::min(s.kpart_max, c.gemv_kpart_max / 8 * 8);
   s.F = c.ffn;
   s.V = c.has_embed_lm_head ? c.vocab : 0;
   s.L = c.n_layers;

@@ -401,6 +401,8 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.QL = s.QL; p.KL = s.KL; p.R = s.R; p.NP = s.NP; p.VD = s.VD;
   p.kpart_max = s.kpart_max;
   p.m = 1;
+  // default: hold (measured faster on the 8B-shaped stack: 0.683 vs 0.665 of peak)
+  p.hold_next_op = cfg->stream_policy != 1;
   p.err = reinterpret_cast<int32_t*>(B + o_err);
   p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
   p.status_host = e->status_dev;

@@ -187,6 +187,7 @@ struct Params {
   int32_t tokens[kMaxTokens];
   uint32_t epoch;
   int flags;
+  int hold_next_op;                // producer waits for this SM's publish at op boundaries
   long long timeout_ns;
   long long pf_window;             // L2 prefetch bytes allowed beyond the ring (0 = off)
 };

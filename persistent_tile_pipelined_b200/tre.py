@@ -49,7 +49,8 @@ class tre_config(ctypes.Structure):
         ("rope_theta", ctypes.c_float), ("norm_eps", ctypes.c_float)] + [
         (n, ctypes.c_int32) for n in (
             "has_embed_lm_head", "debug_flags", "dep_timeout_us", "num_sms", "kv_splits",
-            "stage_bytes", "ring_stages", "l2_prefetch_kb")] + [("reserved", ctypes.c_int32 * 7)]
+            "stage_bytes", "ring_stages", "l2_prefetch_kb", "gemv_kpart_max",
+            "stream_policy")] + [("reserved", ctypes.c_int32 * 5)]
 
 
 class tre_weights(ctypes.Structure):
