@@ -157,6 +157,23 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workload -------------
 
+def max_over_ranks(values, world: int, device: str = "cpu"):
+    """Element-wise maximum of per-rank timings over all ranks (the slowest rank sets the
+    job's time); identity on one rank.  Collective: every rank calls it once."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, steps: int, tokens_per_step: int, slowest_s: float) -> float:
+    """Whole-job tokens/s: every rank runs its own replica, so the job processes world x
+    steps x tokens_per_step tokens in the slowest rank's time."""
+    return world * steps * tokens_per_step / slowest_s
+
+
 def config_overrides(items):
     """FIELD=VALUE strings -> {field: int}."""
     out = {}
@@ -305,11 +322,8 @@ def run_layers(args, rank, world, local_rank):
         print(json.dumps(summ), file=sys.stderr)
     del dmodel
     torch.cuda.empty_cache()
-    t = torch.tensor([dev_s, e2e_s, float(np.mean(launch_ms))], dtype=torch.float64,
-                     device=f"cuda:{local_rank}")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    dev_s, e2e_s, launch_ms_avg = t.tolist()
+    dev_s, e2e_s, launch_ms_avg = max_over_ranks(
+        [dev_s, e2e_s, float(np.mean(launch_ms))], world, f"cuda:{local_rank}")
     return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
 
 
@@ -444,11 +458,8 @@ def run_engine(args, rank, world, local_rank):
     if trace_path:
         write_trace(wl, local_rank, trace_path, args.flags)
 
-    t = torch.tensor([dev_s, e2e_s, float(np.mean(launch_ms))], dtype=torch.float64,
-                     device=f"cuda:{local_rank}")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    dev_s, e2e_s, launch_ms_avg = t.tolist()
+    dev_s, e2e_s, launch_ms_avg = max_over_ranks(
+        [dev_s, e2e_s, float(np.mean(launch_ms))], world, f"cuda:{local_rank}")
     return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
 
 
@@ -499,7 +510,7 @@ def main():
     achieved = step_bytes / (launch_ms / 1e3) / 1e9
     line = {
         "metric": METRIC,
-        "value": world * K * M / dev_s,
+        "value": job_throughput(world, K, M, dev_s),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -530,7 +541,8 @@ def main():
             "kernel": "tre::engine_kernel",
             "algorithmic_bytes_per_launch": step_bytes,
         },
-        "e2e": {"value": world * K * M / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 4 * M,
+        "e2e": {"value": job_throughput(world, K, M, e2e_s), "unit": "tokens/s",
+                "h2d_bytes_per_step": 4 * M,
                 "d2h_bytes_per_step": 4 * M,
                 "note": "greedy loop via tre_decode_step_host: token in as a kernel argument, "
                         "argmax token back to pinned-less host memory, host wall time"},
@@ -570,7 +582,7 @@ def main_layers(args, rank, world, local_rank):
                    nope_dim=wl.nope_dim, v_dim=wl.v_dim, latent_positions=wl.prefill)
     line = {
         "metric": "layer-stack step time and achieved HBM GB/s over the bytes a token reads",
-        "value": world * K / dev_s, "unit": "steps/s", "n_gpus": world, "steps": K,
+        "value": job_throughput(world, K, 1, dev_s), "unit": "steps/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": dev_s / K * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
@@ -581,7 +593,7 @@ def main_layers(args, rank, world, local_rank):
                      "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
                      "kernel": "tre::engine_kernel",
                      "algorithmic_bytes_per_launch": step_bytes},
-        "e2e": {"value": world * K / e2e_s, "unit": "steps/s",
+        "e2e": {"value": job_throughput(world, K, 1, e2e_s), "unit": "steps/s",
                 "h2d_bytes_per_step": 4 * wl.hidden, "d2h_bytes_per_step": 4 * wl.hidden},
         "gpu_launches": K,
         "clocks": clocks,
