@@ -456,23 +456,28 @@ def run_engine(args, rank, world, local_rank):
     torch.cuda.empty_cache()
 
     if trace_path:
-        write_trace(wl, local_rank, trace_path, args.flags)
+        write_trace(wl, local_rank, trace_path, args.flags, config_overrides(args.config))
 
     dev_s, e2e_s, launch_ms_avg = max_over_ranks(
         [dev_s, e2e_s, float(np.mean(launch_ms))], world, f"cuda:{local_rank}")
     return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
 
 
-def write_trace(wl, device, path, flags=0):
+def write_trace(wl, device, path, flags=0, overrides=None):
     """Three traced steps on a fresh engine (debug flag): per-task start / ready / end of
-    the last one, with the plan and its summary."""
+    the last one, with the plan and its summary.  Steps take the workload's tokens per step."""
     import torch
 
     from persistent_tile_pipelined_b200 import trace as trace_mod
     from persistent_tile_pipelined_b200 import tre
-    eng, model = build_engine(wl.replace(decode_steps=3), device, tre.TRE_DEBUG_TRACE | flags)
+    M = max(1, wl.tokens_per_step)
+    eng, model = build_engine(wl.replace(decode_steps=3 * M), device, tre.TRE_DEBUG_TRACE | flags,
+                              overrides)
     for i in range(3):
-        eng.step(1 + i, wl.prefill + i)
+        if M > 1:
+            eng.step_tokens([1 + i * M + v for v in range(M)], wl.prefill + i * M)
+        else:
+            eng.step(1 + i, wl.prefill + i)
     torch.cuda.synchronize(device)
     tr = eng.trace()
     nsm = torch.cuda.get_device_properties(device).multi_processor_count

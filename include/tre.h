@@ -121,7 +121,12 @@ typedef struct {
                                    1 = as soon as ring slots free up; 2 = once this SM
                                    has published the current op (its publish then does
                                    not wait behind in-flight copies); 0 = default (2)   */
-  int32_t reserved[5];          /* must be zero                                         */
+  int32_t multi_token_gemv;     /* GEMV form of a plan with max_tokens_per_step > 1:
+                                   1 = CUDA-core rows; 2 = tensor-core tiles of 16 rows
+                                   (hidden and ffn multiples of 16); 0 = the planner's
+                                   choice: tiles from 3 tokens per step when the sizes
+                                   allow, else rows                                     */
+  int32_t reserved[4];          /* must be zero                                         */
 } tre_config;
 
 /* Per-layer tensor slots.  layer_w[l * TRE_W_SLOTS + slot] is the device pointer of

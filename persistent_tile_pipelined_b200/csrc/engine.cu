@@ -40,6 +40,13 @@ __device__ __noinline__ void record_error(const Params& p, int code, int detail)
 
 __device__ __forceinline__ bool aborted(const Params& p) { return *p.abort_flag != 0; }
 
+// Poll loops look at the abort flag and their time budget once per ~16 us of SM clock: the
+// flag is a global-memory read, and a waiter stalled on it notices its own event late.
+constexpr long long kCheckCycles = 1 << 15;
+
+// GEMV input staging: items each thread fetches before storing any.
+constexpr int kLoadBatch = 2;
+
 // Wait until counter `idx` reaches epoch * count (wrap-safe).  Bounded; on expiry the
 // error names `detail` (a task index).
 __device__ bool wait_counter(const Params& p, int idx, uint32_t count, int detail) {
@@ -47,14 +54,16 @@ __device__ bool wait_counter(const Params& p, int idx, uint32_t count, int detai
   const uint32_t* c = p.counters + idx;
   if ((int32_t)(ld_acquire_gpu(c) - target) >= 0) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  long long c0 = clock64();
+  for (;;) {
     if ((int32_t)(ld_acquire_gpu(c) - target) >= 0) return true;
-    if ((it & 31) == 0) {
+    if (clock64() - c0 > kCheckCycles) {
       if (aborted(p)) return false;
       if ((long long)(globaltimer_ns() - t0) > p.timeout_ns) {
         record_error(p, TRE_ERR_DEP_TIMEOUT, detail);
         return false;
       }
+      c0 = clock64();
     }
   }
 }
@@ -70,14 +79,16 @@ __device__ __forceinline__ bool wait_dep(const Params& p, const Task& t) {
 __device__ bool mbar_wait(const Params& p, uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  long long c0 = clock64();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15) == 0) {
+    if (clock64() - c0 > kCheckCycles) {
       if (aborted(p)) return false;
       if ((long long)(globaltimer_ns() - t0) > 2 * p.timeout_ns) {
         record_error(p, TRE_ERR_DEP_TIMEOUT, -1);
         return false;
       }
+      c0 = clock64();
     }
   }
 }
@@ -88,23 +99,42 @@ __device__ bool mbar_wait(const Params& p, uint64_t* bar, uint32_t parity) {
 // tags each slot with the stage it claimed (after that slot's previous stage was
 // consumed, which implies its full-barrier phase completed); waiting for the tag first
 // keeps every parity wait at most one phase ahead.
+__device__ bool stage_wait_at(const Params& p, uint64_t* full, const uint32_t* tags, uint32_t sidx,
+                              uint32_t slot, uint32_t parity);
+
 __device__ bool stage_wait(const Params& p, uint64_t* full, const uint32_t* tags, uint32_t sidx) {
-  const uint32_t NS = (uint32_t)p.ring_stages, slot = sidx % NS;
+  const uint32_t NS = (uint32_t)p.ring_stages;
+  return stage_wait_at(p, full, tags, sidx, sidx % NS, (sidx / NS) & 1u);
+}
+
+// The ring slot and phase parity of the next stage.
+__device__ __forceinline__ void ring_next(uint32_t& slot, uint32_t& par, uint32_t NS) {
+  if (++slot == NS) {
+    slot = 0;
+    par ^= 1u;
+  }
+}
+
+// The same with the slot and phase parity of stage sidx known to the caller.
+__device__ bool stage_wait_at(const Params& p, uint64_t* full, const uint32_t* tags, uint32_t sidx,
+                              uint32_t slot, uint32_t parity) {
   const volatile uint32_t* tag = tags + slot;
   if (*tag != sidx) {
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1; *tag != sidx; ++it) {
+    long long c0 = clock64();
+    while (*tag != sidx) {
       __nanosleep(64);  // yield issue slots to the warps that are computing
-      if ((it & 63) == 0) {
+      if (clock64() - c0 > kCheckCycles) {
         if (aborted(p)) return false;
         if ((long long)(globaltimer_ns() - t0) > 2 * p.timeout_ns) {
           record_error(p, TRE_ERR_DEP_TIMEOUT, -2);
           return false;
         }
+        c0 = clock64();
       }
     }
   }
-  return mbar_wait(p, &full[slot], (sidx / NS) & 1u);
+  return mbar_wait(p, &full[slot], parity);
 }
 
 // ---- task geometry (shared by producer and consumers) ---------------------------------------
@@ -145,8 +175,10 @@ struct GemvGeom {
   int k0, Kp;   // this part's input columns [k0, k0 + Kp)
   int rps;      // rows per ring stage
   int nstages;
+  int nkk;      // tiles (multi-token plans): stages per row tile and segment (k-chunks)
 };
 
+template <bool TILED>
 __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   GemvGeom g;
   g.K = gemv_K(p, t.op);
@@ -161,11 +193,18 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
     g.part = t.aux & 0xff;
     g.np = max(1, t.aux >> 8);
   }
-  const int len = g.np == 1 ? g.K : gemv_part_len(g.K, g.np);
+  const int len = g.np == 1 ? g.K : gemv_part_len(g.K, g.np, TILED ? 16 : 8);
   g.k0 = g.part * len;
   g.Kp = min(len, g.K - g.k0);
-  g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes);
-  g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
+  if (TILED) {  // row tiles of 16; per tile and segment, k-chunks of kTileK columns
+    g.rps = kTileRows;
+    g.nkk = (g.Kp + kTileK - 1) / kTileK;
+    g.nstages = (t.r1 - t.r0 + kTileRows - 1) / kTileRows * g.nseg * g.nkk;
+  } else {
+    g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes);
+    g.nkk = 1;
+    g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
+  }
   return g;
 }
 
@@ -226,8 +265,9 @@ __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& 
   t1 = (int)(P * (t.r1 + 1) / t.aux);
 }
 
+template <bool TILED>
 __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
-  if (t.type == T_GEMV) return gemv_geom(p, t).nstages;
+  if (t.type == T_GEMV) return gemv_geom<TILED>(p, t).nstages;
   int t0, t1;
   attn_range(p, t, t0, t1);
   return (t1 - t0 + p.pps - 1) / p.pps;
@@ -236,11 +276,14 @@ __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
 // Where a GEMV task's rows come from, resolved once per task (expert ids and layer
 // pointers are looked up here, not per stage): row n of segment s of the task's K-part
 // starts at base[s] + (n - r0) * stride.  QKV rows cross from Wq into Wk into Wv, so QKV
-// stages are resolved per stage instead (lookup = true).
+// whole-row stages are resolved per stage instead (lookup = true); for those ops base[]
+// holds the matrices themselves, row n from base[0] below split[0], base[1] below
+// split[1], else base[2] (used by the tile stages).
 struct RowSrc {
-  const uint16_t* base[2];
+  const uint16_t* base[3];
   long long stride;   // elements between consecutive rows in memory
-  bool lookup;        // resolve every stage with part_row
+  int split[2];
+  bool lookup;        // whole-row stages: resolve every stage with part_row
 };
 
 __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const GemvGeom& g) {
@@ -250,15 +293,76 @@ __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const 
   if (t.op == OP_RGU) r.stride = p.d;
   else if (t.op == OP_MDOWN) r.stride = g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe;
   int contig;
-  r.base[0] = r.lookup ? nullptr : part_row(p, t, g, 0, t.r0, &contig);
-  r.base[1] = (r.lookup || g.nseg < 2) ? nullptr : part_row(p, t, g, 1, t.r0, &contig);
+  r.base[2] = nullptr;
+  r.split[0] = r.split[1] = 0x7fffffff;
+  if (r.lookup) {
+    const LayerPtrs& L = p.layers[t.layer];
+    if (t.op == OP_QKV) {
+      r.base[0] = L.w[TRE_W_Q];
+      r.base[1] = L.w[TRE_W_K];
+      r.base[2] = L.w[TRE_W_V];
+      r.split[0] = p.Hq * p.D;
+      r.split[1] = (p.Hq + p.Hkv) * p.D;
+    } else {
+      r.base[0] = L.w[TRE_W_DQ];
+      r.base[1] = L.w[TRE_W_DKV];
+      r.split[0] = p.QL;
+    }
+    return r;
+  }
+  r.base[0] = part_row(p, t, g, 0, t.r0, &contig);
+  r.base[1] = g.nseg < 2 ? nullptr : part_row(p, t, g, 1, t.r0, &contig);
   return r;
+}
+
+// Row n of segment seg of a GEMV task's K-part, from its resolved row source.
+__device__ __forceinline__ const uint16_t* src_row(const RowSrc& rs, int seg, int n, int r0) {
+  if (!rs.lookup) return (seg ? rs.base[1] : rs.base[0]) + (long long)(n - r0) * rs.stride;
+  if (n < rs.split[0]) return rs.base[0] + (long long)n * rs.stride;
+  if (n < rs.split[1]) return rs.base[1] + (long long)(n - rs.split[0]) * rs.stride;
+  return rs.base[2] + (long long)(n - rs.split[1]) * rs.stride;
 }
 
 // ---- producer -------------------------------------------------------------------------------
 // Bytes of stage i of task t.  GEMV stages are whole rows of the task's K-part (gate/up:
 // the rows of both matrices); attention stages are the K and V rows of up to `pps`
 // consecutive cached positions of one kv head.
+// Tile stages of a multi-token GEMV task in order: row tile, then segment, then k-chunk.
+// A cursor walks them with additions only (the producer and consumers advance it per stage).
+struct TileStage {
+  int n0, nr;    // rows [n0, n0 + nr), nr <= 16
+  int seg;
+  int c0, kw;    // columns [c0, c0 + kw) of the task's K-part, kw <= kTileK
+  bool last;     // last stage of the row tile
+};
+
+__device__ __forceinline__ void tile_set(TileStage& ts, const Task& t, const GemvGeom& g) {
+  ts.nr = min(kTileRows, t.r1 - ts.n0);
+  ts.kw = min(kTileK, g.Kp - ts.c0);
+  ts.last = ts.seg == g.nseg - 1 && ts.c0 + ts.kw == g.Kp;
+}
+
+__device__ __forceinline__ TileStage tile_first(const Task& t, const GemvGeom& g) {
+  TileStage ts;
+  ts.n0 = t.r0;
+  ts.seg = 0;
+  ts.c0 = 0;
+  tile_set(ts, t, g);
+  return ts;
+}
+
+__device__ __forceinline__ void tile_next(TileStage& ts, const Task& t, const GemvGeom& g) {
+  ts.c0 += kTileK;
+  if (ts.c0 >= g.Kp) {
+    ts.c0 = 0;
+    if (++ts.seg == g.nseg) {
+      ts.seg = 0;
+      ts.n0 += kTileRows;
+    }
+  }
+  tile_set(ts, t, g);
+}
+
 __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, const GemvGeom& g,
                                                 int t0, int t1, int i) {
   if (t.type == T_GEMV) {
@@ -344,7 +448,7 @@ __device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, in
   long long bytes[3] = {0, 0, 0};
   if (t.type != T_GEMV) return;  // KV tiles come through the tensor maps
   {
-    const GemvGeom g = gemv_geom(p, t);
+    const GemvGeom g = gemv_geom<false>(p, t);
     if (g.np > 1 || needs_route(p, t)) return;  // strided rows, or addresses not known yet
     const size_t rowb = (size_t)g.K * 2;
     if (g.nseg == 2) {
@@ -389,6 +493,7 @@ __device__ __forceinline__ bool op_boundary(const Task& a, const Task& b) {
   return a.type != b.type || a.op != b.op || a.layer != b.layer;
 }
 
+template <bool TILED>
 __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, uint32_t* tags,
                          const volatile int* done, int lane) {
@@ -397,7 +502,7 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
   const uint32_t SB = (uint32_t)p.stage_bytes;
   const bool no_overlap = (p.flags & TRE_DEBUG_NO_OVERLAP) != 0;
   const long long window = no_overlap ? 0 : p.pf_window;
-  uint32_t gs = 0;
+  uint32_t gs = 0, slot = 0, ph = 0;  // stage count, its ring slot and phase parity (tiles)
   bool ok = true;
   for (int ti = 0; ti < ntask && ok; ++ti) {
     const Task t = my[ti];
@@ -413,12 +518,16 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       bool r = true;
       if (lane == 0) {
         const uint64_t w0 = globaltimer_ns();
-        for (uint32_t it = 1; *done < ti; ++it) {
+        long long c0 = clock64();
+        while (*done < ti) {
           __nanosleep(32);
-          if ((it & 63) == 0 && (aborted(p) || (long long)(globaltimer_ns() - w0) > 2 * p.timeout_ns)) {
-            if (!aborted(p)) record_error(p, TRE_ERR_DEP_TIMEOUT, t.id);
-            r = false;
-            break;
+          if (clock64() - c0 > kCheckCycles) {
+            if (aborted(p) || (long long)(globaltimer_ns() - w0) > 2 * p.timeout_ns) {
+              if (!aborted(p)) record_error(p, TRE_ERR_DEP_TIMEOUT, t.id);
+              r = false;
+              break;
+            }
+            c0 = clock64();
           }
         }
       }
@@ -432,18 +541,24 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       if (!ok) break;
     }
     if (window > 0 && ti + 1 < ntask) task_prefetch(p, my[ti + 1], lane, window);
-    const int ns = task_nstages(p, t);
+    const int ns = task_nstages<TILED>(p, t);
     GemvGeom g{};
     RowSrc rs{};
     int t0 = 0, t1 = 0;
     if (t.type == T_GEMV) {
-      g = gemv_geom(p, t);
+      g = gemv_geom<TILED>(p, t);
       rs = row_src(p, t, g);
     } else {
       attn_range(p, t, t0, t1);
     }
+    const bool tiled = TILED && t.type == T_GEMV;
+    TileStage ts{};
+    if (tiled) ts = tile_first(t, g);
     for (int i = 0; i < ns; ++i, ++gs) {
-      const uint32_t slot = gs % NS, ph = (gs / NS) & 1u;
+      if (!TILED) {  // whole-row kernels: from the stage count (measured faster there)
+        slot = gs % NS;
+        ph = (gs / NS) & 1u;
+      }
       bool r = true;
       if (lane == 0) r = mbar_wait(p, &empty[slot], ph ^ 1u);
       if (__shfl_sync(0xffffffffu, r ? 1 : 0, 0) == 0) {
@@ -452,10 +567,21 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       }
       if (lane == 0) {
         *reinterpret_cast<volatile uint32_t*>(tags + slot) = gs;
-        mbar_arrive_expect_tx(&full[slot], stage_total(p, t, g, t0, t1, i));
+        mbar_arrive_expect_tx(&full[slot], tiled ? (uint32_t)(ts.nr * ts.kw * 2)
+                                                 : stage_total(p, t, g, t0, t1, i));
       }
       __syncwarp();
-      issue_stage(p, t, g, rs, t0, t1, i, lane, ring + (size_t)slot * SB, &full[slot], pol);
+      if (tiled) {
+        // one copy per row of the tile: columns [c0, c0 + kw) into a padded row slot
+        if (lane < ts.nr)
+          bulk_g2s(ring + (size_t)slot * SB + (size_t)lane * kTilePitch,
+                   src_row(rs, ts.seg, ts.n0 + lane, t.r0) + ts.c0, (uint32_t)ts.kw * 2u,
+                   &full[slot], pol);
+        tile_next(ts, t, g);
+      } else {
+        issue_stage(p, t, g, rs, t0, t1, i, lane, ring + (size_t)slot * SB, &full[slot], pol);
+      }
+      if (TILED) ring_next(slot, ph, NS);
     }
   }
   if (!ok && lane == 0) {
@@ -516,7 +642,14 @@ __device__ __forceinline__ int input_key(const Task& t) {
 
 // Stage the GEMV input of each of the MT tokens into its two planes (token v's at
 // ub + v Kp); rn[v] receives token v's RMSNorm scale (1 when the op has no norm).
-template <int MT>
+// FRAG (tensor-core tiles): the inputs are written as the mma B operand instead, split
+// into bf16 hi and lo parts once here (one 8-column group of one token per thread, the
+// tokens interleaved across lanes so that the stores spread over the banks): for k-step s (columns 16 s .. 16 s + 15) and
+// fragment lane c = (part * MT + v) * 4 + tig (part 0 hi, 1 lo), the 32-bit pair at
+// 2 (8 MT s + c) holds columns 16 s + 2 tig, + 1 and the one after it columns
+// 16 s + 8 + 2 tig, + 1 of token v.  A warp reads a k-step's operand as 8 MT consecutive
+// 8-byte words, with no bank conflicts.  Same size as the planes: MT Kp floats.
+template <int MT, bool FRAG = false>
 __device__ void load_input(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
                            float* red, int ctid, float* rn) {
   const int K = gg.Kp;  // this K-part's slice of the input vector
@@ -546,8 +679,80 @@ __device__ void load_input(const Params& p, const Task& t, const GemvGeom& gg, f
   const int K8 = K >> 3;
   float ss[MT];
 #pragma unroll
-  for (int v = 0; v < MT; ++v) {
-    ss[v] = 0.f;
+  for (int v = 0; v < MT; ++v) ss[v] = 0.f;
+  // Fragments: work item w is one 8-column group j of token v, the tokens interleaved
+  // across lanes (so that the fragment stores spread over the banks).  Each thread fetches
+  // a batch of items before it stores any, so that the global reads overlap; indices are
+  // clamped, so the fetches need no guard.
+  const int nitems = MT * K8;
+  for (int w0 = ctid; FRAG && w0 < nitems; w0 += kLoadBatch * kConsumerThreads) {
+    float4 ra[kLoadBatch], rb[kLoadBatch];
+    uint4 gw[kLoadBatch];
+    if (src_bf) {
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) {
+        const int w = min(w0 + u * kConsumerThreads, nitems - 1);
+        const int v = w % MT, j = w / MT;
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(src_bf + (size_t)p.tokens[v] * p.d) + j);
+        ra[u] = make_float4(__uint_as_float(x.x), __uint_as_float(x.y), __uint_as_float(x.z),
+                            __uint_as_float(x.w));
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) {
+        const int w = min(w0 + u * kConsumerThreads, nitems - 1);
+        const int v = w % MT, j = w / MT;
+        const float4* sv = reinterpret_cast<const float4*>(src + v * vstride) + 2 * j;
+        ra[u] = __ldcg(sv);
+        rb[u] = __ldcg(sv + 1);
+      }
+    }
+    if (gain) {
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) {
+        const int w = min(w0 + u * kConsumerThreads, nitems - 1);
+        const int j = w / MT;
+        gw[u] = __ldg(reinterpret_cast<const uint4*>(gain) + j);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kLoadBatch; ++u) {
+      const int w = w0 + u * kConsumerThreads;
+      if (w >= nitems) break;
+      const int v = w % MT, j = w / MT;
+      float e[8];
+      if (src_bf) {
+        const uint32_t x0 = __float_as_uint(ra[u].x), x1 = __float_as_uint(ra[u].y);
+        const uint32_t x2 = __float_as_uint(ra[u].z), x3 = __float_as_uint(ra[u].w);
+        e[0] = bf_lo(x0); e[1] = bf_hi(x0); e[2] = bf_lo(x1); e[3] = bf_hi(x1);
+        e[4] = bf_lo(x2); e[5] = bf_hi(x2); e[6] = bf_lo(x3); e[7] = bf_hi(x3);
+      } else {
+        e[0] = ra[u].x; e[1] = ra[u].y; e[2] = ra[u].z; e[3] = ra[u].w;
+        e[4] = rb[u].x; e[5] = rb[u].y; e[6] = rb[u].z; e[7] = rb[u].w;
+      }
+      if (gain) {
+        float s2 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s2 = fmaf(e[k], e[k], s2);
+#pragma unroll
+        for (int vv = 0; vv < MT; ++vv)
+          if (vv == v) ss[vv] += s2;
+        const uint4 g = gw[u];
+        e[0] *= bf_lo(g.x); e[1] *= bf_hi(g.x); e[2] *= bf_lo(g.y); e[3] *= bf_hi(g.y);
+        e[4] *= bf_lo(g.z); e[5] *= bf_hi(g.z); e[6] *= bf_lo(g.w); e[7] *= bf_hi(g.w);
+      }
+      uint32_t* fr = reinterpret_cast<uint32_t*>(ub) + 2 * (8 * MT * (j >> 1)) + (j & 1);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hi, lo;
+        split_pair(e[2 * q], e[2 * q + 1], hi, lo);
+        fr[2 * (v * 4 + q)] = hi;
+        fr[2 * ((MT + v) * 4 + q)] = lo;
+      }
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < (FRAG ? 0 : MT); ++v) {
     float* xlo = ub + (size_t)v * K;
     float* xhi = xlo + K / 2;
     const float* sv = src ? src + v * vstride : nullptr;
@@ -1469,10 +1674,109 @@ __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
   if (ctid == 0) publish_add(p.counters + t.out, 1u);
 }
 
+
+// ---- multi-token GEMV on the tensor cores ---------------------------------------------------------
+// With m tokens per step a GEMV row is dotted with m input vectors, which makes the stage a
+// small dense contraction (16 rows x kw columns x m tokens): mma.sync m16n8k16 with A = the
+// tile's 16 weight rows (bf16, ldmatrix from the padded row slots) and B = the tokens' input
+// columns split into bf16 hi parts (column v) and lo parts (column 4 + v), so that
+// D[r][v] + D[r][4 + v] is row r . x_v with about 16 significand bits of x (the input
+// staging writes that operand in fragment order).  Every consumer
+// warp takes every stage and a 1/8 share of its 16-column k-steps; the warps' accumulators
+// are summed once per row tile through a double-buffered shared-memory area.
+template <int MT>
+__device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, const GemvGeom& g,
+                                               uint32_t gs, int ns, uint8_t* ring, uint64_t* full,
+                                               uint64_t* empty, const uint32_t* tags,
+                                               const float* xs, float* tred, const float* resid,
+                                               const float (&rnt)[MT], float wsel, int uoff,
+                                               Best (&best)[MT], int warp, int lane, int ctid,
+                                               bool& ab) {
+  const uint32_t NS = (uint32_t)p.ring_stages;
+  const int gq = lane >> 2, tig = lane & 3;
+  // B fragment of this lane (mma column gq: token gq & 3, hi part for gq < 4, else lo), as
+  // the input staging laid it out: 8 MT words of 8 bytes per k-step
+  const int bv = gq & 3;
+  const bool bact = bv < MT;
+  const uint2* xb = reinterpret_cast<const uint2*>(xs) + ((gq >> 2) * MT + (bact ? bv : 0)) * 4 + tig;
+  float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+  int buf = 0;
+  bool bad = false;
+  uint32_t slot = gs % NS, par = (gs / NS) & 1u;
+  TileStage ts = tile_first(t, g);
+  for (int i = 0; i < ns; ++i, tile_next(ts, t, g), ring_next(slot, par, NS)) {
+    const uint32_t sidx = gs + (uint32_t)i;
+    if (!bad) bad = !stage_wait_at(p, full, tags, sidx, slot, par);
+    if (!bad) {
+      const uint32_t sa = smem_u32(ring + (size_t)slot * p.stage_bytes) +
+                          (uint32_t)((lane & 15) * kTilePitch + (lane >> 4) * 16);
+      const int nks = ts.kw >> 4;
+      for (int k = warp; k < nks; k += kConsumerWarps) {
+        uint32_t a[4];
+        ldsm_x4(sa + (uint32_t)k * 32u, a[0], a[1], a[2], a[3]);
+        uint2 b = make_uint2(0u, 0u);
+        if (bact) b = xb[(size_t)((ts.c0 >> 4) + k) * (8 * MT)];
+        const uint32_t b0 = b.x, b1 = b.y;
+        if (ts.seg == 0) mma_bf16(acc0, a, b0, b1);
+        else mma_bf16(acc1, a, b0, b1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
+    }
+    if (!ts.last) continue;
+    // row tile done: hi + lo (columns v and 4 + v are lanes tig and tig ^ 2), then the
+    // lanes tig < 2 store tokens 2 tig, 2 tig + 1 of rows gq and gq + 8
+    float* tb = tred + buf * (2 * kConsumerWarps * kTileRows * kMaxTokens);
+#pragma unroll
+    for (int sg = 0; sg < 2; ++sg) {
+      if (sg == 1 && g.nseg < 2) break;
+      float* acc = sg == 0 ? acc0 : acc1;
+      float d[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        d[e] = acc[e] + __shfl_xor_sync(0xffffffffu, acc[e], 2);
+        acc[e] = 0.f;
+      }
+      if (tig < 2) {
+        float* w = tb + (sg * kConsumerWarps + warp) * (kTileRows * kMaxTokens);
+        *reinterpret_cast<float2*>(w + gq * kMaxTokens + 2 * tig) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(w + (gq + 8) * kMaxTokens + 2 * tig) = make_float2(d[2], d[3]);
+      }
+    }
+    if (consumer_sync_or(bad, kConsumerThreads)) {  // uniform: all warps leave together
+      ab = true;
+      return;
+    }
+    const int r = ctid & (kTileRows - 1), v = ctid >> 4;
+    if (v < MT && r < ts.nr) {
+      float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        y0 += tb[w * (kTileRows * kMaxTokens) + r * kMaxTokens + v];
+        if (g.nseg == 2) y1 += tb[(kConsumerWarps + w) * (kTileRows * kMaxTokens) + r * kMaxTokens + v];
+      }
+      const int n = ts.n0 + r;
+#pragma unroll
+      for (int vv = 0; vv < MT; ++vv) {
+        if (vv != v) continue;
+        if (g.nseg == 2) {
+          const float a = y0 * rnt[vv], bb = y1 * rnt[vv];
+          p.u[(size_t)vv * p.F + uoff + n] = wsel * (a / (1.f + expf(-a)) * bb);
+        } else {
+          gemv_emit(p, t, g, n, y0, rnt[vv], resid + vv * kMaxResidRows, best[vv], vv);
+        }
+      }
+    }
+    buf ^= 1;
+  }
+  if (bad) ab = true;
+}
+
 // ---- consumers -----------------------------------------------------------------------------------
 // MLA = true: the absorbed-MLA stack's kernel (MLA tiles, no GQA attention); false: GQA /
-// MoE.  Two instantiations keep each kernel's register allocation to its own tiles.
-template <bool MLA, int MT>
+// MoE.  Separate instantiations keep each kernel's register allocation to its own tiles.
+// TILED: GEMV stages are 16-row tensor-core tiles (multi-token plans).
+template <bool MLA, int MT, bool TILED>
 __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                          float* misc) {
@@ -1486,7 +1790,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
   bool ab = false;
   for (int ti = 0; ti < ntask; ++ti) {
     const Task t = my[ti];
-    const int ns = task_nstages(p, t);
+    const int ns = task_nstages<TILED>(p, t);
     if (ctid == 0) {
       long long* tr = p.trace ? p.trace + (size_t)t.id * kTraceCols : nullptr;
       if (tr) tr[0] = (long long)globaltimer_ns();
@@ -1512,9 +1816,9 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     } else if (MLA && t.op == OP_UK) {
       cur_key = -1;
       if constexpr (MLA)
-        uk_task(p, t, gemv_geom(p, t), gs, ns, ring, full, empty, tags, ub, red, warp, lane, ctid, ab);
+        uk_task(p, t, gemv_geom<false>(p, t), gs, ns, ring, full, empty, tags, ub, red, warp, lane, ctid, ab);
     } else {
-      const GemvGeom g = gemv_geom(p, t);
+      const GemvGeom g = gemv_geom<TILED>(p, t);
       const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
       const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MO;
@@ -1525,7 +1829,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         cur_key = -1;
       } else if (key != cur_key || key < 0) {
         float rnv[MT];
-        load_input<MT>(p, t, g, ub, red, ctid, rnv);
+        load_input<MT, TILED>(p, t, g, ub, red, ctid, rnv);
         if (ctid == 0)
 #pragma unroll
           for (int v = 0; v < MT; ++v) rn_s[v] = rnv[v];
@@ -1550,9 +1854,14 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         wsel = __ldcg(p.route_w + t.layer * p.topk + t.r0 / p.Fe);
         uoff = p.nshared * p.Fe;
       }
+      if constexpr (TILED) {
+        gemv_tile_task<MT>(p, t, g, gs, ns, ring, full, empty, tags, ub,
+                           ub + p.ub_floats - kTileRedFloats, resid, rnt, wsel, uoff, best, warp,
+                           lane, ctid, ab);
+      }
       // stage gs + i belongs to warp (gs + i) % 8; each warp takes its stages in order
       const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
-      for (int i = first; i < ns; i += kConsumerWarps) {
+      for (int i = first; i < (TILED ? 0 : ns); i += kConsumerWarps) {
         const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
         if (!stage_wait(p, full, tags, sidx)) {
           ab = true;
@@ -1593,6 +1902,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
             const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
             if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
           }
+        } else if (TILED) {
         } else if (g.nseg == 2) {  // MT tokens: gate / up rows as above, per token
           const uint4* up = sp + (size_t)g.rps * K8;
           const int vs = g.Kp / 4;  // float4 stride between the tokens' planes
@@ -1696,7 +2006,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
 }
 
 // ---- the kernel ----------------------------------------------------------------------------------
-template <bool MLA, int MT>
+template <bool MLA, int MT, bool TILED>
 __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t NS = (uint32_t)p.ring_stages;
@@ -1728,31 +2038,40 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
-    producer(p, my, ntask, ring, full, empty, tags,
+    producer<TILED>(p, my, ntask, ring, full, empty, tags,
              reinterpret_cast<const volatile int*>(misc + 80), threadIdx.x & 31);
     return;
   }
-  consumer<MLA, MT>(p, my, ntask, ring, full, empty, tags, ub, misc);
+  consumer<MLA, MT, TILED>(p, my, ntask, ring, full, empty, tags, ub, misc);
 }
 
 // ---- host-side launch helpers ------------------------------------------------------------------
-// The kernel instantiation for a stack kind and a number of tokens per step.
-static const void* kernel_for(bool mla, int m) {
-  if (mla) return reinterpret_cast<const void*>(engine_kernel<true, 1>);
+// The kernel instantiation for a stack kind, a number of tokens per step and the GEMV
+// stage form (tiled: multi-token tensor-core tiles).
+static const void* kernel_for(bool mla, int m, bool tiled) {
+  if (mla) return reinterpret_cast<const void*>(engine_kernel<true, 1, false>);
+  if (tiled) {
+    switch (m) {
+      case 2: return reinterpret_cast<const void*>(engine_kernel<false, 2, true>);
+      case 3: return reinterpret_cast<const void*>(engine_kernel<false, 3, true>);
+      case 4: return reinterpret_cast<const void*>(engine_kernel<false, 4, true>);
+      default: return reinterpret_cast<const void*>(engine_kernel<false, 1, true>);
+    }
+  }
   switch (m) {
-    case 2: return reinterpret_cast<const void*>(engine_kernel<false, 2>);
-    case 3: return reinterpret_cast<const void*>(engine_kernel<false, 3>);
-    case 4: return reinterpret_cast<const void*>(engine_kernel<false, 4>);
-    default: return reinterpret_cast<const void*>(engine_kernel<false, 1>);
+    case 2: return reinterpret_cast<const void*>(engine_kernel<false, 2, false>);
+    case 3: return reinterpret_cast<const void*>(engine_kernel<false, 3, false>);
+    case 4: return reinterpret_cast<const void*>(engine_kernel<false, 4, false>);
+    default: return reinterpret_cast<const void*>(engine_kernel<false, 1, false>);
   }
 }
 
 // Configure the instantiations a plan can launch (m = 1 .. max_m) and report how many
 // CTAs of the largest fit on an SM.
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m) {
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled) {
   *blocks_per_sm = 1 << 30;
   for (int m = 1; m <= (mla ? 1 : max_m); ++m) {
-    const void* k = kernel_for(mla, m);
+    const void* k = kernel_for(mla, m, tiled);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return e;
     int b = 0;
@@ -1775,7 +2094,7 @@ cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   void* args[] = {const_cast<Params*>(&p)};
-  return cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m), args);
+  return cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0), args);
 }
 
 }  // namespace tre

@@ -21,7 +21,7 @@
 #include "tre_internal.h"
 
 namespace tre {
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 }  // namespace tre
@@ -64,7 +64,7 @@ tre_status setup_device(int dev, void** scratch) {
     g_scratch_dev[dev] = ptr;
   }
   int bps = 0;
-  cudaError_t e = engine_configure(kSmemLimit, &bps, false, 1);
+  cudaError_t e = engine_configure(kSmemLimit, &bps, false, 1, false);
   if (e != cudaSuccess) return cuda_fail(e, "engine_configure");
   if (bps < 1) return fail(TRE_ERR_OCCUPANCY, "the persistent CTA does not fit on an SM");
   *scratch = g_scratch_dev[dev];

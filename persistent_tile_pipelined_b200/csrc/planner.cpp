@@ -252,12 +252,16 @@ static tre_status validate(const tre_config& c) {
   if (c.max_tokens_per_step > 1) {
     if (c.kind != TRE_LAYER_GQA)
       return fail(TRE_ERR_UNSUPPORTED, "multi-token steps are implemented for GQA stacks only");
+    if (c.multi_token_gemv == 2 && (c.hidden % 16 || c.ffn % 16))
+      return fail(TRE_ERR_UNSUPPORTED, "multi-token tensor-core tiles need hidden and ffn multiples of 16");
     if (c.max_tokens_per_step * (c.n_q_heads / c.n_kv_heads) > 16)
       return fail(TRE_ERR_UNSUPPORTED, "tokens x (q heads per kv head) above 16");
   }
   if (!(c.rope_theta > 0.f)) return fail(TRE_ERR_INVALID_ARG, "rope_theta must be > 0");
   if (!(c.norm_eps >= 0.f)) return fail(TRE_ERR_INVALID_ARG, "norm_eps must be >= 0");
   if (c.dep_timeout_us < 0) return fail(TRE_ERR_INVALID_ARG, "dep_timeout_us < 0");
+  if (c.multi_token_gemv < 0 || c.multi_token_gemv > 2)
+    return fail(TRE_ERR_INVALID_ARG, "multi_token_gemv must be 0, 1 or 2");
   if (c.stream_policy < 0 || c.stream_policy > 2)
     return fail(TRE_ERR_INVALID_ARG, "stream_policy must be 0, 1 or 2");
   if (c.gemv_kpart_max < 0 || (c.gemv_kpart_max > 0 && c.gemv_kpart_max < 512))
@@ -295,8 +299,14 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // so that the input planes leave room for a 5-deep ring of 36 KB stages; with M tokens
   // per step the M input vectors share the planes
   s.M = c.max_tokens_per_step < 1 ? 1 : c.max_tokens_per_step;
-  s.kpart_max = mla ? 8192 : (kMaxKPart / s.M) / 8 * 8;
-  if (c.gemv_kpart_max > 0) s.kpart_max = std::min(s.kpart_max, c.gemv_kpart_max / 8 * 8);
+  s.kpart_max = mla ? 8192 : (kMaxKPart / s.M) / 16 * 16;  // 16: tile k-steps
+  // multi-token GEMV form: tensor-core tiles cost the same per stage whatever the token
+  // count, CUDA-core rows grow with it (measured on the 8B-shaped stack: rows faster at 2
+  // tokens, tiles at 3 and 4)
+  const bool tiles_fit = c.hidden % 16 == 0 && c.ffn % 16 == 0;
+  s.tiles = s.M > 1 && (c.multi_token_gemv == 2 ||
+                        (c.multi_token_gemv == 0 && s.M >= kTileMinTokens && tiles_fit));
+  if (c.gemv_kpart_max > 0) s.kpart_max = std::min(s.kpart_max, c.gemv_kpart_max / 16 * 16);
   s.F = c.ffn;
   s.V = c.has_embed_lm_head ? c.vocab : 0;
   s.L = c.n_layers;
@@ -337,9 +347,9 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // a stage holds one attention tile: 64 K and V rows (GQA) or 32 latent rows (MLA)
   int xs = 8, need = mla ? (s.KL + s.R) * kMlaPosPerStage * 2 : 4 * s.D * kMaxPosPerStage;
   for (auto& o : ops) {
-    const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max));
+    const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max), s.tiles ? 16 : 8);
     xs = std::max(xs, kp);
-    need = std::max(need, o.nseg * kp * 2);
+    need = std::max(need, s.tiles ? kTileRows * kTilePitch : o.nseg * kp * 2);
   }
   // A ring stage holds whole rows of one K-part (gate/up: a row of each matrix), or the K
   // and V rows of 8-64 cached positions.
@@ -367,7 +377,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
                              2 * kMlaHeadGroup * Smax);
     s.attn_floats = std::max(s.attn_floats, kConsumerWarps * s.KL + s.NP + 64);
   }
-  const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats, s.attn_floats) + 7) / 8 * 8;
+  const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + (s.tiles ? kTileRedFloats : 0),
+                                     s.attn_floats) + 7) / 8 * 8;
   s.ub_floats = ubuf_floats;
   const int misc_bytes = 1024;
   const int fixed = ubuf_floats * 4 + misc_bytes;

@@ -17,7 +17,7 @@
 #include "tre_internal.h"
 
 namespace tre {
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 const char* last_error_cstr();
@@ -251,7 +251,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   }
 
   int bps = 0;
-  CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M));
+  CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M, s.tiles != 0));
   if (bps < 1) {
     set_error("tre_create: the persistent CTA does not fit on an SM");
     return TRE_ERR_OCCUPANCY;
@@ -403,6 +403,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.m = 1;
   // default: hold (measured faster on the 8B-shaped stack: 0.683 vs 0.665 of peak)
   p.hold_next_op = cfg->stream_policy != 1;
+  p.gemv_tiles = s.tiles;
   p.err = reinterpret_cast<int32_t*>(B + o_err);
   p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
   p.status_host = e->status_dev;

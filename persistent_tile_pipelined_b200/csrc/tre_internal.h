@@ -23,6 +23,13 @@ constexpr int kMaxTopK = 32;
 constexpr int kDefaultPrefetchKB = 0;    // next-task L2 prefetch: opt-in (measured 4% slower)
 constexpr int kMaxStageBytes = 65536;
 constexpr int kMaxTokens = 4;            // tokens per step (multi-token verify tiles)
+// Multi-token GEMV on tensor cores: a stage is one tile of 16 weight rows x up to 1024
+// input columns, each row copied into a 16-byte-padded slot (conflict-free ldmatrix).
+constexpr int kTileRows = 16;
+constexpr int kTileMinTokens = 3;                      // the planner's choice of tiles from here
+constexpr int kTileK = 1024;
+constexpr int kTilePitch = kTileK * 2 + 16;            // bytes per row slot
+constexpr int kTileRedFloats = 2 * 2 * kConsumerWarps * kTileRows * kMaxTokens;  // [2 bufs][2 segs]...
 constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per block
 
 #ifdef __CUDACC__
@@ -38,9 +45,9 @@ constexpr int kSmemLimit = 232448;                     // sm_100 opt-in max per 
 // [j * len, min(K, (j + 1) * len)); the parts of one row range are consecutive tasks on
 // one SM, the first adds the residual and later parts accumulate into the output.
 TRE_HD inline int gemv_nparts(int K, int kmax = kMaxKPart) { return (K + kmax - 1) / kmax; }
-TRE_HD inline int gemv_part_len(int K, int nparts) {
+TRE_HD inline int gemv_part_len(int K, int nparts, int align = 8) {
   const int l = (K + nparts - 1) / nparts;
-  return (l + 7) / 8 * 8;
+  return (l + align - 1) / align * align;
 }
 TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes) {
   const int r = stage_bytes / (nseg * K * 2);
@@ -118,6 +125,7 @@ struct PlanShape {
   int E, topk, nshared, Fe;  // MoE: experts, selected per token, shared, expert FFN
   int QL, KL, R, NP, VD;  // MLA: q_lora, kv_lora, rope, nope, v dims
   int kpart_max;       // longest input slice of a GEMV task (floats)
+  int tiles;           // multi-token plan: GEMV stages are 16-row tensor-core tiles
   int u_floats;        // the SwiGLU activation buffer (MoE: shared then routed slices)
   int down_blocks;     // MoE down: row blocks (each summed by its last slot to finish)
   int nsm;
@@ -188,6 +196,7 @@ struct Params {
   uint32_t epoch;
   int flags;
   int hold_next_op;                // producer waits for this SM's publish at op boundaries
+  int gemv_tiles;                  // GEMV stages are 16-row tiles (multi-token plans)
   long long timeout_ns;
   long long pf_window;             // L2 prefetch bytes allowed beyond the ring (0 = off)
 };

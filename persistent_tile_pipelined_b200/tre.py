@@ -50,7 +50,7 @@ class tre_config(ctypes.Structure):
         (n, ctypes.c_int32) for n in (
             "has_embed_lm_head", "debug_flags", "dep_timeout_us", "num_sms", "kv_splits",
             "stage_bytes", "ring_stages", "l2_prefetch_kb", "gemv_kpart_max",
-            "stream_policy")] + [("reserved", ctypes.c_int32 * 5)]
+            "stream_policy", "multi_token_gemv")] + [("reserved", ctypes.c_int32 * 4)]
 
 
 class tre_weights(ctypes.Structure):

@@ -301,9 +301,13 @@ def test_multi_token_plans(wl, m):
     tasks, _ = tre.tre_plan_tasks(cfg)
     T = decode_tasks(tasks)
     down = (T["type"] == T_GEMV) & (T["op"] == OP_DOWN)
-    kmax = (16384 // m) // 8 * 8
+    kmax = (16384 // m) // 16 * 16
     assert (T["aux"][down] >> 8).max() == -(-wl.ffn // kmax)
     assert info.smem_bytes <= 232448 and info.ring_stages >= 2
+    # from 3 tokens the planner picks tensor-core tiles: a stage holds 16 padded row slots
+    # of 1024 columns
+    if m >= 3:
+        assert info.stage_bytes >= 16 * (1024 * 2 + 16)
     resid_ops = (T["type"] == T_GEMV) & np.isin(T["op"], (OP_O, OP_DOWN))
     assert ((T["r1"] - T["r0"])[resid_ops] <= 512).all()
     # the same weights are streamed whatever the token count
@@ -314,13 +318,36 @@ def test_multi_token_plans(wl, m):
 @pytest.mark.parametrize("over,status", [
     (dict(max_tokens_per_step=4, n_q_heads=8, n_kv_heads=1), tre.TRE_ERR_UNSUPPORTED),  # 32 rows
     (dict(max_tokens_per_step=2), tre.TRE_ERR_UNSUPPORTED),                            # MoE
+    (dict(max_tokens_per_step=4, hidden=264, ffn=696, multi_token_gemv=2),
+     tre.TRE_ERR_UNSUPPORTED),                                                          # tiles: K % 16
+    (dict(max_tokens_per_step=2, multi_token_gemv=3), tre.TRE_ERR_INVALID_ARG),
 ])
 def test_multi_token_rejections(over, status):
     import ctypes
-    base = W.TINY if "n_q_heads" in over else MOE_SMALL
+    base = MOE_SMALL if over == dict(max_tokens_per_step=2) else W.TINY
     cfg = tre.config_from_workload(base, **over)
     info = tre.tre_plan_info()
     assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status
+
+
+def test_multi_token_cuda_core_form_takes_any_k():
+    """Whole-row stages (multi_token_gemv = 1, and the planner's choice when the sizes are
+    not multiples of 16) need K only a multiple of 8."""
+    wl = W.TINY.replace(hidden=264, ffn=696)
+    for form in (0, 1):
+        info = tre.tre_plan_inspect(tre.config_from_workload(wl, max_tokens_per_step=4,
+                                                             multi_token_gemv=form))
+        assert info.ring_stages >= 2 and info.stage_bytes < 16 * (1024 * 2 + 16)
+    tiled = tre.tre_plan_inspect(tre.config_from_workload(W.TINY, max_tokens_per_step=4))
+    rows = tre.tre_plan_inspect(tre.config_from_workload(W.TINY, max_tokens_per_step=4,
+                                                         multi_token_gemv=1))
+    assert tiled.weight_bytes == rows.weight_bytes
+    assert tiled.stage_bytes >= 16 * (1024 * 2 + 16) > rows.stage_bytes
+    # two tokens: rows by default, tiles on request
+    two = tre.tre_plan_inspect(tre.config_from_workload(W.TINY, max_tokens_per_step=2))
+    two_t = tre.tre_plan_inspect(tre.config_from_workload(W.TINY, max_tokens_per_step=2,
+                                                          multi_token_gemv=2))
+    assert two.stage_bytes < 16 * (1024 * 2 + 16) <= two_t.stage_bytes
 
 
 def test_reserved_fields_must_be_zero():

@@ -79,21 +79,26 @@ def run_and_compare(wl, steps=1, check_hidden=True, state=None, **cfg):
             assert gtok == rtok, f"greedy token differs at pos {pos}: {gtok} vs {rtok}"
         tok, pos = rtok, pos + 1
     # The KV rows this run appended agree with the oracle's: per appended row (one kv
-    # head, one position) the largest difference is within one bf16 ulp (2^-8 relative)
-    # of the row's largest entry — the two sides round fp32 vs fp64 values to bf16, so an
-    # entry near a rounding boundary may flip, and an entry near zero may differ by a few
-    # of its own (tiny) ulps.  Rows before `start` are untouched bit for bit.
+    # head, one position) the largest difference is within one bf16 ulp of the row's
+    # largest entry.  The two sides round fp32 vs fp64 values to bf16, so an entry near a
+    # rounding boundary may flip by one of its own ulps, which is up to 2^-7 of its
+    # magnitude (bf16 keeps 8 significant bits; at the bottom of a binade the spacing is
+    # 2^-7 relative); an entry near zero may differ by a few of its own (tiny) ulps.  The
+    # prefilled rows are untouched bit for bit (rows an earlier run on the same memory
+    # appended were checked by that run).
     for l in range(wl.n_layers):
         for name in ("k_cache", "v_cache"):
             gw = dev[name][l].view(torch.int16).cpu().numpy().view(np.uint16)
             ow = model[name][l]
             sl = slice(start, pos)
-            assert np.array_equal(gw[:, :start], ow[:, :start])
+            assert np.array_equal(gw[:, :wl.prefill], ow[:, :wl.prefill])
             gv = (gw[:, sl].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             ov = (ow[:, sl].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             row_max = np.abs(ov).max(axis=-1, keepdims=True)
-            bad = np.abs(gv - ov) > 2.0 ** -8 * row_max
-            assert not bad.any(), f"{name}[{l}]: {int(bad.sum())} appended entries off"
+            ratio = np.abs(gv - ov) / row_max
+            bad = ratio > 2.0 ** -7
+            assert not bad.any(), (f"{name}[{l}]: {int(bad.sum())} appended entries off, "
+                                   f"worst {float(ratio.max()):.3g} of the row max")
     eng.close()
     return worst, ties, (model, dev, tok, pos)
 

@@ -68,7 +68,7 @@ def run_mla(wl, steps=1, **cfg_over):
         assert np.array_equal(g[:start], o[:start])
         gv, ov = words_to_f64(g[start:end]), words_to_f64(o[start:end])
         row_max = np.abs(ov).max(axis=-1, keepdims=True)
-        assert not (np.abs(gv - ov) > 2.0 ** -8 * row_max).any()
+        assert not (np.abs(gv - ov) > 2.0 ** -7 * row_max).any()  # one bf16 ulp of the row max
     eng.close()
     return worst
 

@@ -87,7 +87,7 @@ def run_moe(wl, steps=1, **cfg_over):
             gv = (gw_[:, start:end].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             ov = (ow[:, start:end].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             row_max = np.abs(ov).max(axis=-1, keepdims=True)
-            assert not (np.abs(gv - ov) > 2.0 ** -8 * row_max).any()
+            assert not (np.abs(gv - ov) > 2.0 ** -7 * row_max).any()  # one bf16 ulp of the row max
     eng.close()
     return worst
 
