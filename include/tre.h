@@ -124,7 +124,7 @@ typedef struct {
   int32_t multi_token_gemv;     /* GEMV form of a plan with max_tokens_per_step > 1:
                                    1 = CUDA-core rows; 2 = tensor-core tiles of 16 rows
                                    (hidden and ffn multiples of 16); 0 = the planner's
-                                   choice: tiles from 3 tokens per step when the sizes
+                                   choice: tiles at 4 tokens per step when the sizes
                                    allow, else rows                                     */
   int32_t reserved[4];          /* must be zero                                         */
 } tre_config;

@@ -302,7 +302,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   s.kpart_max = mla ? 8192 : (kMaxKPart / s.M) / 16 * 16;  // 16: tile k-steps
   // multi-token GEMV form: tensor-core tiles cost the same per stage whatever the token
   // count, CUDA-core rows grow with it (measured on the 8B-shaped stack: rows faster at 2
-  // tokens, tiles at 3 and 4)
+  // and 3 tokens, tiles at 4)
   const bool tiles_fit = c.hidden % 16 == 0 && c.ffn % 16 == 0;
   s.tiles = s.M > 1 && (c.multi_token_gemv == 2 ||
                         (c.multi_token_gemv == 0 && s.M >= kTileMinTokens && tiles_fit));

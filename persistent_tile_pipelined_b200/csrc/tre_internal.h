@@ -26,7 +26,7 @@ constexpr int kMaxTokens = 4;            // tokens per step (multi-token verify 
 // Multi-token GEMV on tensor cores: a stage is one tile of 16 weight rows x up to 1024
 // input columns, each row copied into a 16-byte-padded slot (conflict-free ldmatrix).
 constexpr int kTileRows = 16;
-constexpr int kTileMinTokens = 3;                      // the planner's choice of tiles from here
+constexpr int kTileMinTokens = 4;                      // the planner's choice of tiles from here
 constexpr int kTileK = 1024;
 constexpr int kTilePitch = kTileK * 2 + 16;            // bytes per row slot
 constexpr int kTileRedFloats = 2 * 2 * kConsumerWarps * kTileRows * kMaxTokens;  // [2 bufs][2 segs]...

@@ -304,9 +304,9 @@ def test_multi_token_plans(wl, m):
     kmax = (16384 // m) // 16 * 16
     assert (T["aux"][down] >> 8).max() == -(-wl.ffn // kmax)
     assert info.smem_bytes <= 232448 and info.ring_stages >= 2
-    # from 3 tokens the planner picks tensor-core tiles: a stage holds 16 padded row slots
+    # at 4 tokens the planner picks tensor-core tiles: a stage holds 16 padded row slots
     # of 1024 columns
-    if m >= 3:
+    if m >= 4:
         assert info.stage_bytes >= 16 * (1024 * 2 + 16)
     resid_ops = (T["type"] == T_GEMV) & np.isin(T["op"], (OP_O, OP_DOWN))
     assert ((T["r1"] - T["r0"])[resid_ops] <= 512).all()
@@ -343,7 +343,9 @@ def test_multi_token_cuda_core_form_takes_any_k():
                                                          multi_token_gemv=1))
     assert tiled.weight_bytes == rows.weight_bytes
     assert tiled.stage_bytes >= 16 * (1024 * 2 + 16) > rows.stage_bytes
-    # two tokens: rows by default, tiles on request
+    # two and three tokens: rows by default, tiles on request
+    three = tre.tre_plan_inspect(tre.config_from_workload(W.TINY, max_tokens_per_step=3))
+    assert three.stage_bytes < 16 * (1024 * 2 + 16)
     two = tre.tre_plan_inspect(tre.config_from_workload(W.TINY, max_tokens_per_step=2))
     two_t = tre.tre_plan_inspect(tre.config_from_workload(W.TINY, max_tokens_per_step=2,
                                                           multi_token_gemv=2))

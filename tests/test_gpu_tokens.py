@@ -95,9 +95,9 @@ def test_multi_token_steps(over, ms, max_m):
 
 
 @pytest.mark.parametrize("over,cfg", [
-    (dict(hidden=272, ffn=720, vocab=1001, decode_steps=7), dict(gemv_kpart_max=512)),
-    (dict(hidden=264, ffn=696, vocab=1001, decode_steps=7), dict(multi_token_gemv=1)),
-    (dict(decode_steps=8), dict(multi_token_gemv=1, num_sms=7)),
+    (dict(hidden=272, ffn=720, vocab=1001, decode_steps=10), dict(gemv_kpart_max=512)),
+    (dict(hidden=264, ffn=696, vocab=1001, decode_steps=10), dict(multi_token_gemv=1)),
+    (dict(decode_steps=10), dict(multi_token_gemv=1, num_sms=7)),
     (dict(n_q_heads=8, n_kv_heads=1, decode_steps=8), dict(multi_token_gemv=2)),
 ], ids=["tiles-kparts", "cuda-cores-ragged-k", "cuda-cores-sms7", "tiles-g8"])
 def test_multi_token_gemv_forms(over, cfg):
