@@ -43,7 +43,9 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 METRIC = "batch-1 decode tokens/s and achieved HBM GB/s (fraction of ~8 TB/s roofline)"
+LAYERS_METRIC = "layer-stack step time and achieved HBM GB/s over the bytes a token reads"
 NOMINAL_HBM_GBS = 8000.0
+REFERENCE_SECONDS = 120.0  # oracle work of a whole reference-arm run
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -86,11 +88,16 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "engine_kernel_llama8b.md")
-    if not os.path.exists(path):
+PROFILES = {("llama3-8b-shaped", 1): "engine_kernel_llama8b.md",
+            ("llama3-8b-shaped", 4): "engine_kernel_llama8b_4tok.md"}
+
+
+def profiled_traffic(workload: str, tokens_per_step: int = 1):
+    """DRAM bytes per launch from the committed ncu summary of this workload's kernel (one
+    per token count), if it was taken on the current kernel source (else None)."""
+    name = PROFILES.get((workload, tokens_per_step))
+    path = os.path.join(ROOT, "profiles", name) if name else ""
+    if not name or not os.path.exists(path):
         return None
     txt = open(path).read()
     m_src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
@@ -327,53 +334,142 @@ def run_layers(args, rank, world, local_rank):
     return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
 
 
-def cpu_baseline(wl, sample_layers: int, reps: int = 1):
-    """The oracle (as it stands) on this machine's cores: one decode step of a
-    `sample_layers`-layer slice of the workload (same layer shapes, same LM head, same KV
-    length) and the same slice's layers alone; the full 32-layer step time is scaled from
-    the per-layer time plus the embedding / final-norm / LM-head time.  With reps > 1 the
-    sample is timed reps times on one generated model and the list is returned."""
-    import oracle
-    from persistent_tile_pipelined_b200.synth import workloads as W
-
-    sw = wl.replace(n_layers=sample_layers, decode_steps=1)
-    model = W.gen_gqa_model(sw)
-    orc = oracle.Oracle(32)
-    if reps > 1:
-        return [_time_sample(orc, wl, sw, model, sample_layers, 3.0) for _ in range(reps)]
-    return _time_sample(orc, wl, sw, model, sample_layers)
+def plan_step_gb(wl) -> float:
+    """GB a step streams at the workload's KV length, from the host planner: the weight
+    bytes of a step plus the KV rows read at `prefill` (both arms state it in `config`)."""
+    from persistent_tile_pipelined_b200 import tre
+    info = tre.tre_plan_inspect(tre.config_from_workload(wl))
+    M = max(1, wl.tokens_per_step)
+    kv = info.kv_bytes_at_capacity * wl.prefill / max(1, wl.kv_capacity - M)
+    return (info.weight_bytes + kv) / 1e9
 
 
-def _time_sample(orc, wl, sw, model, sample_layers, min_seconds: float = 10.0):
-    """Time the sliced step (and its layers alone) repeatedly until at least
-    `min_seconds` of CPU work has run; scale the median to the full stack."""
-    from persistent_tile_pipelined_b200.synth import workloads as W
+def decode_config(wl, M: int, overrides: dict, world: int) -> dict:
+    """`config` of a decode workload (the engine arm and the reference arm report the same)."""
+    return {
+        "workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions" +
+                    (f", {M} tokens per step (causal verify tiles)" if M > 1 else ""),
+        "tokens_per_step": M,
+        "engine_config": overrides,
+        "layers": wl.n_layers, "hidden": wl.hidden, "q_heads": wl.n_q_heads,
+        "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "ffn": wl.ffn,
+        "vocab": wl.vocab, "kv_positions": wl.prefill, "batch": 1,
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        "l2": f"not flushed: each step streams {plan_step_gb(wl):.2f} GB >> 126 MB L2",
+    }
 
-    tok = W.first_token(sw)
-    x = np.full(sw.hidden, 0.01, dtype=np.float32)
-    steps, layers = [], []
-    t_start = time.perf_counter()
-    while time.perf_counter() - t_start < min_seconds or len(steps) < 2:
+
+def layers_config(wl, world: int) -> dict:
+    """`config` of a layers-only workload (MoE, MLA); both arms report the same."""
+    cfg = {"workload": f"{wl.name} layers-only step, batch 1, KV {wl.prefill} positions",
+           "kind": wl.kind, "layers": wl.n_layers, "hidden": wl.hidden,
+           "heads": wl.n_q_heads, "batch": 1,
+           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+           "l2": f"not flushed: each step streams {plan_step_gb(wl):.2f} GB >> 126 MB L2"}
+    if wl.kind == "moe":
+        cfg.update(experts=wl.n_experts, top_k=wl.top_k, shared=wl.n_shared,
+                   expert_ffn=wl.expert_ffn, kv_heads=wl.n_kv_heads, head_dim=wl.head_dim)
+    if wl.kind == "mla":
+        cfg.update(q_lora=wl.q_lora, kv_lora=wl.kv_lora, rope_dim=wl.rope_dim,
+                   nope_dim=wl.nope_dim, v_dim=wl.v_dim, latent_positions=wl.prefill)
+    return cfg
+
+
+class DecodeSample:
+    """One bounded sample of the oracle (as it stands, fp32, on this machine's cores) on a
+    decode workload: a decode step of an `n`-layer slice (same layer shapes, same LM head,
+    same KV length) and the slice's layers alone, scaled to the full stack as
+    per-layer time x layers + the embedding / final-norm / LM-head time."""
+
+    def __init__(self, wl, layers: int):
+        self.wl = wl
+        self.set_layers(layers)
+
+    def set_layers(self, n: int):
+        import oracle
+        from persistent_tile_pipelined_b200.synth import workloads as W
+        self.n = n
+        self.sw = self.wl.replace(n_layers=n, decode_steps=1, tokens_per_step=1)
+        self.model = W.gen_gqa_model(self.sw)
+        self.orc = oracle.Oracle(32)
+        self.tok = W.first_token(self.sw)
+        self.x = np.full(self.sw.hidden, 0.01, dtype=np.float32)
+
+    def step(self) -> float:
+        """Seconds per token of the full stack, from one sample."""
         t0 = time.perf_counter()
-        orc.decode_step(sw, model, tok, sw.prefill, want_hidden=False)
-        steps.append(time.perf_counter() - t0)
+        self.orc.decode_step(self.sw, self.model, self.tok, self.sw.prefill, want_hidden=False)
+        t_step = time.perf_counter() - t0
         t0 = time.perf_counter()
-        orc.layers_step(sw, model, x, sw.prefill)
-        layers.append(time.perf_counter() - t0)
-    t_step, t_layers = float(np.median(steps)), float(np.median(layers))
-    per_layer = t_layers / sample_layers
-    t_full = per_layer * wl.n_layers + max(t_step - t_layers, 0.0)
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+        self.orc.layers_step(self.sw, self.model, self.x, self.sw.prefill)
+        t_layers = time.perf_counter() - t0
+        return t_layers / self.n * self.wl.n_layers + max(t_step - t_layers, 0.0)
+
+    def describe(self) -> str:
+        return (f"fp32 oracle, {self.n} of {self.wl.n_layers} layers + LM head, decode step "
+                f"at pos {self.sw.prefill} (and the layers alone), scaled to the full stack")
+
+
+class LayerSample:
+    """One bounded sample of the oracle on a layers-only workload (MoE, MLA): one layer
+    step of the stack's first layer at `prefill`, scaled by the number of layers."""
+
+    def __init__(self, wl):
+        import oracle
+        from persistent_tile_pipelined_b200.synth import TID_X_IN, normal_f32
+        from persistent_tile_pipelined_b200.synth import workloads as W
+        self.wl = wl
+        self.n = 1
+        self.sw = wl.replace(n_layers=1, decode_steps=1)
+        self.orc = oracle.Oracle(32)
+        self.x = normal_f32(wl.seed, TID_X_IN, (wl.hidden,))
+        if wl.kind == "moe":
+            self.model = W.gen_moe_model(self.sw)
+            self.experts = {}
+
+            def expert(e):
+                if e not in self.experts:
+                    self.experts[e] = W.gen_expert(self.sw, 0, e)
+                return self.experts[e]
+            self.expert = expert
+            self.step()  # the selected experts are generated once, outside the timed samples
+        else:
+            self.model = W.gen_mla_model(self.sw)
+
+    def step(self) -> float:
+        """Seconds per step of the full layer stack, from one sample."""
+        m, pos = self.model, self.sw.prefill
+        t0 = time.perf_counter()
+        if self.wl.kind == "moe":
+            self.orc.moe_layer_step(self.sw, m["layers"][0], m["k_cache"][0], m["v_cache"][0],
+                                    self.expert, pos, self.x)
+        else:
+            self.orc.mla_layer_step(self.sw, m["layers"][0], m["latent_cache"][0], pos, self.x)
+        return (time.perf_counter() - t0) * self.wl.n_layers
+
+    def describe(self) -> str:
+        return (f"fp32 oracle, 1 of {self.wl.n_layers} {self.wl.kind} layers at pos "
+                f"{self.sw.prefill}, scaled to the full stack")
+
+
+def cpu_cores() -> int:
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(wl, sample_layers: int, min_seconds: float = 10.0):
+    """The oracle timed on a bounded sample of the workload (about `min_seconds` of CPU
+    work): the median of repeated samples, scaled to the full stack."""
+    smp = DecodeSample(wl, sample_layers)
+    vals, t_start = [], time.perf_counter()
+    while time.perf_counter() - t_start < min_seconds or len(vals) < 2:
+        vals.append(smp.step())
+    t_full = float(np.median(vals))
     work = time.perf_counter() - t_start
-    return {"value": 1.0 / t_full, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"fp32 oracle, {sample_layers} of {wl.n_layers} layers + LM head, decode "
-                       f"step at pos {sw.prefill}, repeated {len(steps)}x ({work:.1f} s of CPU "
-                       f"work; median step {t_step:.3f} s, layers-only {t_layers:.3f} s), "
-                       f"scaled to the full stack: {t_full:.3f} s/token"),
+    return {"value": 1.0 / t_full, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{smp.describe()}; {len(vals)} samples ({work:.1f} s of CPU work), "
+                      f"median {t_full:.3f} s/token",
             "seconds_per_token": t_full}
 
-
-# ---------------------------------------------------------------- engine arm ----------
 
 def run_engine(args, rank, world, local_rank):
     import torch
@@ -526,23 +622,13 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
-        "config": {
-            "workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions" +
-                        (f", {M} tokens per step (causal verify tiles)" if M > 1 else ""),
-            "tokens_per_step": M,
-            "engine_config": config_overrides(args.config),
-            "layers": wl.n_layers, "hidden": wl.hidden, "q_heads": wl.n_q_heads,
-            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "ffn": wl.ffn,
-            "vocab": wl.vocab, "kv_positions": wl.prefill, "batch": 1,
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": f"not flushed: each step streams {step_bytes / 1e9:.2f} GB >> 126 MB L2",
-        },
+        "config": decode_config(wl, M, config_overrides(args.config), world),
         "hbm_gbs": step_bytes / (dev_s / K) / 1e9,
         "hbm_frac_of_8tbs": step_bytes / (dev_s / K) / 1e9 / NOMINAL_HBM_GBS,
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_kind": peak_kind,
-            "traffic": profiled_traffic(args.workload),
+            "traffic": profiled_traffic(args.workload, M),
             "kernel": "tre::engine_kernel",
             "algorithmic_bytes_per_launch": step_bytes,
         },
@@ -574,19 +660,9 @@ def main_layers(args, rank, world, local_rank):
     K = args.steps
     peak, peak_kind = peaks()
     achieved = step_bytes / (launch_ms / 1e3) / 1e9
-    cfg = {"workload": f"{wl.name} layers-only step, batch 1, KV {wl.prefill} positions",
-           "kind": wl.kind, "layers": wl.n_layers, "hidden": wl.hidden,
-           "heads": wl.n_q_heads, "batch": 1,
-           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-           "l2": f"not flushed: each step streams {step_bytes / 1e9:.2f} GB >> 126 MB L2"}
-    if wl.kind == "moe":
-        cfg.update(experts=wl.n_experts, top_k=wl.top_k, shared=wl.n_shared,
-                   expert_ffn=wl.expert_ffn, kv_heads=wl.n_kv_heads, head_dim=wl.head_dim)
-    if wl.kind == "mla":
-        cfg.update(q_lora=wl.q_lora, kv_lora=wl.kv_lora, rope_dim=wl.rope_dim,
-                   nope_dim=wl.nope_dim, v_dim=wl.v_dim, latent_positions=wl.prefill)
+    cfg = layers_config(wl, world)
     line = {
-        "metric": "layer-stack step time and achieved HBM GB/s over the bytes a token reads",
+        "metric": LAYERS_METRIC,
         "value": job_throughput(world, K, 1, dev_s), "unit": "steps/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": dev_s / K * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -611,25 +687,52 @@ def main_layers(args, rank, world, local_rank):
 
 
 def main_reference(args, rank, world):
-    """The reference arm: the CPU oracle as it stands, on this machine's host cores, on a
-    bounded sample per step of the same workload.  Rank 0 only."""
+    """The reference arm: the CPU oracle as it stands, on this machine's host cores, for the
+    engine arm's workload, metric, unit and config.  W untimed and K timed steps, each step
+    one bounded sample of the workload (a layer slice, scaled to the full stack), the slice
+    sized so the whole run takes about two minutes.  Rank 0 only."""
     if rank != 0:
         return
     from persistent_tile_pipelined_b200.synth import workloads as W
-    wl = W.WORKLOADS[args.workload]
-    K = max(2, min(args.steps, 3))
-    vals = cpu_baseline(wl, args.cpu_sample_layers, reps=K)
-    v = float(np.median([x["value"] for x in vals]))
+    K, Wm, M = args.steps, args.warmup, args.tokens_per_step
+    wl = W.WORKLOADS[args.workload].replace(decode_steps=K + Wm)
+    budget = REFERENCE_SECONDS / max(1, K + Wm)  # seconds of oracle work per step
+    if wl.kind == "gqa":
+        wl = wl.replace(tokens_per_step=M)
+        smp = DecodeSample(wl, args.cpu_sample_layers)
+        while smp.n > 1:  # one sample must fit the per-step budget (untimed calibration)
+            t0 = time.perf_counter()
+            smp.step()
+            if time.perf_counter() - t0 <= budget:
+                break
+            smp.set_layers(max(1, smp.n // 2))
+        metric, unit, per = METRIC, "tokens/s", M  # tokens per step
+        config = decode_config(wl, M, config_overrides(args.config), world)
+    else:
+        M = 1
+        smp = LayerSample(wl)
+        metric, unit, per = LAYERS_METRIC, "steps/s", 1
+        config = layers_config(wl, world)
+    for _ in range(Wm):
+        smp.step()
+    t_start = time.perf_counter()
+    vals = [smp.step() for _ in range(K)]
+    work = time.perf_counter() - t_start
+    t = float(np.median(vals))  # seconds per token (decode) or per stack step (layers)
+    v = 1.0 / t
+    sample = (f"{smp.describe()}; one sample per step, {K} timed after {Wm} warm-up "
+              f"({work:.1f} s of CPU work), median {t:.4f} s per "
+              f"{'token' if wl.kind == 'gqa' else 'stack step'}")
     line = {
-        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": 0, "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions",
-                   "batch": 1, "parallelism": "host cores"},
+        "metric": metric, "value": v, "unit": unit, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": t * per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
+        "config": config,
         "impl": "reference",
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
-                         "kind": "oracle", "sample": vals[0]["sample"]},
-        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
