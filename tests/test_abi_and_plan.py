@@ -63,6 +63,10 @@ PLAN_CASES = [
     (W.MOE4, 148), (MOE_SMALL, 148), (MOE_SMALL, 5),
     (MOE_SMALL.replace(n_shared=0, top_k=1), 19), (MOE_SMALL.replace(n_shared=2), 64),
     (W.MLA4, 148), (MLA_SMALL, 148), (MLA_SMALL, 6),
+    # multi-token plans: tensor-core tiles at 4 tokens, CUDA-core rows at 2 and 3
+    (W.LLAMA8B.replace(tokens_per_step=4), 148), (W.LLAMA8B.replace(tokens_per_step=2), 148),
+    (W.TINY.replace(tokens_per_step=4, hidden=272, ffn=720, vocab=1001), 7),
+    (W.TINY.replace(tokens_per_step=3, hidden=264, ffn=696, vocab=1001), 11),
 ]
 
 
