@@ -5,6 +5,8 @@ import re
 from collections import Counter, defaultdict
 
 import numpy as np
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
 import pytest
 
 from persistent_tile_pipelined_b200 import build
@@ -95,7 +97,14 @@ def rows_of_ops(wl):
 
 @pytest.mark.parametrize("wl,nsm", PLAN_CASES, ids=lambda x: getattr(x, "name", str(x)))
 def test_plan_is_a_valid_task_graph(wl, nsm):
-    cfg = tre.config_from_workload(wl)
+    check_plan(wl, nsm)
+
+
+def check_plan(wl, nsm, **over):
+    """The plan of `wl` on `nsm` SMs is a valid task graph: ids topological per SM queue,
+    every dependency produced earlier with the right count, every op's rows covered
+    exactly once per K-part, attention (head, split) pairs exactly once, balanced."""
+    cfg = tre.config_from_workload(wl, **over)
     tasks, begin = tre.tre_plan_tasks(cfg, num_sms=nsm)
     info = tre.tre_plan_inspect(cfg, num_sms=nsm)
     assert info.num_tasks == len(tasks) and begin[-1] == len(tasks)
@@ -212,6 +221,75 @@ def test_plan_is_a_valid_task_graph(wl, nsm):
     lm = (T["type"] == T_GEMV) & (T["op"] == OP_LM)
     assert (T["aux"][lm] == lm.sum()).all()
     assert info.smem_bytes <= 232448
+    return info
+
+
+@st.composite
+def gqa_plans(draw):
+    """Random valid GQA stacks and launch shapes (sizes, head groups, SM count, KV
+    splits, tokens per step, GEMV form, K-part limit)."""
+    D = draw(st.sampled_from([64, 128]))
+    kv = draw(st.sampled_from([1, 2, 4, 8]))
+    G = draw(st.sampled_from([1, 2, 4, 8]))
+    M = draw(st.integers(1, max(1, min(4, 16 // G))))
+    form = draw(st.sampled_from([0, 1, 2])) if M > 1 else 0
+    q = 16 if form == 2 else 8
+    hidden = q * draw(st.integers(4, 256 // (q // 8)))
+    ffn = q * draw(st.integers(4, 512 // (q // 8)))
+    wl = W.TINY.replace(n_layers=draw(st.integers(1, 3)), hidden=hidden, ffn=ffn,
+                        n_kv_heads=kv, n_q_heads=kv * G, head_dim=D,
+                        vocab=draw(st.integers(1, 3000)), prefill=draw(st.integers(0, 300)),
+                        decode_steps=draw(st.integers(1, 16)), tokens_per_step=M)
+    over = {"multi_token_gemv": form}
+    kmax = draw(st.sampled_from([0, 512, 1024, 4096]))
+    if kmax >= hidden:
+        over["gemv_kpart_max"] = kmax
+    if draw(st.booleans()):
+        over["kv_splits"] = draw(st.integers(1, 4 * D))
+    return wl, draw(st.integers(1, 148)), over
+
+
+@st.composite
+def moe_plans(draw):
+    """Random valid MoE stacks: expert count, top-k, shared experts, expert width."""
+    E = draw(st.integers(1, 64))
+    kv = draw(st.sampled_from([1, 2, 4]))
+    wl = MOE_SMALL.replace(n_layers=draw(st.integers(1, 2)), hidden=8 * draw(st.integers(8, 96)),
+                           n_kv_heads=kv, n_q_heads=kv * draw(st.sampled_from([1, 2, 4, 8])),
+                           head_dim=draw(st.sampled_from([64, 128])), n_experts=E,
+                           top_k=draw(st.integers(1, min(E, 8))), n_shared=draw(st.integers(0, 2)),
+                           expert_ffn=8 * draw(st.integers(1, 64)),
+                           prefill=draw(st.integers(0, 200)))
+    return wl, draw(st.integers(1, 148)), {}
+
+
+@st.composite
+def mla_plans(draw):
+    """Random valid absorbed-MLA stacks: heads, latent and rope widths, q_lora, nope / v."""
+    kl = 128 * draw(st.integers(1, 5))
+    rope = draw(st.sampled_from([r for r in (16, 32, 48, 64, 80, 96, 112, 128)
+                                 if (kl + r) % 64 == 0 and kl + r <= 768] or [64]))
+    wl = MLA_SMALL.replace(n_layers=draw(st.integers(1, 2)), hidden=8 * draw(st.integers(8, 96)),
+                           n_q_heads=16 * draw(st.integers(1, 4)), kv_lora=kl, rope_dim=rope,
+                           q_lora=8 * draw(st.integers(1, 64)), nope_dim=8 * draw(st.integers(1, 16)),
+                           v_dim=8 * draw(st.integers(1, 16)), prefill=draw(st.integers(0, 300)))
+    return wl, draw(st.integers(1, 148)), {}
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(st.one_of(moe_plans(), mla_plans()))
+def test_random_moe_and_mla_plans_are_valid_task_graphs(case):
+    wl, nsm, over = case
+    check_plan(wl, nsm, **over)
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(gqa_plans())
+def test_random_gqa_plans_are_valid_task_graphs(case):
+    wl, nsm, over = case
+    info = check_plan(wl, nsm, **over)
+    if "kv_splits" in over:
+        assert info.kv_splits == over["kv_splits"]
 
 
 def test_llama8b_plan_is_byte_balanced():
