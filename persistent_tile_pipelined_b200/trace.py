@@ -50,11 +50,14 @@ def summarize(trace: np.ndarray, tasks: np.ndarray) -> dict:
         d["wait_ns"] += float(ready[i] - start[i])
         d["busy_ns"] += float(end[i] - ready[i])
         spans[(int(tt["layer"][i]), name)].append((start[i], ready[i], end[i]))
-    # straggler spread: for each (layer, op), last finish minus median finish
+    # straggler spread: for each (layer, op), last finish minus median finish; op span:
+    # first dependency met to last finish (the op's share of the step's critical path)
     spread = defaultdict(list)
+    span = defaultdict(list)
     for (layer, name), v in spans.items():
         ends = np.array([e for _, _, e in v], dtype=np.float64)
         spread[name].append(float(ends.max() - np.median(ends)))
+        span[name].append(float(ends.max() - min(r for _, r, _ in v)))
     nsm = int(trace[:, 3].max()) + 1
     busy = np.zeros(nsm)
     waitt = np.zeros(nsm)
@@ -80,6 +83,7 @@ def summarize(trace: np.ndarray, tasks: np.ndarray) -> dict:
                    for k, v in per_op.items()},
         "finish_spread_us": {k: {"mean": float(np.mean(v)) / 1e3, "max": float(np.max(v)) / 1e3}
                              for k, v in spread.items()},
+        "op_span_us": {k: float(np.mean(v)) / 1e3 for k, v in span.items()},
         "sm_wait_frac_mean": float(np.mean(waitt) / step_ns),
         "sm_busy_frac_mean": float(np.mean(busy) / step_ns),
     }
@@ -90,7 +94,7 @@ def chrome_trace(trace: np.ndarray, tasks: np.ndarray, path: str) -> None:
     t0 = trace[:, 0].min()
     ev = []
     for i in range(len(trace)):
-        s, r, e, sm = (int(x) for x in trace[i])
+        s, r, e, sm = (int(x) for x in trace[i, :4])
         name = f"L{int(tt['layer'][i])}.{op_name(tt, i)}"
         if r > s:
             ev.append({"name": "wait", "ph": "X", "ts": (s - t0) / 1e3, "dur": (r - s) / 1e3,
