@@ -136,30 +136,38 @@ class ClockSampler:
             return None
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        sm, mx, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in out.splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-            except ValueError:
-                continue
-            if self.windows and not any(a - 0.05 <= ts <= b + 0.05 for a, b in self.windows):
-                continue
-            try:
-                sm.append(float(parts[2]))
-                mx = float(parts[3])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return parse_clocks(out, self.windows)
+
+
+def parse_clocks(text: str, windows) -> dict:
+    """The `clocks` entry from nvidia-smi CSV samples (the ClockSampler fields, no header,
+    no units): the median SM clock and the throttle reasons seen during the timed windows
+    (wall-clock (start, end) pairs; every sample when there are none)."""
+    sm, mx, reasons = [], None, set()
+    names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    for line in text.splitlines():
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            continue
+        if windows and not any(a - 0.05 <= ts <= b + 0.05 for a, b in windows):
+            continue
+        try:
+            clk, top = float(parts[2]), float(parts[3])
+        except ValueError:
+            continue
+        sm.append(clk)
+        mx = top
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+    return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+            "samples": len(sm)}
 
 
 # ---------------------------------------------------------------- workload -------------

@@ -65,3 +65,30 @@ def test_plan_step_bytes_in_config():
     kv = 2 * wl.n_layers * wl.n_kv_heads * wl.head_dim * 2 * wl.prefill
     assert bench.plan_step_gb(wl) == pytest.approx((info.weight_bytes + kv) / 1e9, rel=1e-3)
     assert bench.plan_step_gb(wl) == pytest.approx(15.55, abs=0.01)
+
+
+def test_clock_samples_inside_the_timed_windows():
+    """The `clocks` entry: median SM clock and throttle reasons of the samples taken inside
+    the timed windows; malformed and out-of-window samples are ignored."""
+    import datetime
+    sys.path.insert(0, ROOT)
+    import bench
+
+    def row(sec, clk, reasons=("Not Active",) * 4):
+        ts = datetime.datetime(2026, 1, 1, 12, 0, 0) + datetime.timedelta(seconds=sec)
+        return ", ".join([ts.strftime("%Y/%m/%d %H:%M:%S.%f")[:-3], "0", str(clk), "1965",
+                          "700.5", *reasons])
+    t0 = datetime.datetime(2026, 1, 1, 12, 0, 0).timestamp()
+    text = "\n".join([
+        row(0.0, 1200),                                      # before the window: ignored
+        row(1.0, 1965), row(1.2, 1950),
+        row(1.4, 1965, ("Not Active", "Not Active", "Not Active", "Active")),
+        "garbage line", row(1.5, "[N/A]"),                   # malformed: ignored
+        row(3.0, 900, ("Active", "Not Active", "Not Active", "Not Active")),  # after: ignored
+    ])
+    c = bench.parse_clocks(text, [(t0 + 0.9, t0 + 1.6)])
+    assert c == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    every = bench.parse_clocks(text, [])
+    assert every["samples"] == 5 and every["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert bench.parse_clocks("", [(t0, t0 + 1)])["samples"] == 0
