@@ -60,7 +60,7 @@ typedef enum {
   TRE_ERR_OCCUPANCY = -3,     /* one CTA per SM cannot be co-resident                */
   TRE_ERR_DEP_TIMEOUT = -4,   /* a device wait ran out of time (device status word)  */
   TRE_ERR_POS_RANGE = -5,     /* pos (+ tokens) beyond the KV capacity               */
-  TRE_ERR_UNSUPPORTED = -6,   /* config outside what this build implements           */
+  TRE_ERR_UNSUPPORTED = -6,   /* config outside what the engine implements          */
   TRE_ERR_BOUNDS = -7,        /* device bounds check fired (device status word)      */
   TRE_ERR_STATE = -8          /* previous device error not yet cleared by tre_reset  */
 } tre_status;
