@@ -461,7 +461,15 @@ class LayerSample:
 
 
 def cpu_cores() -> int:
-    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    """Threads the OpenMP oracle runs on: OMP_NUM_THREADS, else the CPUs this process may
+    run on (the OpenMP runtime's default)."""
+    env = os.environ.get("OMP_NUM_THREADS", "").split(",")[0].strip()
+    if env.isdigit() and int(env) > 0:
+        return int(env)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def cpu_baseline(wl, sample_layers: int, min_seconds: float = 10.0):
