@@ -342,14 +342,33 @@ def run_layers(args, rank, world, local_rank):
     return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
 
 
+def workload_step_bytes(wl, pos=None) -> int:
+    """Bytes a one-token step streams at `pos` (default: the workload's KV length), from
+    the workload's shape alone: every weight and norm gain the token reads (MoE: the
+    router, the shared and the selected experts only), the K / V (latent) rows read and
+    the new rows written, the embedding row and the logits.  Both arms state it in
+    `config` without loading the engine library."""
+    pos = wl.prefill if pos is None else pos
+    d, L = wl.hidden, wl.n_layers
+    if wl.kind == "mla":
+        H, C = wl.n_q_heads, wl.kv_lora + wl.rope_dim
+        w = ((wl.q_lora + C) * d + H * (wl.nope_dim + wl.rope_dim) * wl.q_lora +
+             H * wl.nope_dim * wl.kv_lora + H * wl.v_dim * wl.kv_lora + d * H * wl.v_dim)
+        total = (w * 2 + (d + wl.q_lora + wl.kv_lora) * 2) * L + L * (pos + 1) * C * 2
+    else:
+        Hq, Hkv, D = wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+        mlp = (wl.n_experts * d + 3 * (wl.n_shared + wl.top_k) * wl.expert_ffn * d
+               if wl.kind == "moe" else 3 * wl.ffn * d)
+        per_layer = ((Hq + 2 * Hkv) * D * d + d * Hq * D + mlp) * 2 + 2 * d * 2
+        total = per_layer * L + L * Hkv * (pos + 1) * D * 2 * 2
+    if wl.vocab > 0:
+        total += wl.vocab * d * 2 + d * 2 + d * 2 + wl.vocab * 4
+    return total
+
+
 def plan_step_gb(wl) -> float:
-    """GB a step streams at the workload's KV length, from the host planner: the weight
-    bytes of a step plus the KV rows read at `prefill` (both arms state it in `config`)."""
-    from persistent_tile_pipelined_b200 import tre
-    info = tre.tre_plan_inspect(tre.config_from_workload(wl))
-    M = max(1, wl.tokens_per_step)
-    kv = info.kv_bytes_at_capacity * wl.prefill / max(1, wl.kv_capacity - M)
-    return (info.weight_bytes + kv) / 1e9
+    """GB a step streams at the workload's KV length (weights + KV), for `config`."""
+    return workload_step_bytes(wl) / 1e9
 
 
 def decode_config(wl, M: int, overrides: dict, world: int) -> dict:

@@ -244,14 +244,17 @@ tre_status tre_decode_step_host(tre_engine* e, int32_t token, int32_t pos, tre_s
  *   cfg, w       as for tre_create (weights and caches caller owned); no debug flags
  *   token, pos   as for tre_decode_step; the step runs on the CURRENT device
  *   logits_dev   device fp32[vocab], required;  token_dev  device int32[1] or NULL
- *   status_dev   device int32[2] or NULL: set to {0, 0}, then on a device error to
- *                {TRE_ERR_DEP_TIMEOUT or TRE_ERR_BOUNDS, task index}
+ *   status_dev   device int32[2] or NULL (4-byte aligned): set to {0, 0}, then on a
+ *                device error to {TRE_ERR_DEP_TIMEOUT or TRE_ERR_BOUNDS, task index}.
+ *                With NULL a device error is NOT reported to the caller: the kernel
+ *                records it in a word of the shared array, which the next call clears.
  * Returns TRE_ERR_UNSUPPORTED, before enqueuing anything, when the model's plan needs
- * more than the 4 MiB array.  The first call on a device looks up the array's device
- * address; make that first call before any stream capture.  Every call shares the array
- * and leaves the previous call's contents in it (the call clears what must start at
- * zero): calls whose work overlaps on the GPU — two streams, two threads — race and give
- * undefined results; calls in one stream are ordered. */
+ * more than the 4 MiB array, and when `stream` is capturing a CUDA graph: every call
+ * copies its plan from host memory that is gone once the call returns, so the call
+ * cannot be captured.  Every call shares the array and leaves the previous call's
+ * contents in it (the call clears what must start at zero): calls whose work overlaps on
+ * the GPU — two streams, two threads — race and give undefined results; calls in one
+ * stream are ordered. */
 tre_status tre_decode_step_static(const tre_config* cfg, const tre_weights* w, int32_t token,
                                   int32_t pos, tre_stream stream, float* logits_dev,
                                   int32_t* token_dev, int32_t* status_dev);

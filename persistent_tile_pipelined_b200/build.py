@@ -23,7 +23,12 @@ ENGINE_LIB = os.path.join(PKG, "libtre.so")
 SYNTH_LIB = os.path.join(PKG, "synth", "libtre_synth.so")
 
 ENGINE_SOURCES = ["planner.cpp", "tre_api.cu", "engine.cu", "noalloc.cu"]
-ENGINE_HEADERS = ["tre_internal.h", "ptx.cuh", "tiles.cuh"]
+
+
+def engine_headers():
+    """Every header in csrc/: an edit to any of them rebuilds the library."""
+    return sorted(f for f in os.listdir(CSRC) if f.endswith((".h", ".cuh")))
+
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -57,7 +62,7 @@ def build_synth(force: bool = False) -> str:
 
 def build_engine(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     srcs = [os.path.join(CSRC, s) for s in ENGINE_SOURCES]
-    deps = srcs + [os.path.join(CSRC, h) for h in ENGINE_HEADERS] + [
+    deps = srcs + [os.path.join(CSRC, h) for h in engine_headers()] + [
         os.path.join(INCLUDE, "tre.h")]
     if not (force or extra_flags or _stale(ENGINE_LIB, deps)):
         return ENGINE_LIB

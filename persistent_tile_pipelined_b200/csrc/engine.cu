@@ -550,6 +550,14 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       rs = row_src(p, t, g);
     } else {
       attn_range(p, t, t0, t1);
+      // each lane that copies through a cache's tensor map acquires the map first (the
+      // allocation-free entry point rewrites its maps in place between launches)
+      const uint8_t* maps = static_cast<const uint8_t*>(p.kv_maps);
+      if (t.type == T_MLA_ATTN) {
+        if (lane < (p.KL + p.R) / kMlaBox) tensormap_acquire(maps + (size_t)t.layer * 128);
+      } else if (lane < 2 * (p.D / 64)) {
+        tensormap_acquire(maps + ((size_t)t.layer * 2 + (lane >= p.D / 64)) * 128);
+      }
     }
     const bool tiled = TILED && t.type == T_GEMV;
     TileStage ts{};

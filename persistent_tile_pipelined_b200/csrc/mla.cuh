@@ -73,6 +73,13 @@ __device__ __forceinline__ uint32_t lat_off(int r, int ch) {
 }
 
 // 2-D tensor copy of one box into shared memory, completing on `bar`.
+// Order this thread's later tensor copies through `map` (a 128-byte tensor map in global
+// memory) after generic-proxy writes of it, such as a host copy that rewrote the map at
+// the same address before this launch.
+__device__ __forceinline__ void tensormap_acquire(const void* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "

@@ -146,8 +146,10 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   // ---- argument checks (nothing is enqueued before they pass)
   if (token < 0 || token >= s.V) return fail(TRE_ERR_INVALID_ARG, "token outside [0, vocab)");
   if (pos < 0 || pos >= s.cap) return fail(TRE_ERR_POS_RANGE, "pos outside [0, kv_capacity)");
-  if (((uintptr_t)logits_dev & 15u) || (status_dev && ((uintptr_t)status_dev & 3u)))
+  if ((uintptr_t)logits_dev & 15u)
     return fail(TRE_ERR_INVALID_ARG, "logits_dev must be 16-byte aligned");
+  if (status_dev && ((uintptr_t)status_dev & 3u))
+    return fail(TRE_ERR_INVALID_ARG, "status_dev must be 4-byte aligned");
   if (!w->layer_w || !w->k_cache || !w->v_cache || !aligned16(w->embed) ||
       !aligned16(w->final_norm) || !aligned16(w->lm_head))
     return fail(TRE_ERR_INVALID_ARG, "weights: NULL or misaligned pointer");
@@ -178,11 +180,21 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
     if (st != TRE_OK) return st;
   }
 
+  // Every call copies its plan from ordinary host memory that is gone once it returns, so
+  // a captured call could never be replayed: refuse capture before enqueuing anything.
+  cudaStream_t sm = (cudaStream_t)stream;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if ((ce = cudaStreamIsCapturing(sm, &cap)) != cudaSuccess)
+    return cuda_fail(ce, "cudaStreamIsCapturing");
+  if (cap != cudaStreamCaptureStatusNone)
+    return fail(TRE_ERR_UNSUPPORTED,
+                "tre_decode_step_static cannot be captured in a CUDA graph (it copies the "
+                "plan from host memory on every call)");
+
   void* scratch = nullptr;
   st = setup_device(dev, &scratch);
   if (st != TRE_OK) return st;
   uint8_t* B = static_cast<uint8_t*>(scratch);
-  cudaStream_t sm = (cudaStream_t)stream;
 
   // ---- fill the array for this call (copies and a memset: no allocation)
   std::vector<double> inv(s.D / 2);

@@ -92,3 +92,31 @@ def test_clock_samples_inside_the_timed_windows():
     every = bench.parse_clocks(text, [])
     assert every["samples"] == 5 and every["reasons"] == ["hw_slowdown", "sw_power_cap"]
     assert bench.parse_clocks("", [(t0, t0 + 1)])["samples"] == 0
+
+
+def test_workload_step_bytes_match_the_planner():
+    """The bytes `config` states come from the workload shape alone (the reference arm
+    loads no engine library); they equal the planner's weight bytes plus the KV rows read
+    at the workload's length, the new rows written, the embedding row and the logits."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from persistent_tile_pipelined_b200 import tre
+    from persistent_tile_pipelined_b200.synth import workloads as W
+    for wl in W.WORKLOADS.values():
+        info = tre.tre_plan_inspect(tre.config_from_workload(wl))
+        row = (wl.kv_lora + wl.rope_dim) * 2 if wl.kind == "mla" else wl.n_kv_heads * wl.head_dim * 4
+        read = info.kv_bytes_at_capacity * wl.prefill // (wl.kv_capacity - 1)
+        lm = wl.vocab * 4 + 2 * wl.hidden if wl.vocab else 0
+        assert bench.workload_step_bytes(wl) == info.weight_bytes + read + wl.n_layers * row + lm
+
+
+def test_reference_arm_loads_no_engine_library():
+    """The CPU baseline describes and times its workload without libtre.so."""
+    code = ("import sys, runpy; sys.argv = ['bench.py', '--impl', 'reference', '--workload', "
+            "'tiny-2L-d256', '--steps', '3', '--warmup', '3'];\n"
+            "try:\n runpy.run_path('bench.py', run_name='__main__')\n"
+            "finally:\n print('LOADED', any('libtre.so' in l for l in open('/proc/self/maps')))")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "LOADED False" in out.stdout, out.stdout[-2000:]

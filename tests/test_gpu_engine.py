@@ -21,6 +21,10 @@ if not torch.cuda.is_available():
 from persistent_tile_pipelined_b200 import tre  # noqa: E402
 
 TOL = 2e-2
+# A second, tight bound near the error the engine actually reaches (fp32 accumulation
+# against the fp64 oracle measures ~1e-6 .. 1e-5): the 2e-2 contract alone would stay green
+# through a 1000x accuracy regression (a dropped eps, a lost lo part of a hi/lo split).
+REG_TOL = 1e-4
 ORC = oracle.Oracle(64)
 
 
@@ -65,11 +69,13 @@ def run_and_compare(wl, steps=1, check_hidden=True, state=None, **cfg):
         e = relerr(g, ref_logits)
         worst = max(worst, e)
         assert e <= TOL, f"logits rel err {e:.3g} at pos {pos}"
+        assert e <= REG_TOL, "regression bound: " + f"logits rel err {e:.3g} at pos {pos}"
         if check_hidden:
             hid = eng.hidden().cpu().numpy()
             for l in range(wl.n_layers):
                 el = relerr(hid[l], ref_hidden[l])
                 assert el <= TOL, f"layer {l} hidden rel err {el:.3g} at pos {pos}"
+                assert el <= REG_TOL, "regression bound: " + f"layer {l} hidden rel err {el:.3g} at pos {pos}"
         gtok = int(tok_dev.item())
         assert gtok == int(np.argmax(g)), "in-kernel argmax differs from host argmax"
         rtok = ORC.argmax(ref_logits)
@@ -140,7 +146,7 @@ def test_decode_step_host_matches_device_path():
     host_logits = np.empty(wl.vocab, dtype=np.float32)
     tok = eng.step_host(W.first_token(wl), wl.prefill, host_logits)
     ref, _ = ORC.decode_step(wl, model, W.first_token(wl), wl.prefill, want_hidden=False)
-    assert relerr(host_logits, ref) <= TOL
+    assert relerr(host_logits, ref) <= REG_TOL
     assert tok == int(np.argmax(host_logits))
     eng.close()
 
@@ -178,5 +184,16 @@ def test_llama8b_64_greedy_steps():
     per-layer hidden state checked."""
     wl = W.LLAMA8B.replace(decode_steps=65)
     worst, ties, state = run_and_compare(wl, steps=64, check_hidden=False)
-    assert worst <= TOL and ties <= 4
+    assert worst <= REG_TOL and ties <= 4
     run_and_compare(wl, steps=1, check_hidden=True, state=state)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("prefill", [32768, 131072], ids=["kv32k", "kv128k"])
+def test_llama8b_long_context(prefill):
+    """Long-context points of the 8B-shaped sweep: the same layer shapes, LM head and launch
+    configuration, on two layers so that the oracle fits host memory and time.  At 131072
+    cached positions each of the 18 splits per kv head streams ~114 stages, so the running
+    (m, l, O) and the combine see magnitudes the 4096-position tests never reach."""
+    wl = W.LLAMA8B.replace(n_layers=2, prefill=prefill, decode_steps=3)
+    run_and_compare(wl, steps=3)

@@ -21,6 +21,10 @@ if not torch.cuda.is_available():
 from persistent_tile_pipelined_b200 import tre  # noqa: E402
 
 TOL = 2e-2
+# A second, tight bound near the error the engine actually reaches (fp32 accumulation
+# against the fp64 oracle measures ~1e-6 .. 1e-5): the 2e-2 contract alone would stay green
+# through a 1000x accuracy regression (a dropped eps, a lost lo part of a hi/lo split).
+REG_TOL = 1e-4
 ORC = oracle.Oracle(64)
 
 SMALL = W.MLA4.replace(name="mla-small", n_layers=2, hidden=512, n_q_heads=16, q_lora=128,
@@ -59,6 +63,7 @@ def run_mla(wl, steps=1, **cfg_over):
             e = relerr(hid[l], h)
             worst = max(worst, e)
             assert e <= TOL, f"layer {l} hidden rel err {e:.3g} at pos {pos}"
+            assert e <= REG_TOL, "regression bound: " + f"layer {l} hidden rel err {e:.3g} at pos {pos}"
         assert np.array_equal(out_dev.cpu().numpy(), hid[-1])
         x = h
     start, end = wl.prefill, wl.prefill + steps
@@ -99,21 +104,6 @@ def test_mla_launch_shapes(cfg):
 @pytest.mark.slow
 def test_mla_full_size_four_layers():
     """The full absorbed-MLA workload: hidden 7168, 128 heads, q_lora 1536, kv_lora 512,
-    rope 64, nope 128, v 128, 4 layers over 8192 cached latent rows."""
-    wl = W.MLA4
-    model = W.gen_mla_model(wl)
-    dev = tre.upload_mla_model(model)
-    eng = tre.Engine(tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_HIDDEN), dev)
-    x = model["x_in"].astype(np.float64)
-    x_dev = torch.from_numpy(x.astype(np.float32)).cuda()
-    out_dev = torch.empty_like(x_dev)
-    eng.layers_step(x_dev, out_dev, wl.prefill)
-    torch.cuda.synchronize()
-    assert eng.status() == (0, 0)
-    hid = eng.hidden().cpu().numpy()
-    h = x
-    for l in range(wl.n_layers):
-        h = ORC.mla_layer_step(wl, model["layers"][l], model["latent_cache"][l].copy(),
-                               wl.prefill, h)
-        assert relerr(hid[l], h) <= TOL
-    eng.close()
+    rope 64, nope 128, v 128, 4 layers over 8192 cached latent rows, 3 steps with each
+    step's input the oracle's output of the previous one."""
+    run_mla(W.MLA4.replace(decode_steps=3), steps=3)
