@@ -65,6 +65,11 @@ def parse():
                     help="engine config override (launch shape, K-part limit); repeatable")
     ap.add_argument("--flags", type=int, default=0,
                     help="engine debug flags for the timed engine (8 = no cross-op prefetch)")
+    ap.add_argument("--launch-mode", default="persistent", choices=["persistent", "per-op"],
+                    help="persistent: one launch per step (the product); per-op: the same "
+                         "tiles, one plain launch per op (measurement form)")
+    ap.add_argument("--no-ablation", action="store_true",
+                    help="skip the kernel-per-op comparison and the device-loop timing")
     return ap.parse_args()
 
 
@@ -518,6 +523,9 @@ def run_engine(args, rank, world, local_rank):
     K, Wm, M = args.steps, args.warmup, args.tokens_per_step
     wl = wl.replace(decode_steps=K + Wm, tokens_per_step=M, seed=wl.seed + rank)
     eng, model = build_engine(wl, local_rank, args.flags, config_overrides(args.config))
+    from persistent_tile_pipelined_b200 import tre
+    timed_launches = eng.set_launch_mode(tre.TRE_LAUNCH_PER_OP if args.launch_mode == "per-op"
+                                         else tre.TRE_LAUNCH_PERSISTENT)
     stream = torch.cuda.current_stream(local_rank)
     s_ptr = stream.cuda_stream
     # step i takes tokens i M .. i M + M - 1 of the seeded stream at positions prefill + i M ..
@@ -581,6 +589,9 @@ def run_engine(args, rank, world, local_rank):
     clocks = sampler.stop()
 
     step_bytes = float(np.mean([eng.step_bytes(positions[Wm + i], M) for i in range(K)]))
+    extra = {}
+    if M == 1 and not args.no_ablation and args.launch_mode == "persistent":
+        extra = ablation(eng, wl, tokens, positions, Wm, K, stream, local_rank, barrier)
     trace_path = args.trace if rank == 0 else ""
     eng.close()
     del model
@@ -591,7 +602,80 @@ def run_engine(args, rank, world, local_rank):
 
     dev_s, e2e_s, launch_ms_avg = max_over_ranks(
         [dev_s, e2e_s, float(np.mean(launch_ms))], world, f"cuda:{local_rank}")
-    return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks
+    if extra:
+        keys = sorted(k for k, v in extra.items() if isinstance(v, float))
+        worst = max_over_ranks([extra[k] for k in keys], world, f"cuda:{local_rank}")
+        extra.update(zip(keys, worst))
+    extra["timed_launches_per_step"] = timed_launches
+    return wl, dev_s, e2e_s, launch_ms_avg, step_bytes, clocks, extra
+
+
+def ablation(eng, wl, tokens, positions, Wm, K, stream, local_rank, barrier):
+    """Beside the timed persistent steps: (1) the kernel-per-op form of the same step (the
+    same tiles on the same plan, one plain launch per op) enqueued launch by launch and
+    replayed from CUDA graphs, timed with CUDA events over steps at the same positions
+    (each step streams the same bytes); (2) the device-resident greedy loop
+    (tre_decode_loop): n steps enqueued at once, each step's argmax feeding the next on the
+    device, timed end to end on the host up to the n tokens back in pinned host memory."""
+    import torch
+
+    from persistent_tile_pipelined_b200 import tre
+    n = min(K, 16)
+    s_ptr = stream.cuda_stream
+    out = {}
+
+    def timed(run):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        barrier()
+        ev[0].record(stream)
+        for i in range(n):
+            run(i)
+        ev[1].record(stream)
+        torch.cuda.synchronize(local_rank)
+        return ev[0].elapsed_time(ev[1]) / n
+
+    out["launches_per_step"] = eng.set_launch_mode(tre.TRE_LAUNCH_PER_OP)
+    for i in range(3):
+        eng.step(tokens[Wm + i][0], positions[Wm + i], stream=s_ptr)
+    out["per_op_ms_per_step"] = timed(lambda i: eng.step(tokens[Wm + i][0], positions[Wm + i],
+                                                         stream=s_ptr))
+    # the same per-op steps captured once and replayed (host launch cost removed)
+    graphs = []
+    side = torch.cuda.Stream(local_rank)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for i in range(n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                eng.step(tokens[Wm + i][0], positions[Wm + i], stream=side.cuda_stream)
+            graphs.append(g)
+    stream.wait_stream(side)
+    torch.cuda.synchronize(local_rank)
+    for i in range(3):
+        graphs[i].replay()
+    out["per_op_graph_ms_per_step"] = timed(lambda i: graphs[i].replay())
+    del graphs
+    st = eng.status()
+    assert st == (0, 0), st
+    eng.set_launch_mode(tre.TRE_LAUNCH_PERSISTENT)
+    for i in range(3):
+        eng.step(tokens[Wm + i][0], positions[Wm + i], stream=s_ptr)
+    out["persistent_ms_per_step"] = timed(lambda i: eng.step(tokens[Wm + i][0], positions[Wm + i],
+                                                             stream=s_ptr))
+    # device-resident greedy loop: n steps, one call, tokens back once
+    toks_dev = torch.empty(n, dtype=torch.int32, device=f"cuda:{local_rank}")
+    toks_pin = torch.empty(n, dtype=torch.int32).pin_memory()
+    eng.decode_loop(tokens[Wm][0], positions[Wm], 3, toks_dev, stream=s_ptr)
+    barrier()
+    t0 = time.perf_counter()
+    eng.decode_loop(tokens[Wm][0], positions[Wm], n, toks_dev, stream=s_ptr)
+    toks_pin.copy_(toks_dev, non_blocking=True)
+    torch.cuda.synchronize(local_rank)
+    out["device_loop_s_per_step"] = (time.perf_counter() - t0) / n
+    st = eng.status()
+    assert st == (0, 0), st
+    out["steps"] = n
+    return out
 
 
 def write_trace(wl, device, path, flags=0, overrides=None):
@@ -640,7 +724,8 @@ def main():
     from persistent_tile_pipelined_b200.synth import workloads as W
     if W.WORKLOADS[args.workload].kind != "gqa":
         return main_layers(args, rank, world, local_rank)
-    wl, dev_s, e2e_s, launch_ms, step_bytes, clocks = run_engine(args, rank, world, local_rank)
+    wl, dev_s, e2e_s, launch_ms, step_bytes, clocks, abl = run_engine(args, rank, world,
+                                                                      local_rank)
     K, M = args.steps, args.tokens_per_step
     peak, peak_kind = peaks()
     achieved = step_bytes / (launch_ms / 1e3) / 1e9
@@ -672,9 +757,31 @@ def main():
                 "d2h_bytes_per_step": 4 * M,
                 "note": "greedy loop via tre_decode_step_host: token in as a kernel argument, "
                         "argmax token back to pinned-less host memory, host wall time"},
-        "gpu_launches": K,
+        "gpu_launches": K * abl["timed_launches_per_step"],
+        "launch_mode": args.launch_mode,
         "clocks": clocks,
     }
+    if "steps" in abl:
+        n = abl["steps"]
+        line["ablation"] = {
+            "what": "the same tiles on the same plan: one persistent launch per step vs one "
+                    "plain launch per op (QKV, attention + combine, O, gate/up, down per layer, "
+                    "LM head), enqueued launch by launch and replayed from CUDA graphs; "
+                    f"{n} steps each at the timed positions, CUDA events",
+            "launches_per_step": abl["launches_per_step"],
+            "persistent_ms_per_step": abl["persistent_ms_per_step"],
+            "per_op_ms_per_step": abl["per_op_ms_per_step"],
+            "per_op_graph_ms_per_step": abl["per_op_graph_ms_per_step"],
+            "per_op_extra_us_per_launch": (abl["per_op_ms_per_step"] -
+                                           abl["persistent_ms_per_step"]) * 1e3 /
+                                          abl["launches_per_step"],
+        }
+        line["e2e_device_loop"] = {
+            "value": world / abl["device_loop_s_per_step"], "unit": "tokens/s",
+            "h2d_bytes_per_step": 4.0 / n, "d2h_bytes_per_step": 4,
+            "note": f"tre_decode_loop: {n} greedy steps in one call, each step's argmax feeds "
+                    "the next step on the device; host wall time up to the tokens back in "
+                    "pinned memory"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_layers)

@@ -259,6 +259,34 @@ tre_status tre_decode_step_static(const tre_config* cfg, const tre_weights* w, i
                                   int32_t pos, tre_stream stream, float* logits_dev,
                                   int32_t* token_dev, int32_t* status_dev);
 
+/* n_steps greedy decode steps with no host round trip between them ([SC] §1: the host
+ * launches once per token and never waits for the model; [TA] blog-vs-code table).  Step
+ * i runs at position pos + i; its input token is `token` for i = 0 and, for i > 0, the
+ * greedy argmax of step i - 1, which the kernel reads from tokens_dev[i - 1] on the
+ * device.  Every step is enqueued on `stream` before the call returns; nothing waits.
+ *   tokens_dev   device int32[n_steps] (4-byte aligned): the argmax token of every step
+ *   logits_dev   device fp32[vocab] or NULL (16-byte aligned): the last step's logits
+ * The caches hold [0, pos) on entry and [0, pos + n_steps) once the steps have run;
+ * pos + n_steps <= kv_capacity.  Each step is one launch in the engine's launch mode.
+ * Requires has_embed_lm_head == 1.  Enqueues asynchronously; returns a previous step's
+ * device error without launching. */
+tre_status tre_decode_loop(tre_engine* e, int32_t token, int32_t pos, int32_t n_steps,
+                           tre_stream stream, int32_t* tokens_dev, float* logits_dev);
+
+/* Launch modes.  PERSISTENT (the default): a step is ONE cooperative launch of the
+ * persistent kernel, in which a task starts as soon as the tasks it reads are done
+ * ([SI] section on breaking the kernel boundary).  PER_OP: the same tasks on the same
+ * plan, with the kernel boundary put back — one plain launch per op group (the tasks of
+ * one layer's op: QKV, attention, O, gate/up, down, ...; ~9 per layer plus the LM head),
+ * each launch starting after the previous one has finished.  PER_OP exists to measure
+ * what the persistent form removes (the launch cost and the drain / ramp at every op
+ * boundary that [SC] §6 names); it computes the same results. */
+enum { TRE_LAUNCH_PERSISTENT = 0, TRE_LAUNCH_PER_OP = 1 };
+
+/* Set the launch mode of every later step call on `e`.  *launches_per_step (may be NULL)
+ * receives the number of kernel launches one step then takes (1, or the op groups). */
+tre_status tre_set_launch_mode(tre_engine* e, int32_t mode, int32_t* launches_per_step);
+
 /* One step of a layers-only stack (has_embed_lm_head == 0): the residual stream after
  * the last layer for one token at `pos`, from the hidden vector entering layer 0.
  *   x_in_dev    device fp32[hidden], read only (16-byte aligned)
@@ -318,6 +346,15 @@ tre_status tre_plan_inspect(const tre_config* cfg, int32_t num_sms, int32_t smem
  * least the task count, out_sm_begin whenever it is not NULL. */
 int32_t tre_plan_tasks(const tre_config* cfg, int32_t num_sms, int32_t smem_per_block,
                        int32_t* out_tasks, int32_t max_tasks, int32_t* out_sm_begin);
+
+/* Plan without a GPU and dump the kernel-per-op form (TRE_LAUNCH_PER_OP): the op groups
+ * are the maximal runs of tasks, in global task order, of one layer, task type and op;
+ * for group g and SM s, out_ranges[2 (g num_sms + s)] .. [+1] is the half-open range of
+ * task indices (into the tre_plan_tasks array) that CTA s runs in launch g.  Returns the
+ * number of groups or a negative tre_status; out_ranges ([groups][num_sms][2] int32) is
+ * written only when max_groups is at least the group count. */
+int32_t tre_plan_op_groups(const tre_config* cfg, int32_t num_sms, int32_t smem_per_block,
+                           int32_t* out_ranges, int32_t max_groups);
 
 /* Human-readable text of the last host-side error of this thread. */
 const char* tre_last_error(void);

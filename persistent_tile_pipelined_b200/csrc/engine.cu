@@ -622,12 +622,25 @@ __device__ __forceinline__ unsigned long long pack_best(const Best& b) {
   return ((unsigned long long)key << 32) | (uint32_t)(0xffffffffu - (uint32_t)b.i);
 }
 
+// Token v of this step: a kernel argument, or (greedy loop) token 0 read from the device
+// word the previous step's argmax wrote.  An id outside [0, V) records a bounds error and
+// is clamped, so that no access leaves the embedding.
+__device__ __forceinline__ int step_token(const Params& p, int v) {
+  if (v > 0 || !p.token_in) return p.tokens[v];
+  const int tok = __ldcg(p.token_in);
+  if (tok < 0 || tok >= p.V) {
+    record_error(p, TRE_ERR_BOUNDS, -4);
+    return 0;
+  }
+  return tok;
+}
+
 // Row n of token v's residual stream entering `layer` (layer 0: the embedding row or the
 // layer-only input).
 __device__ __forceinline__ float resid_in(const Params& p, int layer, int n, int v = 0) {
   if (layer > 0) return __ldcg(p.x + (size_t)v * p.d + n);
   if (p.x_in) return __ldcg(p.x_in + (size_t)v * p.d + n);
-  return bf_lo(p.embed[(size_t)p.tokens[v] * p.d + n]);
+  return bf_lo(p.embed[(size_t)step_token(p, v) * p.d + n]);
 }
 
 // Input-vector identity for reuse across consecutive tasks (same layer, same source,
@@ -701,7 +714,7 @@ __device__ void load_input(const Params& p, const Task& t, const GemvGeom& gg, f
       for (int u = 0; u < kLoadBatch; ++u) {
         const int w = min(w0 + u * kConsumerThreads, nitems - 1);
         const int v = w % MT, j = w / MT;
-        const uint4 x = __ldg(reinterpret_cast<const uint4*>(src_bf + (size_t)p.tokens[v] * p.d) + j);
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(src_bf + (size_t)step_token(p, v) * p.d) + j);
         ra[u] = make_float4(__uint_as_float(x.x), __uint_as_float(x.y), __uint_as_float(x.z),
                             __uint_as_float(x.w));
       }
@@ -764,7 +777,7 @@ __device__ void load_input(const Params& p, const Task& t, const GemvGeom& gg, f
     float* xlo = ub + (size_t)v * K;
     float* xhi = xlo + K / 2;
     const float* sv = src ? src + v * vstride : nullptr;
-    const uint16_t* bv = src_bf ? src_bf + (size_t)p.tokens[v] * p.d : nullptr;
+    const uint16_t* bv = src_bf ? src_bf + (size_t)step_token(p, v) * p.d : nullptr;
     for (int j = ctid; j < K8; j += kConsumerThreads) {
       float e[8];
       if (bv) {
@@ -2027,8 +2040,17 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
   float* misc = ub + p.ub_floats;  // the union buffer covers the input planes and attention scratch
 
   const int b = blockIdx.x;
-  const Task* my = p.tasks + p.sm_begin[b];
-  const int ntask = p.sm_begin[b + 1] - p.sm_begin[b];
+  const Task* my;
+  int ntask;
+  if (p.op_group >= 0) {  // kernel-per-op form: this CTA's tasks of one op
+    const int32_t* r = p.op_ranges + 2 * ((size_t)p.op_group * gridDim.x + b);
+    my = p.tasks + r[0];
+    ntask = r[1] - r[0];
+    if (ntask == 0) return;
+  } else {
+    my = p.tasks + p.sm_begin[b];
+    ntask = p.sm_begin[b + 1] - p.sm_begin[b];
+  }
   // the swizzled latent tiles assume 1024-byte aligned ring slots
   if (p.KL > 0 && (smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) record_error(p, TRE_ERR_BOUNDS, -3);
@@ -2075,12 +2097,21 @@ static const void* kernel_for(bool mla, int m, bool tiled) {
 }
 
 // Configure the instantiations a plan can launch (m = 1 .. max_m) and report how many
-// CTAs of the largest fit on an SM.
+// CTAs of `smem_bytes` fit on an SM.  The shared-memory limit is a property of the kernel
+// function shared by every engine in the process, so it is raised to the device maximum
+// (never lowered to this plan's need: an engine created later must not shrink what an
+// earlier one launches with).
 cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled) {
   *blocks_per_sm = 1 << 30;
+  int dev = 0, optin = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 == cudaSuccess)
+    e0 = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e0 != cudaSuccess) return e0;
+  const int limit = optin > smem_bytes ? optin : smem_bytes;
   for (int m = 1; m <= (mla ? 1 : max_m); ++m) {
     const void* k = kernel_for(mla, m, tiled);
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
     if (e != cudaSuccess) return e;
     int b = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, kThreads, smem_bytes);
@@ -2090,6 +2121,9 @@ cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int m
   return cudaSuccess;
 }
 
+// The persistent form is a cooperative launch (every CTA resident: tasks wait on other
+// CTAs' counters); a kernel-per-op launch (p.op_group >= 0) is a plain one, since every
+// dependency of its tasks was met by the launches before it.
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream, bool mla) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -2100,9 +2134,11 @@ cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.op_group >= 0 ? 0 : 1;
   void* args[] = {const_cast<Params*>(&p)};
-  return cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0), args);
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0), args);
+  if (e != cudaSuccess) cudaGetLastError();  // returned here: do not leave it to the caller
+  return e;
 }
 
 }  // namespace tre

@@ -53,8 +53,8 @@ tre_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 // Once per device, with that device current: resolve the array's device address.  Every
-// call also raises the kernel's shared-memory limit to the device maximum (a host-side
-// attribute, not an allocation), since an engine created meanwhile may have lowered it.
+// call also makes sure the kernel's shared-memory limit is the device maximum (a host-side
+// attribute, not an allocation).
 tre_status setup_device(int dev, void** scratch) {
   std::lock_guard<std::mutex> lock(g_setup_mu);
   if (!g_scratch_dev[dev]) {
@@ -219,6 +219,7 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   Params p{};
   p.tasks = reinterpret_cast<const Task*>(B + o_tasks);
   p.sm_begin = reinterpret_cast<const int32_t*>(B + o_begin);
+  p.op_group = -1;  // the whole step in one persistent launch
   p.counters = reinterpret_cast<uint32_t*>(B + o_ctr);
   p.tickets = reinterpret_cast<uint32_t*>(B + o_tick);
   p.lm_ticket = reinterpret_cast<uint32_t*>(B + o_lmt);

@@ -499,6 +499,52 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   return TRE_OK;
 }
 
+// Kernel-per-op form of a plan: the op groups (maximal runs of tasks, in global task
+// order, of one layer, task type and op) and, per group and SM, the contiguous range of
+// that SM's queue holding the group's tasks ([G][nsm][2] into the task array; empty
+// ranges where an SM has none).  Returns G, or -1 if some SM's tasks of a group are not
+// contiguous in its queue (the planner never builds such a plan).
+int plan_op_groups(const std::vector<Task>& tasks, const std::vector<int32_t>& sm_begin, int nsm,
+                   std::vector<int32_t>* ranges) {
+  const int n = (int)tasks.size();
+  std::vector<int> at(n, -1);  // queue index of each task id
+  for (int i = 0; i < n; ++i) {
+    if (tasks[i].id < 0 || tasks[i].id >= n || at[tasks[i].id] >= 0) return -1;
+    at[tasks[i].id] = i;
+  }
+  std::vector<int> group(n, 0);  // by queue index
+  int G = 0;
+  for (int id = 0; id < n; ++id) {
+    const Task& t = tasks[at[id]];
+    if (id == 0) {
+      G = 1;
+    } else {
+      const Task& u = tasks[at[id - 1]];
+      if (t.layer != u.layer || t.type != u.type || t.op != u.op) ++G;
+    }
+    group[at[id]] = G - 1;
+  }
+  ranges->assign((size_t)G * nsm * 2, 0);
+  for (int s = 0; s < nsm; ++s) {
+    for (int g = 0; g < G; ++g) {
+      (*ranges)[2 * ((size_t)g * nsm + s)] = sm_begin[s];
+      (*ranges)[2 * ((size_t)g * nsm + s) + 1] = sm_begin[s];
+    }
+    int prev = -1;
+    for (int i = sm_begin[s]; i < sm_begin[s + 1]; ++i) {
+      const int g = group[i];
+      int32_t* r = ranges->data() + 2 * ((size_t)g * nsm + s);
+      if (g != prev) {
+        if (g < prev) return -1;
+        r[0] = i;
+        prev = g;
+      }
+      r[1] = i + 1;
+    }
+  }
+  return G;
+}
+
 int64_t step_bytes(const PlanShape& s, int pos, int m) {
   const int64_t d = s.d, D = s.D;
   if (s.kind == TRE_LAYER_MLA) {

@@ -40,6 +40,8 @@ struct tre_engine {
   int32_t* token_buf = nullptr;
   int last_m = 1;                // tokens of the last step (debug hidden layout)
   float* logits_buf = nullptr;
+  int n_groups = 0;              // op groups of the plan (kernel-per-op form)
+  int launch_mode = TRE_LAUNCH_PERSISTENT;
 };
 
 #define TRE_EXPORT extern "C" __attribute__((visibility("default")))
@@ -165,6 +167,26 @@ TRE_EXPORT int32_t tre_plan_tasks(const tre_config* cfg, int32_t num_sms, int32_
   return (int32_t)tasks.size();
 }
 
+TRE_EXPORT int32_t tre_plan_op_groups(const tre_config* cfg, int32_t num_sms,
+                                      int32_t smem_per_block, int32_t* out_ranges,
+                                      int32_t max_groups) {
+  if (!cfg) return TRE_ERR_INVALID_ARG;
+  PlanShape s;
+  std::vector<Task> tasks;
+  std::vector<int32_t> begin, ranges;
+  int nsm = cfg->num_sms ? std::min<int>(cfg->num_sms, num_sms) : num_sms;
+  tre_status st = plan_build(*cfg, nsm, smem_per_block, &s, &tasks, &begin, nullptr);
+  if (st != TRE_OK) return st;
+  const int G = plan_op_groups(tasks, begin, nsm, &ranges);
+  if (G < 0) {
+    set_error("tre_plan_op_groups: an op's tasks are not contiguous in an SM queue");
+    return TRE_ERR_UNSUPPORTED;
+  }
+  if (out_ranges && max_groups >= G)
+    std::memcpy(out_ranges, ranges.data(), ranges.size() * sizeof(int32_t));
+  return G;
+}
+
 TRE_EXPORT void tre_destroy(tre_engine* e) {
   if (!e) return;
   int prev = 0;
@@ -250,6 +272,13 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
     return TRE_ERR_INVALID_ARG;
   }
 
+  std::vector<int32_t> ranges;
+  const int n_groups = plan_op_groups(tasks, begin, nsm, &ranges);
+  if (n_groups < 0) {
+    set_error("tre_create: an op's tasks are not contiguous in an SM queue");
+    return TRE_ERR_UNSUPPORTED;
+  }
+
   int bps = 0;
   CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M, s.tiles != 0));
   if (bps < 1) {
@@ -262,6 +291,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   e->device = device;
   e->shape = s;
   e->n_tasks = (int)tasks.size();
+  e->n_groups = n_groups;
 
   // ---- one device block for all engine-owned state
   const int qkv_n = mla ? s.Hq * (s.NP + s.R) : (s.Hq + 2 * s.Hkv) * s.D;
@@ -281,6 +311,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   Carve cv;
   size_t o_tasks = cv.take<Task>(tasks.size());
   size_t o_begin = cv.take<int32_t>(begin.size());
+  size_t o_ranges = cv.take<int32_t>(ranges.size());
   size_t o_layers = cv.take<LayerPtrs>(s.L);
   size_t o_ctr = cv.take<uint32_t>(s.n_counters);
   size_t o_tick = cv.take<uint32_t>(std::max(s.Hkv, mla ? s.Hq / kMlaHeadGroup : 1));
@@ -336,6 +367,9 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   if ((ce = cudaMemcpy(B + o_begin, begin.data(), begin.size() * sizeof(int32_t),
                        cudaMemcpyHostToDevice)) != cudaSuccess)
     return fail_free(ce, "upload queues");
+  if ((ce = cudaMemcpy(B + o_ranges, ranges.data(), ranges.size() * sizeof(int32_t),
+                       cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail_free(ce, "upload op groups");
   if ((ce = cudaMemcpy(B + o_layers, lp.data(), lp.size() * sizeof(LayerPtrs),
                        cudaMemcpyHostToDevice)) != cudaSuccess)
     return fail_free(ce, "upload layer table");
@@ -364,6 +398,9 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   Params& p = e->base;
   p.tasks = reinterpret_cast<const Task*>(B + o_tasks);
   p.sm_begin = reinterpret_cast<const int32_t*>(B + o_begin);
+  p.op_ranges = reinterpret_cast<const int32_t*>(B + o_ranges);
+  p.op_group = -1;
+  p.token_in = nullptr;
   p.counters = reinterpret_cast<uint32_t*>(B + o_ctr);
   p.tickets = reinterpret_cast<uint32_t*>(B + o_tick);
   p.lm_ticket = reinterpret_cast<uint32_t*>(B + o_lmt);
@@ -432,9 +469,11 @@ static tre_status pending_device_error(tre_engine* e) {
   return (tre_status)code;
 }
 
+// Enqueue one step: one persistent launch, or (kernel-per-op form) one plain launch per
+// op group.  token_in (device, or NULL): token 0 is read there by the kernel.
 static tre_status launch_step(tre_engine* e, const int32_t* tokens, int m, int32_t pos,
                               cudaStream_t stream, float* logits_dev, int32_t* token_dev,
-                              const float* x_in, float* x_out) {
+                              const float* x_in, float* x_out, const int32_t* token_in = nullptr) {
   tre_status st = pending_device_error(e);
   if (st != TRE_OK) return st;
   if (pos < 0 || pos + m > e->shape.cap) {
@@ -446,20 +485,79 @@ static tre_status launch_step(tre_engine* e, const int32_t* tokens, int m, int32
   p.m = m;
   for (int v = 0; v < kMaxTokens; ++v) p.tokens[v] = v < m ? tokens[v] : tokens[0];
   p.token = tokens[0];
+  p.token_in = token_in;
   p.pos = pos;
   p.epoch = ++e->epoch;
   if (logits_dev) p.logits = logits_dev;
   p.token_out = token_dev ? token_dev : e->token_buf;
   p.x_in = x_in;
   p.x_out = x_out;
-  cudaError_t ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream,
-                                 e->shape.kind == TRE_LAYER_MLA);
+  const bool mla = e->shape.kind == TRE_LAYER_MLA;
+  cudaError_t ce = cudaSuccess;
+  if (e->launch_mode == TRE_LAUNCH_PER_OP) {
+    for (int g = 0; g < e->n_groups && ce == cudaSuccess; ++g) {
+      p.op_group = g;
+      ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream, mla);
+    }
+  } else {
+    ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream, mla);
+  }
   if (ce != cudaSuccess) {
     --e->epoch;
-    return cuda_fail(ce, "launch of the persistent engine");
+    return cuda_fail(ce, "launch of the engine kernel");
   }
   e->last_m = m;
   e->last_stream = stream;
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_set_launch_mode(tre_engine* e, int32_t mode,
+                                          int32_t* launches_per_step) {
+  if (!e) {
+    set_error("tre_set_launch_mode: NULL engine");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (mode != TRE_LAUNCH_PERSISTENT && mode != TRE_LAUNCH_PER_OP) {
+    set_error("tre_set_launch_mode: unknown mode");
+    return TRE_ERR_INVALID_ARG;
+  }
+  e->launch_mode = mode;
+  if (launches_per_step) *launches_per_step = mode == TRE_LAUNCH_PER_OP ? e->n_groups : 1;
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_decode_loop(tre_engine* e, int32_t token, int32_t pos, int32_t n_steps,
+                                      tre_stream stream, int32_t* tokens_dev, float* logits_dev) {
+  if (!e || !tokens_dev) {
+    set_error("tre_decode_loop: NULL engine or tokens_dev");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (!e->shape.has_lm) {
+    set_error("tre_decode_loop: engine has no embedding / LM head");
+    return TRE_ERR_UNSUPPORTED;
+  }
+  if (n_steps < 1) {
+    set_error("tre_decode_loop: n_steps must be >= 1");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (token < 0 || token >= e->shape.V) {
+    set_error("tre_decode_loop: token outside [0, vocab)");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (((uintptr_t)tokens_dev & 3u) || (logits_dev && ((uintptr_t)logits_dev & 15u))) {
+    set_error("tre_decode_loop: tokens_dev must be 4-byte and logits_dev 16-byte aligned");
+    return TRE_ERR_INVALID_ARG;
+  }
+  if (pos < 0 || (int64_t)pos + n_steps > e->shape.cap) {
+    set_error("tre_decode_loop: pos .. pos + n_steps - 1 outside [0, kv_capacity)");
+    return TRE_ERR_POS_RANGE;
+  }
+  for (int i = 0; i < n_steps; ++i) {
+    tre_status st = launch_step(e, &token, 1, pos + i, (cudaStream_t)stream, logits_dev,
+                                tokens_dev + i, nullptr, nullptr,
+                                i == 0 ? nullptr : tokens_dev + i - 1);
+    if (st != TRE_OK) return st;
+  }
   return TRE_OK;
 }
 

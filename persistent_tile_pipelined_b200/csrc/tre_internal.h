@@ -145,6 +145,12 @@ struct PlanShape {
 struct Params {
   const Task* tasks;
   const int32_t* sm_begin;         // [nsm + 1] offsets into tasks
+  // Kernel-per-op launches (the measurement form with the kernel boundary put back): this
+  // launch runs op group `op_group` only, CTA b the tasks [op_ranges[2 (g nsm + b)],
+  // op_ranges[2 (g nsm + b) + 1]) of p.tasks; op_group < 0: the whole step (the
+  // persistent form).
+  const int32_t* op_ranges;
+  int op_group;
   uint32_t* counters;
   uint32_t* tickets;               // [Hkv] split-KV arrival tickets
   uint32_t* lm_ticket;
@@ -191,6 +197,7 @@ struct Params {
   int nsplit, pps, stage_bytes, ring_stages, xs_floats, ub_floats;
   float eps;
   int token, pos;
+  const int32_t* token_in;         // device word holding token 0 (greedy loop), or NULL
   int m;                           // tokens this step (1 .. kMaxTokens): positions pos .. pos + m - 1
   int32_t tokens[kMaxTokens];
   uint32_t epoch;
@@ -213,6 +220,8 @@ tre_status plan_build(const tre_config& cfg, int nsm, int smem_limit, PlanShape*
                       std::vector<Task>* tasks, std::vector<int32_t>* sm_begin,
                       std::vector<int64_t>* sm_bytes);
 int64_t step_bytes(const PlanShape& s, int pos, int m = 1);
+int plan_op_groups(const std::vector<Task>& tasks, const std::vector<int32_t>& sm_begin, int nsm,
+                   std::vector<int32_t>* ranges);
 void set_error(const std::string& msg);
 // Host only, allocates nothing: a 2-D tensor map (128 bytes at out128) over a bf16 cache
 // [rows][C] with 64-column x box_rows boxes and the 128-byte swizzle (tre_api.cu).

@@ -68,10 +68,13 @@ class tre_plan_info(ctypes.Structure):
                                       "min_sm_bytes")]
 
 
+TRE_LAUNCH_PERSISTENT, TRE_LAUNCH_PER_OP = 0, 1
+
 EXPORTED = ("tre_create", "tre_destroy", "tre_decode_step", "tre_decode_step_host",
             "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
-            "tre_decode_tokens", "tre_get_status", "tre_reset", "tre_debug_hidden", "tre_debug_trace",
-            "tre_step_bytes", "tre_plan_inspect", "tre_plan_tasks", "tre_last_error")
+            "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
+            "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
+            "tre_plan_inspect", "tre_plan_tasks", "tre_plan_op_groups", "tre_last_error")
 
 
 def _load() -> ctypes.CDLL:
@@ -90,6 +93,10 @@ def _load() -> ctypes.CDLL:
                                          i32, i32, vp, vp, vp, vp]
     L.tre_layers_step.argtypes = [vp, vp, vp, i32, vp]
     L.tre_decode_tokens.argtypes = [vp, vp, i32, i32, vp, vp, vp]
+    L.tre_decode_loop.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    L.tre_set_launch_mode.argtypes = [vp, i32, ctypes.POINTER(i32)]
+    L.tre_plan_op_groups.argtypes = [ctypes.POINTER(tre_config), i32, i32, vp, i32]
+    L.tre_plan_op_groups.restype = i32
     L.tre_debug_routing.argtypes = [vp, vp, vp]
     L.tre_get_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.tre_reset.argtypes = [vp, vp]
@@ -104,7 +111,7 @@ def _load() -> ctypes.CDLL:
     L.tre_last_error.restype = ctypes.c_char_p
     for name in ("tre_create", "tre_decode_step", "tre_decode_step_host",
                  "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
-                 "tre_decode_tokens", "tre_get_status",
+                 "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
                  "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
                  "tre_plan_inspect"):
         getattr(L, name).restype = ctypes.c_int
@@ -203,6 +210,33 @@ def tre_decode_tokens(h, tokens, pos: int, stream: int = 0, logits_dev: int = 0,
     return lib.tre_decode_tokens(h, arr, len(tokens), int(pos), ctypes.c_void_p(stream or None),
                                  ctypes.c_void_p(logits_dev or None),
                                  ctypes.c_void_p(tokens_dev or None))
+
+
+def tre_decode_loop(h, token: int, pos: int, n_steps: int, stream: int = 0, tokens_dev: int = 0,
+                    logits_dev: int = 0) -> int:
+    return lib.tre_decode_loop(h, int(token), int(pos), int(n_steps),
+                               ctypes.c_void_p(stream or None), ctypes.c_void_p(tokens_dev or None),
+                               ctypes.c_void_p(logits_dev or None))
+
+
+def tre_set_launch_mode(h, mode: int) -> int:
+    """Set the engine's launch mode; returns the kernel launches one step takes."""
+    n = ctypes.c_int32()
+    check(lib.tre_set_launch_mode(h, int(mode), ctypes.byref(n)), "tre_set_launch_mode")
+    return n.value
+
+
+def tre_plan_op_groups(cfg: tre_config, num_sms: int = 148, smem_per_block: int = 232448):
+    """Returns ranges int32[groups][num_sms][2] of the kernel-per-op form."""
+    nsm = min(cfg.num_sms, num_sms) if cfg.num_sms else num_sms
+    g = lib.tre_plan_op_groups(ctypes.byref(cfg), num_sms, smem_per_block, None, 0)
+    if g < 0:
+        raise TreError(g, "tre_plan_op_groups")
+    out = np.zeros((g, nsm, 2), dtype=np.int32)
+    g2 = lib.tre_plan_op_groups(ctypes.byref(cfg), num_sms, smem_per_block,
+                                out.ctypes.data_as(ctypes.c_void_p), g)
+    assert g2 == g
+    return out
 
 
 def tre_plan_inspect(cfg: tre_config, num_sms: int = 148, smem_per_block: int = 232448):
@@ -383,6 +417,19 @@ class Engine:
                                 logits.data_ptr() if logits is not None else 0,
                                 tokens_out.data_ptr() if tokens_out is not None else 0),
               "tre_decode_tokens")
+
+    def decode_loop(self, token: int, pos: int, n_steps: int, tokens_out, logits=None,
+                    stream=None) -> None:
+        """Enqueue n_steps greedy steps (each step's argmax feeds the next on the device);
+        tokens_out: device int32[n_steps]."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        check(tre_decode_loop(self.h, token, pos, n_steps, s, tokens_out.data_ptr(),
+                              logits.data_ptr() if logits is not None else 0), "tre_decode_loop")
+
+    def set_launch_mode(self, mode: int) -> int:
+        """TRE_LAUNCH_PERSISTENT or TRE_LAUNCH_PER_OP; returns launches per step."""
+        return tre_set_launch_mode(self.h, mode)
 
     def layers_step(self, x_in, x_out, pos: int, stream=None) -> None:
         """Enqueue one layers-only step: x_out = stack(x_in) (device fp32[hidden] tensors)."""

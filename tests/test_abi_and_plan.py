@@ -451,3 +451,51 @@ def test_fault_inject_plans_one_unsatisfiable_wait():
     fault_ctr = info.num_counters - 1
     assert (T["dep"] == fault_ctr).sum() == 1
     assert not (T["out"] == fault_ctr).any()
+
+
+@pytest.mark.parametrize("wl,nsm", PLAN_CASES, ids=lambda x: getattr(x, "name", str(x)))
+def test_kernel_per_op_groups(wl, nsm):
+    """The kernel-per-op form (TRE_LAUNCH_PER_OP) runs op group g as launch g: every SM's
+    queue is covered exactly once, in order, by its ranges of the groups; a group holds the
+    tasks of one (layer, type, op); and no task waits on a counter that a task of its own
+    or a later group bumps (each launch starts with every dependency of its tasks met, so a
+    plain launch cannot deadlock)."""
+    cfg = tre.config_from_workload(wl, num_sms=nsm)
+    tasks, begin = tre.tre_plan_tasks(cfg, num_sms=148)
+    ranges = tre.tre_plan_op_groups(cfg, num_sms=148)
+    f = decode_tasks(tasks)
+    G = ranges.shape[0]
+    assert ranges.shape == (G, nsm, 2)
+    group = np.full(len(tasks), -1)
+    for s in range(nsm):
+        at = begin[s]
+        for g in range(G):
+            a, b = ranges[g, s]
+            if a == b:
+                continue
+            assert a == at and b > a, "groups must tile the SM queue in order"
+            group[a:b] = g
+            at = b
+        assert at == begin[s + 1]
+    assert (group >= 0).all()
+    for g in range(G):
+        sel = group == g
+        key = {(int(t), int(o), int(l)) for t, o, l in zip(f["type"][sel], f["op"][sel], f["layer"][sel])}
+        assert len(key) == 1, f"group {g} mixes ops {key}"
+    # the last group that bumps each counter (MoE: shared and routed gate/up both bump the
+    # gate/up counter; the router's last task bumps the layer's route counter)
+    bumped = {}
+    for i in range(len(tasks)):
+        c = int(f["out"][i])
+        if c >= 0:
+            bumped[c] = max(bumped.get(c, -1), group[i])
+    for i in np.nonzero((f["type"] == T_GEMV) & (f["op"] == OP_ROUTER))[0]:
+        c = int(f["layer"][i]) * C_PER_LAYER + C_ROUTE
+        bumped[c] = max(bumped.get(c, -1), group[i])
+    for i in range(len(tasks)):
+        d = int(f["dep"][i])
+        if d >= 0:
+            assert d in bumped and bumped[d] < group[i], f"task {i} waits inside its launch"
+    # launches per step: QKV, attention, O, gate/up, down per GQA layer plus the LM head
+    if wl.kind == "gqa":
+        assert G == 5 * wl.n_layers + (1 if wl.vocab else 0)

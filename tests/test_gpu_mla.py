@@ -41,10 +41,12 @@ def words_to_f64(w):
     return (np.asarray(w, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def run_mla(wl, steps=1, **cfg_over):
+def run_mla(wl, steps=1, mode=None, **cfg_over):
     model = W.gen_mla_model(wl)
     dev = tre.upload_mla_model(model)
     eng = tre.Engine(tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_HIDDEN, **cfg_over), dev)
+    if mode is not None:
+        eng.set_launch_mode(mode)
     caches = [c.copy() for c in model["latent_cache"]]
     x = model["x_in"].astype(np.float64)
     x_dev = torch.empty(wl.hidden, dtype=torch.float32, device="cuda")
@@ -107,3 +109,9 @@ def test_mla_full_size_four_layers():
     rope 64, nope 128, v 128, 4 layers over 8192 cached latent rows, 3 steps with each
     step's input the oracle's output of the previous one."""
     run_mla(W.MLA4.replace(decode_steps=3), steps=3)
+
+
+def test_mla_kernel_per_op_form():
+    """Down-projections, q up-projection, W_uk, attention, W_uv and W_o as separate plain
+    launches."""
+    run_mla(SMALL, steps=2, mode=tre.TRE_LAUNCH_PER_OP)

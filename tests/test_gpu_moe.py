@@ -47,7 +47,7 @@ def check_margin(scores, k):
     assert gaps.size == 0 or gaps.min() > MARGIN, f"routing near-tie (gap {gaps.min():.3g})"
 
 
-def run_moe(wl, steps=1, materialize=True, **cfg_over):
+def run_moe(wl, steps=1, materialize=True, mode=None, **cfg_over):
     """`steps` layer-stack steps from pos = prefill, each step's input the oracle's output
     of the previous one.  materialize=False generates every expert on demand (the full
     workload's 256 experts x 4 layers do not fit host memory at once)."""
@@ -61,6 +61,8 @@ def run_moe(wl, steps=1, materialize=True, **cfg_over):
     dev = tre.upload_moe_model(wl, model, expert_fn=expert)
     cfg = tre.config_from_workload(wl, debug_flags=tre.TRE_DEBUG_HIDDEN, **cfg_over)
     eng = tre.Engine(cfg, dev)
+    if mode is not None:
+        eng.set_launch_mode(mode)
     kc = [c.copy() for c in model["k_cache"]]
     vc = [c.copy() for c in model["v_cache"]]
     x = model["x_in"].astype(np.float64)
@@ -151,3 +153,8 @@ def test_moe_full_size_four_layers():
     heads of dim 128 over 4096 cached positions, 4 layers (~92 GB resident), 3 steps with
     each step's input the oracle's output of the previous one."""
     run_moe(W.MOE4.replace(decode_steps=3), steps=3, materialize=False)
+
+
+def test_moe_kernel_per_op_form():
+    """Router, shared and routed gate/up, expert down as separate plain launches."""
+    run_moe(SMALL, steps=2, mode=tre.TRE_LAUNCH_PER_OP)
