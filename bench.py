@@ -598,7 +598,8 @@ def run_engine(args, rank, world, local_rank):
     torch.cuda.empty_cache()
 
     if trace_path:
-        write_trace(wl, local_rank, trace_path, args.flags, config_overrides(args.config))
+        write_trace(wl, local_rank, trace_path, args.flags, config_overrides(args.config),
+                    per_op=args.launch_mode == "per-op")
 
     dev_s, e2e_s, launch_ms_avg = max_over_ranks(
         [dev_s, e2e_s, float(np.mean(launch_ms))], world, f"cuda:{local_rank}")
@@ -657,6 +658,7 @@ def ablation(eng, wl, tokens, positions, Wm, K, stream, local_rank, barrier):
     del graphs
     st = eng.status()
     assert st == (0, 0), st
+    # per-op steps (direct or replayed) leave the persistent form's counters untouched
     eng.set_launch_mode(tre.TRE_LAUNCH_PERSISTENT)
     for i in range(3):
         eng.step(tokens[Wm + i][0], positions[Wm + i], stream=s_ptr)
@@ -678,9 +680,10 @@ def ablation(eng, wl, tokens, positions, Wm, K, stream, local_rank, barrier):
     return out
 
 
-def write_trace(wl, device, path, flags=0, overrides=None):
+def write_trace(wl, device, path, flags=0, overrides=None, per_op=False):
     """Three traced steps on a fresh engine (debug flag): per-task start / ready / end of
-    the last one, with the plan and its summary.  Steps take the workload's tokens per step."""
+    the last one, with the plan and its summary.  Steps take the workload's tokens per step;
+    per_op: the kernel-per-op launch form."""
     import torch
 
     from persistent_tile_pipelined_b200 import trace as trace_mod
@@ -688,6 +691,8 @@ def write_trace(wl, device, path, flags=0, overrides=None):
     M = max(1, wl.tokens_per_step)
     eng, model = build_engine(wl.replace(decode_steps=3 * M), device, tre.TRE_DEBUG_TRACE | flags,
                               overrides)
+    if per_op:
+        eng.set_launch_mode(tre.TRE_LAUNCH_PER_OP)
     for i in range(3):
         if M > 1:
             eng.step_tokens([1 + i * M + v for v in range(M)], wl.prefill + i * M)

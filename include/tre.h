@@ -280,7 +280,11 @@ tre_status tre_decode_loop(tre_engine* e, int32_t token, int32_t pos, int32_t n_
  * one layer's op: QKV, attention, O, gate/up, down, ...; ~9 per layer plus the LM head),
  * each launch starting after the previous one has finished.  PER_OP exists to measure
  * what the persistent form removes (the launch cost and the drain / ramp at every op
- * boundary that [SC] §6 names); it computes the same results. */
+ * boundary that [SC] §6 names); it computes the same results.
+ * Stream capture: PER_OP steps may be captured in a CUDA graph and replayed (their
+ * launches wait on nothing but stream order); a PERSISTENT step returns
+ * TRE_ERR_UNSUPPORTED on a capturing stream (it waits for a new epoch of its dependency
+ * counters, which a replay would not have). */
 enum { TRE_LAUNCH_PERSISTENT = 0, TRE_LAUNCH_PER_OP = 1 };
 
 /* Set the launch mode of every later step call on `e`.  *launches_per_step (may be NULL)

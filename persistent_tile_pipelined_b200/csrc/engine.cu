@@ -48,8 +48,10 @@ constexpr long long kCheckCycles = 1 << 15;
 constexpr int kLoadBatch = 2;
 
 // Wait until counter `idx` reaches epoch * count (wrap-safe).  Bounded; on expiry the
-// error names `detail` (a task index).
+// error names `detail` (a task index).  A kernel-per-op launch never waits: the launches
+// before it in the stream met every dependency of its tasks.
 __device__ bool wait_counter(const Params& p, int idx, uint32_t count, int detail) {
+  if (p.op_group >= 0) return true;
   const uint32_t target = p.epoch * count;
   const uint32_t* c = p.counters + idx;
   if ((int32_t)(ld_acquire_gpu(c) - target) >= 0) return true;

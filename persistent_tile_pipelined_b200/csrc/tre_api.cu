@@ -41,6 +41,7 @@ struct tre_engine {
   int last_m = 1;                // tokens of the last step (debug hidden layout)
   float* logits_buf = nullptr;
   int n_groups = 0;              // op groups of the plan (kernel-per-op form)
+  uint32_t* op_counters = nullptr;  // counters the kernel-per-op launches bump
   int launch_mode = TRE_LAUNCH_PERSISTENT;
 };
 
@@ -314,6 +315,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_ranges = cv.take<int32_t>(ranges.size());
   size_t o_layers = cv.take<LayerPtrs>(s.L);
   size_t o_ctr = cv.take<uint32_t>(s.n_counters);
+  size_t o_ctr_op = cv.take<uint32_t>(s.n_counters);  // bumped by kernel-per-op launches only
   size_t o_tick = cv.take<uint32_t>(std::max(s.Hkv, mla ? s.Hq / kMlaHeadGroup : 1));
   size_t o_lmt = cv.take<uint32_t>(1);
   size_t o_arg = cv.take<unsigned long long>(kMaxTokens);
@@ -402,6 +404,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.op_group = -1;
   p.token_in = nullptr;
   p.counters = reinterpret_cast<uint32_t*>(B + o_ctr);
+  e->op_counters = reinterpret_cast<uint32_t*>(B + o_ctr_op);
   p.tickets = reinterpret_cast<uint32_t*>(B + o_tick);
   p.lm_ticket = reinterpret_cast<uint32_t*>(B + o_lmt);
   p.argmax_slot = reinterpret_cast<unsigned long long*>(B + o_arg);
@@ -481,20 +484,33 @@ static tre_status launch_step(tre_engine* e, const int32_t* tokens, int m, int32
     return TRE_ERR_POS_RANGE;
   }
   CK(cudaSetDevice(e->device));
+  const bool per_op = e->launch_mode == TRE_LAUNCH_PER_OP;
+  if (!per_op) {
+    // A persistent step waits for its counters to reach epoch * count; a replayed capture
+    // would carry a stale epoch and not wait at all, so it is refused.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    CK(cudaStreamIsCapturing(stream, &cap));
+    if (cap != cudaStreamCaptureStatusNone) {
+      set_error("a persistent step cannot be captured in a CUDA graph (each step waits for a "
+                "new epoch of its counters); capture TRE_LAUNCH_PER_OP steps instead");
+      return TRE_ERR_UNSUPPORTED;
+    }
+  }
   Params p = e->base;
   p.m = m;
   for (int v = 0; v < kMaxTokens; ++v) p.tokens[v] = v < m ? tokens[v] : tokens[0];
   p.token = tokens[0];
   p.token_in = token_in;
   p.pos = pos;
-  p.epoch = ++e->epoch;
+  p.epoch = per_op ? e->epoch : ++e->epoch;
+  if (per_op) p.counters = e->op_counters;
   if (logits_dev) p.logits = logits_dev;
   p.token_out = token_dev ? token_dev : e->token_buf;
   p.x_in = x_in;
   p.x_out = x_out;
   const bool mla = e->shape.kind == TRE_LAYER_MLA;
   cudaError_t ce = cudaSuccess;
-  if (e->launch_mode == TRE_LAUNCH_PER_OP) {
+  if (per_op) {
     for (int g = 0; g < e->n_groups && ce == cudaSuccess; ++g) {
       p.op_group = g;
       ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream, mla);
@@ -503,7 +519,7 @@ static tre_status launch_step(tre_engine* e, const int32_t* tokens, int m, int32
     ce = engine_launch(p, e->shape.nsm, e->shape.smem_bytes, stream, mla);
   }
   if (ce != cudaSuccess) {
-    --e->epoch;
+    if (!per_op) --e->epoch;
     return cuda_fail(ce, "launch of the engine kernel");
   }
   e->last_m = m;
@@ -695,6 +711,7 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
   CK(cudaDeviceSynchronize());
   const Params& p = e->base;
   CK(cudaMemsetAsync(p.counters, 0, (size_t)e->shape.n_counters * 4, s));
+  CK(cudaMemsetAsync(e->op_counters, 0, (size_t)e->shape.n_counters * 4, s));
   CK(cudaMemsetAsync(p.tickets, 0,
                      (size_t)std::max(e->shape.Hkv, e->shape.kind == TRE_LAYER_MLA
                                                         ? e->shape.Hq / kMlaHeadGroup : 1) * 4,

@@ -148,7 +148,9 @@ struct Params {
   // Kernel-per-op launches (the measurement form with the kernel boundary put back): this
   // launch runs op group `op_group` only, CTA b the tasks [op_ranges[2 (g nsm + b)],
   // op_ranges[2 (g nsm + b) + 1]) of p.tasks; op_group < 0: the whole step (the
-  // persistent form).
+  // persistent form).  Per-op launches wait on no counter (stream order meets every
+  // dependency) and bump a counter array of their own, so that the persistent form's
+  // counters always stand at epoch * count between steps.
   const int32_t* op_ranges;
   int op_group;
   uint32_t* counters;

@@ -74,7 +74,25 @@ def summarize(trace: np.ndarray, tasks: np.ndarray) -> dict:
                 d[1] += b - a          # stages consumed
                 d[2] += e - (c if c else b)   # tail: epilogue, ticket, combine, publish
                 d[3] += 1
+    # op boundaries, in global task order (the op groups of the kernel-per-op form): the
+    # hand-off from the last task of one op to the first task of the next one to start
+    # computing (dependency met) — a launch boundary in the kernel-per-op form, a counter
+    # publish and wake-up in the persistent form
+    ids = np.arange(len(trace))
+    key = np.stack([tt["layer"], tt["type"], tt["op"]], axis=1)
+    new_group = np.ones(len(ids), dtype=bool)
+    new_group[1:] = (key[1:] != key[:-1]).any(axis=1)
+    gid = np.cumsum(new_group) - 1
+    G = int(gid.max()) + 1
+    g_end = np.full(G, -np.inf)
+    g_ready = np.full(G, np.inf)
+    np.maximum.at(g_end, gid, end.astype(np.float64))
+    np.minimum.at(g_ready, gid, ready.astype(np.float64))
+    gaps = g_ready[1:] - g_end[:-1]
     return {
+        "op_groups": G,
+        "op_gap_us": {"mean": float(np.mean(gaps)) / 1e3, "median": float(np.median(gaps)) / 1e3,
+                      "sum": float(np.sum(np.maximum(gaps, 0))) / 1e3},
         "phases_us": {k: {"prep": v[0] / v[3] / 1e3, "stages": v[1] / v[3] / 1e3,
                           "tail": v[2] / v[3] / 1e3} for k, v in phases.items() if v[3]},
         "step_us": step_ns / 1e3,

@@ -342,3 +342,49 @@ def test_engines_with_different_shared_memory_coexist():
     assert torch.equal(la, lb)  # the ring depth does not change any sum
     big.close()
     small.close()
+
+
+def test_graph_replays_of_per_op_steps_leave_persistent_steps_correct():
+    """Kernel-per-op steps may be captured and replayed (they wait on nothing but stream
+    order); replays must not disturb the counters the persistent form waits on, so
+    persistent steps afterwards still match the oracle.  A persistent step refuses
+    capture (a replay would carry a stale epoch and not wait)."""
+    wl = W.TINY
+    model = W.gen_gqa_model(wl)
+    dev = tre.upload_gqa_model(model)
+    eng = tre.Engine(tre.config_from_workload(wl), dev)
+    tok, pos = W.first_token(wl), wl.prefill
+    logits = torch.empty(wl.vocab, dtype=torch.float32, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    x = torch.zeros(1, device="cuda")
+    with torch.cuda.stream(side):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            x.add_(1.0)
+            st = tre.tre_decode_step(eng.h, tok, pos, side.cuda_stream)
+        assert st == tre.TRE_ERR_UNSUPPORTED
+        eng.set_launch_mode(tre.TRE_LAUNCH_PER_OP)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            eng.step(tok, pos, logits, stream=side.cuda_stream)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    ref, _ = ORC.decode_step(wl, model, tok, pos, want_hidden=False)
+    assert relerr(logits.cpu().numpy(), ref) <= REG_TOL
+    del g
+    eng.set_launch_mode(tre.TRE_LAUNCH_PERSISTENT)
+    # the oracle has appended pos already; continue both from pos + 1
+    tok_dev = torch.empty(1, dtype=torch.int32, device="cuda")
+    tok = ORC.argmax(ref)
+    for step in range(3):
+        eng.step(tok, pos + 1 + step, logits, tok_dev)
+        torch.cuda.synchronize()
+        assert eng.status() == (0, 0)
+        ref, _ = ORC.decode_step(wl, model, tok, pos + 1 + step, want_hidden=False)
+        e = relerr(logits.cpu().numpy(), ref)
+        assert e <= TOL and e <= REG_TOL, f"logits rel err {e:.3g} after per-op graph replays"
+        tok = ORC.argmax(ref)
+    eng.close()
