@@ -68,6 +68,9 @@ def parse():
     ap.add_argument("--launch-mode", default="persistent", choices=["persistent", "per-op"],
                     help="persistent: one launch per step (the product); per-op: the same "
                          "tiles, one plain launch per op (measurement form)")
+    ap.add_argument("--wl", action="append", default=[], metavar="FIELD=VALUE",
+                    help="workload shape override (e.g. n_layers=1, n_experts=16: a small "
+                         "case of the same kernel for profiler captures); repeatable")
     ap.add_argument("--no-ablation", action="store_true",
                     help="skip the kernel-per-op comparison and the device-loop timing")
     return ap.parse_args()
@@ -194,6 +197,17 @@ def job_throughput(world: int, steps: int, tokens_per_step: int, slowest_s: floa
     return world * steps * tokens_per_step / slowest_s
 
 
+def workload_of(args):
+    """The named workload with the --wl shape overrides applied (renamed to show them)."""
+    from persistent_tile_pipelined_b200.synth import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    over = config_overrides(args.wl)
+    if over:
+        wl = wl.replace(name=wl.name + "".join(f",{k}={v}" for k, v in sorted(over.items())),
+                        **over)
+    return wl
+
+
 def config_overrides(items):
     """FIELD=VALUE strings -> {field: int}."""
     out = {}
@@ -266,7 +280,7 @@ def run_layers(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     K, Wm = args.steps, args.warmup
-    wl = W.WORKLOADS[args.workload].replace(decode_steps=K + Wm)
+    wl = workload_of(args).replace(decode_steps=K + Wm)
     wl = wl.replace(seed=wl.seed + rank)
     eng, dmodel = build_layers_engine(wl, local_rank, args.flags, config_overrides(args.config))
     stream = torch.cuda.current_stream(local_rank)
@@ -519,7 +533,7 @@ def run_engine(args, rank, world, local_rank):
     from persistent_tile_pipelined_b200.synth import workloads as W
 
     torch.cuda.set_device(local_rank)
-    wl = W.WORKLOADS[args.workload]
+    wl = workload_of(args)
     K, Wm, M = args.steps, args.warmup, args.tokens_per_step
     wl = wl.replace(decode_steps=K + Wm, tokens_per_step=M, seed=wl.seed + rank)
     eng, model = build_engine(wl, local_rank, args.flags, config_overrides(args.config))
@@ -727,7 +741,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device(f"cuda:{local_rank}"))
     from persistent_tile_pipelined_b200.synth import workloads as W
-    if W.WORKLOADS[args.workload].kind != "gqa":
+    if workload_of(args).kind != "gqa":
         return main_layers(args, rank, world, local_rank)
     wl, dev_s, e2e_s, launch_ms, step_bytes, clocks, abl = run_engine(args, rank, world,
                                                                       local_rank)
@@ -842,7 +856,7 @@ def main_reference(args, rank, world):
         return
     from persistent_tile_pipelined_b200.synth import workloads as W
     K, Wm, M = args.steps, args.warmup, args.tokens_per_step
-    wl = W.WORKLOADS[args.workload].replace(decode_steps=K + Wm)
+    wl = workload_of(args).replace(decode_steps=K + Wm)
     budget = REFERENCE_SECONDS / max(1, K + Wm)  # seconds of oracle work per step
     if wl.kind == "gqa":
         wl = wl.replace(tokens_per_step=M)

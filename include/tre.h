@@ -328,8 +328,8 @@ tre_status tre_debug_hidden(tre_engine* e, float* hidden_dev, tre_stream stream)
 /* Copy the per-task trace of the last step to host memory: 8 int64 per task, in global
  * task order: start ns (dependency wait begins), dependency met ns, end ns, SM id, then
  * phase marks — GEMV: input vector staged, last stage consumed; attention: q ready,
- * stages consumed, partial written (and ticket taken); MLA attention also: ns spent
- * waiting for stages to land — (0 where a mark does not apply).
+ * stages consumed, partial written and published, ns spent waiting for stages to land
+ * (0 where a mark does not apply).
  * Requires TRE_DEBUG_TRACE.  *n_tasks receives the task count; trace_host may be NULL to
  * query. */
 tre_status tre_debug_trace(tre_engine* e, int64_t* trace_host, int32_t* n_tasks);

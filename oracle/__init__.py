@@ -40,16 +40,19 @@ class _GqaConfig(ctypes.Structure):
                 ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("ffn", ctypes.c_int32),
                 ("vocab", ctypes.c_int32), ("kv_capacity", ctypes.c_int32),
-                ("rope_theta", ctypes.c_double), ("norm_eps", ctypes.c_double)]
+                ("rope_theta", ctypes.c_double), ("norm_eps", ctypes.c_double),
+                ("weight_fp8", ctypes.c_int32)]
 
 
 class _GqaLayer(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "wgate", "wup", "wdown",
-                 "k_cache", "v_cache")]
+                 "k_cache", "v_cache", "sq", "sk", "sv", "so", "sgate", "sup", "sdown")]
 
 
 _SLOT_NAMES = ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "wgate", "wup", "wdown")
+# FP8 layers: the block scales of the seven projection matrices sit in slots 9 .. 15
+_SCALE_SLOTS = {"sq": 9, "sk": 10, "sv": 11, "so": 12, "sgate": 13, "sup": 14, "sdown": 15}
 
 
 class _MlaConfig(ctypes.Structure):
@@ -85,6 +88,9 @@ class Oracle:
         assert L.orc_real_bytes() == bits // 8
         L.orc_bf16_to_real.argtypes = [ctypes.c_uint16]
         L.orc_bf16_to_real.restype = creal
+        L.orc_e4m3_to_real.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_to_real.restype = creal
+        L.orc_gemv_fp8.argtypes = [i32, i32, vp, vp, vp, vp]
         L.orc_round_bf16.argtypes = [creal]
         L.orc_round_bf16.restype = ctypes.c_uint16
         L.orc_rmsnorm.argtypes = [i32, vp, vp, dbl, vp]
@@ -112,6 +118,20 @@ class Oracle:
 
     def bf16_to_real(self, w: int) -> float:
         return float(self.lib.orc_bf16_to_real(w))
+
+    def e4m3_to_real(self, b: int) -> float:
+        return float(self.lib.orc_e4m3_to_real(b))
+
+    def gemv_fp8(self, W_e4m3, S, x):
+        """y = (e4m3(W) * S[n / 128][k / 128]) x for W [N][K] bytes, S fp32 block scales."""
+        W = np.ascontiguousarray(W_e4m3, dtype=np.uint8)
+        S = np.ascontiguousarray(S, dtype=np.float32)
+        x = self._r(x)
+        N, K = W.shape
+        assert x.size == K and S.shape == ((N + 127) // 128, (K + 127) // 128)
+        y = np.empty(N, dtype=self.real)
+        self.lib.orc_gemv_fp8(N, K, _ptr(W), _ptr(S), _ptr(x), _ptr(y))
+        return y
 
     def rmsnorm(self, x, g_bf16, eps):
         x = self._r(x)
@@ -157,14 +177,18 @@ class Oracle:
 
     # -- the stack ---------------------------------------------------------------
     def _gqa_structs(self, wl, model):
+        fp8 = getattr(wl, "weight_format", "bf16") == "fp8"
         cfg = _GqaConfig(wl.n_layers, wl.hidden, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
                          wl.ffn, wl.vocab, wl.kv_capacity, float(wl.rope_theta),
-                         float(wl.norm_eps))
+                         float(wl.norm_eps), 1 if fp8 else 0)
         layers = (_GqaLayer * wl.n_layers)()
         for l in range(wl.n_layers):
             t = model["layers"][l]
             for slot, name in enumerate(_SLOT_NAMES):
                 setattr(layers[l], name, _ptr(t[slot]).value)
+            if fp8:
+                for name, slot in _SCALE_SLOTS.items():
+                    setattr(layers[l], name, _ptr(t[slot]).value)
             layers[l].k_cache = _ptr(model["k_cache"][l]).value
             layers[l].v_cache = _ptr(model["v_cache"][l]).value
         return cfg, layers

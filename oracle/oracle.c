@@ -23,7 +23,13 @@
  * current token are rounded to bf16 when appended to the cache and read back from it;
  * every other value stays in `real`.
  *
+ * FP8 weights (optional, the seven projection matrices of a GQA layer): E4M3 bytes with
+ * one fp32 scale per 128 x 128 block, decoded from the format's definition and multiplied
+ * by the block's scale; activations stay in `real`.
+ *
  * Pins (tests/test_oracle_pins.py): bf16 rounding vs torch and vs the two neighbours;
+ * E4M3 decoding of all 256 bytes vs torch and vs the format's closed values; the FP8
+ * matrix-vector product vs numpy on the decoded, scaled matrix;
  * RMSNorm unit RMS; matrix-vector vs numpy matmul; RoPE identity at pos 0, norm
  * preservation, relative-position property and the complex-rotation form; attention
  * brute force in pure Python, one position returns V, equal keys return the mean of V,
@@ -97,6 +103,34 @@ void orc_gemv(int N, int K, const uint16_t* W, const real* x, real* y) {
   }
 }
 
+/* FP8 E4M3 (the OCP 8-bit floating-point format with 4 exponent bits, bias 7, and 3
+ * mantissa bits; no infinities, S.1111.111 is NaN) byte -> value.  Exponent field 0 holds
+ * the subnormals m/8 * 2^-6; otherwise the value is (1 + m/8) * 2^(e - 7). */
+real orc_e4m3_to_real(uint8_t b) {
+  int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+  double v;
+  if (e == 15 && m == 7) return (real)NAN;
+  if (e == 0) v = ldexp((double)m / 8.0, -6);
+  else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+  return (real)(sgn ? -v : v);
+}
+
+/* y = W x with W [N][K] stored as E4M3 bytes and block scales S[ceil(N/128)][ceil(K/128)]
+ * (fp32): element W[n][k] stands for e4m3(W[n][k]) * S[n / 128][k / 128] — the block-scaled
+ * FP8 weight layout (128 x 128 blocks) of DeepSeek-V3-style checkpoints, which the pages'
+ * fused "RMSNorm + QKV + FP8 dequant" op consumes (TileRT code audit, fused-op list). */
+void orc_gemv_fp8(int N, int K, const uint8_t* W, const float* S, const real* x, real* y) {
+  int KB = (K + 127) / 128;
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n) {
+    const uint8_t* row = W + (size_t)n * K;
+    const float* srow = S + (size_t)(n / 128) * KB;
+    real acc = 0;
+    for (int k = 0; k < K; ++k) acc += orc_e4m3_to_real(row[k]) * (real)srow[k / 128] * x[k];
+    y[n] = acc;
+  }
+}
+
 /* Half-split rotary embedding of one head vector v[D] at position pos: the pair
  * (v[i], v[i + D/2]) is rotated by the angle pos * theta^(-2i/D). */
 void orc_rope(int D, int pos, double theta, real* v) {
@@ -161,12 +195,23 @@ int orc_argmax(int n, const real* v) {
 typedef struct {
   int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab, kv_capacity;
   double rope_theta, norm_eps;
+  int32_t weight_fp8;  /* 1: the seven projection matrices are E4M3 with block scales */
 } orc_gqa_config;
 
 typedef struct {
   const uint16_t *attn_norm, *wq, *wk, *wv, *wo, *ffn_norm, *wgate, *wup, *wdown;
   uint16_t *k_cache, *v_cache; /* [Hkv][cap][D] bf16, written at pos */
+  /* weight_fp8: the block scales of wq, wk, wv, wo, wgate, wup, wdown (whose pointers then
+   * address E4M3 bytes) */
+  const float *sq, *sk, *sv, *so, *sgate, *sup, *sdown;
 } orc_gqa_layer;
+
+/* A projection of the stack: bf16 weights, or E4M3 bytes with block scales. */
+static void layer_gemv(const orc_gqa_config* c, int N, int K, const uint16_t* W, const float* S,
+                       const real* x, real* y) {
+  if (c->weight_fp8) orc_gemv_fp8(N, K, (const uint8_t*)W, S, x, y);
+  else orc_gemv(N, K, W, x, y);
+}
 
 /* The attention block of a pre-norm GQA layer at position pos:
  *   xn = RMSNorm(x); q,k,v = Wq xn, Wk xn, Wv xn; RoPE(q, k at pos);
@@ -183,9 +228,9 @@ void orc_gqa_attn_block(const orc_gqa_config* c, const orc_gqa_layer* L, int pos
   real* o = (real*)malloc(sizeof(real) * (size_t)Hq * D);
   real* y = (real*)malloc(sizeof(real) * d);
   orc_rmsnorm(d, x, L->attn_norm, c->norm_eps, xn);
-  orc_gemv(Hq * D, d, L->wq, xn, q);
-  orc_gemv(Hkv * D, d, L->wk, xn, k);
-  orc_gemv(Hkv * D, d, L->wv, xn, v);
+  layer_gemv(c, Hq * D, d, L->wq, L->sq, xn, q);
+  layer_gemv(c, Hkv * D, d, L->wk, L->sk, xn, k);
+  layer_gemv(c, Hkv * D, d, L->wv, L->sv, xn, v);
   for (int h = 0; h < Hq; ++h) orc_rope(D, pos, c->rope_theta, q + (size_t)h * D);
   for (int h = 0; h < Hkv; ++h) orc_rope(D, pos, c->rope_theta, k + (size_t)h * D);
   for (int h = 0; h < Hkv; ++h)
@@ -194,7 +239,7 @@ void orc_gqa_attn_block(const orc_gqa_config* c, const orc_gqa_layer* L, int pos
       L->v_cache[((size_t)h * cap + pos) * D + i] = orc_round_bf16(v[(size_t)h * D + i]);
     }
   orc_attention(Hq, Hkv, D, pos + 1, cap, q, L->k_cache, L->v_cache, o, NULL);
-  orc_gemv(d, Hq * D, L->wo, o, y);
+  layer_gemv(c, d, Hq * D, L->wo, L->so, o, y);
   for (int i = 0; i < d; ++i) h1[i] = x[i] + y[i];
   free(xn); free(q); free(k); free(v); free(o); free(y);
 }
@@ -222,7 +267,19 @@ void orc_gqa_layer_step(const orc_gqa_config* c, const orc_gqa_layer* L, int pos
   real* y = (real*)malloc(sizeof(real) * d);
   orc_gqa_attn_block(c, L, pos, x, h1);
   orc_rmsnorm(d, h1, L->ffn_norm, c->norm_eps, hn);
-  orc_swiglu_mlp(d, c->ffn, L->wgate, L->wup, L->wdown, hn, y);
+  if (c->weight_fp8) {
+    int F = c->ffn;
+    real* g = (real*)malloc(sizeof(real) * F);
+    real* u = (real*)malloc(sizeof(real) * F);
+    orc_gemv_fp8(F, d, (const uint8_t*)L->wgate, L->sgate, hn, g);
+    orc_gemv_fp8(F, d, (const uint8_t*)L->wup, L->sup, hn, u);
+    for (int i = 0; i < F; ++i) g[i] = orc_silu(g[i]) * u[i];
+    orc_gemv_fp8(d, F, (const uint8_t*)L->wdown, L->sdown, g, y);
+    free(g);
+    free(u);
+  } else {
+    orc_swiglu_mlp(d, c->ffn, L->wgate, L->wup, L->wdown, hn, y);
+  }
   for (int i = 0; i < d; ++i) x[i] = h1[i] + y[i];
   free(h1); free(hn); free(y);
 }

@@ -261,10 +261,20 @@ __device__ __forceinline__ const uint16_t* part_row(const Params& p, const Task&
   }
 }
 
+// Cached positions [t0, t1) of split t.r1 of t.aux over [0, pos) (the new positions come
+// from qkv).  GQA: the last split also RoPEs and appends this step's K / V rows and scores
+// them, so it takes half a share of the cached positions (boundaries at 2 s P / (2 S - 1))
+// and the splits finish together.  MLA: equal shares.
 __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& t0, int& t1) {
-  const long long P = p.pos;  // cached positions [0, pos); the new one comes from qkv
-  t0 = (int)(P * t.r1 / t.aux);
-  t1 = (int)(P * (t.r1 + 1) / t.aux);
+  const long long P = p.pos;
+  const long long S = t.aux, sp = t.r1;
+  if (t.type == T_ATTN) {
+    t0 = (int)(P * 2 * sp / (2 * S - 1));
+    t1 = sp + 1 == S ? (int)P : (int)(P * 2 * (sp + 1) / (2 * S - 1));
+    return;
+  }
+  t0 = (int)(P * sp / S);
+  t1 = (int)(P * (sp + 1) / S);
 }
 
 template <bool TILED>
@@ -663,6 +673,79 @@ __device__ __forceinline__ int input_key(const Task& t) {
   return (((int)t.layer * 8 + cls) << 8) | part;
 }
 
+// The O-projection input of each of the MT tokens: the attention output, combined from
+// the KV splits' partials on the way in (the fused combine): for head h,
+// attn_h = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s (splits that saw
+// no position have m_s = -inf and weigh 0).  (1) every split's (m, l) of the K-part's heads
+// in one round trip, one warp per (token, head), lanes over the splits, turned into split
+// weights with shuffles; (2) each thread merges 8-column groups, fetching every split's
+// values before it sums them.  Written as planes, or (FRAG) as the tensor-core B operand,
+// like load_input.
+template <int MT, bool FRAG>
+__device__ void stage_attn_merged(const Params& p, const GemvGeom& gg, float* ub, float* wsc,
+                                  int ctid) {
+  const int D = p.D, S = p.nsplit, pst = D + 2;
+  const int h0 = gg.k0 / D, nh = (gg.k0 + gg.Kp - 1) / D - h0 + 1;
+  float* wm = wsc;                   // [MT][nh][S]: the split weights 2^(m_s - M)
+  float* inv = wsc + MT * nh * S;    // [MT][nh]: 1 / sum_s w_s l_s
+  const int warp = ctid >> 5, lane = ctid & 31;
+  for (int vh = warp; vh < MT * nh; vh += kConsumerWarps) {
+    const int v = vh / nh, h = h0 + vh % nh;
+    const float* ml = p.part + (size_t)(v * p.Hq + h) * S * pst + D;
+    float M = -INFINITY;
+    for (int sp = lane; sp < S; sp += 32) M = fmaxf(M, __ldcg(ml + (size_t)sp * pst));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    for (int sp = lane; sp < S; sp += 32) {
+      const float2 x = __ldcg(reinterpret_cast<const float2*>(ml + (size_t)sp * pst));
+      const float w = x.x == -INFINITY ? 0.f : exp2f(x.x - M);
+      L = fmaf(w, x.y, L);
+      wm[vh * S + sp] = w;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0) inv[vh] = 1.f / L;
+  }
+  consumer_sync(kConsumerThreads);
+  const int K8 = gg.Kp >> 3;
+  for (int it = ctid; it < MT * K8; it += kConsumerThreads) {
+    const int v = FRAG ? it % MT : it / K8, j = FRAG ? it / MT : it % K8;
+    const int k = gg.k0 + 8 * j, h = k / D, dd = k - h * D, vh = v * nh + (h - h0);
+    const float* src = p.part + (size_t)(v * p.Hq + h) * S * pst + dd;
+    const float* w = wm + vh * S;
+    float e[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 6
+    for (int sp = 0; sp < S; ++sp) {
+      const float ws = w[sp];
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(src + (size_t)sp * pst));
+      const float4 b = __ldcg(reinterpret_cast<const float4*>(src + (size_t)sp * pst + 4));
+      e[0] = fmaf(ws, a.x, e[0]); e[1] = fmaf(ws, a.y, e[1]); e[2] = fmaf(ws, a.z, e[2]);
+      e[3] = fmaf(ws, a.w, e[3]); e[4] = fmaf(ws, b.x, e[4]); e[5] = fmaf(ws, b.y, e[5]);
+      e[6] = fmaf(ws, b.z, e[6]); e[7] = fmaf(ws, b.w, e[7]);
+    }
+    const float r = inv[vh];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) e[q] *= r;
+    if constexpr (FRAG) {
+      uint32_t* fr = reinterpret_cast<uint32_t*>(ub) + 2 * (8 * MT * (j >> 1)) + (j & 1);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hi, lo;
+        split_pair(e[2 * q], e[2 * q + 1], hi, lo);
+        fr[2 * (v * 4 + q)] = hi;
+        fr[2 * ((MT + v) * 4 + q)] = lo;
+      }
+    } else {
+      float* xlo = ub + (size_t)v * gg.Kp;
+      float* xhi = xlo + gg.Kp / 2;
+      reinterpret_cast<float4*>(xlo)[j] = make_float4(e[0], e[1], e[2], e[3]);
+      reinterpret_cast<float4*>(xhi)[j] = make_float4(e[4], e[5], e[6], e[7]);
+    }
+  }
+  consumer_sync(kConsumerThreads);
+}
+
 // Stage the GEMV input of each of the MT tokens into its two planes (token v's at
 // ub + v Kp); rn[v] receives token v's RMSNorm scale (1 when the op has no norm).
 // FRAG (tensor-core tiles): the inputs are written as the mma B operand instead, split
@@ -835,10 +918,10 @@ __device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float&
 
 // One split of the split-KV decode attention for kv head g = t.r0 (split t.r1 of t.aux):
 // the G query heads of the group attend to cached positions [t0, t1) streamed through the
-// ring (every warp takes 8 positions of every stage); the last split also takes the new
-// position pos from this step's k / v, appends them to the caches and merges its partial.
-// The last split of the group to finish (arrival ticket) combines all splits — the fused
-// combine — and publishes the group.
+// ring; the last split also takes the new position pos from this step's k / v, appends
+// them to the caches and merges its partial.  Every split writes its partial (m, l, O) and
+// publishes; the O-projection tasks combine the splits while they stage their input
+// (stage_attn_merged), so the combine costs no extra hand-off.
 template <int G, int D, int MT>
 __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
                           uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
@@ -951,12 +1034,15 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   int t0, t1;
   attn_range(p, t, t0, t1);
   const int grp = warp >> 2, r0 = (warp & 3) * 16;
+  long long waited = 0;  // trace: ns thread 0 spent waiting for its stages to land
   for (int i = grp; i < ns; i += 2) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
+    const long long w0 = (p.trace && ctid == 0) ? (long long)globaltimer_ns() : 0;
     if (!stage_wait(p, full, tags, sidx)) {
       abort_out = true;
       break;
     }
+    if (p.trace && ctid == 0) waited += (long long)globaltimer_ns() - w0;
     const int valid = min(16, t1 - (t0 + i * p.pps) - r0);
     if (valid > 0) {
       const uint32_t tb = smem_u32(ring + (size_t)slot * p.stage_bytes);
@@ -1078,7 +1164,10 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     }
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
+  if (ctid == 0 && p.trace) {
+    p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
+    p.trace[(size_t)t.id * kTraceCols + 7] = waited;
+  }
 
   // merge the warps (and, in the last split, the new positions) into this split's partial
   const size_t pstride = (size_t)D + 2;
@@ -1117,50 +1206,9 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     }
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) {
-    const uint32_t old = ticket_add(p.tickets + g, 1u);
-    *flag = ((old + 1u) % (uint32_t)S) == 0u;
+  if (ctid == 0) {  // the O-projection merges the splits while it stages its input
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
-  }
-  consumer_sync(kConsumerThreads);
-  if (*flag) {  // last split of this kv head to finish: combine all splits
-    // (m, l) of every split into shared memory in one round trip (reuses the warp scratch)
-    float* ms = ow;
-    float* ls = ow + ROWS * S;
-    for (int idx = ctid; idx < ROWS * S; idx += kConsumerThreads) {
-      const int r = idx / S, s2 = idx % S, v = r / G, h = r % G;
-      const float* src = p.part + ((size_t)(v * p.Hq + g * G + h) * S + s2) * pstride;
-      ms[idx] = __ldcg(src + D);
-      ls[idx] = __ldcg(src + D + 1);
-    }
-    consumer_sync(kConsumerThreads);
-    if (ctid < ROWS) {  // per row: the splits' weights 2^(m_s - M) and 1 / sum_s w_s l_s
-      float* mh = ms + ctid * S;
-      float* lh = ls + ctid * S;
-      float M = -INFINITY;
-      for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mh[s2]);
-      float Ls = 0.f;
-      for (int s2 = 0; s2 < S; ++s2) {
-        const float w = mh[s2] == -INFINITY ? 0.f : exp2f(mh[s2] - M);
-        mh[s2] = w;
-        Ls = fmaf(w, lh[s2], Ls);
-      }
-      lh[0] = 1.f / Ls;
-    }
-    consumer_sync(kConsumerThreads);
-    for (int idx = ctid; idx < ROWS * D; idx += kConsumerThreads) {
-      const int r = idx / D, dd = idx % D, v = r / G, h = r % G;
-      const float* wh = ms + r * S;
-      const size_t q = (size_t)v * p.Hq + g * G + h;
-      const float* src = p.part + q * S * pstride + dd;
-      // independent loads: the splits' outputs are fetched together, not one at a time
-      float O = 0.f;
-#pragma unroll 16
-      for (int s2 = 0; s2 < S; ++s2) O = fmaf(wh[s2], __ldcg(src + s2 * pstride), O);
-      p.attn[q * D + dd] = O * ls[r * S];
-    }
-    consumer_sync(kConsumerThreads);
-    if (ctid == 0) publish_add(p.counters + t.out, 1u);
+    publish_add(p.counters + t.out, 1u);
   }
 }
 
@@ -1849,6 +1897,13 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       if (MLA && t.op == OP_UV) {
         if constexpr (MLA) mla_combine_input(p, t, ub, ub + p.xs_floats, ctid);
         if (ctid == 0) *rn_s = 1.f;
+        cur_key = -1;
+      } else if (!MLA && t.op == OP_O) {  // the attention splits, combined on the way in
+        if constexpr (!MLA)
+          stage_attn_merged<MT, TILED>(p, g, ub, ub + p.xs_floats + MT * kMaxResidRows, ctid);
+        if (ctid == 0)
+#pragma unroll
+          for (int v = 0; v < MT; ++v) rn_s[v] = 1.f;
         cur_key = -1;
       } else if (key != cur_key || key < 0) {
         float rnv[MT];

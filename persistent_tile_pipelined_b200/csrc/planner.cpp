@@ -362,8 +362,22 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // positions per attention stage: MLA 32 latent rows; GQA 64 (four warps x 16 rows)
   s.pos_per_stage = mla ? kMlaPosPerStage : kMaxPosPerStage;
 
+  // KV splits: enough (kv head, split) tasks to cover the SMs, but no split shorter than
+  // one stage of positions at full capacity.  MLA: (head group, split) tasks.
+  const int units = mla ? s.Hq / kMlaHeadGroup : s.Hkv;
+  int S = c.kv_splits;
+  if (!S) {
+    S = std::max(1, nsm / units);
+    int max_s = std::max(1, (s.cap - 1 + s.pos_per_stage - 1) / s.pos_per_stage);  // >= 1 stage each
+    S = std::min(S, max_s);
+  }
+  if (!mla && S > 4 * s.D) return fail(TRE_ERR_UNSUPPORTED, "kv_splits above 4 * head_dim");
+
   s.xs_floats = (s.M * xs + 7) / 8 * 8;
   s.resid_floats = s.M * kMaxResidRows;
+  // the O projection combines the KV splits while it stages its input: a weight per
+  // (token, head, split) and a scale per (token, head), after the residual rows
+  const int merge_floats = mla ? 0 : (s.M * s.Hq * S + s.M * s.Hq + 7) / 8 * 8;
   // attention scratch: q rows (M tokens x G heads), the M new k / v rows, per-warp
   // (m, l, O) per row, scores of the new positions
   const int rows = s.M * G;
@@ -377,7 +391,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
                              2 * kMlaHeadGroup * Smax);
     s.attn_floats = std::max(s.attn_floats, kConsumerWarps * s.KL + s.NP + 64);
   }
-  const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + (s.tiles ? kTileRedFloats : 0),
+  const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + merge_floats +
+                                         (s.tiles ? kTileRedFloats : 0),
                                      s.attn_floats) + 7) / 8 * 8;
   s.ub_floats = ubuf_floats;
   const int misc_bytes = 1024;
@@ -390,17 +405,6 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   if (s.smem_bytes > smem_limit)
     return fail(TRE_ERR_UNSUPPORTED, "ring + buffers exceed the shared memory per block");
 
-  // KV splits: enough (kv head, split) tasks to cover the SMs, but no split shorter than
-  // one stage of positions at full capacity.  MLA: (head group, split) tasks.
-  const int units = mla ? s.Hq / kMlaHeadGroup : s.Hkv;
-  int S = c.kv_splits;
-  if (!S) {
-    S = std::max(1, nsm / units);
-    int max_s = std::max(1, (s.cap - 1 + s.pos_per_stage - 1) / s.pos_per_stage);  // >= 1 stage each
-    S = std::min(S, max_s);
-  }
-  // the combine stages every split's (m, l) in the attention scratch: 2 G S <= 8 G D
-  if (!mla && S > 4 * s.D) return fail(TRE_ERR_UNSUPPORTED, "kv_splits above 4 * head_dim");
   if (mla && 2 * kMlaHeadGroup * S > s.attn_floats)
     return fail(TRE_ERR_UNSUPPORTED, "kv_splits too large for the MLA combine");
   s.kv_splits = S;
@@ -436,7 +440,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
                             prev_down_count, cq, big);
     const int64_t kv_task_bytes = (int64_t)(s.cap - s.M) / S * s.D * 2 * 2;
     b.attention(l, s.Hkv, S, kv_task_bytes, cq, (uint32_t)nqkv, ca);
-    int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)s.Hkv, co, kMaxResidRows);
+    // every (kv head, split) task publishes its partial; O waits for all of them
+    int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)(s.Hkv * S), co, kMaxResidRows);
     int nd;
     if (!moe) {
       int ng = b.gemv(OP_GU, l, s.F, s.d, 2, co, (uint32_t)no, cg, big);

@@ -32,6 +32,9 @@ def _lib() -> ctypes.CDLL:
             fn.restype = None
         lib.synth_u64.argtypes = [u64, u64, u64]
         lib.synth_u64.restype = u64
+        lib.synth_e4m3_blocks.argtypes = [u64, u64, i64, i64, dbl, ctypes.c_void_p,
+                                          ctypes.c_void_p]
+        lib.synth_e4m3_blocks.restype = None
         _LIB = lib
     return _LIB
 
@@ -64,6 +67,20 @@ def normal_f32(seed: int, tensor_id: int, shape, mean: float = 0.0, std: float =
 def normal_f64(seed: int, tensor_id: int, shape, mean: float = 0.0, std: float = 1.0,
                out: np.ndarray | None = None) -> np.ndarray:
     return _fill("synth_normal_f64", np.float64, seed, tensor_id, shape, mean, std, out)
+
+
+def e4m3_blocks(seed: int, tensor_id: int, shape, std: float):
+    """A block-scaled FP8 matrix [N][K] of values std * N(0,1) (the same stream as
+    normal_f64 with mean 0): E4M3 bytes (uint8) and fp32 scales [ceil(N/128)][ceil(K/128)],
+    each scale = block max |value| / 448, each byte the nearest E4M3 of value / scale."""
+    N, K = (int(s) for s in shape)
+    codes = np.empty((N, K), dtype=np.uint8)
+    scales = np.empty(((N + 127) // 128, (K + 127) // 128), dtype=np.float32)
+    if N and K:
+        _lib().synth_e4m3_blocks(seed, tensor_id, N, K, float(std),
+                                 codes.ctypes.data_as(ctypes.c_void_p),
+                                 scales.ctypes.data_as(ctypes.c_void_p))
+    return codes, scales
 
 
 def u64(seed: int, tensor_id: int, index: int) -> int:

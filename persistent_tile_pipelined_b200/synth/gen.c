@@ -17,6 +17,11 @@
  *              value = mean + std * z, computed in double
  *   bf16       double -> float (C conversion, round to nearest even) -> bf16 by round to
  *              nearest even on the upper 16 bits.
+ *   e4m3 blocks  data preparation of a block-scaled FP8 weight (what an FP8 checkpoint
+ *              holds): the values std * z of a [N][K] matrix, one fp32 scale per 128 x 128
+ *              block = (float)(block max |value| / 448) (1 for an all-zero block), and each
+ *              value divided by its block's scale, rounded to the nearest E4M3 number (ties
+ *              to even, saturated at +-448) and stored as its E4M3 byte.
  */
 #include <math.h>
 #include <stdint.h>
@@ -96,5 +101,59 @@ void synth_normal_bf16(uint64_t seed, uint64_t tensor_id, int64_t n, double mean
     normal_pair(key, (uint64_t)p, &z0, &z1);
     out[2 * p] = float_to_bf16_rne((float)(mean + std * z0));
     if (2 * p + 1 < n) out[2 * p + 1] = float_to_bf16_rne((float)(mean + std * z1));
+  }
+}
+
+/* The E4M3 byte of the E4M3 number nearest to v (ties to even; |v| saturates at 448). */
+static uint8_t e4m3_rne(double v) {
+  uint8_t sgn = (v < 0) ? 0x80 : 0;
+  double a = fabs(v);
+  if (a >= 448.0) return sgn | 0x7E;
+  if (a < ldexp(1.0, -6)) {                     /* subnormal range: steps of 2^-9 */
+    double m = nearbyint(a / ldexp(1.0, -9));
+    if (m >= 8.0) return sgn | 0x08;            /* rounded up to 2^-6 */
+    return sgn | (uint8_t)m;
+  }
+  int e;
+  frexp(a, &e);                                 /* a in [2^(e-1), 2^e) */
+  int E = e - 1;                                /* -6 .. 8 */
+  double r = nearbyint(ldexp(a, 3 - E));        /* 8 .. 16: 1 + m/8 in eighths */
+  if (r >= 16.0) {
+    r = 8.0;
+    E += 1;
+  }
+  if (E > 8 || (E == 8 && r > 14.0)) return sgn | 0x7E;
+  return sgn | (uint8_t)((E + 7) << 3) | (uint8_t)(r - 8.0);
+}
+
+void synth_e4m3_blocks(uint64_t seed, uint64_t tensor_id, int64_t N, int64_t K, double std,
+                       uint8_t* codes, float* scales) {
+  int64_t NB = (N + 127) / 128, KB = (K + 127) / 128;
+  uint64_t key = stream_key(seed, tensor_id);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t nb = 0; nb < NB; ++nb) {
+    int64_t n0 = nb * 128, n1 = n0 + 128 < N ? n0 + 128 : N;
+    for (int64_t kb = 0; kb < KB; ++kb) {
+      int64_t k0 = kb * 128, k1 = k0 + 128 < K ? k0 + 128 : K;
+      double amax = 0.0;
+      for (int64_t n = n0; n < n1; ++n)
+        for (int64_t k = k0; k < k1; ++k) {
+          int64_t i = n * K + k;
+          double z0, z1;
+          normal_pair(key, (uint64_t)(i / 2), &z0, &z1);
+          double v = std * ((i & 1) ? z1 : z0);
+          if (fabs(v) > amax) amax = fabs(v);
+        }
+      float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+      scales[nb * KB + kb] = sc;
+      for (int64_t n = n0; n < n1; ++n)
+        for (int64_t k = k0; k < k1; ++k) {
+          int64_t i = n * K + k;
+          double z0, z1;
+          normal_pair(key, (uint64_t)(i / 2), &z0, &z1);
+          double v = std * ((i & 1) ? z1 : z0);
+          codes[i] = e4m3_rne(v / (double)sc);
+        }
+    }
   }
 }

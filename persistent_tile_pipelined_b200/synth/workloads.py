@@ -14,8 +14,8 @@ from typing import Dict, List, Optional
 
 import numpy as np
 
-from . import (TID_EMBED, TID_FINAL_NORM, TID_LM_HEAD, TID_X_IN, normal_bf16, normal_f32,
-               tid_kcache, tid_layer, tid_vcache, token_id)
+from . import (TID_EMBED, TID_FINAL_NORM, TID_LM_HEAD, TID_X_IN, e4m3_blocks, normal_bf16,
+               normal_f32, tid_kcache, tid_layer, tid_vcache, token_id)
 
 W_STD = 0.02
 GAIN_STD = 0.01
@@ -38,6 +38,7 @@ class Workload:
     norm_eps: float = 1e-5
     tokens_per_step: int = 1
     seed: int = 1234
+    weight_format: str = "bf16"  # "fp8": GQA projections as E4M3 bytes + 128x128 block scales
     # MLA
     q_lora: int = 0
     kv_lora: int = 0
@@ -95,8 +96,12 @@ LLAMA8B_KV8K = LLAMA8B.replace(name="llama3-8b-shaped-kv8k", prefill=8192)
 LLAMA8B_KV32K = LLAMA8B.replace(name="llama3-8b-shaped-kv32k", prefill=32768)
 LLAMA8B_KV128K = LLAMA8B.replace(name="llama3-8b-shaped-kv128k", prefill=131072)
 
+# The 8B-shaped stack with FP8 projections (E4M3, one scale per 128 x 128 block); the
+# embedding, norms and LM head stay bf16.
+LLAMA8B_FP8 = LLAMA8B.replace(name="llama3-8b-shaped-fp8", weight_format="fp8")
+
 WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L, MLA4, MOE4, LLAMA8B_KV8K,
-                                 LLAMA8B_KV32K, LLAMA8B_KV128K)}
+                                 LLAMA8B_KV32K, LLAMA8B_KV128K, LLAMA8B_FP8)}
 
 
 def gqa_layer_shapes(w: Workload) -> List[tuple]:
@@ -200,9 +205,21 @@ def gen_tensor(w: Workload, tensor_id: int, shape, kind: str,
     raise ValueError(kind)
 
 
+# FP8 GQA layers: the block scales of projection slot s sit in slot FP8_SCALE_SLOT[s]
+FP8_SCALE_SLOT = {1: 9, 2: 10, 3: 11, 4: 12, 6: 13, 7: 14, 8: 15}
+
+
 def gen_gqa_layer(w: Workload, layer: int) -> Dict[int, np.ndarray]:
-    return {slot: gen_tensor(w, tid_layer(layer, slot), shape, kind)
-            for slot, shape, kind in gqa_layer_shapes(w)}
+    """bf16 words per slot; FP8 workloads: the projection slots hold E4M3 bytes (uint8) of
+    the same N(0, 0.02) values and slots 9 .. 15 their fp32 block scales."""
+    out = {}
+    for slot, shape, kind in gqa_layer_shapes(w):
+        if w.weight_format == "fp8" and slot in FP8_SCALE_SLOT:
+            out[slot], out[FP8_SCALE_SLOT[slot]] = e4m3_blocks(w.seed, tid_layer(layer, slot),
+                                                               shape, W_STD)
+        else:
+            out[slot] = gen_tensor(w, tid_layer(layer, slot), shape, kind)
+    return out
 
 
 def gen_kv_cache(w: Workload, layer: int, which: str) -> np.ndarray:

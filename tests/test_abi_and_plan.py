@@ -133,8 +133,9 @@ def check_plan(wl, nsm, **over):
             # every MLA attention split publishes; W_uv merges a head's splits
             assert T["dep_count"][i] == (wl.n_q_heads // 16) * info.kv_splits
         elif T["type"][i] == T_GEMV and T["op"][i] == OP_O:
-            # the attention counter is bumped once per kv head (by the combining split)
-            assert T["dep_count"][i] == wl.n_kv_heads
+            # every attention split publishes; the O projection merges them
+            assert T["dep_count"][i] == wl.n_kv_heads * info.kv_splits
+            assert T["dep_count"][i] == len(producers)
         elif wl.kind == "moe" and kind == C_ROUTE and dep < wl.n_layers * C_PER_LAYER:
             # the route counter is bumped once, by the router task that finishes last
             assert T["dep_count"][i] == 1
