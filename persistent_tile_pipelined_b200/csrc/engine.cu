@@ -684,7 +684,7 @@ __device__ __forceinline__ int input_key(const Task& t) {
 template <int MT, bool FRAG>
 __device__ void stage_attn_merged(const Params& p, const GemvGeom& gg, float* ub, float* wsc,
                                   int ctid) {
-  const int D = p.D, S = p.nsplit, pst = D + 2;
+  const int D = p.D, S = p.nsplit, pst = gqa_pstride(D);
   const int h0 = gg.k0 / D, nh = (gg.k0 + gg.Kp - 1) / D - h0 + 1;
   float* wm = wsc;                   // [MT][nh][S]: the split weights 2^(m_s - M)
   float* inv = wsc + MT * nh * S;    // [MT][nh]: 1 / sum_s w_s l_s
@@ -1170,7 +1170,7 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
   }
 
   // merge the warps (and, in the last split, the new positions) into this split's partial
-  const size_t pstride = (size_t)D + 2;
+  const size_t pstride = (size_t)gqa_pstride(D);
   for (int idx = ctid; idx < ROWS * D; idx += kConsumerThreads) {
     const int r = idx / D, dd = idx % D, v = r / G, h = r % G;
     float M = -INFINITY;

@@ -133,7 +133,7 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   const size_t o_qkv = cv.take<float>(qkv_n);
   const size_t o_attn = cv.take<float>((size_t)s.Hq * s.D);
   const size_t o_u = cv.take<float>(s.F);
-  const size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * (s.D + 2));
+  const size_t o_part = cv.take<float>((size_t)s.Hq * s.kv_splits * gqa_pstride(s.D));
   const size_t o_inv = cv.take<double>(s.D / 2);
   cv.off = (cv.off + 127) & ~size_t(127);
   const size_t o_maps = cv.take<uint8_t>((size_t)2 * s.L * 128);  // K and V tensor maps

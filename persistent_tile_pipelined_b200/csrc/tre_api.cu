@@ -333,7 +333,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_rtick = cv.take<uint32_t>(1);
   size_t o_mpart = cv.take<float>(moe ? (size_t)(s.nshared + s.topk) * s.d : 1);
   size_t o_dtick = cv.take<uint32_t>(moe ? s.down_blocks : 1);
-  size_t o_part = cv.take<float>(M * s.Hq * s.kv_splits * (mla ? mla_pstride(s.KL) : s.D + 2));
+  size_t o_part = cv.take<float>(M * s.Hq * s.kv_splits * (mla ? mla_pstride(s.KL) : gqa_pstride(s.D)));
   size_t o_logits = cv.take<float>(s.V > 0 ? M * s.V : 1);
   size_t o_tok = cv.take<int32_t>(kMaxTokens);
   size_t o_inv = cv.take<double>(std::max(1, s.D / 2));

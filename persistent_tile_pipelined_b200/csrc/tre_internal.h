@@ -90,6 +90,9 @@ constexpr int kMlaBox = 64;           // latent columns per tensor-map box (128 
 constexpr int kMlaMaxKSteps = 6;      // 16-column k-steps of the score product per warp
 // floats per MLA split partial: O (KL), m, l, 2 pad -> every row starts on 16 bytes
 TRE_HD inline int mla_pstride(int KL) { return KL + 4; }
+// floats per GQA split partial: O (D), m, l, 2 pad -> every row starts on 16 bytes (the O
+// projection reads the partials with 16-byte loads while it combines them)
+TRE_HD inline int gqa_pstride(int D) { return D + 4; }
 
 // Dependency counters: one per (layer, stage of the layer), then the LM head and a
 // counter nothing ever bumps (used only by the fault-injection debug plan).
@@ -184,7 +187,7 @@ struct Params {
                                    // MLA [L] latent caches
   const double* rope_inv_freq_r;   // [R / 2]
   uint32_t* down_tickets;          // MoE down: arrival ticket per row block
-  float* part;                     // [Hq][splits][D + 2]
+  float* part;                     // [m][Hq][splits][gqa_pstride(D)] (MLA: mla_pstride)
   float* logits;                   // [V]
   int32_t* token_out;              // [1] or NULL
   float* hidden;                   // debug [L][d] or NULL
