@@ -230,13 +230,18 @@ def build_engine(wl, device: int, debug_flags: int = 0, overrides=None):
     dev = f"cuda:{device}"
 
     def up(words):
+        if words.dtype in (np.uint8, np.float32):  # E4M3 bytes, fp32 block scales
+            return torch.from_numpy(words).to(dev)
         t = torch.from_numpy(words.view(np.int16)).view(torch.bfloat16)
         return t.to(dev)
 
     model = {"layers": [], "k_cache": [], "v_cache": []}
     for l in range(wl.n_layers):
-        model["layers"].append({slot: up(W.gen_tensor(wl, tid_layer(l, slot), shape, kind))
-                                for slot, shape, kind in W.gqa_layer_shapes(wl)})
+        if wl.weight_format == "fp8":  # one layer's E4M3 bytes and scales at a time
+            model["layers"].append({slot: up(a) for slot, a in W.gen_gqa_layer(wl, l).items()})
+        else:
+            model["layers"].append({slot: up(W.gen_tensor(wl, tid_layer(l, slot), shape, kind))
+                                    for slot, shape, kind in W.gqa_layer_shapes(wl)})
         model["k_cache"].append(up(W.gen_kv_cache(wl, l, "k")))
         model["v_cache"].append(up(W.gen_kv_cache(wl, l, "v")))
     model["embed"] = up(W.gen_tensor(wl, TID_EMBED, (wl.vocab, wl.hidden), "w"))
@@ -378,7 +383,14 @@ def workload_step_bytes(wl, pos=None) -> int:
         Hq, Hkv, D = wl.n_q_heads, wl.n_kv_heads, wl.head_dim
         mlp = (wl.n_experts * d + 3 * (wl.n_shared + wl.top_k) * wl.expert_ffn * d
                if wl.kind == "moe" else 3 * wl.ffn * d)
-        per_layer = ((Hq + 2 * Hkv) * D * d + d * Hq * D + mlp) * 2 + 2 * d * 2
+        proj = (Hq + 2 * Hkv) * D * d + d * Hq * D + mlp
+        per_layer = proj * 2 + 2 * d * 2
+        if getattr(wl, "weight_format", "bf16") == "fp8":  # E4M3 + a scale per 128x128 block
+            def blocks(N, K):
+                return -(-N // 128) * -(-K // 128)
+            nq, nk = Hq * D, Hkv * D
+            per_layer = proj + 4 * (blocks(nq, d) + 2 * blocks(nk, d) + blocks(d, nq) +
+                                    2 * blocks(wl.ffn, d) + blocks(d, wl.ffn)) + 2 * d * 2
         total = per_layer * L + L * Hkv * (pos + 1) * D * 2 * 2
     if wl.vocab > 0:
         total += wl.vocab * d * 2 + d * 2 + d * 2 + wl.vocab * 4
@@ -396,6 +408,8 @@ def decode_config(wl, M: int, overrides: dict, world: int) -> dict:
         "workload": f"{wl.name} decode, batch 1, KV {wl.prefill} positions" +
                     (f", {M} tokens per step (causal verify tiles)" if M > 1 else ""),
         "tokens_per_step": M,
+        "weights": ("E4M3 projections, 128x128 fp32 block scales; bf16 embedding, norms, LM head"
+                    if wl.weight_format == "fp8" else "bf16"),
         "engine_config": overrides,
         "layers": wl.n_layers, "hidden": wl.hidden, "q_heads": wl.n_q_heads,
         "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "ffn": wl.ffn,
@@ -759,8 +773,10 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
+        "dtype": "fp8e4m3" if wl.weight_format == "fp8" else "bf16",
+        "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))" +
+                ("; projections block-quantised to E4M3 (128x128 fp32 scales)"
+                 if wl.weight_format == "fp8" else ""),
         "config": decode_config(wl, M, config_overrides(args.config), world),
         "hbm_gbs": step_bytes / (dev_s / K) / 1e9,
         "hbm_frac_of_8tbs": step_bytes / (dev_s / K) / 1e9 / NOMINAL_HBM_GBS,

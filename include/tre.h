@@ -126,8 +126,20 @@ typedef struct {
                                    (hidden and ffn multiples of 16); 0 = the planner's
                                    choice: tiles at 4 tokens per step when the sizes
                                    allow, else rows                                     */
-  int32_t reserved[4];          /* must be zero                                         */
+  int32_t weight_format;        /* TRE_WEIGHTS_*: storage of the GQA projections        */
+  int32_t reserved[3];          /* must be zero                                         */
 } tre_config;
+
+/* Weight formats (tre_config.weight_format).  BF16: every matrix bf16.  FP8_BLOCK128 (GQA
+ * stacks, one token per step): the seven projection matrices of every layer (Q, K, V, O,
+ * gate, up, down) are E4M3 bytes (the OCP 8-bit float with 4 exponent and 3 mantissa
+ * bits) with one fp32 scale per 128 x 128 block, element W[n][k] standing for
+ * e4m3(W[n][k]) * SCALE[n / 128][k / 128]; the embedding, the norm gains and the LM head
+ * stay bf16.  The dequantisation is fused into the weight-streaming GEMV ("RMSNorm + QKV
+ * + FP8 dequant", TileRT code audit, fused-op list; fewer bytes per token is the pages'
+ * "tokens per byte" lever, Speed is intelligence talk).  Every K must then be a multiple
+ * of 16 (16-byte rows).  The E4M3 NaN bytes (S.1111.111) are not decoded as NaN. */
+enum { TRE_WEIGHTS_BF16 = 0, TRE_WEIGHTS_FP8_BLOCK128 = 1 };
 
 /* Per-layer tensor slots.  layer_w[l * TRE_W_SLOTS + slot] is the device pointer of
  * tensor `slot` of layer l (NULL for slots the layer kind does not use).
@@ -142,6 +154,9 @@ typedef struct {
  *         then R rope rows), DKV[KL+R][d] (KL latent rows then R rope rows),
  *         KV_NORM[KL], UK[H*NP][KL], UV[H*VD][KL], MLA_O[d][H*VD]
  *         (QL = q_lora, KL = kv_lora, R = rope_dim, NP = nope_dim, VD = v_dim)
+ *   GQA with weight_format FP8_BLOCK128: slots 1-4 and 6-8 hold E4M3 bytes of the same
+ *         shapes, and their fp32 block scales [ceil(N/128)][ceil(K/128)] sit in
+ *         SCALE_Q .. SCALE_DOWN (slots 9-15)
  * KV caches (bf16, written at pos by every step, caller owned):
  *   GQA/MOE : k_cache[l], v_cache[l] = [Hkv][kv_capacity][D]
  *   MLA     : k_cache[l] = latent [kv_capacity][KL + R]: RMSNorm(c_kv) then RoPE(k_pe);
@@ -154,6 +169,8 @@ enum {
   TRE_W_EXPERT_GATE = 10, TRE_W_EXPERT_UP = 11, TRE_W_EXPERT_DOWN = 12,
   TRE_W_DQ = 1, TRE_W_Q_NORM = 2, TRE_W_UQ = 3, TRE_W_DKV = 4, TRE_W_KV_NORM = 5,
   TRE_W_UK = 6, TRE_W_UV = 7, TRE_W_MLA_O = 8,
+  TRE_W_SCALE_Q = 9, TRE_W_SCALE_K = 10, TRE_W_SCALE_V = 11, TRE_W_SCALE_O = 12,
+  TRE_W_SCALE_GATE = 13, TRE_W_SCALE_UP = 14, TRE_W_SCALE_DOWN = 15,
   TRE_W_SLOTS = 16
 };
 

@@ -178,6 +178,7 @@ struct GemvGeom {
   int rps;      // rows per ring stage
   int nstages;
   int nkk;      // tiles (multi-token plans): stages per row tile and segment (k-chunks)
+  int esz;      // bytes per weight: 2 (bf16), 1 (E4M3 projections)
 };
 
 template <bool TILED>
@@ -185,6 +186,7 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   GemvGeom g;
   g.K = gemv_K(p, t.op);
   g.nseg = (t.op == OP_GU || t.op == OP_SGU || t.op == OP_RGU) ? 2 : 1;
+  g.esz = (p.wfp8 && (t.op == OP_QKV || t.op == OP_O || t.op == OP_GU || t.op == OP_DOWN)) ? 1 : 2;
   if (t.op == OP_LM || t.op == OP_ROUTER) {
     g.np = 1;
     g.part = 0;
@@ -195,7 +197,7 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
     g.part = t.aux & 0xff;
     g.np = max(1, t.aux >> 8);
   }
-  const int len = g.np == 1 ? g.K : gemv_part_len(g.K, g.np, TILED ? 16 : 8);
+  const int len = g.np == 1 ? g.K : gemv_part_len(g.K, g.np, gemv_part_align(TILED, g.esz == 1));
   g.k0 = g.part * len;
   g.Kp = min(len, g.K - g.k0);
   if (TILED) {  // row tiles of 16; per tile and segment, k-chunks of kTileK columns
@@ -203,68 +205,112 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
     g.nkk = (g.Kp + kTileK - 1) / kTileK;
     g.nstages = (t.r1 - t.r0 + kTileRows - 1) / kTileRows * g.nseg * g.nkk;
   } else {
-    g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes);
+    g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes, g.esz);
     g.nkk = 1;
     g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
   }
   return g;
 }
 
-// Source of this task's K-part of row n of segment `seg`; *contig receives how many rows
-// from n on follow it contiguously in memory (same matrix, row stride = the part length):
-// QKV rows cross from Wq into Wk into Wv, routed rows end at their expert's last row,
-// K-parts of a wider matrix are one row each.
-__device__ __forceinline__ const uint16_t* part_row(const Params& p, const Task& t,
-                                                    const GemvGeom& g, int seg, int n,
-                                                    int* contig) {
+// Source (byte address) of this task's K-part of row n of segment `seg`; *contig receives
+// how many rows from n on follow it contiguously in memory (same matrix, row stride = the
+// part length): QKV rows cross from Wq into Wk into Wv, routed rows end at their expert's
+// last row, K-parts of a wider matrix are one row each.  Offsets count weights of g.esz
+// bytes (E4M3 projections: 1).
+__device__ __forceinline__ const uint8_t* wbytes(const uint16_t* w) {
+  return reinterpret_cast<const uint8_t*>(w);
+}
+
+__device__ __forceinline__ const uint8_t* part_row(const Params& p, const Task& t,
+                                                   const GemvGeom& g, int seg, int n,
+                                                   int* contig) {
   *contig = 0x7fffffff;
-  if (t.op == OP_LM) return p.lm_head + (size_t)n * g.K;
+  const size_t e = (size_t)g.esz;
+  if (t.op == OP_LM) return wbytes(p.lm_head) + (size_t)n * g.K * 2;
   const LayerPtrs& L = p.layers[t.layer];
   const size_t K = (size_t)g.K;
   switch (t.op) {
     case OP_QKV: {
       const int nq = p.Hq * p.D, nk = p.Hkv * p.D;
-      if (n < nq) { *contig = nq - n; return L.w[TRE_W_Q] + (size_t)n * K; }
-      if (n < nq + nk) { *contig = nq + nk - n; return L.w[TRE_W_K] + (size_t)(n - nq) * K; }
-      return L.w[TRE_W_V] + (size_t)(n - nq - nk) * K;
+      if (n < nq) { *contig = nq - n; return wbytes(L.w[TRE_W_Q]) + (size_t)n * K * e; }
+      if (n < nq + nk) { *contig = nq + nk - n; return wbytes(L.w[TRE_W_K]) + (size_t)(n - nq) * K * e; }
+      return wbytes(L.w[TRE_W_V]) + (size_t)(n - nq - nk) * K * e;
     }
     case OP_O:
     case OP_DOWN:
       if (g.np > 1) *contig = 1;
-      return L.w[t.op == OP_O ? TRE_W_O : TRE_W_DOWN] + (size_t)n * K + g.k0;
-    case OP_GU: return L.w[seg ? TRE_W_UP : TRE_W_GATE] + (size_t)n * K;
-    case OP_ROUTER: return L.w[TRE_W_ROUTER] + (size_t)n * K;
+      return wbytes(L.w[t.op == OP_O ? TRE_W_O : TRE_W_DOWN]) + ((size_t)n * K + g.k0) * e;
+    case OP_GU: return wbytes(L.w[seg ? TRE_W_UP : TRE_W_GATE]) + (size_t)n * K * e;
+    case OP_ROUTER: return wbytes(L.w[TRE_W_ROUTER]) + (size_t)n * K * 2;
     case OP_MDQKV:
-      if (n < p.QL) { *contig = p.QL - n; return L.w[TRE_W_DQ] + (size_t)n * K; }
-      return L.w[TRE_W_DKV] + (size_t)(n - p.QL) * K;
-    case OP_UQ: return L.w[TRE_W_UQ] + (size_t)n * K;
-    case OP_UK: return L.w[TRE_W_UK] + (size_t)n * K;
-    case OP_UV: return L.w[TRE_W_UV] + (size_t)n * K;
+      if (n < p.QL) { *contig = p.QL - n; return wbytes(L.w[TRE_W_DQ]) + (size_t)n * K * 2; }
+      return wbytes(L.w[TRE_W_DKV]) + (size_t)(n - p.QL) * K * 2;
+    case OP_UQ: return wbytes(L.w[TRE_W_UQ]) + (size_t)n * K * 2;
+    case OP_UK: return wbytes(L.w[TRE_W_UK]) + (size_t)n * K * 2;
+    case OP_UV: return wbytes(L.w[TRE_W_UV]) + (size_t)n * K * 2;
     case OP_MO:
       if (g.np > 1) *contig = 1;
-      return L.w[TRE_W_MLA_O] + (size_t)n * K + g.k0;
-    case OP_SGU: return L.w[seg ? TRE_W_SHARED_UP : TRE_W_SHARED_GATE] + (size_t)n * K;
+      return wbytes(L.w[TRE_W_MLA_O]) + ((size_t)n * K + g.k0) * 2;
+    case OP_SGU: return wbytes(L.w[seg ? TRE_W_SHARED_UP : TRE_W_SHARED_GATE]) + (size_t)n * K * 2;
     case OP_RGU: {
       const int j = n / p.Fe, r = n - j * p.Fe;
-      const int e = routed_expert(p, t.layer, j, t.id);
+      const int ex = routed_expert(p, t.layer, j, t.id);
       *contig = p.Fe - r;
-      return L.w[seg ? TRE_W_EXPERT_UP : TRE_W_EXPERT_GATE] + ((size_t)e * p.Fe + r) * K;
+      return wbytes(L.w[seg ? TRE_W_EXPERT_UP : TRE_W_EXPERT_GATE]) + ((size_t)ex * p.Fe + r) * K * 2;
     }
     default: {  // OP_MDOWN: part < nshared is a column slice of the shared down matrix
       if (g.part < p.nshared) {
         if (p.nshared > 1) *contig = 1;
-        return L.w[TRE_W_SHARED_DOWN] + (size_t)n * p.nshared * p.Fe + (size_t)g.part * p.Fe;
+        return wbytes(L.w[TRE_W_SHARED_DOWN]) +
+               ((size_t)n * p.nshared * p.Fe + (size_t)g.part * p.Fe) * 2;
       }
-      const int e = routed_expert(p, t.layer, g.part - p.nshared, t.id);
-      return L.w[TRE_W_EXPERT_DOWN] + ((size_t)e * p.d + n) * p.Fe;
+      const int ex = routed_expert(p, t.layer, g.part - p.nshared, t.id);
+      return wbytes(L.w[TRE_W_EXPERT_DOWN]) + ((size_t)ex * p.d + n) * p.Fe * 2;
     }
   }
 }
 
-// Cached positions [t0, t1) of split t.r1 of t.aux over [0, pos) (the new positions come
-// from qkv).  GQA: the last split also RoPEs and appends this step's K / V rows and scores
-// them, so it takes half a share of the cached positions (boundaries at 2 s P / (2 S - 1))
-// and the splits finish together.  MLA: equal shares.
+// Block scales of an E4M3 GEMV task, resolved once per task: row n of segment seg uses the
+// scale row base[...] + (row within its matrix / 128) * KB, where KB = ceil(K / 128); QKV
+// rows cross from Wq's scales into Wk's into Wv's at split[0], split[1].
+struct Fp8Scales {
+  const float* base[3];
+  int split[2];
+  int KB;
+};
+
+__device__ __forceinline__ Fp8Scales fp8_scales(const Params& p, const Task& t, const GemvGeom& g) {
+  const LayerPtrs& L = p.layers[t.layer];
+  auto sc = [&](int slot) { return reinterpret_cast<const float*>(L.w[slot]); };
+  Fp8Scales f;
+  f.KB = (g.K + 127) >> 7;
+  f.split[0] = f.split[1] = 0x7fffffff;
+  f.base[1] = f.base[2] = nullptr;
+  switch (t.op) {
+    case OP_QKV:
+      f.base[0] = sc(TRE_W_SCALE_Q);
+      f.base[1] = sc(TRE_W_SCALE_K);
+      f.base[2] = sc(TRE_W_SCALE_V);
+      f.split[0] = p.Hq * p.D;
+      f.split[1] = (p.Hq + p.Hkv) * p.D;
+      break;
+    case OP_O: f.base[0] = sc(TRE_W_SCALE_O); break;
+    case OP_GU:
+      f.base[0] = sc(TRE_W_SCALE_GATE);
+      f.base[1] = sc(TRE_W_SCALE_UP);
+      break;
+    default: f.base[0] = sc(TRE_W_SCALE_DOWN); break;
+  }
+  return f;
+}
+
+__device__ __forceinline__ const float* fp8_scale_row(const Fp8Scales& f, int seg, int n) {
+  if (seg) return f.base[1] + (size_t)(n >> 7) * f.KB;                 // gate/up: up rows
+  if (n < f.split[0]) return f.base[0] + (size_t)(n >> 7) * f.KB;
+  if (n < f.split[1]) return f.base[1] + (size_t)((n - f.split[0]) >> 7) * f.KB;
+  return f.base[2] + (size_t)((n - f.split[1]) >> 7) * f.KB;
+}
+
 __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& t0, int& t1) {
   const long long P = p.pos;
   const long long S = t.aux, sp = t.r1;
@@ -292,8 +338,8 @@ __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
 // holds the matrices themselves, row n from base[0] below split[0], base[1] below
 // split[1], else base[2] (used by the tile stages).
 struct RowSrc {
-  const uint16_t* base[3];
-  long long stride;   // elements between consecutive rows in memory
+  const uint8_t* base[3];
+  long long stride;   // bytes between consecutive rows in memory
   int split[2];
   bool lookup;        // whole-row stages: resolve every stage with part_row
 };
@@ -301,23 +347,23 @@ struct RowSrc {
 __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const GemvGeom& g) {
   RowSrc r;
   r.lookup = t.op == OP_QKV || t.op == OP_MDQKV;
-  r.stride = g.K;
-  if (t.op == OP_RGU) r.stride = p.d;
-  else if (t.op == OP_MDOWN) r.stride = g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe;
+  r.stride = (long long)g.K * g.esz;
+  if (t.op == OP_RGU) r.stride = 2LL * p.d;
+  else if (t.op == OP_MDOWN) r.stride = 2LL * (g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe);
   int contig;
   r.base[2] = nullptr;
   r.split[0] = r.split[1] = 0x7fffffff;
   if (r.lookup) {
     const LayerPtrs& L = p.layers[t.layer];
     if (t.op == OP_QKV) {
-      r.base[0] = L.w[TRE_W_Q];
-      r.base[1] = L.w[TRE_W_K];
-      r.base[2] = L.w[TRE_W_V];
+      r.base[0] = wbytes(L.w[TRE_W_Q]);
+      r.base[1] = wbytes(L.w[TRE_W_K]);
+      r.base[2] = wbytes(L.w[TRE_W_V]);
       r.split[0] = p.Hq * p.D;
       r.split[1] = (p.Hq + p.Hkv) * p.D;
     } else {
-      r.base[0] = L.w[TRE_W_DQ];
-      r.base[1] = L.w[TRE_W_DKV];
+      r.base[0] = wbytes(L.w[TRE_W_DQ]);
+      r.base[1] = wbytes(L.w[TRE_W_DKV]);
       r.split[0] = p.QL;
     }
     return r;
@@ -328,7 +374,7 @@ __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const 
 }
 
 // Row n of segment seg of a GEMV task's K-part, from its resolved row source.
-__device__ __forceinline__ const uint16_t* src_row(const RowSrc& rs, int seg, int n, int r0) {
+__device__ __forceinline__ const uint8_t* src_row(const RowSrc& rs, int seg, int n, int r0) {
   if (!rs.lookup) return (seg ? rs.base[1] : rs.base[0]) + (long long)(n - r0) * rs.stride;
   if (n < rs.split[0]) return rs.base[0] + (long long)n * rs.stride;
   if (n < rs.split[1]) return rs.base[1] + (long long)(n - rs.split[0]) * rs.stride;
@@ -394,9 +440,9 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
                                             uint8_t* dst, uint64_t* bar, uint64_t pol) {
   if (t.type == T_GEMV) {
     const int n0 = t.r0 + i * g.rps, n1 = min(t.r1, n0 + g.rps);
-    const uint32_t rowb = (uint32_t)g.Kp * 2u;
+    const uint32_t rowb = (uint32_t)g.Kp * (uint32_t)g.esz;
     if (!rs.lookup) {
-      if (rs.stride == g.Kp) {  // rows adjacent in memory: one copy per segment
+      if (rs.stride == (long long)rowb) {  // rows adjacent in memory: one copy per segment
         if (lane < g.nseg)
           bulk_g2s(dst + (size_t)lane * g.rps * rowb, rs.base[lane] + (n0 - t.r0) * rs.stride,
                    (uint32_t)(n1 - n0) * rowb, bar, pol);
@@ -411,7 +457,7 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
     }
     // QKV: each segment's rows of the stage in at most three runs
     int contig = 0;
-    const uint16_t* w0 = lane < g.nseg ? part_row(p, t, g, lane, n0, &contig) : nullptr;
+    const uint8_t* w0 = lane < g.nseg ? part_row(p, t, g, lane, n0, &contig) : nullptr;
     if (__all_sync(0xffffffffu, lane >= g.nseg || contig >= n1 - n0)) {
       if (lane < g.nseg)
         bulk_g2s(dst + (size_t)lane * g.rps * rowb, w0, (uint32_t)(n1 - n0) * rowb, bar, pol);
@@ -421,7 +467,7 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
     for (int seg = 0; seg < g.nseg; ++seg) {
       for (int n = n0; n < n1;) {
         int contig;
-        const uint16_t* w = part_row(p, t, g, seg, n, &contig);
+        const uint8_t* w = part_row(p, t, g, seg, n, &contig);
         const int take = min(n1 - n, contig);
         if ((piece & 31) == lane)
           bulk_g2s(dst + (size_t)(seg * g.rps + (n - n0)) * rowb, w, (uint32_t)take * rowb, bar, pol);
@@ -462,18 +508,18 @@ __device__ __forceinline__ void task_prefetch(const Params& p, const Task& t, in
   {
     const GemvGeom g = gemv_geom<false>(p, t);
     if (g.np > 1 || needs_route(p, t)) return;  // strided rows, or addresses not known yet
-    const size_t rowb = (size_t)g.K * 2;
+    const size_t rowb = (size_t)g.K * g.esz;
     if (g.nseg == 2) {
       for (int s = 0; s < 2; ++s) {
         int run;
-        src[s] = reinterpret_cast<const uint8_t*>(part_row(p, t, g, s, t.r0, &run));
+        src[s] = part_row(p, t, g, s, t.r0, &run);
         bytes[s] = (long long)(t.r1 - t.r0) * rowb;
       }
     } else {
       int n = t.r0, left = t.r1 - t.r0;
       for (int piece = 0; left > 0 && piece < 3; ++piece) {
         int run;
-        src[piece] = reinterpret_cast<const uint8_t*>(part_row(p, t, g, 0, n, &run));
+        src[piece] = part_row(p, t, g, 0, n, &run);
         const int take = min(left, run);
         bytes[piece] = (long long)take * rowb;
         n += take;
@@ -595,7 +641,7 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
         // one copy per row of the tile: columns [c0, c0 + kw) into a padded row slot
         if (lane < ts.nr)
           bulk_g2s(ring + (size_t)slot * SB + (size_t)lane * kTilePitch,
-                   src_row(rs, ts.seg, ts.n0 + lane, t.r0) + ts.c0, (uint32_t)ts.kw * 2u,
+                   src_row(rs, ts.seg, ts.n0 + lane, t.r0) + 2 * ts.c0, (uint32_t)ts.kw * 2u,
                    &full[slot], pol);
         tile_next(ts, t, g);
       } else {
@@ -671,79 +717,6 @@ __device__ __forceinline__ int input_key(const Task& t) {
   }
   const int part = (t.op == OP_LM || t.op == OP_ROUTER) ? 0 : (t.aux & 0xff);
   return (((int)t.layer * 8 + cls) << 8) | part;
-}
-
-// The O-projection input of each of the MT tokens: the attention output, combined from
-// the KV splits' partials on the way in (the fused combine): for head h,
-// attn_h = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s (splits that saw
-// no position have m_s = -inf and weigh 0).  (1) every split's (m, l) of the K-part's heads
-// in one round trip, one warp per (token, head), lanes over the splits, turned into split
-// weights with shuffles; (2) each thread merges 8-column groups, fetching every split's
-// values before it sums them.  Written as planes, or (FRAG) as the tensor-core B operand,
-// like load_input.
-template <int MT, bool FRAG>
-__device__ void stage_attn_merged(const Params& p, const GemvGeom& gg, float* ub, float* wsc,
-                                  int ctid) {
-  const int D = p.D, S = p.nsplit, pst = gqa_pstride(D);
-  const int h0 = gg.k0 / D, nh = (gg.k0 + gg.Kp - 1) / D - h0 + 1;
-  float* wm = wsc;                   // [MT][nh][S]: the split weights 2^(m_s - M)
-  float* inv = wsc + MT * nh * S;    // [MT][nh]: 1 / sum_s w_s l_s
-  const int warp = ctid >> 5, lane = ctid & 31;
-  for (int vh = warp; vh < MT * nh; vh += kConsumerWarps) {
-    const int v = vh / nh, h = h0 + vh % nh;
-    const float* ml = p.part + (size_t)(v * p.Hq + h) * S * pst + D;
-    float M = -INFINITY;
-    for (int sp = lane; sp < S; sp += 32) M = fmaxf(M, __ldcg(ml + (size_t)sp * pst));
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int sp = lane; sp < S; sp += 32) {
-      const float2 x = __ldcg(reinterpret_cast<const float2*>(ml + (size_t)sp * pst));
-      const float w = x.x == -INFINITY ? 0.f : exp2f(x.x - M);
-      L = fmaf(w, x.y, L);
-      wm[vh * S + sp] = w;
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    if (lane == 0) inv[vh] = 1.f / L;
-  }
-  consumer_sync(kConsumerThreads);
-  const int K8 = gg.Kp >> 3;
-  for (int it = ctid; it < MT * K8; it += kConsumerThreads) {
-    const int v = FRAG ? it % MT : it / K8, j = FRAG ? it / MT : it % K8;
-    const int k = gg.k0 + 8 * j, h = k / D, dd = k - h * D, vh = v * nh + (h - h0);
-    const float* src = p.part + (size_t)(v * p.Hq + h) * S * pst + dd;
-    const float* w = wm + vh * S;
-    float e[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 6
-    for (int sp = 0; sp < S; ++sp) {
-      const float ws = w[sp];
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(src + (size_t)sp * pst));
-      const float4 b = __ldcg(reinterpret_cast<const float4*>(src + (size_t)sp * pst + 4));
-      e[0] = fmaf(ws, a.x, e[0]); e[1] = fmaf(ws, a.y, e[1]); e[2] = fmaf(ws, a.z, e[2]);
-      e[3] = fmaf(ws, a.w, e[3]); e[4] = fmaf(ws, b.x, e[4]); e[5] = fmaf(ws, b.y, e[5]);
-      e[6] = fmaf(ws, b.z, e[6]); e[7] = fmaf(ws, b.w, e[7]);
-    }
-    const float r = inv[vh];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) e[q] *= r;
-    if constexpr (FRAG) {
-      uint32_t* fr = reinterpret_cast<uint32_t*>(ub) + 2 * (8 * MT * (j >> 1)) + (j & 1);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t hi, lo;
-        split_pair(e[2 * q], e[2 * q + 1], hi, lo);
-        fr[2 * (v * 4 + q)] = hi;
-        fr[2 * ((MT + v) * 4 + q)] = lo;
-      }
-    } else {
-      float* xlo = ub + (size_t)v * gg.Kp;
-      float* xhi = xlo + gg.Kp / 2;
-      reinterpret_cast<float4*>(xlo)[j] = make_float4(e[0], e[1], e[2], e[3]);
-      reinterpret_cast<float4*>(xhi)[j] = make_float4(e[4], e[5], e[6], e[7]);
-    }
-  }
-  consumer_sync(kConsumerThreads);
 }
 
 // Stage the GEMV input of each of the MT tokens into its two planes (token v's at
@@ -920,8 +893,8 @@ __device__ __forceinline__ void rope_cs(const Params& p, int i, float& c, float&
 // the G query heads of the group attend to cached positions [t0, t1) streamed through the
 // ring; the last split also takes the new position pos from this step's k / v, appends
 // them to the caches and merges its partial.  Every split writes its partial (m, l, O) and
-// publishes; the O-projection tasks combine the splits while they stage their input
-// (stage_attn_merged), so the combine costs no extra hand-off.
+// takes an arrival ticket; the last split of the group to arrive combines all splits —
+// the fused combine — and publishes the group.
 template <int G, int D, int MT>
 __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
                           uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
@@ -1206,10 +1179,74 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     }
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) {  // the O-projection merges the splits while it stages its input
+  if (ctid == 0) {
+    const uint32_t old = ticket_add(p.tickets + g, 1u);
+    *flag = ((old + 1u) % (uint32_t)S) == 0u;
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
-    publish_add(p.counters + t.out, 1u);
   }
+  consumer_sync(kConsumerThreads);
+  if (!*flag) return;
+  // The last split of this kv head to finish combines all splits (the fused combine):
+  // attn = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (splits that saw no
+  // position have m_s = -inf and weigh 0).  Two threads share each group of 4 output
+  // columns and take alternate splits; each fetches its splits' (m, l) and 4 O values
+  // before it sums them (one round trip for up to 18 splits), the pair merges with
+  // shuffles.
+  constexpr int CH = 9;      // splits a thread fetches at once
+  const int sub = ctid & 1;
+  constexpr int NIT = ROWS * D / 4;
+  for (int it0 = 0; it0 < NIT; it0 += kConsumerThreads / 2) {
+    const int it = it0 + (ctid >> 1);
+    const bool act = it < NIT;
+    const int r = act ? it / (D / 4) : 0, dd = act ? (it % (D / 4)) * 4 : 0;
+    const int v = r / G, h = r % G;
+    const size_t q = (size_t)v * p.Hq + g * G + h;
+    const float* base = p.part + q * S * pstride;
+    float M = -INFINITY, L = 0.f, O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+    for (int s0 = sub; act && s0 < S; s0 += 2 * CH) {
+      float2 ml[CH];
+      float4 ov[CH];
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int sp = s0 + 2 * u;
+        if (sp < S) {
+          ml[u] = __ldcg(reinterpret_cast<const float2*>(base + (size_t)sp * pstride + D));
+          ov[u] = __ldcg(reinterpret_cast<const float4*>(base + (size_t)sp * pstride + dd));
+        } else {
+          ml[u] = make_float2(-INFINITY, 0.f);
+          ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float Mn = M;
+#pragma unroll
+      for (int u = 0; u < CH; ++u) Mn = fmaxf(Mn, ml[u].x);
+      if (Mn == -INFINITY) continue;
+      const float a = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      L *= a; O0 *= a; O1 *= a; O2 *= a; O3 *= a;
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const float w = ml[u].x == -INFINITY ? 0.f : exp2f(ml[u].x - Mn);
+        L = fmaf(w, ml[u].y, L);
+        O0 = fmaf(w, ov[u].x, O0); O1 = fmaf(w, ov[u].y, O1);
+        O2 = fmaf(w, ov[u].z, O2); O3 = fmaf(w, ov[u].w, O3);
+      }
+      M = Mn;
+    }
+    const float Mo = __shfl_xor_sync(0xffffffffu, M, 1), Lo = __shfl_xor_sync(0xffffffffu, L, 1);
+    const float P0 = __shfl_xor_sync(0xffffffffu, O0, 1), P1 = __shfl_xor_sync(0xffffffffu, O1, 1);
+    const float P2 = __shfl_xor_sync(0xffffffffu, O2, 1), P3 = __shfl_xor_sync(0xffffffffu, O3, 1);
+    if (act && sub == 0) {  // the last split holds the new position: M is finite
+      const float Mm = fmaxf(M, Mo);
+      const float a0 = M == -INFINITY ? 0.f : exp2f(M - Mm);
+      const float a1 = Mo == -INFINITY ? 0.f : exp2f(Mo - Mm);
+      const float inv = 1.f / fmaf(L, a0, Lo * a1);
+      *reinterpret_cast<float4*>(p.attn + q * D + dd) =
+          make_float4(fmaf(O0, a0, P0 * a1) * inv, fmaf(O1, a0, P1 * a1) * inv,
+                      fmaf(O2, a0, P2 * a1) * inv, fmaf(O3, a0, P3 * a1) * inv);
+    }
+  }
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) publish_add(p.counters + t.out, 1u);
 }
 
 template <int MT>
@@ -1898,13 +1935,6 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         if constexpr (MLA) mla_combine_input(p, t, ub, ub + p.xs_floats, ctid);
         if (ctid == 0) *rn_s = 1.f;
         cur_key = -1;
-      } else if (!MLA && t.op == OP_O) {  // the attention splits, combined on the way in
-        if constexpr (!MLA)
-          stage_attn_merged<MT, TILED>(p, g, ub, ub + p.xs_floats + MT * kMaxResidRows, ctid);
-        if (ctid == 0)
-#pragma unroll
-          for (int v = 0; v < MT; ++v) rn_s[v] = 1.f;
-        cur_key = -1;
       } else if (key != cur_key || key < 0) {
         float rnv[MT];
         load_input<MT, TILED>(p, t, g, ub, red, ctid, rnv);
@@ -1947,7 +1977,51 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
-        if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+        if (MT == 1 && !TILED && g.esz == 1) {  // E4M3 rows (rows of Kp bytes, K8 8-byte groups)
+          const uint2* s8 = reinterpret_cast<const uint2*>(sp);
+          const Fp8Scales fs = fp8_scales(p, t, g);
+          if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+            const uint2* up = s8 + (size_t)g.rps * K8;
+            for (int r = 0; r < nr; r += 2) {
+              const int np = min(2, nr - r), n = n0 + r, n1 = n0 + r + np - 1;
+              float o0, o1, o2, o3;
+              const uint2* g0 = s8 + (size_t)r * K8;
+              const uint2* u0 = up + (size_t)r * K8;
+              if (np == 2) {
+                gemv_rows_fp8<4, 1>(g0, g0 + K8, u0, u0 + K8, fp8_scale_row(fs, 0, n),
+                                    fp8_scale_row(fs, 0, n1), fp8_scale_row(fs, 1, n),
+                                    fp8_scale_row(fs, 1, n1), K8, g.k0, xl, xh, lane, o0, o1, o2, o3);
+              } else {
+                const float* sg = fp8_scale_row(fs, 0, n);
+                const float* su = fp8_scale_row(fs, 1, n);
+                gemv_rows_fp8<2, 2>(g0, u0, u0, u0, sg, su, su, su, K8, g.k0, xl, xh, lane, o0,
+                                    o1, o2, o3);
+              }
+              const float v = reduce4(o0, o1, o2, o3, lane);
+              const float upv = __shfl_xor_sync(0xffffffffu, v, np == 2 ? 16 : 8);
+              const int k = (lane >> 3) & 1;
+              if ((np == 2 && (lane & 23) == 0) || (np == 1 && lane == 0)) {
+                const float a = v * rn, bb = upv * rn;
+                p.u[uoff + n0 + r + k] = wsel * (a / (1.f + expf(-a)) * bb);
+              }
+            }
+          } else {
+            for (int r = 0; r < nr; r += 4) {
+              const int nv = min(4, nr - r), n = n0 + r;
+              const uint2* r0 = s8 + (size_t)r * K8;
+              float o0, o1, o2, o3;
+              gemv_rows_fp8_n(nv, r0, r0 + (size_t)min(1, nv - 1) * K8,
+                              r0 + (size_t)min(2, nv - 1) * K8, r0 + (size_t)min(3, nv - 1) * K8,
+                              fp8_scale_row(fs, 0, n), fp8_scale_row(fs, 0, n + min(1, nv - 1)),
+                              fp8_scale_row(fs, 0, n + min(2, nv - 1)),
+                              fp8_scale_row(fs, 0, n + min(3, nv - 1)), K8, g.k0, xl, xh, lane,
+                              o0, o1, o2, o3);
+              const float v = reduce4(o0, o1, o2, o3, lane);
+              const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+              if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
+            }
+          }
+        } else if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;
           for (int r = 0; r < nr; r += 2) {
             const int np = min(2, nr - r);

@@ -114,6 +114,8 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
     return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: GQA stacks, one token per step");
   if (cfg->debug_flags & (TRE_DEBUG_HIDDEN | TRE_DEBUG_TRACE))
     return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: debug buffers are not available");
+  if (s.wfp8)
+    return fail(TRE_ERR_UNSUPPORTED, "tre_decode_step_static: bf16 weights only");
 
   // ---- scratch layout inside the static array; reject plans that do not fit
   const int qkv_n = (s.Hq + 2 * s.Hkv) * s.D;

@@ -85,10 +85,13 @@ struct Builder {
   // `cut` (> 0: rows of different experts never share a task), and each sub-range is one
   // task per K-part (only the last part bumps `out`).  `np` > 0 fixes the number of
   // K-parts (else they follow from K).  Returns the number of tasks that bump `out`.
+  int esz_proj = 2;  // bytes per weight of the GQA projections (1: E4M3)
+
   int gemv(uint8_t op, int layer, int N, int K, int nseg, int dep, uint32_t dep_count, int out,
            int cap, int np = 0, int cut = 0) {
     if (np <= 0) np = (op == OP_LM || op == OP_ROUTER) ? 1 : gemv_nparts(K, kpart_max);
-    auto ranges = assign_rows(N, (int64_t)nseg * K * 2, cum);
+    const int esz = (op == OP_QKV || op == OP_O || op == OP_GU || op == OP_DOWN) ? esz_proj : 2;
+    auto ranges = assign_rows(N, (int64_t)nseg * K * esz, cum);
     int n = 0;
     for (int s = 0; s < nsm; ++s) {
       for (int r = ranges[s].first; r < ranges[s].second;) {
@@ -257,6 +260,16 @@ static tre_status validate(const tre_config& c) {
     if (c.max_tokens_per_step * (c.n_q_heads / c.n_kv_heads) > 16)
       return fail(TRE_ERR_UNSUPPORTED, "tokens x (q heads per kv head) above 16");
   }
+  if (c.weight_format != TRE_WEIGHTS_BF16 && c.weight_format != TRE_WEIGHTS_FP8_BLOCK128)
+    return fail(TRE_ERR_INVALID_ARG, "unknown weight_format");
+  if (c.weight_format == TRE_WEIGHTS_FP8_BLOCK128) {
+    if (c.kind != TRE_LAYER_GQA)
+      return fail(TRE_ERR_UNSUPPORTED, "FP8 weights are implemented for GQA stacks only");
+    if (c.max_tokens_per_step > 1)
+      return fail(TRE_ERR_UNSUPPORTED, "FP8 weights are implemented for one token per step");
+    if (c.hidden % 16 || c.ffn % 16)
+      return fail(TRE_ERR_UNSUPPORTED, "FP8 weights need hidden and ffn multiples of 16");
+  }
   if (!(c.rope_theta > 0.f)) return fail(TRE_ERR_INVALID_ARG, "rope_theta must be > 0");
   if (!(c.norm_eps >= 0.f)) return fail(TRE_ERR_INVALID_ARG, "norm_eps must be >= 0");
   if (c.dep_timeout_us < 0) return fail(TRE_ERR_INVALID_ARG, "dep_timeout_us < 0");
@@ -331,25 +344,29 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   if (s.d > s.kpart_max)
     return fail(TRE_ERR_UNSUPPORTED, "hidden above 16384 / tokens per step (normalised inputs are staged whole)");
   // (input length, segments, K-part length) of every op the stack uses
-  struct OpShape { int K, nseg, kp; };
-  std::vector<OpShape> ops = {{s.d, 1, 0}, {s.Hq * s.D, 1, 0}, {s.d, 1, s.d}};
+  // E4M3 projections (GQA): QKV, O, gate/up and down rows are 1 byte per weight
+  s.wfp8 = c.weight_format == TRE_WEIGHTS_FP8_BLOCK128;
+  const int pesz = s.wfp8 ? 1 : 2;  // bytes per weight of the layer projections
+  struct OpShape { int K, nseg, kp, esz; };
+  std::vector<OpShape> ops = {{s.d, 1, 0, pesz}, {s.Hq * s.D, 1, 0, pesz}, {s.d, 1, s.d, 2}};
   if (mla) {
-    ops = {{s.d, 1, s.d}, {s.QL, 1, s.QL}, {s.KL, 1, s.KL}, {s.Hq * s.VD, 1, 0},
-           {s.NP, 1, s.NP}};
-    if (s.has_lm) ops.push_back({s.d, 1, s.d});
+    ops = {{s.d, 1, s.d, 2}, {s.QL, 1, s.QL, 2}, {s.KL, 1, s.KL, 2}, {s.Hq * s.VD, 1, 0, 2},
+           {s.NP, 1, s.NP, 2}};
+    if (s.has_lm) ops.push_back({s.d, 1, s.d, 2});
   } else if (moe) {
-    ops.push_back({s.d, 2, 0});                                  // shared / routed gate-up
-    ops.push_back({(s.nshared + s.topk) * s.Fe, 1, s.Fe});       // MoE down: one part per expert
+    ops.push_back({s.d, 2, 0, 2});                               // shared / routed gate-up
+    ops.push_back({(s.nshared + s.topk) * s.Fe, 1, s.Fe, 2});    // MoE down: one part per expert
   } else {
-    ops.push_back({s.d, 2, 0});
-    ops.push_back({s.F, 1, 0});
+    ops.push_back({s.d, 2, 0, pesz});
+    ops.push_back({s.F, 1, 0, pesz});
   }
   // a stage holds one attention tile: 64 K and V rows (GQA) or 32 latent rows (MLA)
   int xs = 8, need = mla ? (s.KL + s.R) * kMlaPosPerStage * 2 : 4 * s.D * kMaxPosPerStage;
   for (auto& o : ops) {
-    const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max), s.tiles ? 16 : 8);
+    const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max),
+                                               gemv_part_align(s.tiles, o.esz == 1));
     xs = std::max(xs, kp);
-    need = std::max(need, s.tiles ? kTileRows * kTilePitch : o.nseg * kp * 2);
+    need = std::max(need, s.tiles ? kTileRows * kTilePitch : o.nseg * kp * o.esz);
   }
   // A ring stage holds whole rows of one K-part (gate/up: a row of each matrix), or the K
   // and V rows of 8-64 cached positions.
@@ -375,9 +392,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
 
   s.xs_floats = (s.M * xs + 7) / 8 * 8;
   s.resid_floats = s.M * kMaxResidRows;
-  // the O projection combines the KV splits while it stages its input: a weight per
-  // (token, head, split) and a scale per (token, head), after the residual rows
-  const int merge_floats = mla ? 0 : (s.M * s.Hq * S + s.M * s.Hq + 7) / 8 * 8;
+
   // attention scratch: q rows (M tokens x G heads), the M new k / v rows, per-warp
   // (m, l, O) per row, scores of the new positions
   const int rows = s.M * G;
@@ -391,8 +406,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
                              2 * kMlaHeadGroup * Smax);
     s.attn_floats = std::max(s.attn_floats, kConsumerWarps * s.KL + s.NP + 64);
   }
-  const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + merge_floats +
-                                         (s.tiles ? kTileRedFloats : 0),
+  const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + (s.tiles ? kTileRedFloats : 0),
                                      s.attn_floats) + 7) / 8 * 8;
   s.ub_floats = ubuf_floats;
   const int misc_bytes = 1024;
@@ -411,6 +425,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
 
   Builder b(nsm);
   b.kpart_max = s.kpart_max;
+  b.esz_proj = pesz;
   int prev_down = -1;
   uint32_t prev_down_count = 0;
   for (int l = 0; l < s.L && mla; ++l) {
@@ -440,8 +455,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
                             prev_down_count, cq, big);
     const int64_t kv_task_bytes = (int64_t)(s.cap - s.M) / S * s.D * 2 * 2;
     b.attention(l, s.Hkv, S, kv_task_bytes, cq, (uint32_t)nqkv, ca);
-    // every (kv head, split) task publishes its partial; O waits for all of them
-    int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)(s.Hkv * S), co, kMaxResidRows);
+    // the last split of each kv head to finish combines the head's splits and publishes
+    int no = b.gemv(OP_O, l, s.d, s.Hq * s.D, 1, ca, (uint32_t)s.Hkv, co, kMaxResidRows);
     int nd;
     if (!moe) {
       int ng = b.gemv(OP_GU, l, s.F, s.d, 2, co, (uint32_t)no, cg, big);
@@ -565,7 +580,14 @@ int64_t step_bytes(const PlanShape& s, int pos, int m) {
   const int64_t mlp = s.kind == TRE_LAYER_MOE
                           ? (int64_t)s.E * d + 3LL * (s.nshared + s.topk) * s.Fe * d
                           : 3LL * s.F * d;
-  int64_t per_layer = ((int64_t)(s.Hq + 2 * s.Hkv) * D * d + d * s.Hq * D + mlp) * 2 + 2 * d * 2;
+  const int64_t proj = (int64_t)(s.Hq + 2 * s.Hkv) * D * d + d * s.Hq * D + mlp;
+  int64_t per_layer = proj * 2 + 2 * d * 2;
+  if (s.wfp8) {  // E4M3 bytes plus one fp32 scale per 128 x 128 block of every matrix
+    auto blocks = [](int64_t N, int64_t K) { return ((N + 127) / 128) * ((K + 127) / 128); };
+    const int64_t nq = (int64_t)s.Hq * D, nk = (int64_t)s.Hkv * D;
+    per_layer = proj + 4 * (blocks(nq, d) + 2 * blocks(nk, d) + blocks(d, nq) +
+                            2 * blocks(s.F, d) + blocks(d, s.F)) + 2 * d * 2;
+  }
   int64_t bytes = per_layer * s.L;
   bytes += (int64_t)s.L * s.Hkv * (int64_t)pos * D * 2 * 2;  // K and V read
   bytes += (int64_t)s.L * s.Hkv * D * 2 * 2 * m;             // the m tokens' K and V written

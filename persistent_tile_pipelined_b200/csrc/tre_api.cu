@@ -239,6 +239,9 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   static const int gqa_slots[] = {TRE_W_ATTN_NORM, TRE_W_Q,        TRE_W_K,  TRE_W_V,   TRE_W_O,
                                   TRE_W_FFN_NORM,  TRE_W_GATE,     TRE_W_UP, TRE_W_DOWN};
   std::vector<int> slots(gqa_slots, gqa_slots + 9);
+  if (s.wfp8)  // the E4M3 projections' block scales
+    slots.insert(slots.end(), {TRE_W_SCALE_Q, TRE_W_SCALE_K, TRE_W_SCALE_V, TRE_W_SCALE_O,
+                               TRE_W_SCALE_GATE, TRE_W_SCALE_UP, TRE_W_SCALE_DOWN});
   const bool mla = s.kind == TRE_LAYER_MLA;
   if (mla) {
     slots = {TRE_W_ATTN_NORM, TRE_W_DQ, TRE_W_Q_NORM, TRE_W_UQ, TRE_W_DKV, TRE_W_KV_NORM,
@@ -444,6 +447,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   // default: hold (measured faster on the 8B-shaped stack: 0.683 vs 0.665 of peak)
   p.hold_next_op = cfg->stream_policy != 1;
   p.gemv_tiles = s.tiles;
+  p.wfp8 = s.wfp8;
   p.err = reinterpret_cast<int32_t*>(B + o_err);
   p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
   p.status_host = e->status_dev;

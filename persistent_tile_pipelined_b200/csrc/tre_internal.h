@@ -49,10 +49,14 @@ TRE_HD inline int gemv_part_len(int K, int nparts, int align = 8) {
   const int l = (K + nparts - 1) / nparts;
   return (l + align - 1) / align * align;
 }
-TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes) {
-  const int r = stage_bytes / (nseg * K * 2);
+// esz: bytes per weight element (2 bf16, 1 E4M3)
+TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes, int esz = 2) {
+  const int r = stage_bytes / (nseg * K * esz);
   return r < 1 ? 1 : r;
 }
+// K-part boundaries: multiples of 8 columns (16 bytes of bf16), of 16 for tensor-core tiles
+// and for E4M3 rows (16 bytes)
+TRE_HD inline int gemv_part_align(bool tiles, bool fp8) { return tiles || fp8 ? 16 : 8; }
 
 // ---- tasks --------------------------------------------------------------------------
 enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1, T_MLA_ATTN = 2 };
@@ -129,6 +133,7 @@ struct PlanShape {
   int QL, KL, R, NP, VD;  // MLA: q_lora, kv_lora, rope, nope, v dims
   int kpart_max;       // longest input slice of a GEMV task (floats)
   int tiles;           // multi-token plan: GEMV stages are 16-row tensor-core tiles
+  int wfp8;            // GQA projections are E4M3 with 128 x 128 block scales
   int u_floats;        // the SwiGLU activation buffer (MoE: shared then routed slices)
   int down_blocks;     // MoE down: row blocks (each summed by its last slot to finish)
   int nsm;
@@ -209,6 +214,7 @@ struct Params {
   int flags;
   int hold_next_op;                // producer waits for this SM's publish at op boundaries
   int gemv_tiles;                  // GEMV stages are 16-row tiles (multi-token plans)
+  int wfp8;                        // QKV / O / gate-up / down weights are E4M3 + block scales
   long long timeout_ns;
   long long pf_window;             // L2 prefetch bytes allowed beyond the ring (0 = off)
 };

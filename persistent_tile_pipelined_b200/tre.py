@@ -26,6 +26,7 @@ TRE_ERR_UNSUPPORTED = -6
 TRE_ERR_BOUNDS = -7
 TRE_ERR_STATE = -8
 TRE_LAYER_GQA, TRE_LAYER_MLA, TRE_LAYER_MOE = 0, 1, 2
+TRE_WEIGHTS_BF16, TRE_WEIGHTS_FP8_BLOCK128 = 0, 1
 TRE_DEBUG_HIDDEN, TRE_DEBUG_TRACE, TRE_DEBUG_FAULT_INJECT, TRE_DEBUG_NO_OVERLAP = 1, 2, 4, 8
 TRE_W_SLOTS = 16
 TRACE_COLS = 8
@@ -50,7 +51,8 @@ class tre_config(ctypes.Structure):
         (n, ctypes.c_int32) for n in (
             "has_embed_lm_head", "debug_flags", "dep_timeout_us", "num_sms", "kv_splits",
             "stage_bytes", "ring_stages", "l2_prefetch_kb", "gemv_kpart_max",
-            "stream_policy", "multi_token_gemv")] + [("reserved", ctypes.c_int32 * 4)]
+            "stream_policy", "multi_token_gemv", "weight_format")] + [
+        ("reserved", ctypes.c_int32 * 3)]
 
 
 class tre_weights(ctypes.Structure):
@@ -275,14 +277,20 @@ def config_from_workload(wl, **overrides) -> tre_config:
     c.rope_theta = wl.rope_theta
     c.norm_eps = wl.norm_eps
     c.has_embed_lm_head = 1 if wl.has_embed_lm_head else 0
+    c.weight_format = TRE_WEIGHTS_FP8_BLOCK128 if getattr(wl, "weight_format", "bf16") == "fp8" \
+        else TRE_WEIGHTS_BF16
     for k, v in overrides.items():
         setattr(c, k, v)
     return c
 
 
 def _dev_tensor(words: np.ndarray, device):
+    """bf16 words (uint16) as a bf16 tensor; E4M3 bytes (uint8) and fp32 scales as they are."""
     import torch
-    t = torch.from_numpy(np.ascontiguousarray(words).view(np.int16)).view(torch.bfloat16)
+    a = np.ascontiguousarray(words)
+    if a.dtype == np.uint8 or a.dtype == np.float32:
+        return torch.from_numpy(a).to(device, non_blocking=False)
+    t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
     return t.to(device, non_blocking=False)
 
 

@@ -133,9 +133,8 @@ def check_plan(wl, nsm, **over):
             # every MLA attention split publishes; W_uv merges a head's splits
             assert T["dep_count"][i] == (wl.n_q_heads // 16) * info.kv_splits
         elif T["type"][i] == T_GEMV and T["op"][i] == OP_O:
-            # every attention split publishes; the O projection merges them
-            assert T["dep_count"][i] == wl.n_kv_heads * info.kv_splits
-            assert T["dep_count"][i] == len(producers)
+            # the attention counter is bumped once per kv head (by the combining split)
+            assert T["dep_count"][i] == wl.n_kv_heads
         elif wl.kind == "moe" and kind == C_ROUTE and dep < wl.n_layers * C_PER_LAYER:
             # the route counter is bumped once, by the router task that finishes last
             assert T["dep_count"][i] == 1
@@ -438,7 +437,7 @@ def test_multi_token_cuda_core_form_takes_any_k():
 def test_reserved_fields_must_be_zero():
     import ctypes
     cfg = tre.config_from_workload(W.TINY)
-    cfg.reserved[3] = 1
+    cfg.reserved[2] = 1
     info = tre.tre_plan_info()
     assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448,
                                     ctypes.byref(info)) == tre.TRE_ERR_INVALID_ARG
@@ -500,3 +499,36 @@ def test_kernel_per_op_groups(wl, nsm):
     # launches per step: QKV, attention, O, gate/up, down per GQA layer plus the LM head
     if wl.kind == "gqa":
         assert G == 5 * wl.n_layers + (1 if wl.vocab else 0)
+
+
+def test_fp8_plans():
+    """FP8 projections: the same task graph, every projection row streamed at one byte per
+    weight (plus one fp32 scale per 128 x 128 block), the LM head still bf16; the format is
+    refused where it is not implemented."""
+    fp8 = W.LLAMA8B_FP8
+    check_plan(fp8, 148)
+    check_plan(W.TINY.replace(weight_format="fp8", hidden=272, ffn=720, vocab=1001), 7)
+    info8 = tre.tre_plan_inspect(tre.config_from_workload(fp8))
+    info16 = tre.tre_plan_inspect(tre.config_from_workload(W.LLAMA8B))
+    d, L, V, F = fp8.hidden, fp8.n_layers, fp8.vocab, fp8.ffn
+    nq, nk = fp8.n_q_heads * fp8.head_dim, fp8.n_kv_heads * fp8.head_dim
+    proj = (nq + 2 * nk) * d + d * nq + 3 * F * d
+    blocks = lambda N, K: -(-N // 128) * -(-K // 128)  # noqa: E731
+    scales = 4 * (blocks(nq, d) + 2 * blocks(nk, d) + blocks(d, nq) + 2 * blocks(F, d) + blocks(d, F))
+    assert info16.weight_bytes - info8.weight_bytes == L * (proj - scales)
+    # byte-balanced over the SMs (within 0.5 % of the busiest SM's bytes)
+    assert info8.max_sm_bytes - info8.min_sm_bytes <= 0.005 * info8.max_sm_bytes
+    for over, status in [(dict(kind="moe"), tre.TRE_ERR_UNSUPPORTED),
+                         (dict(max_tokens_per_step=2), tre.TRE_ERR_UNSUPPORTED),
+                         (dict(hidden=264), tre.TRE_ERR_UNSUPPORTED),
+                         (dict(weight_format=7), tre.TRE_ERR_INVALID_ARG)]:
+        cfg = tre.config_from_workload(W.TINY.replace(weight_format="fp8"))
+        for k, v in over.items():
+            if k == "kind":
+                cfg.kind = tre.TRE_LAYER_MOE
+                cfg.n_experts, cfg.top_k, cfg.expert_ffn = 8, 2, 64
+            else:
+                setattr(cfg, k, v)
+        import ctypes
+        info = tre.tre_plan_info()
+        assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status, over

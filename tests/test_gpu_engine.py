@@ -388,3 +388,31 @@ def test_graph_replays_of_per_op_steps_leave_persistent_steps_correct():
         assert e <= TOL and e <= REG_TOL, f"logits rel err {e:.3g} after per-op graph replays"
         tok = ORC.argmax(ref)
     eng.close()
+
+
+# ---- FP8 projections (E4M3 bytes, one fp32 scale per 128 x 128 block) ---------------------
+@pytest.mark.parametrize("over,cfg,steps", [
+    (dict(), dict(), 3),
+    (dict(hidden=272, ffn=720, vocab=1001, prefill=77), dict(), 2),     # partial blocks, ragged N
+    (dict(n_q_heads=8, n_kv_heads=1, n_layers=3), dict(num_sms=7), 2),  # rows cross Wq/Wk/Wv blocks
+    (dict(), dict(gemv_kpart_max=512), 2),                              # down in K-parts (k0 = 352)
+    (dict(), dict(num_sms=3, ring_stages=2, stage_bytes=16384), 2),
+], ids=["tiny", "ragged", "g8-sms7", "kparts", "sms3-ring2"])
+def test_fp8_projections(over, cfg, steps):
+    """The engine with E4M3 projections (dequantised inside the weight-streaming GEMV)
+    against the oracle's block-scaled FP8 decode step."""
+    run_and_compare(W.TINY.replace(weight_format="fp8", **over), steps=steps, **cfg)
+
+
+def test_fp8_kernel_per_op_form():
+    run_and_compare(W.TINY.replace(weight_format="fp8"), steps=2, mode=tre.TRE_LAUNCH_PER_OP)
+
+
+@pytest.mark.slow
+def test_llama8b_fp8_greedy_steps():
+    """The 8B-shaped stack with E4M3 projections in the benchmark's launch configuration:
+    8 greedy steps, then one more with every layer's hidden state checked."""
+    wl = W.LLAMA8B_FP8.replace(decode_steps=9)
+    worst, ties, state = run_and_compare(wl, steps=8, check_hidden=False, reg_tol=REG_TOL_LONG)
+    assert ties <= 1
+    run_and_compare(wl, steps=1, check_hidden=True, state=state, reg_tol=REG_TOL_LONG)
