@@ -44,8 +44,10 @@ __device__ __forceinline__ bool aborted(const Params& p) { return *p.abort_flag 
 // flag is a global-memory read, and a waiter stalled on it notices its own event late.
 constexpr long long kCheckCycles = 1 << 15;
 
-// GEMV input staging: items each thread fetches before storing any.
+// GEMV input staging: items each thread fetches before storing any (tensor-core fragments;
+// fp32 planes).
 constexpr int kLoadBatch = 2;
+constexpr int kPlaneBatch = 4;
 
 // Wait until counter `idx` reaches epoch * count (wrap-safe).  Bounded; on expiry the
 // error names `detail` (a task index).  A kernel-per-op launch never waits: the launches
@@ -425,7 +427,7 @@ __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, 
                                                 int t0, int t1, int i) {
   if (t.type == T_GEMV) {
     const int nr = min(g.rps, t.r1 - (t.r0 + i * g.rps));
-    return (uint32_t)(g.nseg * nr * g.Kp * 2);
+    return (uint32_t)(g.nseg * nr * g.Kp * g.esz);
   }
   if (t.type == T_MLA_ATTN)  // whole boxes (rows past the cache are zero-filled)
     return (uint32_t)((p.KL + p.R) / kMlaBox * kMlaPosPerStage * 128);
@@ -836,26 +838,50 @@ __device__ void load_input(const Params& p, const Task& t, const GemvGeom& gg, f
     float* xhi = xlo + K / 2;
     const float* sv = src ? src + v * vstride : nullptr;
     const uint16_t* bv = src_bf ? src_bf + (size_t)step_token(p, v) * p.d : nullptr;
-    for (int j = ctid; j < K8; j += kConsumerThreads) {
-      float e[8];
-      if (bv) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(bv) + j);
-        e[0] = bf_lo(w.x); e[1] = bf_hi(w.x); e[2] = bf_lo(w.y); e[3] = bf_hi(w.y);
-        e[4] = bf_lo(w.z); e[5] = bf_hi(w.z); e[6] = bf_lo(w.w); e[7] = bf_hi(w.w);
-      } else {
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(sv) + 2 * j);
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(sv) + 2 * j + 1);
-        e[0] = a.x; e[1] = a.y; e[2] = a.z; e[3] = a.w; e[4] = b.x; e[5] = b.y; e[6] = b.z; e[7] = b.w;
-      }
-      if (gain) {
+    // each thread fetches kPlaneBatch 8-column groups (and their gains) before it stores
+    // any, so that the global reads overlap instead of costing one round trip per group;
+    // indices are clamped, so the fetches need no guard
+    constexpr int PB = MT == 1 ? kPlaneBatch : 1;  // (more tokens: registers are short)
+    for (int j0 = ctid; j0 < K8; j0 += PB * kConsumerThreads) {
+      float4 ra[PB], rb[PB];
+      uint4 gw[PB];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) ss[v] = fmaf(e[k], e[k], ss[v]);
-        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain) + j);
-        e[0] *= bf_lo(g.x); e[1] *= bf_hi(g.x); e[2] *= bf_lo(g.y); e[3] *= bf_hi(g.y);
-        e[4] *= bf_lo(g.z); e[5] *= bf_hi(g.z); e[6] *= bf_lo(g.w); e[7] *= bf_hi(g.w);
+      for (int u = 0; u < PB; ++u) {
+        const int j = min(j0 + u * kConsumerThreads, K8 - 1);
+        if (bv) {
+          const uint4 w = __ldg(reinterpret_cast<const uint4*>(bv) + j);
+          ra[u] = make_float4(__uint_as_float(w.x), __uint_as_float(w.y), __uint_as_float(w.z),
+                              __uint_as_float(w.w));
+        } else {
+          ra[u] = __ldcg(reinterpret_cast<const float4*>(sv) + 2 * j);
+          rb[u] = __ldcg(reinterpret_cast<const float4*>(sv) + 2 * j + 1);
+        }
+        if (gain) gw[u] = __ldg(reinterpret_cast<const uint4*>(gain) + j);
       }
-      reinterpret_cast<float4*>(xlo)[j] = make_float4(e[0], e[1], e[2], e[3]);
-      reinterpret_cast<float4*>(xhi)[j] = make_float4(e[4], e[5], e[6], e[7]);
+#pragma unroll
+      for (int u = 0; u < PB; ++u) {
+        const int j = j0 + u * kConsumerThreads;
+        if (j >= K8) break;
+        float e[8];
+        if (bv) {
+          const uint32_t x0 = __float_as_uint(ra[u].x), x1 = __float_as_uint(ra[u].y);
+          const uint32_t x2 = __float_as_uint(ra[u].z), x3 = __float_as_uint(ra[u].w);
+          e[0] = bf_lo(x0); e[1] = bf_hi(x0); e[2] = bf_lo(x1); e[3] = bf_hi(x1);
+          e[4] = bf_lo(x2); e[5] = bf_hi(x2); e[6] = bf_lo(x3); e[7] = bf_hi(x3);
+        } else {
+          e[0] = ra[u].x; e[1] = ra[u].y; e[2] = ra[u].z; e[3] = ra[u].w;
+          e[4] = rb[u].x; e[5] = rb[u].y; e[6] = rb[u].z; e[7] = rb[u].w;
+        }
+        if (gain) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) ss[v] = fmaf(e[k], e[k], ss[v]);
+          const uint4 g = gw[u];
+          e[0] *= bf_lo(g.x); e[1] *= bf_hi(g.x); e[2] *= bf_lo(g.y); e[3] *= bf_hi(g.y);
+          e[4] *= bf_lo(g.z); e[5] *= bf_hi(g.z); e[6] *= bf_lo(g.w); e[7] *= bf_hi(g.w);
+        }
+        reinterpret_cast<float4*>(xlo)[j] = make_float4(e[0], e[1], e[2], e[3]);
+        reinterpret_cast<float4*>(xhi)[j] = make_float4(e[4], e[5], e[6], e[7]);
+      }
     }
   }
   if (gain) {
