@@ -47,7 +47,7 @@ constexpr long long kCheckCycles = 1 << 15;
 // GEMV input staging: items each thread fetches before storing any (tensor-core fragments;
 // fp32 planes).
 constexpr int kLoadBatch = 2;
-constexpr int kPlaneBatch = 4;
+constexpr int kPlaneBatch = 2;
 
 // Wait until counter `idx` reaches epoch * count (wrap-safe).  Bounded; on expiry the
 // error names `detail` (a task index).  A kernel-per-op launch never waits: the launches
@@ -207,7 +207,8 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
     g.nkk = (g.Kp + kTileK - 1) / kTileK;
     g.nstages = (t.r1 - t.r0 + kTileRows - 1) / kTileRows * g.nseg * g.nkk;
   } else {
-    g.rps = gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes, g.esz);
+    g.rps = g.esz == 1 ? fp8_rows_per_stage(g.Kp, g.nseg, p.stage_bytes)
+                       : gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes, g.esz);
     g.nkk = 1;
     g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
   }
@@ -443,6 +444,15 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
   if (t.type == T_GEMV) {
     const int n0 = t.r0 + i * g.rps, n1 = min(t.r1, n0 + g.rps);
     const uint32_t rowb = (uint32_t)g.Kp * (uint32_t)g.esz;
+    if (g.esz == 1) {  // E4M3 rows: one copy per row, rows at the padded pitch
+      const uint32_t pitch = (uint32_t)fp8_row_pitch(g.Kp);
+      for (int k = lane; k < g.nseg * (n1 - n0); k += 32) {
+        const int seg = k / (n1 - n0), r = k % (n1 - n0);
+        bulk_g2s(dst + (size_t)(seg * g.rps + r) * pitch, src_row(rs, seg, n0 + r, t.r0), rowb,
+                 bar, pol);
+      }
+      return;
+    }
     if (!rs.lookup) {
       if (rs.stride == (long long)rowb) {  // rows adjacent in memory: one copy per segment
         if (lane < g.nseg)
@@ -719,6 +729,93 @@ __device__ __forceinline__ int input_key(const Task& t) {
   }
   const int part = (t.op == OP_LM || t.op == OP_ROUTER) ? 0 : (t.aux & 0xff);
   return (((int)t.layer * 8 + cls) << 8) | part;
+}
+
+// The input of a GEMV over E4M3 rows (one token) as the B operand of mma.sync m16n8k16
+// (f16 in, fp32 accumulate), in fragment order: column c of the K-part belongs to k-step
+// s = c / 16 and column group t4 = (c % 16) / 4, and entry [s][part][t4] (8 bytes) holds
+// (x[c0], x[c0 + 1]) and (x[c0 + 2], x[c0 + 3]) of c0 = 16 s + 4 t4 as f16x2 — part 0 the
+// f16 rounding hi of each x, part 1 the rounding of x - hi (about 22 significand bits in
+// all).  The A fragments take the weights' columns in the same order.  Columns from Kp up
+// to the next multiple of 64 are zero.  An |x| of 65504 or more (beyond f16) records a
+// bounds error.  rn receives the RMSNorm scale (1 when the op has no norm).
+__device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
+                                float* red, int ctid, float* rn) {
+  const int K = gg.Kp, NG = ((K + 63) / 64 * 64) / 4;  // 4-column groups
+  const float* src = nullptr;
+  const uint16_t* src_bf = nullptr;
+  const uint16_t* gain = nullptr;
+  switch (t.op) {
+    case OP_QKV:
+      gain = p.layers[t.layer].w[TRE_W_ATTN_NORM];
+      if (t.layer > 0) src = p.x;
+      else if (p.x_in) src = p.x_in;
+      else src_bf = p.embed + (size_t)step_token(p, 0) * p.d;
+      break;
+    case OP_O: src = p.attn; break;
+    case OP_GU: src = p.h1; gain = p.layers[t.layer].w[TRE_W_FFN_NORM]; break;
+    default: src = p.u; break;  // OP_DOWN
+  }
+  if (src) src += gg.k0;
+  float ss = 0.f;
+  bool bad = false;
+  uint2* fr = reinterpret_cast<uint2*>(ub);
+  constexpr int B = 4;  // groups a thread fetches before it stores any
+  for (int q0 = ctid; q0 < NG; q0 += B * kConsumerThreads) {
+    float4 xv[B];
+    uint2 gv[B];
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      const int q = q0 + u * kConsumerThreads, c = min(4 * q, K - 4);  // clamped fetch
+      if (src_bf) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(src_bf + c));
+        xv[u] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+      } else {
+        xv[u] = __ldcg(reinterpret_cast<const float4*>(src + c));
+      }
+      if (gain) gv[u] = __ldg(reinterpret_cast<const uint2*>(gain + c));
+    }
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      const int q = q0 + u * kConsumerThreads;
+      if (q >= NG) break;
+      float e[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+      if (4 * q >= K) {
+        e[0] = e[1] = e[2] = e[3] = 0.f;
+      } else if (gain) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ss = fmaf(e[k], e[k], ss);
+        e[0] *= bf_lo(gv[u].x); e[1] *= bf_hi(gv[u].x);
+        e[2] *= bf_lo(gv[u].y); e[3] *= bf_hi(gv[u].y);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) bad |= !(fabsf(e[k]) < 65504.f) && !isnan(e[k]);
+      const __half2 h01 = __floats2half2_rn(e[0], e[1]), h23 = __floats2half2_rn(e[2], e[3]);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(e[0] - f01.x, e[1] - f01.y);
+      const __half2 l23 = __floats2half2_rn(e[2] - f23.x, e[3] - f23.y);
+      const int sidx = q >> 2, t4 = q & 3;
+      fr[(sidx * 2 + 0) * 4 + t4] = make_uint2(*reinterpret_cast<const uint32_t*>(&h01),
+                                               *reinterpret_cast<const uint32_t*>(&h23));
+      fr[(sidx * 2 + 1) * 4 + t4] = make_uint2(*reinterpret_cast<const uint32_t*>(&l01),
+                                               *reinterpret_cast<const uint32_t*>(&l23));
+    }
+  }
+  if (bad) record_error(p, TRE_ERR_BOUNDS, t.id);
+  if (gain) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if ((ctid & 31) == 0) red[ctid >> 5] = ss;
+  }
+  consumer_sync(kConsumerThreads);
+  float r = 1.f;
+  if (gain) {
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) tot += red[w];
+    r = 1.f / sqrtf(tot / (float)K + p.eps);
+  }
+  rn[0] = r;
 }
 
 // Stage the GEMV input of each of the MT tokens into its two planes (token v's at
@@ -1910,7 +2007,7 @@ __device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, c
 // MLA = true: the absorbed-MLA stack's kernel (MLA tiles, no GQA attention); false: GQA /
 // MoE.  Separate instantiations keep each kernel's register allocation to its own tiles.
 // TILED: GEMV stages are 16-row tensor-core tiles (multi-token plans).
-template <bool MLA, int MT, bool TILED>
+template <bool MLA, int MT, bool TILED, bool F8>
 __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                          float* misc) {
@@ -1961,6 +2058,11 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         if constexpr (MLA) mla_combine_input(p, t, ub, ub + p.xs_floats, ctid);
         if (ctid == 0) *rn_s = 1.f;
         cur_key = -1;
+      } else if (F8 && g.esz == 1 && (key != cur_key || key < 0)) {
+        float rnv[1];
+        if constexpr (F8) load_input_e4m3(p, t, g, ub, red, ctid, rnv);
+        if (ctid == 0) rn_s[0] = rnv[0];
+        cur_key = key;
       } else if (key != cur_key || key < 0) {
         float rnv[MT];
         load_input<MT, TILED>(p, t, g, ub, red, ctid, rnv);
@@ -2003,48 +2105,54 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
-        if (MT == 1 && !TILED && g.esz == 1) {  // E4M3 rows (rows of Kp bytes, K8 8-byte groups)
-          const uint2* s8 = reinterpret_cast<const uint2*>(sp);
+        if (F8 && g.esz == 1) {
+          // E4M3 rows on the tensor cores: mma.sync m16n8k16 (f16) with A = 8 weight rows
+          // (rows 0-7 of the tile; rows 8-15 zero) and B = the input's hi / lo columns (n = 0,
+          // 1; the rest zero).  An ldmatrix.x4 brings 64 columns of the 8 rows (E4M3 bytes
+          // read as 16-bit pairs: lane (g, t4) gets columns 4 t4 .. 4 t4 + 3 of row g of each
+          // 16-column block), converted in registers to f16 — columns 4 t4, + 1 as k 2 t4,
+          // + 1 and columns 4 t4 + 2, + 3 as k 2 t4 + 8, + 9, the order the input fragments
+          // follow.  Each 64 columns lie in one 128-column scale block: lane (g, 0) adds
+          // (hi + lo) * scale of row g.  Gate / up stages take 4 gate rows and the same 4 up
+          // rows per tile.
+          const uint32_t sb = smem_u32(ring + (size_t)slot * p.stage_bytes);
           const Fp8Scales fs = fp8_scales(p, t, g);
-          if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
-            const uint2* up = s8 + (size_t)g.rps * K8;
-            for (int r = 0; r < nr; r += 2) {
-              const int np = min(2, nr - r), n = n0 + r, n1 = n0 + r + np - 1;
-              float o0, o1, o2, o3;
-              const uint2* g0 = s8 + (size_t)r * K8;
-              const uint2* u0 = up + (size_t)r * K8;
-              if (np == 2) {
-                gemv_rows_fp8<4, 1>(g0, g0 + K8, u0, u0 + K8, fp8_scale_row(fs, 0, n),
-                                    fp8_scale_row(fs, 0, n1), fp8_scale_row(fs, 1, n),
-                                    fp8_scale_row(fs, 1, n1), K8, g.k0, xl, xh, lane, o0, o1, o2, o3);
-              } else {
-                const float* sg = fp8_scale_row(fs, 0, n);
-                const float* su = fp8_scale_row(fs, 1, n);
-                gemv_rows_fp8<2, 2>(g0, u0, u0, u0, sg, su, su, su, K8, g.k0, xl, xh, lane, o0,
-                                    o1, o2, o3);
+          const int P = fp8_row_pitch(g.Kp), K64 = (g.Kp + 63) / 64 * 64;
+          const int gq = lane >> 2, t4 = lane & 3;
+          const uint2* bfr = reinterpret_cast<const uint2*>(ub);
+          const bool two = g.nseg == 2;
+          const int step = two ? 4 : 8;
+          for (int r = 0; r < nr; r += step) {
+            const int nv = min(step, nr - r);
+            const int i = lane & 7;  // tile row this lane addresses for ldmatrix
+            const int seg_i = two ? i >> 2 : 0, ri = r + min(two ? (i & 3) : i, nv - 1);
+            const uint32_t arow = sb + (uint32_t)((seg_i * g.rps + ri) * P + (lane >> 3) * 16);
+            const int seg_q = two ? gq >> 2 : 0;
+            const float* srow = fp8_scale_row(fs, seg_q, n0 + r + min(two ? (gq & 3) : gq, nv - 1));
+            float tot = 0.f;
+            for (int c = 0; c < K64; c += 64) {
+              uint32_t w[4];
+              ldsm_x4(arow + (uint32_t)c, w[0], w[1], w[2], w[3]);
+              float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int m = 0; m < 4; ++m) {
+                const bool in = c + 16 * m + 4 * t4 < g.Kp;  // columns past Kp: zero
+                const uint32_t a[4] = {in ? e4m3x2_to_f16x2(w[m]) : 0u, 0u,
+                                       in ? e4m3x2_to_f16x2(w[m] >> 16) : 0u, 0u};
+                uint2 b = make_uint2(0u, 0u);
+                if (gq < 2) b = bfr[(((c >> 4) + m) * 2 + gq) * 4 + t4];
+                mma_f16(d, a, b.x, b.y);
               }
-              const float v = reduce4(o0, o1, o2, o3, lane);
-              const float upv = __shfl_xor_sync(0xffffffffu, v, np == 2 ? 16 : 8);
-              const int k = (lane >> 3) & 1;
-              if ((np == 2 && (lane & 23) == 0) || (np == 1 && lane == 0)) {
-                const float a = v * rn, bb = upv * rn;
-                p.u[uoff + n0 + r + k] = wsel * (a / (1.f + expf(-a)) * bb);
-              }
+              tot = fmaf(d[0] + d[1], __ldg(srow + ((g.k0 + c) >> 7)), tot);
             }
-          } else {
-            for (int r = 0; r < nr; r += 4) {
-              const int nv = min(4, nr - r), n = n0 + r;
-              const uint2* r0 = s8 + (size_t)r * K8;
-              float o0, o1, o2, o3;
-              gemv_rows_fp8_n(nv, r0, r0 + (size_t)min(1, nv - 1) * K8,
-                              r0 + (size_t)min(2, nv - 1) * K8, r0 + (size_t)min(3, nv - 1) * K8,
-                              fp8_scale_row(fs, 0, n), fp8_scale_row(fs, 0, n + min(1, nv - 1)),
-                              fp8_scale_row(fs, 0, n + min(2, nv - 1)),
-                              fp8_scale_row(fs, 0, n + min(3, nv - 1)), K8, g.k0, xl, xh, lane,
-                              o0, o1, o2, o3);
-              const float v = reduce4(o0, o1, o2, o3, lane);
-              const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-              if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
+            if (two) {
+              const float upv = __shfl_sync(0xffffffffu, tot, ((gq + 4) & 7) * 4);
+              if (t4 == 0 && gq < nv) {
+                const float a = tot * rn, bb = upv * rn;
+                p.u[uoff + n0 + r + gq] = wsel * (a / (1.f + expf(-a)) * bb);
+              }
+            } else if (t4 == 0 && gq < nv) {
+              gemv_emit(p, t, g, n0 + r + gq, tot, rn, resid, best[0]);
             }
           }
         } else if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
@@ -2184,7 +2292,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
 }
 
 // ---- the kernel ----------------------------------------------------------------------------------
-template <bool MLA, int MT, bool TILED>
+template <bool MLA, int MT, bool TILED, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t NS = (uint32_t)p.ring_stages;
@@ -2229,14 +2337,16 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
              reinterpret_cast<const volatile int*>(misc + 80), threadIdx.x & 31);
     return;
   }
-  consumer<MLA, MT, TILED>(p, my, ntask, ring, full, empty, tags, ub, misc);
+  consumer<MLA, MT, TILED, F8>(p, my, ntask, ring, full, empty, tags, ub, misc);
 }
 
 // ---- host-side launch helpers ------------------------------------------------------------------
-// The kernel instantiation for a stack kind, a number of tokens per step and the GEMV
-// stage form (tiled: multi-token tensor-core tiles).
-static const void* kernel_for(bool mla, int m, bool tiled) {
+// The kernel instantiation for a stack kind, a number of tokens per step, the GEMV stage
+// form (tiled: multi-token tensor-core tiles) and the weight format (fp8: E4M3 projections
+// on the tensor cores; their own instantiation keeps the bf16 kernel's registers as they are).
+static const void* kernel_for(bool mla, int m, bool tiled, bool fp8 = false) {
   if (mla) return reinterpret_cast<const void*>(engine_kernel<true, 1, false>);
+  if (fp8) return reinterpret_cast<const void*>(engine_kernel<false, 1, false, true>);
   if (tiled) {
     switch (m) {
       case 2: return reinterpret_cast<const void*>(engine_kernel<false, 2, true>);
@@ -2258,7 +2368,8 @@ static const void* kernel_for(bool mla, int m, bool tiled) {
 // function shared by every engine in the process, so it is raised to the device maximum
 // (never lowered to this plan's need: an engine created later must not shrink what an
 // earlier one launches with).
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled) {
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled,
+                             bool fp8) {
   *blocks_per_sm = 1 << 30;
   int dev = 0, optin = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
@@ -2266,8 +2377,8 @@ cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int m
     e0 = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e0 != cudaSuccess) return e0;
   const int limit = optin > smem_bytes ? optin : smem_bytes;
-  for (int m = 1; m <= (mla ? 1 : max_m); ++m) {
-    const void* k = kernel_for(mla, m, tiled);
+  for (int m = 1; m <= (mla || fp8 ? 1 : max_m); ++m) {
+    const void* k = kernel_for(mla, m, tiled, fp8);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
     if (e != cudaSuccess) return e;
     int b = 0;
@@ -2293,7 +2404,8 @@ cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_
   cfg.attrs = attr;
   cfg.numAttrs = p.op_group >= 0 ? 0 : 1;
   void* args[] = {const_cast<Params*>(&p)};
-  const cudaError_t e = cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0), args);
+  const cudaError_t e =
+      cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0, p.wfp8 != 0), args);
   if (e != cudaSuccess) cudaGetLastError();  // returned here: do not leave it to the caller
   return e;
 }

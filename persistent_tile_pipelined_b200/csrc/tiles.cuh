@@ -2,6 +2,8 @@
 // of one shared-memory ring stage (the stage layout matches issue_stage() in engine.cu).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "tre_internal.h"
@@ -100,98 +102,13 @@ __device__ __forceinline__ void gemv_rows_n(int nr, const uint4* r0, const uint4
   }
 }
 
-// ---- GEMV over E4M3 rows with 128 x 128 block scales ----------------------------------------
-// The binary32 whose sign, exponent and mantissa fields are the sign, 4 exponent and 3
-// mantissa bits of the E4M3 byte held in bits 24-31 of w: an arithmetic shift right by 4
-// moves them to bits 31 / 23-26 / 20-22 (the sign copies that land in bits 27-30 are
-// masked off).  Its value is exactly the byte's E4M3 value times 2^-120 (E4M3 exponent bias
-// 7 against binary32's 127; E4M3 subnormals land on binary32 subnormals, which the FMA
-// keeps), so a dot product over such floats is scaled by 2^120 afterwards.  The E4M3 NaN
-// bytes (S.1111.111) decode as finite numbers.
-__device__ __forceinline__ float e4m3_top_byte(uint32_t w) {
-  return __int_as_float((static_cast<int32_t>(w) >> 4) & static_cast<int32_t>(0x87F00000u));
-}
-
-// 2^-120 * sum_k e4m3(W[k]) x[k] over 8 E4M3 weights (bytes 0-3 of w.x, then of w.y; element
-// k in byte k % 4); x split in planes a = x[0:4], b = x[4:8].
-__device__ __forceinline__ float dot8_e4m3(const uint2 w, const float4 a, const float4 b) {
-  float acc = e4m3_top_byte(w.x << 24) * a.x;
-  acc = fmaf(e4m3_top_byte(w.x << 16), a.y, acc);
-  acc = fmaf(e4m3_top_byte(w.x << 8), a.z, acc);
-  acc = fmaf(e4m3_top_byte(w.x), a.w, acc);
-  acc = fmaf(e4m3_top_byte(w.y << 24), b.x, acc);
-  acc = fmaf(e4m3_top_byte(w.y << 16), b.y, acc);
-  acc = fmaf(e4m3_top_byte(w.y << 8), b.z, acc);
-  acc = fmaf(e4m3_top_byte(w.y), b.w, acc);
-  return acc;
-}
-
-// One warp computes NR (<= 4) whole E4M3 rows of a stage: rows[r] points at row r's K8
-// 8-byte groups in shared memory; sc[r] at the row's block-scale row (fp32, global, one per
-// 128 input columns); k0 is the first input column of this K-part.  Each lane's 8-column
-// group lies inside one 128-column block, whose scale (times 2^120) weighs the group's
-// partial sum.
-template <int NR, int NACC>
-__device__ __forceinline__ void gemv_rows_fp8(const uint2* r0, const uint2* r1, const uint2* r2,
-                                              const uint2* r3, const float* s0, const float* s1,
-                                              const float* s2, const float* s3, int K8, int k0,
-                                              const float4* __restrict__ xl,
-                                              const float4* __restrict__ xh, int lane, float& o0,
-                                              float& o1, float& o2, float& o3) {
-  const uint2* rp[4] = {r0, r1, r2, r3};
-  const float* sp[4] = {s0, s1, s2, s3};
-  float acc[NR][NACC];
-#pragma unroll
-  for (int r = 0; r < NR; ++r)
-#pragma unroll
-    for (int a = 0; a < NACC; ++a) acc[r][a] = 0.f;
-  int j = lane;
-#pragma unroll 2
-  for (; j + 32 * (NACC - 1) < K8; j += 32 * NACC) {
-#pragma unroll
-    for (int a = 0; a < NACC; ++a) {
-      const int jj = j + 32 * a, blk = (k0 + 8 * jj) >> 7;
-      const float4 x0 = xl[jj], x1 = xh[jj];
-#pragma unroll
-      for (int r = 0; r < NR; ++r)
-        acc[r][a] = fmaf(dot8_e4m3(rp[r][jj], x0, x1), __ldg(sp[r] + blk) * 0x1p120f, acc[r][a]);
-    }
-  }
-  for (; j < K8; j += 32) {
-    const int blk = (k0 + 8 * j) >> 7;
-    const float4 x0 = xl[j], x1 = xh[j];
-#pragma unroll
-    for (int r = 0; r < NR; ++r)
-      acc[r][0] = fmaf(dot8_e4m3(rp[r][j], x0, x1), __ldg(sp[r] + blk) * 0x1p120f, acc[r][0]);
-  }
-  float out[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    float v = 0.f;
-    if (r < NR) {
-#pragma unroll
-      for (int a = 0; a < NACC; ++a) v += acc[r][a];
-    }
-    out[r] = v;
-  }
-  o0 = out[0];
-  o1 = out[1];
-  o2 = out[2];
-  o3 = out[3];
-}
-
-__device__ __forceinline__ void gemv_rows_fp8_n(int nr, const uint2* r0, const uint2* r1,
-                                                const uint2* r2, const uint2* r3, const float* s0,
-                                                const float* s1, const float* s2, const float* s3,
-                                                int K8, int k0, const float4* xl, const float4* xh,
-                                                int lane, float& o0, float& o1, float& o2,
-                                                float& o3) {
-  switch (nr) {
-    case 4: gemv_rows_fp8<4, 1>(r0, r1, r2, r3, s0, s1, s2, s3, K8, k0, xl, xh, lane, o0, o1, o2, o3); break;
-    case 3: gemv_rows_fp8<3, 1>(r0, r1, r2, r3, s0, s1, s2, s3, K8, k0, xl, xh, lane, o0, o1, o2, o3); break;
-    case 2: gemv_rows_fp8<2, 2>(r0, r1, r2, r3, s0, s1, s2, s3, K8, k0, xl, xh, lane, o0, o1, o2, o3); break;
-    default: gemv_rows_fp8<1, 4>(r0, r1, r2, r3, s0, s1, s2, s3, K8, k0, xl, xh, lane, o0, o1, o2, o3); break;
-  }
+// ---- E4M3 weights on the tensor cores ---------------------------------------------------------
+// Two E4M3 bytes (bits 0-7 and 8-15 of v) as f16x2, the lower byte in the low half: exact —
+// every E4M3 number, subnormals included, is an f16 number.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
+  const __half2_raw h =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xffffu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
 // ---- GEMV for MT tokens: one warp computes NR (<= 4) whole rows against MT input vectors -----

@@ -17,7 +17,8 @@
 #include "tre_internal.h"
 
 namespace tre {
-cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled);
+cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled,
+                             bool fp8 = false);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 const char* last_error_cstr();
@@ -284,7 +285,8 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   }
 
   int bps = 0;
-  CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M, s.tiles != 0));
+  CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M, s.tiles != 0,
+                      s.wfp8 != 0));
   if (bps < 1) {
     set_error("tre_create: the persistent CTA does not fit on an SM");
     return TRE_ERR_OCCUPANCY;
