@@ -2059,9 +2059,11 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         if (ctid == 0) *rn_s = 1.f;
         cur_key = -1;
       } else if (F8 && g.esz == 1 && (key != cur_key || key < 0)) {
-        float rnv[1];
-        if constexpr (F8) load_input_e4m3(p, t, g, ub, red, ctid, rnv);
-        if (ctid == 0) rn_s[0] = rnv[0];
+        if constexpr (F8) {
+          float rnv[1];
+          load_input_e4m3(p, t, g, ub, red, ctid, rnv);
+          if (ctid == 0) rn_s[0] = rnv[0];
+        }
         cur_key = key;
       } else if (key != cur_key || key < 0) {
         float rnv[MT];
