@@ -737,11 +737,11 @@ __device__ __forceinline__ int input_key(const Task& t) {
 // (x[c0], x[c0 + 1]) and (x[c0 + 2], x[c0 + 3]) of c0 = 16 s + 4 t4 as f16x2 — part 0 the
 // f16 rounding hi of each x, part 1 the rounding of x - hi (about 22 significand bits in
 // all).  The A fragments take the weights' columns in the same order.  Columns from Kp up
-// to the next multiple of 64 are zero.  An |x| of 65504 or more (beyond f16) records a
+// to the end of the 4 row segments (fp8_span) are zero.  An |x| of 65504 or more (beyond f16) records a
 // bounds error.  rn receives the RMSNorm scale (1 when the op has no norm).
 __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
                                 float* red, int ctid, float* rn) {
-  const int K = gg.Kp, NG = ((K + 63) / 64 * 64) / 4;  // 4-column groups
+  const int K = gg.Kp, NG = fp8_span(K) / 4;  // 4-column groups
   const float* src = nullptr;
   const uint16_t* src_bf = nullptr;
   const uint16_t* gain = nullptr;
@@ -2108,54 +2108,86 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
         if (F8 && g.esz == 1) {
-          // E4M3 rows on the tensor cores: mma.sync m16n8k16 (f16) with A = 8 weight rows
-          // (rows 0-7 of the tile; rows 8-15 zero) and B = the input's hi / lo columns (n = 0,
-          // 1; the rest zero).  An ldmatrix.x4 brings 64 columns of the 8 rows (E4M3 bytes
-          // read as 16-bit pairs: lane (g, t4) gets columns 4 t4 .. 4 t4 + 3 of row g of each
-          // 16-column block), converted in registers to f16 — columns 4 t4, + 1 as k 2 t4,
-          // + 1 and columns 4 t4 + 2, + 3 as k 2 t4 + 8, + 9, the order the input fragments
-          // follow.  Each 64 columns lie in one 128-column scale block: lane (g, 0) adds
-          // (hi + lo) * scale of row g.  Gate / up stages take 4 gate rows and the same 4 up
-          // rows per tile.
+          // E4M3 rows on the tensor cores, mma.sync m16n8k16 (f16 in, fp32 accumulate).  A
+          // tile is 4 weight rows, each cut into 4 segments of L columns: tile row
+          // 4 j + q (j < 2) is segment q of weight row j, tile row 8 + 4 j + q segment q of row
+          // 2 + j; column n of the input operand is segment n / 2 of the input, hi part for
+          // even n, lo part for odd.  So D[4 j + q][2 q] + D[4 j + q][2 q + 1] is segment q of
+          // row j's dot product (the other products are discarded), held by lane
+          // (g = 4 j + q, t4 = q).  An ldmatrix.x4 brings 32 columns of all 16 tile rows (E4M3
+          // bytes read as 16-bit pairs: lane (g, t4) gets columns 4 t4 .. 4 t4 + 3 of each
+          // 16-column block), converted in registers to f16 — columns 4 t4, + 1 as k 2 t4, + 1
+          // and 4 t4 + 2, + 3 as k 2 t4 + 8, + 9, the order the input fragments follow.  32
+          // columns lie in one 128-column scale block; the segments are summed with shuffles.
+          // Gate / up tiles take gate rows r, r + 1 as rows 0, 1 and the same up rows as 2, 3.
           const uint32_t sb = smem_u32(ring + (size_t)slot * p.stage_bytes);
           const Fp8Scales fs = fp8_scales(p, t, g);
-          const int P = fp8_row_pitch(g.Kp), K64 = (g.Kp + 63) / 64 * 64;
-          const int gq = lane >> 2, t4 = lane & 3;
+          const int P = fp8_row_pitch(g.Kp), Ls = fp8_seg_len(g.Kp);
+          const int gq = lane >> 2, t4 = lane & 3, qs = gq & 3;
+          const bool mine = t4 == qs;             // this lane holds a useful segment sum
           const uint2* bfr = reinterpret_cast<const uint2*>(ub);
           const bool two = g.nseg == 2;
-          const int step = two ? 4 : 8;
+          const int step = two ? 2 : 4;           // weight rows per tile and segment
+          // ldmatrix row addresses: matrix lane >> 3 (0: tile rows 0-7, 1: rows 8-15, 2 / 3 the
+          // same 16 columns further), tile row lane & 7
+          const int mat = lane >> 3, trow = (mat & 1) * 8 + (lane & 7);
+          const int tj = (trow >> 3) * 2 + ((trow & 7) >> 2), tq = trow & 3;
           for (int r = 0; r < nr; r += step) {
             const int nv = min(step, nr - r);
-            const int i = lane & 7;  // tile row this lane addresses for ldmatrix
-            const int seg_i = two ? i >> 2 : 0, ri = r + min(two ? (i & 3) : i, nv - 1);
-            const uint32_t arow = sb + (uint32_t)((seg_i * g.rps + ri) * P + (lane >> 3) * 16);
-            const int seg_q = two ? gq >> 2 : 0;
-            const float* srow = fp8_scale_row(fs, seg_q, n0 + r + min(two ? (gq & 3) : gq, nv - 1));
-            float tot = 0.f;
-            for (int c = 0; c < K64; c += 64) {
+            // weight row of tile row index jj (0..3) and its stage slot
+            auto slot_row = [&](int jj) {
+              if (two) return (jj >> 1) * g.rps + r + min(jj & 1, nv - 1);  // gate, gate, up, up
+              return r + min(jj, nv - 1);
+            };
+            auto weight_row = [&](int jj, int& seg) {
+              seg = two ? jj >> 1 : 0;
+              return n0 + r + min(two ? (jj & 1) : jj, nv - 1);
+            };
+            const uint32_t arow = sb + (uint32_t)(slot_row(tj) * P + tq * Ls + (mat >> 1) * 16);
+            int sg0, sg1;
+            const int wr0 = weight_row(gq >> 2, sg0), wr1 = weight_row(2 + (gq >> 2), sg1);
+            const float* srow0 = fp8_scale_row(fs, sg0, wr0);
+            const float* srow1 = fp8_scale_row(fs, sg1, wr1);
+            float tot0 = 0.f, tot1 = 0.f;
+            for (int c = 0; c < Ls; c += 32) {
               uint32_t w[4];
               ldsm_x4(arow + (uint32_t)c, w[0], w[1], w[2], w[3]);
-              float d[4] = {0.f, 0.f, 0.f, 0.f};
+              float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int m = 0; m < 4; ++m) {
-                const bool in = c + 16 * m + 4 * t4 < g.Kp;  // columns past Kp: zero
-                const uint32_t a[4] = {in ? e4m3x2_to_f16x2(w[m]) : 0u, 0u,
-                                       in ? e4m3x2_to_f16x2(w[m] >> 16) : 0u, 0u};
-                uint2 b = make_uint2(0u, 0u);
-                if (gq < 2) b = bfr[(((c >> 4) + m) * 2 + gq) * 4 + t4];
-                mma_f16(d, a, b.x, b.y);
+              for (int j = 0; j < 2; ++j) {
+                // this lane's A columns: segment qs of its rows, columns c + 16 j + 4 t4 ..
+                const bool in = qs * Ls + c + 16 * j + 4 * t4 < g.Kp;
+                const uint32_t lo = w[2 * j], hi = w[2 * j + 1];
+                const uint32_t a[4] = {in ? e4m3x2_to_f16x2(lo) : 0u, in ? e4m3x2_to_f16x2(hi) : 0u,
+                                       in ? e4m3x2_to_f16x2(lo >> 16) : 0u,
+                                       in ? e4m3x2_to_f16x2(hi >> 16) : 0u};
+                const uint2 b = bfr[((((gq >> 1) * Ls + c) >> 4) + j) * 8 + (gq & 1) * 4 + t4];
+                mma_f16(j ? d1 : d0, a, b.x, b.y);
               }
-              tot = fmaf(d[0] + d[1], __ldg(srow + ((g.k0 + c) >> 7)), tot);
-            }
-            if (two) {
-              const float upv = __shfl_sync(0xffffffffu, tot, ((gq + 4) & 7) * 4);
-              if (t4 == 0 && gq < nv) {
-                const float a = tot * rn, bb = upv * rn;
-                p.u[uoff + n0 + r + gq] = wsel * (a / (1.f + expf(-a)) * bb);
+              if (mine) {
+                const int blk = (g.k0 + qs * Ls + c) >> 7;
+                tot0 = fmaf((d0[0] + d0[1]) + (d1[0] + d1[1]), __ldg(srow0 + blk), tot0);
+                tot1 = fmaf((d0[2] + d0[3]) + (d1[2] + d1[3]), __ldg(srow1 + blk), tot1);
               }
-            } else if (t4 == 0 && gq < nv) {
-              gemv_emit(p, t, g, n0 + r + gq, tot, rn, resid, best[0]);
             }
+            // sum the 4 segments: lanes 16 j + 5 q hold segment q of rows j (tot0), 2 + j (tot1)
+            float v0 = mine ? tot0 : 0.f, v1 = mine ? tot1 : 0.f;
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1) {
+              v0 += __shfl_xor_sync(0xffffffffu, v0, off);
+              v1 += __shfl_xor_sync(0xffffffffu, v1, off);
+            }
+            const int jrow = lane >> 4;  // lanes 0 / 16 emit rows jrow and 2 + jrow
+            if ((lane & 15) == 0 && jrow < (two ? nv : min(2, nv))) {
+              if (two) {  // rows: gate jrow (v0), up jrow (v1)
+                const float a = v0 * rn, bb = v1 * rn;
+                p.u[uoff + n0 + r + jrow] = wsel * (a / (1.f + expf(-a)) * bb);
+              } else {
+                gemv_emit(p, t, g, n0 + r + jrow, v0, rn, resid, best[0]);
+              }
+            }
+            if (!two && (lane & 15) == 0 && 2 + jrow < nv)
+              gemv_emit(p, t, g, n0 + r + 2 + jrow, v1, rn, resid, best[0]);
           }
         } else if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;

@@ -365,8 +365,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   for (auto& o : ops) {
     const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max),
                                                gemv_part_align(s.tiles, o.esz == 1));
-    // E4M3 rows: the tensor-core operand of the input covers the row rounded up to 64
-    xs = std::max(xs, o.esz == 1 ? (kp + 63) / 64 * 64 : kp);
+    // E4M3 rows: the tensor-core operand of the input covers the 4 row segments
+    xs = std::max(xs, o.esz == 1 ? fp8_span(kp) : kp);
     need = std::max(need, s.tiles ? kTileRows * kTilePitch
                                   : o.esz == 1 ? o.nseg * fp8_row_pitch(kp) : o.nseg * kp * o.esz);
   }

@@ -57,10 +57,14 @@ TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes, int esz 
 // K-part boundaries: multiples of 8 columns (16 bytes of bf16), of 16 for tensor-core
 // tiles, of 128 for E4M3 rows (a K-part then covers whole 128-column scale blocks)
 TRE_HD inline int gemv_part_align(bool tiles, bool fp8) { return fp8 ? 128 : tiles ? 16 : 8; }
-// E4M3 rows sit in a stage at this pitch (bytes): the row rounded up to 64 columns (the
-// tensor-core loop reads 64 columns at a time) plus 16 bytes, so that the 8 rows an
-// ldmatrix reads fall on 8 different 16-byte bank groups
-TRE_HD inline int fp8_row_pitch(int Kp) { return (Kp + 63) / 64 * 64 + 16; }
+// E4M3 rows on the tensor cores are read as 4 segments of fp8_seg_len(Kp) columns (a
+// multiple of 32: the loop takes 32 columns of every segment at a time); the input operand
+// covers the 4 segments (fp8_span columns, zero past Kp).  Rows sit in a stage at a pitch
+// of the span plus 16 bytes, so that the 8 rows an ldmatrix reads fall on 8 different
+// 16-byte bank groups.
+TRE_HD inline int fp8_seg_len(int Kp) { return ((Kp + 3) / 4 + 31) / 32 * 32; }
+TRE_HD inline int fp8_span(int Kp) { return 4 * fp8_seg_len(Kp); }
+TRE_HD inline int fp8_row_pitch(int Kp) { return fp8_span(Kp) + 16; }
 TRE_HD inline int fp8_rows_per_stage(int Kp, int nseg, int stage_bytes) {
   const int r = stage_bytes / (nseg * fp8_row_pitch(Kp));
   return r < 1 ? 1 : r;
