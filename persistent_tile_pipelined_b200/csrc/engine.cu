@@ -47,7 +47,10 @@ constexpr long long kCheckCycles = 1 << 15;
 // GEMV input staging: items each thread fetches before storing any (tensor-core fragments;
 // fp32 planes).
 constexpr int kLoadBatch = 2;
-constexpr int kPlaneBatch = 2;
+#ifndef TRE_PLANE_BATCH
+#define TRE_PLANE_BATCH 2
+#endif
+constexpr int kPlaneBatch = TRE_PLANE_BATCH;
 
 // Wait until counter `idx` reaches epoch * count (wrap-safe).  Bounded; on expiry the
 // error names `detail` (a task index).  A kernel-per-op launch never waits: the launches
@@ -732,9 +735,10 @@ __device__ __forceinline__ int input_key(const Task& t) {
 }
 
 // The input of a GEMV over E4M3 rows (one token) as the B operand of mma.sync m16n8k16
-// (f16 in, fp32 accumulate), in fragment order: column c of the K-part belongs to k-step
-// s = c / 16 and column group t4 = (c % 16) / 4, and entry [s][part][t4] (8 bytes) holds
-// (x[c0], x[c0 + 1]) and (x[c0 + 2], x[c0 + 3]) of c0 = 16 s + 4 t4 as f16x2 — part 0 the
+// (f16 in, fp32 accumulate), in fragment order: column c of the K-part lies in row segment
+// q = c / Ls at local k-step sl and column group t4, and entry [q][sl][part][t4] (8 bytes;
+// segments fp8_frag_seg_bytes apart) holds (x[c0], x[c0 + 1]) and (x[c0 + 2], x[c0 + 3]) of
+// the group's first column c0 as f16x2 — part 0 the
 // f16 rounding hi of each x, part 1 the rounding of x - hi (about 22 significand bits in
 // all).  The A fragments take the weights' columns in the same order.  Columns from Kp up
 // to the end of the 4 row segments (fp8_span) are zero.  An |x| of 65504 or more (beyond f16) records a
@@ -742,6 +746,7 @@ __device__ __forceinline__ int input_key(const Task& t) {
 __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
                                 float* red, int ctid, float* rn) {
   const int K = gg.Kp, NG = fp8_span(K) / 4;  // 4-column groups
+  const int Ls = fp8_seg_len(K), segb = fp8_frag_seg_bytes(K);
   const float* src = nullptr;
   const uint16_t* src_bf = nullptr;
   const uint16_t* gain = nullptr;
@@ -759,7 +764,6 @@ __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& 
   if (src) src += gg.k0;
   float ss = 0.f;
   bool bad = false;
-  uint2* fr = reinterpret_cast<uint2*>(ub);
   constexpr int B = 4;  // groups a thread fetches before it stores any
   for (int q0 = ctid; q0 < NG; q0 += B * kConsumerThreads) {
     float4 xv[B];
@@ -794,11 +798,13 @@ __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& 
       const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
       const __half2 l01 = __floats2half2_rn(e[0] - f01.x, e[1] - f01.y);
       const __half2 l23 = __floats2half2_rn(e[2] - f23.x, e[3] - f23.y);
-      const int sidx = q >> 2, t4 = q & 3;
-      fr[(sidx * 2 + 0) * 4 + t4] = make_uint2(*reinterpret_cast<const uint32_t*>(&h01),
-                                               *reinterpret_cast<const uint32_t*>(&h23));
-      fr[(sidx * 2 + 1) * 4 + t4] = make_uint2(*reinterpret_cast<const uint32_t*>(&l01),
-                                               *reinterpret_cast<const uint32_t*>(&l23));
+      // column 4 q of the K-part: segment sg, local k-step sl, column group t4
+      const int col = 4 * q, sg = col / Ls, cl = col - sg * Ls, sl = cl >> 4, t4 = (cl >> 2) & 3;
+      uint2* e0 = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(ub) + sg * segb) + sl * 8 + t4;
+      e0[0] = make_uint2(*reinterpret_cast<const uint32_t*>(&h01),
+                         *reinterpret_cast<const uint32_t*>(&h23));
+      e0[4] = make_uint2(*reinterpret_cast<const uint32_t*>(&l01),
+                         *reinterpret_cast<const uint32_t*>(&l23));
     }
   }
   if (bad) record_error(p, TRE_ERR_BOUNDS, t.id);
@@ -2125,7 +2131,9 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
           const int P = fp8_row_pitch(g.Kp), Ls = fp8_seg_len(g.Kp);
           const int gq = lane >> 2, t4 = lane & 3, qs = gq & 3;
           const bool mine = t4 == qs;             // this lane holds a useful segment sum
-          const uint2* bfr = reinterpret_cast<const uint2*>(ub);
+          // this lane's B column n = gq: segment gq / 2, part gq % 2
+          const uint2* bseg = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(ub) +
+                                                             (gq >> 1) * fp8_frag_seg_bytes(g.Kp));
           const bool two = g.nseg == 2;
           const int step = two ? 2 : 4;           // weight rows per tile and segment
           // ldmatrix row addresses: matrix lane >> 3 (0: tile rows 0-7, 1: rows 8-15, 2 / 3 the
@@ -2161,13 +2169,13 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
                 const uint32_t a[4] = {in ? e4m3x2_to_f16x2(lo) : 0u, in ? e4m3x2_to_f16x2(hi) : 0u,
                                        in ? e4m3x2_to_f16x2(lo >> 16) : 0u,
                                        in ? e4m3x2_to_f16x2(hi >> 16) : 0u};
-                const uint2 b = bfr[((((gq >> 1) * Ls + c) >> 4) + j) * 8 + (gq & 1) * 4 + t4];
+                const uint2 b = bseg[((c >> 4) + j) * 8 + (gq & 1) * 4 + t4];
                 mma_f16(j ? d1 : d0, a, b.x, b.y);
               }
               if (mine) {
                 const int blk = (g.k0 + qs * Ls + c) >> 7;
-                tot0 = fmaf((d0[0] + d0[1]) + (d1[0] + d1[1]), __ldg(srow0 + blk), tot0);
-                tot1 = fmaf((d0[2] + d0[3]) + (d1[2] + d1[3]), __ldg(srow1 + blk), tot1);
+                tot0 = fmaf((d0[0] + d0[1]) + (d1[0] + d1[1]), __ldg(srow0 + blk) * kE4M3Unit, tot0);
+                tot1 = fmaf((d0[2] + d0[3]) + (d1[2] + d1[3]), __ldg(srow1 + blk) * kE4M3Unit, tot1);
               }
             }
             // sum the 4 segments: lanes 16 j + 5 q hold segment q of rows j (tot0), 2 + j (tot1)
