@@ -734,19 +734,20 @@ __device__ __forceinline__ int input_key(const Task& t) {
   return (((int)t.layer * 8 + cls) << 8) | part;
 }
 
-// The input of a GEMV over E4M3 rows (one token) as the B operand of mma.sync m16n8k16
-// (f16 in, fp32 accumulate), in fragment order: column c of the K-part lies in row segment
-// q = c / Ls at local k-step sl and column group t4, and entry [q][sl][part][t4] (8 bytes;
-// segments fp8_frag_seg_bytes apart) holds (x[c0], x[c0 + 1]) and (x[c0 + 2], x[c0 + 3]) of
-// the group's first column c0 as f16x2 — part 0 the
-// f16 rounding hi of each x, part 1 the rounding of x - hi (about 22 significand bits in
-// all).  The A fragments take the weights' columns in the same order.  Columns from Kp up
-// to the end of the 4 row segments (fp8_span) are zero.  An |x| of 65504 or more (beyond f16) records a
-// bounds error.  rn receives the RMSNorm scale (1 when the op has no norm).
+// The input of a GEMV over E4M3 rows (one token) as the B operand of mma.sync m16n8k32
+// E4M3.  Each input x (times its gain) becomes 4 E4M3 terms: with 2^sg the power of two
+// that brings the largest |x| of its 32-column chunk into [128, 256),
+// x 2^sg ~ t0 + t1 / 16 + t2 / 256 + t3 / 4096, each term the nearest E4M3 number to what
+// the earlier ones left, times 16 (about 16 significand bits in all).  Fragment order:
+// column c of the K-part lies in row segment q = c / Ls, 32-column chunk cc = (c % Ls) / 32,
+// half h and column group t4 (c % 32 = 16 h + 4 t4 + i), and the 4 bytes of term tau for
+// (q, cc, h, t4) sit at byte q 4 Ls + cc 128 + tau 32 + t4 8 + h 4 (a lane reads its term's
+// two halves as one 8-byte word, a warp's 32 words two 128-byte rows).  After the 4
+// segments: 2^-sg per chunk (span / 32 floats).  Columns past Kp are zero.  rn receives
+// the RMSNorm scale (1 when the op has no norm).
 __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
                                 float* red, int ctid, float* rn) {
-  const int K = gg.Kp, NG = fp8_span(K) / 4;  // 4-column groups
-  const int Ls = fp8_seg_len(K), segb = fp8_frag_seg_bytes(K);
+  const int K = gg.Kp, Ls = fp8_seg_len(K), span = 4 * Ls, NG = span / 4;  // 4-column groups
   const float* src = nullptr;
   const uint16_t* src_bf = nullptr;
   const uint16_t* gain = nullptr;
@@ -762,10 +763,11 @@ __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& 
     default: src = p.u; break;  // OP_DOWN
   }
   if (src) src += gg.k0;
+  uint8_t* fr = reinterpret_cast<uint8_t*>(ub);
+  float* cs = ub + span;
   float ss = 0.f;
-  bool bad = false;
   constexpr int B = 4;  // groups a thread fetches before it stores any
-  for (int q0 = ctid; q0 < NG; q0 += B * kConsumerThreads) {
+  for (int q0 = ctid; q0 < NG; q0 += B * kConsumerThreads) {  // warp-uniform trip count
     float4 xv[B];
     uint2 gv[B];
 #pragma unroll
@@ -781,10 +783,10 @@ __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& 
     }
 #pragma unroll
     for (int u = 0; u < B; ++u) {
-      const int q = q0 + u * kConsumerThreads;
-      if (q >= NG) break;
+      const int q = q0 + u * kConsumerThreads, col = 4 * q;
+      const bool live = col < K;  // (all lanes run the shuffles below)
       float e[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-      if (4 * q >= K) {
+      if (!live) {
         e[0] = e[1] = e[2] = e[3] = 0.f;
       } else if (gain) {
 #pragma unroll
@@ -792,22 +794,31 @@ __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& 
         e[0] *= bf_lo(gv[u].x); e[1] *= bf_hi(gv[u].x);
         e[2] *= bf_lo(gv[u].y); e[3] *= bf_hi(gv[u].y);
       }
+      // the chunk's largest |x| (its 8 groups sit on 8 consecutive lanes)
+      float am = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+      int sg = 0;
+      if (am > 0.f && am < INFINITY)
+        sg = min(100, max(-100, 7 - (((int)(__float_as_uint(am) >> 23) & 0xff) - 127)));
+      const float up = __int_as_float((127 + sg) << 23);  // 2^sg, exact
+      float y[4] = {e[0] * up, e[1] * up, e[2] * up, e[3] * up};
+      if (q < NG) {
+        const int sgm = col / Ls, cl = col - sgm * Ls;
+        uint8_t* dst = fr + sgm * 4 * Ls + (cl >> 5) * 128 + ((cl >> 2) & 3) * 8 + ((cl >> 4) & 1) * 4;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) bad |= !(fabsf(e[k]) < 65504.f) && !isnan(e[k]);
-      const __half2 h01 = __floats2half2_rn(e[0], e[1]), h23 = __floats2half2_rn(e[2], e[3]);
-      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-      const __half2 l01 = __floats2half2_rn(e[0] - f01.x, e[1] - f01.y);
-      const __half2 l23 = __floats2half2_rn(e[2] - f23.x, e[3] - f23.y);
-      // column 4 q of the K-part: segment sg, local k-step sl, column group t4
-      const int col = 4 * q, sg = col / Ls, cl = col - sg * Ls, sl = cl >> 4, t4 = (cl >> 2) & 3;
-      uint2* e0 = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(ub) + sg * segb) + sl * 8 + t4;
-      e0[0] = make_uint2(*reinterpret_cast<const uint32_t*>(&h01),
-                         *reinterpret_cast<const uint32_t*>(&h23));
-      e0[4] = make_uint2(*reinterpret_cast<const uint32_t*>(&l01),
-                         *reinterpret_cast<const uint32_t*>(&l23));
+        for (int tau = 0; tau < 4; ++tau) {
+          const uint32_t w01 = f2_to_e4m3x2(y[0], y[1]), w23 = f2_to_e4m3x2(y[2], y[3]);
+          *reinterpret_cast<uint32_t*>(dst + tau * 32) = w01 | (w23 << 16);
+          const float2 b01 = e4m3x2_to_f2(w01), b23 = e4m3x2_to_f2(w23);
+          y[0] = (y[0] - b01.x) * 16.f; y[1] = (y[1] - b01.y) * 16.f;
+          y[2] = (y[2] - b23.x) * 16.f; y[3] = (y[3] - b23.y) * 16.f;
+        }
+        if ((col & 31) == 0) cs[col >> 5] = __int_as_float((127 - sg) << 23);  // 2^-sg
+      }
     }
   }
-  if (bad) record_error(p, TRE_ERR_BOUNDS, t.id);
   if (gain) {
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -2114,35 +2125,36 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
         if (F8 && g.esz == 1) {
-          // E4M3 rows on the tensor cores, mma.sync m16n8k16 (f16 in, fp32 accumulate).  A
-          // tile is 4 weight rows, each cut into 4 segments of L columns: tile row
-          // 4 j + q (j < 2) is segment q of weight row j, tile row 8 + 4 j + q segment q of row
-          // 2 + j; column n of the input operand is segment n / 2 of the input, hi part for
-          // even n, lo part for odd.  So D[4 j + q][2 q] + D[4 j + q][2 q + 1] is segment q of
-          // row j's dot product (the other products are discarded), held by lane
-          // (g = 4 j + q, t4 = q).  An ldmatrix.x4 brings 32 columns of all 16 tile rows (E4M3
-          // bytes read as 16-bit pairs: lane (g, t4) gets columns 4 t4 .. 4 t4 + 3 of each
-          // 16-column block), converted in registers to f16 — columns 4 t4, + 1 as k 2 t4, + 1
-          // and 4 t4 + 2, + 3 as k 2 t4 + 8, + 9, the order the input fragments follow.  32
-          // columns lie in one 128-column scale block; the segments are summed with shuffles.
-          // Gate / up tiles take gate rows r, r + 1 as rows 0, 1 and the same up rows as 2, 3.
+          // E4M3 rows on the tensor cores, mma.sync m16n8k32 E4M3 x E4M3 -> fp32, the weights
+          // as stored (no conversion).  A tile is 4 weight rows, each cut into 4 segments of
+          // Ls columns: tile row 4 j + q (j < 2) is segment q of weight row j, tile row
+          // 8 + 4 j + q segment q of row 2 + j.  Two mma per 32 columns, n-tile 0 with the
+          // input terms of segments 0, 1 as columns (column 4 s + tau: segment s, term tau),
+          // n-tile 1 with segments 2, 3; lane (g, t4) of the n-tile holding its segment
+          // keeps terms 2 (t4 & 1) and + 1 when t4 / 2 = q % 2 (the other products are
+          // discarded).  An ldmatrix.x4 of 32 columns of the 16 tile rows is exactly the A
+          // fragment.  32 columns lie in one 128-column scale block and one input chunk: the
+          // lane weighs its terms by 16^-tau, the block scale and the chunk's 2^-sg; the
+          // segments and terms are summed with shuffles.  Gate / up tiles take gate rows
+          // r, r + 1 as rows 0, 1 and the same up rows as 2, 3.
           const uint32_t sb = smem_u32(ring + (size_t)slot * p.stage_bytes);
           const Fp8Scales fs = fp8_scales(p, t, g);
           const int P = fp8_row_pitch(g.Kp), Ls = fp8_seg_len(g.Kp);
           const int gq = lane >> 2, t4 = lane & 3, qs = gq & 3;
-          const bool mine = t4 == qs;             // this lane holds a useful segment sum
-          // this lane's B column n = gq: segment gq / 2, part gq % 2
-          const uint2* bseg = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(ub) +
-                                                             (gq >> 1) * fp8_frag_seg_bytes(g.Kp));
+          const bool mine = (t4 >> 1) == (qs & 1);
+          const float wa = (t4 & 1) ? 1.f / 256.f : 1.f, wb = wa * (1.f / 16.f);
+          const uint8_t* frb = reinterpret_cast<const uint8_t*>(ub);
+          const float* csc = ub + 4 * Ls;
+          const uint8_t* bp0 = frb + ((gq >> 2) * 4 * Ls + (gq & 3) * 32 + t4 * 8);
+          const uint8_t* bp1 = bp0 + 2 * 4 * Ls;
           const bool two = g.nseg == 2;
-          const int step = two ? 2 : 4;           // weight rows per tile and segment
+          const int step = two ? 2 : 4;           // weight rows per tile
           // ldmatrix row addresses: matrix lane >> 3 (0: tile rows 0-7, 1: rows 8-15, 2 / 3 the
-          // same 16 columns further), tile row lane & 7
+          // same rows 16 columns further), tile row lane & 7
           const int mat = lane >> 3, trow = (mat & 1) * 8 + (lane & 7);
           const int tj = (trow >> 3) * 2 + ((trow & 7) >> 2), tq = trow & 3;
           for (int r = 0; r < nr; r += step) {
             const int nv = min(step, nr - r);
-            // weight row of tile row index jj (0..3) and its stage slot
             auto slot_row = [&](int jj) {
               if (two) return (jj >> 1) * g.rps + r + min(jj & 1, nv - 1);  // gate, gate, up, up
               return r + min(jj, nv - 1);
@@ -2158,27 +2170,27 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
             const float* srow1 = fp8_scale_row(fs, sg1, wr1);
             float tot0 = 0.f, tot1 = 0.f;
             for (int c = 0; c < Ls; c += 32) {
-              uint32_t w[4];
-              ldsm_x4(arow + (uint32_t)c, w[0], w[1], w[2], w[3]);
-              float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                // this lane's A columns: segment qs of its rows, columns c + 16 j + 4 t4 ..
-                const bool in = qs * Ls + c + 16 * j + 4 * t4 < g.Kp;
-                const uint32_t lo = w[2 * j], hi = w[2 * j + 1];
-                const uint32_t a[4] = {in ? e4m3x2_to_f16x2(lo) : 0u, in ? e4m3x2_to_f16x2(hi) : 0u,
-                                       in ? e4m3x2_to_f16x2(lo >> 16) : 0u,
-                                       in ? e4m3x2_to_f16x2(hi >> 16) : 0u};
-                const uint2 b = bseg[((c >> 4) + j) * 8 + (gq & 1) * 4 + t4];
-                mma_f16(j ? d1 : d0, a, b.x, b.y);
-              }
+              uint32_t a[4];
+              ldsm_x4(arow + (uint32_t)c, a[0], a[1], a[2], a[3]);
+              // weight bytes past Kp are stale shared memory: zero them (the input is zero there)
+              const int colA = qs * Ls + c + 4 * t4;
+              if (colA >= g.Kp) a[0] = a[1] = 0u;
+              if (colA + 16 >= g.Kp) a[2] = a[3] = 0u;
+              const uint2 b0 = *reinterpret_cast<const uint2*>(bp0 + (c >> 5) * 128);
+              const uint2 b1 = *reinterpret_cast<const uint2*>(bp1 + (c >> 5) * 128);
+              float d0[4], d1[4];
+              mma_e4m3(d0, a, b0.x, b0.y);
+              mma_e4m3(d1, a, b1.x, b1.y);
               if (mine) {
-                const int blk = (g.k0 + qs * Ls + c) >> 7;
-                tot0 = fmaf((d0[0] + d0[1]) + (d1[0] + d1[1]), __ldg(srow0 + blk) * kE4M3Unit, tot0);
-                tot1 = fmaf((d0[2] + d0[3]) + (d1[2] + d1[3]), __ldg(srow1 + blk) * kE4M3Unit, tot1);
+                const float* dd = (qs >> 1) ? d1 : d0;
+                const int col = qs * Ls + c;
+                const float cscale = csc[col >> 5];
+                const int blk = (g.k0 + col) >> 7;
+                tot0 = fmaf(fmaf(dd[1], wb, dd[0] * wa), __ldg(srow0 + blk) * cscale, tot0);
+                tot1 = fmaf(fmaf(dd[3], wb, dd[2] * wa), __ldg(srow1 + blk) * cscale, tot1);
               }
             }
-            // sum the 4 segments: lanes 16 j + 5 q hold segment q of rows j (tot0), 2 + j (tot1)
+            // sum the segments and terms: the 16 lanes of half j hold rows j (tot0), 2 + j (tot1)
             float v0 = mine ? tot0 : 0.f, v1 = mine ? tot1 : 0.f;
 #pragma unroll
             for (int off = 1; off < 16; off <<= 1) {
@@ -2188,8 +2200,8 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
             const int jrow = lane >> 4;  // lanes 0 / 16 emit rows jrow and 2 + jrow
             if ((lane & 15) == 0 && jrow < (two ? nv : min(2, nv))) {
               if (two) {  // rows: gate jrow (v0), up jrow (v1)
-                const float a = v0 * rn, bb = v1 * rn;
-                p.u[uoff + n0 + r + jrow] = wsel * (a / (1.f + expf(-a)) * bb);
+                const float aa = v0 * rn, bb = v1 * rn;
+                p.u[uoff + n0 + r + jrow] = wsel * (aa / (1.f + expf(-aa)) * bb);
               } else {
                 gemv_emit(p, t, g, n0 + r + jrow, v0, rn, resid, best[0]);
               }

@@ -312,7 +312,10 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // so that the input planes leave room for a 5-deep ring of 36 KB stages; with M tokens
   // per step the M input vectors share the planes
   s.M = c.max_tokens_per_step < 1 ? 1 : c.max_tokens_per_step;
-  s.kpart_max = mla ? 8192 : (kMaxKPart / s.M) / 16 * 16;  // 16: tile k-steps
+  // E4M3 plans: K-parts of at most 8192 columns, so that a long row (the down projection)
+  // leaves 4 rows to a stage and its input operand leaves room for the ring
+  s.kpart_max = mla || c.weight_format == TRE_WEIGHTS_FP8_BLOCK128
+                    ? 8192 : (kMaxKPart / s.M) / 16 * 16;  // 16: tile k-steps
   // multi-token GEMV form: tensor-core tiles cost the same per stage whatever the token
   // count, CUDA-core rows grow with it (measured on the 8B-shaped stack: rows faster at 2
   // and 3 tokens, tiles at 4)
@@ -375,7 +378,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   int sb = c.stage_bytes ? c.stage_bytes : std::max(kDefaultStageBytes, (need + 1023) / 1024 * 1024);
   // E4M3 plans: a stage of 8 hidden-wide rows (two full 4-row tensor-core tiles; gate / up:
   // 4 row pairs) when that is at least the default
-  if (!c.stage_bytes && s.wfp8 && 8 * fp8_row_pitch(s.d) >= sb) sb = 8 * fp8_row_pitch(s.d);
+  if (!c.stage_bytes && s.wfp8 && 8 * fp8_row_pitch(s.d) >= sb)
+    sb = (8 * fp8_row_pitch(s.d) + 1023) / 1024 * 1024;  // ring slots stay 1024-byte aligned
   if (!c.stage_bytes)
     while (sb < need && sb < kMaxStageBytes) sb += 1024;
   if (sb < need)

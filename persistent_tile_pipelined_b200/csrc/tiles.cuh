@@ -103,27 +103,16 @@ __device__ __forceinline__ void gemv_rows_n(int nr, const uint4* r0, const uint4
 }
 
 // ---- E4M3 weights on the tensor cores ---------------------------------------------------------
-// Two E4M3 bytes (bits 0-7 and 8-15 of v) as f16x2, the lower byte in the low half, exact
-// (every E4M3 number, subnormals included, is an f16 number).  Two ways: the conversion
-// instruction, or (TRE_E4M3_BITS) placing the byte's sign / exponent / mantissa bits into
-// the f16 fields with integer operations, which yields the value times 2^-8 (E4M3 exponent
-// bias 7 against f16's 15; E4M3 subnormals land on f16 subnormals) — the caller then scales
-// by kE4M3Unit.
-#ifndef TRE_E4M3_BITS
-#define TRE_E4M3_BITS 0
-#endif
-constexpr float kE4M3Unit = TRE_E4M3_BITS ? 256.f : 1.f;
-
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
-#if TRE_E4M3_BITS
-  uint32_t p;  // byte 0 -> bits 8-15, byte 1 -> bits 24-31
-  asm("prmt.b32 %0, %1, 0, 0x1404;" : "=r"(p) : "r"(v));
-  return ((p & 0x7F007F00u) >> 1) | (p & 0x80008000u);
-#else
+// f32 -> E4M3 (nearest, saturating) for two values, the first in the low byte; and back.
+__device__ __forceinline__ uint32_t f2_to_e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t v) {
   const __half2_raw h =
       __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xffffu), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-#endif
+  __half2 hh;
+  *reinterpret_cast<__half2_raw*>(&hh) = h;
+  return __half22float2(hh);
 }
 
 // ---- GEMV for MT tokens: one warp computes NR (<= 4) whole rows against MT input vectors -----
