@@ -58,13 +58,14 @@ _SCALE_SLOTS = {"sq": 9, "sk": 10, "sv": 11, "so": 12, "sgate": 13, "sup": 14, "
 class _MlaConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("hidden", "n_heads", "q_lora", "kv_lora",
                                                "rope_dim", "nope_dim", "v_dim", "kv_capacity")] + [
-        ("rope_theta", ctypes.c_double), ("norm_eps", ctypes.c_double)]
+        ("rope_theta", ctypes.c_double), ("norm_eps", ctypes.c_double)] + [
+        (n, ctypes.c_int32) for n in ("index_heads", "index_dim", "index_topk")]
 
 
 class _MlaLayer(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("attn_norm", "w_dq", "q_norm", "w_uq", "w_dkv", "kv_norm", "w_uk", "w_uv", "w_o",
-                 "latent_cache")]
+                 "latent_cache", "w_iq", "w_ik", "index_cache")]
 
 
 def _ptr(a: np.ndarray) -> ctypes.c_void_p:
@@ -108,6 +109,9 @@ class Oracle:
         L.orc_swiglu_mlp.argtypes = [i32, i32, vp, vp, vp, vp, vp]
         L.orc_router_topk.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
         L.orc_mla_layer_step.argtypes = [vp, vp, i32, vp]
+        L.orc_mla_layer_step_ex.argtypes = [vp, vp, i32, vp, vp, i32, vp, vp]
+        L.orc_index_select.argtypes = [i32, i32, vp, vp]
+        L.orc_index_select.restype = i32
 
     # -- pieces ------------------------------------------------------------------
     def _r(self, a) -> np.ndarray:
@@ -256,18 +260,47 @@ class Oracle:
             return h1 + y, idx, w, scores
         return h1 + y, idx, w
 
-    def mla_layer_step(self, wl, layer: dict, latent_cache, pos: int, x):
-        """One absorbed-MLA layer (attention only); appends this token's latent row."""
+    def index_select(self, scores, k: int):
+        """The k positions of largest score (ties to the lower position), increasing."""
+        sc = self._r(scores)
+        out = np.empty(max(1, min(k, sc.size)), dtype=np.int32)
+        n = self.lib.orc_index_select(sc.size, int(k), _ptr(sc), _ptr(out))
+        return out[:n]
+
+    def mla_layer_step(self, wl, layer: dict, latent_cache, pos: int, x, index_cache=None,
+                       sel=None, want_index: bool = False):
+        """One absorbed-MLA layer (attention only); appends this token's latent row (and, with
+        the sparse indexer, its index key).  sel (positions, increasing) overrides the
+        indexer's choice.  want_index: also return (index scores [pos + 1], chosen positions)."""
+        topk = getattr(wl, "index_topk", 0)
         cfg = _MlaConfig(wl.hidden, wl.n_q_heads, wl.q_lora, wl.kv_lora, wl.rope_dim,
                          wl.nope_dim, wl.v_dim, wl.kv_capacity, float(wl.rope_theta),
-                         float(wl.norm_eps))
+                         float(wl.norm_eps), getattr(wl, "index_heads", 0),
+                         getattr(wl, "index_dim", 0), topk)
         L = _MlaLayer()
         for slot, name in enumerate(("attn_norm", "w_dq", "q_norm", "w_uq", "w_dkv", "kv_norm",
                                      "w_uk", "w_uv", "w_o")):
             setattr(L, name, _ptr(layer[slot]).value)
         L.latent_cache = _ptr(latent_cache).value
+        P = pos + 1
+        iscore = np.empty(P, dtype=self.real)
+        chosen = np.empty(max(1, min(P, topk)) if topk else 1, dtype=np.int32)
+        sel_arr = None
+        if topk:
+            assert index_cache is not None
+            L.w_iq = _ptr(layer[9]).value
+            L.w_ik = _ptr(layer[10]).value
+            L.index_cache = _ptr(index_cache).value
+            if sel is not None:
+                sel_arr = np.ascontiguousarray(sel, dtype=np.int32)
         x = self._r(x).copy()
-        self.lib.orc_mla_layer_step(ctypes.byref(cfg), ctypes.byref(L), int(pos), _ptr(x))
+        self.lib.orc_mla_layer_step_ex(ctypes.byref(cfg), ctypes.byref(L), int(pos), _ptr(x),
+                                       _ptr(sel_arr) if sel_arr is not None else None,
+                                       int(sel_arr.size) if sel_arr is not None else 0,
+                                       _ptr(iscore) if topk else None,
+                                       _ptr(chosen) if topk else None)
+        if want_index:
+            return x, (iscore if topk else None), (chosen[:min(P, topk)] if topk else None)
         return x
 
     def layers_step(self, wl, model, x, pos: int):

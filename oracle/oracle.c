@@ -343,6 +343,8 @@ void orc_router_topk(int E, int top_k, int d, const uint16_t* wr, const real* hn
 typedef struct {
   int32_t hidden, n_heads, q_lora, kv_lora, rope_dim, nope_dim, v_dim, kv_capacity;
   double rope_theta, norm_eps;
+  /* sparse attention (0 = dense): index heads H_I, index dim D_I, positions kept K */
+  int32_t index_heads, index_dim, index_topk;
 } orc_mla_config;
 
 typedef struct {
@@ -356,7 +358,47 @@ typedef struct {
   const uint16_t *w_uv;      /* [H * v][kv_lora]             */
   const uint16_t *w_o;       /* [d][H * v]                   */
   uint16_t *latent_cache;    /* [cap][kv_lora + rope] bf16   */
+  const uint16_t *w_iq;      /* sparse: [H_I * D_I][q_lora]  (index queries)          */
+  const uint16_t *w_ik;      /* sparse: [D_I + H_I][d]       (index key, head weights) */
+  uint16_t *index_cache;     /* sparse: [cap][D_I] bf16                               */
 } orc_mla_layer;
+
+/* The sparse-attention indexer (the pages: 64 index heads choose the top-2048 KV positions
+ * of a 160K context, TileRT code audit, sparse-index paragraph; weights named
+ * self_attn.indexer.* come with the DeepSeek-V3.2 checkpoint; no formula is printed): read
+ * as DeepSeek-V3.2's lightning indexer, with plain projections (no RoPE, no norm):
+ *   k_I = W_ik[0:D_I] xn (this position's index key, appended to the index cache as bf16),
+ *   w_I = W_ik[D_I:D_I+H_I] xn,  q_I = W_iq c_q (c_q after its RMSNorm),
+ *   I[t] = sum_j (w_I[j] / sqrt(H_I)) * ReLU(q_I[j] . k_I[t] / sqrt(D_I))  for t in [0, pos];
+ * the attention keeps the K positions of largest I (ties to the lower position; every
+ * position when pos + 1 <= K).  sel[] receives them in increasing order; returns their count. */
+static int cmp_score_desc(const void* a, const void* b) {
+  const real* x = (const real*)a;
+  const real* y = (const real*)b;
+  if (x[0] > y[0]) return -1;
+  if (x[0] < y[0]) return 1;
+  return (x[1] < y[1]) ? -1 : (x[1] > y[1]);  /* lower position first */
+}
+static int cmp_int(const void* a, const void* b) {
+  const int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+  return (x > y) - (x < y);
+}
+int orc_index_select(int P, int K, const real* score, int32_t* sel) {
+  if (P <= K) {
+    for (int t = 0; t < P; ++t) sel[t] = t;
+    return P;
+  }
+  real* pairs = (real*)malloc(sizeof(real) * 2 * (size_t)P);
+  for (int t = 0; t < P; ++t) {
+    pairs[2 * t] = score[t];
+    pairs[2 * t + 1] = (real)t;
+  }
+  qsort(pairs, (size_t)P, 2 * sizeof(real), cmp_score_desc);
+  for (int i = 0; i < K; ++i) sel[i] = (int32_t)pairs[2 * i + 1];
+  qsort(sel, (size_t)K, sizeof(int32_t), cmp_int);
+  free(pairs);
+  return K;
+}
 
 /* One absorbed multi-head latent attention layer (attention only) at position pos, residual
  * x[d] updated in place.  The pages name FlashSparseMLA (batch == 1) and TokenSpeed's
@@ -367,7 +409,21 @@ typedef struct {
  *   cache[pos] = bf16([c_kv, k_pe]);
  *   q_lat_h = W_uk,h^T q_nope_h;  s_h[t] = (q_lat_h . c_kv[t] + q_pe_h . k_pe[t]) / sqrt(nope+rope);
  *   o_lat_h = sum_t softmax(s_h)[t] c_kv[t];  o_h = W_uv,h o_lat_h;  x = x + W_o [o_h]. */
+/* The layer with the attention over a chosen set of positions.  Sparse configs compute the
+ * index scores into iscore_out ([pos + 1], may be NULL) and the chosen positions into
+ * sel_out ([K], may be NULL); sel_in (n_sel_in positions, increasing) overrides the choice
+ * when not NULL.  Dense configs (index_topk 0) attend to every position in [0, pos]. */
+void orc_mla_layer_step_ex(const orc_mla_config* c, const orc_mla_layer* L, int pos, real* x,
+                           const int32_t* sel_in, int n_sel_in, real* iscore_out,
+                           int32_t* sel_out);
+
 void orc_mla_layer_step(const orc_mla_config* c, const orc_mla_layer* L, int pos, real* x) {
+  orc_mla_layer_step_ex(c, L, pos, x, NULL, 0, NULL, NULL);
+}
+
+void orc_mla_layer_step_ex(const orc_mla_config* c, const orc_mla_layer* L, int pos, real* x,
+                           const int32_t* sel_in, int n_sel_in, real* iscore_out,
+                           int32_t* sel_out) {
   const int d = c->hidden, H = c->n_heads, QL = c->q_lora, KL = c->kv_lora, R = c->rope_dim;
   const int NP = c->nope_dim, VD = c->v_dim, QH = NP + R, C = KL + R, cap = c->kv_capacity;
   real* xn = (real*)malloc(sizeof(real) * d);
@@ -403,28 +459,71 @@ void orc_mla_layer_step(const orc_mla_config* c, const orc_mla_layer* L, int pos
         acc += bf16_val(L->w_uk[((size_t)h * NP + n) * KL + j]) * q[(size_t)h * QH + n];
       qlat[(size_t)h * KL + j] = acc;
     }
+  /* the positions attended: all of [0, pos], or the indexer's choice */
+  int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)P);
+  int NS = P;
+  for (int t = 0; t < P; ++t) sel[t] = t;
+  if (c->index_topk > 0) {
+    const int HI = c->index_heads, DI = c->index_dim;
+    real* ki = (real*)malloc(sizeof(real) * (size_t)(DI + HI));
+    real* qi = (real*)malloc(sizeof(real) * (size_t)HI * DI);
+    real* isc = (real*)malloc(sizeof(real) * (size_t)P);
+    orc_gemv(DI + HI, d, L->w_ik, xn, ki);
+    orc_gemv(HI * DI, QL, L->w_iq, cqn, qi);
+    uint16_t* irow = L->index_cache + (size_t)pos * DI;
+    for (int i = 0; i < DI; ++i) irow[i] = orc_round_bf16(ki[i]);
+    const double sq = 1.0 / sqrt((double)DI), sw = 1.0 / sqrt((double)HI);
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < P; ++t) {
+      const uint16_t* kt = L->index_cache + (size_t)t * DI;
+      real acc = 0;
+      for (int j = 0; j < HI; ++j) {
+        real dot = 0;
+        for (int i = 0; i < DI; ++i) dot += qi[(size_t)j * DI + i] * bf16_val(kt[i]);
+        dot *= (real)sq;
+        if (dot > 0) acc += ki[DI + j] * (real)sw * dot;
+      }
+      isc[t] = acc;
+    }
+    int32_t* mine = (int32_t*)malloc(sizeof(int32_t) * (size_t)P);
+    const int nm = orc_index_select(P, c->index_topk, isc, mine);
+    if (sel_out) memcpy(sel_out, mine, sizeof(int32_t) * (size_t)nm);
+    if (iscore_out) memcpy(iscore_out, isc, sizeof(real) * (size_t)P);
+    if (sel_in) {
+      NS = n_sel_in;
+      memcpy(sel, sel_in, sizeof(int32_t) * (size_t)n_sel_in);
+    } else {
+      NS = nm;
+      memcpy(sel, mine, sizeof(int32_t) * (size_t)nm);
+    }
+    free(ki); free(qi); free(isc); free(mine);
+  }
+
   const real scale = (real)(1.0 / sqrt((double)QH));
   for (int h = 0; h < H; ++h) {
     real m = -INFINITY;
-    for (int t = 0; t < P; ++t) {
+    for (int u = 0; u < NS; ++u) {
+      const int t = sel[u];
       const uint16_t* ct = L->latent_cache + (size_t)t * C;
       real a = 0;
       for (int j = 0; j < KL; ++j) a += qlat[(size_t)h * KL + j] * bf16_val(ct[j]);
       for (int j = 0; j < R; ++j) a += q[(size_t)h * QH + NP + j] * bf16_val(ct[KL + j]);
-      sc[t] = a * scale;
-      if (sc[t] > m) m = sc[t];
+      sc[u] = a * scale;
+      if (sc[u] > m) m = sc[u];
     }
     real l = 0;
-    for (int t = 0; t < P; ++t) {
-      sc[t] = (real)exp((double)(sc[t] - m));
-      l += sc[t];
+    for (int u = 0; u < NS; ++u) {
+      sc[u] = (real)exp((double)(sc[u] - m));
+      l += sc[u];
     }
     for (int j = 0; j < KL; ++j) {
       real acc = 0;
-      for (int t = 0; t < P; ++t) acc += sc[t] / l * bf16_val(L->latent_cache[(size_t)t * C + j]);
+      for (int u = 0; u < NS; ++u)
+        acc += sc[u] / l * bf16_val(L->latent_cache[(size_t)sel[u] * C + j]);
       olat[(size_t)h * KL + j] = acc;
     }
   }
+  free(sel);
   /* o_h = W_uv,h o_lat_h */
   for (int h = 0; h < H; ++h)
     orc_gemv(VD, KL, L->w_uv + (size_t)h * VD * KL, olat + (size_t)h * KL, o + (size_t)h * VD);

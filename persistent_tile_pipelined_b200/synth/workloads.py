@@ -39,6 +39,10 @@ class Workload:
     tokens_per_step: int = 1
     seed: int = 1234
     weight_format: str = "bf16"  # "fp8": GQA projections as E4M3 bytes + 128x128 block scales
+    # MLA sparse attention (0 = dense): index heads, index dim, positions kept per step
+    index_heads: int = 0
+    index_dim: int = 0
+    index_topk: int = 0
     # MLA
     q_lora: int = 0
     kv_lora: int = 0
@@ -100,8 +104,16 @@ LLAMA8B_KV128K = LLAMA8B.replace(name="llama3-8b-shaped-kv128k", prefill=131072)
 # embedding, norms and LM head stay bf16.
 LLAMA8B_FP8 = LLAMA8B.replace(name="llama3-8b-shaped-fp8", weight_format="fp8")
 
+# Absorbed-MLA layers x4 with the sparse-attention indexer (64 index heads of dim 128 keep
+# the top 2048 of 131072 cached positions: the pages' 160K-context setting), and the same
+# layers dense at that length for comparison.
+MLA4_SPARSE128K = MLA4.replace(name="mla-4L-d7168-sparse-kv128k", prefill=131072, index_heads=64,
+                               index_dim=128, index_topk=2048)
+MLA4_KV128K = MLA4.replace(name="mla-4L-d7168-kv128k", prefill=131072)
+
 WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L, MLA4, MOE4, LLAMA8B_KV8K,
-                                 LLAMA8B_KV32K, LLAMA8B_KV128K, LLAMA8B_FP8)}
+                                 LLAMA8B_KV32K, LLAMA8B_KV128K, LLAMA8B_FP8, MLA4_SPARSE128K,
+                                 MLA4_KV128K)}
 
 
 def gqa_layer_shapes(w: Workload) -> List[tuple]:
@@ -134,7 +146,10 @@ def mla_layer_shapes(w: Workload) -> List[tuple]:
         (6, (H * nope, kl), "w"),           # W_uk
         (7, (H * v, kl), "w"),              # W_uv
         (8, (d, H * v), "w"),               # W_o
-    ]
+    ] + ([
+        (9, (w.index_heads * w.index_dim, ql), "w"),      # indexer queries W_iq
+        (10, (w.index_dim + w.index_heads, d), "w"),      # indexer key rows, head-weight rows
+    ] if w.index_topk else [])
 
 
 def moe_layer_shapes(w: Workload) -> List[tuple]:
@@ -174,6 +189,12 @@ def gen_mla_model(w: Workload) -> dict:
         if w.prefill:
             cache[: w.prefill] = normal_bf16(w.seed, tid_kcache(l), (w.prefill, C), 0.0, 1.0)
         model["latent_cache"].append(cache)
+        if w.index_topk:  # the indexer's key cache [capacity][index_dim], N(0, 1) like the latents
+            icache = np.zeros((w.kv_capacity, w.index_dim), dtype=np.uint16)
+            if w.prefill:
+                icache[: w.prefill] = normal_bf16(w.seed, tid_vcache(l), (w.prefill, w.index_dim),
+                                                  0.0, 1.0)
+            model.setdefault("index_cache", []).append(icache)
     return model
 
 
