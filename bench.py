@@ -378,7 +378,16 @@ def workload_step_bytes(wl, pos=None) -> int:
         H, C = wl.n_q_heads, wl.kv_lora + wl.rope_dim
         w = ((wl.q_lora + C) * d + H * (wl.nope_dim + wl.rope_dim) * wl.q_lora +
              H * wl.nope_dim * wl.kv_lora + H * wl.v_dim * wl.kv_lora + d * H * wl.v_dim)
-        total = (w * 2 + (d + wl.q_lora + wl.kv_lora) * 2) * L + L * (pos + 1) * C * 2
+        HI, DI, KI = wl.index_heads, wl.index_dim, wl.index_topk
+        if KI:  # the indexer's projections
+            w += HI * DI * wl.q_lora + (DI + HI) * d
+        total = (w * 2 + (d + wl.q_lora + wl.kv_lora) * 2) * L
+        if KI and pos + 1 > KI:
+            # every index key read (+ this one written), the K chosen latent rows read and
+            # this position's latent row written
+            total += L * ((pos + 1) * DI * 2 + (KI + 1) * C * 2)
+        else:
+            total += L * (pos + 1) * C * 2 + (L * (pos + 1) * DI * 2 if KI else 0)
     else:
         Hq, Hkv, D = wl.n_q_heads, wl.n_kv_heads, wl.head_dim
         mlp = (wl.n_experts * d + 3 * (wl.n_shared + wl.top_k) * wl.expert_ffn * d

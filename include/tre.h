@@ -127,8 +127,23 @@ typedef struct {
                                    choice: tiles at 4 tokens per step when the sizes
                                    allow, else rows                                     */
   int32_t weight_format;        /* TRE_WEIGHTS_*: storage of the GQA projections        */
-  int32_t reserved[3];          /* must be zero                                         */
+  int32_t index_heads;          /* MLA sparse attention (index_topk > 0): H_I index heads,
+                                   16, 32 or 64                                         */
+  int32_t index_dim;            /* D_I, the index key width: 64 or 128                  */
+  int32_t index_topk;           /* K: positions each step attends to (0 = dense MLA)    */
 } tre_config;
+
+/* Sparse MLA (index_topk > 0; one token per step).  The pages give the sparse attention of
+ * a DeepSeek-V3.2-class model as 64 index heads that choose the top-2048 cached positions
+ * of a 160K context for the attention kernel (TileRT code audit, sparse-index paragraph)
+ * and print no formula; the indexer is read as DeepSeek-V3.2's lightning indexer with
+ * plain projections.  At position pos, with xn = RMSNorm(x) and c_q = RMSNorm(W_dq xn):
+ *   k_I = W_ik[0:D_I] xn (this position's index key, appended to the index cache as bf16),
+ *   w_I = W_ik[D_I:D_I+H_I] xn,  q_I = W_iq c_q (H_I heads of D_I),
+ *   I[t] = sum_j (w_I[j] / sqrt(H_I)) * ReLU(q_I[j] . k_I[t] / sqrt(D_I)),  t in [0, pos];
+ * the attention then runs over the K positions of largest I (ties to the lower position);
+ * when pos + 1 <= K that is every position.  The score of every position and the chosen
+ * set are kept per layer for tre_debug_index. */
 
 /* Weight formats (tre_config.weight_format).  BF16: every matrix bf16.  FP8_BLOCK128 (GQA
  * stacks, one token per step): the seven projection matrices of every layer (Q, K, V, O,
@@ -154,13 +169,16 @@ enum { TRE_WEIGHTS_BF16 = 0, TRE_WEIGHTS_FP8_BLOCK128 = 1 };
  *         then R rope rows), DKV[KL+R][d] (KL latent rows then R rope rows),
  *         KV_NORM[KL], UK[H*NP][KL], UV[H*VD][KL], MLA_O[d][H*VD]
  *         (QL = q_lora, KL = kv_lora, R = rope_dim, NP = nope_dim, VD = v_dim)
+ *   MLA sparse (index_topk > 0), also: INDEX_Q[H_I*D_I][QL] (the index queries W_iq),
+ *         INDEX_K[D_I+H_I][d] (D_I index-key rows, then H_I head-weight rows: W_ik)
  *   GQA with weight_format FP8_BLOCK128: slots 1-4 and 6-8 hold E4M3 bytes of the same
  *         shapes, and their fp32 block scales [ceil(N/128)][ceil(K/128)] sit in
  *         SCALE_Q .. SCALE_DOWN (slots 9-15)
  * KV caches (bf16, written at pos by every step, caller owned):
  *   GQA/MOE : k_cache[l], v_cache[l] = [Hkv][kv_capacity][D]
  *   MLA     : k_cache[l] = latent [kv_capacity][KL + R]: RMSNorm(c_kv) then RoPE(k_pe);
- *             v_cache unused (may be NULL)
+ *             v_cache unused (may be NULL); sparse: v_cache[l] = the index-key cache
+             [kv_capacity][D_I] bf16
  */
 enum {
   TRE_W_ATTN_NORM = 0, TRE_W_Q = 1, TRE_W_K = 2, TRE_W_V = 3, TRE_W_O = 4,
@@ -171,6 +189,7 @@ enum {
   TRE_W_UK = 6, TRE_W_UV = 7, TRE_W_MLA_O = 8,
   TRE_W_SCALE_Q = 9, TRE_W_SCALE_K = 10, TRE_W_SCALE_V = 11, TRE_W_SCALE_O = 12,
   TRE_W_SCALE_GATE = 13, TRE_W_SCALE_UP = 14, TRE_W_SCALE_DOWN = 15,
+  TRE_W_INDEX_Q = 9, TRE_W_INDEX_K = 10,
   TRE_W_SLOTS = 16
 };
 
@@ -328,6 +347,15 @@ tre_status tre_layers_step(tre_engine* e, const float* x_in_dev, float* x_out_de
  * [n_layers][top_k] (their normalised weights); either may be NULL.  Waits for the
  * engine's last stream.  TRE_ERR_UNSUPPORTED for other kinds. */
 tre_status tre_debug_routing(tre_engine* e, int32_t* idx_host, float* w_host);
+
+/* Sparse MLA: wait for the engine's last stream, then copy layer `layer`'s index scores
+ * of the last step (score_host: float[pos + 1], I[0 .. pos] as defined above, may be
+ * NULL) and its chosen positions (sel_host: int32[index_topk], in no particular order,
+ * may be NULL); *n_sel_out receives how many were chosen (min(pos + 1, K)).  pos is the
+ * position of that step.  TRE_ERR_INVALID_ARG for a dense engine or a layer or pos out
+ * of range. */
+tre_status tre_debug_index(tre_engine* e, int32_t layer, int32_t pos, float* score_host,
+                           int32_t* sel_host, int32_t* n_sel_out);
 
 /* Wait for the engine's last stream, then report the device status word: 0, or a
  * negative tre_status (TRE_ERR_DEP_TIMEOUT / TRE_ERR_BOUNDS).  *detail_out (may be

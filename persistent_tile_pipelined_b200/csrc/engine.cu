@@ -248,10 +248,20 @@ __device__ __forceinline__ const uint8_t* part_row(const Params& p, const Task& 
       return wbytes(L.w[t.op == OP_O ? TRE_W_O : TRE_W_DOWN]) + ((size_t)n * K + g.k0) * e;
     case OP_GU: return wbytes(L.w[seg ? TRE_W_UP : TRE_W_GATE]) + (size_t)n * K * e;
     case OP_ROUTER: return wbytes(L.w[TRE_W_ROUTER]) + (size_t)n * K * 2;
-    case OP_MDQKV:
+    case OP_MDQKV: {  // W_dq, W_dkv, then (sparse) W_ik
+      const int C = p.KL + p.R;
       if (n < p.QL) { *contig = p.QL - n; return wbytes(L.w[TRE_W_DQ]) + (size_t)n * K * 2; }
-      return wbytes(L.w[TRE_W_DKV]) + (size_t)(n - p.QL) * K * 2;
-    case OP_UQ: return wbytes(L.w[TRE_W_UQ]) + (size_t)n * K * 2;
+      if (n < p.QL + C) {
+        *contig = p.QL + C - n;
+        return wbytes(L.w[TRE_W_DKV]) + (size_t)(n - p.QL) * K * 2;
+      }
+      return wbytes(L.w[TRE_W_INDEX_K]) + (size_t)(n - p.QL - C) * K * 2;
+    }
+    case OP_UQ: {  // W_uq, then (sparse) W_iq
+      const int nq = p.Hq * (p.NP + p.R);
+      if (n < nq) { *contig = nq - n; return wbytes(L.w[TRE_W_UQ]) + (size_t)n * K * 2; }
+      return wbytes(L.w[TRE_W_INDEX_Q]) + (size_t)(n - nq) * K * 2;
+    }
     case OP_UK: return wbytes(L.w[TRE_W_UK]) + (size_t)n * K * 2;
     case OP_UV: return wbytes(L.w[TRE_W_UV]) + (size_t)n * K * 2;
     case OP_MO:
@@ -317,9 +327,28 @@ __device__ __forceinline__ const float* fp8_scale_row(const Fp8Scales& f, int se
   return f.base[2] + (size_t)((n - f.split[1]) >> 7) * f.KB;
 }
 
+// ---- sparse MLA ----------------------------------------------------------------------------------
+// A sparse plan's step attends to chosen positions once pos + 1 > K (before that, to all).
+__device__ __forceinline__ bool sparse_step(const Params& p) { return p.KI > 0 && p.pos + 1 > p.KI; }
+__device__ __forceinline__ uint32_t* index_meta(const Params& p, int layer) {
+  return p.ix_meta + (size_t)layer * IM_WORDS;
+}
+// Order key of a float: larger floats have larger keys (one key for -0 and +0 is the
+// caller's business).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Positions of a task's stages.  GQA attention: split sp of [0, pos) (the last split a
+// half share: it also takes the new positions); MLA attention: split sp of [0, pos), or
+// in a sparse step entries [t0, t1) of the layer's chosen positions (read once the
+// selection is published); index scoring: split sp of the cached positions [0, pos).
 __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& t0, int& t1) {
-  const long long P = p.pos;
+  long long P = p.pos;
   const long long S = t.aux, sp = t.r1;
+  if (t.type == T_MLA_ATTN && sparse_step(p))
+    P = min(__ldcg(index_meta(p, t.layer) + IM_NSEL), (uint32_t)p.KI);
   if (t.type == T_ATTN) {
     t0 = (int)(P * 2 * sp / (2 * S - 1));
     t1 = sp + 1 == S ? (int)P : (int)(P * 2 * (sp + 1) / (2 * S - 1));
@@ -332,9 +361,11 @@ __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& 
 template <bool TILED>
 __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
   if (t.type == T_GEMV) return gemv_geom<TILED>(p, t).nstages;
+  if (t.type == T_ISEL) return 0;
   int t0, t1;
   attn_range(p, t, t0, t1);
-  return (t1 - t0 + p.pps - 1) / p.pps;
+  const int rows = t.type == T_INDEX ? kIndexRows : p.pps;
+  return (t1 - t0 + rows - 1) / rows;
 }
 
 // Where a GEMV task's rows come from, resolved once per task (expert ids and layer
@@ -352,7 +383,7 @@ struct RowSrc {
 
 __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const GemvGeom& g) {
   RowSrc r;
-  r.lookup = t.op == OP_QKV || t.op == OP_MDQKV;
+  r.lookup = t.op == OP_QKV || t.op == OP_MDQKV || (t.op == OP_UQ && p.KI > 0);
   r.stride = (long long)g.K * g.esz;
   if (t.op == OP_RGU) r.stride = 2LL * p.d;
   else if (t.op == OP_MDOWN) r.stride = 2LL * (g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe);
@@ -367,10 +398,16 @@ __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const 
       r.base[2] = wbytes(L.w[TRE_W_V]);
       r.split[0] = p.Hq * p.D;
       r.split[1] = (p.Hq + p.Hkv) * p.D;
-    } else {
+    } else if (t.op == OP_MDQKV) {
       r.base[0] = wbytes(L.w[TRE_W_DQ]);
       r.base[1] = wbytes(L.w[TRE_W_DKV]);
+      r.base[2] = wbytes(L.w[TRE_W_INDEX_K]);  // sparse only (rows past QL + C)
       r.split[0] = p.QL;
+      r.split[1] = p.QL + p.KL + p.R;
+    } else {  // sparse q up-projection: W_uq rows, then W_iq rows
+      r.base[0] = wbytes(L.w[TRE_W_UQ]);
+      r.base[1] = wbytes(L.w[TRE_W_INDEX_Q]);
+      r.split[0] = p.Hq * (p.NP + p.R);
     }
     return r;
   }
@@ -433,8 +470,13 @@ __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, 
     const int nr = min(g.rps, t.r1 - (t.r0 + i * g.rps));
     return (uint32_t)(g.nseg * nr * g.Kp * g.esz);
   }
-  if (t.type == T_MLA_ATTN)  // whole boxes (rows past the cache are zero-filled)
+  if (t.type == T_INDEX) return (uint32_t)(p.DI * 2 * kIndexRows);  // whole boxes
+  if (t.type == T_MLA_ATTN) {
+    // sparse: every row of the stage is gathered (rows past the split repeat its first)
+    if (sparse_step(p)) return (uint32_t)(kMlaPosPerStage * (p.KL + p.R) * 2);
+    // whole boxes (rows past the cache are zero-filled)
     return (uint32_t)((p.KL + p.R) / kMlaBox * kMlaPosPerStage * 128);
+  }
   return (uint32_t)(2 * (p.D / 64) * p.pps * 128);  // K and V boxes of pps rows
 }
 
@@ -490,6 +532,26 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
         n += take;
       }
     }
+  } else if (t.type == T_INDEX) {
+    // 64-column boxes of kIndexRows index keys, 128-byte swizzled
+    if (lane < p.DI / 64) {
+      const uint8_t* map = static_cast<const uint8_t*>(p.ix_maps) + (size_t)t.layer * 128;
+      tma_load_2d(dst + (size_t)lane * kIndexRows * 128, map, lane * 64, t0 + i * kIndexRows, bar);
+    }
+  } else if (t.type == T_MLA_ATTN && sparse_step(p)) {
+    // gather: lane r copies the latent row of chosen entry t0 + 32 i + r (past the split:
+    // entry t0 again, so that the masked rows hold finite values) at the padded pitch
+    const int C = p.KL + p.R;
+    int j = t0 + i * kMlaPosPerStage + lane;
+    if (j >= t1) j = t0;
+    int pos = __ldcg(p.ix_sel + (size_t)t.layer * p.KI + j);
+    if (pos < 0 || pos >= p.pos) {
+      record_error(p, TRE_ERR_BOUNDS, t.id);
+      pos = 0;
+    }
+    bulk_g2s(dst + (size_t)lane * sparse_lat_pitch(C),
+             reinterpret_cast<const uint8_t*>(p.layers[t.layer].k_cache) + (size_t)pos * C * 2,
+             (uint32_t)C * 2u, bar, pol);
   } else if (t.type == T_MLA_ATTN) {
     // 64-column boxes of 32 latent rows, 128-byte swizzled (see mla.cuh)
     if (lane < (p.KL + p.R) / kMlaBox) {
@@ -613,6 +675,13 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
       if (!ok) break;
     }
+    if (t.type == T_MLA_ATTN && sparse_step(p)) {  // the chosen positions pick the rows
+      bool r = true;
+      if (lane == 0) r = wait_dep(p, t);
+      ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      __syncwarp();  // orders the other lanes' reads of the selection after lane 0's acquire
+    }
     if (window > 0 && ti + 1 < ntask) task_prefetch(p, my[ti + 1], lane, window);
     const int ns = task_nstages<TILED>(p, t);
     GemvGeom g{};
@@ -626,7 +695,11 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       // each lane that copies through a cache's tensor map acquires the map first (the
       // allocation-free entry point rewrites its maps in place between launches)
       const uint8_t* maps = static_cast<const uint8_t*>(p.kv_maps);
-      if (t.type == T_MLA_ATTN) {
+      if (t.type == T_INDEX) {
+        if (lane < p.DI / 64)
+          tensormap_acquire(static_cast<const uint8_t*>(p.ix_maps) + (size_t)t.layer * 128);
+      } else if (t.type == T_ISEL) {
+      } else if (t.type == T_MLA_ATTN) {
         if (lane < (p.KL + p.R) / kMlaBox) tensormap_acquire(maps + (size_t)t.layer * 128);
       } else if (lane < 2 * (p.D / 64)) {
         tensormap_acquire(maps + ((size_t)t.layer * 2 + (lane >= p.D / 64)) * 128);
@@ -1543,7 +1616,12 @@ __device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int n
                               int warp, int lane, int ctid, bool& ab) {
   constexpr int HG = kMlaHeadGroup, PS = kMlaPosPerStage, RP = 36;  // score row pitch (floats)
   const int KL = p.KL, C = KL + p.R, hg = t.r0, split = t.r1, S = t.aux;
-  const bool last = (split == S - 1);
+  // sparse step: the stage rows are the chosen positions' latent rows at a padded pitch,
+  // and the new position joins only when the indexer chose it
+  const bool sp = sparse_step(p);
+  const uint32_t LP = (uint32_t)sparse_lat_pitch(C);
+  const bool last = (split == S - 1) && (!sp || __ldcg(index_meta(p, t.layer) + IM_HASPOS) != 0u);
+  auto row_off = [&](int r, int ch) { return sp ? (uint32_t)r * LP + (uint32_t)ch * 16u : lat_off(r, ch); };
   float* red = ub;                                        // [8][16][RP] partial scores
   __nv_bfloat16* phi = reinterpret_cast<__nv_bfloat16*>(ub + kConsumerWarps * HG * RP);  // [16][40]
   __nv_bfloat16* plo = phi + HG * 40;                                                    // [16][40]
@@ -1609,7 +1687,7 @@ __device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int n
         for (int np = 0; np < 2; ++np) {   // n-tile pairs (rows 16 np .. 16 np + 15)
           const int m = lane >> 3, r = np * 16 + (m >> 1) * 8 + (lane & 7);
           uint32_t b0, b1, b2, b3;
-          ldsm_x4(tb + lat_off(r, ch + (m & 1)), b0, b1, b2, b3);
+          ldsm_x4(tb + row_off(r, ch + (m & 1)), b0, b1, b2, b3);
           mma_bf16(c[2 * np], ahi[j], b0, b1);
           mma_bf16(c[2 * np], alo[j], b0, b1);
           mma_bf16(c[2 * np + 1], ahi[j], b2, b3);
@@ -1691,7 +1769,7 @@ __device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int n
             const int r = ks * 16 + (m & 1) * 8 + (lane & 7);
             const int ch = (col0 + n * 8) / 8 + (m >> 1);
             uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(tb + lat_off(r, ch), b0, b1, b2, b3);
+            ldsm_x4_t(tb + row_off(r, ch), b0, b1, b2, b3);
             mma_bf16(o[n], ah, b0, b1);
             mma_bf16(o[n], al, b0, b1);
             mma_bf16(o[n + 1], ah, b2, b3);
@@ -1776,6 +1854,390 @@ __device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int n
   }
 }
 
+// ---- sparse MLA: index scoring and top-K selection ----------------------------------------------
+// Index scoring task = split sp of the cached positions [0, pos).  Per stage of kIndexRows
+// index keys: S[j][t] = q_I[j] . k_I[t] on the tensor cores (mma.sync m16n8k16, fp32
+// accumulation; the queries, rounded to bf16, as A from shared memory, 16 heads per
+// m-tile; the bf16 keys as B straight from the swizzled tile), then
+// I[t] = sum_j w'_j ReLU(S[j][t]) with w' = w_I / sqrt(H_I D_I).  Warp w takes the
+// stage's positions 16 w .. 16 w + 15 against every head, so ReLU, weights and the sum
+// over heads stay in the warp (per thread, then shuffles).  The scores go to
+// iscore[layer]; a shared histogram of their order keys' top bits is added into the
+// layer's global histogram.  The last split also scores the new position from its
+// on-chip key (rounded to bf16 as the cache holds it); the split that arrives last picks
+// the threshold bin (index_threshold).
+__device__ void index_threshold(const Params& p, const Task& t, float* scratch, int warp,
+                                int lane, int ctid);
+
+// Byte offset of 16-byte chunk c of row r of the [H_I][D_I] bf16 query tile (rows of
+// 2 D_I bytes, chunks XOR-swizzled by r & 7 so that ldmatrix reads 8 rows conflict-free).
+__device__ __forceinline__ uint32_t qtile_off(int r, int c, int DI) {
+  return (uint32_t)(r * DI * 2 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ void index_task(const Params& p, const Task& t, uint32_t gs, int ns, uint8_t* ring,
+                           uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
+                           int* tk, int warp, int lane, int ctid, bool& ab) {
+  const int HI = p.HI, DI = p.DI, MTI = HI / 16, KS = DI / 16;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ub);                   // [kIndexBins]
+  uint8_t* qt = reinterpret_cast<uint8_t*>(ub + kIndexBins);          // [H_I][D_I] bf16
+  float* wsc = ub + kIndexBins + kIndexMaxHeads * 128 / 2;            // [kIndexMaxHeads]
+  float* nsum = wsc + kIndexMaxHeads;                                 // [kConsumerWarps]
+  const int C = p.KL + p.R;
+  const float* qi = p.qkv + (size_t)p.Hq * (p.NP + p.R);  // q_I [H_I][D_I]
+  const float* kin = p.cqkv + p.QL + C;                    // k_I of this position [D_I]
+  const float* win = kin + DI;                             // w_I [H_I]
+  for (int b = ctid; b < kIndexBins; b += kConsumerThreads) hist[b] = 0u;
+  for (int e = ctid; e < HI * DI / 8; e += kConsumerThreads) {  // 8 columns per item
+    const int r = e / (DI / 8), c = e % (DI / 8);
+    const float4 x0 = __ldcg(reinterpret_cast<const float4*>(qi + (size_t)r * DI + 8 * c));
+    const float4 x1 = __ldcg(reinterpret_cast<const float4*>(qi + (size_t)r * DI + 8 * c + 4));
+    uint4 v;
+    v.x = bf2_bits(__floats2bfloat162_rn(x0.x, x0.y));
+    v.y = bf2_bits(__floats2bfloat162_rn(x0.z, x0.w));
+    v.z = bf2_bits(__floats2bfloat162_rn(x1.x, x1.y));
+    v.w = bf2_bits(__floats2bfloat162_rn(x1.z, x1.w));
+    *reinterpret_cast<uint4*>(qt + qtile_off(r, c, DI)) = v;
+  }
+  const float wnorm = 1.f / sqrtf((float)(HI * DI));
+  if (ctid < HI) wsc[ctid] = __ldcg(win + ctid) * wnorm;
+  consumer_sync(kConsumerThreads);
+  float wt[4][2];  // this thread's head weights: rows g8, g8 + 8 of every m-tile
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    wt[mt][0] = mt < MTI ? wsc[mt * 16 + g8] : 0.f;
+    wt[mt][1] = mt < MTI ? wsc[mt * 16 + g8 + 8] : 0.f;
+  }
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
+  float* score = p.iscore + (size_t)t.layer * p.cap;
+  int t0, t1;
+  attn_range(p, t, t0, t1);
+  const uint32_t NS = (uint32_t)p.ring_stages;
+  const uint32_t qb = smem_u32(qt);
+  const int m = lane >> 3;
+  const int rb = warp * 16 + (m >> 1) * 8 + (lane & 7);   // this lane's key row (ldmatrix)
+  const int ra = (m & 1) * 8 + (lane & 7);                // this lane's query row in an m-tile
+  for (int i = 0; i < ns; ++i) {
+    const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
+    const bool landed = stage_wait(p, full, tags, sidx);
+    const uint32_t tb = smem_u32(ring + (size_t)slot * p.stage_bytes);
+    float c[4][2][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) c[mt][n][k] = 0.f;
+    if (landed) {
+#pragma unroll 2
+      for (int j = 0; j < KS; ++j) {
+        uint32_t b0, b1, b2, b3;
+        const int chb = 2 * j + (m & 1);  // key chunk: k 0-7 (even) or 8-15 of the step
+        ldsm_x4(tb + swz_off(chb >> 3, rb, chb & 7, kIndexRows), b0, b1, b2, b3);
+        const int cha = 2 * j + (m >> 1);  // query chunk of matrices 2, 3: k 8-15
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          if (mt < MTI) {
+            uint32_t a[4];
+            ldsm_x4(qb + qtile_off(mt * 16 + ra, cha, DI), a[0], a[1], a[2], a[3]);
+            mma_bf16(c[mt][0], a, b0, b1);
+            mma_bf16(c[mt][1], a, b2, b3);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
+    }
+    if (__any_sync(0xffffffffu, !landed)) {  // one warp's view is enough to stop
+      ab = true;
+      break;
+    }
+    // ReLU, head weights, sum over the heads: positions 16 warp + 8 n + 2 t4 (+ 1)
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        v0 = fmaf(fmaxf(c[mt][n][0], 0.f), wt[mt][0], v0);
+        v0 = fmaf(fmaxf(c[mt][n][2], 0.f), wt[mt][1], v0);
+        v1 = fmaf(fmaxf(c[mt][n][1], 0.f), wt[mt][0], v1);
+        v1 = fmaf(fmaxf(c[mt][n][3], 0.f), wt[mt][1], v1);
+      }
+#pragma unroll
+      for (int off = 4; off <= 16; off <<= 1) {
+        v0 += __shfl_xor_sync(0xffffffffu, v0, off);
+        v1 += __shfl_xor_sync(0xffffffffu, v1, off);
+      }
+      if (g8 == 0) {
+        const int tt = t0 + i * kIndexRows + warp * 16 + 8 * n + 2 * t4;
+        if (tt < t1) {
+          const float sc = v0 == 0.f ? 0.f : v0;  // -0 and +0 are one score
+          score[tt] = sc;
+          atomicAdd(hist + (order_key(sc) >> (32 - kIndexBinBits)), 1u);
+        }
+        if (tt + 1 < t1) {
+          const float sc = v1 == 0.f ? 0.f : v1;
+          score[tt + 1] = sc;
+          atomicAdd(hist + (order_key(sc) >> (32 - kIndexBinBits)), 1u);
+        }
+      }
+    }
+  }
+  // every warp must agree on an abort before the barriers below
+  if (consumer_sync_or(ab, kConsumerThreads)) {
+    ab = true;
+    return;
+  }
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
+  if (t.r1 == t.aux - 1) {  // the new position, from its key on chip
+    float part = 0.f;
+    for (int h = warp; h < HI; h += kConsumerWarps) {
+      float d = 0.f;
+      for (int k = lane; k < DI; k += 32) {
+        const float q = __bfloat162float(__float2bfloat16_rn(__ldcg(qi + (size_t)h * DI + k)));
+        d = fmaf(q, __bfloat162float(__float2bfloat16_rn(__ldcg(kin + k))), d);
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      part = fmaf(fmaxf(d, 0.f), wsc[h], part);
+    }
+    if (lane == 0) nsum[warp] = part;
+    consumer_sync(kConsumerThreads);
+    if (ctid == 0) {
+      float sc = 0.f;
+      for (int w = 0; w < kConsumerWarps; ++w) sc += nsum[w];
+      if (sc == 0.f) sc = 0.f;
+      score[p.pos] = sc;
+      atomicAdd(hist + (order_key(sc) >> (32 - kIndexBinBits)), 1u);
+    }
+  }
+  consumer_sync(kConsumerThreads);
+  uint32_t* gh = p.ix_hist + (size_t)t.layer * kIndexBins;
+  for (int b = ctid; b < kIndexBins; b += kConsumerThreads) {
+    const uint32_t v = hist[b];
+    if (v) atomicAdd(gh + b, v);
+  }
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) *tk = ((ticket_add(index_meta(p, t.layer) + IM_TICK_A, 1u) + 1u) % (uint32_t)t.aux) == 0u;
+  consumer_sync(kConsumerThreads);
+  if (*tk) index_threshold(p, t, ub, warp, lane, ctid);
+}
+
+// Run by the index scoring task that arrives last: the bin of the K-th largest score.
+// Thread j holds bins kIndexBins - 1 - (16 j + k), k < 16 (descending); a scan over the
+// threads finds the bin b where the count above it is below K and the count from it on
+// reaches K.  The layer's state receives b, the count above it, how many of b are still to
+// take and b's count; the histogram is cleared and the chosen count reset for the next
+// step, then the layer's index counter is published.
+__device__ void index_threshold(const Params& p, const Task& t, float* scratch, int warp,
+                                int lane, int ctid) {
+  static_assert(kIndexBins == 16 * kConsumerThreads, "16 bins per consumer thread");
+  uint32_t* gh = p.ix_hist + (size_t)t.layer * kIndexBins;
+  uint32_t* meta = index_meta(p, t.layer);
+  uint32_t* wt = reinterpret_cast<uint32_t*>(scratch);  // [kConsumerWarps]
+  const uint32_t K = (uint32_t)p.KI, P = (uint32_t)p.pos + 1u;
+  uint32_t cnt[16], sum = 0;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    cnt[k] = __ldcg(gh + kIndexBins - 1 - (16 * ctid + k));
+    sum += cnt[k];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) wt[warp] = incl;
+  consumer_sync(kConsumerThreads);
+  uint32_t excl = incl - sum;
+  for (int w = 0; w < warp; ++w) excl += wt[w];
+  if (P > K && excl < K && excl + sum >= K) {
+    uint32_t run = excl;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (run < K && run + cnt[k] >= K) {
+        meta[IM_THR] = (uint32_t)(kIndexBins - 1 - (16 * ctid + k));
+        meta[IM_ABOVE] = run;
+        meta[IM_NEED] = K - run;
+        meta[IM_BINCNT] = cnt[k];
+      }
+      run += cnt[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) gh[kIndexBins - 1 - (16 * ctid + k)] = 0u;
+  if (ctid == 0) {
+    meta[IM_NSEL] = 0u;
+    meta[IM_NCAND] = 0u;
+    meta[IM_HASPOS] = 0u;
+  }
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) publish_add(p.counters + t.out, 1u);
+}
+
+// Append `take` lanes' values to list[] at the counter *ctr (one atomic per warp); an
+// index at or past `cap` records a bounds error instead.
+__device__ __forceinline__ void warp_append(const Params& p, bool take, uint32_t* ctr, int32_t* list,
+                                            int32_t val, int cap, int lane, int detail) {
+  const uint32_t mask = __ballot_sync(0xffffffffu, take);
+  if (!mask) return;
+  const int leader = __ffs(mask) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(ctr, (uint32_t)__popc(mask));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (take) {
+    const uint32_t idx = base + (uint32_t)__popc(mask & ((1u << lane) - 1u));
+    if (idx < (uint32_t)cap) list[idx] = val;
+    else record_error(p, TRE_ERR_BOUNDS, detail);
+  }
+}
+
+// Run by the selection task that arrives last when the threshold bin holds more than are
+// still to take: the `need` largest (score, then lower position) of its candidates, by an
+// MSD radix select on keys (low 20 bits of the order key << pb) | (2^pb - 1 - position),
+// pb = bits of a position (all candidates share the top 12 bits); the keys are unique, so
+// exactly `need` of them reach the selected one.
+__device__ void index_pick(const Params& p, const Task& t, float* scratch, int warp, int lane,
+                           int ctid) {
+  uint32_t* meta = index_meta(p, t.layer);
+  const unsigned long long* cand = p.ix_cand + (size_t)t.layer * p.cap;
+  int32_t* sel = p.ix_sel + (size_t)t.layer * p.KI;
+  const uint32_t n = min(__ldcg(meta + IM_NCAND), (uint32_t)p.cap);
+  uint32_t* h = reinterpret_cast<uint32_t*>(scratch);  // [256]
+  uint32_t* sh = h + 256;                               // digit, still to take
+  const int pb = 32 - __clz(max(p.cap - 1, 1));
+  const unsigned long long pmask = (1ull << pb) - 1ull;
+  auto keyof = [&](unsigned long long c) {
+    const unsigned long long k20 = (c >> 32) & 0xFFFFFull;
+    const unsigned long long pos = 0xffffffffull - (c & 0xffffffffull);
+    return (k20 << pb) | (pmask - pos);
+  };
+  const int bits = 20 + pb;
+  unsigned long long prefix = 0;
+  uint32_t rem = __ldcg(meta + IM_NEED);
+  for (int sft = (bits + 7) / 8 * 8 - 8; sft >= 0; sft -= 8) {
+    for (int i = ctid; i < 256; i += kConsumerThreads) h[i] = 0u;
+    consumer_sync(kConsumerThreads);
+    for (uint32_t i = ctid; i < n; i += kConsumerThreads) {
+      const unsigned long long k = keyof(__ldcg(cand + i));
+      if ((k >> (sft + 8)) == prefix) atomicAdd(h + ((k >> sft) & 255u), 1u);
+    }
+    consumer_sync(kConsumerThreads);
+    if (warp == 0) {  // lane l holds digits 255 - 8 l - k, k < 8 (descending)
+      uint32_t c8[8], s8 = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        c8[k] = h[255 - 8 * lane - k];
+        s8 += c8[k];
+      }
+      uint32_t incl = s8;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      uint32_t run = incl - s8;
+      if (run < rem && run + s8 >= rem) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (run < rem && run + c8[k] >= rem) {
+            sh[0] = (uint32_t)(255 - 8 * lane - k);
+            sh[1] = rem - run;
+          }
+          run += c8[k];
+        }
+      }
+    }
+    consumer_sync(kConsumerThreads);
+    prefix = (prefix << 8) | sh[0];
+    rem = sh[1];
+    consumer_sync(kConsumerThreads);  // sh and h are rewritten by the next pass
+  }
+  // every candidate whose key reaches the selected one
+  for (uint32_t i0 = 0; i0 < n; i0 += kConsumerThreads) {
+    const uint32_t i = i0 + ctid;
+    bool take = false;
+    int pos = 0;
+    if (i < n) {
+      const unsigned long long c = __ldcg(cand + i);
+      take = keyof(c) >= prefix;
+      pos = (int)(0xffffffffu - (uint32_t)(c & 0xffffffffull));
+    }
+    if (take && pos == p.pos) {
+      meta[IM_HASPOS] = 1u;
+      take = false;
+    }
+    warp_append(p, take, meta + IM_NSEL, sel, pos, p.KI, lane, t.id);
+  }
+}
+
+// Selection task = split sp of the positions [0, pos]: positions whose bin is above the
+// threshold bin are chosen (the whole threshold bin when all of it is to take), the
+// threshold bin's others become candidates; the new position is flagged instead of listed
+// (its latent row comes from on chip).  The task that arrives last runs index_pick when
+// needed, then (the attention also reads this layer's W_uk contraction) waits for the
+// W_uk tasks and publishes the layer's selection counter.  Steps with pos + 1 <= K only
+// do the last part.
+__device__ void isel_task(const Params& p, const Task& t, float* ub, int* tk, int warp, int lane,
+                          int ctid, bool& ab) {
+  uint32_t* meta = index_meta(p, t.layer);
+  const bool sparse = sparse_step(p);
+  uint32_t need = 0, bincnt = 0;
+  if (sparse) {
+    const uint32_t thr = __ldcg(meta + IM_THR);
+    need = __ldcg(meta + IM_NEED);
+    bincnt = __ldcg(meta + IM_BINCNT);
+    const bool whole_bin = need == bincnt;
+    const long long P = p.pos + 1;
+    const int t0 = (int)(P * t.r1 / t.aux), t1 = (int)(P * (t.r1 + 1) / t.aux);
+    const float* score = p.iscore + (size_t)t.layer * p.cap;
+    int32_t* sel = p.ix_sel + (size_t)t.layer * p.KI;
+    unsigned long long* cand = p.ix_cand + (size_t)t.layer * p.cap;
+    for (int b0 = t0; b0 < t1; b0 += kConsumerThreads) {
+      const int tt = b0 + ctid;
+      const bool live = tt < t1;
+      const float sc = live ? __ldcg(score + tt) : 0.f;
+      const uint32_t key = order_key(sc), bin = key >> (32 - kIndexBinBits);
+      bool above = live && (bin > thr || (whole_bin && bin == thr));
+      const bool cnd = live && !whole_bin && bin == thr;
+      if (above && tt == p.pos) {
+        meta[IM_HASPOS] = 1u;
+        above = false;
+      }
+      warp_append(p, above, meta + IM_NSEL, sel, tt, p.KI, lane, t.id);
+      const uint32_t mask = __ballot_sync(0xffffffffu, cnd);
+      if (mask) {
+        const int leader = __ffs(mask) - 1;
+        uint32_t base = 0;
+        if (lane == leader) base = atomicAdd(meta + IM_NCAND, (uint32_t)__popc(mask));
+        base = __shfl_sync(0xffffffffu, base, leader);
+        if (cnd) {
+          const uint32_t idx = base + (uint32_t)__popc(mask & ((1u << lane) - 1u));
+          if (idx < (uint32_t)p.cap)
+            cand[idx] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)tt);
+          else
+            record_error(p, TRE_ERR_BOUNDS, t.id);
+        }
+      }
+    }
+  }
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) *tk = ((ticket_add(meta + IM_TICK_B, 1u) + 1u) % (uint32_t)t.aux) == 0u;
+  consumer_sync(kConsumerThreads);
+  if (!*tk) return;
+  if (sparse && need != bincnt) index_pick(p, t, ub, warp, lane, ctid);
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) {
+    const bool ok = wait_counter(p, t.layer * C_PER_LAYER + C_MLA_UK, (uint32_t)p.Hq, t.id);
+    if (ok) publish_add(p.counters + t.out, 1u);
+    *tk = ok ? 0 : 1;
+  }
+  consumer_sync(kConsumerThreads);
+  if (*tk) ab = true;
+}
+
 // The W_uv task of head h stages o_lat_h, merging the head's KV splits on the way:
 // o_lat_h = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s (splits that saw no position
 // have m_s = -inf and weigh 0).  128 heads merge on 128 SMs at once.
@@ -1849,7 +2311,14 @@ __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const 
   switch (t.op) {
     case OP_QKV: p.qkv[(size_t)tok * (p.Hq + 2 * p.Hkv) * p.D + n] = v * rn; break;
     case OP_UQ: p.qkv[n] = v * rn; break;
-    case OP_MDQKV: p.cqkv[n] = v * rn; break;
+    case OP_MDQKV: {
+      const float y = v * rn;
+      p.cqkv[n] = y;
+      const int ki = n - (p.QL + p.KL + p.R);  // sparse: this position's index key
+      if (ki >= 0 && ki < p.DI)
+        reinterpret_cast<__nv_bfloat16*>(p.layers[t.layer].v_cache)[(size_t)p.pos * p.DI + ki] =
+            __float2bfloat16_rn(y);
+    } break;
     case OP_UV: p.mla_o[n] = v; break;
     case OP_O: p.h1[(size_t)tok * p.d + n] = resid[n - t.r0] + v; break;
     case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
@@ -2024,7 +2493,7 @@ __device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, c
 // MLA = true: the absorbed-MLA stack's kernel (MLA tiles, no GQA attention); false: GQA /
 // MoE.  Separate instantiations keep each kernel's register allocation to its own tiles.
 // TILED: GEMV stages are 16-row tensor-core tiles (multi-token plans).
-template <bool MLA, int MT, bool TILED, bool F8>
+template <bool MLA, int MT, bool TILED, bool F8, bool SP>
 __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                          float* misc) {
@@ -2038,7 +2507,6 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
   bool ab = false;
   for (int ti = 0; ti < ntask; ++ti) {
     const Task t = my[ti];
-    const int ns = task_nstages<TILED>(p, t);
     if (ctid == 0) {
       long long* tr = p.trace ? p.trace + (size_t)t.id * kTraceCols : nullptr;
       if (tr) tr[0] = (long long)globaltimer_ns();
@@ -2052,6 +2520,8 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     }
     consumer_sync(kConsumerThreads);
     if (flags[0]) break;  // uniform: every consumer thread read the same flag
+    // after the wait: a sparse attention task's stages follow this step's selection
+    const int ns = task_nstages<TILED>(p, t);
 
     if (!MLA && t.type == T_ATTN) {
       cur_key = -1;  // the attention scratch aliases the input-vector planes
@@ -2061,6 +2531,13 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       cur_key = -1;
       if constexpr (MLA)
         mla_attn_task(p, t, gs, ns, ring, full, empty, tags, ub, warp, lane, ctid, ab);
+    } else if (SP && t.type == T_INDEX) {
+      cur_key = -1;
+      if constexpr (SP)
+        index_task(p, t, gs, ns, ring, full, empty, tags, ub, flags + 1, warp, lane, ctid, ab);
+    } else if (SP && t.type == T_ISEL) {
+      cur_key = -1;
+      if constexpr (SP) isel_task(p, t, ub, flags + 1, warp, lane, ctid, ab);
     } else if (MLA && t.op == OP_UK) {
       cur_key = -1;
       if constexpr (MLA)
@@ -2346,7 +2823,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
 }
 
 // ---- the kernel ----------------------------------------------------------------------------------
-template <bool MLA, int MT, bool TILED, bool F8 = false>
+template <bool MLA, int MT, bool TILED, bool F8 = false, bool SP = false>
 __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t NS = (uint32_t)p.ring_stages;
@@ -2391,14 +2868,15 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
              reinterpret_cast<const volatile int*>(misc + 80), threadIdx.x & 31);
     return;
   }
-  consumer<MLA, MT, TILED, F8>(p, my, ntask, ring, full, empty, tags, ub, misc);
+  consumer<MLA, MT, TILED, F8, SP>(p, my, ntask, ring, full, empty, tags, ub, misc);
 }
 
 // ---- host-side launch helpers ------------------------------------------------------------------
 // The kernel instantiation for a stack kind, a number of tokens per step, the GEMV stage
 // form (tiled: multi-token tensor-core tiles) and the weight format (fp8: E4M3 projections
 // on the tensor cores; their own instantiation keeps the bf16 kernel's registers as they are).
-static const void* kernel_for(bool mla, int m, bool tiled, bool fp8 = false) {
+static const void* kernel_for(bool mla, int m, bool tiled, bool fp8 = false, bool sparse = false) {
+  if (mla && sparse) return reinterpret_cast<const void*>(engine_kernel<true, 1, false, false, true>);
   if (mla) return reinterpret_cast<const void*>(engine_kernel<true, 1, false>);
   if (fp8) return reinterpret_cast<const void*>(engine_kernel<false, 1, false, true>);
   if (tiled) {
@@ -2423,7 +2901,7 @@ static const void* kernel_for(bool mla, int m, bool tiled, bool fp8 = false) {
 // (never lowered to this plan's need: an engine created later must not shrink what an
 // earlier one launches with).
 cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled,
-                             bool fp8) {
+                             bool fp8, bool sparse) {
   *blocks_per_sm = 1 << 30;
   int dev = 0, optin = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
@@ -2432,7 +2910,7 @@ cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int m
   if (e0 != cudaSuccess) return e0;
   const int limit = optin > smem_bytes ? optin : smem_bytes;
   for (int m = 1; m <= (mla || fp8 ? 1 : max_m); ++m) {
-    const void* k = kernel_for(mla, m, tiled, fp8);
+    const void* k = kernel_for(mla, m, tiled, fp8, sparse);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
     if (e != cudaSuccess) return e;
     int b = 0;
@@ -2459,7 +2937,7 @@ cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_
   cfg.numAttrs = p.op_group >= 0 ? 0 : 1;
   void* args[] = {const_cast<Params*>(&p)};
   const cudaError_t e =
-      cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0, p.wfp8 != 0), args);
+      cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0, p.wfp8 != 0, p.KI > 0), args);
   if (e != cudaSuccess) cudaGetLastError();  // returned here: do not leave it to the caller
   return e;
 }

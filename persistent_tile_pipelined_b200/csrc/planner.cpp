@@ -154,6 +154,21 @@ struct Builder {
       }
   }
 
+  // Sparse MLA: `n` tasks of one type (index scoring or selection), split sp = r1 of n
+  // (aux = n), each on the SM with the least streamed bytes so far.
+  void splits(uint8_t type, int layer, int n, int64_t bytes_per_task, int dep,
+              uint32_t dep_count, int out) {
+    const std::vector<int> sms = spread(n);
+    for (int sp = 0; sp < n; ++sp) {
+      Task t = make(type, 0, layer, dep, dep_count, out);
+      t.r0 = 0;
+      t.r1 = sp;
+      t.aux = n;
+      q[sms[sp]].push_back(t);
+      cum[sms[sp]] += bytes_per_task;
+    }
+  }
+
   // Set aux = count on every task of `op` created since task id `first`.
   void set_count(int first, uint8_t op, int count) {
     for (auto& qq : q)
@@ -211,6 +226,17 @@ static tre_status validate_mla(const tre_config& c) {
     return fail(TRE_ERR_INVALID_ARG, "MLA q_lora, nope_dim and v_dim must be positive multiples of 8");
   if (c.q_lora > kMaxKPart) return fail(TRE_ERR_UNSUPPORTED, "MLA q_lora above 16384");
   if (c.nope_dim > kMaxResidRows) return fail(TRE_ERR_UNSUPPORTED, "MLA nope_dim above 512");
+  if (c.index_topk < 0) return fail(TRE_ERR_INVALID_ARG, "index_topk must be >= 0");
+  if (c.index_topk > 0) {
+    if (c.index_heads != 16 && c.index_heads != 32 && c.index_heads != 64)
+      return fail(TRE_ERR_UNSUPPORTED, "index_heads must be 16, 32 or 64");
+    if (c.index_dim != 64 && c.index_dim != 128)
+      return fail(TRE_ERR_UNSUPPORTED, "index_dim must be 64 or 128");
+    if (c.index_topk > c.kv_capacity)
+      return fail(TRE_ERR_INVALID_ARG, "index_topk above kv_capacity");
+  } else if (c.index_heads || c.index_dim) {
+    return fail(TRE_ERR_INVALID_ARG, "index_heads / index_dim set without index_topk");
+  }
   return TRE_OK;
 }
 
@@ -231,8 +257,8 @@ static tre_status validate(const tre_config& c) {
     if (c.expert_ffn < 8 || c.expert_ffn % 8)
       return fail(TRE_ERR_INVALID_ARG, "expert_ffn must be a positive multiple of 8");
   }
-  for (int r : c.reserved)
-    if (r != 0) return fail(TRE_ERR_INVALID_ARG, "reserved config fields must be zero");
+  if (c.kind != TRE_LAYER_MLA && (c.index_heads || c.index_dim || c.index_topk))
+    return fail(TRE_ERR_INVALID_ARG, "index_heads / index_dim / index_topk are MLA fields");
   if (c.n_layers < 1 || c.n_layers > 1024) return fail(TRE_ERR_INVALID_ARG, "n_layers out of range");
   if (c.hidden < 8 || c.hidden % 8) return fail(TRE_ERR_INVALID_ARG, "hidden must be a positive multiple of 8");
   if (c.kind != TRE_LAYER_MLA) {
@@ -307,6 +333,12 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     s.R = c.rope_dim;
     s.NP = c.nope_dim;
     s.VD = c.v_dim;
+    if (c.index_topk > 0) {
+      s.HI = c.index_heads;
+      s.DI = c.index_dim;
+      s.KI = c.index_topk;
+      s.isplits = nsm;
+    }
   }
   // an MLA output projection (K = H * v_dim) is staged in halves of at most 8192 inputs,
   // so that the input planes leave room for a 5-deep ring of 36 KB stages; with M tokens
@@ -363,8 +395,11 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     ops.push_back({s.d, 2, 0, pesz});
     ops.push_back({s.F, 1, 0, pesz});
   }
-  // a stage holds one attention tile: 64 K and V rows (GQA) or 32 latent rows (MLA)
+  // a stage holds one attention tile: 64 K and V rows (GQA) or 32 latent rows (MLA; sparse:
+  // 32 gathered rows at a padded pitch, or kIndexRows index keys)
   int xs = 8, need = mla ? (s.KL + s.R) * kMlaPosPerStage * 2 : 4 * s.D * kMaxPosPerStage;
+  if (s.KI) need = std::max({need, kMlaPosPerStage * sparse_lat_pitch(s.KL + s.R),
+                             kIndexRows * s.DI * 2});
   for (auto& o : ops) {
     const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max),
                                                gemv_part_align(s.tiles, o.esz == 1));
@@ -414,6 +449,11 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     s.attn_floats = std::max(kConsumerWarps * kMlaHeadGroup * 36 + 640 + 128,
                              2 * kMlaHeadGroup * Smax);
     s.attn_floats = std::max(s.attn_floats, kConsumerWarps * s.KL + s.NP + 64);
+    // index scoring: the score histogram, the bf16 query tile [H_I][D_I], the head weights,
+    // the new position's per-warp sums
+    if (s.KI)
+      s.attn_floats = std::max(s.attn_floats, kIndexBins + kIndexMaxHeads * 128 / 2 +
+                                                  kIndexMaxHeads + 64);
   }
   const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + (s.tiles ? kTileRedFloats : 0),
                                      s.attn_floats) + 7) / 8 * 8;
@@ -444,11 +484,24 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
               cuk = counter_of(l, C_MLA_UK), ca = counter_of(l, C_ATTN),
               cuv = counter_of(l, C_MLA_UV), co = counter_of(l, C_O);
     const int big = 1 << 30, C = s.KL + s.R, H = s.Hq, groups = H / kMlaHeadGroup;
-    const int n1 = b.gemv(OP_MDQKV, l, s.QL + C, s.d, 1, prev_down, prev_down_count, cdq, big);
-    const int n2 = b.gemv(OP_UQ, l, H * (s.NP + s.R), s.QL, 1, cdq, (uint32_t)n1, cuq, big);
+    // sparse: the down-projection also yields the index key and head weights, the q
+    // up-projection the index queries; index scoring tasks (after the q up-projection)
+    // score every cached position, selection tasks keep the top K, and the attention
+    // waits for the selection (whose last task also waits for the W_uk contraction)
+    const int n1 = b.gemv(OP_MDQKV, l, s.QL + C + (s.KI ? s.DI + s.HI : 0), s.d, 1, prev_down,
+                          prev_down_count, cdq, big);
+    const int n2 = b.gemv(OP_UQ, l, H * (s.NP + s.R) + s.HI * s.DI, s.QL, 1, cdq, (uint32_t)n1,
+                          cuq, big);
+    const int cix = counter_of(l, C_MLA_IDX), csel = counter_of(l, C_MLA_SEL);
+    if (s.KI)
+      b.splits(T_INDEX, l, s.isplits, (int64_t)s.cap / s.isplits * s.DI * 2, cuq, (uint32_t)n2,
+               cix);
     const int n3 = b.per_unit(OP_UK, l, H, s.NP, (int64_t)s.NP * s.KL * 2, cuq, (uint32_t)n2, cuk);
-    const int64_t lat_task = (int64_t)(s.cap - s.M) / S * C * 2;
-    b.mla_attention(l, groups, S, lat_task, cuk, (uint32_t)n3, ca);
+    if (s.KI) b.splits(T_ISEL, l, s.isplits, 0, cix, 1u, csel);
+    const int64_t lat_task =
+        (int64_t)((s.KI ? std::min(s.KI, s.cap) : s.cap) - s.M) / S * C * 2;
+    if (s.KI) b.mla_attention(l, groups, S, lat_task, csel, 1u, ca);
+    else b.mla_attention(l, groups, S, lat_task, cuk, (uint32_t)n3, ca);
     const int n5 = b.per_unit(OP_UV, l, H, s.VD, (int64_t)s.VD * s.KL * 2, ca,
                               (uint32_t)(groups * S), cuv);
     const int n6 = b.gemv(OP_MO, l, s.d, H * s.VD, 1, cuv, (uint32_t)n5, co, kMaxResidRows);
@@ -580,8 +633,16 @@ int64_t step_bytes(const PlanShape& s, int pos, int m) {
     const int64_t H = s.Hq, C = s.KL + s.R;
     const int64_t w = (s.QL + C) * d + H * (s.NP + s.R) * s.QL +
                       H * s.NP * s.KL + H * s.VD * s.KL + d * H * s.VD;
-    int64_t bytes = (w * 2 + (d + s.QL + s.KL) * 2) * s.L;   // weights and norm gains
-    bytes += (int64_t)s.L * (pos + 1) * C * 2;                // latent rows read + written
+    const int64_t wi = s.KI ? (int64_t)s.HI * s.DI * s.QL + (int64_t)(s.DI + s.HI) * d : 0;
+    int64_t bytes = ((w + wi) * 2 + (d + s.QL + s.KL) * 2) * s.L;   // weights and norm gains
+    if (s.KI && pos + 1 > s.KI) {
+      // sparse: the index keys read + this one written, the K chosen latent rows read (the
+      // new one from on chip when chosen) + this position's written
+      bytes += (int64_t)s.L * ((int64_t)(pos + 1) * s.DI * 2 + (int64_t)(s.KI + 1) * C * 2);
+    } else {
+      bytes += (int64_t)s.L * (pos + 1) * C * 2;              // latent rows read + written
+      if (s.KI) bytes += (int64_t)s.L * (pos + 1) * s.DI * 2;  // the index keys too
+    }
     if (s.has_lm) bytes += (int64_t)s.V * d * 2 + d * 2 + d * 2 + (int64_t)s.V * 4;
     return bytes;
   }

@@ -18,7 +18,7 @@
 
 namespace tre {
 cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled,
-                             bool fp8 = false);
+                             bool fp8 = false, bool sparse = false);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 const char* last_error_cstr();
@@ -139,9 +139,12 @@ TRE_EXPORT tre_status tre_plan_inspect(const tre_config* cfg, int32_t num_sms,
   info->max_tasks_per_sm = mx;
   const int64_t row_new = s.kind == TRE_LAYER_MLA ? (int64_t)(s.KL + s.R) * 2 : (int64_t)s.Hkv * s.D * 4;
   const int64_t row_read = s.kind == TRE_LAYER_MLA ? (int64_t)(s.KL + s.R) * 2 : (int64_t)s.Hkv * s.D * 4;
-  info->weight_bytes = step_bytes(s, 0) - (int64_t)s.L * row_new -
+  info->weight_bytes = step_bytes(s, 0) - (int64_t)s.L * (row_new + (int64_t)s.DI * 2) -
                        (s.has_lm ? (int64_t)s.V * 4 + 2LL * s.d : 0);
   info->kv_bytes_at_capacity = (int64_t)s.L * (int64_t)(s.cap - s.M) * row_read;
+  if (s.KI)  // sparse MLA: every index key, and only the K chosen latent rows
+    info->kv_bytes_at_capacity = (int64_t)s.L * ((int64_t)(s.cap - 1) * s.DI * 2 +
+                                                 (int64_t)std::min(s.KI, s.cap - 1) * row_read);
   int64_t lo = INT64_MAX, hi = 0;
   for (int64_t b : bytes) {
     lo = std::min(lo, b);
@@ -233,7 +236,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   if (st != TRE_OK) return st;
 
   // ---- pointer validation: everything the plan reads must be present and 16B-aligned.
-  if (!w->layer_w || !w->k_cache || (!w->v_cache && s.kind != TRE_LAYER_MLA)) {
+  if (!w->layer_w || !w->k_cache || (!w->v_cache && (s.kind != TRE_LAYER_MLA || s.KI))) {
     set_error("tre_create: layer_w / k_cache / v_cache tables must be non-NULL");
     return TRE_ERR_INVALID_ARG;
   }
@@ -247,6 +250,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   if (mla) {
     slots = {TRE_W_ATTN_NORM, TRE_W_DQ, TRE_W_Q_NORM, TRE_W_UQ, TRE_W_DKV, TRE_W_KV_NORM,
              TRE_W_UK, TRE_W_UV, TRE_W_MLA_O};
+    if (s.KI) slots.insert(slots.end(), {TRE_W_INDEX_Q, TRE_W_INDEX_K});
   } else if (s.kind == TRE_LAYER_MOE) {
     slots = {TRE_W_ATTN_NORM, TRE_W_Q, TRE_W_K, TRE_W_V, TRE_W_O, TRE_W_FFN_NORM, TRE_W_ROUTER,
              TRE_W_EXPERT_GATE, TRE_W_EXPERT_UP, TRE_W_EXPERT_DOWN};
@@ -265,12 +269,14 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
       }
       lp[l].w[slot] = static_cast<const uint16_t*>(p);
     }
-    if (!aligned16(w->k_cache[l]) || (!mla && !aligned16(w->v_cache[l]))) {
-      set_error("tre_create: KV cache of layer " + std::to_string(l) + " NULL or misaligned");
+    const bool has_v = !mla || s.KI;  // sparse MLA: v_cache holds the index keys
+    if (!aligned16(w->k_cache[l]) || (has_v && (!w->v_cache || !aligned16(w->v_cache[l])))) {
+      set_error("tre_create: KV (or index-key) cache of layer " + std::to_string(l) +
+                " NULL or misaligned");
       return TRE_ERR_INVALID_ARG;
     }
     lp[l].k_cache = static_cast<uint16_t*>(w->k_cache[l]);
-    lp[l].v_cache = mla ? nullptr : static_cast<uint16_t*>(w->v_cache[l]);
+    lp[l].v_cache = has_v ? static_cast<uint16_t*>(w->v_cache[l]) : nullptr;
   }
   if (s.has_lm && (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(w->lm_head))) {
     set_error("tre_create: embed / final_norm / lm_head NULL or not 16-byte aligned");
@@ -286,7 +292,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
 
   int bps = 0;
   CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M, s.tiles != 0,
-                      s.wfp8 != 0));
+                      s.wfp8 != 0, s.KI > 0));
   if (bps < 1) {
     set_error("tre_create: the persistent CTA does not fit on an SM");
     return TRE_ERR_OCCUPANCY;
@@ -300,7 +306,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   e->n_groups = n_groups;
 
   // ---- one device block for all engine-owned state
-  const int qkv_n = mla ? s.Hq * (s.NP + s.R) : (s.Hq + 2 * s.Hkv) * s.D;
+  const int qkv_n = mla ? s.Hq * (s.NP + s.R) + s.HI * s.DI : (s.Hq + 2 * s.Hkv) * s.D;
   const int C = s.KL + s.R;
   // MLA: one map per layer over the latent cache; GQA / MoE: K and V maps per layer over
   // the caches viewed as [Hkv * capacity][D]
@@ -312,6 +318,12 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
     if (ms == TRE_OK && !mla)
       ms = encode_cache_map(w->v_cache[l], s.D, (long long)s.Hkv * s.cap, s.pos_per_stage,
                             &maps[2 * l + 1]);
+    if (ms != TRE_OK) return ms;
+  }
+  // sparse MLA: one map per layer over the index-key cache, boxes of kIndexRows keys
+  std::vector<CUtensorMap> imaps(s.KI ? s.L : 0);
+  for (int l = 0; l < (int)imaps.size(); ++l) {
+    const tre_status ms = encode_cache_map(w->v_cache[l], s.DI, s.cap, kIndexRows, &imaps[l]);
     if (ms != TRE_OK) return ms;
   }
   Carve cv;
@@ -343,13 +355,20 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_tok = cv.take<int32_t>(kMaxTokens);
   size_t o_inv = cv.take<double>(std::max(1, s.D / 2));
   size_t o_invr = cv.take<double>(std::max(1, s.R / 2));
-  size_t o_cqkv = cv.take<float>(mla ? s.QL + C : 1);
+  size_t o_cqkv = cv.take<float>(mla ? s.QL + C + s.DI + s.HI : 1);
   size_t o_qf = cv.take<float>(mla ? (size_t)s.Hq * C : 1);
   size_t o_latn = cv.take<float>(mla ? C : 1);
   size_t o_olat = cv.take<float>(mla ? (size_t)s.Hq * s.KL : 1);
   size_t o_mlao = cv.take<float>(mla ? (size_t)s.Hq * s.VD : 1);
+  const bool sp = s.KI > 0;
+  size_t o_isc = cv.take<float>(sp ? (size_t)s.L * s.cap : 1);
+  size_t o_isel = cv.take<int32_t>(sp ? (size_t)s.L * s.KI : 1);
+  size_t o_icand = cv.take<unsigned long long>(sp ? (size_t)s.L * s.cap : 1);
+  size_t o_ihist = cv.take<uint32_t>(sp ? (size_t)s.L * kIndexBins : 1);
+  size_t o_imeta = cv.take<uint32_t>(sp ? (size_t)s.L * IM_WORDS : 1);
   cv.off = (cv.off + 127) & ~size_t(127);
   size_t o_maps = cv.take<CUtensorMap>(maps.size() ? maps.size() : 1);
+  size_t o_imaps = cv.take<CUtensorMap>(imaps.size() ? imaps.size() : 1);
   const bool dbg_hidden = cfg->debug_flags & TRE_DEBUG_HIDDEN;
   const bool dbg_trace = cfg->debug_flags & TRE_DEBUG_TRACE;
   size_t o_hidden = dbg_hidden ? cv.take<float>((size_t)s.L * M * s.d) : 0;
@@ -394,6 +413,10 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
       (ce = cudaMemcpy(B + o_maps, maps.data(), maps.size() * sizeof(CUtensorMap),
                        cudaMemcpyHostToDevice)) != cudaSuccess)
     return fail_free(ce, "upload tensor maps");
+  if (!imaps.empty() &&
+      (ce = cudaMemcpy(B + o_imaps, imaps.data(), imaps.size() * sizeof(CUtensorMap),
+                       cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail_free(ce, "upload index tensor maps");
   if ((ce = cudaHostAlloc(reinterpret_cast<void**>(&e->status_host), 4 * sizeof(int32_t),
                           cudaHostAllocMapped)) != cudaSuccess)
     return fail_free(ce, "cudaHostAlloc(status)");
@@ -444,6 +467,13 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.mla_o = reinterpret_cast<float*>(B + o_mlao);
   p.kv_maps = B + o_maps;
   p.QL = s.QL; p.KL = s.KL; p.R = s.R; p.NP = s.NP; p.VD = s.VD;
+  p.HI = s.HI; p.DI = s.DI; p.KI = s.KI; p.isplits = s.isplits;
+  p.iscore = reinterpret_cast<float*>(B + o_isc);
+  p.ix_sel = reinterpret_cast<int32_t*>(B + o_isel);
+  p.ix_cand = reinterpret_cast<unsigned long long*>(B + o_icand);
+  p.ix_hist = reinterpret_cast<uint32_t*>(B + o_ihist);
+  p.ix_meta = reinterpret_cast<uint32_t*>(B + o_imeta);
+  p.ix_maps = B + o_imaps;
   p.kpart_max = s.kpart_max;
   p.m = 1;
   // default: hold (measured faster on the 8B-shaped stack: 0.683 vs 0.665 of peak)
@@ -693,6 +723,41 @@ TRE_EXPORT tre_status tre_debug_routing(tre_engine* e, int32_t* idx_host, float*
   return TRE_OK;
 }
 
+TRE_EXPORT tre_status tre_debug_index(tre_engine* e, int32_t layer, int32_t pos, float* score_host,
+                                      int32_t* sel_host, int32_t* n_sel_out) {
+  if (!e || !n_sel_out) {
+    set_error("tre_debug_index: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  const PlanShape& s = e->shape;
+  if (!s.KI || layer < 0 || layer >= s.L || pos < 0 || pos >= s.cap) {
+    set_error("tre_debug_index: not a sparse MLA engine, or layer / pos out of range");
+    return TRE_ERR_INVALID_ARG;
+  }
+  CK(cudaSetDevice(e->device));
+  if (e->last_stream) CK(cudaStreamSynchronize(e->last_stream));
+  CK(cudaDeviceSynchronize());
+  const Params& p = e->base;
+  if (score_host)
+    CK(cudaMemcpy(score_host, p.iscore + (size_t)layer * s.cap, (size_t)(pos + 1) * 4,
+                  cudaMemcpyDeviceToHost));
+  if (pos + 1 <= s.KI) {  // every position
+    *n_sel_out = pos + 1;
+    if (sel_host)
+      for (int i = 0; i <= pos; ++i) sel_host[i] = i;
+    return TRE_OK;
+  }
+  uint32_t meta[IM_WORDS];
+  CK(cudaMemcpy(meta, p.ix_meta + (size_t)layer * IM_WORDS, sizeof(meta), cudaMemcpyDeviceToHost));
+  const int n = (int)std::min<uint32_t>(meta[IM_NSEL], (uint32_t)s.KI);
+  if (sel_host) {
+    CK(cudaMemcpy(sel_host, p.ix_sel + (size_t)layer * s.KI, (size_t)n * 4, cudaMemcpyDeviceToHost));
+    if (meta[IM_HASPOS] && n < s.KI) sel_host[n] = pos;
+  }
+  *n_sel_out = n + (meta[IM_HASPOS] && n < s.KI ? 1 : 0);
+  return TRE_OK;
+}
+
 TRE_EXPORT tre_status tre_get_status(tre_engine* e, int32_t* device_status, int32_t* detail_out) {
   if (!e || !device_status) {
     set_error("tre_get_status: NULL argument");
@@ -728,6 +793,10 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
     CK(cudaMemsetAsync(p.down_tickets, 0, (size_t)e->shape.down_blocks * 4, s));
   CK(cudaMemsetAsync(p.argmax_slot, 0, 8 * kMaxTokens, s));
   CK(cudaMemsetAsync(p.err, 0, 8, s));  // error word + abort flag
+  if (e->shape.KI) {  // sparse MLA: histograms and selection state (tickets included)
+    CK(cudaMemsetAsync(p.ix_hist, 0, (size_t)e->shape.L * kIndexBins * 4, s));
+    CK(cudaMemsetAsync(p.ix_meta, 0, (size_t)e->shape.L * IM_WORDS * 4, s));
+  }
   CK(cudaStreamSynchronize(s));
   std::memset(e->status_host, 0, 4 * sizeof(int32_t));
   e->epoch = 0;

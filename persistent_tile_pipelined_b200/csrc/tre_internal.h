@@ -77,7 +77,7 @@ TRE_HD inline int fp8_rows_per_stage(int Kp, int nseg, int stage_bytes) {
 }
 
 // ---- tasks --------------------------------------------------------------------------
-enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1, T_MLA_ATTN = 2 };
+enum TaskType : uint8_t { T_GEMV = 0, T_ATTN = 1, T_MLA_ATTN = 2, T_INDEX = 3, T_ISEL = 4 };
 
 // GEMV ops: which matrix, which input vector, which epilogue.
 enum GemvOp : uint8_t {
@@ -105,7 +105,23 @@ enum GemvOp : uint8_t {
 
 // MLA counters reuse the per-layer slots: QKV = down-projections, ATTN, O = output
 // projection, and these three.
-enum MlaCounter { C_MLA_UQ = 3, C_MLA_UK = 4, C_MLA_UV = 5 };
+enum MlaCounter { C_MLA_UQ = 3, C_MLA_UK = 4, C_MLA_UV = 5, C_MLA_IDX = 6, C_MLA_SEL = 7 };
+// Sparse MLA (the lightning-indexer reading): index scoring tasks stream the index-key
+// cache in stages of kIndexRows positions (64-column swizzled boxes, like the latent
+// stages) and histogram the scores on the top kIndexBinBits bits of their order key; the
+// chosen positions' latent rows are gathered by per-row bulk copies into stages of
+// kMlaPosPerStage rows at a padded pitch (conflict-free ldmatrix without the swizzle).
+constexpr int kIndexRows = 128;
+constexpr int kIndexBinBits = 12;
+constexpr int kIndexBins = 1 << kIndexBinBits;
+constexpr int kIndexMaxHeads = 64;
+TRE_HD inline int sparse_lat_pitch(int C) { return C * 2 + 16; }  // bytes per gathered row
+// Per-layer selection state (uint32 words): the threshold bin, how many positions lie in
+// bins above it, how many of the threshold bin are still to take, that bin's count, the
+// chosen-position count, the candidate count, whether the new position was chosen, and
+// the arrival tickets of the scoring and selection tasks.
+enum IndexMeta { IM_THR = 0, IM_ABOVE = 1, IM_NEED = 2, IM_BINCNT = 3, IM_NSEL = 4,
+                 IM_NCAND = 5, IM_HASPOS = 6, IM_TICK_A = 7, IM_TICK_B = 8, IM_WORDS = 16 };
 constexpr int kMlaHeadGroup = 16;     // query heads per MLA attention tile (the mma M)
 constexpr int kMlaPosPerStage = 32;   // latent rows per MLA attention stage
 constexpr int kMlaBox = 64;           // latent columns per tensor-map box (128 B, swizzled)
@@ -121,7 +137,7 @@ TRE_HD inline int gqa_pstride(int D) { return D + 4; }
 // C_ROUTE (MoE) is bumped once per step by the router task that finishes last, after it
 // has written the layer's selected experts and weights.
 enum CounterKind { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, C_ROUTE = 5,
-                   C_PER_LAYER = 6 };
+                   C_PER_LAYER = 8 };
 
 struct Task {          // 32 bytes, 16-byte aligned array
   uint8_t type;        // TaskType
@@ -130,8 +146,10 @@ struct Task {          // 32 bytes, 16-byte aligned array
   int32_t dep;         // counter to wait on, -1 = none
   uint32_t dep_count;  // increments of `dep` per step
   int32_t out;         // counter to bump when done, -1 = none
-  int32_t r0, r1;      // GEMV: output rows [r0, r1).  ATTN: kv head, split index
-  int32_t aux;         // ATTN: number of splits.  LM / ROUTER: number of tasks of the op.
+  int32_t r0, r1;      // GEMV: output rows [r0, r1).  ATTN: kv head, split index.
+                       // INDEX / ISEL: -, split index
+  int32_t aux;         // ATTN / INDEX / ISEL: number of splits.  LM / ROUTER: number of
+                       // tasks of the op.
                        // other GEMV: K-part index | (number of K-parts << 8)
   int32_t id;          // global task index (trace rows, error detail)
 };
@@ -140,7 +158,7 @@ static_assert(sizeof(Task) == 32, "task descriptor is 32 bytes");
 struct LayerPtrs {     // device-side per-layer pointer table
   const uint16_t* w[TRE_W_SLOTS];
   uint16_t* k_cache;
-  uint16_t* v_cache;
+  uint16_t* v_cache;   // MLA sparse: the index-key cache [cap][D_I]
 };
 
 // ---- the plan (host side) -----------------------------------------------------------
@@ -149,6 +167,8 @@ struct PlanShape {
   int d, Hq, Hkv, D, F, V, L, cap, M;
   int E, topk, nshared, Fe;  // MoE: experts, selected per token, shared, expert FFN
   int QL, KL, R, NP, VD;  // MLA: q_lora, kv_lora, rope, nope, v dims
+  int HI, DI, KI;         // MLA sparse: index heads, index dim, positions kept (0: dense)
+  int isplits;            // MLA sparse: index scoring tasks = selection tasks per layer
   int kpart_max;       // longest input slice of a GEMV task (floats)
   int tiles;           // multi-token plan: GEMV stages are 16-row tensor-core tiles
   int wfp8;            // GQA projections are E4M3 with 128 x 128 block scales
@@ -206,6 +226,15 @@ struct Params {
   float* lat_new;                  // [KL + R]: this token's latent row (bf16 values)
   float* o_lat;                    // [H][KL]
   float* mla_o;                    // [H * VD]
+  // sparse MLA (HI > 0): per layer scores [L][cap], chosen positions [L][KI], threshold-bin
+  // candidates [L][cap] (order key << 32 | ~position), score histograms [L][kIndexBins],
+  // selection state [L][IM_WORDS]; index-cache tensor maps [L] (128 B each)
+  float* iscore;
+  int32_t* ix_sel;
+  unsigned long long* ix_cand;
+  uint32_t* ix_hist;
+  uint32_t* ix_meta;
+  const void* ix_maps;
   const void* kv_maps;             // tensor maps (128 B each): GQA / MoE [L][K, V] caches,
                                    // MLA [L] latent caches
   const double* rope_inv_freq_r;   // [R / 2]
@@ -222,6 +251,7 @@ struct Params {
   int d, Hq, Hkv, D, F, V, L, cap;
   int E, topk, nshared, Fe;
   int QL, KL, R, NP, VD, kpart_max;
+  int HI, DI, KI, isplits;
   int nsplit, pps, stage_bytes, ring_stages, xs_floats, ub_floats;
   float eps;
   int token, pos;

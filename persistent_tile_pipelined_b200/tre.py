@@ -51,8 +51,8 @@ class tre_config(ctypes.Structure):
         (n, ctypes.c_int32) for n in (
             "has_embed_lm_head", "debug_flags", "dep_timeout_us", "num_sms", "kv_splits",
             "stage_bytes", "ring_stages", "l2_prefetch_kb", "gemv_kpart_max",
-            "stream_policy", "multi_token_gemv", "weight_format")] + [
-        ("reserved", ctypes.c_int32 * 3)]
+            "stream_policy", "multi_token_gemv", "weight_format", "index_heads", "index_dim",
+            "index_topk")]
 
 
 class tre_weights(ctypes.Structure):
@@ -73,7 +73,7 @@ class tre_plan_info(ctypes.Structure):
 TRE_LAUNCH_PERSISTENT, TRE_LAUNCH_PER_OP = 0, 1
 
 EXPORTED = ("tre_create", "tre_destroy", "tre_decode_step", "tre_decode_step_host",
-            "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
+            "tre_decode_step_static", "tre_layers_step", "tre_debug_routing", "tre_debug_index",
             "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
             "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
             "tre_plan_inspect", "tre_plan_tasks", "tre_plan_op_groups", "tre_last_error")
@@ -100,6 +100,7 @@ def _load() -> ctypes.CDLL:
     L.tre_plan_op_groups.argtypes = [ctypes.POINTER(tre_config), i32, i32, vp, i32]
     L.tre_plan_op_groups.restype = i32
     L.tre_debug_routing.argtypes = [vp, vp, vp]
+    L.tre_debug_index.argtypes = [vp, i32, i32, vp, vp, ctypes.POINTER(i32)]
     L.tre_get_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.tre_reset.argtypes = [vp, vp]
     L.tre_debug_hidden.argtypes = [vp, vp, vp]
@@ -113,7 +114,7 @@ def _load() -> ctypes.CDLL:
     L.tre_last_error.restype = ctypes.c_char_p
     for name in ("tre_create", "tre_decode_step", "tre_decode_step_host",
                  "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
-                 "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
+                 "tre_debug_index", "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
                  "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
                  "tre_plan_inspect"):
         getattr(L, name).restype = ctypes.c_int
@@ -188,6 +189,18 @@ def tre_debug_routing(h, n_layers: int, top_k: int):
     check(lib.tre_debug_routing(h, idx.ctypes.data_as(ctypes.c_void_p),
                                 w.ctypes.data_as(ctypes.c_void_p)), "tre_debug_routing")
     return idx, w
+
+
+def tre_debug_index(h, layer: int, pos: int, index_topk: int):
+    """(scores float32[pos + 1], chosen positions int32[n], unordered) of layer `layer` at
+    the last step (position pos) of a sparse MLA engine."""
+    sc = np.zeros(pos + 1, dtype=np.float32)
+    sel = np.zeros(max(index_topk, pos + 1), dtype=np.int32)
+    n = ctypes.c_int32()
+    check(lib.tre_debug_index(h, int(layer), int(pos), sc.ctypes.data_as(ctypes.c_void_p),
+                              sel.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)),
+          "tre_debug_index")
+    return sc, sel[:n.value].copy()
 
 
 def tre_get_status(h):
@@ -270,8 +283,8 @@ def config_from_workload(wl, **overrides) -> tre_config:
     c.kind = {"gqa": TRE_LAYER_GQA, "mla": TRE_LAYER_MLA, "moe": TRE_LAYER_MOE}[wl.kind]
     for f in ("n_layers", "hidden", "n_q_heads", "n_kv_heads", "head_dim", "ffn", "vocab",
               "q_lora", "kv_lora", "rope_dim", "nope_dim", "v_dim", "n_experts", "top_k",
-              "n_shared", "expert_ffn"):
-        setattr(c, f, int(getattr(wl, f)))
+              "n_shared", "expert_ffn", "index_heads", "index_dim", "index_topk"):
+        setattr(c, f, int(getattr(wl, f, 0)))
     c.kv_capacity = wl.kv_capacity
     c.max_tokens_per_step = wl.tokens_per_step
     c.rope_theta = wl.rope_theta
@@ -337,11 +350,12 @@ def upload_moe_model(wl, model: dict, device="cuda:0", expert_fn=None) -> dict:
 
 def upload_mla_model(model: dict, device="cuda:0") -> dict:
     """Copy a host absorbed-MLA model (bf16 words) to device tensors: the layer slots as
-    they are and each layer's latent cache [capacity][kv_lora + rope] as its k_cache."""
+    they are, each layer's latent cache [capacity][kv_lora + rope] as its k_cache and (sparse
+    attention) its index-key cache [capacity][index_dim] as its v_cache."""
     return {"layers": [{slot: _dev_tensor(a, device) for slot, a in layer.items()}
                        for layer in model["layers"]],
             "k_cache": [_dev_tensor(c, device) for c in model["latent_cache"]],
-            "v_cache": []}
+            "v_cache": [_dev_tensor(c, device) for c in model.get("index_cache", [])]}
 
 
 def make_weights(cfg: tre_config, dev_model: dict):
@@ -447,6 +461,10 @@ class Engine:
 
     def routing(self):
         return tre_debug_routing(self.h, self.cfg.n_layers, self.cfg.top_k)
+
+    def index(self, layer: int, pos: int):
+        """Sparse MLA: (index scores [pos + 1], chosen positions) of `layer` at the last step."""
+        return tre_debug_index(self.h, layer, pos, self.cfg.index_topk)
 
     def status(self):
         return tre_get_status(self.h)

@@ -20,8 +20,10 @@ from persistent_tile_pipelined_b200 import tre  # noqa: E402
 T_GEMV, T_ATTN = 0, 1
 OP_QKV, OP_O, OP_GU, OP_DOWN, OP_LM, OP_ROUTER, OP_SGU, OP_RGU, OP_MDOWN = range(9)
 OP_MDQKV, OP_UQ, OP_UK, OP_UV, OP_MO = range(9, 14)
-T_MLA_ATTN = 2
-C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_ROUTE, C_PER_LAYER = range(7)
+T_MLA_ATTN, T_INDEX, T_ISEL = 2, 3, 4
+C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_ROUTE = range(6)
+C_MLA_UK, C_MLA_IDX, C_MLA_SEL = 4, 6, 7
+C_PER_LAYER = 8
 WHOLE_ROW_OPS = (OP_LM, OP_ROUTER)   # aux holds the op's task count, not K-parts
 
 
@@ -58,6 +60,8 @@ MOE_SMALL = W.MOE4.replace(name="moe-small", n_layers=2, hidden=512, n_q_heads=8
                           expert_ffn=200)
 MLA_SMALL = W.MLA4.replace(name="mla-small", n_layers=2, hidden=512, n_q_heads=32, q_lora=128,
                           kv_lora=128, rope_dim=64, nope_dim=64, v_dim=64, prefill=100)
+MLA_SPARSE = MLA_SMALL.replace(name="mla-sparse-small", prefill=300, index_heads=64, index_dim=128,
+                              index_topk=64)
 PLAN_CASES = [
     (W.TINY, 148), (W.TINY, 7), (W.LLAMA8B, 148), (W.LLAMA8B, 132),
     (W.TINY.replace(n_q_heads=8, n_kv_heads=1, ffn=696, vocab=1001), 148),
@@ -65,6 +69,8 @@ PLAN_CASES = [
     (W.MOE4, 148), (MOE_SMALL, 148), (MOE_SMALL, 5),
     (MOE_SMALL.replace(n_shared=0, top_k=1), 19), (MOE_SMALL.replace(n_shared=2), 64),
     (W.MLA4, 148), (MLA_SMALL, 148), (MLA_SMALL, 6),
+    (MLA_SPARSE, 148), (MLA_SPARSE, 6), (W.MLA4_SPARSE128K, 148),
+    (MLA_SPARSE.replace(index_heads=16, index_dim=64, index_topk=300), 37),
     # multi-token plans: tensor-core tiles at 4 tokens, CUDA-core rows at 2 and 3
     (W.LLAMA8B.replace(tokens_per_step=4), 148), (W.LLAMA8B.replace(tokens_per_step=2), 148),
     (W.TINY.replace(tokens_per_step=4, hidden=272, ffn=720, vocab=1001), 7),
@@ -76,8 +82,9 @@ def rows_of_ops(wl):
     """Output rows of every GEMV op of one layer."""
     if wl.kind == "mla":
         H = wl.n_q_heads
-        rows = {OP_MDQKV: wl.q_lora + wl.kv_lora + wl.rope_dim,
-                OP_UQ: H * (wl.nope_dim + wl.rope_dim), OP_UK: H * wl.nope_dim,
+        rows = {OP_MDQKV: wl.q_lora + wl.kv_lora + wl.rope_dim + wl.index_dim + wl.index_heads,
+                OP_UQ: H * (wl.nope_dim + wl.rope_dim) + wl.index_heads * wl.index_dim,
+                OP_UK: H * wl.nope_dim,
                 OP_UV: H * wl.v_dim, OP_MO: wl.hidden}
         if wl.vocab:
             rows[OP_LM] = wl.vocab
@@ -129,7 +136,14 @@ def check_plan(wl, nsm, **over):
         # every producer of a dependency precedes its consumer in global order
         assert all(T["id"][j] < T["id"][i] for j in producers)
         kind = dep % C_PER_LAYER
-        if T["type"][i] == T_GEMV and T["op"][i] == OP_UV:
+        if wl.kind == "mla" and kind in (C_MLA_IDX, C_MLA_SEL):
+            # sparse: the index and selection counters are bumped once, by the scoring /
+            # selection task that arrives last; attention waits for the selection
+            assert T["dep_count"][i] == 1
+            want = T_INDEX if kind == C_MLA_IDX else T_ISEL
+            assert producers and all(T["type"][j] == want for j in producers)
+            assert T["type"][i] == (T_ISEL if kind == C_MLA_IDX else T_MLA_ATTN)
+        elif T["type"][i] == T_GEMV and T["op"][i] == OP_UV:
             # every MLA attention split publishes; W_uv merges a head's splits
             assert T["dep_count"][i] == (wl.n_q_heads // 16) * info.kv_splits
         elif T["type"][i] == T_GEMV and T["op"][i] == OP_O:
@@ -201,6 +215,14 @@ def check_plan(wl, nsm, **over):
         assert set(pairs) == {(g, s) for g in range(units) for s in range(S)}
         assert all(v == 1 for v in pairs.values())
         assert (T["aux"][sel] == S).all()
+        for typ in (T_INDEX, T_ISEL):  # sparse: splits 0 .. n - 1 once each, n on every task
+            sel = (T["type"] == typ) & (T["layer"] == l)
+            if wl.index_topk:
+                nsp = int(sel.sum())
+                assert nsp >= 1 and sorted(T["r1"][sel].tolist()) == list(range(nsp))
+                assert (T["aux"][sel] == nsp).all()
+            else:
+                assert not sel.any()
     # per layer, attention and MoE-down tasks are spread evenly: no SM holds more than
     # ceil(n / nsm) of one op's tasks (an op ends at a dependency; its slowest SM sets it)
     sm_of = np.zeros(n, dtype=np.int64)
@@ -434,13 +456,34 @@ def test_multi_token_cuda_core_form_takes_any_k():
     assert two.stage_bytes < 16 * (1024 * 2 + 16) <= two_t.stage_bytes
 
 
-def test_reserved_fields_must_be_zero():
+def test_index_fields_are_validated():
     import ctypes
-    cfg = tre.config_from_workload(W.TINY)
-    cfg.reserved[2] = 1
     info = tre.tre_plan_info()
-    assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448,
-                                    ctypes.byref(info)) == tre.TRE_ERR_INVALID_ARG
+
+    def status(wl, **over):
+        cfg = tre.config_from_workload(wl, **over)
+        return tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info))
+
+    assert status(MLA_SPARSE) == tre.TRE_OK
+    assert status(W.TINY, index_topk=8) == tre.TRE_ERR_INVALID_ARG       # GQA stack
+    assert status(MLA_SMALL, index_heads=16) == tre.TRE_ERR_INVALID_ARG  # without a K
+    assert status(MLA_SPARSE, index_heads=48) == tre.TRE_ERR_UNSUPPORTED
+    assert status(MLA_SPARSE, index_dim=96) == tre.TRE_ERR_UNSUPPORTED
+    assert status(MLA_SPARSE, index_topk=MLA_SPARSE.kv_capacity + 1) == tre.TRE_ERR_INVALID_ARG
+    assert status(MLA_SPARSE, index_topk=-1) == tre.TRE_ERR_INVALID_ARG
+
+
+def test_sparse_plan_bytes_follow_the_selection():
+    # dense reads every latent row; sparse reads every index key but only K latent rows
+    d = tre.tre_plan_inspect(tre.config_from_workload(W.MLA4_KV128K))
+    s = tre.tre_plan_inspect(tre.config_from_workload(W.MLA4_SPARSE128K))
+    wl = W.MLA4_SPARSE128K
+    C, L, cap = wl.kv_lora + wl.rope_dim, wl.n_layers, wl.kv_capacity
+    assert d.kv_bytes_at_capacity == L * (cap - 1) * C * 2
+    assert s.kv_bytes_at_capacity == L * ((cap - 1) * wl.index_dim * 2 + wl.index_topk * C * 2)
+    extra = L * 2 * (wl.index_heads * wl.index_dim * wl.q_lora +
+                     (wl.index_dim + wl.index_heads) * wl.hidden)
+    assert s.weight_bytes == d.weight_bytes + extra
 
 
 def test_fault_inject_plans_one_unsatisfiable_wait():

@@ -107,6 +107,10 @@ def test_workload_step_bytes_match_the_planner():
         row = (wl.kv_lora + wl.rope_dim) * 2 if wl.kind == "mla" else wl.n_kv_heads * wl.head_dim * 4
         read = info.kv_bytes_at_capacity * wl.prefill // (wl.kv_capacity - 1)
         lm = wl.vocab * 4 + 2 * wl.hidden if wl.vocab else 0
+        if wl.index_topk and wl.prefill + 1 > wl.index_topk:
+            # sparse MLA: every index key (+ the new one), the K chosen latent rows + the new one
+            read = wl.n_layers * (wl.prefill * wl.index_dim * 2 + wl.index_topk * row)
+            row += wl.index_dim * 2
         assert bench.workload_step_bytes(wl) == info.weight_bytes + read + wl.n_layers * row + lm
 
 
