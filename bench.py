@@ -513,7 +513,9 @@ class LayerSample:
             self.orc.moe_layer_step(self.sw, m["layers"][0], m["k_cache"][0], m["v_cache"][0],
                                     self.expert, pos, self.x)
         else:
-            self.orc.mla_layer_step(self.sw, m["layers"][0], m["latent_cache"][0], pos, self.x)
+            ic = m["index_cache"][0] if self.sw.index_topk else None  # sparse: the indexer too
+            self.orc.mla_layer_step(self.sw, m["layers"][0], m["latent_cache"][0], pos, self.x,
+                                    index_cache=ic)
         return (time.perf_counter() - t0) * self.wl.n_layers
 
     def describe(self) -> str:

@@ -210,7 +210,8 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
     g.nkk = (g.Kp + kTileK - 1) / kTileK;
     g.nstages = (t.r1 - t.r0 + kTileRows - 1) / kTileRows * g.nseg * g.nkk;
   } else {
-    g.rps = g.esz == 1 ? fp8_rows_per_stage(g.Kp, g.nseg, p.stage_bytes)
+    // E4M3: one tensor-core tile of 8 rows (gate / up: 4 of each) per stage at most
+    g.rps = g.esz == 1 ? min(8 / g.nseg, fp8_rows_per_stage(g.Kp, g.nseg, p.stage_bytes))
                        : gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes, g.esz);
     g.nkk = 1;
     g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
@@ -820,7 +821,7 @@ __device__ __forceinline__ int input_key(const Task& t) {
 // the RMSNorm scale (1 when the op has no norm).
 __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& gg, float* ub,
                                 float* red, int ctid, float* rn) {
-  const int K = gg.Kp, Ls = fp8_seg_len(K), span = 4 * Ls, NG = span / 4;  // 4-column groups
+  const int K = gg.Kp, Ls = fp8_half_len(K), span = 2 * Ls, NG = span / 4;  // 4-column groups
   const float* src = nullptr;
   const uint16_t* src_bf = nullptr;
   const uint16_t* gain = nullptr;
@@ -2490,6 +2491,92 @@ __device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, c
 }
 
 // ---- consumers -----------------------------------------------------------------------------------
+// ---- E4M3 GEMV on the tensor cores ------------------------------------------------------------
+// A stage holds up to 8 weight rows (gate / up: up to 4 rows of each) of the task's K-part at
+// a pitch of span + 16 bytes, span = 2 Lh (Lh: half the K-part, rounded up to 32 columns).
+// One mma.sync m16n8k32 E4M3 x E4M3 -> fp32 tile covers 32 columns of both halves of the 8
+// rows, the weights as stored: tile row r < 8 is weight row r at columns [c, c + 32), tile
+// row 8 + r the same row at [Lh + c, Lh + c + 32), so an ldmatrix.x4 is exactly the A
+// fragment.  The B operand holds the input's 4 E4M3 terms of those columns (load_input_e4m3):
+// columns 0-3 the terms of half 0, 4-7 those of half 1.  Of the 16 x 8 products a lane keeps
+// its row g's pair of terms of its half (lanes t4 < 2: half 0, t4 >= 2: half 1), weighed by
+// 16^-tau, the chunk's 2^-sg and the weight block scale (32 columns never straddle a
+// 128-column block).  All 8 warps share each stage, warp w taking the chunks w, w + 8, ...;
+// the lanes of a row and then the warps are summed (shuffles, shared memory), and one thread
+// per row finishes it.
+__device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint32_t gs, int ns,
+                         uint8_t* ring, uint64_t* full, uint64_t* empty, const uint32_t* tags,
+                         float* ub, const float* resid, float rn, float wsel, int uoff, int warp,
+                         int lane, int ctid, bool& ab, Best& best) {
+  const int Lh = fp8_half_len(g.Kp), P = fp8_row_pitch(g.Kp), nch = Lh / 32;
+  const uint8_t* frag = reinterpret_cast<const uint8_t*>(ub);
+  const float* csc = ub + 2 * Lh;            // 2^-sg per 32 columns of the span
+  float* red = ub + fp8_frag_floats(g.Kp);   // [2][kConsumerWarps][8]
+  const Fp8Scales fs = fp8_scales(p, t, g);
+  const bool two = g.nseg == 2;
+  const int gq = lane >> 2, t4 = lane & 3, half = t4 >> 1;
+  const float wa = (t4 & 1) ? 1.f / 256.f : 1.f, wb = wa * (1.f / 16.f);
+  // B: this lane's 8 bytes are term gq & 3 of half gq >> 2, column group t4 (+ 128 per chunk)
+  const uint8_t* bp = frag + (gq >> 2) * 4 * Lh + (gq & 3) * 32 + t4 * 8;
+  const int mat = lane >> 3, trow = lane & 7;  // ldmatrix: this lane's matrix and row
+  const uint32_t NS = (uint32_t)p.ring_stages;
+  for (int i = 0; i < ns; ++i) {
+    const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
+    const bool landed = stage_wait(p, full, tags, sidx);
+    const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
+    // tile row trow's stage row (gate / up: rows 0-3 gate, 4-7 up), clamped to a loaded row
+    const int sr = two ? ((trow >> 2) ? g.rps : 0) + min(trow & 3, nr - 1) : min(trow, nr - 1);
+    const uint32_t arow = smem_u32(ring + (size_t)slot * p.stage_bytes) +
+                          (uint32_t)(sr * P + (mat & 1) * Lh + (mat >> 1) * 16);
+    // the weight row of this lane's output row gq, for its block scales
+    const float* srow = two ? fp8_scale_row(fs, gq >> 2, n0 + min(gq & 3, nr - 1))
+                            : fp8_scale_row(fs, 0, n0 + min(gq, nr - 1));
+    float acc = 0.f;
+    if (landed) {
+      for (int cc = warp; cc < nch; cc += kConsumerWarps) {
+        uint32_t a[4];
+        ldsm_x4(arow + (uint32_t)(cc * 32), a[0], a[1], a[2], a[3]);
+        // columns past Kp are stale shared memory: zero them (the input is zero there)
+        const int c0 = cc * 32 + 4 * t4, c1 = Lh + c0;
+        if (c0 >= g.Kp) a[0] = 0u;
+        if (c0 + 16 >= g.Kp) a[2] = 0u;
+        if (c1 >= g.Kp) a[1] = 0u;
+        if (c1 + 16 >= g.Kp) a[3] = 0u;
+        const uint2 b = *reinterpret_cast<const uint2*>(bp + cc * 128);
+        float d[4];
+        mma_e4m3(d, a, b.x, b.y);
+        const int col = half * Lh + cc * 32;
+        const float v = half ? fmaf(d[3], wb, d[2] * wa) : fmaf(d[1], wb, d[0] * wa);
+        acc = fmaf(v, __ldg(srow + ((g.k0 + col) >> 7)) * csc[col >> 5], acc);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    float* rb = red + (i & 1) * kConsumerWarps * 8;
+    if (t4 == 0) rb[warp * 8 + gq] = acc;
+    if (consumer_sync_or(!landed, kConsumerThreads)) {
+      ab = true;
+      return;
+    }
+    if (ctid < nr && (!two || ctid < 4)) {
+      float v = 0.f, u = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        v += rb[w * 8 + ctid];
+        if (two) u += rb[w * 8 + 4 + ctid];
+      }
+      if (two) {  // gate row ctid (v), up row ctid (u)
+        const float aa = v * rn, bb = u * rn;
+        p.u[uoff + n0 + ctid] = wsel * (aa / (1.f + expf(-aa)) * bb);
+      } else {
+        gemv_emit(p, t, g, n0 + ctid, v, rn, resid, best);
+      }
+    }
+  }
+}
+
 // MLA = true: the absorbed-MLA stack's kernel (MLA tiles, no GQA attention); false: GQA /
 // MoE.  Separate instantiations keep each kernel's register allocation to its own tiles.
 // TILED: GEMV stages are 16-row tensor-core tiles (multi-token plans).
@@ -2591,9 +2678,15 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
                            ub + p.ub_floats - kTileRedFloats, resid, rnt, wsel, uoff, best, warp,
                            lane, ctid, ab);
       }
+      const bool coop = F8 && g.esz == 1;  // E4M3 stages: every warp takes part in each
+      if constexpr (F8) {
+        if (coop)
+          fp8_task(p, t, g, gs, ns, ring, full, empty, tags, ub, resid, rn, wsel, uoff, warp,
+                   lane, ctid, ab, best[0]);
+      }
       // stage gs + i belongs to warp (gs + i) % 8; each warp takes its stages in order
       const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
-      for (int i = first; i < (TILED ? 0 : ns); i += kConsumerWarps) {
+      for (int i = first; i < (TILED || coop ? 0 : ns); i += kConsumerWarps) {
         const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
         if (!stage_wait(p, full, tags, sidx)) {
           ab = true;
@@ -2601,92 +2694,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
-        if (F8 && g.esz == 1) {
-          // E4M3 rows on the tensor cores, mma.sync m16n8k32 E4M3 x E4M3 -> fp32, the weights
-          // as stored (no conversion).  A tile is 4 weight rows, each cut into 4 segments of
-          // Ls columns: tile row 4 j + q (j < 2) is segment q of weight row j, tile row
-          // 8 + 4 j + q segment q of row 2 + j.  Two mma per 32 columns, n-tile 0 with the
-          // input terms of segments 0, 1 as columns (column 4 s + tau: segment s, term tau),
-          // n-tile 1 with segments 2, 3; lane (g, t4) of the n-tile holding its segment
-          // keeps terms 2 (t4 & 1) and + 1 when t4 / 2 = q % 2 (the other products are
-          // discarded).  An ldmatrix.x4 of 32 columns of the 16 tile rows is exactly the A
-          // fragment.  32 columns lie in one 128-column scale block and one input chunk: the
-          // lane weighs its terms by 16^-tau, the block scale and the chunk's 2^-sg; the
-          // segments and terms are summed with shuffles.  Gate / up tiles take gate rows
-          // r, r + 1 as rows 0, 1 and the same up rows as 2, 3.
-          const uint32_t sb = smem_u32(ring + (size_t)slot * p.stage_bytes);
-          const Fp8Scales fs = fp8_scales(p, t, g);
-          const int P = fp8_row_pitch(g.Kp), Ls = fp8_seg_len(g.Kp);
-          const int gq = lane >> 2, t4 = lane & 3, qs = gq & 3;
-          const bool mine = (t4 >> 1) == (qs & 1);
-          const float wa = (t4 & 1) ? 1.f / 256.f : 1.f, wb = wa * (1.f / 16.f);
-          const uint8_t* frb = reinterpret_cast<const uint8_t*>(ub);
-          const float* csc = ub + 4 * Ls;
-          const uint8_t* bp0 = frb + ((gq >> 2) * 4 * Ls + (gq & 3) * 32 + t4 * 8);
-          const uint8_t* bp1 = bp0 + 2 * 4 * Ls;
-          const bool two = g.nseg == 2;
-          const int step = two ? 2 : 4;           // weight rows per tile
-          // ldmatrix row addresses: matrix lane >> 3 (0: tile rows 0-7, 1: rows 8-15, 2 / 3 the
-          // same rows 16 columns further), tile row lane & 7
-          const int mat = lane >> 3, trow = (mat & 1) * 8 + (lane & 7);
-          const int tj = (trow >> 3) * 2 + ((trow & 7) >> 2), tq = trow & 3;
-          for (int r = 0; r < nr; r += step) {
-            const int nv = min(step, nr - r);
-            auto slot_row = [&](int jj) {
-              if (two) return (jj >> 1) * g.rps + r + min(jj & 1, nv - 1);  // gate, gate, up, up
-              return r + min(jj, nv - 1);
-            };
-            auto weight_row = [&](int jj, int& seg) {
-              seg = two ? jj >> 1 : 0;
-              return n0 + r + min(two ? (jj & 1) : jj, nv - 1);
-            };
-            const uint32_t arow = sb + (uint32_t)(slot_row(tj) * P + tq * Ls + (mat >> 1) * 16);
-            int sg0, sg1;
-            const int wr0 = weight_row(gq >> 2, sg0), wr1 = weight_row(2 + (gq >> 2), sg1);
-            const float* srow0 = fp8_scale_row(fs, sg0, wr0);
-            const float* srow1 = fp8_scale_row(fs, sg1, wr1);
-            float tot0 = 0.f, tot1 = 0.f;
-            for (int c = 0; c < Ls; c += 32) {
-              uint32_t a[4];
-              ldsm_x4(arow + (uint32_t)c, a[0], a[1], a[2], a[3]);
-              // weight bytes past Kp are stale shared memory: zero them (the input is zero there)
-              const int colA = qs * Ls + c + 4 * t4;
-              if (colA >= g.Kp) a[0] = a[1] = 0u;
-              if (colA + 16 >= g.Kp) a[2] = a[3] = 0u;
-              const uint2 b0 = *reinterpret_cast<const uint2*>(bp0 + (c >> 5) * 128);
-              const uint2 b1 = *reinterpret_cast<const uint2*>(bp1 + (c >> 5) * 128);
-              float d0[4], d1[4];
-              mma_e4m3(d0, a, b0.x, b0.y);
-              mma_e4m3(d1, a, b1.x, b1.y);
-              if (mine) {
-                const float* dd = (qs >> 1) ? d1 : d0;
-                const int col = qs * Ls + c;
-                const float cscale = csc[col >> 5];
-                const int blk = (g.k0 + col) >> 7;
-                tot0 = fmaf(fmaf(dd[1], wb, dd[0] * wa), __ldg(srow0 + blk) * cscale, tot0);
-                tot1 = fmaf(fmaf(dd[3], wb, dd[2] * wa), __ldg(srow1 + blk) * cscale, tot1);
-              }
-            }
-            // sum the segments and terms: the 16 lanes of half j hold rows j (tot0), 2 + j (tot1)
-            float v0 = mine ? tot0 : 0.f, v1 = mine ? tot1 : 0.f;
-#pragma unroll
-            for (int off = 1; off < 16; off <<= 1) {
-              v0 += __shfl_xor_sync(0xffffffffu, v0, off);
-              v1 += __shfl_xor_sync(0xffffffffu, v1, off);
-            }
-            const int jrow = lane >> 4;  // lanes 0 / 16 emit rows jrow and 2 + jrow
-            if ((lane & 15) == 0 && jrow < (two ? nv : min(2, nv))) {
-              if (two) {  // rows: gate jrow (v0), up jrow (v1)
-                const float aa = v0 * rn, bb = v1 * rn;
-                p.u[uoff + n0 + r + jrow] = wsel * (aa / (1.f + expf(-aa)) * bb);
-              } else {
-                gemv_emit(p, t, g, n0 + r + jrow, v0, rn, resid, best[0]);
-              }
-            }
-            if (!two && (lane & 15) == 0 && 2 + jrow < nv)
-              gemv_emit(p, t, g, n0 + r + 2 + jrow, v1, rn, resid, best[0]);
-          }
-        } else if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+        if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;
           for (int r = 0; r < nr; r += 2) {
             const int np = min(2, nr - r);

@@ -404,15 +404,15 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max),
                                                gemv_part_align(s.tiles, o.esz == 1));
     // E4M3 rows: the tensor-core operand of the input covers the 4 row segments
-    xs = std::max(xs, o.esz == 1 ? fp8_frag_floats(kp) : kp);
+    xs = std::max(xs, o.esz == 1 ? fp8_frag_floats(kp) + kFp8RedFloats : kp);
     need = std::max(need, s.tiles ? kTileRows * kTilePitch
                                   : o.esz == 1 ? o.nseg * fp8_row_pitch(kp) : o.nseg * kp * o.esz);
   }
   // A ring stage holds whole rows of one K-part (gate/up: a row of each matrix), or the K
   // and V rows of 8-64 cached positions.
   int sb = c.stage_bytes ? c.stage_bytes : std::max(kDefaultStageBytes, (need + 1023) / 1024 * 1024);
-  // E4M3 plans: a stage of 8 hidden-wide rows (two full 4-row tensor-core tiles; gate / up:
-  // 4 row pairs) when that is at least the default
+  // E4M3 plans: a stage of 8 hidden-wide rows (one full tensor-core tile; gate / up: 4 row
+  // pairs) when that is at least the default
   if (!c.stage_bytes && s.wfp8 && 8 * fp8_row_pitch(s.d) >= sb)
     sb = (8 * fp8_row_pitch(s.d) + 1023) / 1024 * 1024;  // ring slots stay 1024-byte aligned
   if (!c.stage_bytes)

@@ -57,20 +57,17 @@ TRE_HD inline int gemv_rows_per_stage(int K, int nseg, int stage_bytes, int esz 
 // K-part boundaries: multiples of 8 columns (16 bytes of bf16), of 16 for tensor-core
 // tiles, of 128 for E4M3 rows (a K-part then covers whole 128-column scale blocks)
 TRE_HD inline int gemv_part_align(bool tiles, bool fp8) { return fp8 ? 128 : tiles ? 16 : 8; }
-// E4M3 rows on the tensor cores are read as 4 segments of fp8_seg_len(Kp) columns, an odd
-// multiple of 32 (the loop takes 32 columns of every segment at a time; the 4 segments of
-// a row then start on 4 different 32-byte bank offsets, and with the pitch's 16-byte skew
-// between rows an ldmatrix's 8 tile rows hit 8 different 16-byte bank groups).  The input
-// operand covers the 4 segments (fp8_span columns, zero past Kp).
-TRE_HD inline int fp8_seg_len(int Kp) {
-  const int l = ((Kp + 3) / 4 + 31) / 32 * 32;
-  return l % 64 ? l : l + 32;
-}
-TRE_HD inline int fp8_span(int Kp) { return 4 * fp8_seg_len(Kp); }
+// E4M3 rows on the tensor cores are read as 2 halves of fp8_half_len(Kp) columns (a
+// multiple of 32: the tiles take 32 columns of both halves at a time); the input operand
+// covers both (fp8_span columns, zero past Kp).  Rows sit at a pitch of span + 16 bytes, an
+// odd number of 16-byte units, so that an ldmatrix's 8 rows hit 8 different bank groups.
+TRE_HD inline int fp8_half_len(int Kp) { return (Kp + 63) / 64 * 32; }
+TRE_HD inline int fp8_span(int Kp) { return 2 * fp8_half_len(Kp); }
 TRE_HD inline int fp8_row_pitch(int Kp) { return fp8_span(Kp) + 16; }
 // The input operand of an E4M3 GEMV: 4 E4M3 terms per input (4 bytes) in fragment order,
-// then one scale per 32 columns: its size in floats
+// then one scale per 32 columns: its size in floats (the cross-warp sums follow it)
 TRE_HD inline int fp8_frag_floats(int Kp) { return fp8_span(Kp) + fp8_span(Kp) / 32; }
+constexpr int kFp8RedFloats = 2 * kConsumerWarps * 8;
 TRE_HD inline int fp8_rows_per_stage(int Kp, int nseg, int stage_bytes) {
   const int r = stage_bytes / (nseg * fp8_row_pitch(Kp));
   return r < 1 ? 1 : r;

@@ -158,7 +158,7 @@ def test_sparse_plan_before_and_after_k():
 
 def test_sparse_small_contexts():
     """Fewer cached positions than scoring splits (most splits score nothing), pos 0."""
-    run_sparse(SMALL.replace(prefill=0, index_topk=4, decode_steps=3, n_layers=1), steps=3)
+    run_sparse(SMALL.replace(prefill=0, index_topk=2, decode_steps=3, n_layers=1), steps=3)
     run_sparse(SMALL.replace(prefill=9, index_topk=4, decode_steps=2, n_layers=1), steps=2)
 
 
