@@ -841,12 +841,15 @@ __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& 
   float* cs = ub + span;
   float ss = 0.f;
   constexpr int B = 4;  // groups a thread fetches before it stores any
-  for (int q0 = ctid; q0 < NG; q0 += B * kConsumerThreads) {  // warp-uniform trip count
+  // the loop runs from the warp's first group, so every lane of a warp takes the same number
+  // of trips (the shuffles below need all 32); groups past NG only skip their stores
+  const int lane = ctid & 31;
+  for (int q0 = ctid - lane; q0 < NG; q0 += B * kConsumerThreads) {
     float4 xv[B];
     uint2 gv[B];
 #pragma unroll
     for (int u = 0; u < B; ++u) {
-      const int q = q0 + u * kConsumerThreads, c = min(4 * q, K - 4);  // clamped fetch
+      const int q = q0 + lane + u * kConsumerThreads, c = min(4 * q, K - 4);  // clamped fetch
       if (src_bf) {
         const uint2 w = __ldg(reinterpret_cast<const uint2*>(src_bf + c));
         xv[u] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
@@ -857,7 +860,7 @@ __device__ void load_input_e4m3(const Params& p, const Task& t, const GemvGeom& 
     }
 #pragma unroll
     for (int u = 0; u < B; ++u) {
-      const int q = q0 + u * kConsumerThreads, col = 4 * q;
+      const int q = q0 + lane + u * kConsumerThreads, col = 4 * q;
       const bool live = col < K;  // (all lanes run the shuffles below)
       float e[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
       if (!live) {
