@@ -348,6 +348,15 @@ tre_status tre_layers_step(tre_engine* e, const float* x_in_dev, float* x_out_de
  * engine's last stream.  TRE_ERR_UNSUPPORTED for other kinds. */
 tre_status tre_debug_routing(tre_engine* e, int32_t* idx_host, float* w_host);
 
+/* Per-step invariants, a debug check that stands in for a memory checker: wait for the
+ * engine's last stream, then check that every dependency counter some task waits on stands
+ * at (persistent steps run since create / tre_reset) x (its increments per step), and that
+ * the guard words the engine keeps after every buffer it owns still hold their fill
+ * pattern.  *bad_counter_out receives the first counter that does not (or -1),
+ * *bad_guard_out the index of the first overwritten guard (or -1).  The counters of
+ * kernel-per-op launches (their own array) are not checked.  Host copies only. */
+tre_status tre_debug_check(tre_engine* e, int32_t* bad_counter_out, int32_t* bad_guard_out);
+
 /* Sparse MLA: wait for the engine's last stream, then copy layer `layer`'s index scores
  * of the last step (score_host: float[pos + 1], I[0 .. pos] as defined above, may be
  * NULL) and its chosen positions (sel_host: int32[index_topk], in no particular order,

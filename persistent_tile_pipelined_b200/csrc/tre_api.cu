@@ -44,6 +44,8 @@ struct tre_engine {
   int n_groups = 0;              // op groups of the plan (kernel-per-op form)
   uint32_t* op_counters = nullptr;  // counters the kernel-per-op launches bump
   int launch_mode = TRE_LAUNCH_PERSISTENT;
+  std::vector<uint32_t> expected;  // per counter: increments per step (0: no task waits on it)
+  std::vector<size_t> guards;      // offsets of the guard words after every owned buffer
 };
 
 #define TRE_EXPORT extern "C" __attribute__((visibility("default")))
@@ -99,13 +101,19 @@ tre_status encode_cache_map(void* cache, int C, long long rows, int box_rows, vo
 }  // namespace tre
 
 namespace {
+constexpr size_t kGuardBytes = 64;       // guard words after every engine-owned buffer
+constexpr unsigned char kGuardFill = 0x5A;
+
 struct Carve {  // bump allocator over the engine's single device block
   size_t off = 0;
+  std::vector<size_t> guards;
   template <class T>
   size_t take(size_t count) {
     off = (off + 255) & ~size_t(255);
     size_t at = off;
     off += count * sizeof(T);
+    guards.push_back(off);  // kGuardBytes of fill pattern right after the buffer
+    off += kGuardBytes;
     return at;
   }
 };
@@ -387,6 +395,13 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   };
   if ((ce = cudaMemset(e->block, 0, e->block_bytes)) != cudaSuccess)
     return fail_free(ce, "cudaMemset(engine state)");
+  e->guards = cv.guards;
+  for (size_t g : e->guards)
+    if ((ce = cudaMemset(B + g, kGuardFill, kGuardBytes)) != cudaSuccess)
+      return fail_free(ce, "cudaMemset(guards)");
+  e->expected.assign(s.n_counters, 0u);
+  for (const Task& t : tasks)
+    if (t.dep >= 0) e->expected[t.dep] = t.dep_count;
   if ((ce = cudaMemcpy(B + o_tasks, tasks.data(), tasks.size() * sizeof(Task),
                        cudaMemcpyHostToDevice)) != cudaSuccess)
     return fail_free(ce, "upload tasks");
@@ -720,6 +735,38 @@ TRE_EXPORT tre_status tre_debug_routing(tre_engine* e, int32_t* idx_host, float*
   const size_t n = (size_t)e->shape.L * e->shape.topk;
   if (idx_host) CK(cudaMemcpy(idx_host, e->base.route_idx, n * 4, cudaMemcpyDeviceToHost));
   if (w_host) CK(cudaMemcpy(w_host, e->base.route_w, n * 4, cudaMemcpyDeviceToHost));
+  return TRE_OK;
+}
+
+TRE_EXPORT tre_status tre_debug_check(tre_engine* e, int32_t* bad_counter_out,
+                                      int32_t* bad_guard_out) {
+  if (!e || !bad_counter_out || !bad_guard_out) {
+    set_error("tre_debug_check: NULL argument");
+    return TRE_ERR_INVALID_ARG;
+  }
+  CK(cudaSetDevice(e->device));
+  if (e->last_stream) CK(cudaStreamSynchronize(e->last_stream));
+  CK(cudaDeviceSynchronize());
+  const int n = e->shape.n_counters;
+  std::vector<uint32_t> c(n);
+  CK(cudaMemcpy(c.data(), e->base.counters, (size_t)n * 4, cudaMemcpyDeviceToHost));
+  *bad_counter_out = -1;
+  for (int i = 0; i < n; ++i)
+    if (e->expected[i] && c[i] != e->epoch * e->expected[i]) {
+      *bad_counter_out = i;
+      break;
+    }
+  *bad_guard_out = -1;
+  std::vector<unsigned char> g(kGuardBytes);
+  const uint8_t* B = static_cast<const uint8_t*>(e->block);
+  for (size_t k = 0; k < e->guards.size() && *bad_guard_out < 0; ++k) {
+    CK(cudaMemcpy(g.data(), B + e->guards[k], kGuardBytes, cudaMemcpyDeviceToHost));
+    for (unsigned char b : g)
+      if (b != kGuardFill) {
+        *bad_guard_out = (int32_t)k;
+        break;
+      }
+  }
   return TRE_OK;
 }
 

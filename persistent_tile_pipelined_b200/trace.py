@@ -32,6 +32,10 @@ def op_name(tt: dict, i: int) -> str:
         return "attention"
     if tt["type"][i] == 2:
         return "mla_attention"
+    if tt["type"][i] == 3:
+        return "index_score"
+    if tt["type"][i] == 4:
+        return "index_select"
     return OP_NAMES.get(int(tt["op"][i]), "?")
 
 

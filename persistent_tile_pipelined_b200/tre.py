@@ -74,6 +74,7 @@ TRE_LAUNCH_PERSISTENT, TRE_LAUNCH_PER_OP = 0, 1
 
 EXPORTED = ("tre_create", "tre_destroy", "tre_decode_step", "tre_decode_step_host",
             "tre_decode_step_static", "tre_layers_step", "tre_debug_routing", "tre_debug_index",
+            "tre_debug_check",
             "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
             "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
             "tre_plan_inspect", "tre_plan_tasks", "tre_plan_op_groups", "tre_last_error")
@@ -101,6 +102,7 @@ def _load() -> ctypes.CDLL:
     L.tre_plan_op_groups.restype = i32
     L.tre_debug_routing.argtypes = [vp, vp, vp]
     L.tre_debug_index.argtypes = [vp, i32, i32, vp, vp, ctypes.POINTER(i32)]
+    L.tre_debug_check.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.tre_get_status.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.tre_reset.argtypes = [vp, vp]
     L.tre_debug_hidden.argtypes = [vp, vp, vp]
@@ -114,7 +116,7 @@ def _load() -> ctypes.CDLL:
     L.tre_last_error.restype = ctypes.c_char_p
     for name in ("tre_create", "tre_decode_step", "tre_decode_step_host",
                  "tre_decode_step_static", "tre_layers_step", "tre_debug_routing",
-                 "tre_debug_index", "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
+                 "tre_debug_index", "tre_debug_check", "tre_decode_tokens", "tre_decode_loop", "tre_set_launch_mode", "tre_get_status",
                  "tre_reset", "tre_debug_hidden", "tre_debug_trace", "tre_step_bytes",
                  "tre_plan_inspect"):
         getattr(L, name).restype = ctypes.c_int
@@ -201,6 +203,13 @@ def tre_debug_index(h, layer: int, pos: int, index_topk: int):
                               sel.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)),
           "tre_debug_index")
     return sc, sel[:n.value].copy()
+
+
+def tre_debug_check(h):
+    """(first counter off its per-step invariant or -1, first overwritten guard or -1)."""
+    c, g = ctypes.c_int32(), ctypes.c_int32()
+    check(lib.tre_debug_check(h, ctypes.byref(c), ctypes.byref(g)), "tre_debug_check")
+    return c.value, g.value
 
 
 def tre_get_status(h):
@@ -461,6 +470,10 @@ class Engine:
 
     def routing(self):
         return tre_debug_routing(self.h, self.cfg.n_layers, self.cfg.top_k)
+
+    def check(self):
+        """Per-step invariants: (bad counter or -1, overwritten guard or -1)."""
+        return tre_debug_check(self.h)
 
     def index(self, layer: int, pos: int):
         """Sparse MLA: (index scores [pos + 1], chosen positions) of `layer` at the last step."""

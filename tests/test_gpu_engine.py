@@ -174,6 +174,33 @@ def test_fault_inject_times_out_without_hanging_and_context_survives():
     run_and_compare(wl, steps=1)
 
 
+def test_step_invariants_hold_and_catch_a_stalled_step():
+    """tre_debug_check: after persistent steps (with a kernel-per-op step between them)
+    every waited-on counter stands at steps x increments and every guard word is intact; a
+    step stalled by the fault-injection plan leaves a counter behind (guards intact), and
+    tre_reset restores the invariant."""
+    wl = W.TINY
+    model, dev, eng = make(wl, debug=0)
+    for i in range(3):
+        if i == 1:
+            eng.set_launch_mode(tre.TRE_LAUNCH_PER_OP)
+        eng.step(W.first_token(wl), wl.prefill + i)
+        eng.set_launch_mode(tre.TRE_LAUNCH_PERSISTENT)
+    torch.cuda.synchronize()
+    assert eng.status() == (0, 0)
+    assert eng.check() == (-1, -1)
+    eng.close()
+    model, dev, eng = make(wl, debug=tre.TRE_DEBUG_FAULT_INJECT, dep_timeout_us=20000)
+    eng.step(W.first_token(wl), wl.prefill)
+    torch.cuda.synchronize()
+    assert eng.status()[0] == tre.TRE_ERR_DEP_TIMEOUT
+    bad_counter, bad_guard = eng.check()
+    assert bad_counter >= 0 and bad_guard == -1
+    eng.reset()
+    assert eng.check() == (-1, -1)
+    eng.close()
+
+
 def test_host_side_argument_errors():
     wl = W.TINY
     model, dev, eng = make(wl, debug=0)
