@@ -120,7 +120,8 @@ typedef struct {
   int32_t stream_policy;        /* when the producer streams the next op's tiles:
                                    1 = as soon as ring slots free up; 2 = once this SM
                                    has published the current op (its publish then does
-                                   not wait behind in-flight copies); 0 = default (2)   */
+                                   not wait behind in-flight copies); 3..6 = its first
+                                   1..4 stages at once, the rest as 2; 0 = default (2)   */
   int32_t multi_token_gemv;     /* GEMV form of a plan with max_tokens_per_step > 1:
                                    1 = CUDA-core rows; 2 = tensor-core tiles of 16 rows
                                    (hidden and ffn multiples of 16); 0 = the planner's

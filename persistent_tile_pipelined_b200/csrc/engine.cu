@@ -629,6 +629,28 @@ __device__ __forceinline__ bool op_boundary(const Task& a, const Task& b) {
   return a.type != b.type || a.op != b.op || a.layer != b.layer;
 }
 
+// Producer: wait (bounded) until this SM's consumers have finished task ti - 1.
+__device__ bool hold_for_consumers(const Params& p, const volatile int* done, int ti, int detail,
+                                   int lane) {
+  bool r = true;
+  if (lane == 0) {
+    const uint64_t w0 = globaltimer_ns();
+    long long c0 = clock64();
+    while (*done < ti) {
+      __nanosleep(32);
+      if (clock64() - c0 > kCheckCycles) {
+        if (aborted(p) || (long long)(globaltimer_ns() - w0) > 2 * p.timeout_ns) {
+          if (!aborted(p)) record_error(p, TRE_ERR_DEP_TIMEOUT, detail);
+          r = false;
+          break;
+        }
+        c0 = clock64();
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+}
+
 template <bool TILED>
 __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, uint32_t* tags,
@@ -648,27 +670,14 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
       if (!ok) break;
     }
-    if (p.hold_next_op && ti > 0 && op_boundary(my[ti - 1], t)) {
-      // hold the next op's tiles until this SM's consumers have finished (and published)
-      // the previous task, so that their publish does not wait behind queued copies
-      bool r = true;
-      if (lane == 0) {
-        const uint64_t w0 = globaltimer_ns();
-        long long c0 = clock64();
-        while (*done < ti) {
-          __nanosleep(32);
-          if (clock64() - c0 > kCheckCycles) {
-            if (aborted(p) || (long long)(globaltimer_ns() - w0) > 2 * p.timeout_ns) {
-              if (!aborted(p)) record_error(p, TRE_ERR_DEP_TIMEOUT, t.id);
-              r = false;
-              break;
-            }
-            c0 = clock64();
-          }
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
-      if (!ok) break;
+    // at an op boundary, hold the next op's tiles (all of them, or those after its first
+    // hold_next_op - 1 stages) until this SM's consumers have finished (and published) the
+    // previous task, so that their publish does not wait behind queued copies
+    int hold_at = -1;
+    if (p.hold_next_op > 0 && ti > 0 && op_boundary(my[ti - 1], t)) hold_at = p.hold_next_op - 1;
+    if (hold_at == 0 && !hold_for_consumers(p, done, ti, t.id, lane)) {
+      ok = false;
+      break;
     }
     if (needs_route(p, t)) {  // the expert ids pick the addresses: wait for the routing
       bool r = true;
@@ -710,6 +719,10 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
     TileStage ts{};
     if (tiled) ts = tile_first(t, g);
     for (int i = 0; i < ns; ++i, ++gs) {
+      if (i > 0 && i == hold_at && !hold_for_consumers(p, done, ti, t.id, lane)) {
+        ok = false;
+        break;
+      }
       if (!TILED) {  // whole-row kernels: from the stage count (measured faster there)
         slot = gs % NS;
         ph = (gs / NS) & 1u;
@@ -2536,22 +2549,43 @@ __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint
                             : fp8_scale_row(fs, 0, n0 + min(gq, nr - 1));
     float acc = 0.f;
     if (landed) {
-      for (int cc = warp; cc < nch; cc += kConsumerWarps) {
-        uint32_t a[4];
-        ldsm_x4(arow + (uint32_t)(cc * 32), a[0], a[1], a[2], a[3]);
-        // columns past Kp are stale shared memory: zero them (the input is zero there)
-        const int c0 = cc * 32 + 4 * t4, c1 = Lh + c0;
-        if (c0 >= g.Kp) a[0] = 0u;
-        if (c0 + 16 >= g.Kp) a[2] = 0u;
-        if (c1 >= g.Kp) a[1] = 0u;
-        if (c1 + 16 >= g.Kp) a[3] = 0u;
-        const uint2 b = *reinterpret_cast<const uint2*>(bp + cc * 128);
-        float d[4];
-        mma_e4m3(d, a, b.x, b.y);
-        const int col = half * Lh + cc * 32;
-        const float v = half ? fmaf(d[3], wb, d[2] * wa) : fmaf(d[1], wb, d[0] * wa);
-        acc = fmaf(v, __ldg(srow + ((g.k0 + col) >> 7)) * csc[col >> 5], acc);
+      // kU chunks at a time (chunks w, w + 8, ...), every load issued before the products,
+      // so that a warp keeps several ldmatrix / scale loads and mma in flight
+      constexpr int kU = 4;
+      float accu[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) accu[u] = 0.f;
+      for (int cb = warp; cb < nch; cb += kU * kConsumerWarps) {
+        uint32_t a[kU][4];
+        uint2 b[kU];
+        float sc[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int cc = min(cb + u * kConsumerWarps, nch - 1);  // clamped: in-range reads
+          ldsm_x4(arow + (uint32_t)(cc * 32), a[u][0], a[u][1], a[u][2], a[u][3]);
+          b[u] = *reinterpret_cast<const uint2*>(bp + cc * 128);
+          const int col = half * Lh + cc * 32;
+          sc[u] = __ldg(srow + ((g.k0 + col) >> 7)) * csc[col >> 5];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int cc = cb + u * kConsumerWarps;
+          // columns past Kp are stale shared memory: zero them (the input is zero there); a
+          // chunk past the last one (clamped above) counts nothing
+          const int c0 = cc * 32 + 4 * t4, c1 = Lh + c0;
+          const bool live = cc < nch;
+          if (!live || c0 >= g.Kp) a[u][0] = 0u;
+          if (!live || c0 + 16 >= g.Kp) a[u][2] = 0u;
+          if (!live || c1 >= g.Kp) a[u][1] = 0u;
+          if (!live || c1 + 16 >= g.Kp) a[u][3] = 0u;
+          float d[4];
+          mma_e4m3(d, a[u], b[u].x, b[u].y);
+          const float v = half ? fmaf(d[3], wb, d[2] * wa) : fmaf(d[1], wb, d[0] * wa);
+          accu[u] = fmaf(v, sc[u], accu[u]);
+        }
       }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) acc += accu[u];
       __syncwarp();
       if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
     }

@@ -258,7 +258,7 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   p.pf_window = cfg->l2_prefetch_kb > 0 ? 1024LL * cfg->l2_prefetch_kb : 1024LL * kDefaultPrefetchKB;
   p.token = token;
   p.m = 1;
-  p.hold_next_op = cfg->stream_policy != 1;
+  p.hold_next_op = cfg->stream_policy == 1 ? 0 : cfg->stream_policy >= 3 ? cfg->stream_policy - 1 : 1;
   for (int v = 0; v < kMaxTokens; ++v) p.tokens[v] = token;
   p.pos = pos;
   p.epoch = 1;  // counters were just cleared

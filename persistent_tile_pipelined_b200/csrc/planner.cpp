@@ -301,8 +301,8 @@ static tre_status validate(const tre_config& c) {
   if (c.dep_timeout_us < 0) return fail(TRE_ERR_INVALID_ARG, "dep_timeout_us < 0");
   if (c.multi_token_gemv < 0 || c.multi_token_gemv > 2)
     return fail(TRE_ERR_INVALID_ARG, "multi_token_gemv must be 0, 1 or 2");
-  if (c.stream_policy < 0 || c.stream_policy > 2)
-    return fail(TRE_ERR_INVALID_ARG, "stream_policy must be 0, 1 or 2");
+  if (c.stream_policy < 0 || c.stream_policy > 6)
+    return fail(TRE_ERR_INVALID_ARG, "stream_policy must be in [0, 6]");
   if (c.gemv_kpart_max < 0 || (c.gemv_kpart_max > 0 && c.gemv_kpart_max < 512))
     return fail(TRE_ERR_INVALID_ARG, "gemv_kpart_max must be 0 or >= 512");
   if (c.num_sms < 0 || c.kv_splits < 0 || c.stage_bytes < 0 || c.ring_stages < 0)

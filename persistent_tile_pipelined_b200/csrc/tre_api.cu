@@ -492,7 +492,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.kpart_max = s.kpart_max;
   p.m = 1;
   // default: hold (measured faster on the 8B-shaped stack: 0.683 vs 0.665 of peak)
-  p.hold_next_op = cfg->stream_policy != 1;
+  p.hold_next_op = cfg->stream_policy == 1 ? 0 : cfg->stream_policy >= 3 ? cfg->stream_policy - 1 : 1;
   p.gemv_tiles = s.tiles;
   p.wfp8 = s.wfp8;
   p.err = reinterpret_cast<int32_t*>(B + o_err);

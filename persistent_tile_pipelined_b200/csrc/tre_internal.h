@@ -257,7 +257,8 @@ struct Params {
   int32_t tokens[kMaxTokens];
   uint32_t epoch;
   int flags;
-  int hold_next_op;                // producer waits for this SM's publish at op boundaries
+  int hold_next_op;                // > 0: at op boundaries the producer issues hold_next_op - 1
+                                   // stages, then waits for this SM's publish; 0: no wait
   int gemv_tiles;                  // GEMV stages are 16-row tiles (multi-token plans)
   int wfp8;                        // QKV / O / gate-up / down weights are E4M3 + block scales
   long long timeout_ns;
