@@ -154,7 +154,7 @@ __device__ __forceinline__ int gemv_K(const Params& p, int op) {
     case OP_MDOWN: return (p.nshared + p.topk) * p.Fe;
     case OP_UQ: return p.QL;
     case OP_UK: case OP_UV: return p.KL;   // W_uk / W_uv rows are KL wide
-    case OP_MO: return p.Hq * p.VD;
+    case OP_MO: case OP_MOS: return p.Hq * p.VD;
     default: return p.d;
   }
 }
@@ -198,6 +198,9 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   } else if (t.op == OP_MDOWN) {  // aux = slot | block << 8
     g.part = t.aux & 0xff;
     g.np = p.nshared + p.topk;
+  } else if (t.op == OP_MOS) {    // aux = slice | block << 8 | slices << 16
+    g.part = t.aux & 0xff;
+    g.np = (t.aux >> 16) & 0xff;
   } else {
     g.part = t.aux & 0xff;
     g.np = max(1, t.aux >> 8);
@@ -266,6 +269,7 @@ __device__ __forceinline__ const uint8_t* part_row(const Params& p, const Task& 
     case OP_UK: return wbytes(L.w[TRE_W_UK]) + (size_t)n * K * 2;
     case OP_UV: return wbytes(L.w[TRE_W_UV]) + (size_t)n * K * 2;
     case OP_MO:
+    case OP_MOS:
       if (g.np > 1) *contig = 1;
       return wbytes(L.w[TRE_W_MLA_O]) + ((size_t)n * K + g.k0) * 2;
     case OP_SGU: return wbytes(L.w[seg ? TRE_W_SHARED_UP : TRE_W_SHARED_GATE]) + (size_t)n * K * 2;
@@ -810,7 +814,7 @@ __device__ __forceinline__ int input_key(const Task& t) {
   int cls;
   switch (t.op) {
     case OP_QKV: case OP_MDQKV: cls = 0; break;
-    case OP_O: case OP_MO: cls = 1; break;
+    case OP_O: case OP_MO: case OP_MOS: cls = 1; break;
     case OP_GU: case OP_ROUTER: case OP_SGU: case OP_RGU: cls = 2; break;
     case OP_DOWN: case OP_MDOWN: cls = 3; break;
     case OP_UQ: cls = 5; break;
@@ -957,7 +961,7 @@ __device__ void load_input(const Params& p, const Task& t, const GemvGeom& gg, f
     case OP_DOWN: case OP_MDOWN: src = p.u; vstride = p.F; break;
     case OP_UQ: src = p.cqkv; gain = p.layers[t.layer].w[TRE_W_Q_NORM]; break;
     case OP_UV: src = p.o_lat + (size_t)(t.r0 / p.VD) * p.KL; break;
-    case OP_MO: src = p.mla_o; break;
+    case OP_MO: case OP_MOS: src = p.mla_o; break;
     default: src = p.x; vstride = p.d; gain = p.final_norm; break;
   }
   if (src) src += gg.k0;        // normalised inputs are single-part (k0 = 0)
@@ -2124,6 +2128,10 @@ __device__ void index_pick(const Params& p, const Task& t, float* scratch, int w
   const uint32_t n = min(__ldcg(meta + IM_NCAND), (uint32_t)p.cap);
   uint32_t* h = reinterpret_cast<uint32_t*>(scratch);  // [256]
   uint32_t* sh = h + 256;                               // digit, still to take
+  // the candidates' keys in shared memory when they fit (the usual case: the threshold
+  // bin holds a small share of the positions), else read from L2 on every pass
+  unsigned long long* ks = reinterpret_cast<unsigned long long*>(scratch + 512);
+  const bool in_smem = n <= kPickSmemKeys;
   const int pb = 32 - __clz(max(p.cap - 1, 1));
   const unsigned long long pmask = (1ull << pb) - 1ull;
   auto keyof = [&](unsigned long long c) {
@@ -2131,6 +2139,9 @@ __device__ void index_pick(const Params& p, const Task& t, float* scratch, int w
     const unsigned long long pos = 0xffffffffull - (c & 0xffffffffull);
     return (k20 << pb) | (pmask - pos);
   };
+  auto key_at = [&](uint32_t i) { return in_smem ? ks[i] : keyof(__ldcg(cand + i)); };
+  if (in_smem)
+    for (uint32_t i = ctid; i < n; i += kConsumerThreads) ks[i] = keyof(__ldcg(cand + i));
   const int bits = 20 + pb;
   unsigned long long prefix = 0;
   uint32_t rem = __ldcg(meta + IM_NEED);
@@ -2138,7 +2149,7 @@ __device__ void index_pick(const Params& p, const Task& t, float* scratch, int w
     for (int i = ctid; i < 256; i += kConsumerThreads) h[i] = 0u;
     consumer_sync(kConsumerThreads);
     for (uint32_t i = ctid; i < n; i += kConsumerThreads) {
-      const unsigned long long k = keyof(__ldcg(cand + i));
+      const unsigned long long k = key_at(i);
       if ((k >> (sft + 8)) == prefix) atomicAdd(h + ((k >> sft) & 255u), 1u);
     }
     consumer_sync(kConsumerThreads);
@@ -2178,9 +2189,9 @@ __device__ void index_pick(const Params& p, const Task& t, float* scratch, int w
     bool take = false;
     int pos = 0;
     if (i < n) {
-      const unsigned long long c = __ldcg(cand + i);
-      take = keyof(c) >= prefix;
-      pos = (int)(0xffffffffu - (uint32_t)(c & 0xffffffffull));
+      const unsigned long long k = key_at(i);
+      take = k >= prefix;
+      pos = (int)(pmask - (k & pmask));
     }
     if (take && pos == p.pos) {
       meta[IM_HASPOS] = 1u;
@@ -2258,14 +2269,28 @@ __device__ void isel_task(const Params& p, const Task& t, float* ub, int* tk, in
 // The W_uv task of head h stages o_lat_h, merging the head's KV splits on the way:
 // o_lat_h = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s (splits that saw no position
 // have m_s = -inf and weigh 0).  128 heads merge on 128 SMs at once.
-__device__ void mla_combine_input(const Params& p, const Task& t, float* ub, float* scratch,
+__device__ __noinline__ void mla_combine_input(const Params& p, const Task& t, float* ub, float* scratch,
                                   int ctid) {
   const int h = t.r0 / p.VD, KL = p.KL, S = p.nsplit;
   const size_t pstride = (size_t)mla_pstride(KL);
   const float* base = p.part + (size_t)h * S * pstride;
-  float* ms = scratch;       // [S] split weights 2^(m_s - M)
-  float* ls = scratch + S;  // [1] 1 / sum_s w_s l_s
-  for (int s2 = ctid; s2 < S; s2 += kConsumerThreads) ms[s2] = __ldcg(base + s2 * pstride + KL);
+  float* ms = scratch;       // [S] split maxima, then weights 2^(m_s - M)
+  float* lsum = scratch + S; // [S] split sums
+  float* ls = lsum + S;      // [1] 1 / sum_s w_s l_s
+  // Every load is issued before the weights are known: (m, l) of each split, and this
+  // thread's two columns of the first kPre splits' partials (the loads of one thread are
+  // independent, so they overlap: one L2 round trip instead of one per phase).
+  constexpr int kPre = 16;
+  const int c = 2 * ctid;
+  float2 pv[kPre];
+#pragma unroll
+  for (int s2 = 0; s2 < kPre; ++s2)
+    if (s2 < S && c < KL)
+      pv[s2] = __ldcg(reinterpret_cast<const float2*>(base + s2 * pstride + c));
+  for (int s2 = ctid; s2 < S; s2 += kConsumerThreads) {
+    ms[s2] = __ldcg(base + s2 * pstride + KL);
+    lsum[s2] = __ldcg(base + s2 * pstride + KL + 1);
+  }
   consumer_sync(kConsumerThreads);
   if (ctid < 32) {
     float M = -INFINITY;
@@ -2275,7 +2300,7 @@ __device__ void mla_combine_input(const Params& p, const Task& t, float* ub, flo
     float L = 0.f;
     for (int s2 = ctid; s2 < S; s2 += 32) {
       const float w = ms[s2] == -INFINITY ? 0.f : exp2f(ms[s2] - M);
-      L = fmaf(w, __ldcg(base + s2 * pstride + KL + 1), L);
+      L = fmaf(w, lsum[s2], L);
       ms[s2] = w;
     }
 #pragma unroll
@@ -2286,19 +2311,28 @@ __device__ void mla_combine_input(const Params& p, const Task& t, float* ub, flo
   const float inv = ls[0];
   float* xlo = ub;
   float* xhi = ub + KL / 2;
-  for (int j = ctid; j < KL / 8; j += kConsumerThreads) {
-    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int s2 = 0; s2 < S; ++s2) {
-      const float w = ms[s2];
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(base + s2 * pstride + 8 * j));
-      const float4 b = __ldcg(reinterpret_cast<const float4*>(base + s2 * pstride + 8 * j + 4));
-      v[0] = fmaf(w, a.x, v[0]); v[1] = fmaf(w, a.y, v[1]); v[2] = fmaf(w, a.z, v[2]);
-      v[3] = fmaf(w, a.w, v[3]); v[4] = fmaf(w, b.x, v[4]); v[5] = fmaf(w, b.y, v[5]);
-      v[6] = fmaf(w, b.z, v[6]); v[7] = fmaf(w, b.w, v[7]);
+  // columns c, c + 1 of the input planes (plane lo holds x[8j .. 8j + 3], hi x[8j + 4 ..])
+  auto put = [&](int col, float v) {
+    const int j = col >> 3, w = col & 7;
+    (w < 4 ? xlo : xhi)[4 * j + (w & 3)] = v * inv;
+  };
+  for (int cc = c; cc < KL; cc += 2 * kConsumerThreads) {
+    float v0 = 0.f, v1 = 0.f;
+    if (cc == c) {
+#pragma unroll
+      for (int s2 = 0; s2 < kPre; ++s2)
+        if (s2 < S) {
+          v0 = fmaf(ms[s2], pv[s2].x, v0);
+          v1 = fmaf(ms[s2], pv[s2].y, v1);
+        }
     }
-    reinterpret_cast<float4*>(xlo)[j] = make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
-    reinterpret_cast<float4*>(xhi)[j] = make_float4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
+    for (int s2 = cc == c ? kPre : 0; s2 < S; ++s2) {
+      const float2 a = __ldcg(reinterpret_cast<const float2*>(base + s2 * pstride + cc));
+      v0 = fmaf(ms[s2], a.x, v0);
+      v1 = fmaf(ms[s2], a.y, v1);
+    }
+    put(cc, v0);
+    put(cc + 1, v1);
   }
   consumer_sync(kConsumerThreads);
 }
@@ -2339,7 +2373,8 @@ __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const 
     case OP_UV: p.mla_o[n] = v; break;
     case OP_O: p.h1[(size_t)tok * p.d + n] = resid[n - t.r0] + v; break;
     case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
-    case OP_MDOWN: p.mpart[(size_t)g.part * p.d + n] = v; break;
+    case OP_MDOWN:
+    case OP_MOS: p.mpart[(size_t)g.part * p.d + n] = v; break;
     case OP_DOWN:
     case OP_MO: {
       const float y = resid[n - t.r0] + v;
@@ -2395,6 +2430,20 @@ __device__ void route_topk(const Params& p, int layer, float* sc, int warp, int 
 
 // The last slot of a MoE-down row block to finish: x = h1 + sum of the slots' partial rows
 // in slot order (deterministic), then the block is published.
+// The last K-slice of an MLA output row block to finish: x = x + sum_j partial_j (slice
+// order, deterministic), then the layer's output counter.
+__device__ void mo_slices_combine(const Params& p, const Task& t, int np, int ctid) {
+  for (int n = t.r0 + ctid; n < t.r1; n += kConsumerThreads) {
+    float y = resid_in(p, t.layer, n);
+    for (int j = 0; j < np; ++j) y += __ldcg(p.mpart + (size_t)j * p.d + n);
+    p.x[n] = y;
+    if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
+    if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
+  }
+  consumer_sync(kConsumerThreads);
+  if (ctid == 0) publish_add(p.counters + t.out, 1u);
+}
+
 __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
   const int np = p.nshared + p.topk;
   for (int n = t.r0 + ctid; n < t.r1; n += kConsumerThreads) {
@@ -2517,17 +2566,16 @@ __device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, c
 // columns 0-3 the terms of half 0, 4-7 those of half 1.  Of the 16 x 8 products a lane keeps
 // its row g's pair of terms of its half (lanes t4 < 2: half 0, t4 >= 2: half 1), weighed by
 // 16^-tau, the chunk's 2^-sg and the weight block scale (32 columns never straddle a
-// 128-column block).  All 8 warps share each stage, warp w taking the chunks w, w + 8, ...;
-// the lanes of a row and then the warps are summed (shuffles, shared memory), and one thread
-// per row finishes it.
+// 128-column block).  As for bf16 rows, stage gs + i belongs to warp (gs + i) % 8, which
+// walks all its chunks (four at a time, every load issued first), sums a row's 4 lanes with
+// two shuffles and emits the rows: no barrier per stage, several stages in flight at once.
 __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint32_t gs, int ns,
                          uint8_t* ring, uint64_t* full, uint64_t* empty, const uint32_t* tags,
                          float* ub, const float* resid, float rn, float wsel, int uoff, int warp,
-                         int lane, int ctid, bool& ab, Best& best) {
+                         int lane, bool& ab, Best& best) {
   const int Lh = fp8_half_len(g.Kp), P = fp8_row_pitch(g.Kp), nch = Lh / 32;
   const uint8_t* frag = reinterpret_cast<const uint8_t*>(ub);
   const float* csc = ub + 2 * Lh;            // 2^-sg per 32 columns of the span
-  float* red = ub + fp8_frag_floats(g.Kp);   // [2][kConsumerWarps][8]
   const Fp8Scales fs = fp8_scales(p, t, g);
   const bool two = g.nseg == 2;
   const int gq = lane >> 2, t4 = lane & 3, half = t4 >> 1;
@@ -2536,9 +2584,13 @@ __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint
   const uint8_t* bp = frag + (gq >> 2) * 4 * Lh + (gq & 3) * 32 + t4 * 8;
   const int mat = lane >> 3, trow = lane & 7;  // ldmatrix: this lane's matrix and row
   const uint32_t NS = (uint32_t)p.ring_stages;
-  for (int i = 0; i < ns; ++i) {
+  const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
+  for (int i = first; i < ns; i += kConsumerWarps) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
-    const bool landed = stage_wait(p, full, tags, sidx);
+    if (!stage_wait(p, full, tags, sidx)) {
+      ab = true;
+      return;
+    }
     const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
     // tile row trow's stage row (gate / up: rows 0-3 gate, 4-7 up), clamped to a loaded row
     const int sr = two ? ((trow >> 2) ? g.rps : 0) + min(trow & 3, nr - 1) : min(trow, nr - 1);
@@ -2547,69 +2599,54 @@ __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint
     // the weight row of this lane's output row gq, for its block scales
     const float* srow = two ? fp8_scale_row(fs, gq >> 2, n0 + min(gq & 3, nr - 1))
                             : fp8_scale_row(fs, 0, n0 + min(gq, nr - 1));
+    constexpr int kU = 4;
+    float accu[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) accu[u] = 0.f;
+    for (int cb = 0; cb < nch; cb += kU) {
+      uint32_t a[kU][4];
+      uint2 b[kU];
+      float sc[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int cc = min(cb + u, nch - 1);  // clamped: in-range reads
+        ldsm_x4(arow + (uint32_t)(cc * 32), a[u][0], a[u][1], a[u][2], a[u][3]);
+        b[u] = *reinterpret_cast<const uint2*>(bp + cc * 128);
+        const int col = half * Lh + cc * 32;
+        sc[u] = __ldg(srow + ((g.k0 + col) >> 7)) * csc[col >> 5];
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int cc = cb + u;
+        // columns past Kp are stale shared memory: zero them (the input is zero there); a
+        // chunk past the last one (clamped above) counts nothing
+        const int c0 = cc * 32 + 4 * t4, c1 = Lh + c0;
+        const bool live = cc < nch;
+        if (!live || c0 >= g.Kp) a[u][0] = 0u;
+        if (!live || c0 + 16 >= g.Kp) a[u][2] = 0u;
+        if (!live || c1 >= g.Kp) a[u][1] = 0u;
+        if (!live || c1 + 16 >= g.Kp) a[u][3] = 0u;
+        float d[4];
+        mma_e4m3(d, a[u], b[u].x, b[u].y);
+        const float v = half ? fmaf(d[3], wb, d[2] * wa) : fmaf(d[1], wb, d[0] * wa);
+        accu[u] = fmaf(v, sc[u], accu[u]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_n(&empty[slot], kConsumerWarps);
     float acc = 0.f;
-    if (landed) {
-      // kU chunks at a time (chunks w, w + 8, ...), every load issued before the products,
-      // so that a warp keeps several ldmatrix / scale loads and mma in flight
-      constexpr int kU = 4;
-      float accu[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) accu[u] = 0.f;
-      for (int cb = warp; cb < nch; cb += kU * kConsumerWarps) {
-        uint32_t a[kU][4];
-        uint2 b[kU];
-        float sc[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int cc = min(cb + u * kConsumerWarps, nch - 1);  // clamped: in-range reads
-          ldsm_x4(arow + (uint32_t)(cc * 32), a[u][0], a[u][1], a[u][2], a[u][3]);
-          b[u] = *reinterpret_cast<const uint2*>(bp + cc * 128);
-          const int col = half * Lh + cc * 32;
-          sc[u] = __ldg(srow + ((g.k0 + col) >> 7)) * csc[col >> 5];
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int cc = cb + u * kConsumerWarps;
-          // columns past Kp are stale shared memory: zero them (the input is zero there); a
-          // chunk past the last one (clamped above) counts nothing
-          const int c0 = cc * 32 + 4 * t4, c1 = Lh + c0;
-          const bool live = cc < nch;
-          if (!live || c0 >= g.Kp) a[u][0] = 0u;
-          if (!live || c0 + 16 >= g.Kp) a[u][2] = 0u;
-          if (!live || c1 >= g.Kp) a[u][1] = 0u;
-          if (!live || c1 + 16 >= g.Kp) a[u][3] = 0u;
-          float d[4];
-          mma_e4m3(d, a[u], b[u].x, b[u].y);
-          const float v = half ? fmaf(d[3], wb, d[2] * wa) : fmaf(d[1], wb, d[0] * wa);
-          accu[u] = fmaf(v, sc[u], accu[u]);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kU; ++u) acc += accu[u];
-      __syncwarp();
-      if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
-    }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    for (int u = 0; u < kU; ++u) acc += accu[u];
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);  // the row's two halves and term pairs
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    float* rb = red + (i & 1) * kConsumerWarps * 8;
-    if (t4 == 0) rb[warp * 8 + gq] = acc;
-    if (consumer_sync_or(!landed, kConsumerThreads)) {
-      ab = true;
-      return;
-    }
-    if (ctid < nr && (!two || ctid < 4)) {
-      float v = 0.f, u = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        v += rb[w * 8 + ctid];
-        if (two) u += rb[w * 8 + 4 + ctid];
+    if (two) {  // lane (j, 0) holds gate row j, lane (4 + j, 0) up row j
+      const float u = __shfl_down_sync(0xffffffffu, acc, 16);
+      if (t4 == 0 && gq < 4 && gq < nr) {
+        const float aa = acc * rn, bb = u * rn;
+        p.u[uoff + n0 + gq] = wsel * (aa / (1.f + expf(-aa)) * bb);
       }
-      if (two) {  // gate row ctid (v), up row ctid (u)
-        const float aa = v * rn, bb = u * rn;
-        p.u[uoff + n0 + ctid] = wsel * (aa / (1.f + expf(-aa)) * bb);
-      } else {
-        gemv_emit(p, t, g, n0 + ctid, v, rn, resid, best);
-      }
+    } else if (t4 == 0 && gq < nr) {
+      gemv_emit(p, t, g, n0 + gq, acc, rn, resid, best);
     }
   }
 }
@@ -2715,11 +2752,11 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
                            ub + p.ub_floats - kTileRedFloats, resid, rnt, wsel, uoff, best, warp,
                            lane, ctid, ab);
       }
-      const bool coop = F8 && g.esz == 1;  // E4M3 stages: every warp takes part in each
+      const bool coop = F8 && g.esz == 1;  // E4M3 stages: the tensor-core tile
       if constexpr (F8) {
         if (coop)
           fp8_task(p, t, g, gs, ns, ring, full, empty, tags, ub, resid, rn, wsel, uoff, warp,
-                   lane, ctid, ab, best[0]);
+                   lane, ab, best[0]);
       }
       // stage gs + i belongs to warp (gs + i) % 8; each warp takes its stages in order
       const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
@@ -2848,6 +2885,14 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         consumer_sync(kConsumerThreads);
         if (flags[1]) route_topk(p, t.layer, ub + p.xs_floats, warp, lane, ctid);
+      } else if (t.op == OP_MOS) {  // the block's last slice sums the partial rows
+        const int np = (t.aux >> 16) & 0xff;
+        if (ctid == 0) {
+          const uint32_t old = ticket_add(p.down_tickets + ((t.aux >> 8) & 0xff), 1u);
+          flags[1] = ((old + 1u) % (uint32_t)np) == 0u;
+        }
+        consumer_sync(kConsumerThreads);
+        if (flags[1]) mo_slices_combine(p, t, np, ctid);
       } else if (t.op == OP_MDOWN) {  // the block's last slot sums the partial rows
         if (ctid == 0) {
           const uint32_t old = ticket_add(p.down_tickets + (t.aux >> 8), 1u);

@@ -169,6 +169,27 @@ struct Builder {
     }
   }
 
+  // MLA output projection in K-slices on different SMs: nb row blocks x np slices, each
+  // placed on the SM with the least streamed bytes so far; aux = slice | block << 8 |
+  // np << 16.  Returns nb (one bump per block, by its last slice).
+  int mo_slices(int layer, int d, int K, int np, int nb, int dep, uint32_t dep_count, int out) {
+    const std::vector<int> sms = spread(np * nb);
+    const int len = gemv_part_len(K, np, 8);
+    for (int bl = 0; bl < nb; ++bl) {
+      const int r0 = (int)((int64_t)d * bl / nb), r1 = (int)((int64_t)d * (bl + 1) / nb);
+      for (int j = 0; j < np; ++j) {
+        const int best = sms[bl * np + j];
+        Task t = make(T_GEMV, OP_MOS, layer, dep, dep_count, out);
+        t.r0 = r0;
+        t.r1 = r1;
+        t.aux = j | (bl << 8) | (np << 16);
+        q[best].push_back(t);
+        cum[best] += (int64_t)(r1 - r0) * std::min(len, K - j * len) * 2;
+      }
+    }
+    return nb;
+  }
+
   // Set aux = count on every task of `op` created since task id `first`.
   void set_count(int first, uint8_t op, int count) {
     for (auto& qq : q)
@@ -372,6 +393,15 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   s.u_floats = moe ? (s.nshared + s.topk) * s.Fe : s.F;
   // MoE down row blocks: enough (slot, block) tasks to cover the SMs once
   if (moe) s.down_blocks = std::max(1, std::min(s.d / 8, nsm / (s.nshared + s.topk)));
+  // MLA output projection: its K-parts as slices on different SMs, row blocks to cover the
+  // SMs once (up to 255 blocks and slices: the task's aux fields)
+  if (mla) {
+    const int np = gemv_nparts(s.Hq * s.VD, s.kpart_max);
+    if (np > 1 && np <= 255) {
+      s.mo_slices = np;
+      s.down_blocks = std::max(1, std::min({s.d / 8, nsm / np, 255}));
+    }
+  }
   const int G = s.Hq / s.Hkv;
 
   // Inputs longer than kMaxKPart are staged in K-parts; ops that normalise their input
@@ -404,7 +434,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max),
                                                gemv_part_align(s.tiles, o.esz == 1));
     // E4M3 rows: the tensor-core operand of the input covers the 4 row segments
-    xs = std::max(xs, o.esz == 1 ? fp8_frag_floats(kp) + kFp8RedFloats : kp);
+    xs = std::max(xs, o.esz == 1 ? fp8_frag_floats(kp) : kp);
     need = std::max(need, s.tiles ? kTileRows * kTilePitch
                                   : o.esz == 1 ? o.nseg * fp8_row_pitch(kp) : o.nseg * kp * o.esz);
   }
@@ -452,8 +482,9 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     // index scoring: the score histogram, the bf16 query tile [H_I][D_I], the head weights,
     // the new position's per-warp sums
     if (s.KI)
-      s.attn_floats = std::max(s.attn_floats, kIndexBins + kIndexMaxHeads * 128 / 2 +
-                                                  kIndexMaxHeads + 64);
+      s.attn_floats = std::max({s.attn_floats, kIndexBins + kIndexMaxHeads * 128 / 2 +
+                                                   kIndexMaxHeads + 64,
+                                512 + 2 * kPickSmemKeys});  // the pick's keys
   }
   const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + (s.tiles ? kTileRedFloats : 0),
                                      s.attn_floats) + 7) / 8 * 8;
@@ -504,7 +535,12 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     else b.mla_attention(l, groups, S, lat_task, cuk, (uint32_t)n3, ca);
     const int n5 = b.per_unit(OP_UV, l, H, s.VD, (int64_t)s.VD * s.KL * 2, ca,
                               (uint32_t)(groups * S), cuv);
-    const int n6 = b.gemv(OP_MO, l, s.d, H * s.VD, 1, cuv, (uint32_t)n5, co, kMaxResidRows);
+    // W_o (K = H v_dim) in K-slices: the slices of a row block run on different SMs and the
+    // last to finish adds them to the residual (one K-part per SM instead of two in a row)
+    const int n6 = s.mo_slices > 1
+                       ? b.mo_slices(l, s.d, H * s.VD, s.mo_slices, s.down_blocks, cuv,
+                                     (uint32_t)n5, co)
+                       : b.gemv(OP_MO, l, s.d, H * s.VD, 1, cuv, (uint32_t)n5, co, kMaxResidRows);
     prev_down = co;
     prev_down_count = (uint32_t)n6;
   }

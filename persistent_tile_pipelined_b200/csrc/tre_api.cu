@@ -356,8 +356,9 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_ridx = cv.take<int32_t>(moe ? (size_t)s.L * s.topk : 1);
   size_t o_rw = cv.take<float>(moe ? (size_t)s.L * s.topk : 1);
   size_t o_rtick = cv.take<uint32_t>(1);
-  size_t o_mpart = cv.take<float>(moe ? (size_t)(s.nshared + s.topk) * s.d : 1);
-  size_t o_dtick = cv.take<uint32_t>(moe ? s.down_blocks : 1);
+  size_t o_mpart = cv.take<float>(moe ? (size_t)(s.nshared + s.topk) * s.d
+                                       : s.mo_slices ? (size_t)s.mo_slices * s.d : 1);
+  size_t o_dtick = cv.take<uint32_t>(s.down_blocks ? s.down_blocks : 1);
   size_t o_part = cv.take<float>(M * s.Hq * s.kv_splits * (mla ? mla_pstride(s.KL) : gqa_pstride(s.D)));
   size_t o_logits = cv.take<float>(s.V > 0 ? M * s.V : 1);
   size_t o_tok = cv.take<int32_t>(kMaxTokens);
@@ -836,7 +837,7 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
                      s));
   CK(cudaMemsetAsync(p.lm_ticket, 0, 4, s));
   CK(cudaMemsetAsync(p.router_ticket, 0, 4, s));
-  if (e->shape.kind == TRE_LAYER_MOE)
+  if (e->shape.down_blocks)
     CK(cudaMemsetAsync(p.down_tickets, 0, (size_t)e->shape.down_blocks * 4, s));
   CK(cudaMemsetAsync(p.argmax_slot, 0, 8 * kMaxTokens, s));
   CK(cudaMemsetAsync(p.err, 0, 8, s));  // error word + abort flag

@@ -65,9 +65,8 @@ TRE_HD inline int fp8_half_len(int Kp) { return (Kp + 63) / 64 * 32; }
 TRE_HD inline int fp8_span(int Kp) { return 2 * fp8_half_len(Kp); }
 TRE_HD inline int fp8_row_pitch(int Kp) { return fp8_span(Kp) + 16; }
 // The input operand of an E4M3 GEMV: 4 E4M3 terms per input (4 bytes) in fragment order,
-// then one scale per 32 columns: its size in floats (the cross-warp sums follow it)
+// then one scale per 32 columns: its size in floats
 TRE_HD inline int fp8_frag_floats(int Kp) { return fp8_span(Kp) + fp8_span(Kp) / 32; }
-constexpr int kFp8RedFloats = 2 * kConsumerWarps * 8;
 TRE_HD inline int fp8_rows_per_stage(int Kp, int nseg, int stage_bytes) {
   const int r = stage_bytes / (nseg * fp8_row_pitch(Kp));
   return r < 1 ? 1 : r;
@@ -97,7 +96,10 @@ enum GemvOp : uint8_t {
                   //                               also RoPE(q_pe); head 0 appends the latent
   OP_UV = 12,     // in: o_lat of one head      -> o = Wuv_h o_lat
   OP_MO = 13,     // in: o                      -> x = x + Wo o
-  OP_COUNT = 14
+  OP_MOS = 14,    // in: o, K-slice j           -> partial rows of slice j of a row block
+                  //                               (aux = j | block << 8 | slices << 16); the
+                  //                               block's last slice sums x = x + sum_j partial_j
+  OP_COUNT = 15
 };
 
 // MLA counters reuse the per-layer slots: QKV = down-projections, ATTN, O = output
@@ -112,6 +114,7 @@ constexpr int kIndexRows = 128;
 constexpr int kIndexBinBits = 12;
 constexpr int kIndexBins = 1 << kIndexBinBits;
 constexpr int kIndexMaxHeads = 64;
+constexpr int kPickSmemKeys = 3840;  // threshold-bin candidates the pick keeps in shared memory
 TRE_HD inline int sparse_lat_pitch(int C) { return C * 2 + 16; }  // bytes per gathered row
 // Per-layer selection state (uint32 words): the threshold bin, how many positions lie in
 // bins above it, how many of the threshold bin are still to take, that bin's count, the
@@ -170,7 +173,9 @@ struct PlanShape {
   int tiles;           // multi-token plan: GEMV stages are 16-row tensor-core tiles
   int wfp8;            // GQA projections are E4M3 with 128 x 128 block scales
   int u_floats;        // the SwiGLU activation buffer (MoE: shared then routed slices)
-  int down_blocks;     // MoE down: row blocks (each summed by its last slot to finish)
+  int down_blocks;     // MoE down / MLA output slices: row blocks (each summed by its last
+                       // slot or slice to finish)
+  int mo_slices;       // MLA output projection: K-slices on different SMs (0: one K-part)
   int nsm;
   int stage_bytes, ring_stages;
   int kv_splits, pos_per_stage;

@@ -15,7 +15,7 @@ import numpy as np
 
 OP_NAMES = {0: "qkv", 1: "o_proj", 2: "gate_up", 3: "down", 4: "lm_head", 5: "router",
             6: "shared_gate_up", 7: "routed_gate_up", 8: "moe_down", 9: "mla_down",
-            10: "q_up", 11: "uk", 12: "uv", 13: "mla_o"}
+            10: "q_up", 11: "uk", 12: "uv", 13: "mla_o", 14: "mla_o"}
 
 
 def task_table(tasks: np.ndarray) -> dict:

@@ -19,7 +19,7 @@ from persistent_tile_pipelined_b200 import tre  # noqa: E402
 
 T_GEMV, T_ATTN = 0, 1
 OP_QKV, OP_O, OP_GU, OP_DOWN, OP_LM, OP_ROUTER, OP_SGU, OP_RGU, OP_MDOWN = range(9)
-OP_MDQKV, OP_UQ, OP_UK, OP_UV, OP_MO = range(9, 14)
+OP_MDQKV, OP_UQ, OP_UK, OP_UV, OP_MO, OP_MOS = range(9, 15)
 T_MLA_ATTN, T_INDEX, T_ISEL = 2, 3, 4
 C_QKV, C_ATTN, C_O, C_GU, C_DOWN, C_ROUTE = range(6)
 C_MLA_UK, C_MLA_IDX, C_MLA_SEL = 4, 6, 7
@@ -157,17 +157,24 @@ def check_plan(wl, nsm, **over):
             # the MoE down counter is bumped once per row block (by its last slot)
             blocks = {int(T["aux"][j]) >> 8 for j in producers}
             assert T["dep_count"][i] == len(blocks)
+        elif producers and T["op"][producers[0]] == OP_MOS:
+            # the MLA output counter: once per row block (by its last K-slice)
+            blocks = {(int(T["aux"][j]) >> 8) & 0xFF for j in producers}
+            assert T["dep_count"][i] == len(blocks)
         else:
             assert T["dep_count"][i] == len(producers), (i, dep, kind)
     # every GEMV op's output rows are partitioned exactly once per layer
     rows_of = rows_of_ops(wl)
     whole = np.isin(T["op"], WHOLE_ROW_OPS)
     mdown = T["op"] == OP_MDOWN
+    mos = T["op"] == OP_MOS
     part = np.where(whole, 0, T["aux"] & 0xFF)
-    nparts = np.where(whole, 1, np.where(mdown, 1, T["aux"] >> 8))
+    nparts = np.where(whole, 1, np.where(mdown, 1, np.where(mos, (T["aux"] >> 16) & 0xFF,
+                                                            T["aux"] >> 8)))
     gemv = T["type"] == T_GEMV
-    # only the last K-part of a row range publishes (MoE down: every slot task may)
-    kp = gemv & ~mdown
+    # only the last K-part of a row range publishes (MoE down, MLA output slices: every
+    # slot task may; the last to arrive does)
+    kp = gemv & ~mdown & ~mos
     assert ((T["out"][kp] >= 0) == (part[kp] == nparts[kp] - 1)).all()
     if wl.kind == "moe":
         # every (slot, row block) pair exactly once; blocks partition the rows
@@ -193,8 +200,19 @@ def check_plan(wl, nsm, **over):
             ro = gemv & (T["op"] == OP_ROUTER) & (T["layer"] == l)
             assert (T["aux"][ro] == ro.sum()).all()
     for l in range(wl.n_layers):
+        sl = np.flatnonzero(gemv & mos & (T["layer"] == l))
+        if len(sl):  # every (slice, block) pair once; blocks partition the rows; 2+ slices
+            pairs = Counter((int(T["aux"][i]) & 0xFF, (int(T["aux"][i]) >> 8) & 0xFF) for i in sl)
+            ns_ = int(nparts[sl[0]])
+            nb = len({b for _, b in pairs})
+            assert ns_ >= 2 and set(pairs) == {(j, b) for j in range(ns_) for b in range(nb)}
+            cover = np.zeros(wl.hidden, dtype=np.int64)
+            for i in sl:
+                if int(T["aux"][i]) & 0xFF == 0:
+                    cover[T["r0"][i]:T["r1"][i]] += 1
+            assert (cover == 1).all()
         for op, N in rows_of.items():
-            if op == OP_MDOWN:
+            if op == OP_MDOWN or (op == OP_MO and len(sl)):
                 continue
             if op == OP_LM and l != wl.n_layers - 1:
                 continue

@@ -98,7 +98,9 @@ def test_mla_layers(over, steps):
     dict(num_sms=5),
     dict(kv_splits=1),
     dict(num_sms=3, ring_stages=2),
-], ids=["sms5", "split1", "sms3-ring2"])
+    dict(gemv_kpart_max=512),             # W_o in 2 K-slices on different SMs
+    dict(gemv_kpart_max=512, num_sms=3),  # ... 2 slices x 1 row block
+], ids=["sms5", "split1", "sms3-ring2", "wo-slices", "wo-slices-sms3"])
 def test_mla_launch_shapes(cfg):
     run_mla(SMALL, steps=2, **cfg)
 

@@ -177,7 +177,8 @@ def test_sparse_ties_go_to_the_lower_position():
 
 
 @pytest.mark.parametrize("cfg", [dict(num_sms=5), dict(num_sms=3, ring_stages=2),
-                                 dict(kv_splits=1)], ids=["sms5", "sms3-ring2", "split1"])
+                                 dict(kv_splits=1), dict(gemv_kpart_max=512)],
+                         ids=["sms5", "sms3-ring2", "split1", "wo-slices"])
 def test_sparse_launch_shapes(cfg):
     run_sparse(SMALL, steps=2, **cfg)
 
