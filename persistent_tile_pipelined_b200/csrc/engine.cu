@@ -1525,6 +1525,7 @@ __device__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint3
   const float* qh = p.qkv + (size_t)h * (p.NP + p.R);
   for (int i = ctid; i < p.NP; i += kConsumerThreads) qn[i] = __ldcg(qh + i);
   consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
   const uint32_t NS = (uint32_t)p.ring_stages;
   const int nblk = KL / 256 + ((KL % 256) ? 1 : 0);   // 256-column blocks (lane: 8 columns each)
   float acc[3][8];
@@ -1571,6 +1572,7 @@ __device__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint3
       for (int k = 0; k < 8; ++k) red[warp * KL + c0 + k] = acc[b][k];
   }
   consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
   float* qf = p.qf + (size_t)h * C;
   for (int c = ctid; c < KL; c += kConsumerThreads) {
     float v = 0.f;
@@ -1586,6 +1588,7 @@ __device__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint3
     qf[KL + i] = x0 * cs - x1 * sn;
     qf[KL + i + R2] = x0 * sn + x1 * cs;
   }
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
   if (h == 0) {  // this token's latent row
     const float* kv = p.cqkv + p.QL;
     const uint16_t* gain = p.layers[t.layer].w[TRE_W_KV_NORM];
@@ -1887,9 +1890,6 @@ __device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int n
 // layer's global histogram.  The last split also scores the new position from its
 // on-chip key (rounded to bf16 as the cache holds it); the split that arrives last picks
 // the threshold bin (index_threshold).
-__device__ void index_threshold(const Params& p, const Task& t, float* scratch, int warp,
-                                int lane, int ctid);
-
 // Byte offset of 16-byte chunk c of row r of the [H_I][D_I] bf16 query tile (rows of
 // 2 D_I bytes, chunks XOR-swizzled by r & 7 so that ldmatrix reads 8 rows conflict-free).
 __device__ __forceinline__ uint32_t qtile_off(int r, int c, int DI) {
@@ -1939,9 +1939,12 @@ __device__ void index_task(const Params& p, const Task& t, uint32_t gs, int ns, 
   const int m = lane >> 3;
   const int rb = warp * 16 + (m >> 1) * 8 + (lane & 7);   // this lane's key row (ldmatrix)
   const int ra = (m & 1) * 8 + (lane & 7);                // this lane's query row in an m-tile
+  long long waited = 0;  // trace: ns warp 0 spent waiting for stages to land
   for (int i = 0; i < ns; ++i) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
+    const long long w0 = p.trace ? (long long)globaltimer_ns() : 0;
     const bool landed = stage_wait(p, full, tags, sidx);
+    if (p.trace) waited += (long long)globaltimer_ns() - w0;
     const uint32_t tb = smem_u32(ring + (size_t)slot * p.stage_bytes);
     float c[4][2][4];
 #pragma unroll
@@ -2010,14 +2013,26 @@ __device__ void index_task(const Params& p, const Task& t, uint32_t gs, int ns, 
     ab = true;
     return;
   }
-  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
-  if (t.r1 == t.aux - 1) {  // the new position, from its key on chip
+  if (ctid == 0 && p.trace) {
+    p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
+    p.trace[(size_t)t.id * kTraceCols + 7] = waited;
+  }
+  if (t.r1 == t.aux - 1) {  // the new position, from its key on chip (rounded to bf16)
+    // warp w takes heads w, w + 8, ...; lane l columns 4 l .. 4 l + 3 (D_I <= 128), the
+    // queries from the bf16 tile the stages used
     float part = 0.f;
+    const int k0 = 4 * lane;
+    float kv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      kv[k] = k0 + k < DI ? __bfloat162float(__float2bfloat16_rn(__ldcg(kin + k0 + k))) : 0.f;
     for (int h = warp; h < HI; h += kConsumerWarps) {
       float d = 0.f;
-      for (int k = lane; k < DI; k += 32) {
-        const float q = __bfloat162float(__float2bfloat16_rn(__ldcg(qi + (size_t)h * DI + k)));
-        d = fmaf(q, __bfloat162float(__float2bfloat16_rn(__ldcg(kin + k))), d);
+      if (k0 < DI) {
+        const __nv_bfloat16* qr =
+            reinterpret_cast<const __nv_bfloat16*>(qt + qtile_off(h, k0 >> 3, DI)) + (k0 & 7);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) d = fmaf(__bfloat162float(qr[k]), kv[k], d);
       }
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
@@ -2034,30 +2049,33 @@ __device__ void index_task(const Params& p, const Task& t, uint32_t gs, int ns, 
     }
   }
   consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
   uint32_t* gh = p.ix_hist + (size_t)t.layer * kIndexBins;
   for (int b = ctid; b < kIndexBins; b += kConsumerThreads) {
     const uint32_t v = hist[b];
     if (v) atomicAdd(gh + b, v);
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) *tk = ((ticket_add(index_meta(p, t.layer) + IM_TICK_A, 1u) + 1u) % (uint32_t)t.aux) == 0u;
-  consumer_sync(kConsumerThreads);
-  if (*tk) index_threshold(p, t, ub, warp, lane, ctid);
+  if (ctid == 0) {
+    if (t.r1 == 0) {  // this step's selection starts from no chosen positions
+      uint32_t* meta = index_meta(p, t.layer);
+      meta[IM_NSEL] = 0u;
+      meta[IM_NCAND] = 0u;
+      meta[IM_HASPOS] = 0u;
+    }
+    publish_add(p.counters + t.out, 1u);  // after the CTA's histogram adds (barrier above)
+  }
 }
 
-// Run by the index scoring task that arrives last: the bin of the K-th largest score.
-// Thread j holds bins kIndexBins - 1 - (16 j + k), k < 16 (descending); a scan over the
-// threads finds the bin b where the count above it is below K and the count from it on
-// reaches K.  The layer's state receives b, the count above it, how many of b are still to
-// take and b's count; the histogram is cleared and the chosen count reset for the next
-// step, then the layer's index counter is published.
-__device__ void index_threshold(const Params& p, const Task& t, float* scratch, int warp,
-                                int lane, int ctid) {
+// The bin of the K-th largest score of the layer's complete histogram, found by every
+// selection task: thread j holds bins kIndexBins - 1 - (16 j + k), k < 16 (descending); a
+// scan over the threads finds the bin b where the count above it is below K and the count
+// from it on reaches K.  thr[0..2] receive b, how many of b are still to take, b's count.
+__device__ void index_threshold(const Params& p, int layer, uint32_t* thr, uint32_t* wt,
+                                int warp, int lane, int ctid) {
   static_assert(kIndexBins == 16 * kConsumerThreads, "16 bins per consumer thread");
-  uint32_t* gh = p.ix_hist + (size_t)t.layer * kIndexBins;
-  uint32_t* meta = index_meta(p, t.layer);
-  uint32_t* wt = reinterpret_cast<uint32_t*>(scratch);  // [kConsumerWarps]
-  const uint32_t K = (uint32_t)p.KI, P = (uint32_t)p.pos + 1u;
+  const uint32_t* gh = p.ix_hist + (size_t)layer * kIndexBins;
+  const uint32_t K = (uint32_t)p.KI;
   uint32_t cnt[16], sum = 0;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -2074,28 +2092,19 @@ __device__ void index_threshold(const Params& p, const Task& t, float* scratch, 
   consumer_sync(kConsumerThreads);
   uint32_t excl = incl - sum;
   for (int w = 0; w < warp; ++w) excl += wt[w];
-  if (P > K && excl < K && excl + sum >= K) {
+  if (excl < K && excl + sum >= K) {
     uint32_t run = excl;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       if (run < K && run + cnt[k] >= K) {
-        meta[IM_THR] = (uint32_t)(kIndexBins - 1 - (16 * ctid + k));
-        meta[IM_ABOVE] = run;
-        meta[IM_NEED] = K - run;
-        meta[IM_BINCNT] = cnt[k];
+        thr[0] = (uint32_t)(kIndexBins - 1 - (16 * ctid + k));
+        thr[1] = K - run;
+        thr[2] = cnt[k];
       }
       run += cnt[k];
     }
   }
-#pragma unroll
-  for (int k = 0; k < 16; ++k) gh[kIndexBins - 1 - (16 * ctid + k)] = 0u;
-  if (ctid == 0) {
-    meta[IM_NSEL] = 0u;
-    meta[IM_NCAND] = 0u;
-    meta[IM_HASPOS] = 0u;
-  }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) publish_add(p.counters + t.out, 1u);
 }
 
 // Append `take` lanes' values to list[] at the counter *ctr (one atomic per warp); an
@@ -2120,8 +2129,8 @@ __device__ __forceinline__ void warp_append(const Params& p, bool take, uint32_t
 // MSD radix select on keys (low 20 bits of the order key << pb) | (2^pb - 1 - position),
 // pb = bits of a position (all candidates share the top 12 bits); the keys are unique, so
 // exactly `need` of them reach the selected one.
-__device__ void index_pick(const Params& p, const Task& t, float* scratch, int warp, int lane,
-                           int ctid) {
+__device__ void index_pick(const Params& p, const Task& t, float* scratch, uint32_t need, int warp,
+                           int lane, int ctid) {
   uint32_t* meta = index_meta(p, t.layer);
   const unsigned long long* cand = p.ix_cand + (size_t)t.layer * p.cap;
   int32_t* sel = p.ix_sel + (size_t)t.layer * p.KI;
@@ -2144,7 +2153,7 @@ __device__ void index_pick(const Params& p, const Task& t, float* scratch, int w
     for (uint32_t i = ctid; i < n; i += kConsumerThreads) ks[i] = keyof(__ldcg(cand + i));
   const int bits = 20 + pb;
   unsigned long long prefix = 0;
-  uint32_t rem = __ldcg(meta + IM_NEED);
+  uint32_t rem = need;
   for (int sft = (bits + 7) / 8 * 8 - 8; sft >= 0; sft -= 8) {
     for (int i = ctid; i < 256; i += kConsumerThreads) h[i] = 0u;
     consumer_sync(kConsumerThreads);
@@ -2212,11 +2221,13 @@ __device__ void isel_task(const Params& p, const Task& t, float* ub, int* tk, in
                           int ctid, bool& ab) {
   uint32_t* meta = index_meta(p, t.layer);
   const bool sparse = sparse_step(p);
+  uint32_t* th = reinterpret_cast<uint32_t*>(ub);  // threshold bin, still to take, its count
   uint32_t need = 0, bincnt = 0;
   if (sparse) {
-    const uint32_t thr = __ldcg(meta + IM_THR);
-    need = __ldcg(meta + IM_NEED);
-    bincnt = __ldcg(meta + IM_BINCNT);
+    index_threshold(p, t.layer, th, th + 4, warp, lane, ctid);
+    const uint32_t thr = th[0];
+    need = th[1];
+    bincnt = th[2];
     const bool whole_bin = need == bincnt;
     const long long P = p.pos + 1;
     const int t0 = (int)(P * t.r1 / t.aux), t1 = (int)(P * (t.r1 + 1) / t.aux);
@@ -2252,11 +2263,18 @@ __device__ void isel_task(const Params& p, const Task& t, float* ub, int* tk, in
     }
   }
   consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 4] = (long long)globaltimer_ns();
   if (ctid == 0) *tk = ((ticket_add(meta + IM_TICK_B, 1u) + 1u) % (uint32_t)t.aux) == 0u;
   consumer_sync(kConsumerThreads);
   if (!*tk) return;
-  if (sparse && need != bincnt) index_pick(p, t, ub, warp, lane, ctid);
+  // every selection task has read the histogram: clear it for the next step
+  {
+    uint32_t* gh = p.ix_hist + (size_t)t.layer * kIndexBins;
+    for (int b = ctid; b < kIndexBins; b += kConsumerThreads) gh[b] = 0u;
+  }
+  if (sparse && need != bincnt) index_pick(p, t, ub + 16, need, warp, lane, ctid);
   consumer_sync(kConsumerThreads);
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
   if (ctid == 0) {
     const bool ok = wait_counter(p, t.layer * C_PER_LAYER + C_MLA_UK, (uint32_t)p.Hq, t.id);
     if (ok) publish_add(p.counters + t.out, 1u);
@@ -2566,16 +2584,17 @@ __device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, c
 // columns 0-3 the terms of half 0, 4-7 those of half 1.  Of the 16 x 8 products a lane keeps
 // its row g's pair of terms of its half (lanes t4 < 2: half 0, t4 >= 2: half 1), weighed by
 // 16^-tau, the chunk's 2^-sg and the weight block scale (32 columns never straddle a
-// 128-column block).  As for bf16 rows, stage gs + i belongs to warp (gs + i) % 8, which
-// walks all its chunks (four at a time, every load issued first), sums a row's 4 lanes with
-// two shuffles and emits the rows: no barrier per stage, several stages in flight at once.
+// 128-column block).  All 8 warps share each stage, warp w taking the chunks w, w + 8, ...;
+// the lanes of a row and then the warps are summed (shuffles, shared memory), and one thread
+// per row finishes it.
 __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint32_t gs, int ns,
                          uint8_t* ring, uint64_t* full, uint64_t* empty, const uint32_t* tags,
                          float* ub, const float* resid, float rn, float wsel, int uoff, int warp,
-                         int lane, bool& ab, Best& best) {
+                         int lane, int ctid, bool& ab, Best& best) {
   const int Lh = fp8_half_len(g.Kp), P = fp8_row_pitch(g.Kp), nch = Lh / 32;
   const uint8_t* frag = reinterpret_cast<const uint8_t*>(ub);
   const float* csc = ub + 2 * Lh;            // 2^-sg per 32 columns of the span
+  float* red = ub + fp8_frag_floats(g.Kp);   // [2][kConsumerWarps][8]
   const Fp8Scales fs = fp8_scales(p, t, g);
   const bool two = g.nseg == 2;
   const int gq = lane >> 2, t4 = lane & 3, half = t4 >> 1;
@@ -2584,13 +2603,9 @@ __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint
   const uint8_t* bp = frag + (gq >> 2) * 4 * Lh + (gq & 3) * 32 + t4 * 8;
   const int mat = lane >> 3, trow = lane & 7;  // ldmatrix: this lane's matrix and row
   const uint32_t NS = (uint32_t)p.ring_stages;
-  const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);
-  for (int i = first; i < ns; i += kConsumerWarps) {
+  for (int i = 0; i < ns; ++i) {
     const uint32_t sidx = gs + (uint32_t)i, slot = sidx % NS;
-    if (!stage_wait(p, full, tags, sidx)) {
-      ab = true;
-      return;
-    }
+    const bool landed = stage_wait(p, full, tags, sidx);
     const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
     // tile row trow's stage row (gate / up: rows 0-3 gate, 4-7 up), clamped to a loaded row
     const int sr = two ? ((trow >> 2) ? g.rps : 0) + min(trow & 3, nr - 1) : min(trow, nr - 1);
@@ -2599,54 +2614,69 @@ __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint
     // the weight row of this lane's output row gq, for its block scales
     const float* srow = two ? fp8_scale_row(fs, gq >> 2, n0 + min(gq & 3, nr - 1))
                             : fp8_scale_row(fs, 0, n0 + min(gq, nr - 1));
-    constexpr int kU = 4;
-    float accu[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) accu[u] = 0.f;
-    for (int cb = 0; cb < nch; cb += kU) {
-      uint32_t a[kU][4];
-      uint2 b[kU];
-      float sc[kU];
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int cc = min(cb + u, nch - 1);  // clamped: in-range reads
-        ldsm_x4(arow + (uint32_t)(cc * 32), a[u][0], a[u][1], a[u][2], a[u][3]);
-        b[u] = *reinterpret_cast<const uint2*>(bp + cc * 128);
-        const int col = half * Lh + cc * 32;
-        sc[u] = __ldg(srow + ((g.k0 + col) >> 7)) * csc[col >> 5];
-      }
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int cc = cb + u;
-        // columns past Kp are stale shared memory: zero them (the input is zero there); a
-        // chunk past the last one (clamped above) counts nothing
-        const int c0 = cc * 32 + 4 * t4, c1 = Lh + c0;
-        const bool live = cc < nch;
-        if (!live || c0 >= g.Kp) a[u][0] = 0u;
-        if (!live || c0 + 16 >= g.Kp) a[u][2] = 0u;
-        if (!live || c1 >= g.Kp) a[u][1] = 0u;
-        if (!live || c1 + 16 >= g.Kp) a[u][3] = 0u;
-        float d[4];
-        mma_e4m3(d, a[u], b[u].x, b[u].y);
-        const float v = half ? fmaf(d[3], wb, d[2] * wa) : fmaf(d[1], wb, d[0] * wa);
-        accu[u] = fmaf(v, sc[u], accu[u]);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive_n(&empty[slot], kConsumerWarps);
     float acc = 0.f;
+    if (landed) {
+      // kU chunks at a time (chunks w, w + 8, ...), every load issued before the products,
+      // so that a warp keeps several ldmatrix / scale loads and mma in flight
+      constexpr int kU = 4;
+      float accu[kU];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) acc += accu[u];
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);  // the row's two halves and term pairs
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (two) {  // lane (j, 0) holds gate row j, lane (4 + j, 0) up row j
-      const float u = __shfl_down_sync(0xffffffffu, acc, 16);
-      if (t4 == 0 && gq < 4 && gq < nr) {
-        const float aa = acc * rn, bb = u * rn;
-        p.u[uoff + n0 + gq] = wsel * (aa / (1.f + expf(-aa)) * bb);
+      for (int u = 0; u < kU; ++u) accu[u] = 0.f;
+      for (int cb = warp; cb < nch; cb += kU * kConsumerWarps) {
+        uint32_t a[kU][4];
+        uint2 b[kU];
+        float sc[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int cc = min(cb + u * kConsumerWarps, nch - 1);  // clamped: in-range reads
+          ldsm_x4(arow + (uint32_t)(cc * 32), a[u][0], a[u][1], a[u][2], a[u][3]);
+          b[u] = *reinterpret_cast<const uint2*>(bp + cc * 128);
+          const int col = half * Lh + cc * 32;
+          sc[u] = __ldg(srow + ((g.k0 + col) >> 7)) * csc[col >> 5];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int cc = cb + u * kConsumerWarps;
+          // columns past Kp are stale shared memory: zero them (the input is zero there); a
+          // chunk past the last one (clamped above) counts nothing
+          const int c0 = cc * 32 + 4 * t4, c1 = Lh + c0;
+          const bool live = cc < nch;
+          if (!live || c0 >= g.Kp) a[u][0] = 0u;
+          if (!live || c0 + 16 >= g.Kp) a[u][2] = 0u;
+          if (!live || c1 >= g.Kp) a[u][1] = 0u;
+          if (!live || c1 + 16 >= g.Kp) a[u][3] = 0u;
+          float d[4];
+          mma_e4m3(d, a[u], b[u].x, b[u].y);
+          const float v = half ? fmaf(d[3], wb, d[2] * wa) : fmaf(d[1], wb, d[0] * wa);
+          accu[u] = fmaf(v, sc[u], accu[u]);
+        }
       }
-    } else if (t4 == 0 && gq < nr) {
-      gemv_emit(p, t, g, n0 + gq, acc, rn, resid, best);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) acc += accu[u];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(&empty[slot], 1u);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    float* rb = red + (i & 1) * kConsumerWarps * 8;
+    if (t4 == 0) rb[warp * 8 + gq] = acc;
+    if (consumer_sync_or(!landed, kConsumerThreads)) {
+      ab = true;
+      return;
+    }
+    if (ctid < nr && (!two || ctid < 4)) {
+      float v = 0.f, u = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        v += rb[w * 8 + ctid];
+        if (two) u += rb[w * 8 + 4 + ctid];
+      }
+      if (two) {  // gate row ctid (v), up row ctid (u)
+        const float aa = v * rn, bb = u * rn;
+        p.u[uoff + n0 + ctid] = wsel * (aa / (1.f + expf(-aa)) * bb);
+      } else {
+        gemv_emit(p, t, g, n0 + ctid, v, rn, resid, best);
+      }
     }
   }
 }
@@ -2752,11 +2782,11 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
                            ub + p.ub_floats - kTileRedFloats, resid, rnt, wsel, uoff, best, warp,
                            lane, ctid, ab);
       }
-      const bool coop = F8 && g.esz == 1;  // E4M3 stages: the tensor-core tile
+      const bool coop = F8 && g.esz == 1;  // E4M3 stages: every warp takes part in each
       if constexpr (F8) {
         if (coop)
           fp8_task(p, t, g, gs, ns, ring, full, empty, tags, ub, resid, rn, wsel, uoff, warp,
-                   lane, ab, best[0]);
+                   lane, ctid, ab, best[0]);
       }
       // stage gs + i belongs to warp (gs + i) % 8; each warp takes its stages in order
       const int first = (int)((warp - (int)(gs % kConsumerWarps) + kConsumerWarps) % kConsumerWarps);

@@ -434,7 +434,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     const int kp = o.kp ? o.kp : gemv_part_len(o.K, gemv_nparts(o.K, s.kpart_max),
                                                gemv_part_align(s.tiles, o.esz == 1));
     // E4M3 rows: the tensor-core operand of the input covers the 4 row segments
-    xs = std::max(xs, o.esz == 1 ? fp8_frag_floats(kp) : kp);
+    xs = std::max(xs, o.esz == 1 ? fp8_frag_floats(kp) + kFp8RedFloats : kp);
     need = std::max(need, s.tiles ? kTileRows * kTilePitch
                                   : o.esz == 1 ? o.nseg * fp8_row_pitch(kp) : o.nseg * kp * o.esz);
   }
@@ -484,7 +484,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
     if (s.KI)
       s.attn_floats = std::max({s.attn_floats, kIndexBins + kIndexMaxHeads * 128 / 2 +
                                                    kIndexMaxHeads + 64,
-                                512 + 2 * kPickSmemKeys});  // the pick's keys
+                                16 + 512 + 2 * kPickSmemKeys});  // the pick's keys
   }
   const int ubuf_floats = (std::max(s.xs_floats + s.resid_floats + (s.tiles ? kTileRedFloats : 0),
                                      s.attn_floats) + 7) / 8 * 8;
@@ -528,7 +528,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
       b.splits(T_INDEX, l, s.isplits, (int64_t)s.cap / s.isplits * s.DI * 2, cuq, (uint32_t)n2,
                cix);
     const int n3 = b.per_unit(OP_UK, l, H, s.NP, (int64_t)s.NP * s.KL * 2, cuq, (uint32_t)n2, cuk);
-    if (s.KI) b.splits(T_ISEL, l, s.isplits, 0, cix, 1u, csel);
+    if (s.KI) b.splits(T_ISEL, l, s.isplits, 0, cix, (uint32_t)s.isplits, csel);
     const int64_t lat_task =
         (int64_t)((s.KI ? std::min(s.KI, s.cap) : s.cap) - s.M) / S * C * 2;
     if (s.KI) b.mla_attention(l, groups, S, lat_task, csel, 1u, ca);

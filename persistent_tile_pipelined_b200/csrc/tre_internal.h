@@ -65,8 +65,9 @@ TRE_HD inline int fp8_half_len(int Kp) { return (Kp + 63) / 64 * 32; }
 TRE_HD inline int fp8_span(int Kp) { return 2 * fp8_half_len(Kp); }
 TRE_HD inline int fp8_row_pitch(int Kp) { return fp8_span(Kp) + 16; }
 // The input operand of an E4M3 GEMV: 4 E4M3 terms per input (4 bytes) in fragment order,
-// then one scale per 32 columns: its size in floats
+// then one scale per 32 columns: its size in floats (the cross-warp sums follow it)
 TRE_HD inline int fp8_frag_floats(int Kp) { return fp8_span(Kp) + fp8_span(Kp) / 32; }
+constexpr int kFp8RedFloats = 2 * kConsumerWarps * 8;
 TRE_HD inline int fp8_rows_per_stage(int Kp, int nseg, int stage_bytes) {
   const int r = stage_bytes / (nseg * fp8_row_pitch(Kp));
   return r < 1 ? 1 : r;
@@ -116,12 +117,9 @@ constexpr int kIndexBins = 1 << kIndexBinBits;
 constexpr int kIndexMaxHeads = 64;
 constexpr int kPickSmemKeys = 3840;  // threshold-bin candidates the pick keeps in shared memory
 TRE_HD inline int sparse_lat_pitch(int C) { return C * 2 + 16; }  // bytes per gathered row
-// Per-layer selection state (uint32 words): the threshold bin, how many positions lie in
-// bins above it, how many of the threshold bin are still to take, that bin's count, the
-// chosen-position count, the candidate count, whether the new position was chosen, and
-// the arrival tickets of the scoring and selection tasks.
-enum IndexMeta { IM_THR = 0, IM_ABOVE = 1, IM_NEED = 2, IM_BINCNT = 3, IM_NSEL = 4,
-                 IM_NCAND = 5, IM_HASPOS = 6, IM_TICK_A = 7, IM_TICK_B = 8, IM_WORDS = 16 };
+// Per-layer selection state (uint32 words): the chosen-position count, the candidate
+// count, whether the new position was chosen, and the selection tasks' arrival ticket.
+enum IndexMeta { IM_NSEL = 4, IM_NCAND = 5, IM_HASPOS = 6, IM_TICK_B = 8, IM_WORDS = 16 };
 constexpr int kMlaHeadGroup = 16;     // query heads per MLA attention tile (the mma M)
 constexpr int kMlaPosPerStage = 32;   // latent rows per MLA attention stage
 constexpr int kMlaBox = 64;           // latent columns per tensor-map box (128 B, swizzled)

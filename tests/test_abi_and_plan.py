@@ -137,11 +137,11 @@ def check_plan(wl, nsm, **over):
         assert all(T["id"][j] < T["id"][i] for j in producers)
         kind = dep % C_PER_LAYER
         if wl.kind == "mla" and kind in (C_MLA_IDX, C_MLA_SEL):
-            # sparse: the index and selection counters are bumped once, by the scoring /
-            # selection task that arrives last; attention waits for the selection
-            assert T["dep_count"][i] == 1
+            # sparse: every scoring task bumps the index counter; the selection counter is
+            # bumped once, by the selection task that arrives last; attention waits for it
             want = T_INDEX if kind == C_MLA_IDX else T_ISEL
             assert producers and all(T["type"][j] == want for j in producers)
+            assert T["dep_count"][i] == (len(producers) if kind == C_MLA_IDX else 1)
             assert T["type"][i] == (T_ISEL if kind == C_MLA_IDX else T_MLA_ATTN)
         elif T["type"][i] == T_GEMV and T["op"][i] == OP_UV:
             # every MLA attention split publishes; W_uv merges a head's splits
