@@ -58,7 +58,7 @@ constexpr int kPlaneBatch = TRE_PLANE_BATCH;
 __device__ bool wait_counter(const Params& p, int idx, uint32_t count, int detail) {
   if (p.op_group >= 0) return true;
   const uint32_t target = p.epoch * count;
-  const uint32_t* c = p.counters + idx;
+  const uint32_t* c = p.counters + (size_t)idx * kCtrStride;
   if ((int32_t)(ld_acquire_gpu(c) - target) >= 0) return true;
   const uint64_t t0 = globaltimer_ns();
   long long c0 = clock64();
@@ -1480,7 +1480,7 @@ __device__ void attn_task(const Params& p, const Task& t, uint32_t gs, int ns, u
     }
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) publish_add(p.counters + t.out, 1u);
+  if (ctid == 0) publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);
 }
 
 template <int MT>
@@ -1621,7 +1621,7 @@ __device__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint3
     }
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) publish_add(p.counters + t.out, 1u);
+  if (ctid == 0) publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);
 }
 
 // ---- absorbed MLA: latent attention on tensor cores ---------------------------------------------
@@ -1874,7 +1874,7 @@ __device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int n
   consumer_sync(kConsumerThreads);
   if (ctid == 0) {
     if (p.trace) p.trace[(size_t)t.id * kTraceCols + 6] = (long long)globaltimer_ns();
-    publish_add(p.counters + t.out, 1u);
+    publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);
   }
 }
 
@@ -2063,7 +2063,7 @@ __device__ void index_task(const Params& p, const Task& t, uint32_t gs, int ns, 
       meta[IM_NCAND] = 0u;
       meta[IM_HASPOS] = 0u;
     }
-    publish_add(p.counters + t.out, 1u);  // after the CTA's histogram adds (barrier above)
+    publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);  // after the CTA's histogram adds (barrier above)
   }
 }
 
@@ -2277,7 +2277,7 @@ __device__ void isel_task(const Params& p, const Task& t, float* ub, int* tk, in
   if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 5] = (long long)globaltimer_ns();
   if (ctid == 0) {
     const bool ok = wait_counter(p, t.layer * C_PER_LAYER + C_MLA_UK, (uint32_t)p.Hq, t.id);
-    if (ok) publish_add(p.counters + t.out, 1u);
+    if (ok) publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);
     *tk = ok ? 0 : 1;
   }
   consumer_sync(kConsumerThreads);
@@ -2443,7 +2443,7 @@ __device__ void route_topk(const Params& p, int layer, float* sc, int warp, int 
   }
   if (lane < p.topk) p.route_w[layer * p.topk + lane] = mine / tot;
   __syncwarp();
-  if (lane == 0) publish_add(p.counters + layer * C_PER_LAYER + C_ROUTE, 1u);
+  if (lane == 0) publish_add(p.counters + (size_t)(layer * C_PER_LAYER + C_ROUTE) * kCtrStride, 1u);
 }
 
 // The last slot of a MoE-down row block to finish: x = h1 + sum of the slots' partial rows
@@ -2459,7 +2459,7 @@ __device__ void mo_slices_combine(const Params& p, const Task& t, int np, int ct
     if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) publish_add(p.counters + t.out, 1u);
+  if (ctid == 0) publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);
 }
 
 __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
@@ -2472,7 +2472,7 @@ __device__ void moe_down_combine(const Params& p, const Task& t, int ctid) {
     if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
   }
   consumer_sync(kConsumerThreads);
-  if (ctid == 0) publish_add(p.counters + t.out, 1u);
+  if (ctid == 0) publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);
 }
 
 
@@ -2698,6 +2698,9 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
   bool ab = false;
   for (int ti = 0; ti < ntask; ++ti) {
     const Task t = my[ti];
+    // stage count before the dependency wait (off the hand-off's critical path), except for
+    // tasks whose stages follow this step's sparse selection
+    const int ns_early = (MLA && t.type == T_MLA_ATTN) ? -1 : task_nstages<TILED>(p, t);
     if (ctid == 0) {
       long long* tr = p.trace ? p.trace + (size_t)t.id * kTraceCols : nullptr;
       if (tr) tr[0] = (long long)globaltimer_ns();
@@ -2711,8 +2714,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     }
     consumer_sync(kConsumerThreads);
     if (flags[0]) break;  // uniform: every consumer thread read the same flag
-    // after the wait: a sparse attention task's stages follow this step's selection
-    const int ns = task_nstages<TILED>(p, t);
+    const int ns = ns_early >= 0 ? ns_early : task_nstages<TILED>(p, t);
 
     if (!MLA && t.type == T_ATTN) {
       cur_key = -1;  // the attention scratch aliases the input-vector planes
@@ -2931,7 +2933,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         consumer_sync(kConsumerThreads);
         if (flags[1]) moe_down_combine(p, t, ctid);
       } else if (ctid == 0 && t.out >= 0) {
-        publish_add(p.counters + t.out, 1u);
+        publish_add(p.counters + (size_t)t.out * kCtrStride, 1u);
       }
     }
     if (ctid == 0) {

@@ -125,7 +125,7 @@ extern "C" __attribute__((visibility("default"))) tre_status tre_decode_step_sta
   const size_t o_begin = cv.take<int32_t>(begin.size());
   const size_t o_layers = cv.take<LayerPtrs>(s.L);
   const size_t o_zero = cv.take<uint32_t>(0);  // everything from here to o_zero_end starts at 0
-  const size_t o_ctr = cv.take<uint32_t>(s.n_counters);
+  const size_t o_ctr = cv.take<uint32_t>((size_t)s.n_counters * kCtrStride);
   const size_t o_tick = cv.take<uint32_t>(s.Hkv);
   const size_t o_lmt = cv.take<uint32_t>(1);
   const size_t o_arg = cv.take<unsigned long long>(kMaxTokens);

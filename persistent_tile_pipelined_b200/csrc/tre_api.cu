@@ -339,8 +339,8 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   size_t o_begin = cv.take<int32_t>(begin.size());
   size_t o_ranges = cv.take<int32_t>(ranges.size());
   size_t o_layers = cv.take<LayerPtrs>(s.L);
-  size_t o_ctr = cv.take<uint32_t>(s.n_counters);
-  size_t o_ctr_op = cv.take<uint32_t>(s.n_counters);  // bumped by kernel-per-op launches only
+  size_t o_ctr = cv.take<uint32_t>((size_t)s.n_counters * kCtrStride);
+  size_t o_ctr_op = cv.take<uint32_t>((size_t)s.n_counters * kCtrStride);  // bumped by kernel-per-op launches only
   size_t o_tick = cv.take<uint32_t>(std::max(s.Hkv, mla ? s.Hq / kMlaHeadGroup : 1));
   size_t o_lmt = cv.take<uint32_t>(1);
   size_t o_arg = cv.take<unsigned long long>(kMaxTokens);
@@ -749,11 +749,11 @@ TRE_EXPORT tre_status tre_debug_check(tre_engine* e, int32_t* bad_counter_out,
   if (e->last_stream) CK(cudaStreamSynchronize(e->last_stream));
   CK(cudaDeviceSynchronize());
   const int n = e->shape.n_counters;
-  std::vector<uint32_t> c(n);
-  CK(cudaMemcpy(c.data(), e->base.counters, (size_t)n * 4, cudaMemcpyDeviceToHost));
+  std::vector<uint32_t> c((size_t)n * kCtrStride);
+  CK(cudaMemcpy(c.data(), e->base.counters, c.size() * 4, cudaMemcpyDeviceToHost));
   *bad_counter_out = -1;
   for (int i = 0; i < n; ++i)
-    if (e->expected[i] && c[i] != e->epoch * e->expected[i]) {
+    if (e->expected[i] && c[(size_t)i * kCtrStride] != e->epoch * e->expected[i]) {
       *bad_counter_out = i;
       break;
     }
@@ -829,8 +829,8 @@ TRE_EXPORT tre_status tre_reset(tre_engine* e, tre_stream stream) {
   cudaStream_t s = (cudaStream_t)stream;
   CK(cudaDeviceSynchronize());
   const Params& p = e->base;
-  CK(cudaMemsetAsync(p.counters, 0, (size_t)e->shape.n_counters * 4, s));
-  CK(cudaMemsetAsync(e->op_counters, 0, (size_t)e->shape.n_counters * 4, s));
+  CK(cudaMemsetAsync(p.counters, 0, (size_t)e->shape.n_counters * kCtrStride * 4, s));
+  CK(cudaMemsetAsync(e->op_counters, 0, (size_t)e->shape.n_counters * kCtrStride * 4, s));
   CK(cudaMemsetAsync(p.tickets, 0,
                      (size_t)std::max(e->shape.Hkv, e->shape.kind == TRE_LAYER_MLA
                                                         ? e->shape.Hq / kMlaHeadGroup : 1) * 4,

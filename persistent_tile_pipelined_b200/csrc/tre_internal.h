@@ -23,6 +23,9 @@ constexpr int kMaxTopK = 32;
 constexpr int kDefaultPrefetchKB = 0;    // next-task L2 prefetch: opt-in (measured 4% slower)
 constexpr int kMaxStageBytes = 65536;
 constexpr int kMaxTokens = 4;            // tokens per step (multi-token verify tiles)
+// Dependency counters sit kCtrStride words apart (packed: padding them to 128 bytes each
+// measured no different)
+constexpr int kCtrStride = 1;
 // Multi-token GEMV on tensor cores: a stage is one tile of 16 weight rows x up to 1024
 // input columns, each row copied into a 16-byte-padded slot (conflict-free ldmatrix).
 constexpr int kTileRows = 16;
