@@ -1580,6 +1580,7 @@ __device__ void uk_task(const Params& p, const Task& t, const GemvGeom& g, uint3
     for (int w = 0; w < kConsumerWarps; ++w) v += red[w * KL + c];
     qf[c] = v;
   }
+  if (ctid == 0 && p.trace) p.trace[(size_t)t.id * kTraceCols + 7] = (long long)globaltimer_ns();
   const int R2 = p.R / 2;
   for (int i = ctid; i < R2; i += kConsumerThreads) {
     const float x0 = __ldcg(qh + p.NP + i), x1 = __ldcg(qh + p.NP + i + R2);
