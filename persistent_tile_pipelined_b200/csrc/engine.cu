@@ -469,18 +469,21 @@ __device__ __forceinline__ void tile_next(TileStage& ts, const Task& t, const Ge
   tile_set(ts, t, g);
 }
 
+template <bool MLA, bool SP>
 __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, const GemvGeom& g,
                                                 int t0, int t1, int i) {
   if (t.type == T_GEMV) {
     const int nr = min(g.rps, t.r1 - (t.r0 + i * g.rps));
     return (uint32_t)(g.nseg * nr * g.Kp * g.esz);
   }
-  if (t.type == T_INDEX) return (uint32_t)(p.DI * 2 * kIndexRows);  // whole boxes
-  if (t.type == T_MLA_ATTN) {
+  if constexpr (SP) {
+    if (t.type == T_INDEX) return (uint32_t)(p.DI * 2 * kIndexRows);  // whole boxes
     // sparse: every row of the stage is gathered (rows past the split repeat its first)
-    if (sparse_step(p)) return (uint32_t)(kMlaPosPerStage * (p.KL + p.R) * 2);
+    if (t.type == T_MLA_ATTN && sparse_step(p)) return (uint32_t)(kMlaPosPerStage * (p.KL + p.R) * 2);
+  }
+  if constexpr (MLA) {
     // whole boxes (rows past the cache are zero-filled)
-    return (uint32_t)((p.KL + p.R) / kMlaBox * kMlaPosPerStage * 128);
+    if (t.type == T_MLA_ATTN) return (uint32_t)((p.KL + p.R) / kMlaBox * kMlaPosPerStage * 128);
   }
   return (uint32_t)(2 * (p.D / 64) * p.pps * 128);  // K and V boxes of pps rows
 }
@@ -488,6 +491,7 @@ __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, 
 // Issue the bulk copies of stage i into `dst`: one copy per contiguous run of rows (per
 // segment; gate rows at the stage's start, up rows after `rps` rows), spread over the
 // producer lanes; attention: the K rows then the V rows (lanes 0 and 1).
+template <bool MLA, bool SP>
 __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, const GemvGeom& g,
                                             const RowSrc& rs, int t0, int t1, int i, int lane,
                                             uint8_t* dst, uint64_t* bar, uint64_t pol) {
@@ -537,13 +541,13 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
         n += take;
       }
     }
-  } else if (t.type == T_INDEX) {
+  } else if (SP && t.type == T_INDEX) {
     // 64-column boxes of kIndexRows index keys, 128-byte swizzled
     if (lane < p.DI / 64) {
       const uint8_t* map = static_cast<const uint8_t*>(p.ix_maps) + (size_t)t.layer * 128;
       tma_load_2d(dst + (size_t)lane * kIndexRows * 128, map, lane * 64, t0 + i * kIndexRows, bar);
     }
-  } else if (t.type == T_MLA_ATTN && sparse_step(p)) {
+  } else if (SP && t.type == T_MLA_ATTN && sparse_step(p)) {
     // gather: lane r copies the latent row of chosen entry t0 + 32 i + r (past the split:
     // entry t0 again, so that the masked rows hold finite values) at the padded pitch
     const int C = p.KL + p.R;
@@ -557,7 +561,7 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
     bulk_g2s(dst + (size_t)lane * sparse_lat_pitch(C),
              reinterpret_cast<const uint8_t*>(p.layers[t.layer].k_cache) + (size_t)pos * C * 2,
              (uint32_t)C * 2u, bar, pol);
-  } else if (t.type == T_MLA_ATTN) {
+  } else if (MLA && t.type == T_MLA_ATTN) {
     // 64-column boxes of 32 latent rows, 128-byte swizzled (see mla.cuh)
     if (lane < (p.KL + p.R) / kMlaBox) {
       const uint8_t* map = static_cast<const uint8_t*>(p.kv_maps) + (size_t)t.layer * 128;
@@ -655,7 +659,7 @@ __device__ bool hold_for_consumers(const Params& p, const volatile int* done, in
   return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
 }
 
-template <bool TILED>
+template <bool TILED, bool MLA, bool SP>
 __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, uint32_t* tags,
                          const volatile int* done, int lane) {
@@ -689,7 +693,7 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
       if (!ok) break;
     }
-    if (t.type == T_MLA_ATTN && sparse_step(p)) {  // the chosen positions pick the rows
+    if (SP && t.type == T_MLA_ATTN && sparse_step(p)) {  // the chosen positions pick the rows
       bool r = true;
       if (lane == 0) r = wait_dep(p, t);
       ok = __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
@@ -709,11 +713,11 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       // each lane that copies through a cache's tensor map acquires the map first (the
       // allocation-free entry point rewrites its maps in place between launches)
       const uint8_t* maps = static_cast<const uint8_t*>(p.kv_maps);
-      if (t.type == T_INDEX) {
+      if (SP && t.type == T_INDEX) {
         if (lane < p.DI / 64)
           tensormap_acquire(static_cast<const uint8_t*>(p.ix_maps) + (size_t)t.layer * 128);
-      } else if (t.type == T_ISEL) {
-      } else if (t.type == T_MLA_ATTN) {
+      } else if (SP && t.type == T_ISEL) {
+      } else if (MLA && t.type == T_MLA_ATTN) {
         if (lane < (p.KL + p.R) / kMlaBox) tensormap_acquire(maps + (size_t)t.layer * 128);
       } else if (lane < 2 * (p.D / 64)) {
         tensormap_acquire(maps + ((size_t)t.layer * 2 + (lane >= p.D / 64)) * 128);
@@ -740,7 +744,7 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       if (lane == 0) {
         *reinterpret_cast<volatile uint32_t*>(tags + slot) = gs;
         mbar_arrive_expect_tx(&full[slot], tiled ? (uint32_t)(ts.nr * ts.kw * 2)
-                                                 : stage_total(p, t, g, t0, t1, i));
+                                                 : stage_total<MLA, SP>(p, t, g, t0, t1, i));
       }
       __syncwarp();
       if (tiled) {
@@ -751,7 +755,7 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
                    &full[slot], pol);
         tile_next(ts, t, g);
       } else {
-        issue_stage(p, t, g, rs, t0, t1, i, lane, ring + (size_t)slot * SB, &full[slot], pol);
+        issue_stage<MLA, SP>(p, t, g, rs, t0, t1, i, lane, ring + (size_t)slot * SB, &full[slot], pol);
       }
       if (TILED) ring_next(slot, ph, NS);
     }
@@ -2375,39 +2379,59 @@ __device__ __forceinline__ void prefetch_resid(const Params& p, const Task& t, c
   }
 }
 
+// One output row of a GEMV task (MLA: the absorbed-MLA ops' epilogues; else GQA / MoE),
+// specialised per stack so that each kernel dispatches over its own ops only.
+template <bool MLA>
 __device__ __forceinline__ void gemv_emit(const Params& p, const Task& t, const GemvGeom& g, int n,
                                           float v, float rn, const float* resid, Best& best,
                                           int tok = 0) {
-  switch (t.op) {
-    case OP_QKV: p.qkv[(size_t)tok * (p.Hq + 2 * p.Hkv) * p.D + n] = v * rn; break;
-    case OP_UQ: p.qkv[n] = v * rn; break;
-    case OP_MDQKV: {
-      const float y = v * rn;
-      p.cqkv[n] = y;
-      const int ki = n - (p.QL + p.KL + p.R);  // sparse: this position's index key
-      if (ki >= 0 && ki < p.DI)
-        reinterpret_cast<__nv_bfloat16*>(p.layers[t.layer].v_cache)[(size_t)p.pos * p.DI + ki] =
-            __float2bfloat16_rn(y);
-    } break;
-    case OP_UV: p.mla_o[n] = v; break;
-    case OP_O: p.h1[(size_t)tok * p.d + n] = resid[n - t.r0] + v; break;
-    case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
-    case OP_MDOWN:
-    case OP_MOS: p.mpart[(size_t)g.part * p.d + n] = v; break;
-    case OP_DOWN:
-    case OP_MO: {
-      const float y = resid[n - t.r0] + v;
-      p.x[(size_t)tok * p.d + n] = y;
-      if (g.part == g.np - 1) {
-        if (p.hidden) p.hidden[((size_t)t.layer * p.m + tok) * p.d + n] = y;
-        if (p.x_out && t.layer == p.L - 1) p.x_out[(size_t)tok * p.d + n] = y;
-      }
-    } break;
-    default: {
-      const float y = v * rn;
-      p.logits[(size_t)tok * p.V + n] = y;
-      best_update(best, y, n);
-    } break;
+  if constexpr (MLA) {
+    switch (t.op) {
+      case OP_UQ: p.qkv[n] = v * rn; break;
+      case OP_MDQKV: {
+        const float y = v * rn;
+        p.cqkv[n] = y;
+        const int ki = n - (p.QL + p.KL + p.R);  // sparse: this position's index key
+        if (ki >= 0 && ki < p.DI)
+          reinterpret_cast<__nv_bfloat16*>(p.layers[t.layer].v_cache)[(size_t)p.pos * p.DI + ki] =
+              __float2bfloat16_rn(y);
+      } break;
+      case OP_UV: p.mla_o[n] = v; break;
+      case OP_MOS: p.mpart[(size_t)g.part * p.d + n] = v; break;
+      case OP_MO: {
+        const float y = resid[n - t.r0] + v;
+        p.x[n] = y;
+        if (g.part == g.np - 1) {
+          if (p.hidden) p.hidden[(size_t)t.layer * p.d + n] = y;
+          if (p.x_out && t.layer == p.L - 1) p.x_out[n] = y;
+        }
+      } break;
+      default: {
+        const float y = v * rn;
+        p.logits[n] = y;
+        best_update(best, y, n);
+      } break;
+    }
+  } else {
+    switch (t.op) {
+      case OP_QKV: p.qkv[(size_t)tok * (p.Hq + 2 * p.Hkv) * p.D + n] = v * rn; break;
+      case OP_O: p.h1[(size_t)tok * p.d + n] = resid[n - t.r0] + v; break;
+      case OP_ROUTER: p.scores[n] = 1.f / (1.f + expf(-v * rn)); break;
+      case OP_MDOWN: p.mpart[(size_t)g.part * p.d + n] = v; break;
+      case OP_DOWN: {
+        const float y = resid[n - t.r0] + v;
+        p.x[(size_t)tok * p.d + n] = y;
+        if (g.part == g.np - 1) {
+          if (p.hidden) p.hidden[((size_t)t.layer * p.m + tok) * p.d + n] = y;
+          if (p.x_out && t.layer == p.L - 1) p.x_out[(size_t)tok * p.d + n] = y;
+        }
+      } break;
+      default: {
+        const float y = v * rn;
+        p.logits[(size_t)tok * p.V + n] = y;
+        best_update(best, y, n);
+      } break;
+    }
   }
 }
 
@@ -2565,7 +2589,7 @@ __device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, c
           const float a = y0 * rnt[vv], bb = y1 * rnt[vv];
           p.u[(size_t)vv * p.F + uoff + n] = wsel * (a / (1.f + expf(-a)) * bb);
         } else {
-          gemv_emit(p, t, g, n, y0, rnt[vv], resid + vv * kMaxResidRows, best[vv], vv);
+          gemv_emit<false>(p, t, g, n, y0, rnt[vv], resid + vv * kMaxResidRows, best[vv], vv);
         }
       }
     }
@@ -2676,7 +2700,7 @@ __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint
         const float aa = v * rn, bb = u * rn;
         p.u[uoff + n0 + ctid] = wsel * (aa / (1.f + expf(-aa)) * bb);
       } else {
-        gemv_emit(p, t, g, n0 + ctid, v, rn, resid, best);
+        gemv_emit<false>(p, t, g, n0 + ctid, v, rn, resid, best);
       }
     }
   }
@@ -2832,7 +2856,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
                         r0 + (size_t)min(3, nv - 1) * K8, K8, xl, xh, lane, o0, o1, o2, o3);
             const float v = reduce4(o0, o1, o2, o3, lane);
             const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-            if ((lane & 7) == 0 && idx < nv) gemv_emit(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
+            if ((lane & 7) == 0 && idx < nv) gemv_emit<MLA>(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
           }
         } else if (TILED) {
         } else if (g.nseg == 2) {  // MT tokens: gate / up rows as above, per token
@@ -2869,7 +2893,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
             for (int v = 0; v < MT; ++v) {
               const float val = reduce4(out[v][0], out[v][1], out[v][2], out[v][3], lane);
               if ((lane & 7) == 0 && idx < nv)
-                gemv_emit(p, t, g, n0 + r + idx, val, rnt[v], resid + v * kMaxResidRows, best[v], v);
+                gemv_emit<MLA>(p, t, g, n0 + r + idx, val, rnt[v], resid + v * kMaxResidRows, best[v], v);
             }
           }
         }
@@ -2987,7 +3011,7 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
-    producer<TILED>(p, my, ntask, ring, full, empty, tags,
+    producer<TILED, MLA, SP>(p, my, ntask, ring, full, empty, tags,
              reinterpret_cast<const volatile int*>(misc + 80), threadIdx.x & 31);
     return;
   }
