@@ -638,7 +638,7 @@ __device__ __forceinline__ bool op_boundary(const Task& a, const Task& b) {
 }
 
 // Producer: wait (bounded) until this SM's consumers have finished task ti - 1.
-__device__ bool hold_for_consumers(const Params& p, const volatile int* done, int ti, int detail,
+__device__ __forceinline__ bool hold_for_consumers(const Params& p, const volatile int* done, int ti, int detail,
                                    int lane) {
   bool r = true;
   if (lane == 0) {
