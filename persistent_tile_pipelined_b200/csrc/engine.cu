@@ -1892,9 +1892,10 @@ __device__ void mla_attn_task(const Params& p, const Task& t, uint32_t gs, int n
 // stage's positions 16 w .. 16 w + 15 against every head, so ReLU, weights and the sum
 // over heads stay in the warp (per thread, then shuffles).  The scores go to
 // iscore[layer]; a shared histogram of their order keys' top bits is added into the
-// layer's global histogram.  The last split also scores the new position from its
-// on-chip key (rounded to bf16 as the cache holds it); the split that arrives last picks
-// the threshold bin (index_threshold).
+// layer's global histogram, and every split publishes the layer's index counter (split 0
+// first resets the chosen counts).  The last split also scores the new position from its
+// on-chip key (rounded to bf16 as the cache holds it).
+
 // Byte offset of 16-byte chunk c of row r of the [H_I][D_I] bf16 query tile (rows of
 // 2 D_I bytes, chunks XOR-swizzled by r & 7 so that ldmatrix reads 8 rows conflict-free).
 __device__ __forceinline__ uint32_t qtile_off(int r, int c, int DI) {
@@ -2215,10 +2216,11 @@ __device__ void index_pick(const Params& p, const Task& t, float* scratch, uint3
   }
 }
 
-// Selection task = split sp of the positions [0, pos]: positions whose bin is above the
-// threshold bin are chosen (the whole threshold bin when all of it is to take), the
-// threshold bin's others become candidates; the new position is flagged instead of listed
-// (its latent row comes from on chip).  The task that arrives last runs index_pick when
+// Selection task = split sp of the positions [0, pos]: it finds the threshold bin in the
+// complete histogram (index_threshold), then positions whose bin is above it are chosen
+// (the whole threshold bin when all of it is to take) and the threshold bin's others
+// become candidates; the new position is flagged instead of listed (its latent row comes
+// from on chip).  The task that arrives last clears the histogram, runs index_pick when
 // needed, then (the attention also reads this layer's W_uk contraction) waits for the
 // W_uk tasks and publishes the layer's selection counter.  Steps with pos + 1 <= K only
 // do the last part.
