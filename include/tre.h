@@ -211,6 +211,8 @@ typedef struct {
   int32_t kv_splits;
   int32_t ring_stages, stage_bytes, smem_bytes;
   int32_t max_tasks_per_sm;
+  int32_t gemv_tiles;             /* 1: multi-token GEMV stages are 16-row tensor-core tiles */
+  int32_t index_splits;           /* sparse MLA: index scoring (= selection) tasks per layer */
   int64_t weight_bytes;           /* weight bytes streamed per step                     */
   int64_t kv_bytes_at_capacity;   /* KV bytes streamed per step at pos = capacity - M   */
   int64_t max_sm_bytes, min_sm_bytes;  /* per-CTA streamed bytes (balance)              */

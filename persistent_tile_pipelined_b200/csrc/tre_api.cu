@@ -145,6 +145,8 @@ TRE_EXPORT tre_status tre_plan_inspect(const tre_config* cfg, int32_t num_sms,
   int mx = 0;
   for (int i = 0; i < s.nsm; ++i) mx = std::max(mx, begin[i + 1] - begin[i]);
   info->max_tasks_per_sm = mx;
+  info->gemv_tiles = s.tiles;
+  info->index_splits = s.isplits;
   const int64_t row_new = s.kind == TRE_LAYER_MLA ? (int64_t)(s.KL + s.R) * 2 : (int64_t)s.Hkv * s.D * 4;
   const int64_t row_read = s.kind == TRE_LAYER_MLA ? (int64_t)(s.KL + s.R) * 2 : (int64_t)s.Hkv * s.D * 4;
   info->weight_bytes = step_bytes(s, 0) - (int64_t)s.L * (row_new + (int64_t)s.DI * 2) -

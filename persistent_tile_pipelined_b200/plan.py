@@ -18,19 +18,6 @@ from . import tre
 from .synth import workloads as W
 from .trace import OP_NAMES
 
-TILE_STAGE_BYTES = 16 * (1024 * 2 + 16)  # one 16-row tile of 1024 padded columns
-
-
-def gemv_tiles(cfg) -> bool:
-    """The GEMV form rule of tre_config.multi_token_gemv: tensor-core tiles when asked for
-    (2), or by the planner's choice (0) at 4 tokens per step when hidden and ffn are
-    multiples of 16; CUDA-core rows otherwise (and always at one token)."""
-    M = max(1, cfg.max_tokens_per_step)
-    if M == 1 or cfg.multi_token_gemv == 1:
-        return False
-    return cfg.multi_token_gemv == 2 or (M >= 4 and cfg.hidden % 16 == 0 and cfg.ffn % 16 == 0)
-
-
 def report(wl, num_sms: int = 148, **overrides) -> dict:
     cfg = tre.config_from_workload(wl, **overrides)
     info = tre.tre_plan_inspect(cfg, num_sms=num_sms)
@@ -38,10 +25,10 @@ def report(wl, num_sms: int = 148, **overrides) -> dict:
     w0 = tasks[:, 0].astype("int64") & 0xFFFFFFFF
     kinds = Counter()
     for typ, op in zip((w0 & 0xFF).tolist(), ((w0 >> 8) & 0xFF).tolist()):
-        kinds["attention" if typ == 1 else "mla_attention" if typ == 2
-              else OP_NAMES.get(op, str(op))] += 1
+        kinds[{1: "attention", 2: "mla_attention", 3: "index_score",
+               4: "index_select"}.get(typ) or OP_NAMES.get(op, str(op))] += 1
     M = max(1, cfg.max_tokens_per_step)
-    tiles = gemv_tiles(cfg)
+    tiles = bool(info.gemv_tiles)  # the planner's choice of GEMV form
     kv_at_prefill = info.kv_bytes_at_capacity * wl.prefill / max(1, cfg.kv_capacity - M)
     return {
         "workload": wl.name, "kind": wl.kind, "tokens_per_step": M,

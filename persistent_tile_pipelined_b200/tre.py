@@ -65,7 +65,7 @@ class tre_weights(ctypes.Structure):
 class tre_plan_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_sms", "num_tasks", "num_counters", "kv_splits", "ring_stages", "stage_bytes",
-        "smem_bytes", "max_tasks_per_sm")] + [
+        "smem_bytes", "max_tasks_per_sm", "gemv_tiles", "index_splits")] + [
         (n, ctypes.c_int64) for n in ("weight_bytes", "kv_bytes_at_capacity", "max_sm_bytes",
                                       "min_sm_bytes")]
 

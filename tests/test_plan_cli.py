@@ -5,7 +5,7 @@ import sys
 
 import pytest
 
-from persistent_tile_pipelined_b200 import plan, tre
+from persistent_tile_pipelined_b200 import tre
 from persistent_tile_pipelined_b200.synth import workloads as W
 
 
@@ -19,12 +19,19 @@ from persistent_tile_pipelined_b200.synth import workloads as W
     (W.TINY.replace(tokens_per_step=4, hidden=264, ffn=696), {}, False),
 ])
 def test_gemv_form_rule_matches_the_plan(wl, over, tiles):
-    """The documented form rule agrees with the planner: tile plans carry one 16-row tile of
-    1024 padded columns per stage, row plans (32 KB stages here) do not."""
+    """The documented form rule (tre.h, multi_token_gemv) is what the planner reports, and
+    tile plans carry one 16-row tile of 1024 padded columns per stage, row plans (32 KB
+    stages here) do not."""
     cfg = tre.config_from_workload(wl, **over)
-    assert plan.gemv_tiles(cfg) == tiles
     info = tre.tre_plan_inspect(cfg)
-    assert (info.stage_bytes >= plan.TILE_STAGE_BYTES) == tiles
+    assert bool(info.gemv_tiles) == tiles
+    assert (info.stage_bytes >= 16 * (1024 * 2 + 16)) == tiles
+
+
+def test_plan_reports_sparse_splits():
+    info = tre.tre_plan_inspect(tre.config_from_workload(W.MLA4_SPARSE128K))
+    assert info.index_splits == info.num_sms == 148
+    assert tre.tre_plan_inspect(tre.config_from_workload(W.MLA4)).index_splits == 0
 
 
 def test_plan_report_cli():
