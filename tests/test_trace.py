@@ -53,6 +53,16 @@ def test_summary_of_a_synthetic_trace():
         assert s["finish_spread_us"][op]["mean"] == pytest.approx(np.mean(spread))
 
 
+def test_sparse_plan_op_names():
+    """Index scoring and selection tasks and the W_o K-slices are named in the summary."""
+    cfg = tre.config_from_workload(W.MLA4_SPARSE128K.replace(n_layers=1))
+    tasks, begin = tre.tre_plan_tasks(cfg, num_sms=148)
+    tt = T.task_table(tasks)
+    names = {T.op_name(tt, i) for i in range(len(tasks))}
+    assert {"index_score", "index_select", "mla_attention", "uk", "uv", "mla_o"} <= names
+    assert "?" not in names
+
+
 def test_chrome_trace_export():
     tr, tasks = synthetic()
     out = os.path.join(ROOT, "tests", "_build")
