@@ -92,6 +92,14 @@ class Oracle:
         L.orc_e4m3_to_real.argtypes = [ctypes.c_uint8]
         L.orc_e4m3_to_real.restype = creal
         L.orc_gemv_fp8.argtypes = [i32, i32, vp, vp, vp, vp]
+        L.orc_e2m1_to_real.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_to_real.restype = creal
+        L.orc_e8m0_to_real.argtypes = [ctypes.c_uint8]
+        L.orc_e8m0_to_real.restype = creal
+        L.orc_mxfp4_pitch.argtypes = [i32]
+        L.orc_mxfp4_pitch.restype = i32
+        L.orc_gemv_mxfp4.argtypes = [i32, i32, vp, vp, vp]
+        L.orc_swiglu_mlp_mxfp4.argtypes = [i32, i32, vp, vp, vp, vp, vp]
         L.orc_round_bf16.argtypes = [creal]
         L.orc_round_bf16.restype = ctypes.c_uint16
         L.orc_rmsnorm.argtypes = [i32, vp, vp, dbl, vp]
@@ -135,6 +143,36 @@ class Oracle:
         assert x.size == K and S.shape == ((N + 127) // 128, (K + 127) // 128)
         y = np.empty(N, dtype=self.real)
         self.lib.orc_gemv_fp8(N, K, _ptr(W), _ptr(S), _ptr(x), _ptr(y))
+        return y
+
+    def e2m1_to_real(self, c: int) -> float:
+        return float(self.lib.orc_e2m1_to_real(c))
+
+    def e8m0_to_real(self, s: int) -> float:
+        return float(self.lib.orc_e8m0_to_real(s))
+
+    def mxfp4_pitch(self, K: int) -> int:
+        return int(self.lib.orc_mxfp4_pitch(K))
+
+    def gemv_mxfp4(self, W_rows, K: int, x):
+        """y = W x for W [N][K] as MXFP4 rows (uint8 [N][mxfp4_pitch(K)])."""
+        W = np.ascontiguousarray(W_rows, dtype=np.uint8)
+        x = self._r(x)
+        N = W.shape[0]
+        assert x.size == K and W.shape[1] == self.mxfp4_pitch(K)
+        y = np.empty(N, dtype=self.real)
+        self.lib.orc_gemv_mxfp4(N, K, _ptr(W), _ptr(x), _ptr(y))
+        return y
+
+    def swiglu_mlp_mxfp4(self, wgate, wup, wdown, hn):
+        """SwiGLU of one FP4 expert: gate / up [F][pitch(d)], down [d][pitch(F)] rows."""
+        wg, wu, wd = (np.ascontiguousarray(a, dtype=np.uint8) for a in (wgate, wup, wdown))
+        F, d = wg.shape[0], wd.shape[0]
+        assert wg.shape == wu.shape == (F, self.mxfp4_pitch(d))
+        assert wd.shape == (d, self.mxfp4_pitch(F))
+        hn = self._r(hn)
+        y = np.empty(d, dtype=self.real)
+        self.lib.orc_swiglu_mlp_mxfp4(d, F, _ptr(wg), _ptr(wu), _ptr(wd), _ptr(hn), _ptr(y))
         return y
 
     def rmsnorm(self, x, g_bf16, eps):
@@ -247,14 +285,17 @@ class Oracle:
                        want_scores: bool = False):
         """One MoE decoder layer: the GQA attention block, then
         x = h1 + sum_i w_i Expert_{idx_i}(hn) + Shared(hn), hn = RMSNorm(h1).
-        `experts(e)` returns routed expert e's (W_gate, W_up, W_down).
+        `experts(e)` returns routed expert e's (W_gate, W_up, W_down): bf16 words, or MXFP4
+        rows when the workload's weight_format is "fp4".
         Returns (x_out, idx, w), and the router's scores of all experts when want_scores."""
         h1 = self.gqa_attn_block(wl, layer, k_cache, v_cache, pos, x)
         hn = self.rmsnorm(h1, layer[5], wl.norm_eps)
         idx, w, scores = self.router_topk(layer[6], hn, wl.top_k)
         y = np.zeros(wl.hidden, dtype=self.real)
+        mlp = self.swiglu_mlp_mxfp4 if getattr(wl, "weight_format", "bf16") == "fp4" \
+            else self.swiglu_mlp
         for i, e in enumerate(idx):
-            y += w[i] * self.swiglu_mlp(*experts(int(e)), hn)
+            y += w[i] * mlp(*experts(int(e)), hn)
         y += self.swiglu_mlp(layer[7], layer[8], layer[9], hn)
         if want_scores:
             return h1 + y, idx, w, scores

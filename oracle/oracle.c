@@ -27,9 +27,15 @@
  * one fp32 scale per 128 x 128 block, decoded from the format's definition and multiplied
  * by the block's scale; activations stay in `real`.
  *
+ * FP4 experts (optional, the routed experts of a MoE layer): MXFP4 rows (OCP Microscaling,
+ * E2M1 elements with one E8M0 scale per 32), decoded from the formats' definitions;
+ * activations stay in `real`.
+ *
  * Pins (tests/test_oracle_pins.py): bf16 rounding vs torch and vs the two neighbours;
  * E4M3 decoding of all 256 bytes vs torch and vs the format's closed values; the FP8
- * matrix-vector product vs numpy on the decoded, scaled matrix;
+ * matrix-vector product vs numpy on the decoded, scaled matrix; E2M1 and E8M0 decoding vs
+ * the formats' value tables, the nibble order on a hand-made row, the MXFP4 product vs
+ * numpy, the FP4-expert MoE layer vs the bf16 one on the decoded weights;
  * RMSNorm unit RMS; matrix-vector vs numpy matmul; RoPE identity at pos 0, norm
  * preservation, relative-position property and the complex-rotation form; attention
  * brute force in pure Python, one position returns V, equal keys return the mean of V,
@@ -127,6 +133,45 @@ void orc_gemv_fp8(int N, int K, const uint8_t* W, const float* S, const real* x,
     const float* srow = S + (size_t)(n / 128) * KB;
     real acc = 0;
     for (int k = 0; k < K; ++k) acc += orc_e4m3_to_real(row[k]) * (real)srow[k / 128] * x[k];
+    y[n] = acc;
+  }
+}
+
+/* FP4 E2M1 (the OCP Microscaling 4-bit float: sign, 2 exponent bits with bias 1, 1 mantissa
+ * bit; no infinities, no NaN) code in the low 4 bits of c -> value.  Exponent field 0 holds
+ * the subnormals m/2 (0 and 0.5); otherwise the value is (1 + m/2) * 2^(e - 1). */
+real orc_e2m1_to_real(uint8_t c) {
+  int sgn = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+  double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return (real)(sgn ? -v : v);
+}
+
+/* E8M0 (the OCP Microscaling shared scale: an unsigned 8-bit exponent with bias 127, no
+ * mantissa) -> 2^(s - 127); 255 is NaN. */
+real orc_e8m0_to_real(uint8_t s) {
+  if (s == 255) return (real)NAN;
+  return (real)ldexp(1.0, (int)s - 127);
+}
+
+/* Bytes of one stored MXFP4 row of K elements: K/2 code bytes, K/32 scale bytes, padded to
+ * a multiple of 16. */
+int orc_mxfp4_pitch(int K) { return (K / 2 + K / 32 + 15) / 16 * 16; }
+
+/* y = W x with W [N][K] stored as MXFP4 rows (OCP Microscaling MXFP4, block size 32) of
+ * orc_mxfp4_pitch(K) bytes: element k of row n is the E2M1 code in the low nibble (k even)
+ * or high nibble (k odd) of byte k / 2, times the E8M0 scale in byte K / 2 + k / 32.  The
+ * pages quantise only the MoE experts to FP4 (Speed is intelligence talk, the MiMo
+ * co-design passage) and name no layout; this is the OCP MXFP4 format. */
+void orc_gemv_mxfp4(int N, int K, const uint8_t* W, const real* x, real* y) {
+  const int pitch = orc_mxfp4_pitch(K);
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n) {
+    const uint8_t* row = W + (size_t)n * pitch;
+    real acc = 0;
+    for (int k = 0; k < K; ++k) {
+      const uint8_t code = (k & 1) ? (uint8_t)(row[k / 2] >> 4) : (uint8_t)(row[k / 2] & 15);
+      acc += orc_e2m1_to_real(code) * orc_e8m0_to_real(row[K / 2 + k / 32]) * x[k];
+    }
     y[n] = acc;
   }
 }
@@ -254,6 +299,20 @@ void orc_swiglu_mlp(int d, int F, const uint16_t* wgate, const uint16_t* wup,
   orc_gemv(F, d, wup, hn, u);
   for (int i = 0; i < F; ++i) g[i] = orc_silu(g[i]) * u[i];
   orc_gemv(d, F, wdown, g, y);
+  free(g);
+  free(u);
+}
+
+/* SwiGLU MLP of one FP4 expert: gate and up rows [F] of d elements, down rows [d] of F
+ * elements, all MXFP4 (orc_gemv_mxfp4). */
+void orc_swiglu_mlp_mxfp4(int d, int F, const uint8_t* wgate, const uint8_t* wup,
+                          const uint8_t* wdown, const real* hn, real* y) {
+  real* g = (real*)malloc(sizeof(real) * F);
+  real* u = (real*)malloc(sizeof(real) * F);
+  orc_gemv_mxfp4(F, d, wgate, hn, g);
+  orc_gemv_mxfp4(F, d, wup, hn, u);
+  for (int i = 0; i < F; ++i) g[i] = orc_silu(g[i]) * u[i];
+  orc_gemv_mxfp4(d, F, wdown, g, y);
   free(g);
   free(u);
 }

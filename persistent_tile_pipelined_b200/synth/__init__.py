@@ -35,6 +35,9 @@ def _lib() -> ctypes.CDLL:
         lib.synth_e4m3_blocks.argtypes = [u64, u64, i64, i64, dbl, ctypes.c_void_p,
                                           ctypes.c_void_p]
         lib.synth_e4m3_blocks.restype = None
+        lib.synth_mxfp4_rows.argtypes = [u64, u64, i64, i64, i64, ctypes.c_int32,
+                                         ctypes.c_void_p]
+        lib.synth_mxfp4_rows.restype = None
         _LIB = lib
     return _LIB
 
@@ -81,6 +84,24 @@ def e4m3_blocks(seed: int, tensor_id: int, shape, std: float):
                                  codes.ctypes.data_as(ctypes.c_void_p),
                                  scales.ctypes.data_as(ctypes.c_void_p))
     return codes, scales
+
+
+def mxfp4_pitch(K: int) -> int:
+    """Bytes per stored MXFP4 row of K elements: K/2 code bytes and K/32 scale bytes,
+    padded to a multiple of 16."""
+    return (K // 2 + K // 32 + 15) // 16 * 16
+
+
+def mxfp4_rows(seed: int, tensor_id: int, N: int, K: int, scale_lo: int = 119) -> np.ndarray:
+    """[N][mxfp4_pitch(K)] bytes of random MXFP4 rows (K a multiple of 32): uniform random
+    E2M1 code bytes, then K/32 scale exponents scale_lo or scale_lo + 1, then zero padding."""
+    N, K = int(N), int(K)
+    assert K % 32 == 0
+    out = np.empty((N, mxfp4_pitch(K)), dtype=np.uint8)
+    if N and K:
+        _lib().synth_mxfp4_rows(seed, tensor_id, N, K, out.shape[1], int(scale_lo),
+                                out.ctypes.data_as(ctypes.c_void_p))
+    return out
 
 
 def u64(seed: int, tensor_id: int, index: int) -> int:

@@ -22,6 +22,11 @@
  *              block = (float)(block max |value| / 448) (1 for an all-zero block), and each
  *              value divided by its block's scale, rounded to the nearest E4M3 number (ties
  *              to even, saturated at +-448) and stored as its E4M3 byte.
+ *   mxfp4 rows bytes of an [N] x pitch matrix of FP4 weight rows (K elements each): the
+ *              row's first K/2 bytes are draws' bytes (byte b of the matrix is byte b % 8
+ *              of draw(b / 8)), the next K/32 bytes are scale exponents lo + (that byte & 1),
+ *              the rest of the row is zero.  Random codes, not a quantised matrix: every
+ *              E2M1 pair (and, with lo = 119, scales of 2^-8 or 2^-7) is equally likely.
  */
 #include <math.h>
 #include <stdint.h>
@@ -154,6 +159,22 @@ void synth_e4m3_blocks(uint64_t seed, uint64_t tensor_id, int64_t N, int64_t K, 
           double v = std * ((i & 1) ? z1 : z0);
           codes[i] = e4m3_rne(v / (double)sc);
         }
+    }
+  }
+}
+
+void synth_mxfp4_rows(uint64_t seed, uint64_t tensor_id, int64_t N, int64_t K, int64_t pitch,
+                      int32_t lo, uint8_t* out) {
+  uint64_t key = stream_key(seed, tensor_id);
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    uint8_t* row = out + n * pitch;
+    for (int64_t j = 0; j < pitch; ++j) {
+      const uint64_t b = (uint64_t)(n * pitch + j);
+      const uint8_t v = (uint8_t)(draw(key, b / 8) >> (8 * (b % 8)));
+      if (j < K / 2) row[j] = v;
+      else if (j < K / 2 + K / 32) row[j] = (uint8_t)(lo + (v & 1));
+      else row[j] = 0;
     }
   }
 }

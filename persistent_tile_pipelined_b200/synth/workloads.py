@@ -14,8 +14,8 @@ from typing import Dict, List, Optional
 
 import numpy as np
 
-from . import (TID_EMBED, TID_FINAL_NORM, TID_LM_HEAD, TID_X_IN, e4m3_blocks, normal_bf16,
-               normal_f32, tid_kcache, tid_layer, tid_vcache, token_id)
+from . import (TID_EMBED, TID_FINAL_NORM, TID_LM_HEAD, TID_X_IN, e4m3_blocks, mxfp4_rows,
+               normal_bf16, normal_f32, tid_kcache, tid_layer, tid_vcache, token_id)
 
 W_STD = 0.02
 GAIN_STD = 0.01
@@ -38,7 +38,8 @@ class Workload:
     norm_eps: float = 1e-5
     tokens_per_step: int = 1
     seed: int = 1234
-    weight_format: str = "bf16"  # "fp8": GQA projections as E4M3 bytes + 128x128 block scales
+    weight_format: str = "bf16"  # "fp8": GQA projections as E4M3 bytes + 128x128 block scales;
+    #                              "fp4": MoE routed experts as MXFP4 rows (E2M1 + E8M0 per 32)
     # MLA sparse attention (0 = dense): index heads, index dim, positions kept per step
     index_heads: int = 0
     index_dim: int = 0
@@ -111,9 +112,13 @@ MLA4_SPARSE128K = MLA4.replace(name="mla-4L-d7168-sparse-kv128k", prefill=131072
                                index_dim=128, index_topk=2048)
 MLA4_KV128K = MLA4.replace(name="mla-4L-d7168-kv128k", prefill=131072)
 
+# The MoE layers with FP4 routed experts (MXFP4 rows: E2M1 codes, one power-of-two scale per
+# 32 weights); attention, router and shared expert stay bf16.
+MOE4_FP4 = MOE4.replace(name="moe-4L-d7168-fp4", weight_format="fp4")
+
 WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, LLAMA8B_4L, MLA4, MOE4, LLAMA8B_KV8K,
                                  LLAMA8B_KV32K, LLAMA8B_KV128K, LLAMA8B_FP8, MLA4_SPARSE128K,
-                                 MLA4_KV128K)}
+                                 MLA4_KV128K, MOE4_FP4)}
 
 
 def gqa_layer_shapes(w: Workload) -> List[tuple]:
@@ -171,8 +176,14 @@ def tid_expert(layer: int, expert: int, which: int) -> int:
 
 
 def gen_expert(w: Workload, layer: int, expert: int) -> tuple:
-    """(W_gate [F][d], W_up [F][d], W_down [d][F]) of one routed expert, on demand."""
+    """(W_gate [F][d], W_up [F][d], W_down [d][F]) of one routed expert, on demand: bf16
+    words N(0, 0.02), or (weight_format "fp4") MXFP4 rows of bytes [F][pitch(d)], [F][pitch(d)],
+    [d][pitch(F)] with scales 2^-8 / 2^-7 (rms about 0.018)."""
     F, d = w.expert_ffn, w.hidden
+    if w.weight_format == "fp4":
+        return (mxfp4_rows(w.seed, tid_expert(layer, expert, 0), F, d),
+                mxfp4_rows(w.seed, tid_expert(layer, expert, 1), F, d),
+                mxfp4_rows(w.seed, tid_expert(layer, expert, 2), d, F))
     return (gen_tensor(w, tid_expert(layer, expert, 0), (F, d), "w"),
             gen_tensor(w, tid_expert(layer, expert, 1), (F, d), "w"),
             gen_tensor(w, tid_expert(layer, expert, 2), (d, F), "w"))
