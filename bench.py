@@ -394,6 +394,10 @@ def workload_step_bytes(wl, pos=None) -> int:
                if wl.kind == "moe" else 3 * wl.ffn * d)
         proj = (Hq + 2 * Hkv) * D * d + d * Hq * D + mlp
         per_layer = proj * 2 + 2 * d * 2
+        if getattr(wl, "weight_format", "bf16") == "fp4":  # the selected experts as MXFP4 rows
+            from persistent_tile_pipelined_b200.synth import mxfp4_pitch
+            Fe = wl.expert_ffn
+            per_layer += wl.top_k * (2 * Fe * mxfp4_pitch(d) + d * mxfp4_pitch(Fe) - 3 * Fe * d * 2)
         if getattr(wl, "weight_format", "bf16") == "fp8":  # E4M3 + a scale per 128x128 block
             def blocks(N, K):
                 return -(-N // 128) * -(-K // 128)
@@ -438,6 +442,8 @@ def layers_config(wl, world: int) -> dict:
     if wl.kind == "moe":
         cfg.update(experts=wl.n_experts, top_k=wl.top_k, shared=wl.n_shared,
                    expert_ffn=wl.expert_ffn, kv_heads=wl.n_kv_heads, head_dim=wl.head_dim)
+        if getattr(wl, "weight_format", "bf16") == "fp4":
+            cfg.update(weights="routed experts MXFP4 (E2M1 + E8M0 scale per 32); the rest bf16")
     if wl.kind == "mla":
         cfg.update(q_lora=wl.q_lora, kv_lora=wl.kv_lora, rope_dim=wl.rope_dim,
                    nope_dim=wl.nope_dim, v_dim=wl.v_dim, latent_positions=wl.prefill)
@@ -853,8 +859,11 @@ def main_layers(args, rank, world, local_rank):
         "metric": LAYERS_METRIC,
         "value": job_throughput(world, K, 1, dev_s), "unit": "steps/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": dev_s / K * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp4e2m1-experts" if wl.weight_format == "fp4" else "bf16",
+        "data": "synthetic (seeded random-init weights N(0,0.02), KV N(0,1))" +
+                ("; routed experts random MXFP4 codes, scales 2^-8 / 2^-7"
+                 if wl.weight_format == "fp4" else ""),
         "config": cfg,
         "hbm_gbs": step_bytes / (dev_s / K) / 1e9,
         "hbm_frac_of_8tbs": step_bytes / (dev_s / K) / 1e9 / NOMINAL_HBM_GBS,

@@ -127,7 +127,8 @@ typedef struct {
                                    (hidden and ffn multiples of 16); 0 = the planner's
                                    choice: tiles at 4 tokens per step when the sizes
                                    allow, else rows                                     */
-  int32_t weight_format;        /* TRE_WEIGHTS_*: storage of the GQA projections        */
+  int32_t weight_format;        /* TRE_WEIGHTS_*: storage of the GQA projections (FP8)
+                                   or of the MoE routed experts (FP4)                   */
   int32_t index_heads;          /* MLA sparse attention (index_topk > 0): H_I index heads,
                                    16, 32 or 64                                         */
   int32_t index_dim;            /* D_I, the index key width: 64 or 128                  */
@@ -154,8 +155,16 @@ typedef struct {
  * stay bf16.  The dequantisation is fused into the weight-streaming GEMV ("RMSNorm + QKV
  * + FP8 dequant", TileRT code audit, fused-op list; fewer bytes per token is the pages'
  * "tokens per byte" lever, Speed is intelligence talk).  Every K must then be a multiple
- * of 16 (16-byte rows).  The E4M3 NaN bytes (S.1111.111) are not decoded as NaN. */
-enum { TRE_WEIGHTS_BF16 = 0, TRE_WEIGHTS_FP8_BLOCK128 = 1 };
+ * of 16 (16-byte rows).  The E4M3 NaN bytes (S.1111.111) are not decoded as NaN.
+ * FP4_EXPERTS (MoE stacks, one token per step): the routed experts' gate, up and down
+ * matrices are MXFP4 rows (the OCP Microscaling MXFP4 format): a row of K weights is K/2
+ * bytes of E2M1 codes (weight k in the low nibble of byte k/2 when k is even, in the high
+ * nibble when odd; E2M1 = sign, 2 exponent bits of bias 1, 1 mantissa bit), then K/32 E8M0
+ * scale bytes (weights [32b, 32b + 32) are scaled by 2^(byte b - 127); byte 255 is NaN),
+ * zero-padded to a pitch of round_up(K/2 + K/32, 16) bytes.  Attention, router and shared
+ * experts stay bf16.  The pages quantise only the MoE experts to FP4 (Speed is intelligence
+ * talk, the MiMo co-design passage).  hidden and expert_ffn must be multiples of 32. */
+enum { TRE_WEIGHTS_BF16 = 0, TRE_WEIGHTS_FP8_BLOCK128 = 1, TRE_WEIGHTS_FP4_EXPERTS = 2 };
 
 /* Per-layer tensor slots.  layer_w[l * TRE_W_SLOTS + slot] is the device pointer of
  * tensor `slot` of layer l (NULL for slots the layer kind does not use).
@@ -165,7 +174,9 @@ enum { TRE_WEIGHTS_BF16 = 0, TRE_WEIGHTS_FP8_BLOCK128 = 1 };
  *         ROUTER[E][d], SHARED_GATE[Fs][d], SHARED_UP[Fs][d], SHARED_DOWN[d][Fs]
  *         (NULL when n_shared == 0), and the routed experts stacked expert-major:
  *         EXPERT_GATE[E][Fe][d], EXPERT_UP[E][Fe][d], EXPERT_DOWN[E][d][Fe]
- *         (the layout of a fused-MoE weight: expert e's matrix starts at e * Fe * d).
+ *         (the layout of a fused-MoE weight: expert e's matrix starts at e * Fe * d);
+ *         FP4_EXPERTS: the same matrices as MXFP4 rows, [E][Fe] rows of pitch(d) bytes
+ *         (gate, up) and [E][d] rows of pitch(Fe) bytes (down).
  *   MLA : ATTN_NORM[d], DQ[QL][d], Q_NORM[QL], UQ[H*(NP+R)][QL] (per head: NP nope rows
  *         then R rope rows), DKV[KL+R][d] (KL latent rows then R rope rows),
  *         KV_NORM[KL], UK[H*NP][KL], UV[H*VD][KL], MLA_O[d][H*VD]

@@ -184,6 +184,8 @@ struct GemvGeom {
   int nstages;
   int nkk;      // tiles (multi-token plans): stages per row tile and segment (k-chunks)
   int esz;      // bytes per weight: 2 (bf16), 1 (E4M3 projections)
+  int rowb;     // bytes of one row of the K-part as stored and copied (MXFP4: the pitch)
+  bool f4;      // MXFP4 rows (FP4 routed experts)
 };
 
 template <bool TILED>
@@ -208,6 +210,8 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   const int len = g.np == 1 ? g.K : gemv_part_len(g.K, g.np, gemv_part_align(TILED, g.esz == 1));
   g.k0 = g.part * len;
   g.Kp = min(len, g.K - g.k0);
+  g.f4 = p.wfp4 && (t.op == OP_RGU || (t.op == OP_MDOWN && g.part >= p.nshared));
+  g.rowb = g.f4 ? fp4_row_pitch(g.Kp) : g.Kp * g.esz;
   if (TILED) {  // row tiles of 16; per tile and segment, k-chunks of kTileK columns
     g.rps = kTileRows;
     g.nkk = (g.Kp + kTileK - 1) / kTileK;
@@ -215,6 +219,7 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   } else {
     // E4M3: one tensor-core tile of 8 rows (gate / up: 4 of each) per stage at most
     g.rps = g.esz == 1 ? min(8 / g.nseg, fp8_rows_per_stage(g.Kp, g.nseg, p.stage_bytes))
+            : g.f4     ? max(1, p.stage_bytes / (g.nseg * g.rowb))
                        : gemv_rows_per_stage(g.Kp, g.nseg, p.stage_bytes, g.esz);
     g.nkk = 1;
     g.nstages = (t.r1 - t.r0 + g.rps - 1) / g.rps;
@@ -226,7 +231,7 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
 // how many rows from n on follow it contiguously in memory (same matrix, row stride = the
 // part length): QKV rows cross from Wq into Wk into Wv, routed rows end at their expert's
 // last row, K-parts of a wider matrix are one row each.  Offsets count weights of g.esz
-// bytes (E4M3 projections: 1).
+// bytes (E4M3 projections: 1); MXFP4 expert rows count whole rows of their pitch.
 __device__ __forceinline__ const uint8_t* wbytes(const uint16_t* w) {
   return reinterpret_cast<const uint8_t*>(w);
 }
@@ -277,7 +282,8 @@ __device__ __forceinline__ const uint8_t* part_row(const Params& p, const Task& 
       const int j = n / p.Fe, r = n - j * p.Fe;
       const int ex = routed_expert(p, t.layer, j, t.id);
       *contig = p.Fe - r;
-      return wbytes(L.w[seg ? TRE_W_EXPERT_UP : TRE_W_EXPERT_GATE]) + ((size_t)ex * p.Fe + r) * K * 2;
+      return wbytes(L.w[seg ? TRE_W_EXPERT_UP : TRE_W_EXPERT_GATE]) +
+             ((size_t)ex * p.Fe + r) * (g.f4 ? (size_t)g.rowb : K * 2);
     }
     default: {  // OP_MDOWN: part < nshared is a column slice of the shared down matrix
       if (g.part < p.nshared) {
@@ -286,7 +292,8 @@ __device__ __forceinline__ const uint8_t* part_row(const Params& p, const Task& 
                ((size_t)n * p.nshared * p.Fe + (size_t)g.part * p.Fe) * 2;
       }
       const int ex = routed_expert(p, t.layer, g.part - p.nshared, t.id);
-      return wbytes(L.w[TRE_W_EXPERT_DOWN]) + ((size_t)ex * p.d + n) * p.Fe * 2;
+      return wbytes(L.w[TRE_W_EXPERT_DOWN]) +
+             ((size_t)ex * p.d + n) * (g.f4 ? (size_t)g.rowb : (size_t)p.Fe * 2);
     }
   }
 }
@@ -390,8 +397,9 @@ __device__ __forceinline__ RowSrc row_src(const Params& p, const Task& t, const 
   RowSrc r;
   r.lookup = t.op == OP_QKV || t.op == OP_MDQKV || (t.op == OP_UQ && p.KI > 0);
   r.stride = (long long)g.K * g.esz;
-  if (t.op == OP_RGU) r.stride = 2LL * p.d;
-  else if (t.op == OP_MDOWN) r.stride = 2LL * (g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe);
+  if (t.op == OP_RGU) r.stride = g.f4 ? (long long)g.rowb : 2LL * p.d;
+  else if (t.op == OP_MDOWN)
+    r.stride = g.f4 ? (long long)g.rowb : 2LL * (g.part < p.nshared ? (long long)p.nshared * p.Fe : p.Fe);
   int contig;
   r.base[2] = nullptr;
   r.split[0] = r.split[1] = 0x7fffffff;
@@ -474,7 +482,7 @@ __device__ __forceinline__ uint32_t stage_total(const Params& p, const Task& t, 
                                                 int t0, int t1, int i) {
   if (t.type == T_GEMV) {
     const int nr = min(g.rps, t.r1 - (t.r0 + i * g.rps));
-    return (uint32_t)(g.nseg * nr * g.Kp * g.esz);
+    return (uint32_t)(g.nseg * nr * g.rowb);
   }
   if constexpr (SP) {
     if (t.type == T_INDEX) return (uint32_t)(p.DI * 2 * kIndexRows);  // whole boxes
@@ -497,7 +505,7 @@ __device__ __forceinline__ void issue_stage(const Params& p, const Task& t, cons
                                             uint8_t* dst, uint64_t* bar, uint64_t pol) {
   if (t.type == T_GEMV) {
     const int n0 = t.r0 + i * g.rps, n1 = min(t.r1, n0 + g.rps);
-    const uint32_t rowb = (uint32_t)g.Kp * (uint32_t)g.esz;
+    const uint32_t rowb = (uint32_t)g.rowb;
     if (g.esz == 1) {  // E4M3 rows: one copy per row, rows at the padded pitch
       const uint32_t pitch = (uint32_t)fp8_row_pitch(g.Kp);
       for (int k = lane; k < g.nseg * (n1 - n0); k += 32) {
@@ -2711,7 +2719,7 @@ __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint
 // MLA = true: the absorbed-MLA stack's kernel (MLA tiles, no GQA attention); false: GQA /
 // MoE.  Separate instantiations keep each kernel's register allocation to its own tiles.
 // TILED: GEMV stages are 16-row tensor-core tiles (multi-token plans).
-template <bool MLA, int MT, bool TILED, bool F8, bool SP>
+template <bool MLA, int MT, bool TILED, bool F8, bool SP, bool F4>
 __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, const uint32_t* tags, float* ub,
                          float* misc) {
@@ -2827,7 +2835,38 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
-        if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+        if (F4 && g.f4) {  // MXFP4 expert rows at their pitch (as the bf16 rows below)
+          const uint8_t* sb = ring + (size_t)slot * p.stage_bytes;
+          const size_t rb = (size_t)g.rowb;
+          if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+            for (int r = 0; r < nr; r += 2) {
+              const int np = min(2, nr - r);
+              const uint8_t* g0 = sb + (size_t)r * rb;
+              const uint8_t* u0 = sb + (size_t)(g.rps + r) * rb;
+              float o0, o1, o2, o3;
+              if (np == 2) gemv_rows_e2m1<4>(g0, g0 + rb, u0, u0 + rb, g.Kp, xl, xh, lane, o0, o1, o2, o3);
+              else gemv_rows_e2m1<2>(g0, u0, u0, u0, g.Kp, xl, xh, lane, o0, o1, o2, o3);
+              const float v = reduce4(o0, o1, o2, o3, lane);
+              const float upv = __shfl_xor_sync(0xffffffffu, v, np == 2 ? 16 : 8);
+              const int k = (lane >> 3) & 1;
+              if ((np == 2 && (lane & 23) == 0) || (np == 1 && lane == 0)) {
+                const float a = v * rn, bb = upv * rn;
+                p.u[uoff + n0 + r + k] = wsel * (a / (1.f + expf(-a)) * bb);
+              }
+            }
+          } else {
+            for (int r = 0; r < nr; r += 4) {
+              const int nv = min(4, nr - r);
+              const uint8_t* r0 = sb + (size_t)r * rb;
+              float o0, o1, o2, o3;
+              gemv_rows_e2m1_n(nv, r0, r0 + (size_t)min(1, nv - 1) * rb, r0 + (size_t)min(2, nv - 1) * rb,
+                               r0 + (size_t)min(3, nv - 1) * rb, g.Kp, xl, xh, lane, o0, o1, o2, o3);
+              const float v = reduce4(o0, o1, o2, o3, lane);
+              const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+              if ((lane & 7) == 0 && idx < nv) gemv_emit<MLA>(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
+            }
+          }
+        } else if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;
           for (int r = 0; r < nr; r += 2) {
             const int np = min(2, nr - r);
@@ -2972,7 +3011,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
 }
 
 // ---- the kernel ----------------------------------------------------------------------------------
-template <bool MLA, int MT, bool TILED, bool F8 = false, bool SP = false>
+template <bool MLA, int MT, bool TILED, bool F8 = false, bool SP = false, bool F4 = false>
 __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t NS = (uint32_t)p.ring_stages;
@@ -3017,17 +3056,20 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
              reinterpret_cast<const volatile int*>(misc + 80), threadIdx.x & 31);
     return;
   }
-  consumer<MLA, MT, TILED, F8, SP>(p, my, ntask, ring, full, empty, tags, ub, misc);
+  consumer<MLA, MT, TILED, F8, SP, F4>(p, my, ntask, ring, full, empty, tags, ub, misc);
 }
 
 // ---- host-side launch helpers ------------------------------------------------------------------
 // The kernel instantiation for a stack kind, a number of tokens per step, the GEMV stage
 // form (tiled: multi-token tensor-core tiles) and the weight format (fp8: E4M3 projections
-// on the tensor cores; their own instantiation keeps the bf16 kernel's registers as they are).
-static const void* kernel_for(bool mla, int m, bool tiled, bool fp8 = false, bool sparse = false) {
+// on the tensor cores; fp4: MXFP4 routed experts; their own instantiations keep the bf16
+// kernel's code and registers as they are).
+static const void* kernel_for(bool mla, int m, bool tiled, bool fp8 = false, bool sparse = false,
+                              bool fp4 = false) {
   if (mla && sparse) return reinterpret_cast<const void*>(engine_kernel<true, 1, false, false, true>);
   if (mla) return reinterpret_cast<const void*>(engine_kernel<true, 1, false>);
   if (fp8) return reinterpret_cast<const void*>(engine_kernel<false, 1, false, true>);
+  if (fp4) return reinterpret_cast<const void*>(engine_kernel<false, 1, false, false, false, true>);
   if (tiled) {
     switch (m) {
       case 2: return reinterpret_cast<const void*>(engine_kernel<false, 2, true>);
@@ -3050,7 +3092,7 @@ static const void* kernel_for(bool mla, int m, bool tiled, bool fp8 = false, boo
 // (never lowered to this plan's need: an engine created later must not shrink what an
 // earlier one launches with).
 cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled,
-                             bool fp8, bool sparse) {
+                             bool fp8, bool sparse, bool fp4) {
   *blocks_per_sm = 1 << 30;
   int dev = 0, optin = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
@@ -3058,8 +3100,8 @@ cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int m
     e0 = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e0 != cudaSuccess) return e0;
   const int limit = optin > smem_bytes ? optin : smem_bytes;
-  for (int m = 1; m <= (mla || fp8 ? 1 : max_m); ++m) {
-    const void* k = kernel_for(mla, m, tiled, fp8, sparse);
+  for (int m = 1; m <= (mla || fp8 || fp4 ? 1 : max_m); ++m) {
+    const void* k = kernel_for(mla, m, tiled, fp8, sparse, fp4);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
     if (e != cudaSuccess) return e;
     int b = 0;
@@ -3086,7 +3128,8 @@ cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_
   cfg.numAttrs = p.op_group >= 0 ? 0 : 1;
   void* args[] = {const_cast<Params*>(&p)};
   const cudaError_t e =
-      cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0, p.wfp8 != 0, p.KI > 0), args);
+      cudaLaunchKernelExC(&cfg, kernel_for(mla, p.m, p.gemv_tiles != 0, p.wfp8 != 0, p.KI > 0, p.wfp4 != 0),
+                          args);
   if (e != cudaSuccess) cudaGetLastError();  // returned here: do not leave it to the caller
   return e;
 }

@@ -22,7 +22,7 @@
 
 namespace tre {
 cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled,
-                             bool fp8 = false, bool sparse = false);
+                             bool fp8 = false, bool sparse = false, bool fp4 = false);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 }  // namespace tre

@@ -86,12 +86,14 @@ struct Builder {
   // task per K-part (only the last part bumps `out`).  `np` > 0 fixes the number of
   // K-parts (else they follow from K).  Returns the number of tasks that bump `out`.
   int esz_proj = 2;  // bytes per weight of the GQA projections (1: E4M3)
+  bool fp4 = false;  // routed experts are MXFP4 rows
 
   int gemv(uint8_t op, int layer, int N, int K, int nseg, int dep, uint32_t dep_count, int out,
            int cap, int np = 0, int cut = 0) {
     if (np <= 0) np = (op == OP_LM || op == OP_ROUTER) ? 1 : gemv_nparts(K, kpart_max);
     const int esz = (op == OP_QKV || op == OP_O || op == OP_GU || op == OP_DOWN) ? esz_proj : 2;
-    auto ranges = assign_rows(N, (int64_t)nseg * K * esz, cum);
+    const int64_t rowb = (fp4 && op == OP_RGU) ? fp4_row_pitch(K) : (int64_t)K * esz;
+    auto ranges = assign_rows(N, (int64_t)nseg * rowb, cum);
     int n = 0;
     for (int s = 0; s < nsm; ++s) {
       for (int r = ranges[s].first; r < ranges[s].second;) {
@@ -199,18 +201,25 @@ struct Builder {
 
   // MoE down: np slots x nb row blocks of d rows, each placed on the SM with the least
   // streamed bytes so far; aux = slot | block << 8.  Returns nb (one bump per block).
+  int nshared = 0;   // MoE: slots below nshared are the shared experts (bf16)
   int moe_down(int layer, int d, int np, int Fe, int nb, int dep, uint32_t dep_count, int out) {
     const std::vector<int> sms = spread(np * nb);
+    // MXFP4 routed slots stream fewer bytes than the bf16 shared ones: the shared slots'
+    // tasks take the least loaded SMs first
+    const bool cheap_routed = fp4 && nshared > 0;
     for (int bl = 0; bl < nb; ++bl) {
       const int r0 = (int)((int64_t)d * bl / nb), r1 = (int)((int64_t)d * (bl + 1) / nb);
       for (int j = 0; j < np; ++j) {
-        const int best = sms[bl * np + j];
+        const int k = !cheap_routed ? bl * np + j
+                      : j < nshared ? bl * nshared + j
+                                    : nb * nshared + bl * (np - nshared) + (j - nshared);
+        const int best = sms[k];
         Task t = make(T_GEMV, OP_MDOWN, layer, dep, dep_count, out);
         t.r0 = r0;
         t.r1 = r1;
         t.aux = j | (bl << 8);
         q[best].push_back(t);
-        cum[best] += (int64_t)(r1 - r0) * Fe * 2;
+        cum[best] += (int64_t)(r1 - r0) * (fp4 && j >= nshared ? fp4_row_pitch(Fe) : Fe * 2);
       }
     }
     return nb;
@@ -307,8 +316,17 @@ static tre_status validate(const tre_config& c) {
     if (c.max_tokens_per_step * (c.n_q_heads / c.n_kv_heads) > 16)
       return fail(TRE_ERR_UNSUPPORTED, "tokens x (q heads per kv head) above 16");
   }
-  if (c.weight_format != TRE_WEIGHTS_BF16 && c.weight_format != TRE_WEIGHTS_FP8_BLOCK128)
+  if (c.weight_format != TRE_WEIGHTS_BF16 && c.weight_format != TRE_WEIGHTS_FP8_BLOCK128 &&
+      c.weight_format != TRE_WEIGHTS_FP4_EXPERTS)
     return fail(TRE_ERR_INVALID_ARG, "unknown weight_format");
+  if (c.weight_format == TRE_WEIGHTS_FP4_EXPERTS) {
+    if (c.kind != TRE_LAYER_MOE)
+      return fail(TRE_ERR_UNSUPPORTED, "FP4 weights are implemented for the routed experts of MoE stacks");
+    if (c.max_tokens_per_step > 1)
+      return fail(TRE_ERR_UNSUPPORTED, "FP4 experts are implemented for one token per step");
+    if (c.hidden % 32 || c.expert_ffn % 32)
+      return fail(TRE_ERR_UNSUPPORTED, "FP4 experts need hidden and expert_ffn multiples of 32");
+  }
   if (c.weight_format == TRE_WEIGHTS_FP8_BLOCK128) {
     if (c.kind != TRE_LAYER_GQA)
       return fail(TRE_ERR_UNSUPPORTED, "FP8 weights are implemented for GQA stacks only");
@@ -411,6 +429,7 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   // (input length, segments, K-part length) of every op the stack uses
   // E4M3 projections (GQA): QKV, O, gate/up and down rows are 1 byte per weight
   s.wfp8 = c.weight_format == TRE_WEIGHTS_FP8_BLOCK128;
+  s.wfp4 = c.weight_format == TRE_WEIGHTS_FP4_EXPERTS;
   const int pesz = s.wfp8 ? 1 : 2;  // bytes per weight of the layer projections
   struct OpShape { int K, nseg, kp, esz; };
   std::vector<OpShape> ops = {{s.d, 1, 0, pesz}, {s.Hq * s.D, 1, 0, pesz}, {s.d, 1, s.d, 2}};
@@ -506,6 +525,8 @@ tre_status plan_build(const tre_config& c, int nsm, int smem_limit, PlanShape* s
   Builder b(nsm);
   b.kpart_max = s.kpart_max;
   b.esz_proj = pesz;
+  b.fp4 = s.wfp4 != 0;
+  b.nshared = s.nshared;
   int prev_down = -1;
   uint32_t prev_down_count = 0;
   for (int l = 0; l < s.L && mla; ++l) {
@@ -688,6 +709,9 @@ int64_t step_bytes(const PlanShape& s, int pos, int m) {
                           : 3LL * s.F * d;
   const int64_t proj = (int64_t)(s.Hq + 2 * s.Hkv) * D * d + d * s.Hq * D + mlp;
   int64_t per_layer = proj * 2 + 2 * d * 2;
+  if (s.wfp4)  // the selected experts' rows are MXFP4 rows instead of bf16
+    per_layer += (int64_t)s.topk * (2LL * s.Fe * fp4_row_pitch(d) + (int64_t)d * fp4_row_pitch(s.Fe) -
+                                    3LL * s.Fe * d * 2);
   if (s.wfp8) {  // E4M3 bytes plus one fp32 scale per 128 x 128 block of every matrix
     auto blocks = [](int64_t N, int64_t K) { return ((N + 127) / 128) * ((K + 127) / 128); };
     const int64_t nq = (int64_t)s.Hq * D, nk = (int64_t)s.Hkv * D;

@@ -3,6 +3,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -113,6 +114,84 @@ __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t v) {
   __half2 hh;
   *reinterpret_cast<__half2_raw*>(&hh) = h;
   return __half22float2(hh);
+}
+
+// ---- MXFP4 rows (FP4 routed experts) --------------------------------------------------------
+// Two E2M1 codes (the low byte of v: the first in the low nibble) -> their values.
+__device__ __forceinline__ float2 e2m1x2_to_f2(uint32_t v) {
+  const __half2_raw h =
+      __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(v & 0xffu), __NV_E2M1);
+  __half2 hh;
+  *reinterpret_cast<__half2_raw*>(&hh) = h;
+  return __half22float2(hh);
+}
+
+// E8M0 scale byte -> 2^(s - 127) (s = 0: 2^-127, a subnormal; s = 255: NaN).
+__device__ __forceinline__ float e8m0_to_f(uint32_t s) {
+  return __uint_as_float(s == 0u ? 0x00400000u : s == 255u ? 0x7fc00000u : s << 23);
+}
+
+// sum_k W[k] x[k] over 8 E2M1 weights (one 32-bit word: weight 2i in the low nibble of
+// byte i) against the x planes a = x[0:4], b = x[4:8] (the bf16 rows' planes).
+__device__ __forceinline__ float dot8_e2m1(uint32_t w, const float4 a, const float4 b) {
+  const float2 p0 = e2m1x2_to_f2(w), p1 = e2m1x2_to_f2(w >> 8);
+  const float2 p2 = e2m1x2_to_f2(w >> 16), p3 = e2m1x2_to_f2(w >> 24);
+  float s = p0.x * a.x;
+  s = fmaf(p0.y, a.y, s);
+  s = fmaf(p1.x, a.z, s);
+  s = fmaf(p1.y, a.w, s);
+  s = fmaf(p2.x, b.x, s);
+  s = fmaf(p2.y, b.y, s);
+  s = fmaf(p3.x, b.z, s);
+  s = fmaf(p3.y, b.w, s);
+  return s;
+}
+
+// One warp computes NR (<= 4) whole MXFP4 rows of Kp weights (Kp a multiple of 32) of a
+// stage: row r's codes are Kp / 2 bytes at rows[r], its scales the Kp / 32 bytes after
+// them.  Lane l takes the 8-weight groups j = l, l + 32, ...: a 32-bit code word, the x
+// planes of the bf16 rows (xl[j] = x[8j:8j+4], xh[j] = x[8j+4:8j+8]) and the scale of
+// group j / 4; each group's 8 products are summed before its scale multiplies them.
+template <int NR>
+__device__ __forceinline__ void gemv_rows_e2m1(const uint8_t* r0, const uint8_t* r1,
+                                               const uint8_t* r2, const uint8_t* r3, int Kp,
+                                               const float4* __restrict__ xl,
+                                               const float4* __restrict__ xh, int lane,
+                                               float& o0, float& o1, float& o2, float& o3) {
+  const uint8_t* rp[4] = {r0, r1, r2, r3};
+  const int K8 = Kp >> 3, half = Kp >> 1;
+  float acc[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) acc[r] = 0.f;
+#pragma unroll 2
+  for (int j = lane; j < K8; j += 32) {
+    const float4 x0 = xl[j], x1 = xh[j];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(rp[r])[j];
+      const float sc = e8m0_to_f(rp[r][half + (j >> 2)]);
+      acc[r] = fmaf(dot8_e2m1(w, x0, x1), sc, acc[r]);
+    }
+  }
+  float out[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) out[r] = r < NR ? acc[r] : 0.f;
+  o0 = out[0];
+  o1 = out[1];
+  o2 = out[2];
+  o3 = out[3];
+}
+
+__device__ __forceinline__ void gemv_rows_e2m1_n(int nr, const uint8_t* r0, const uint8_t* r1,
+                                                 const uint8_t* r2, const uint8_t* r3, int Kp,
+                                                 const float4* xl, const float4* xh, int lane,
+                                                 float& o0, float& o1, float& o2, float& o3) {
+  switch (nr) {
+    case 4: gemv_rows_e2m1<4>(r0, r1, r2, r3, Kp, xl, xh, lane, o0, o1, o2, o3); break;
+    case 3: gemv_rows_e2m1<3>(r0, r1, r2, r3, Kp, xl, xh, lane, o0, o1, o2, o3); break;
+    case 2: gemv_rows_e2m1<2>(r0, r1, r2, r3, Kp, xl, xh, lane, o0, o1, o2, o3); break;
+    default: gemv_rows_e2m1<1>(r0, r1, r2, r3, Kp, xl, xh, lane, o0, o1, o2, o3); break;
+  }
 }
 
 // ---- GEMV for MT tokens: one warp computes NR (<= 4) whole rows against MT input vectors -----

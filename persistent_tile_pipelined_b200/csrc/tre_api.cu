@@ -18,7 +18,7 @@
 
 namespace tre {
 cudaError_t engine_configure(int smem_bytes, int* blocks_per_sm, bool mla, int max_m, bool tiled,
-                             bool fp8 = false, bool sparse = false);
+                             bool fp8 = false, bool sparse = false, bool fp4 = false);
 cudaError_t engine_launch(const Params& p, int grid, int smem_bytes, cudaStream_t stream,
                           bool mla = false);
 const char* last_error_cstr();
@@ -302,7 +302,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
 
   int bps = 0;
   CK(engine_configure(s.smem_bytes, &bps, s.kind == TRE_LAYER_MLA, s.M, s.tiles != 0,
-                      s.wfp8 != 0, s.KI > 0));
+                      s.wfp8 != 0, s.KI > 0, s.wfp4 != 0));
   if (bps < 1) {
     set_error("tre_create: the persistent CTA does not fit on an SM");
     return TRE_ERR_OCCUPANCY;
@@ -498,6 +498,7 @@ TRE_EXPORT tre_status tre_create(const tre_config* cfg, const tre_weights* w, in
   p.hold_next_op = cfg->stream_policy == 1 ? 0 : cfg->stream_policy >= 3 ? cfg->stream_policy - 1 : 1;
   p.gemv_tiles = s.tiles;
   p.wfp8 = s.wfp8;
+  p.wfp4 = s.wfp4;
   p.err = reinterpret_cast<int32_t*>(B + o_err);
   p.abort_flag = reinterpret_cast<volatile int32_t*>(B + o_err + 4);
   p.status_host = e->status_dev;

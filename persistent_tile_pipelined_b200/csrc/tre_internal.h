@@ -71,6 +71,9 @@ TRE_HD inline int fp8_row_pitch(int Kp) { return fp8_span(Kp) + 16; }
 // then one scale per 32 columns: its size in floats (the cross-warp sums follow it)
 TRE_HD inline int fp8_frag_floats(int Kp) { return fp8_span(Kp) + fp8_span(Kp) / 32; }
 constexpr int kFp8RedFloats = 2 * kConsumerWarps * 8;
+// MXFP4 rows (FP4 routed experts): K/2 bytes of E2M1 codes, then K/32 E8M0 scale bytes,
+// padded to a multiple of 16 bytes; rows are stored, copied and staged at this pitch
+TRE_HD inline int fp4_row_pitch(int K) { return (K / 2 + K / 32 + 15) / 16 * 16; }
 TRE_HD inline int fp8_rows_per_stage(int Kp, int nseg, int stage_bytes) {
   const int r = stage_bytes / (nseg * fp8_row_pitch(Kp));
   return r < 1 ? 1 : r;
@@ -173,6 +176,7 @@ struct PlanShape {
   int kpart_max;       // longest input slice of a GEMV task (floats)
   int tiles;           // multi-token plan: GEMV stages are 16-row tensor-core tiles
   int wfp8;            // GQA projections are E4M3 with 128 x 128 block scales
+  int wfp4;            // MoE routed experts are MXFP4 rows
   int u_floats;        // the SwiGLU activation buffer (MoE: shared then routed slices)
   int down_blocks;     // MoE down / MLA output slices: row blocks (each summed by its last
                        // slot or slice to finish)
@@ -267,6 +271,7 @@ struct Params {
                                    // stages, then waits for this SM's publish; 0: no wait
   int gemv_tiles;                  // GEMV stages are 16-row tiles (multi-token plans)
   int wfp8;                        // QKV / O / gate-up / down weights are E4M3 + block scales
+  int wfp4;                        // routed experts' gate / up / down rows are MXFP4
   long long timeout_ns;
   long long pf_window;             // L2 prefetch bytes allowed beyond the ring (0 = off)
 };

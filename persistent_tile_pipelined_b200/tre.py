@@ -26,7 +26,7 @@ TRE_ERR_UNSUPPORTED = -6
 TRE_ERR_BOUNDS = -7
 TRE_ERR_STATE = -8
 TRE_LAYER_GQA, TRE_LAYER_MLA, TRE_LAYER_MOE = 0, 1, 2
-TRE_WEIGHTS_BF16, TRE_WEIGHTS_FP8_BLOCK128 = 0, 1
+TRE_WEIGHTS_BF16, TRE_WEIGHTS_FP8_BLOCK128, TRE_WEIGHTS_FP4_EXPERTS = 0, 1, 2
 TRE_DEBUG_HIDDEN, TRE_DEBUG_TRACE, TRE_DEBUG_FAULT_INJECT, TRE_DEBUG_NO_OVERLAP = 1, 2, 4, 8
 TRE_W_SLOTS = 16
 TRACE_COLS = 8
@@ -299,8 +299,8 @@ def config_from_workload(wl, **overrides) -> tre_config:
     c.rope_theta = wl.rope_theta
     c.norm_eps = wl.norm_eps
     c.has_embed_lm_head = 1 if wl.has_embed_lm_head else 0
-    c.weight_format = TRE_WEIGHTS_FP8_BLOCK128 if getattr(wl, "weight_format", "bf16") == "fp8" \
-        else TRE_WEIGHTS_BF16
+    c.weight_format = {"fp8": TRE_WEIGHTS_FP8_BLOCK128, "fp4": TRE_WEIGHTS_FP4_EXPERTS}.get(
+        getattr(wl, "weight_format", "bf16"), TRE_WEIGHTS_BF16)
     for k, v in overrides.items():
         setattr(c, k, v)
     return c
@@ -332,21 +332,34 @@ def upload_gqa_model(model: dict, device="cuda:0") -> dict:
 def upload_moe_model(wl, model: dict, device="cuda:0", expert_fn=None) -> dict:
     """Copy a host MoE model to device tensors: the non-expert slots as they are, and the
     routed experts of every layer stacked expert-major into slots 10-12 ([E][Fe][d] gate
-    and up, [E][d][Fe] down).  `expert_fn(layer, e)` returns an expert's host tensors
-    (default: the workload's generator, one expert at a time)."""
+    and up, [E][d][Fe] down; FP4 workloads: MXFP4 row bytes [E][Fe][pitch(d)] and
+    [E][d][pitch(Fe)]).  `expert_fn(layer, e)` returns an expert's host tensors (default: the
+    workload's generator, one expert at a time)."""
     import torch
+    from .synth import mxfp4_pitch
     from .synth import workloads as W
     expert_fn = expert_fn or (lambda l, e: W.gen_expert(wl, l, e))
     E, Fe, d = wl.n_experts, wl.expert_ffn, wl.hidden
+    fp4 = getattr(wl, "weight_format", "bf16") == "fp4"
     out = {"layers": [], "k_cache": [], "v_cache": []}
     for l, layer in enumerate(model["layers"]):
         dev = {slot: _dev_tensor(a, device) for slot, a in layer.items()
                if not (slot in (7, 8, 9) and a.size == 0)}
-        g = torch.empty((E, Fe, d), dtype=torch.bfloat16, device=device)
-        u = torch.empty((E, Fe, d), dtype=torch.bfloat16, device=device)
-        dn = torch.empty((E, d, Fe), dtype=torch.bfloat16, device=device)
+        if fp4:
+            g = torch.empty((E, Fe, mxfp4_pitch(d)), dtype=torch.uint8, device=device)
+            u = torch.empty_like(g)
+            dn = torch.empty((E, d, mxfp4_pitch(Fe)), dtype=torch.uint8, device=device)
+        else:
+            g = torch.empty((E, Fe, d), dtype=torch.bfloat16, device=device)
+            u = torch.empty((E, Fe, d), dtype=torch.bfloat16, device=device)
+            dn = torch.empty((E, d, Fe), dtype=torch.bfloat16, device=device)
         for e in range(E):
             eg, eu, ed = expert_fn(l, e)
+            if fp4:
+                for dst, a in ((g[e], eg), (u[e], eu), (dn[e], ed)):
+                    assert a.dtype == np.uint8 and tuple(a.shape) == tuple(dst.shape)
+                    dst.copy_(torch.from_numpy(a))
+                continue
             g[e].copy_(torch.from_numpy(eg.view(np.int16)).view(torch.bfloat16))
             u[e].copy_(torch.from_numpy(eu.view(np.int16)).view(torch.bfloat16))
             dn[e].copy_(torch.from_numpy(ed.view(np.int16)).view(torch.bfloat16))

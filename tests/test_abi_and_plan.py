@@ -593,3 +593,34 @@ def test_fp8_plans():
         import ctypes
         info = tre.tre_plan_info()
         assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status, over
+
+
+def test_fp4_expert_plans():
+    """FP4 routed experts: the same MoE task graph, each selected expert's rows streamed as
+    MXFP4 rows (K/2 code bytes + K/32 scale bytes, 16-byte pitch) while attention, router
+    and shared expert stay bf16; the format is refused where it is not implemented."""
+    from persistent_tile_pipelined_b200.synth import mxfp4_pitch
+    fp4 = W.MOE4_FP4
+    check_plan(fp4, 148)
+    check_plan(MOE_SMALL.replace(weight_format="fp4", hidden=544, expert_ffn=224), 7)
+    check_plan(MOE_SMALL.replace(weight_format="fp4", n_shared=0, top_k=1, expert_ffn=96), 19)
+    info4 = tre.tre_plan_inspect(tre.config_from_workload(fp4))
+    info16 = tre.tre_plan_inspect(tre.config_from_workload(W.MOE4))
+    d, Fe, L, k = fp4.hidden, fp4.expert_ffn, fp4.n_layers, fp4.top_k
+    assert info16.weight_bytes - info4.weight_bytes == L * k * (
+        3 * Fe * d * 2 - 2 * Fe * mxfp4_pitch(d) - d * mxfp4_pitch(Fe))
+    # byte-balanced over the SMs (the bf16 shared-expert down slots take the lighter SMs)
+    assert info4.max_sm_bytes <= 1.1 * info4.min_sm_bytes
+    import ctypes
+    for over, status in [(dict(), tre.TRE_OK),
+                         (dict(kind=tre.TRE_LAYER_GQA), tre.TRE_ERR_UNSUPPORTED),
+                         (dict(max_tokens_per_step=2), tre.TRE_ERR_UNSUPPORTED),
+                         (dict(hidden=528), tre.TRE_ERR_UNSUPPORTED),
+                         (dict(expert_ffn=200), tre.TRE_ERR_UNSUPPORTED)]:
+        cfg = tre.config_from_workload(MOE_SMALL.replace(weight_format="fp4", expert_ffn=224))
+        for kk, v in over.items():
+            setattr(cfg, kk, v)
+        if "kind" in over:
+            cfg.ffn = 512
+        info = tre.tre_plan_info()
+        assert tre.lib.tre_plan_inspect(ctypes.byref(cfg), 148, 232448, ctypes.byref(info)) == status, over

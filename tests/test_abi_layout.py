@@ -18,7 +18,7 @@ CONSTANTS = ["TRE_OK", "TRE_ERR_INVALID_ARG", "TRE_ERR_CUDA", "TRE_ERR_OCCUPANCY
              "TRE_ERR_STATE", "TRE_LAYER_GQA", "TRE_LAYER_MLA", "TRE_LAYER_MOE",
              "TRE_DEBUG_HIDDEN", "TRE_DEBUG_TRACE", "TRE_DEBUG_FAULT_INJECT",
              "TRE_DEBUG_NO_OVERLAP", "TRE_W_SLOTS", "TRE_LAUNCH_PERSISTENT", "TRE_LAUNCH_PER_OP",
-             "TRE_WEIGHTS_BF16", "TRE_WEIGHTS_FP8_BLOCK128"]
+             "TRE_WEIGHTS_BF16", "TRE_WEIGHTS_FP8_BLOCK128", "TRE_WEIGHTS_FP4_EXPERTS"]
 
 
 def probe_source():

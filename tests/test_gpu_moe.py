@@ -158,3 +158,32 @@ def test_moe_full_size_four_layers():
 def test_moe_kernel_per_op_form():
     """Router, shared and routed gate/up, expert down as separate plain launches."""
     run_moe(SMALL, steps=2, mode=tre.TRE_LAUNCH_PER_OP)
+
+
+# FP4 routed experts (MXFP4 rows): hidden and expert_ffn multiples of 32
+SMALL_FP4 = SMALL.replace(name="moe-small-fp4", weight_format="fp4", expert_ffn=224)
+
+
+@pytest.mark.parametrize("over,steps,cfg", [
+    (dict(), 3, {}),                                                        # E 12, top 3
+    (dict(hidden=1024, n_q_heads=16, n_kv_heads=2, head_dim=128, n_experts=40, top_k=8,
+          expert_ffn=256, n_layers=1), 2, {}),                              # top 8, d 1024
+    (dict(n_shared=0, top_k=1, expert_ffn=96), 2, {}),                      # routed only
+    (dict(n_shared=2, expert_ffn=64), 2, {}),                               # strided shared parts
+    (dict(), 2, dict(num_sms=3, ring_stages=2, stage_bytes=16384)),        # few SMs, small ring
+    (dict(prefill=0, decode_steps=2), 2, {}),                               # pos 0
+], ids=["e12-k3", "e40-k8-d1024", "no-shared-k1", "two-shared", "sms3-ring2-16k", "pos0"])
+def test_moe_fp4_expert_layers(over, steps, cfg):
+    """MXFP4 routed experts against the oracle's MXFP4 definition, with the bf16 bars."""
+    run_moe(SMALL_FP4.replace(**over), steps=steps, **cfg)
+
+
+def test_moe_fp4_kernel_per_op_form():
+    run_moe(SMALL_FP4, steps=2, mode=tre.TRE_LAUNCH_PER_OP)
+
+
+@pytest.mark.slow
+def test_moe_fp4_full_size_two_layers():
+    """The full MoE layer shapes with FP4 routed experts (hidden 7168, 256 experts top 8 + 1
+    shared, Fe 2048, 4096 cached positions), 2 layers, 2 steps."""
+    run_moe(W.MOE4_FP4.replace(n_layers=2, decode_steps=2), steps=2, materialize=False)
