@@ -126,6 +126,13 @@ __device__ __forceinline__ float2 e2m1x2_to_f2(uint32_t v) {
   return __half22float2(hh);
 }
 
+// Two E2M1 codes (the low byte of v) -> an f16x2 word, the first code in the low half.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2bits(uint32_t v) {
+  const __half2_raw h =
+      __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(v & 0xffu), __NV_E2M1);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
 // E8M0 scale byte -> 2^(s - 127) (s = 0: 2^-127, a subnormal; s = 255: NaN).
 __device__ __forceinline__ float e8m0_to_f(uint32_t s) {
   return __uint_as_float(s == 0u ? 0x00400000u : s == 255u ? 0x7fc00000u : s << 23);
@@ -136,42 +143,55 @@ __device__ __forceinline__ float e8m0_to_f(uint32_t s) {
 __device__ __forceinline__ float dot8_e2m1(uint32_t w, const float4 a, const float4 b) {
   const float2 p0 = e2m1x2_to_f2(w), p1 = e2m1x2_to_f2(w >> 8);
   const float2 p2 = e2m1x2_to_f2(w >> 16), p3 = e2m1x2_to_f2(w >> 24);
-  float s = p0.x * a.x;
-  s = fmaf(p0.y, a.y, s);
-  s = fmaf(p1.x, a.z, s);
-  s = fmaf(p1.y, a.w, s);
-  s = fmaf(p2.x, b.x, s);
-  s = fmaf(p2.y, b.y, s);
-  s = fmaf(p3.x, b.z, s);
-  s = fmaf(p3.y, b.w, s);
-  return s;
+  float s0 = p0.x * a.x, s1 = p0.y * a.y;  // two chains of four
+  s0 = fmaf(p1.x, a.z, s0);
+  s1 = fmaf(p1.y, a.w, s1);
+  s0 = fmaf(p2.x, b.x, s0);
+  s1 = fmaf(p2.y, b.y, s1);
+  s0 = fmaf(p3.x, b.z, s0);
+  s1 = fmaf(p3.y, b.w, s1);
+  return s0 + s1;
 }
 
 // One warp computes NR (<= 4) whole MXFP4 rows of Kp weights (Kp a multiple of 32) of a
 // stage: row r's codes are Kp / 2 bytes at rows[r], its scales the Kp / 32 bytes after
 // them.  Lane l takes the 8-weight groups j = l, l + 32, ...: a 32-bit code word, the x
 // planes of the bf16 rows (xl[j] = x[8j:8j+4], xh[j] = x[8j+4:8j+8]) and the scale of
-// group j / 4; each group's 8 products are summed before its scale multiplies them.
+// group j / 4; each group's 8 products are summed before its scale multiplies them.  Two
+// groups per lane at a time, every shared-memory load issued before the products, so
+// that a warp keeps NR x 2 independent decode + product chains in flight.
 template <int NR>
 __device__ __forceinline__ void gemv_rows_e2m1(const uint8_t* r0, const uint8_t* r1,
                                                const uint8_t* r2, const uint8_t* r3, int Kp,
                                                const float4* __restrict__ xl,
                                                const float4* __restrict__ xh, int lane,
                                                float& o0, float& o1, float& o2, float& o3) {
+  constexpr int U = 2;
   const uint8_t* rp[4] = {r0, r1, r2, r3};
   const int K8 = Kp >> 3, half = Kp >> 1;
   float acc[NR];
 #pragma unroll
   for (int r = 0; r < NR; ++r) acc[r] = 0.f;
-#pragma unroll 2
-  for (int j = lane; j < K8; j += 32) {
-    const float4 x0 = xl[j], x1 = xh[j];
+  for (int j0 = lane; j0 < K8; j0 += 32 * U) {
+    uint32_t w[U][NR];
+    float sc[U][NR];
+    float4 x0[U], x1[U];
 #pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      const uint32_t w = reinterpret_cast<const uint32_t*>(rp[r])[j];
-      const float sc = e8m0_to_f(rp[r][half + (j >> 2)]);
-      acc[r] = fmaf(dot8_e2m1(w, x0, x1), sc, acc[r]);
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + 32 * u;
+      const int jj = j < K8 ? j : j0;  // in range; a group past the row counts nothing
+      x0[u] = xl[jj];
+      x1[u] = xh[jj];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        w[u][r] = reinterpret_cast<const uint32_t*>(rp[r])[jj];
+        sc[u][r] = j < K8 ? e8m0_to_f(rp[r][half + (jj >> 2)]) : 0.f;
+      }
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int r = 0; r < NR; ++r) acc[r] = fmaf(dot8_e2m1(w[u][r], x0[u], x1[u]), sc[u][r], acc[r]);
   }
   float out[4];
 #pragma unroll
