@@ -2622,109 +2622,6 @@ __device__ __forceinline__ void gemv_tile_task(const Params& p, const Task& t, c
 // 128-column block).  All 8 warps share each stage, warp w taking the chunks w, w + 8, ...;
 // the lanes of a row and then the warps are summed (shuffles, shared memory), and one thread
 // per row finishes it.
-// ---- FP4 routed experts on the tensor cores ---------------------------------------------------
-// The input of an MXFP4 expert GEMV as the B operand of mma.sync m16n8k16 f16.  Per 32-column
-// block c, B column 0 / 1 holds the f16 hi / lo parts of x[32c, 32c + 16) and column 2 / 3
-// those of x[32c + 16, 32c + 32) (x = hi + lo to about 22 significant bits); the 16 lanes
-// L = 4 g + t4 (g < 4) that hold them keep 8 bytes each: (x[k], x[k + 1]) and
-// (x[k + 8], x[k + 9]), k = 32c + 16 (g >> 1) + 2 t4, hi for even g, lo for odd.  Lanes 0-7's
-// entries take the place of the block's 64 bytes of the xl plane, lanes 8-15's those of
-// its xh plane, so the fp32 planes of load_input() turn into this operand block by block.
-__device__ __forceinline__ uint32_t fp4_bfrag_off(int c, int L, int Kp) {  // bytes from ub
-  return L < 8 ? (uint32_t)(64 * c + 8 * L) : (uint32_t)(2 * Kp + 64 * c + 8 * (L - 8));
-}
-
-// In place, every consumer thread: 8 lanes of a warp per block read its 32 inputs, the
-// warp synchronises, then they write the block's 16 entries.  An input outside the f16
-// range records a bounds error (its product would be lost).
-__device__ void fp4_bplane(const Params& p, const Task& t, float* ub, int Kp, int ctid) {
-  const int nblk = Kp >> 5, lane = ctid & 31, warp = ctid >> 5;
-  const int slot = lane >> 3, h = (lane >> 2) & 1, t4 = lane & 3;
-  uint8_t* base = reinterpret_cast<uint8_t*>(ub);
-  for (int c0 = warp * 4; c0 < nblk; c0 += kConsumerWarps * 4) {  // uniform in the warp
-    const int c = c0 + slot;
-    const bool live = c < nblk;
-    float2 a = make_float2(0.f, 0.f), b = a;
-    if (live) {
-      const int j = 4 * c + 2 * h, e = 2 * t4;  // x[k]: group j, element e (k + 8: group j + 1)
-      const float* pl = e < 4 ? ub : ub + Kp / 2;
-      a = *reinterpret_cast<const float2*>(pl + 4 * j + (e & 3));
-      b = *reinterpret_cast<const float2*>(pl + 4 * (j + 1) + (e & 3));
-    }
-    __syncwarp();
-    if (live) {
-      const __half2 ha = __floats2half2_rn(a.x, a.y), hb = __floats2half2_rn(b.x, b.y);
-      const float2 ra = __half22float2(ha), rb = __half22float2(hb);
-      const __half2 la = __floats2half2_rn(a.x - ra.x, a.y - ra.y);
-      const __half2 lb = __floats2half2_rn(b.x - rb.x, b.y - rb.y);
-      if (!(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))) < 65504.f))
-        record_error(p, TRE_ERR_BOUNDS, t.id);
-      const int Lh = 8 * h + t4;
-      *reinterpret_cast<uint2*>(base + fp4_bfrag_off(c, Lh, Kp)) =
-          make_uint2(*reinterpret_cast<const uint32_t*>(&ha), *reinterpret_cast<const uint32_t*>(&hb));
-      *reinterpret_cast<uint2*>(base + fp4_bfrag_off(c, Lh + 4, Kp)) =
-          make_uint2(*reinterpret_cast<const uint32_t*>(&la), *reinterpret_cast<const uint32_t*>(&lb));
-    }
-  }
-}
-
-// One warp computes the rows of one MXFP4 stage in tiles of 8 (gate / up: 4 rows of each),
-// one m16n8k16 per 32-column block c: A rows 0-7 are the tile's rows at columns
-// [32c, 32c + 16), rows 8-15 the same rows at [32c + 16, 32c + 32), decoded from the stage
-// (lane (g, t4) takes byte t4 of each 32-bit word of row g's 16-byte chunk c: exact E2M1 ->
-// f16 pairs); B is the operand above.  Lane (g, 0) then holds row g's first-half dot
-// (columns 0 + 1), lane (g, 1) its second half (columns 2 + 3); the block's E8M0 scale
-// multiplies each before it is added up.
-template <bool MLA>
-__device__ __forceinline__ void fp4_stage(const Params& p, const Task& t, const GemvGeom& g,
-                                          const uint8_t* sb, int n0, int nr, const uint8_t* bpl,
-                                          float rn, float wsel, int uoff, const float* resid,
-                                          int lane, Best& best) {
-  const bool two = g.nseg == 2;
-  const int gq = lane >> 2, t4 = lane & 3, nblk = g.Kp >> 5, half = g.Kp >> 1;
-  const uint32_t sh = 8u * (uint32_t)t4;
-  const bool bl = lane < 16;
-  for (int q = 0; q < nr; q += two ? 4 : 8) {
-    const int sr = two ? (gq >= 4 ? g.rps : 0) + min(q + (gq & 3), nr - 1) : min(q + gq, nr - 1);
-    const uint8_t* arow = sb + (size_t)sr * g.rowb;
-    float acc = 0.f;
-    constexpr int U = 4;
-    for (int c0 = 0; c0 < nblk; c0 += U) {
-      uint4 a[U];
-      uint2 b[U];
-      uint32_t s8[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c = min(c0 + u, nblk - 1);  // in range; blocks past the row count nothing
-        a[u] = *reinterpret_cast<const uint4*>(arow + 16 * c);
-        b[u] = bl ? *reinterpret_cast<const uint2*>(bpl + fp4_bfrag_off(c, lane, g.Kp)) : make_uint2(0u, 0u);
-        s8[u] = arow[half + c];
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (c0 + u < nblk) {
-          const uint32_t af[4] = {e2m1x2_to_h2bits(a[u].x >> sh), e2m1x2_to_h2bits(a[u].z >> sh),
-                                  e2m1x2_to_h2bits(a[u].y >> sh), e2m1x2_to_h2bits(a[u].w >> sh)};
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_f16(d, af, b[u].x, b[u].y);
-          const float v = t4 == 0 ? d[0] + d[1] : t4 == 1 ? d[2] + d[3] : 0.f;
-          acc = fmaf(v, e8m0_to_f(s8[u]), acc);
-        }
-      }
-    }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);  // lanes (g, 0) and (g, 1): row g's dot
-    if (two) {
-      const float upv = __shfl_down_sync(0xffffffffu, acc, 16);  // up row: lane (g + 4, 0)
-      if (t4 == 0 && gq < 4 && q + gq < nr) {
-        const float aa = acc * rn, bb = upv * rn;
-        p.u[uoff + n0 + q + gq] = wsel * (aa / (1.f + expf(-aa)) * bb);
-      }
-    } else if (t4 == 0 && q + gq < nr) {
-      gemv_emit<MLA>(p, t, g, n0 + q + gq, acc, rn, resid, best);
-    }
-  }
-}
-
 __device__ void fp8_task(const Params& p, const Task& t, const GemvGeom& g, uint32_t gs, int ns,
                          uint8_t* ring, uint64_t* full, uint64_t* empty, const uint32_t* tags,
                          float* ub, const float* resid, float rn, float wsel, int uoff, int warp,
@@ -2875,9 +2772,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         uk_task(p, t, gemv_geom<false>(p, t), gs, ns, ring, full, empty, tags, ub, red, warp, lane, ctid, ab);
     } else {
       const GemvGeom g = gemv_geom<TILED>(p, t);
-      // MXFP4 tasks keep their input as the tensor-core operand (fp4_bplane): its own key
-      const int key0 = input_key(t);
-      const int key = F4 && g.f4 && key0 >= 0 ? key0 | (1 << 30) : key0;
+      const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
       const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MO;
       if (has_resid) prefetch_resid<MT>(p, t, g, resid, ctid);
@@ -2898,12 +2793,6 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         if (ctid == 0)
 #pragma unroll
           for (int v = 0; v < MT; ++v) rn_s[v] = rnv[v];
-        if constexpr (F4) {
-          if (g.f4) {
-            consumer_sync(kConsumerThreads);
-            fp4_bplane(p, t, ub, g.Kp, ctid);
-          }
-        }
         cur_key = key;
       }
       consumer_sync(kConsumerThreads);
@@ -2946,9 +2835,37 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
         }
         const int n0 = t.r0 + i * g.rps, nr = min(g.rps, t.r1 - n0);
         const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)slot * p.stage_bytes);
-        if (F4 && g.f4) {  // MXFP4 expert rows at their pitch: tensor-core tiles of 8 rows
-          fp4_stage<MLA>(p, t, g, ring + (size_t)slot * p.stage_bytes, n0, nr,
-                         reinterpret_cast<const uint8_t*>(ub), rn, wsel, uoff, resid, lane, best[0]);
+        if (F4 && g.f4) {  // MXFP4 expert rows at their pitch (as the bf16 rows below)
+          const uint8_t* sb = ring + (size_t)slot * p.stage_bytes;
+          const size_t rb = (size_t)g.rowb;
+          if (g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
+            for (int r = 0; r < nr; r += 2) {
+              const int np = min(2, nr - r);
+              const uint8_t* g0 = sb + (size_t)r * rb;
+              const uint8_t* u0 = sb + (size_t)(g.rps + r) * rb;
+              float o0, o1, o2, o3;
+              if (np == 2) gemv_rows_e2m1<4>(g0, g0 + rb, u0, u0 + rb, g.Kp, xl, xh, lane, o0, o1, o2, o3);
+              else gemv_rows_e2m1<2>(g0, u0, u0, u0, g.Kp, xl, xh, lane, o0, o1, o2, o3);
+              const float v = reduce4(o0, o1, o2, o3, lane);
+              const float upv = __shfl_xor_sync(0xffffffffu, v, np == 2 ? 16 : 8);
+              const int k = (lane >> 3) & 1;
+              if ((np == 2 && (lane & 23) == 0) || (np == 1 && lane == 0)) {
+                const float a = v * rn, bb = upv * rn;
+                p.u[uoff + n0 + r + k] = wsel * (a / (1.f + expf(-a)) * bb);
+              }
+            }
+          } else {
+            for (int r = 0; r < nr; r += 4) {
+              const int nv = min(4, nr - r);
+              const uint8_t* r0 = sb + (size_t)r * rb;
+              float o0, o1, o2, o3;
+              gemv_rows_e2m1_n(nv, r0, r0 + (size_t)min(1, nv - 1) * rb, r0 + (size_t)min(2, nv - 1) * rb,
+                               r0 + (size_t)min(3, nv - 1) * rb, g.Kp, xl, xh, lane, o0, o1, o2, o3);
+              const float v = reduce4(o0, o1, o2, o3, lane);
+              const int idx = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+              if ((lane & 7) == 0 && idx < nv) gemv_emit<MLA>(p, t, g, n0 + r + idx, v, rn, resid, best[0]);
+            }
+          }
         } else if (MT == 1 && g.nseg == 2) {  // gate rows [0, nr), up rows at +rps rows
           const uint4* up = sp + (size_t)g.rps * K8;
           for (int r = 0; r < nr; r += 2) {

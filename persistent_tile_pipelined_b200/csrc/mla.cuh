@@ -49,16 +49,6 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// d += a * b for one 16x8x16 tile of f16 operands (fp32 accumulate; fragments as mma_bf16).
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                        uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // d = a * b for one 16x8x32 tile of E4M3 operands (A row-major 16x32, B column-major 32x8,
 // fp32 D): thread (g, t4) holds A bytes (row g, k 4 t4 .. + 3), (row g + 8, same k),
 // (row g, k 16 + 4 t4 ..), (row g + 8, ...) and B bytes (k 4 t4 .., n = g), (k 16 + 4 t4 ..).

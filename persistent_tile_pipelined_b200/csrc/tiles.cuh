@@ -3,7 +3,6 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -117,20 +116,20 @@ __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t v) {
 }
 
 // ---- MXFP4 rows (FP4 routed experts) --------------------------------------------------------
-// Two E2M1 codes (the low byte of v: the first in the low nibble) -> their values.
-__device__ __forceinline__ float2 e2m1x2_to_f2(uint32_t v) {
-  const __half2_raw h =
-      __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(v & 0xffu), __NV_E2M1);
-  __half2 hh;
-  *reinterpret_cast<__half2_raw*>(&hh) = h;
-  return __half22float2(hh);
+// Eight E2M1 codes (a 32-bit word, code 2i in the low nibble of byte i) -> four f16x2 words,
+// the first code of each byte in the low half: the sm_100a conversion instruction, exact
+// (CUDA's header helper falls back to a software conversion for arch-specific targets).
+__device__ __forceinline__ void e2m1x8_to_h2bits(uint32_t w, uint32_t (&h)[4]) {
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(w));
 }
 
-// Two E2M1 codes (the low byte of v) -> an f16x2 word, the first code in the low half.
-__device__ __forceinline__ uint32_t e2m1x2_to_h2bits(uint32_t v) {
-  const __half2_raw h =
-      __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(v & 0xffu), __NV_E2M1);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+__device__ __forceinline__ float2 h2bits_to_f2(uint32_t v) {
+  __half2 hh;
+  *reinterpret_cast<uint32_t*>(&hh) = v;
+  return __half22float2(hh);
 }
 
 // E8M0 scale byte -> 2^(s - 127) (s = 0: 2^-127, a subnormal; s = 255: NaN).
@@ -141,8 +140,10 @@ __device__ __forceinline__ float e8m0_to_f(uint32_t s) {
 // sum_k W[k] x[k] over 8 E2M1 weights (one 32-bit word: weight 2i in the low nibble of
 // byte i) against the x planes a = x[0:4], b = x[4:8] (the bf16 rows' planes).
 __device__ __forceinline__ float dot8_e2m1(uint32_t w, const float4 a, const float4 b) {
-  const float2 p0 = e2m1x2_to_f2(w), p1 = e2m1x2_to_f2(w >> 8);
-  const float2 p2 = e2m1x2_to_f2(w >> 16), p3 = e2m1x2_to_f2(w >> 24);
+  uint32_t h[4];
+  e2m1x8_to_h2bits(w, h);
+  const float2 p0 = h2bits_to_f2(h[0]), p1 = h2bits_to_f2(h[1]);
+  const float2 p2 = h2bits_to_f2(h[2]), p3 = h2bits_to_f2(h[3]);
   float s0 = p0.x * a.x, s1 = p0.y * a.y;  // two chains of four
   s0 = fmaf(p1.x, a.z, s0);
   s1 = fmaf(p1.y, a.w, s1);
