@@ -3,6 +3,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 
@@ -116,19 +117,12 @@ __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t v) {
 }
 
 // ---- MXFP4 rows (FP4 routed experts) --------------------------------------------------------
-// Eight E2M1 codes (a 32-bit word, code 2i in the low nibble of byte i) -> four f16x2 words,
-// the first code of each byte in the low half: the sm_100a conversion instruction, exact
-// (CUDA's header helper falls back to a software conversion for arch-specific targets).
-__device__ __forceinline__ void e2m1x8_to_h2bits(uint32_t w, uint32_t (&h)[4]) {
-  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
-      " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
-      " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(w));
-}
-
-__device__ __forceinline__ float2 h2bits_to_f2(uint32_t v) {
+// Two E2M1 codes (the low byte of v: the first in the low nibble) -> their values.
+__device__ __forceinline__ float2 e2m1x2_to_f2(uint32_t v) {
+  const __half2_raw h =
+      __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(v & 0xffu), __NV_E2M1);
   __half2 hh;
-  *reinterpret_cast<uint32_t*>(&hh) = v;
+  *reinterpret_cast<__half2_raw*>(&hh) = h;
   return __half22float2(hh);
 }
 
@@ -140,59 +134,44 @@ __device__ __forceinline__ float e8m0_to_f(uint32_t s) {
 // sum_k W[k] x[k] over 8 E2M1 weights (one 32-bit word: weight 2i in the low nibble of
 // byte i) against the x planes a = x[0:4], b = x[4:8] (the bf16 rows' planes).
 __device__ __forceinline__ float dot8_e2m1(uint32_t w, const float4 a, const float4 b) {
-  uint32_t h[4];
-  e2m1x8_to_h2bits(w, h);
-  const float2 p0 = h2bits_to_f2(h[0]), p1 = h2bits_to_f2(h[1]);
-  const float2 p2 = h2bits_to_f2(h[2]), p3 = h2bits_to_f2(h[3]);
-  float s0 = p0.x * a.x, s1 = p0.y * a.y;  // two chains of four
-  s0 = fmaf(p1.x, a.z, s0);
-  s1 = fmaf(p1.y, a.w, s1);
-  s0 = fmaf(p2.x, b.x, s0);
-  s1 = fmaf(p2.y, b.y, s1);
-  s0 = fmaf(p3.x, b.z, s0);
-  s1 = fmaf(p3.y, b.w, s1);
-  return s0 + s1;
+  const float2 p0 = e2m1x2_to_f2(w), p1 = e2m1x2_to_f2(w >> 8);
+  const float2 p2 = e2m1x2_to_f2(w >> 16), p3 = e2m1x2_to_f2(w >> 24);
+  float s = p0.x * a.x;
+  s = fmaf(p0.y, a.y, s);
+  s = fmaf(p1.x, a.z, s);
+  s = fmaf(p1.y, a.w, s);
+  s = fmaf(p2.x, b.x, s);
+  s = fmaf(p2.y, b.y, s);
+  s = fmaf(p3.x, b.z, s);
+  s = fmaf(p3.y, b.w, s);
+  return s;
 }
 
 // One warp computes NR (<= 4) whole MXFP4 rows of Kp weights (Kp a multiple of 32) of a
 // stage: row r's codes are Kp / 2 bytes at rows[r], its scales the Kp / 32 bytes after
 // them.  Lane l takes the 8-weight groups j = l, l + 32, ...: a 32-bit code word, the x
 // planes of the bf16 rows (xl[j] = x[8j:8j+4], xh[j] = x[8j+4:8j+8]) and the scale of
-// group j / 4; each group's 8 products are summed before its scale multiplies them.  Two
-// groups per lane at a time, every shared-memory load issued before the products, so
-// that a warp keeps NR x 2 independent decode + product chains in flight.
+// group j / 4; each group's 8 products are summed before its scale multiplies them.
 template <int NR>
 __device__ __forceinline__ void gemv_rows_e2m1(const uint8_t* r0, const uint8_t* r1,
                                                const uint8_t* r2, const uint8_t* r3, int Kp,
                                                const float4* __restrict__ xl,
                                                const float4* __restrict__ xh, int lane,
                                                float& o0, float& o1, float& o2, float& o3) {
-  constexpr int U = 2;
   const uint8_t* rp[4] = {r0, r1, r2, r3};
   const int K8 = Kp >> 3, half = Kp >> 1;
   float acc[NR];
 #pragma unroll
   for (int r = 0; r < NR; ++r) acc[r] = 0.f;
-  for (int j0 = lane; j0 < K8; j0 += 32 * U) {
-    uint32_t w[U][NR];
-    float sc[U][NR];
-    float4 x0[U], x1[U];
+#pragma unroll 2
+  for (int j = lane; j < K8; j += 32) {
+    const float4 x0 = xl[j], x1 = xh[j];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int j = j0 + 32 * u;
-      const int jj = j < K8 ? j : j0;  // in range; a group past the row counts nothing
-      x0[u] = xl[jj];
-      x1[u] = xh[jj];
-#pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        w[u][r] = reinterpret_cast<const uint32_t*>(rp[r])[jj];
-        sc[u][r] = j < K8 ? e8m0_to_f(rp[r][half + (jj >> 2)]) : 0.f;
-      }
+    for (int r = 0; r < NR; ++r) {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(rp[r])[j];
+      const float sc = e8m0_to_f(rp[r][half + (j >> 2)]);
+      acc[r] = fmaf(dot8_e2m1(w, x0, x1), sc, acc[r]);
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int r = 0; r < NR; ++r) acc[r] = fmaf(dot8_e2m1(w[u][r], x0[u], x1[u]), sc[u][r], acc[r]);
   }
   float out[4];
 #pragma unroll
