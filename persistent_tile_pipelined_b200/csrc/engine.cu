@@ -188,7 +188,8 @@ struct GemvGeom {
   bool f4;      // MXFP4 rows (FP4 routed experts)
 };
 
-template <bool TILED>
+// F4: the FP4-expert kernel (only its tasks can be MXFP4 rows; the other kernels fold f4 away)
+template <bool TILED, bool F4 = false>
 __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   GemvGeom g;
   g.K = gemv_K(p, t.op);
@@ -210,7 +211,7 @@ __device__ __forceinline__ GemvGeom gemv_geom(const Params& p, const Task& t) {
   const int len = g.np == 1 ? g.K : gemv_part_len(g.K, g.np, gemv_part_align(TILED, g.esz == 1));
   g.k0 = g.part * len;
   g.Kp = min(len, g.K - g.k0);
-  g.f4 = p.wfp4 && (t.op == OP_RGU || (t.op == OP_MDOWN && g.part >= p.nshared));
+  g.f4 = F4 && p.wfp4 && (t.op == OP_RGU || (t.op == OP_MDOWN && g.part >= p.nshared));
   g.rowb = g.f4 ? fp4_row_pitch(g.Kp) : g.Kp * g.esz;
   if (TILED) {  // row tiles of 16; per tile and segment, k-chunks of kTileK columns
     g.rps = kTileRows;
@@ -370,9 +371,9 @@ __device__ __forceinline__ void attn_range(const Params& p, const Task& t, int& 
   t1 = (int)(P * (sp + 1) / S);
 }
 
-template <bool TILED>
+template <bool TILED, bool F4 = false>
 __device__ __forceinline__ int task_nstages(const Params& p, const Task& t) {
-  if (t.type == T_GEMV) return gemv_geom<TILED>(p, t).nstages;
+  if (t.type == T_GEMV) return gemv_geom<TILED, F4>(p, t).nstages;
   if (t.type == T_ISEL) return 0;
   int t0, t1;
   attn_range(p, t, t0, t1);
@@ -667,7 +668,7 @@ __device__ __forceinline__ bool hold_for_consumers(const Params& p, const volati
   return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
 }
 
-template <bool TILED, bool MLA, bool SP>
+template <bool TILED, bool MLA, bool SP, bool F4 = false>
 __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ring,
                          uint64_t* full, uint64_t* empty, uint32_t* tags,
                          const volatile int* done, int lane) {
@@ -709,12 +710,12 @@ __device__ void producer(const Params& p, const Task* my, int ntask, uint8_t* ri
       __syncwarp();  // orders the other lanes' reads of the selection after lane 0's acquire
     }
     if (window > 0 && ti + 1 < ntask) task_prefetch(p, my[ti + 1], lane, window);
-    const int ns = task_nstages<TILED>(p, t);
+    const int ns = task_nstages<TILED, F4>(p, t);
     GemvGeom g{};
     RowSrc rs{};
     int t0 = 0, t1 = 0;
     if (t.type == T_GEMV) {
-      g = gemv_geom<TILED>(p, t);
+      g = gemv_geom<TILED, F4>(p, t);
       rs = row_src(p, t, g);
     } else {
       attn_range(p, t, t0, t1);
@@ -2735,7 +2736,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     const Task t = my[ti];
     // stage count before the dependency wait (off the hand-off's critical path), except for
     // tasks whose stages follow this step's sparse selection
-    const int ns_early = (MLA && t.type == T_MLA_ATTN) ? -1 : task_nstages<TILED>(p, t);
+    const int ns_early = (MLA && t.type == T_MLA_ATTN) ? -1 : task_nstages<TILED, F4>(p, t);
     if (ctid == 0) {
       long long* tr = p.trace ? p.trace + (size_t)t.id * kTraceCols : nullptr;
       if (tr) tr[0] = (long long)globaltimer_ns();
@@ -2749,7 +2750,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
     }
     consumer_sync(kConsumerThreads);
     if (flags[0]) break;  // uniform: every consumer thread read the same flag
-    const int ns = ns_early >= 0 ? ns_early : task_nstages<TILED>(p, t);
+    const int ns = ns_early >= 0 ? ns_early : task_nstages<TILED, F4>(p, t);
 
     if (!MLA && t.type == T_ATTN) {
       cur_key = -1;  // the attention scratch aliases the input-vector planes
@@ -2771,7 +2772,7 @@ __device__ void consumer(const Params& p, const Task* my, int ntask, uint8_t* ri
       if constexpr (MLA)
         uk_task(p, t, gemv_geom<false>(p, t), gs, ns, ring, full, empty, tags, ub, red, warp, lane, ctid, ab);
     } else {
-      const GemvGeom g = gemv_geom<TILED>(p, t);
+      const GemvGeom g = gemv_geom<TILED, F4>(p, t);
       const int key = input_key(t);
       float* resid = ub + p.xs_floats;  // residual rows of this task (O-proj, down)
       const bool has_resid = t.op == OP_O || t.op == OP_DOWN || t.op == OP_MO;
@@ -3052,7 +3053,7 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
-    producer<TILED, MLA, SP>(p, my, ntask, ring, full, empty, tags,
+    producer<TILED, MLA, SP, F4>(p, my, ntask, ring, full, empty, tags,
              reinterpret_cast<const volatile int*>(misc + 80), threadIdx.x & 31);
     return;
   }
