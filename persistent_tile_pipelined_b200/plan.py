@@ -33,6 +33,8 @@ def report(wl, num_sms: int = 148, **overrides) -> dict:
     return {
         "workload": wl.name, "kind": wl.kind, "tokens_per_step": M,
         "gemv_form": "tensor-core tiles (16 x 1024)" if tiles else "CUDA-core rows",
+        "weights": {1: "E4M3 projections, 128 x 128 fp32 block scales",
+                    2: "MXFP4 routed experts (E2M1 + E8M0 per 32)"}.get(cfg.weight_format, "bf16"),
         "num_sms": info.num_sms, "ring": f"{info.ring_stages} x {info.stage_bytes} B",
         "smem_bytes_per_cta": info.smem_bytes, "kv_splits": info.kv_splits,
         "tasks": info.num_tasks, "tasks_by_kind_per_step": dict(sorted(kinds.items())),

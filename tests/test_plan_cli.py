@@ -43,3 +43,11 @@ def test_plan_report_cli():
     assert r["kv_splits"] == 8 and r["tasks_by_kind_per_step"]["attention"] == 32 * 8 * 8
     assert r["weight_gb_per_step"] == pytest.approx(15.01, abs=0.01)
     assert 1.0 <= r["sm_bytes_max_over_min"] < 1.1
+
+
+def test_plan_report_names_the_weight_format():
+    out = subprocess.run([sys.executable, "-m", "persistent_tile_pipelined_b200.plan",
+                          "--workload", "moe-4L-d7168-fp4"],
+                         capture_output=True, text=True, check=True, timeout=120)
+    r = json.loads(out.stdout)
+    assert r["weights"].startswith("MXFP4") and r["weight_gb_per_step"] == pytest.approx(2.173, abs=1e-3)
