@@ -304,6 +304,16 @@ def moe_plans(draw):
 
 
 @st.composite
+def moe_fp4_plans(draw):
+    """Random valid MoE stacks with MXFP4 routed experts (hidden and expert width multiples
+    of 32), on any SM count."""
+    wl, nsm, over = draw(moe_plans())
+    wl = wl.replace(weight_format="fp4", hidden=32 * draw(st.integers(2, 24)),
+                    expert_ffn=32 * draw(st.integers(1, 16)))
+    return wl, nsm, over
+
+
+@st.composite
 def mla_plans(draw):
     """Random valid absorbed-MLA stacks: heads, latent and rope widths, q_lora, nope / v."""
     kl = 128 * draw(st.integers(1, 5))
@@ -317,7 +327,7 @@ def mla_plans(draw):
 
 
 @settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
-@given(st.one_of(moe_plans(), mla_plans()))
+@given(st.one_of(moe_plans(), moe_fp4_plans(), mla_plans()))
 def test_random_moe_and_mla_plans_are_valid_task_graphs(case):
     wl, nsm, over = case
     check_plan(wl, nsm, **over)
